@@ -1,0 +1,25 @@
+"""Compile the CPU oracle (plain C, gcc, OpenMP) into oracle/liboracle.so.
+
+Test infrastructure only: the product library never links or loads it.
+"""
+import os
+import subprocess
+import sys
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+SRC = os.path.join(HERE, "lb_oracle.c")
+LIB = os.path.join(HERE, "liboracle.so")
+
+
+def build(force: bool = False, src: str = SRC, out: str = LIB) -> str:
+    """Build the oracle shared library if it is missing or older than its source."""
+    if not force and os.path.exists(out) and os.path.getmtime(out) >= os.path.getmtime(src):
+        return out
+    cmd = ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-fopenmp",
+           "-Wall", "-Wextra", "-Wno-unused-parameter", src, "-o", out]
+    subprocess.run(cmd, check=True)
+    return out
+
+
+if __name__ == "__main__":
+    print(build(force="--force" in sys.argv))
