@@ -1,0 +1,452 @@
+"""Benchmark of the MoE expert-parallel load-balancing decision path on B200.
+
+python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--config NAME]
+
+A step is one pass of the whole decision path (lookahead gate + top-k,
+per-rank counts, replica plan, normal gate + top-k, counts, Relief split,
+destinations + stable permutation) over every layer of the workload's model,
+all layers batched into one launch per kernel, replayed from a CUDA graph.
+Inputs (hidden states, gate weights, biases) are resident in HBM before the
+timed region; the per-step hidden-state stream (285 MB for the default
+workload) is larger than the 126 MB L2, so no L2 flush is needed.
+
+One JSON line is printed by rank 0.  `value` is whole-job routed
+token-assignments per second (all ranks; each rank runs its own independent
+copy of the workload: weak scaling, no collective on the data path).
+
+`--impl reference` times the CPU oracle (the only reference implementation
+this method has) on the host cores, on a bounded sample of the same workload.
+"""
+import argparse
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "routed token-assignments/s and per-layer T_solve (µs); % of HBM roofline"
+UNIT = "token-assignments/s"
+DEFAULT_WORKLOAD = "olmoe"
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), "measured"
+    except Exception:
+        return 6650.0, 1590.0, "fallback"
+
+
+def profile_traffic(kernel_tag, source_files):
+    """Per-launch DRAM bytes from a committed ncu summary, if the kernel's
+    source has not changed since the capture (else None)."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", f"{kernel_tag}.md")
+    if not os.path.exists(path):
+        return None
+    h = hashlib.sha256()
+    for f in source_files:
+        with open(os.path.join(ROOT, f), "rb") as fh:
+            h.update(fh.read())
+    want = h.hexdigest()[:16]
+    got, traffic = None, None
+    for line in open(path):
+        if line.startswith("source_sha:"):
+            got = line.split(":", 1)[1].strip()
+        if line.startswith("traffic_bytes_per_launch:"):
+            traffic = float(line.split(":", 1)[1].strip())
+    return traffic if got == want else None
+
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons with NVML in a background thread."""
+
+    def __init__(self, index, period=0.005):
+        self.index, self.period = index, period
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self._stop = threading.Event()
+        self._t = None
+
+    def __enter__(self):
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nvml = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(self.index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self._nvml = None
+            return self
+        self._t = threading.Thread(target=self._run, daemon=True)
+        self._t.start()
+        return self
+
+    def _run(self):
+        nv = self._nvml
+        names = {
+            getattr(nv, "nvmlClocksEventReasonHwSlowdown", 0x8): "hw_slowdown",
+            getattr(nv, "nvmlClocksEventReasonHwThermalSlowdown", 0x40): "hw_thermal_slowdown",
+            getattr(nv, "nvmlClocksEventReasonSwThermalSlowdown", 0x20): "sw_thermal_slowdown",
+            getattr(nv, "nvmlClocksEventReasonSwPowerCap", 0x4): "sw_power_cap",
+            getattr(nv, "nvmlClocksEventReasonHwPowerBrakeSlowdown", 0x80): "hw_power_brake_slowdown",
+        }
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                r = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                for bit, name in names.items():
+                    if r & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._t is not None:
+            self._t.join()
+        return False
+
+    def summary(self):
+        return {"sm_mhz": int(statistics.median(self.samples)) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+def dist_setup(n_gpus):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local))
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+def max_over_ranks(x, world):
+    if world == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ----------------------------------------------------------------------------- GPU arm
+def run_ours(args, world, rank, local):
+    from moe_expert_load_bf16_b200 import _lib, build, workloads
+    from moe_expert_load_bf16_b200.pipeline import DecisionPath
+
+    build.build()
+    wl = workloads.WORKLOADS[args.config]
+    if rank:
+        wl = wl.with_(seed=wl.seed + 1000 * rank)     # independent problems per rank
+    Lyr, T, H, E, k, G, N, L = wl.layers, wl.T, wl.H, wl.E, wl.k, wl.G, wl.N, wl.L
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.current_stream()
+
+    # hidden slot 0 = h_0 again: the lookahead input of layer 0
+    hid = torch.empty(Lyr + 1, T, H, dtype=torch.bfloat16, device=dev)
+    workloads.hidden_chain(wl, Lyr, T=T, out=hid[1:])
+    hid[0].copy_(hid[1])
+    W = workloads.gate_weights(wl, Lyr, device=dev)
+    bias = workloads.biases(wl, Lyr).to(dev)
+    path = DecisionPath(Lyr, T, H, E, k, G, N, L, device=dev)
+
+    def step():
+        path.run(hid[:-1], hid[1:], W, bias)
+
+    # warm-up (also loads the library, sets kernel attributes, builds maps)
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if _lib.lb_get_status():
+        raise RuntimeError("device status flagged during warm-up")
+
+    g_step = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_step):
+        step()
+    g_step.replay()
+    torch.cuda.synchronize()
+
+    # ---------------- timed region: K graph replays
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        barrier(world)
+        torch.cuda.synchronize()
+        ev0.record(stream)
+        for _ in range(args.steps):
+            g_step.replay()
+        ev1.record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+    ms_total = max_over_ranks(ev0.elapsed_time(ev1), world)
+    ms_step = ms_total / args.steps
+    assign_per_step = Lyr * T * k
+    value = assign_per_step * world / (ms_step * 1e-3)
+
+    # ---------------- dominant kernel: the gate (two launches per step)
+    g_gate = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_gate):
+        _lib.lb_predict_topk(hid[:-1], W, bias, k, ids=path.ids_pred)
+        _lib.lb_predict_topk(hid[1:], W, bias, k, ids=path.ids)
+    g_gate.replay()
+    torch.cuda.synchronize()
+    barrier(world)
+    ev0.record(stream)
+    for _ in range(args.steps):
+        g_gate.replay()
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    gate_ms = ev0.elapsed_time(ev1) / (2 * args.steps)
+    gate_bytes = Lyr * (2 * T * H + 2 * H * E + 4 * E + 4 * T * k)
+    gate_flops = Lyr * 2.0 * T * H * E
+    hbm, tflops, peak_kind = peaks()
+    achieved = gate_bytes / (gate_ms * 1e-3) / 1e9
+    traffic = profile_traffic("gate_topk_olmoe16", ["moe_expert_load_bf16_b200/csrc/gate_topk.cuh",
+                                                    "moe_expert_load_bf16_b200/csrc/common.cuh"])
+
+    # ---------------- per-layer latencies (single problem, graph replays)
+    lat = per_layer_latency(wl, hid, W, bias, dev, reps=max(50, args.steps))
+
+    # ---------------- end to end through the C ABI with host buffers
+    e2e = end_to_end(args, wl, hid, W, bias, path, dev, world)
+
+    torch.cuda.synchronize()
+    flags = _lib.lb_get_status()
+    if flags:
+        raise RuntimeError(f"device status flagged: {flags}")
+
+    out = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": f"{wl.name}: {Lyr} layers x T={T} tokens, H={H}, E={E}, top-{k}, "
+                               f"G={G} ranks, N={N} replica slots (L={L})",
+                   "layers": Lyr, "T": T, "H": H, "E": E, "k": k, "G": G, "N": N, "L": L, "passes": 12,
+                   "batching": "all layers of a step in one launch per kernel, CUDA-graph replay",
+                   "l2": "inputs larger than L2 (hidden states %.0f MB per step)" % (2 * Lyr * T * H * 2 / 1e6),
+                   "parallelism": f"{world} independent replicas"},
+        "t_solve_us": lat["solve"], "t_split_us": lat["split"], "t_lookahead_us": lat["lookahead"],
+        "per_kernel_us": lat["kernels"],
+        "roofline": {"kernel": "gate_topk", "bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
+                     "frac": achieved / hbm, "traffic": traffic, "peak_kind": peak_kind,
+                     "algorithmic_bytes_per_launch": gate_bytes, "launch_us": gate_ms * 1e3,
+                     "tensor_frac": gate_flops / (gate_ms * 1e-3) / (tflops * 1e12)},
+        "e2e": e2e,
+        "gpu_launches": path.LAUNCHES_PER_RUN * args.steps,
+        "clocks": clk.summary(),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline(wl, budget_s=args.cpu_budget)
+    return out
+
+
+def per_layer_latency(wl, hid, W, bias, dev, reps):
+    """Median-free mean latency per layer (one problem, CUDA-graph replays) of
+    T_solve = count + split + assign on actual ids, T_split, T_lookahead =
+    2 gate + count + plan, and each kernel group alone."""
+    from moe_expert_load_bf16_b200 import _lib
+    from moe_expert_load_bf16_b200.pipeline import DecisionPath
+    T, H, E, k, G, N, L = wl.T, wl.H, wl.E, wl.k, wl.G, wl.N, wl.L
+    p1 = DecisionPath(1, T, H, E, k, G, N, L, device=dev)
+    p1.run(hid[0:1], hid[1:2], W[0:1], bias[0:1])
+    torch.cuda.synchronize()
+
+    def timed(fn):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            fn()
+        g.replay()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(reps):
+            g.replay()
+        b.record()
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) * 1e3 / reps
+
+    res = {
+        "solve": timed(p1.solve),
+        "split": timed(lambda: _lib.lb_split(p1.cnt, p1.plan, N, 12,
+                                             out=(p1.tok, p1.mass, p1.loads, p1.passes_run))),
+        "lookahead": timed(lambda: (p1.lookahead(hid[0:1], W[0:1], bias[0:1]), p1.route(hid[1:2], W[0:1],
+                                                                                        bias[0:1]))),
+    }
+    res["kernels"] = {
+        "gate": timed(lambda: _lib.lb_predict_topk(hid[1:2], W[0:1], bias[0:1], k, ids=p1.ids)),
+        "count": timed(lambda: _lib.lb_count(p1.ids, G, E, cnt=p1.cnt)),
+        "plan": timed(lambda: _lib.lb_plan_replicas(p1.cnt_pred, N, L, plan=p1.plan)),
+        "split": res["split"],
+        "assign": timed(lambda: _lib.lb_assign(p1.ids, p1.cnt, p1.plan, p1.tok, p1.mass, N,
+                                               out=(p1.dest, p1.perm, p1.offs), workspace=p1.ws)),
+    }
+    return res
+
+
+def end_to_end(args, wl, hid, W, bias, path, dev, world):
+    """Same metric through the public API with host buffers: every step
+    copies its inputs from pinned host memory and reads its results back."""
+    Lyr, T, k = wl.layers, wl.T, wl.k
+    h_host = hid.cpu().pin_memory()
+    w_host = W.cpu().pin_memory()
+    b_host = bias.cpu().pin_memory()
+    outs = (path.dest, path.perm, path.offs, path.loads)
+    o_host = [torch.empty(o.shape, dtype=o.dtype).pin_memory() for o in outs]
+    h2d = h_host.numel() * 2 + w_host.numel() * 2 + b_host.numel() * 4
+    d2h = sum(o.numel() * o.element_size() for o in o_host)
+
+    def step():
+        hid.copy_(h_host, non_blocking=True)
+        W.copy_(w_host, non_blocking=True)
+        bias.copy_(b_host, non_blocking=True)
+        path.run(hid[:-1], hid[1:], W, bias)
+        for o, oh in zip(outs, o_host):
+            oh.copy_(o, non_blocking=True)
+
+    for _ in range(max(1, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    n = max(3, min(args.steps, 20))
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    a.record()
+    for _ in range(n):
+        step()
+    b.record()
+    torch.cuda.synchronize()
+    barrier(world)
+    ms = max_over_ranks(a.elapsed_time(b), world) / n
+    return {"value": Lyr * T * k * world / (ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": int(h2d),
+            "d2h_bytes_per_step": int(d2h), "ms_per_step": ms, "steps": n}
+
+
+# ----------------------------------------------------------------------------- CPU oracle
+def cpu_baseline(wl, budget_s=15.0):
+    """The oracle, as it stands, on this host's cores, over whole layers of
+    the workload (both gate calls, count, plan, count, split, assign) until
+    the time budget is spent.  If one layer's gate would not fit the budget,
+    the gate runs on evenly spaced sampled rows and its time is scaled to the
+    full layer (the integer stages always run on the whole layer)."""
+    import oracle
+    from moe_expert_load_bf16_b200 import workloads
+    o = oracle.default()
+    T, H, E, k, G, N, L = wl.T, wl.H, wl.E, wl.k, wl.G, wl.N, wl.L
+    hid = workloads.hidden_chain(wl, 2)
+    hb = [workloads.bf16_bits(hid[0]), workloads.bf16_bits(hid[1])]
+    wb = workloads.bf16_bits(workloads.gate_weights(wl, 1)[0])
+    b = workloads.biases(wl, 1)[0].numpy()
+    probe = np.arange(min(T, 64))
+    t0 = time.perf_counter()
+    o.gate(hb[1][probe], wb, b, k)
+    per_row = (time.perf_counter() - t0) / len(probe)
+    rows = T if 2 * per_row * T <= 0.5 * budget_s else max(64, int(0.5 * budget_s / (2 * per_row)))
+    sel = np.linspace(0, T - 1, rows).astype(np.int64)
+    # full ids for the integer stages (computed once, untimed, when the gate is sampled)
+    ids_pred_full = ids_full = None
+    if rows < T:
+        ids_pred_full = o.gate(hb[0], wb, b, k)[1]
+        ids_full = o.gate(hb[1], wb, b, k)[1]
+    total, layers, t_start = 0.0, 0, time.perf_counter()
+    while layers == 0 or (time.perf_counter() - t_start < budget_s and layers < wl.layers):
+        t0 = time.perf_counter()
+        _, ids_pred = o.gate(hb[0][sel], wb, b, k)
+        t_gate = time.perf_counter() - t0
+        if rows < T:
+            ids_pred = ids_pred_full
+        t1 = time.perf_counter()
+        p = o.plan(o.count(ids_pred, G, E), N, L)
+        t_int = time.perf_counter() - t1
+        t0 = time.perf_counter()
+        _, ids = o.gate(hb[1][sel], wb, b, k)
+        t_gate += time.perf_counter() - t0
+        if rows < T:
+            ids = ids_full
+        t1 = time.perf_counter()
+        cnt = o.count(ids, G, E)
+        s = o.split(cnt, p, 12)
+        o.assign(ids, p, s, G, E)
+        t_int += time.perf_counter() - t1
+        total += t_gate * T / rows + t_int
+        layers += 1
+    sample = (f"{layers} full layer(s) of {wl.name} (T={T}, H={H}, E={E}, top-{k}): both gate calls, "
+              f"count, plan, count, split, assign")
+    if rows < T:
+        sample += f"; gate on {rows} of {T} rows per call, time scaled to the full layer"
+    return {"value": layers * T * k / total, "unit": UNIT, "cores": o.threads(), "kind": "oracle",
+            "sample": sample, "seconds": total}
+
+
+def run_reference(args, world, rank):
+    from moe_expert_load_bf16_b200 import workloads
+    wl = workloads.WORKLOADS[args.config]
+    if rank != 0:
+        return None
+    for _ in range(min(args.warmup, 1)):
+        cpu_baseline(wl, budget_s=1.0)
+    per = max(2.0, min(20.0, 120.0 / max(1, args.steps)))
+    t0 = time.perf_counter()
+    vals = [cpu_baseline(wl, budget_s=per) for _ in range(args.steps)]
+    wall = time.perf_counter() - t0
+    value = statistics.mean(v["value"] for v in vals)
+    cb = dict(vals[-1])
+    cb["value"] = value
+    Lyr, T, k = wl.layers, wl.T, wl.k
+    return {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": Lyr * T * k / value * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic",
+            "config": {"workload": f"{wl.name}: {Lyr} layers x T={T} tokens, H={wl.H}, E={wl.E}, top-{k}, "
+                                   f"G={wl.G} ranks, N={wl.N} replica slots (L={wl.L})"},
+            "cpu_baseline": cb, "wall_s": wall,
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--config", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        rank = int(os.environ.get("RANK", "0"))
+        world = int(os.environ.get("WORLD_SIZE", str(args.gpus)))
+        out = run_reference(args, world, rank)
+        if out is not None:
+            print(json.dumps(out), flush=True)
+        return
+    world, rank, local = dist_setup(args.gpus)
+    try:
+        out = run_ours(args, world, rank, local)
+        if rank == 0:
+            print(json.dumps(out), flush=True)
+    finally:
+        if world > 1 and torch.distributed.is_initialized():
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,220 @@
+/*
+ * lb.h -- C ABI of the B200 (sm_100a) library for the per-layer MoE
+ * expert-parallel load-balancing decision path.
+ *
+ * Sources the operations follow (page titles and sections):
+ *   [Libra]  "Libra: Effective yet Efficient Load Balancing for Large-Scale
+ *            MoE Inference" (project README), Key Ideas.
+ *   [FB]     "FreeBalance: Pre-Routing Online MoE Load Balancing via Residual
+ *            Workload Prediction", sec. 2.1-2.2, sec. 3.2 eq. 2-5, Algorithm 1.
+ *   [Relief] "A Per-Step Load-Balancing Engine for Expert-Parallel MoE
+ *            Serving", The Per-Step Optimum Problem; Methodology, The Relief
+ *            Algorithm, Algorithm 1; Three Deployments.
+ *
+ * Model.  G expert-parallel ranks are modelled logically on one GPU.  A
+ * problem has T tokens; token t comes from source rank src(t) = t / (T/G)
+ * (one contiguous batch per rank), expert e lives at home(e) = e / (E/G).
+ *
+ * Conventions for every entry point:
+ *   - All array pointers are DEVICE pointers to caller-owned memory; the
+ *     library allocates no device memory and keeps no pointer after return.
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Calls are
+ *     stream-ordered and asynchronous; none of them synchronizes the host,
+ *     except lb_get_status.
+ *   - `nbatch` >= 1 independent problems of identical shape are processed
+ *     by one call; every per-problem array is laid out problem-major and
+ *     contiguous (problem b starts at b * per-problem size).
+ *   - Return codes: LB_OK; LB_EINVAL for a bad argument (nothing launched);
+ *     LB_ECUDA if a launch failed; LB_ENOSPACE if a workspace is too small.
+ *     Bad DATA found on the device (an expert id out of range, a repeated id
+ *     in a token's row, an inconsistent plan or split) never traps: the
+ *     kernel skips the offending element and sets a bit in a per-device
+ *     status word that lb_get_status reads.
+ *   - int32 counts: T * k * nbatch must be < 2^31.
+ */
+#ifndef LB_H_
+#define LB_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+enum {
+    LB_OK = 0,
+    LB_EINVAL = 1,    /* bad argument, nothing launched */
+    LB_ECUDA = 2,     /* a CUDA call or launch failed */
+    LB_EDATA = 3,     /* bad data seen on the device (lb_get_status) */
+    LB_ENOSPACE = 4   /* workspace smaller than required */
+};
+
+/* Bits of the device status word (lb_get_status). */
+enum {
+    LB_DEV_BAD_IDS = 1,      /* expert id out of [0,E) or repeated in a row */
+    LB_DEV_TIMEOUT = 2,      /* a bounded wait inside a kernel gave up */
+    LB_DEV_BAD_PLAN = 4,     /* plan blob inconsistent (e.g. round not rank-disjoint) */
+    LB_DEV_BAD_SPLIT = 8     /* split does not cover the remote tokens it should */
+};
+
+/* Limits. */
+#define LB_MAX_E_GATE 256    /* experts per gate call (one tcgen05 MMA N) */
+#define LB_MAX_K_GATE 16     /* top-k of the gate */
+#define LB_MAX_G 64          /* logical ranks */
+#define LB_MAX_E 1024        /* experts in the integer stages */
+#define LB_MAX_K 32          /* experts per token in the integer stages */
+#define LB_MAX_N 32          /* replica slots per rank */
+
+/* ------------------------------------------------------------------------
+ * Step 1 -- lookahead gate + top-k   [FB sec. 3.2 eq. 2-5, sec. 2.1; Libra,
+ * Key Ideas, lookahead predictor]
+ *   logit[b,t,e] = sum_h h[b,t,h] * w[b,e,h] + bias[b,e]   (fp32 accumulate)
+ *   ids[b,t,0..k-1] = the k largest logits of row t, in descending order,
+ *                     equal logits ordered by ascending expert id.
+ * The same call is the "normal" router when given the layer's own input.
+ *   h       bf16 [nbatch, T, H] row-major, 16-byte aligned
+ *   w       bf16 [nbatch, E, H] (row e = expert e's gate weights), 16-byte aligned
+ *   bias    fp32 [nbatch, E] or NULL (no bias)
+ *   ids     int32 [nbatch, T, k]                          (output)
+ *   logits  fp32 [nbatch, T, E] or NULL                    (optional output)
+ * Limits: 1 <= E <= LB_MAX_E_GATE, 1 <= k <= min(E, LB_MAX_K_GATE),
+ * H >= 8 and H % 8 == 0, T >= 0.  T need not be a multiple of the tile.
+ * ------------------------------------------------------------------------ */
+int lb_predict_topk(const void *h, const void *w, const float *bias,
+                    int nbatch, int T, int H, int E, int k,
+                    int32_t *ids, float *logits, void *stream);
+
+/* Tuning knobs of lb_predict_topk (process-wide; 0 = automatic choice):
+ * pipeline stages per CTA (2..8) and split of H across a CTA cluster
+ * (1, 2, 4, 8 or 16).  Results do not depend on them beyond fp32 rounding
+ * of the split-H partial sums.  Returns LB_EINVAL for values out of range. */
+int lb_gate_tuning(int stages, int split);
+
+/* ------------------------------------------------------------------------
+ * Step 2 -- per-rank histograms   [FB sec. 3.2 eq. 5; Algorithm 1,
+ * aggregation of expert workloads; Libra, Key Ideas, "its own tokens"]
+ *   cnt[b,g,e] = #{(t,j) : src(t) = g, ids[b,t,j] = e}
+ *   ids  int32 [nbatch, T, k];   cnt int32 [nbatch, G, E]   (output)
+ * Limits: T % G == 0, 1 <= G <= LB_MAX_G, 1 <= E <= LB_MAX_E,
+ * 1 <= k <= LB_MAX_K.  Ids out of range or repeated in a row are skipped and
+ * flagged (LB_DEV_BAD_IDS).
+ * ------------------------------------------------------------------------ */
+int lb_count(const int32_t *ids, int nbatch, int T, int k, int E, int G,
+             int32_t *cnt, void *stream);
+
+/* ------------------------------------------------------------------------
+ * Step 3 -- locality-aware replica plan   [Libra, Key Ideas, locality-aware
+ * expert replication planning, phases 1 and 2; Relief, The Relief
+ * Algorithm (replica edges, edge-coloured round schedule)]
+ * Phase 1: each rank g imports up to L experts it does not host, those its
+ *   own tokens request most, order (cnt[g,e] desc, e asc); never one with
+ *   cnt[g,e] == 0.
+ * Load model: a token whose source holds its expert is served there; the
+ *   rest of expert e's tokens (m[e]) are served at home(e).
+ * Phase 2: at most sum_g (N - used[g]) times: u = most-loaded rank (lowest
+ *   id on ties); among u's home experts with m[e] > 0 that some rank can
+ *   still take (does not hold e, has a free slot), the one with the largest
+ *   m[e] (lowest id on ties); v = least-loaded such rank (lowest id on ties);
+ *   c = cnt[v,e] becomes local to v and d = min(m[e]-c, max(0, lu-lv) >> 1)
+ *   more is credited to v (lu = load[u]-c, lv = load[v]+c); stop if no
+ *   candidate or c + d == 0.
+ * Edges: one transfer (home(e) -> r, e) per replica, ordered by e then r;
+ *   schedule: greedy edge colouring in that order (lowest round free at both
+ *   ends); rounds are rank-disjoint.
+ *   cnt   int32 [nbatch, G, E] (predicted counts)
+ *   plan  caller-allocated [nbatch] blobs of lb_plan_bytes(G,E,N) bytes each
+ *         (output; layout below)
+ * Limits: E % G == 0, G <= LB_MAX_G, E <= LB_MAX_E, G*E <= 24576,
+ * 0 <= L <= N <= min(LB_MAX_N, E - E/G).
+ * ------------------------------------------------------------------------ */
+size_t lb_plan_bytes(int G, int E, int N);
+int lb_plan_replicas(const int32_t *cnt, int nbatch, int G, int E, int N, int L,
+                     void *plan, void *stream);
+
+/* Plan blob layout (byte offsets from the start of one problem's blob).
+ * All fields int32 except holds (uint8).  Edge arrays hold n_edges valid
+ * entries in schedule order (round by round, edge order inside a round).
+ *   hdr[16]        n_edges, n_rounds, n_phase1, n_phase2, G, E, N, L, 0...
+ *   used[G]        replica slots used per rank
+ *   slots[G*N]     expert id per slot, -1 if empty (phase-1 slots first)
+ *   slot_phase[G*N] 1 or 2, 0 if empty
+ *   plan_load[G]   load model after phase 2
+ *   edge_u[G*N]    home rank of the transfer
+ *   edge_v[G*N]    replica rank
+ *   edge_e[G*N]    expert
+ *   edge_round[G*N]
+ *   round_ptr[G*N+1] edges of round r are [round_ptr[r], round_ptr[r+1])
+ *   rep_ptr[E+1]   edges of expert e, by ascending replica rank, are
+ *   rep_edge[G*N]    rep_edge[rep_ptr[e] .. rep_ptr[e+1]) (schedule indices)
+ *   holds[G*E]     uint8, 1 if rank g holds expert e (home or replica)   */
+typedef struct {
+    size_t hdr, used, slots, slot_phase, plan_load, edge_u, edge_v, edge_e,
+        edge_round, round_ptr, rep_ptr, rep_edge, holds, total;
+} lb_plan_layout;
+int lb_plan_layout_of(int G, int E, int N, lb_plan_layout *out);
+
+/* ------------------------------------------------------------------------
+ * Step 4 -- Relief split   [Relief, Methodology, Algorithm 1; The Per-Step
+ * Optimum Problem]
+ * Remote mass of expert e: R_e = tokens of e whose source does not hold e.
+ * For a replicated expert with m edges (ascending replica rank j=0..m-1):
+ *   tok_j = R_e/m + (j < R_e % m), mass_j = tok_j (all start at home).
+ * L[i] = own tokens of experts i holds + R_e of every expert homed on i.
+ * Each pass visits the rounds in order and, inside a round, every transfer:
+ *   gap = L[u]-L[v]; delta = min(|gap| >> 1, gap > 0 ? mass : tok - mass);
+ *   if delta > 0: L[u] -= sgn(gap) delta; L[v] += sgn(gap) delta;
+ *                 mass -= sgn(gap) delta.
+ * At most `passes` passes; stops after a pass that moved nothing.
+ *   cnt        int32 [nbatch, G, E] (actual counts)
+ *   plan       [nbatch] plan blobs from lb_plan_replicas
+ *   tok, mass  int32 [nbatch, G*N] (schedule order; entries past n_edges = 0;
+ *              may be NULL when G*N == 0)
+ *   loads      int32 [nbatch, G];  passes_run int32 [nbatch]   (outputs)
+ * Limits: as lb_plan_replicas; 0 <= passes <= 4096.
+ * ------------------------------------------------------------------------ */
+int lb_split(const int32_t *cnt, const void *plan, int nbatch, int G, int E, int N,
+             int passes, int32_t *tok, int32_t *mass, int32_t *loads,
+             int32_t *passes_run, void *stream);
+
+/* ------------------------------------------------------------------------
+ * Step 5 -- destinations + stable permutation   [Libra, Key Ideas,
+ * two-stage locality-aware execution and token sharding; FB sec. 2.2]
+ * For assignment f = t*k + j (e = ids[t,j], s = src(t)):
+ *   s holds e -> dest = s; e unreplicated -> dest = home(e); otherwise
+ *   q = rank of f among e's remote assignments (ascending f); edge j covers
+ *   q in [sum_{i<j} tok_i, ... + tok_j): its first mass_j stay at home(e),
+ *   the rest go to the edge's replica rank.
+ * perm = stable sort of f by key dest*E + e; offs = exclusive prefix sum of
+ * the bucket sizes over all G*E keys, offs[G*E] = T*k.
+ *   ids        int32 [nbatch, T, k];  cnt int32 [nbatch, G, E] (lb_count of ids)
+ *   plan, tok, mass: from lb_plan_replicas and lb_split
+ *   dest       int32 [nbatch, T, k]; perm int32 [nbatch, T*k] (problem-local f)
+ *   offs       int32 [nbatch, G*E+1]                       (outputs)
+ *   workspace  device scratch of >= lb_assign_workspace_bytes(...) bytes,
+ *              256-byte aligned, caller-owned; contents need not be cleared.
+ * Limits: T % G == 0, G <= LB_MAX_G, E <= LB_MAX_E, k <= LB_MAX_K.
+ * ------------------------------------------------------------------------ */
+size_t lb_assign_workspace_bytes(int nbatch, int T, int k, int G, int E, int N);
+int lb_assign(const int32_t *ids, const int32_t *cnt, const void *plan,
+              const int32_t *tok, const int32_t *mass, int nbatch, int T, int k,
+              int G, int E, int N, int32_t *dest, int32_t *perm, int32_t *offs,
+              void *workspace, size_t workspace_bytes, void *stream);
+
+/* ------------------------------------------------------------------------
+ * Status and diagnostics (not from the pages).
+ * lb_get_status: synchronizes the current device, writes the status word of
+ * the current device to *flags (LB_DEV_* bits) and clears it when `clear`
+ * is non-zero.  Returns LB_OK, LB_EDATA if any data bit is set, or LB_ECUDA.
+ * lb_strerror: static text for a return code.
+ * ------------------------------------------------------------------------ */
+int lb_get_status(int32_t *flags, int clear);
+const char *lb_strerror(int code);
+/* Text of the CUDA error behind this thread's last LB_ECUDA return. */
+const char *lb_last_error(void);
+int lb_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* LB_H_ */

@@ -1,0 +1,312 @@
+// Step 1: lookahead gate GEMM + top-k, fused (FreeBalance sec. 3.2 eq. 2-5;
+// Libra README, Key Ideas, lookahead predictor).
+//
+// One CTA owns a 128-token tile of one problem.  TMA streams h[128 x 64] and
+// W[Epad x 64] bf16 tiles (128-byte swizzle) through a ring of shared-memory
+// stages; one thread issues tcgen05.mma (M=128, N=Epad, K=16) into a TMEM
+// accumulator of Epad fp32 columns; after the last k-block, TMEM holds the
+// 128 x E logit tile and the epilogue does the top-k without another pass
+// over memory.
+//
+// Split of H across a cluster (SPLITK): when there are too few token tiles to
+// fill the GPU, `split` CTAs of one cluster each take 1/split of H; each CTA
+// stages its partial tile in its own shared memory, and after a cluster
+// barrier CTA r reduces rows [r*128/split, (r+1)*128/split) over all
+// partials (in fixed CTA order, so results are deterministic), adds the bias
+// and ranks them, with `split` threads per row merged by warp shuffles.
+//
+// Top-k: each thread keeps a sorted list of its KMAX best (value desc, id
+// asc) fed in ascending expert order with a strict '>' so equal logits keep
+// the lower id first; lists of several threads merge by repeated
+// (max value, min id) shuffles.
+#pragma once
+#include "common.cuh"
+
+namespace lb {
+namespace gate {
+
+constexpr int BM = 128;        // tokens per tile (UMMA M)
+constexpr int BK = 64;         // bf16 per k-block: one 128-byte swizzle row
+constexpr int UK = 16;         // UMMA K for bf16
+constexpr int THREADS = 128;   // 4 warps; warp 0 lane 0 = TMA, warp 1 lane 0 = MMA
+constexpr int MAX_STAGES = 8;
+
+struct Params {
+    const float *bias;   // [B,E] or null
+    int32_t *ids;        // [B,T,k]
+    float *logits;       // [B,T,E] or null
+    int T, H, E, Epad, k, nkb, split, stages;
+    uint32_t tmem_cols;
+};
+
+template <int KMAX>
+struct TopK {
+    float v[KMAX];
+    int i[KMAX];
+    __device__ __forceinline__ void init() {
+#pragma unroll
+        for (int j = 0; j < KMAX; ++j) {
+            v[j] = -INFINITY;
+            i[j] = 0x7fffffff;
+        }
+    }
+    // Candidates must arrive in ascending id order.
+    __device__ __forceinline__ void push(float x, int id) {
+        if (!(x > v[KMAX - 1])) return;
+#pragma unroll
+        for (int j = KMAX - 1; j > 0; --j) {
+            const bool up = x > v[j - 1];          // x goes above slot j-1
+            const bool here = !up && x > v[j];     // x lands exactly in slot j
+            const float nv = up ? v[j - 1] : (here ? x : v[j]);
+            const int ni = up ? i[j - 1] : (here ? id : i[j]);
+            v[j] = nv;
+            i[j] = ni;
+        }
+        if (x > v[0]) {
+            v[0] = x;
+            i[0] = id;
+        }
+    }
+    // Merge the lists of `width` adjacent lanes (width a power of two <= 32);
+    // every lane of the group ends up with the merged list in `out`.
+    __device__ __forceinline__ void merge(int width, float (&ov)[KMAX], int (&oi)[KMAX]) {
+#pragma unroll
+        for (int j = 0; j < KMAX; ++j) {
+            float hv = v[0];
+            int hi = i[0];
+            for (int off = width >> 1; off > 0; off >>= 1) {
+                const float xv = __shfl_xor_sync(kFull, hv, off);
+                const int xi = __shfl_xor_sync(kFull, hi, off);
+                if (xv > hv || (xv == hv && xi < hi)) {
+                    hv = xv;
+                    hi = xi;
+                }
+            }
+            ov[j] = hv;
+            oi[j] = hi;
+            const bool pop = (i[0] == hi);
+#pragma unroll
+            for (int q = 0; q < KMAX - 1; ++q) {
+                v[q] = pop ? v[q + 1] : v[q];
+                i[q] = pop ? i[q + 1] : i[q];
+            }
+            if (pop) {
+                v[KMAX - 1] = -INFINITY;
+                i[KMAX - 1] = 0x7fffffff;
+            }
+        }
+    }
+};
+
+template <int KMAX, bool SPLITK>
+__global__ void __launch_bounds__(THREADS, 1)
+    gate_topk_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                     const Params p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                                ~static_cast<uintptr_t>(1023));
+    __shared__ __align__(8) uint64_t full_bar[MAX_STAGES];
+    __shared__ __align__(8) uint64_t empty_bar[MAX_STAGES];
+    __shared__ __align__(8) uint64_t acc_bar;
+    __shared__ uint32_t tmem_slot;
+    __shared__ int aborted;
+    __shared__ float bias_s[LB_MAX_E_GATE];
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int b = blockIdx.y;
+    const int S = SPLITK ? p.split : 1;
+    const int crank = SPLITK ? static_cast<int>(cluster_ctarank()) : 0;
+    const int mtile = blockIdx.x / S;
+    const int m0 = mtile * BM;
+    const int kb_per = (p.nkb + S - 1) / S;
+    const int kb0 = crank * kb_per;
+    const int nk = max(0, min(p.nkb, kb0 + kb_per) - kb0);
+    const uint32_t a_bytes = BM * 128u;
+    const uint32_t stage_bytes = a_bytes + static_cast<uint32_t>(p.Epad) * 128u;
+    const int stages = p.stages;
+
+    for (int c = tid; c < p.Epad; c += THREADS)
+        bias_s[c] = (p.bias != nullptr && c < p.E) ? p.bias[static_cast<int64_t>(b) * p.E + c] : 0.f;
+    if (tid == 0) {
+        for (int s = 0; s < stages; ++s) {
+            mbar_init(&full_bar[s], 1);
+            mbar_init(&empty_bar[s], 1);
+        }
+        mbar_init(&acc_bar, 1);
+        aborted = 0;
+        fence_mbar_init();
+        tma_prefetch_desc(&tmA);
+        tma_prefetch_desc(&tmB);
+    }
+    if (warp == 1) {
+        tmem_alloc(&tmem_slot, p.tmem_cols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = tmem_slot;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            // ---------------- TMA producer
+            int issued = 0;
+            for (int i = 0; i < nk; ++i) {
+                const int s = i % stages;
+                const uint32_t ph = (i / stages) & 1;
+                if (!mbar_wait(&empty_bar[s], ph ^ 1)) {
+                    atomicExch(&aborted, 1);
+                    flag(LB_DEV_TIMEOUT);
+                    break;
+                }
+                if (*reinterpret_cast<volatile int *>(&aborted)) break;
+                uint8_t *sa = smem + static_cast<size_t>(s) * stage_bytes;
+                mbar_arrive_expect_tx(&full_bar[s], stage_bytes);
+                tma_load_3d(&tmA, sa, &full_bar[s], (kb0 + i) * BK, m0, b);
+                tma_load_3d(&tmB, sa + a_bytes, &full_bar[s], (kb0 + i) * BK, 0, b);
+                ++issued;
+            }
+            // Never leave with copies in flight into this CTA's shared memory:
+            // wait (bounded) for the latest phase of every stage used.
+            for (int s = 0; s < stages && s < issued; ++s) {
+                const int last = s + ((issued - 1 - s) / stages) * stages;
+                if (!mbar_wait(&full_bar[s], (last / stages) & 1)) flag(LB_DEV_TIMEOUT);
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            // ---------------- MMA issuer
+            const uint32_t idesc = umma_idesc_bf16(BM, p.Epad);
+            for (int i = 0; i < nk; ++i) {
+                const int s = i % stages;
+                const uint32_t ph = (i / stages) & 1;
+                if (!mbar_wait(&full_bar[s], ph)) {
+                    atomicExch(&aborted, 1);
+                    flag(LB_DEV_TIMEOUT);
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t sa = smem_u32(smem + static_cast<size_t>(s) * stage_bytes);
+                const uint32_t sb = sa + a_bytes;
+#pragma unroll
+                for (int kk = 0; kk < BK / UK; ++kk) {
+                    umma_bf16(tmem, sw128_kmajor_desc(sa + kk * UK * 2), sw128_kmajor_desc(sb + kk * UK * 2),
+                              idesc, (i > 0 || kk > 0) ? 1u : 0u);
+                }
+                umma_commit(&empty_bar[s]);   // stage free once these MMAs have read it
+            }
+            umma_commit(&acc_bar);            // accumulator complete
+        }
+    }
+    __syncwarp();
+
+    // ---------------- epilogue: all four warps, thread tid <-> TMEM lane tid
+    bool ok = mbar_wait(&acc_bar, 0);
+    if (!ok) flag(LB_DEV_TIMEOUT);
+    tc_fence_after();
+    ok = ok && (nk > 0) && !*reinterpret_cast<volatile int *>(&aborted);
+    ok = __all_sync(kFull, ok);   // tcgen05.ld below is warp-collective
+    const int64_t rowbase = static_cast<int64_t>(b) * p.T;
+    const uint32_t tl = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+
+    if constexpr (!SPLITK) {
+        const int row = m0 + tid;
+        const bool valid = ok && row < p.T;
+        TopK<KMAX> tk;
+        tk.init();
+        float *lrow = (p.logits != nullptr && valid) ? p.logits + (rowbase + row) * p.E : nullptr;
+        if (ok) {
+            for (int c0 = 0; c0 < p.Epad; c0 += 16) {
+                uint32_t r[16];
+                tmem_ld16(tl + c0, r);
+                tmem_wait_ld();
+#pragma unroll
+                for (int q = 0; q < 16; ++q) {
+                    const int c = c0 + q;
+                    if (c < p.E) {
+                        const float x = __uint_as_float(r[q]) + bias_s[c];
+                        tk.push(x, c);
+                        if (lrow) lrow[c] = x;
+                    }
+                }
+            }
+        }
+        if (valid) {
+            int32_t *out = p.ids + (rowbase + row) * p.k;
+#pragma unroll
+            for (int j = 0; j < KMAX; ++j)
+                if (j < p.k) out[j] = tk.i[j];
+        }
+    } else {
+        // Stage the partial tile in this CTA's shared memory (pipeline buffers
+        // are free: every TMA write landed and every MMA read finished before
+        // acc_bar completed).
+        const int PS = p.Epad + 4;   // padded row stride in floats
+        float *part = reinterpret_cast<float *>(smem);
+        if (ok) {
+            for (int c0 = 0; c0 < p.Epad; c0 += 16) {
+                uint32_t r[16];
+                tmem_ld16(tl + c0, r);
+                tmem_wait_ld();
+                float4 *dst = reinterpret_cast<float4 *>(part + tid * PS + c0);
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+                    dst[q] = make_float4(__uint_as_float(r[4 * q]), __uint_as_float(r[4 * q + 1]),
+                                         __uint_as_float(r[4 * q + 2]), __uint_as_float(r[4 * q + 3]));
+            }
+        } else {
+            for (int c = 0; c < p.Epad; ++c) part[tid * PS + c] = 0.f;
+        }
+        cluster_sync();   // every CTA of the cluster passes both barriers, always
+        const int R = BM / S;          // rows this CTA finishes
+        const int rl = tid / S, pp = tid % S;
+        const int trow = crank * R + rl;
+        const int row = m0 + trow;
+        const int C = p.Epad / S;      // columns per thread (multiple of 4)
+        TopK<KMAX> tk;
+        tk.init();
+        const bool valid = row < p.T;
+        float *lrow = (p.logits != nullptr && valid) ? p.logits + (rowbase + row) * p.E : nullptr;
+        const uint32_t pbase = smem_u32(part + trow * PS);
+        for (int c = pp * C; c < pp * C + C; c += 4) {
+            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+            for (int s = 0; s < S; ++s) {
+                const float4 x = ld_cluster_f4(mapa_shared(pbase + c * 4, s));
+                acc.x += x.x;
+                acc.y += x.y;
+                acc.z += x.z;
+                acc.w += x.w;
+            }
+            const float xs[4] = {acc.x, acc.y, acc.z, acc.w};
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const int cc = c + q;
+                if (cc < p.E) {
+                    const float x = xs[q] + bias_s[cc];
+                    tk.push(x, cc);
+                    if (lrow) lrow[cc] = x;
+                }
+            }
+        }
+        float ov[KMAX];
+        int oi[KMAX];
+        tk.merge(S, ov, oi);
+        if (valid && pp == 0) {
+            int32_t *out = p.ids + (rowbase + row) * p.k;
+#pragma unroll
+            for (int j = 0; j < KMAX; ++j)
+                if (j < p.k) out[j] = oi[j];
+        }
+        cluster_sync();   // keep this CTA's partials alive until all readers are done
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, p.tmem_cols);
+    }
+}
+
+}  // namespace gate
+}  // namespace lb

@@ -1,0 +1,399 @@
+// C-ABI entry points of liblb.so (declared and documented in include/lb.h).
+// Host code only validates arguments, computes launch shapes and launches;
+// every step of the decision path runs in the kernels included below.
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <climits>
+#include <cstdio>
+#include <mutex>
+
+#include "assign.cuh"
+#include "common.cuh"
+#include "count.cuh"
+#include "gate_topk.cuh"
+#include "plan.cuh"
+#include "split.cuh"
+
+namespace {
+
+using namespace lb;
+
+int g_tune_stages = 0;
+int g_tune_split = 0;
+
+inline bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// Text of the last CUDA error a call of this thread returned LB_ECUDA for.
+thread_local char g_last_error[256] = "";
+
+inline int cuda_fail(cudaError_t e, const char *where) {
+    std::snprintf(g_last_error, sizeof g_last_error, "%s: %s (%d)", where, cudaGetErrorString(e),
+                  static_cast<int>(e));
+    return LB_ECUDA;
+}
+
+inline int launched(const char *where = "launch") {
+    const cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? LB_OK : cuda_fail(e, where);
+}
+
+int device_sms() {
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) return 148;
+    return n;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+// 3-D bf16 tensor map [d2][d1][d0] (d0 innermost), box {64, box1, 1},
+// 128-byte swizzle, out-of-range elements read as zero.
+bool make_map(CUtensorMap *map, const void *base, uint64_t d0, uint64_t d1, uint64_t d2, uint32_t box1) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[3] = {d0, d1, d2};
+    cuuint64_t strides[2] = {d0 * 2, d0 * d1 * 2};
+    cuuint32_t box[3] = {static_cast<cuuint32_t>(gate::BK), box1, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Raise a kernel's dynamic shared-memory limit to at least `bytes` (the
+// limit plus the kernel's static shared memory must stay within the
+// per-block opt-in maximum, so it is raised only as far as needed).
+struct SmemLimit {
+    std::mutex mu;
+    size_t current = 0;
+    bool cluster_set = false;
+};
+
+template <typename F>
+bool allow_smem(F *kernel, SmemLimit &lim, size_t bytes, bool cluster16) {
+    std::lock_guard<std::mutex> lock(lim.mu);
+    if (bytes > lim.current) {
+        const cudaError_t e =
+            cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(bytes));
+        if (e != cudaSuccess) {
+            cuda_fail(e, "cudaFuncSetAttribute(max dynamic shared memory)");
+            return false;
+        }
+        lim.current = bytes;
+    }
+    if (cluster16 && !lim.cluster_set) {
+        const cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+        if (e != cudaSuccess) {
+            cuda_fail(e, "cudaFuncSetAttribute(non-portable cluster size)");
+            return false;
+        }
+        lim.cluster_set = true;
+    }
+    return true;
+}
+
+template <int KMAX, bool SPLITK>
+int launch_gate(const CUtensorMap &ma, const CUtensorMap &mb, const gate::Params &p, int mtiles, int nbatch,
+                size_t smem, cudaStream_t s) {
+    auto kern = gate::gate_topk_kernel<KMAX, SPLITK>;
+    static SmemLimit lim;
+    if (!allow_smem(kern, lim, smem, SPLITK)) return LB_ECUDA;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(mtiles * p.split, nbatch, 1);
+    cfg.blockDim = dim3(gate::THREADS, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    if (SPLITK) {
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = p.split;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+    }
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, ma, mb, p);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaLaunchKernelEx(gate_topk)");
+    return launched("gate_topk");
+}
+
+template <bool SPLITK>
+int launch_gate_k(int k, const CUtensorMap &ma, const CUtensorMap &mb, const gate::Params &p, int mtiles,
+                  int nbatch, size_t smem, cudaStream_t s) {
+    if (k <= 2) return launch_gate<2, SPLITK>(ma, mb, p, mtiles, nbatch, smem, s);
+    if (k <= 4) return launch_gate<4, SPLITK>(ma, mb, p, mtiles, nbatch, smem, s);
+    if (k <= 8) return launch_gate<8, SPLITK>(ma, mb, p, mtiles, nbatch, smem, s);
+    return launch_gate<16, SPLITK>(ma, mb, p, mtiles, nbatch, smem, s);
+}
+
+template <int K, bool VEC>
+int launch_count(const int32_t *ids, int nbatch, int T, int k, int E, int G, int32_t *cnt, cudaStream_t s) {
+    count::count_kernel<K, VEC><<<dim3(G, nbatch), count::THREADS, E * sizeof(int), s>>>(ids, T, k, E, G, cnt);
+    return launched("count");
+}
+
+template <int K>
+int launch_count_v(bool vec, const int32_t *ids, int nbatch, int T, int k, int E, int G, int32_t *cnt,
+                   cudaStream_t s) {
+    return vec ? launch_count<K, true>(ids, nbatch, T, k, E, G, cnt, s)
+               : launch_count<K, false>(ids, nbatch, T, k, E, G, cnt, s);
+}
+
+bool plan_shape_ok(int G, int E, int N, int L) {
+    if (G < 1 || G > LB_MAX_G || E < 1 || E > LB_MAX_E || E % G != 0) return false;
+    if (static_cast<long long>(G) * E > 24576) return false;
+    if (N < 0 || N > LB_MAX_N || N > E - E / G || L < 0 || L > N) return false;
+    return true;
+}
+
+}  // namespace
+
+extern "C" {
+
+int lb_version(void) { return 100; }
+
+const char *lb_strerror(int code) {
+    switch (code) {
+        case LB_OK: return "ok";
+        case LB_EINVAL: return "invalid argument";
+        case LB_ECUDA: return "CUDA error";
+        case LB_EDATA: return "bad data seen on the device";
+        case LB_ENOSPACE: return "workspace too small";
+        default: return "unknown error";
+    }
+}
+
+int lb_get_status(int32_t *flags, int clear) {
+    if (!flags) return LB_EINVAL;
+    cudaError_t e = cudaDeviceSynchronize();
+    if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceSynchronize");
+    int v = 0;
+    e = cudaMemcpyFromSymbol(&v, lb::g_status, sizeof(int));
+    if (e != cudaSuccess) return cuda_fail(e, "read status word");
+    *flags = v;
+    if (clear) {
+        const int z = 0;
+        e = cudaMemcpyToSymbol(lb::g_status, &z, sizeof(int));
+        if (e != cudaSuccess) return cuda_fail(e, "clear status word");
+    }
+    return v ? LB_EDATA : LB_OK;
+}
+
+const char *lb_last_error(void) { return g_last_error; }
+
+int lb_gate_tuning(int stages, int split) {
+    if (stages != 0 && (stages < 2 || stages > gate::MAX_STAGES)) return LB_EINVAL;
+    if (split != 0 && split != 1 && split != 2 && split != 4 && split != 8 && split != 16) return LB_EINVAL;
+    g_tune_stages = stages;
+    g_tune_split = split;
+    return LB_OK;
+}
+
+int lb_predict_topk(const void *h, const void *w, const float *bias, int nbatch, int T, int H, int E, int k,
+                    int32_t *ids, float *logits, void *stream) {
+    if (nbatch < 1 || nbatch > 65535 || T < 0 || H < 8 || H % 8 != 0 || E < 1 || E > LB_MAX_E_GATE || k < 1 ||
+        k > E || k > LB_MAX_K_GATE)
+        return LB_EINVAL;
+    if (!h || !w || !ids || !aligned(h, 16) || !aligned(w, 16) || !aligned(ids, 4)) return LB_EINVAL;
+    if (bias && !aligned(bias, 4)) return LB_EINVAL;
+    if (logits && !aligned(logits, 4)) return LB_EINVAL;
+    if (static_cast<long long>(T) * nbatch * std::max(k, E) >= INT_MAX) return LB_EINVAL;
+    if (T == 0) return LB_OK;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+
+    gate::Params p;
+    p.bias = bias;
+    p.ids = ids;
+    p.logits = logits;
+    p.T = T;
+    p.H = H;
+    p.E = E;
+    p.Epad = (E + 15) / 16 * 16;
+    p.k = k;
+    p.nkb = (H + gate::BK - 1) / gate::BK;
+    uint32_t cols = 32;
+    while (cols < static_cast<uint32_t>(p.Epad)) cols <<= 1;
+    p.tmem_cols = cols;
+    const int mtiles = (T + gate::BM - 1) / gate::BM;
+
+    // split of H across a cluster when the token tiles alone underfill the GPU
+    int S = 1;
+    if (g_tune_split) {
+        S = g_tune_split;
+    } else {
+        const int sms = device_sms();
+        while (static_cast<long long>(mtiles) * nbatch * S < sms && S * 2 <= 16 && S * 2 <= p.nkb / 2 &&
+               p.Epad % (4 * S * 2) == 0)
+            S *= 2;
+    }
+    // each of the S CTAs of a cluster reduces Epad/S columns per row with
+    // 16-byte shared-memory loads, so Epad/S must be a multiple of 4
+    if (S > p.nkb || p.Epad % (4 * S) != 0 || gate::BM % S != 0) return LB_EINVAL;
+    p.split = S;
+
+    const size_t stage_bytes = 16384 + static_cast<size_t>(p.Epad) * 128;
+    int stages = g_tune_stages;
+    if (!stages) stages = static_cast<int>(std::min<size_t>(8, std::max<size_t>(2, (110 * 1024 - 1024) / stage_bytes)));
+    size_t smem = stages * stage_bytes + 1024;
+    if (S > 1) smem = std::max(smem, static_cast<size_t>(gate::BM) * (p.Epad + 4) * 4 + 1024);
+    if (smem > 224 * 1024) {
+        stages = static_cast<int>((224 * 1024 - 1024) / stage_bytes);
+        smem = stages * stage_bytes + 1024;
+        if (S > 1) smem = std::max(smem, static_cast<size_t>(gate::BM) * (p.Epad + 4) * 4 + 1024);
+        if (stages < 2 || smem > 224 * 1024) return LB_EINVAL;
+    }
+    p.stages = stages;
+    // Never let more CTAs share an SM than its 512 TMEM columns can serve at
+    // once: pad the shared-memory request so the extra CTA does not fit.  (In
+    // a cluster, a CTA blocked in tcgen05.alloc behind a sibling that waits at
+    // the cluster barrier would never proceed.)
+    {
+        const size_t sm_per_sm = 228 * 1024;
+        const size_t max_ctas = 512 / p.tmem_cols;
+        smem = std::max(smem, sm_per_sm / (max_ctas + 1) + 1);
+        if (smem > 224 * 1024) return LB_EINVAL;
+    }
+
+    CUtensorMap ma, mb;
+    if (!make_map(&ma, h, static_cast<uint64_t>(H), static_cast<uint64_t>(T), static_cast<uint64_t>(nbatch),
+                  gate::BM)) {
+        std::snprintf(g_last_error, sizeof g_last_error, "cuTensorMapEncodeTiled failed for h");
+        return LB_ECUDA;
+    }
+    if (!make_map(&mb, w, static_cast<uint64_t>(H), static_cast<uint64_t>(E), static_cast<uint64_t>(nbatch),
+                  static_cast<uint32_t>(p.Epad))) {
+        std::snprintf(g_last_error, sizeof g_last_error, "cuTensorMapEncodeTiled failed for w");
+        return LB_ECUDA;
+    }
+    return S > 1 ? launch_gate_k<true>(k, ma, mb, p, mtiles, nbatch, smem, s)
+                 : launch_gate_k<false>(k, ma, mb, p, mtiles, nbatch, smem, s);
+}
+
+int lb_count(const int32_t *ids, int nbatch, int T, int k, int E, int G, int32_t *cnt, void *stream) {
+    if (nbatch < 1 || nbatch > 65535 || T < 0 || G < 1 || G > LB_MAX_G || T % G != 0 || E < 1 || E > LB_MAX_E ||
+        k < 1 || k > LB_MAX_K)
+        return LB_EINVAL;
+    if (!cnt || (T > 0 && !ids) || !aligned(cnt, 4) || (ids && !aligned(ids, 4))) return LB_EINVAL;
+    if (static_cast<long long>(T) * k * nbatch >= INT_MAX) return LB_EINVAL;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const bool vec = ids && aligned(ids, 16);
+    if (k <= 2) return launch_count_v<2>(vec, ids, nbatch, T, k, E, G, cnt, s);
+    if (k <= 4) return launch_count_v<4>(vec, ids, nbatch, T, k, E, G, cnt, s);
+    if (k <= 8) return launch_count_v<8>(vec, ids, nbatch, T, k, E, G, cnt, s);
+    if (k <= 16) return launch_count_v<16>(vec, ids, nbatch, T, k, E, G, cnt, s);
+    return launch_count_v<32>(vec, ids, nbatch, T, k, E, G, cnt, s);
+}
+
+size_t lb_plan_bytes(int G, int E, int N) {
+    if (G < 1 || E < 1 || N < 0) return 0;
+    return plan::layout(G, E, N).total;
+}
+
+int lb_plan_layout_of(int G, int E, int N, lb_plan_layout *out) {
+    if (!out || G < 1 || E < 1 || N < 0) return LB_EINVAL;
+    const plan::Layout L = plan::layout(G, E, N);
+    out->hdr = L.hdr;
+    out->used = L.used;
+    out->slots = L.slots;
+    out->slot_phase = L.slot_phase;
+    out->plan_load = L.plan_load;
+    out->edge_u = L.edge_u;
+    out->edge_v = L.edge_v;
+    out->edge_e = L.edge_e;
+    out->edge_round = L.edge_round;
+    out->round_ptr = L.round_ptr;
+    out->rep_ptr = L.rep_ptr;
+    out->rep_edge = L.rep_edge;
+    out->holds = L.holds;
+    out->total = L.total;
+    return LB_OK;
+}
+
+int lb_plan_replicas(const int32_t *cnt, int nbatch, int G, int E, int N, int L, void *plan, void *stream) {
+    if (nbatch < 1 || !plan_shape_ok(G, E, N, L) || !cnt || !plan || !aligned(plan, 256) || !aligned(cnt, 4))
+        return LB_EINVAL;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const size_t smem = plan::smem_bytes(G, E, N);
+    if (smem > 224 * 1024) return LB_EINVAL;
+    static SmemLimit lim;
+    if (!allow_smem(plan::plan_kernel, lim, smem, false)) return LB_ECUDA;
+    plan::plan_kernel<<<nbatch, plan::THREADS, smem, s>>>(cnt, G, E, N, L, static_cast<uint8_t *>(plan),
+                                                            plan::layout(G, E, N).total);
+    return launched("plan");
+}
+
+int lb_split(const int32_t *cnt, const void *plan, int nbatch, int G, int E, int N, int passes, int32_t *tok,
+             int32_t *mass, int32_t *loads, int32_t *passes_run, void *stream) {
+    if (nbatch < 1 || !plan_shape_ok(G, E, N, 0) || passes < 0 || passes > 4096) return LB_EINVAL;
+    if (!cnt || !plan || !loads || !passes_run || !aligned(plan, 256)) return LB_EINVAL;
+    if (G * N > 0 && (!tok || !mass)) return LB_EINVAL;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const size_t smem = split::smem_bytes(G, E, N);
+    static SmemLimit lim;
+    if (!allow_smem(split::split_kernel, lim, smem, false)) return LB_ECUDA;
+    split::split_kernel<<<nbatch, split::THREADS, smem, s>>>(cnt, static_cast<const uint8_t *>(plan),
+                                                              plan::layout(G, E, N).total, G, E, N, passes, tok,
+                                                              mass, loads, passes_run);
+    return launched("split");
+}
+
+size_t lb_assign_workspace_bytes(int nbatch, int T, int k, int G, int E, int N) {
+    (void)T;
+    (void)k;
+    if (nbatch < 1 || G < 1 || E < 1 || N < 0) return 0;
+    return static_cast<size_t>(nbatch) * assign::ws_words(G, E, N) * 4;
+}
+
+int lb_assign(const int32_t *ids, const int32_t *cnt, const void *plan, const int32_t *tok, const int32_t *mass,
+              int nbatch, int T, int k, int G, int E, int N, int32_t *dest, int32_t *perm, int32_t *offs,
+              void *workspace, size_t workspace_bytes, void *stream) {
+    if (nbatch < 1 || nbatch > 65535 || T < 0 || T % G != 0 || k < 1 || k > LB_MAX_K || !plan_shape_ok(G, E, N, 0))
+        return LB_EINVAL;
+    if (!cnt || !plan || !offs || !workspace || !aligned(plan, 256) || !aligned(workspace, 256)) return LB_EINVAL;
+    if (G * N > 0 && (!tok || !mass)) return LB_EINVAL;
+    if (T > 0 && (!ids || !dest || !perm)) return LB_EINVAL;
+    if (static_cast<long long>(T) * k * nbatch >= INT_MAX) return LB_EINVAL;
+    if (assign::scatter_smem_bytes(E) > 224 * 1024) return LB_EINVAL;
+    if (workspace_bytes < lb_assign_workspace_bytes(nbatch, T, k, G, E, N)) return LB_ENOSPACE;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    assign::Args a;
+    a.ids = ids;
+    a.cnt = cnt;
+    a.tok = tok;
+    a.mass = mass;
+    a.plan = static_cast<const uint8_t *>(plan);
+    a.plan_stride = plan::layout(G, E, N).total;
+    a.T = T;
+    a.k = k;
+    a.G = G;
+    a.E = E;
+    a.N = N;
+    a.dest = dest;
+    a.perm = perm;
+    a.offs = offs;
+    a.ws = static_cast<int32_t *>(workspace);
+    a.ws_stride = assign::ws_words(G, E, N);
+    const size_t sm1 = assign::prep_smem_bytes(E), sm2 = assign::scatter_smem_bytes(E);
+    static SmemLimit lim1, lim2;
+    if (!allow_smem(assign::prep_kernel, lim1, sm1, false) || !allow_smem(assign::scatter_kernel, lim2, sm2, false))
+        return LB_ECUDA;
+    assign::prep_kernel<<<nbatch, assign::PREP_THREADS, sm1, s>>>(a);
+    if (launched("assign prep") != LB_OK) return LB_ECUDA;
+    if (T == 0) return LB_OK;
+    assign::scatter_kernel<<<dim3(G, nbatch), assign::SC_THREADS, sm2, s>>>(a);
+    return launched("assign scatter");
+}
+
+}  // extern "C"

@@ -1,0 +1,64 @@
+"""One pass of the decision path over a batch of independent problems (layers,
+steps or micro-batches of identical shape), with every buffer preallocated so
+the pass can be captured in a CUDA graph.
+
+Per problem (Libra README, Key Ideas; FreeBalance sec. 3.2, Algorithm 1;
+Relief, Algorithm 1):
+  ids_pred = top-k(gate(h_prev))           lookahead        lb_predict_topk
+  cnt_pred = counts(ids_pred)                               lb_count
+  plan     = replica plan(cnt_pred)                         lb_plan_replicas
+  ids      = top-k(gate(h_cur))            normal router    lb_predict_topk
+  cnt      = counts(ids)                                    lb_count
+  tok, mass, loads = split(cnt, plan)                       lb_split
+  dest, perm, offs = assign(ids, cnt, plan, split)          lb_assign
+"""
+import torch
+
+from . import _lib
+
+
+class DecisionPath:
+    def __init__(self, B, T, H, E, k, G, N, L, passes=12, device="cuda"):
+        self.B, self.T, self.H, self.E, self.k, self.G, self.N, self.L = B, T, H, E, k, G, N, L
+        self.passes = passes
+        dev = torch.device(device)
+        i32 = dict(dtype=torch.int32, device=dev)
+        self.ids_pred = torch.empty(B, T, k, **i32)
+        self.cnt_pred = torch.empty(B, G, E, **i32)
+        self.plan = torch.empty(B, _lib.lb_plan_bytes(G, E, N), dtype=torch.uint8, device=dev)
+        self.ids = torch.empty(B, T, k, **i32)
+        self.cnt = torch.empty(B, G, E, **i32)
+        self.tok = torch.empty(B, G * N, **i32)
+        self.mass = torch.empty(B, G * N, **i32)
+        self.loads = torch.empty(B, G, **i32)
+        self.passes_run = torch.empty(B, **i32)
+        self.dest = torch.empty(B, T, k, **i32)
+        self.perm = torch.empty(B, T * k, **i32)
+        self.offs = torch.empty(B, G * E + 1, **i32)
+        self.ws = torch.empty(max(256, _lib.lb_assign_workspace_bytes(B, T, k, G, E, N)), dtype=torch.uint8,
+                              device=dev)
+
+    # lookahead half: prediction and placement (off the per-step critical path)
+    def lookahead(self, h_prev, w, bias):
+        _lib.lb_predict_topk(h_prev, w, bias, self.k, ids=self.ids_pred)
+        _lib.lb_count(self.ids_pred, self.G, self.E, cnt=self.cnt_pred)
+        _lib.lb_plan_replicas(self.cnt_pred, self.N, self.L, plan=self.plan)
+
+    def route(self, h_cur, w, bias):
+        _lib.lb_predict_topk(h_cur, w, bias, self.k, ids=self.ids)
+
+    # the per-step decision on actual ids (T_solve)
+    def solve(self, ids=None):
+        ids = self.ids if ids is None else ids
+        _lib.lb_count(ids, self.G, self.E, cnt=self.cnt)
+        _lib.lb_split(self.cnt, self.plan, self.N, self.passes,
+                      out=(self.tok, self.mass, self.loads, self.passes_run))
+        _lib.lb_assign(ids, self.cnt, self.plan, self.tok, self.mass, self.N,
+                       out=(self.dest, self.perm, self.offs), workspace=self.ws)
+
+    def run(self, h_prev, h_cur, w, bias):
+        self.lookahead(h_prev, w, bias)
+        self.route(h_cur, w, bias)
+        self.solve()
+
+    LAUNCHES_PER_RUN = 8   # 2 gate, 2 count, plan, split, assign prep + scatter

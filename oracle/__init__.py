@@ -98,6 +98,7 @@ class Oracle:
         lib.orc_split_optimum.restype = ctypes.c_int64
         for f in (lib.orc_gate, lib.orc_count, lib.orc_plan, lib.orc_split, lib.orc_assign):
             f.restype = ctypes.c_int
+        lib.orc_threads.restype = ctypes.c_int
         self.lib = lib
         self.path = path
 
@@ -179,6 +180,9 @@ class Oracle:
             _ptr(ids), T, k, G, E, _ptr(holds), eu.shape[0], _ptr(eu), _ptr(ev), _ptr(ee),
             _ptr(tok), _ptr(mass), _ptr(dest), _ptr(perm), _ptr(offs)))
         return dest, perm, offs
+
+    def threads(self):
+        return int(self.lib.orc_threads())
 
     def split_optimum(self, cnt, p):
         cnt = _c(cnt, np.int32)

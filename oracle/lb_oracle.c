@@ -36,10 +36,23 @@
 #include <stdint.h>
 #include <stdlib.h>
 #include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
 
 #define ORC_OK 0
 #define ORC_EINVAL 1
 #define ORC_EDATA 3
+
+/* Threads the OpenMP parts (the gate) use; reported with CPU timings. */
+int orc_threads(void)
+{
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
 
 /* bf16 -> double, exactly: a bf16 value is the high half of an IEEE float. */
 static double orc_bf16(uint16_t x)

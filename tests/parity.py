@@ -1,0 +1,123 @@
+"""Helpers that run the CUDA path through the C ABI and compare it with the CPU
+oracle on the same inputs.
+
+Tolerance of the gate (floating point): logits agree within 1e-2 relative,
+with an absolute floor of 1e-2 for logits of magnitude below 1
+(|gpu - oracle| <= 1e-2 * max(|oracle|, 1)).  The kernel accumulates bf16
+products in fp32 over H terms; for these inputs (|logit| ~ 1-3) its error is
+orders of magnitude below that bound, which is the one the method's
+description states.  Top-k ids may differ from the oracle's only between
+near-ties: the oracle logit of the kernel's j-th id must be within the same
+tolerance of the oracle logit of the oracle's j-th id, for every j.
+
+Integer stages are compared bit for bit, each on the kernel's own inputs
+(the kernel's ids go into the oracle's count, its counts into the oracle's
+plan, and so on), so a logit near-tie upstream never excuses a difference
+downstream.
+"""
+import numpy as np
+import torch
+
+import oracle
+from moe_expert_load_bf16_b200 import _lib, workloads
+
+TOL = 1e-2
+
+
+def gate_check(h, w, bias, k, ids_gpu, logits_gpu=None, rows=None):
+    """h [T,H] bf16 tensor, w [E,H], bias [E] or None; ids_gpu [T,k] tensor.
+    Returns (max_rel_err, n_id_mismatch_rows)."""
+    T = h.shape[0]
+    rows = np.arange(T) if rows is None else np.asarray(rows)
+    hb = workloads.bf16_bits(h)[rows]
+    wb = workloads.bf16_bits(w)
+    b = None if bias is None else bias.detach().cpu().numpy()
+    o_logits, o_ids = oracle.gate(hb, wb, b, k)
+    g_ids = ids_gpu.detach().cpu().numpy()[rows]
+    max_err = 0.0
+    if logits_gpu is not None:
+        g_logits = logits_gpu.detach().cpu().numpy()[rows]
+        err = np.abs(g_logits.astype(np.float64) - o_logits) / np.maximum(np.abs(o_logits), 1.0)
+        max_err = float(err.max()) if err.size else 0.0
+        assert max_err <= TOL, f"logit error {max_err}"
+    mism = 0
+    for r in range(len(rows)):
+        if np.array_equal(g_ids[r], o_ids[r]):
+            continue
+        mism += 1
+        assert len(set(g_ids[r].tolist())) == k, f"row {rows[r]}: repeated id {g_ids[r]}"
+        ol = o_logits[r]
+        for j in range(k):
+            a, c = ol[g_ids[r, j]], ol[o_ids[r, j]]
+            assert abs(a - c) <= TOL * max(abs(c), 1.0), (
+                f"row {rows[r]}: id {g_ids[r, j]} vs {o_ids[r, j]} at rank {j} (logits {a} vs {c})")
+    return max_err, mism
+
+
+def plan_check(cnt_np, plan_dec, N, L):
+    """Kernel plan (decoded) vs the oracle's plan of the same counts: bit-exact."""
+    p = oracle.plan(cnt_np, N, L)
+    for f in ("holds", "used", "slots", "slot_phase"):
+        assert np.array_equal(plan_dec[f], getattr(p, f)), f
+    assert np.array_equal(plan_dec["plan_load"].astype(np.int64), p.plan_load), "plan_load"
+    for f in ("edge_u", "edge_v", "edge_e", "edge_round", "round_ptr"):
+        assert np.array_equal(plan_dec[f], getattr(p, f)), f
+    assert plan_dec["n_edges"] == p.n_edges and plan_dec["n_rounds"] == p.n_rounds
+    assert plan_dec["n_phase1"] == int((p.slot_phase == 1).sum())
+    assert plan_dec["n_phase2"] == int((p.slot_phase == 2).sum())
+    # per-expert CSR: edges of e by ascending replica rank
+    E = cnt_np.shape[1]
+    for e in range(E):
+        js = plan_dec["rep_edge"][plan_dec["rep_ptr"][e]:plan_dec["rep_ptr"][e + 1]]
+        assert all(plan_dec["edge_e"][j] == e for j in js)
+        assert list(plan_dec["edge_v"][js]) == sorted(plan_dec["edge_v"][js])
+    return p
+
+
+def split_check(cnt_np, p, tok, mass, loads, passes_run, passes):
+    s = oracle.split(cnt_np, p, passes)
+    ne = p.n_edges
+    assert np.array_equal(tok[:ne], s.tok), "tok"
+    assert np.array_equal(mass[:ne], s.mass), "mass"
+    assert (tok[ne:] == 0).all() and (mass[ne:] == 0).all()
+    assert np.array_equal(loads.astype(np.int64), s.loads), "loads"
+    assert int(passes_run) == s.passes_run, "passes_run"
+    return s
+
+
+def assign_check(ids_np, p, s, G, E, dest, perm, offs):
+    d, pm, of = oracle.assign(ids_np, p, s, G, E)
+    assert np.array_equal(dest, d), "dest"
+    assert np.array_equal(perm, pm), "perm"
+    assert np.array_equal(offs, of), "offs"
+
+
+def check_path(path, b, passes, ids_pred=None):
+    """Integer stages of problem b of a DecisionPath against the oracle."""
+    G, E, N, L = path.G, path.E, path.N, path.L
+    ids_pred = path.ids_pred[b] if ids_pred is None else ids_pred
+    ip = ids_pred.cpu().numpy()
+    cnt_pred = path.cnt_pred[b].cpu().numpy()
+    assert np.array_equal(cnt_pred, oracle.count(ip, G, E)), "cnt_pred"
+    dec = _lib.decode_plan(path.plan[b], G, E, N)[0]
+    p = plan_check(cnt_pred, dec, N, L)
+    ids = path.ids[b].cpu().numpy()
+    cnt = path.cnt[b].cpu().numpy()
+    assert np.array_equal(cnt, oracle.count(ids, G, E)), "cnt"
+    s = split_check(cnt, p, path.tok[b].cpu().numpy(), path.mass[b].cpu().numpy(),
+                    path.loads[b].cpu().numpy(), path.passes_run[b].item(), passes)
+    assign_check(ids, p, s, G, E, path.dest[b].cpu().numpy(), path.perm[b].cpu().numpy(),
+                 path.offs[b].cpu().numpy())
+    return p, s
+
+
+def model_inputs(w: workloads.Workload, layers, device, T=None):
+    """hidden [layers+1, T, H] (slot 0 = h_0 again, the lookahead input of
+    layer 0), weights [layers, E, H], bias [layers, E] on `device`."""
+    T = w.T if T is None else T
+    hid = torch.empty(layers + 1, T, w.H, dtype=torch.bfloat16, device=device)
+    workloads.hidden_chain(w, layers, T=T, out=hid[1:])
+    hid[0].copy_(hid[1])
+    W = workloads.gate_weights(w, layers, device=device)
+    bias = workloads.biases(w, layers).to(device)
+    return hid, W, bias

@@ -1,0 +1,75 @@
+"""The C-ABI library loads and exports every symbol include/lb.h declares
+(CPU only: no compute call, only host-side functions and argument checks)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from moe_expert_load_bf16_b200 import _lib, build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "lb.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return _lib._load()
+
+
+def declared():
+    src = open(HEADER).read()
+    return sorted(set(re.findall(r"^\s*(?:int|size_t|const char \*)\s*(lb_\w+)\s*\(", src, re.M)))
+
+
+def test_header_declares_the_five_steps():
+    names = declared()
+    for n in ("lb_predict_topk", "lb_count", "lb_plan_replicas", "lb_split", "lb_assign"):
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for n in declared():
+        assert hasattr(lib, n), n
+        assert n in _lib.EXPORTS, n
+
+
+def test_host_only_functions(lib):
+    assert lib.lb_version() == 100
+    assert lib.lb_strerror(_lib.LB_EINVAL) == b"invalid argument"
+    nb = _lib.lb_plan_bytes(64, 256, 2)
+    assert nb % 256 == 0
+    lay = _lib.plan_layout(64, 256, 2)
+    offs = [lay[k] for k in ("hdr", "used", "slots", "slot_phase", "plan_load", "edge_u", "edge_v", "edge_e",
+                             "edge_round", "round_ptr", "rep_ptr", "rep_edge", "holds")]
+    assert offs == sorted(offs) and all(o % 4 == 0 for o in offs)
+    assert lay["holds"] + 64 * 256 <= lay["total"] == nb
+    assert _lib.lb_assign_workspace_bytes(3, 100, 8, 8, 64, 2) % 256 == 0
+
+
+def test_arguments_rejected_before_any_launch(lib):
+    P = ctypes.c_void_p
+    s = P(0)
+    # nbatch = 0, E too large, k > E: rejected without touching the GPU
+    assert lib.lb_predict_topk(P(16), P(16), None, 0, 128, 64, 16, 2, P(16), None, s) == _lib.LB_EINVAL
+    assert lib.lb_predict_topk(P(16), P(16), None, 1, 128, 64, 300, 2, P(16), None, s) == _lib.LB_EINVAL
+    assert lib.lb_predict_topk(P(16), P(16), None, 1, 128, 64, 4, 5, P(16), None, s) == _lib.LB_EINVAL
+    assert lib.lb_predict_topk(P(16), P(16), None, 1, 128, 60, 16, 2, P(16), None, s) == _lib.LB_EINVAL
+    assert lib.lb_count(P(16), 1, 10, 2, 16, 4, P(16), s) == _lib.LB_EINVAL          # T % G
+    assert lib.lb_plan_replicas(P(256), 1, 3, 16, 1, 0, P(256), s) == _lib.LB_EINVAL  # E % G
+    assert lib.lb_plan_replicas(P(256), 1, 4, 16, 20, 0, P(256), s) == _lib.LB_EINVAL  # N > E - E/G
+    assert lib.lb_plan_replicas(P(256), 1, 4, 16, 1, 2, P(256), s) == _lib.LB_EINVAL  # L > N
+    assert lib.lb_plan_replicas(P(256), 1, 128, 128, 1, 0, P(256), s) == _lib.LB_EINVAL  # G > 64
+    assert lib.lb_split(P(256), P(256), 1, 4, 16, 1, -1, P(16), P(16), P(16), P(16), s) == _lib.LB_EINVAL
+    assert lib.lb_assign(P(16), P(16), P(256), P(16), P(16), 1, 8, 2, 4, 16, 1, P(16), P(16), P(16), P(256),
+                         1, s) == _lib.LB_ENOSPACE
+    assert lib.lb_gate_tuning(3, 5) == _lib.LB_EINVAL
+    assert lib.lb_gate_tuning(0, 0) == _lib.LB_OK
+
+
+def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
+    monkeypatch.setattr(_lib, "_lib", None)
+    monkeypatch.setattr(_lib, "LIB_PATH", str(tmp_path / "missing.so"))
+    with pytest.raises(ImportError):
+        _lib._load()

@@ -1,0 +1,293 @@
+"""CUDA path vs the CPU oracle, through the C ABI (needs a B200)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import parity
+from moe_expert_load_bf16_b200 import _lib, workloads
+from moe_expert_load_bf16_b200.pipeline import DecisionPath
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+
+
+@pytest.fixture(autouse=True)
+def _clean_status():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    _lib.lb_gate_tuning(0, 0)
+    _lib.lb_get_status(clear=True)
+    yield
+    _lib.lb_gate_tuning(0, 0)
+
+
+def run_model(w, layers, passes=12, T=None, sample_rows=None):
+    hid, W, bias = parity.model_inputs(w, layers, DEV, T=T)
+    T = hid.shape[1]
+    path = DecisionPath(layers, T, w.H, w.E, w.k, w.G, w.N, w.L, passes=passes, device=DEV)
+    path.run(hid[:-1], hid[1:], W, bias)
+    torch.cuda.synchronize()
+    assert _lib.lb_get_status() == 0
+    return hid, W, bias, path
+
+
+@pytest.mark.parametrize("name", ["tiny", "tiny-p1"])
+def test_small_full_path(name):
+    w = workloads.WORKLOADS[name]
+    hid, W, bias, path = run_model(w, w.layers)
+    # gate: every row, both calls, with logits
+    for src, ids in ((hid[0], path.ids_pred[0]), (hid[1], path.ids[0])):
+        ids2, logits = _lib.lb_predict_topk(src, W[0], bias[0], w.k, want_logits=True)
+        assert torch.equal(ids2, ids)
+        parity.gate_check(src, W[0], bias[0], w.k, ids, logits)
+    parity.check_path(path, 0, 12)
+
+
+def test_olmoe_all_layers_as_benchmarked():
+    """The benchmark's launch configuration: all 16 OLMoE-shaped layers in one
+    batched pass; gate on sampled rows of every layer, integer stages exact."""
+    w = workloads.WORKLOADS["olmoe"]
+    hid, W, bias, path = run_model(w, w.layers)
+    rng = np.random.default_rng(0)
+    for l in range(w.layers):
+        rows = np.concatenate([rng.choice(w.T, 48, replace=False), [0, w.T - 1]])
+        parity.gate_check(hid[l + 1], W[l], bias[l], w.k, path.ids[l], rows=rows)
+        parity.gate_check(hid[l], W[l], bias[l], w.k, path.ids_pred[l], rows=rows)
+        parity.check_path(path, l, 12)
+
+
+def test_olmoe_one_layer_all_rows_with_logits():
+    w = workloads.WORKLOADS["olmoe"]
+    hid, W, bias = parity.model_inputs(w, 1, DEV)
+    ids, logits = _lib.lb_predict_topk(hid[1], W[0], bias[0], w.k, want_logits=True)
+    err, mism = parity.gate_check(hid[1], W[0], bias[0], w.k, ids, logits)
+    assert mism <= 8
+
+
+@pytest.mark.parametrize("name,layers", [("qwen3-30b", 2), ("qwen3-235b", 1)])
+def test_large_configs(name, layers):
+    w = workloads.WORKLOADS[name]
+    hid, W, bias, path = run_model(w, layers)
+    rng = np.random.default_rng(1)
+    rows = np.concatenate([rng.choice(w.T, 96, replace=False), [0, w.T - 1]])
+    for l in range(layers):
+        # one problem alone may take the cluster split of H (another fp32
+        # summation order than the batched call), so each is held to the oracle
+        ids, logits = _lib.lb_predict_topk(hid[l + 1], W[l], bias[l], w.k, want_logits=True)
+        parity.gate_check(hid[l + 1], W[l], bias[l], w.k, ids, logits, rows=rows)
+        parity.gate_check(hid[l + 1], W[l], bias[l], w.k, path.ids[l], rows=rows)
+        assert (ids == path.ids[l]).float().mean().item() > 0.999
+        parity.check_path(path, l, 12)
+
+
+@pytest.mark.parametrize("T", [64, 1024, 8192])
+def test_decode_steps(T):
+    """Decode sweep shape: plan from step 0, split + assign for several steps."""
+    w = workloads.WORKLOADS["decode"]
+    steps = [0, 1, 2, 3]
+    ids = workloads.decode_ids(w, T, steps).to(DEV)
+    path = DecisionPath(len(steps), T, w.H, w.E, w.k, w.G, w.N, w.L, device=DEV)
+    cnt0 = _lib.lb_count(ids[0], w.G, w.E)
+    _lib.lb_plan_replicas(cnt0, w.N, w.L, plan=path.plan[0:1])
+    path.plan[1:].copy_(path.plan[0:1].expand(len(steps) - 1, -1))
+    path.ids.copy_(ids)
+    path.ids_pred.copy_(ids[0:1].expand(len(steps), -1, -1))
+    path.cnt_pred.copy_(cnt0.unsqueeze(0).expand(len(steps), -1, -1))
+    path.solve()
+    torch.cuda.synchronize()
+    assert _lib.lb_get_status() == 0
+    for b in range(len(steps)):
+        parity.check_path(path, b, 12)
+
+
+@pytest.mark.parametrize("T", [64, 8192])
+def test_decode_gate(T):
+    """Gate at the decode shape (H=7168, E=256): the cluster split of H is
+    what runs at small T."""
+    w = workloads.WORKLOADS["decode"]
+    h = workloads.hidden_chain(w, 1, device=DEV, T=T)[0]
+    W = workloads.gate_weights(w, 1, device=DEV)[0]
+    bias = workloads.biases(w, 1)[0].to(DEV)
+    ids, logits = _lib.lb_predict_topk(h, W, bias, w.k, want_logits=True)
+    rows = np.arange(T) if T <= 256 else np.random.default_rng(2).choice(T, 128, replace=False)
+    parity.gate_check(h, W, bias, w.k, ids, logits, rows=rows)
+
+
+@pytest.mark.parametrize("T,H,E,k", [(200, 72, 60, 5), (1, 8, 16, 1), (333, 128, 256, 16), (130, 64, 17, 3),
+                                     (4096, 256, 128, 8), (96, 2048, 32, 2)])
+@pytest.mark.parametrize("split", [0, 1, 2, 4])
+def test_gate_shapes(T, H, E, k, split):
+    """Ragged token tails, E not a multiple of 16, H not a multiple of 64,
+    tiny and maximum k, every split of H."""
+    nkb = (H + 63) // 64
+    Epad = (E + 15) // 16 * 16
+    if split > nkb or (split and Epad % (4 * split) != 0):
+        pytest.skip("split not valid for this shape")
+    _lib.lb_gate_tuning(0, split)
+    g = torch.Generator(device=DEV).manual_seed(T * 7 + H + E + k)
+    h = torch.randn(T, H, generator=g, device=DEV).to(torch.bfloat16)
+    W = (torch.randn(E, H, generator=g, device=DEV) / H ** 0.5).to(torch.bfloat16)
+    bias = torch.randn(E, generator=g, device=DEV)
+    ids, logits = _lib.lb_predict_topk(h, W, bias, k, want_logits=True)
+    parity.gate_check(h, W, bias, k, ids, logits)
+    ids0 = _lib.lb_predict_topk(h, W, None, k)
+    parity.gate_check(h, W, None, k, ids0)
+
+
+@pytest.mark.parametrize("split", [2, 4, 8, 16])
+def test_gate_split_cluster(split):
+    """Forced split of H across clusters of 2..16 CTAs."""
+    _lib.lb_gate_tuning(0, split)
+    T, H, E, k = 300, 4096, 256, 8
+    g = torch.Generator(device=DEV).manual_seed(split)
+    h = torch.randn(T, H, generator=g, device=DEV).to(torch.bfloat16)
+    W = (torch.randn(E, H, generator=g, device=DEV) / H ** 0.5).to(torch.bfloat16)
+    ids, logits = _lib.lb_predict_topk(h, W, None, k, want_logits=True)
+    parity.gate_check(h, W, None, k, ids, logits)
+
+
+@pytest.mark.parametrize("stages", [2, 3, 5, 8])
+def test_gate_stages(stages):
+    _lib.lb_gate_tuning(stages, 1)
+    T, H, E, k = 512, 1024, 64, 8
+    g = torch.Generator(device=DEV).manual_seed(stages)
+    h = torch.randn(T, H, generator=g, device=DEV).to(torch.bfloat16)
+    W = (torch.randn(E, H, generator=g, device=DEV) / H ** 0.5).to(torch.bfloat16)
+    ids, logits = _lib.lb_predict_topk(h, W, None, k, want_logits=True)
+    parity.gate_check(h, W, None, k, ids, logits)
+
+
+def test_gate_ties_lower_id():
+    """Exactly equal logits: lower expert id first (identical weight rows)."""
+    T, H, E, k = 256, 128, 32, 6
+    g = torch.Generator(device=DEV).manual_seed(5)
+    h = torch.randn(T, H, generator=g, device=DEV).to(torch.bfloat16)
+    W = (torch.randn(E, H, generator=g, device=DEV) / H ** 0.5).to(torch.bfloat16)
+    W[7] = W[3]
+    W[20] = W[3]
+    W[9] = W[1]
+    ids = _lib.lb_predict_topk(h, W, None, k)
+    _, o_ids = oracle.gate(workloads.bf16_bits(h), workloads.bf16_bits(W), None, k)
+    got = ids.cpu().numpy()
+    for r in range(T):
+        row = list(got[r])
+        for lo, hi in ((3, 7), (3, 20), (7, 20), (1, 9)):
+            if lo in row and hi in row:
+                assert row.index(lo) < row.index(hi)
+    assert (got == o_ids).mean() > 0.99
+
+
+def test_integer_stages_random_shapes():
+    rng = np.random.default_rng(3)
+    for trial in range(12):
+        G = int(rng.choice([1, 2, 3, 4, 8, 16, 64]))
+        Eg = int(rng.choice([1, 2, 4, 8]))
+        E = G * Eg
+        if E > 512:
+            continue
+        k = int(rng.integers(1, min(E, 8) + 1))
+        T = G * int(rng.integers(0, 40))
+        N = int(rng.integers(0, min(4, E - Eg) + 1))
+        L = int(rng.integers(0, N + 1))
+        pr = rng.permutation(np.arange(1, E + 1)) ** -1.3
+        pr /= pr.sum()
+        ids_np = np.stack([rng.choice(E, k, replace=False, p=pr) for _ in range(T)]).astype(np.int32) \
+            if T else np.zeros((0, k), np.int32)
+        ids = torch.from_numpy(ids_np).to(DEV)
+        B = 2
+        path = DecisionPath(B, T, 8, E, k, G, N, L, device=DEV)
+        path.ids.copy_(ids.unsqueeze(0).expand(B, -1, -1))
+        # problem 1 plans on counts of a shuffled copy: different prediction
+        shuffled = ids_np[rng.permutation(T)] if T else ids_np
+        path.ids_pred[0].copy_(ids)
+        path.ids_pred[1].copy_(torch.from_numpy(np.ascontiguousarray(shuffled)).to(DEV))
+        _lib.lb_count(path.ids_pred, G, E, cnt=path.cnt_pred)
+        _lib.lb_plan_replicas(path.cnt_pred, N, L, plan=path.plan)
+        path.solve()
+        torch.cuda.synchronize()
+        assert _lib.lb_get_status() == 0
+        for b in range(B):
+            parity.check_path(path, b, 12)
+
+
+@pytest.mark.parametrize("passes", [0, 1, 2, 64])
+def test_split_pass_counts(passes):
+    w = workloads.WORKLOADS["qwen3-30b"]
+    ids = workloads.decode_ids(w.with_(T=2048), 2048, [0]).to(DEV)[0]
+    path = DecisionPath(1, 2048, 8, w.E, w.k, w.G, w.N, w.L, passes=passes, device=DEV)
+    path.ids_pred.copy_(ids)
+    path.ids.copy_(ids)
+    _lib.lb_count(path.ids_pred, w.G, w.E, cnt=path.cnt_pred)
+    _lib.lb_plan_replicas(path.cnt_pred, w.N, w.L, plan=path.plan)
+    path.solve()
+    torch.cuda.synchronize()
+    parity.check_path(path, 0, passes)
+
+
+def test_all_tokens_one_expert():
+    G, E, k, T, N, L = 8, 64, 1, 1024, 4, 2
+    ids = torch.zeros(T, k, dtype=torch.int32, device=DEV)
+    path = DecisionPath(1, T, 8, E, k, G, N, L, device=DEV)
+    path.ids_pred.copy_(ids)
+    path.ids.copy_(ids)
+    _lib.lb_count(path.ids_pred, G, E, cnt=path.cnt_pred)
+    _lib.lb_plan_replicas(path.cnt_pred, N, L, plan=path.plan)
+    path.solve()
+    torch.cuda.synchronize()
+    p, s = parity.check_path(path, 0, 12)
+    assert int(s.loads.max()) == oracle.split_optimum(path.cnt[0].cpu().numpy(), p)
+
+
+def test_empty_batch():
+    G, E, k, N, L = 4, 16, 2, 1, 0
+    path = DecisionPath(1, 0, 8, E, k, G, N, L, device=DEV)
+    _lib.lb_count(path.ids_pred, G, E, cnt=path.cnt_pred)
+    _lib.lb_plan_replicas(path.cnt_pred, N, L, plan=path.plan)
+    path.solve()
+    torch.cuda.synchronize()
+    assert (path.cnt == 0).all() and (path.offs == 0).all()
+    parity.check_path(path, 0, 12)
+
+
+def test_bad_ids_are_flagged_not_fatal():
+    G, E, k, T = 4, 16, 2, 64
+    ids = torch.randint(0, E, (T, k), dtype=torch.int32, device=DEV)
+    ids[:, 1] = (ids[:, 0] + 1) % E
+    ids[5, 0] = E + 3           # out of range
+    ids[9, 1] = ids[9, 0]       # repeated in a row
+    _lib.lb_count(ids, G, E)
+    flags = _lib.lb_get_status(clear=True)
+    assert flags & _lib.LB_DEV_BAD_IDS
+    # the context is still usable
+    ok = torch.ones(4, device=DEV).sum().item()
+    assert ok == 4.0
+
+
+def test_invalid_arguments_rejected():
+    h = torch.zeros(128, 64, dtype=torch.bfloat16, device=DEV)
+    W = torch.zeros(300, 64, dtype=torch.bfloat16, device=DEV)
+    with pytest.raises(_lib.LBError) as e:
+        _lib.lb_predict_topk(h, W, None, 8)       # E > 256
+    assert e.value.code == _lib.LB_EINVAL
+    ids = torch.zeros(10, 2, dtype=torch.int32, device=DEV)
+    with pytest.raises(_lib.LBError):
+        _lib.lb_count(ids, 4, 16)                 # T % G != 0
+    cnt = torch.zeros(3, 16, dtype=torch.int32, device=DEV)
+    with pytest.raises(_lib.LBError):
+        _lib.lb_plan_replicas(cnt, 1, 0)          # E % G != 0
+    assert _lib.lb_get_status() == 0
+
+
+def test_batched_equals_unbatched():
+    w = workloads.WORKLOADS["tiny-p1"].with_(layers=3)
+    hid, W, bias = parity.model_inputs(w, 3, DEV)
+    ids_b = _lib.lb_predict_topk(hid[1:], W, bias, w.k)
+    for l in range(3):
+        assert torch.equal(ids_b[l], _lib.lb_predict_topk(hid[l + 1], W[l], bias[l], w.k))
+    cnt_b = _lib.lb_count(ids_b, w.G, w.E)
+    plan_b = _lib.lb_plan_replicas(cnt_b, w.N, w.L)
+    for l in range(3):
+        assert torch.equal(cnt_b[l], _lib.lb_count(ids_b[l], w.G, w.E))
+        assert torch.equal(plan_b[l], _lib.lb_plan_replicas(cnt_b[l], w.N, w.L)[0])
