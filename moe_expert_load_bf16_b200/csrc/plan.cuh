@@ -331,6 +331,9 @@ __global__ void __launch_bounds__(THREADS)
         const int g = i / E, e = i - g * E;
         o_holds[i] = static_cast<uint8_t>((hold[e] >> g) & 1ull);
     }
+    // padding to the blob's 256-byte size: written too, so a blob is fully
+    // determined by its inputs
+    for (size_t i = LY.holds + static_cast<size_t>(G) * E + tid; i < LY.total; i += blockDim.x) blob[i] = 0;
 }
 
 }  // namespace plan
