@@ -202,6 +202,34 @@ int lb_assign(const int32_t *ids, const int32_t *cnt, const void *plan,
               void *workspace, size_t workspace_bytes, void *stream);
 
 /* ------------------------------------------------------------------------
+ * lb_assign without a caller workspace (the pages have no counterpart; this
+ * is a convenience of this library).
+ * For callers that cannot provide device scratch memory: a runtime whose
+ * device memory all belongs to its own arena, or a plain-C caller with no
+ * device allocator (cudaMalloc would also synchronize the device mid-step).
+ * Same arguments, outputs and limits as lb_assign, minus the workspace; the
+ * scratch is a fixed device array of LB_NOALLOC_SCRATCH_BYTES inside the
+ * library, which every GPU that loads the library holds until exit.
+ *   - Calls whose lb_assign_workspace_bytes(...) exceeds
+ *     LB_NOALLOC_SCRATCH_BYTES return LB_ENOSPACE (lb_last_error says why);
+ *     use lb_assign for those.
+ *   - It allocates nothing: no cudaMalloc, no cudaFree, no allocating
+ *     library routine.
+ *   - The first call on a device looks up the array's device address and
+ *     raises two kernels' shared-memory limits (once per device); make that
+ *     first call before any stream capture.
+ *   - All calls share the one array: calls that overlap on the GPU (for
+ *     example on two streams) race and give wrong results.  The scratch keeps
+ *     the last call's contents; every call fully rewrites what it reads, so
+ *     nothing needs clearing.
+ * ------------------------------------------------------------------------ */
+#define LB_NOALLOC_SCRATCH_BYTES (1u << 20)
+int lb_assign_noalloc(const int32_t *ids, const int32_t *cnt, const void *plan,
+                      const int32_t *tok, const int32_t *mass, int nbatch, int T, int k,
+                      int G, int E, int N, int32_t *dest, int32_t *perm, int32_t *offs,
+                      void *stream);
+
+/* ------------------------------------------------------------------------
  * Status and diagnostics (not from the pages).
  * lb_get_status: synchronizes the current device, writes the status word of
  * the current device to *flags (LB_DEV_* bits) and clears it when `clear`

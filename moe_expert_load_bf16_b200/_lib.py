@@ -55,13 +55,14 @@ def _load():
     lib.lb_assign_workspace_bytes.argtypes = [I, I, I, I, I, I]
     lib.lb_assign_workspace_bytes.restype = SZ
     lib.lb_assign.argtypes = [P, P, P, P, P, I, I, I, I, I, I, P, P, P, P, SZ, P]
+    lib.lb_assign_noalloc.argtypes = [P, P, P, P, P, I, I, I, I, I, I, P, P, P, P]
     lib.lb_get_status.argtypes = [ctypes.POINTER(ctypes.c_int32), I]
     lib.lb_strerror.argtypes = [I]
     lib.lb_strerror.restype = ctypes.c_char_p
     lib.lb_last_error.argtypes = []
     lib.lb_last_error.restype = ctypes.c_char_p
     for f in ("lb_predict_topk", "lb_gate_tuning", "lb_count", "lb_plan_layout_of", "lb_plan_replicas",
-              "lb_split", "lb_assign", "lb_get_status", "lb_version"):
+              "lb_split", "lb_assign", "lb_assign_noalloc", "lb_get_status", "lb_version"):
         getattr(lib, f).restype = ctypes.c_int
     _lib = lib
     return lib
@@ -237,6 +238,27 @@ def lb_assign(ids, cnt, plan, tok, mass, N, out=None, workspace=None):
     return dest, perm, offs
 
 
+def lb_assign_noalloc(ids, cnt, plan, tok, mass, N, out=None):
+    """lb_assign for callers that cannot provide device scratch memory: the
+    library uses its own fixed device array instead (see include/lb.h).
+    Output buffers are still the caller's; pass `out` to avoid allocating
+    them here.  Calls that overlap on the GPU race on the shared array."""
+    lib = _load()
+    ids, cnt = _batched(ids, 3), _batched(cnt, 3)
+    _need(ids, torch.int32, "ids")
+    _need(cnt, torch.int32, "cnt")
+    B, T, k = ids.shape
+    _, G, E = cnt.shape
+    dev = ids.device
+    if out is None:
+        out = (torch.empty(B, T, k, dtype=torch.int32, device=dev), torch.empty(B, T * k, dtype=torch.int32, device=dev),
+               torch.empty(B, G * E + 1, dtype=torch.int32, device=dev))
+    dest, perm, offs = out
+    _check("lb_assign_noalloc", lib.lb_assign_noalloc(_p(ids), _p(cnt), _p(plan), _p(tok), _p(mass), B, T, k, G, E,
+                                                      N, _p(dest), _p(perm), _p(offs), _stream()))
+    return dest, perm, offs
+
+
 # ------------------------------------------------------------------ status
 def lb_get_status(clear=True):
     """Synchronizes the device; returns the LB_DEV_* bits seen since the last clear."""
@@ -252,5 +274,6 @@ def lb_version():
 
 
 EXPORTS = ("lb_predict_topk", "lb_gate_tuning", "lb_count", "lb_plan_bytes", "lb_plan_layout_of",
-           "lb_plan_replicas", "lb_split", "lb_assign_workspace_bytes", "lb_assign", "lb_get_status",
+           "lb_plan_replicas", "lb_split", "lb_assign_workspace_bytes", "lb_assign", "lb_assign_noalloc",
+           "lb_get_status",
            "lb_strerror", "lb_last_error", "lb_version")

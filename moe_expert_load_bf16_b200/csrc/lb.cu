@@ -397,3 +397,105 @@ int lb_assign(const int32_t *ids, const int32_t *cnt, const void *plan, const in
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Allocation-free variant of lb_assign.
+//
+// Some callers cannot hand this library a device workspace: a serving
+// runtime that gave all device memory to its own arena at start-up, or a
+// plain-C host loop with no device allocator of its own (and cudaMalloc
+// would synchronize the device in the middle of a step).  For them the
+// scratch lives in a file-scope device array of fixed size instead.  Every
+// GPU that loads this library holds that array (LB_NOALLOC_SCRATCH_BYTES)
+// until the process exits.
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = LB_NOALLOC_SCRATCH_BYTES;
+static __device__ __align__(256) int32_t g_noalloc_scratch[kNoAllocScratchBytes / sizeof(int32_t)];
+
+constexpr int kMaxDevices = 256;
+std::mutex g_noalloc_mu;
+int32_t *g_noalloc_ptr[kMaxDevices] = {};
+
+// Device address of the scratch array on the current device (the array's
+// name in host code is only a host-side stand-in).  Looked up once per
+// device, together with the kernels' shared-memory limits.
+int32_t *noalloc_scratch() {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) {
+        cuda_fail(e, "cudaGetDevice");
+        return nullptr;
+    }
+    if (dev < 0 || dev >= kMaxDevices) {
+        std::snprintf(g_last_error, sizeof g_last_error, "device ordinal %d out of range", dev);
+        return nullptr;
+    }
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (g_noalloc_ptr[dev] == nullptr) {
+        void *p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (e != cudaSuccess) {
+            cuda_fail(e, "cudaGetSymbolAddress(scratch)");
+            return nullptr;
+        }
+        // Raise the limits to the largest shared-memory size these kernels
+        // accept, so this never lowers a limit another entry point relies on.
+        e = cudaFuncSetAttribute(assign::prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 224 * 1024);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(assign::scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     224 * 1024);
+        if (e != cudaSuccess) {
+            cuda_fail(e, "cudaFuncSetAttribute(noalloc)");
+            return nullptr;
+        }
+        g_noalloc_ptr[dev] = static_cast<int32_t *>(p);
+    }
+    return g_noalloc_ptr[dev];
+}
+
+}  // namespace
+
+extern "C" int lb_assign_noalloc(const int32_t *ids, const int32_t *cnt, const void *plan, const int32_t *tok,
+                                 const int32_t *mass, int nbatch, int T, int k, int G, int E, int N,
+                                 int32_t *dest, int32_t *perm, int32_t *offs, void *stream) {
+    if (nbatch < 1 || nbatch > 65535 || T < 0 || T % G != 0 || k < 1 || k > LB_MAX_K || !plan_shape_ok(G, E, N, 0))
+        return LB_EINVAL;
+    if (!cnt || !plan || !offs || !aligned(plan, 256)) return LB_EINVAL;
+    if (G * N > 0 && (!tok || !mass)) return LB_EINVAL;
+    if (T > 0 && (!ids || !dest || !perm)) return LB_EINVAL;
+    if (static_cast<long long>(T) * k * nbatch >= INT_MAX) return LB_EINVAL;
+    if (assign::scatter_smem_bytes(E) > 224 * 1024) return LB_EINVAL;
+    const size_t need = lb_assign_workspace_bytes(nbatch, T, k, G, E, N);
+    if (need > kNoAllocScratchBytes) {
+        std::snprintf(g_last_error, sizeof g_last_error,
+                      "lb_assign_noalloc needs %zu bytes of scratch, more than its fixed %zu; use lb_assign", need,
+                      kNoAllocScratchBytes);
+        return LB_ENOSPACE;
+    }
+    int32_t *scratch = noalloc_scratch();
+    if (scratch == nullptr) return LB_ECUDA;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    assign::Args a;
+    a.ids = ids;
+    a.cnt = cnt;
+    a.tok = tok;
+    a.mass = mass;
+    a.plan = static_cast<const uint8_t *>(plan);
+    a.plan_stride = plan::layout(G, E, N).total;
+    a.T = T;
+    a.k = k;
+    a.G = G;
+    a.E = E;
+    a.N = N;
+    a.dest = dest;
+    a.perm = perm;
+    a.offs = offs;
+    a.ws = scratch;
+    a.ws_stride = assign::ws_words(G, E, N);
+    assign::prep_kernel<<<nbatch, assign::PREP_THREADS, assign::prep_smem_bytes(E), s>>>(a);
+    if (launched("assign prep (noalloc)") != LB_OK) return LB_ECUDA;
+    if (T == 0) return LB_OK;
+    assign::scatter_kernel<<<dim3(G, nbatch), assign::SC_THREADS, assign::scatter_smem_bytes(E), s>>>(a);
+    return launched("assign scatter (noalloc)");
+}
