@@ -199,6 +199,10 @@ def run_ours(args, world, rank, local):
     ms_step = ms_total / args.steps
     assign_per_step = Lyr * T * k
     value = assign_per_step * world / (ms_step * 1e-3)
+    if args.lean:
+        return {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": ms_step, "lean": True,
+                "gpu_launches": path.LAUNCHES_PER_RUN * args.steps, "clocks": clk.summary()}
 
     # ---------------- dominant kernel: the gate (two launches per step)
     g_gate = torch.cuda.CUDAGraph()
@@ -428,6 +432,9 @@ def main():
     ap.add_argument("--config", default=DEFAULT_WORKLOAD)
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--lean", action="store_true",
+                    help="time the steps only (no gate-only loop, per-layer latencies, end-to-end or CPU "
+                         "baseline): the command used for ncu launch lists")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
