@@ -125,8 +125,10 @@ int lb_count(const int32_t *ids, int nbatch, int T, int k, int E, int G,
  *   cnt   int32 [nbatch, G, E] (predicted counts)
  *   plan  caller-allocated [nbatch] blobs of lb_plan_bytes(G,E,N) bytes each
  *         (output; layout below)
- * Limits: E % G == 0, G <= LB_MAX_G, E <= LB_MAX_E, G*E <= 24576,
- * 0 <= L <= N <= min(LB_MAX_N, E - E/G).
+ * Limits: E % G == 0, G <= LB_MAX_G, E <= LB_MAX_E, 0 <= L <= N <=
+ * min(LB_MAX_N, E - E/G), and the counts plus planning tables fit in one
+ * SM's shared memory (about G*E*4 + 32*G*N bytes <= 224 KB; every shape of
+ * the pages fits: G*E <= 32768 at N <= 16).
  * ------------------------------------------------------------------------ */
 size_t lb_plan_bytes(int G, int E, int N);
 int lb_plan_replicas(const int32_t *cnt, int nbatch, int G, int E, int N, int L,

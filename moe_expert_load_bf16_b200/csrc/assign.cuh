@@ -11,14 +11,15 @@
 //               (or q0 for a replicated expert's remote assignments, whose
 //               destination depends on their rank q among e's remote ones).
 // The prep kernel (one CTA per problem) computes these from cnt, plan and
-// split without reading the ids.  The scatter kernel (one CTA per (problem,
-// source block)) then needs only each assignment's rank among the earlier
-// assignments of the same expert in its block: warps take consecutive
-// 32-assignment steps with __match_any_sync ranks and per-warp counters in
-// shared memory, a per-expert scan across warps keeps block order, and each
-// assignment's slot is base + rank (plus the segment arithmetic for a
-// replicated expert).  Positions never come from atomics, so the permutation
-// is deterministic and stable.
+// split without reading the ids; counts and plan are staged in shared memory
+// first.  The scatter kernel (one CTA per (problem, source block)) then needs
+// only each assignment's rank among the earlier assignments of the same
+// expert in its block: warps take consecutive 32-assignment steps with
+// __match_any_sync ranks and per-warp counters in shared memory, a warp
+// shuffle scan across warps keeps block order, and each assignment's slot is
+// base + rank, or, for a replicated expert's remote assignment, a short walk
+// over the expert's replica segments (staged in shared memory).  Positions
+// never come from atomics, so the permutation is deterministic and stable.
 #pragma once
 #include "common.cuh"
 #include "plan.cuh"
@@ -29,7 +30,8 @@ namespace assign {
 constexpr int PREP_THREADS = 1024;
 constexpr int SC_THREADS = 1024;
 constexpr int SC_WARPS = SC_THREADS / 32;
-constexpr int SC_STEPS = 4;   // 32-assignment steps per warp per chunk
+constexpr int SC_STEPS = 8;   // 32-assignment steps per warp per chunk
+static_assert(SC_WARPS == 32, "the cross-warp scan maps one warp's counts to one lane");
 
 // Workspace per problem (int32 words): base[G*E], seg_qoff[GN], seg_cum[GN],
 // seg_rep[GN]; rounded to 256 bytes.
@@ -38,13 +40,16 @@ __host__ __device__ inline size_t ws_words(int G, int E, int N) {
     return (w + 63) & ~static_cast<size_t>(63);
 }
 
-__host__ __device__ inline size_t prep_smem_bytes(int E) {
-    return static_cast<size_t>(E) * 8 + static_cast<size_t>(E) * 4 * 2;
+__host__ __device__ inline size_t prep_smem_bytes(int G, int E, int N) {
+    const size_t GN = static_cast<size_t>(G) * N;
+    return static_cast<size_t>(E) * 8 + static_cast<size_t>(G) * E * 4 * 2 + static_cast<size_t>(E) * 4 * 3 +
+           (static_cast<size_t>(E) + 1) * 4 + GN * 4 * 7 + 64;
 }
 
-__host__ __device__ inline size_t scatter_smem_bytes(int E) {
-    return static_cast<size_t>(E) * 8 + static_cast<size_t>(E) * 4 * 3 +
-           static_cast<size_t>(SC_WARPS) * E * 4 * 2;
+__host__ __device__ inline size_t scatter_smem_bytes(int G, int E, int N) {
+    const size_t GN = static_cast<size_t>(G) * N;
+    return static_cast<size_t>(E) * 8 + static_cast<size_t>(E) * 4 * 3 + (static_cast<size_t>(E) + 1) * 4 +
+           static_cast<size_t>(SC_WARPS) * (E + 1) * 4 * 2 + GN * 4 * 6 + 64;
 }
 
 struct Args {
@@ -62,8 +67,19 @@ __global__ void __launch_bounds__(PREP_THREADS) prep_kernel(const Args a) {
     extern __shared__ __align__(16) uint8_t sm[];
     const int G = a.G, E = a.E, N = a.N, GN = G * N, NK = G * E;
     uint64_t *hold = reinterpret_cast<uint64_t *>(sm);
-    int32_t *homeadd = reinterpret_cast<int32_t *>(hold + E);
+    int32_t *cnt_s = reinterpret_cast<int32_t *>(hold + E);
+    int32_t *homeadd = cnt_s + NK;
     int32_t *rcnt = homeadd + E;
+    int32_t *rtot = rcnt + E;
+    int32_t *rep_ptr = rtot + E;     // [E+1]
+    int32_t *rep_edge = rep_ptr + E + 1;
+    int32_t *ev = rep_edge + GN;
+    int32_t *ee = ev + GN;
+    int32_t *tk = ee + GN;
+    int32_t *ms = tk + GN;
+    int32_t *sq = ms + GN;           // segment start in q
+    int32_t *sc = sq + GN;           // mass of earlier segments
+    int32_t *osz = sc + GN;          // [NK] bucket sizes, then their exclusive scan
     __shared__ int wsum[PREP_THREADS / 32];
     __shared__ int bad;
 
@@ -73,12 +89,6 @@ __global__ void __launch_bounds__(PREP_THREADS) prep_kernel(const Args a) {
     const uint8_t *blob = a.plan + static_cast<size_t>(b) * a.plan_stride;
     const plan::Layout LY = plan::layout(G, E, N);
     const int32_t *hdr = reinterpret_cast<const int32_t *>(blob + LY.hdr);
-    const int32_t *p_ev = reinterpret_cast<const int32_t *>(blob + LY.edge_v);
-    const int32_t *p_ee = reinterpret_cast<const int32_t *>(blob + LY.edge_e);
-    const int32_t *rep_ptr = reinterpret_cast<const int32_t *>(blob + LY.rep_ptr);
-    const int32_t *rep_edge = reinterpret_cast<const int32_t *>(blob + LY.rep_edge);
-    const int32_t *tok = a.tok + static_cast<int64_t>(b) * GN;
-    const int32_t *mass = a.mass + static_cast<int64_t>(b) * GN;
     int32_t *offs = a.offs + static_cast<int64_t>(b) * (NK + 1);
     int32_t *base = a.ws + static_cast<size_t>(b) * a.ws_stride;
     int32_t *seg_qoff = base + NK;
@@ -89,143 +99,188 @@ __global__ void __launch_bounds__(PREP_THREADS) prep_kernel(const Args a) {
     if (tid == 0) bad = 0;
     if (ne < 0 || ne > GN) ne = 0;
 
-    for (int e = tid; e < E; e += blockDim.x) hold[e] = 1ull << (e / Eg);
-    __syncthreads();
-    for (int i = tid; i < ne; i += blockDim.x) {
-        const int e = p_ee[i], v = p_ev[i];
-        if (e >= 0 && e < E && v >= 0 && v < G)
-            atomicOr(reinterpret_cast<unsigned long long *>(&hold[e]), 1ull << v);
-        else
-            bad = 1;
+    // ---- stage inputs
+    LB_TICK(20);
+    stage_i32(cnt_s, cnt, NK);
+    {
+        const int32_t *p_ev = reinterpret_cast<const int32_t *>(blob + LY.edge_v);
+        const int32_t *p_ee = reinterpret_cast<const int32_t *>(blob + LY.edge_e);
+        const int32_t *p_rep_edge = reinterpret_cast<const int32_t *>(blob + LY.rep_edge);
+        const int32_t *p_rep_ptr = reinterpret_cast<const int32_t *>(blob + LY.rep_ptr);
+        const int32_t *tok = a.tok + static_cast<int64_t>(b) * GN;
+        const int32_t *mass = a.mass + static_cast<int64_t>(b) * GN;
+        for (int i = tid; i < ne; i += blockDim.x) {
+            ev[i] = p_ev[i];
+            ee[i] = p_ee[i];
+            rep_edge[i] = p_rep_edge[i];
+            tk[i] = tok[i];
+            ms[i] = mass[i];
+        }
+        for (int e = tid; e <= E; e += blockDim.x) rep_ptr[e] = p_rep_ptr[e];
     }
     __syncthreads();
 
-    // q0 (into base, temporarily), remote mass, replica segments
+    // ---- per expert: holders, remote mass, replica segments
     for (int e = tid; e < E; e += blockDim.x) {
-        const uint64_t hm = hold[e];
-        int run = 0;
-        for (int g = 0; g < G; ++g) {
-            base[g * E + e] = run;
-            if (!((hm >> g) & 1ull)) run += cnt[g * E + e];
-        }
+        const int h = e / Eg;
         int r0 = rep_ptr[e], r1 = rep_ptr[e + 1];
         if (r0 < 0 || r1 > ne || r1 < r0) {
             bad = 1;
             r0 = r1 = 0;
         }
-        rcnt[e] = r1 - r0;
+        uint64_t hm = 1ull << h;
         int qo = 0, cm = 0;
         for (int j = r0; j < r1; ++j) {
             const int i = rep_edge[j];
-            if (i < 0 || i >= ne) {
+            if (i < 0 || i >= ne || ee[i] != e || ev[i] < 0 || ev[i] >= G) {
                 bad = 1;
                 continue;
             }
-            seg_qoff[i] = qo;
-            seg_cum[i] = cm;
-            qo += tok[i];
-            cm += mass[i];
+            hm |= 1ull << ev[i];
+            sq[i] = qo;
+            sc[i] = cm;
+            qo += tk[i];
+            cm += ms[i];
         }
-        if (r1 > r0 && qo != run) bad = 1;
-        homeadd[e] = (r1 > r0) ? cm : run;
+        int R = 0;
+        for (int g = 0; g < G; ++g)
+            if (!((hm >> g) & 1ull)) R += cnt_s[g * E + e];
+        if (r1 > r0 && qo != R) bad = 1;
+        hold[e] = hm;
+        rcnt[e] = r1 - r0;
+        rtot[e] = R;
+        homeadd[e] = (r1 > r0) ? cm : R;
     }
     __syncthreads();
+    LB_TICK(21);
 
-    // bucket sizes over keys r*E+e, block-wide exclusive scan -> offs
-    const int per = (NK + blockDim.x - 1) / blockDim.x;
-    const int k0 = min(NK, tid * per), k1 = min(NK, k0 + per);
-    auto bucket = [&](int key) -> int {
-        const int r = key / E, e = key - r * E;
-        const int h = e / Eg;
-        int s = 0;
-        if ((hold[e] >> r) & 1ull) s += cnt[key];
-        if (r == h) {
-            s += homeadd[e];
-        } else if (((hold[e] >> r) & 1ull) && rcnt[e] > 0) {
-            for (int j = rep_ptr[e]; j < rep_ptr[e + 1]; ++j) {
-                const int i = rep_edge[j];
-                if (i >= 0 && i < ne && p_ev[i] == r) s += tok[i] - mass[i];
+    // ---- bucket sizes over keys r*E+e: own tokens of held experts, the home
+    // share of each expert, and every edge's replica share (tok - mass)
+    for (int r = warp; r < G; r += (blockDim.x >> 5)) {
+        for (int e = lane; e < E; e += 32) {
+            const uint64_t hm = hold[e];
+            int sz = ((hm >> r) & 1ull) ? cnt_s[r * E + e] : 0;
+            sz += (e >= r * Eg && e < (r + 1) * Eg) ? homeadd[e] : 0;
+            osz[r * E + e] = sz;
+        }
+    }
+    __syncthreads();
+    for (int i = tid; i < ne; i += blockDim.x) {
+        const int e = ee[i], v = ev[i];
+        if (e >= 0 && e < E && v >= 0 && v < G) osz[v * E + e] += tk[i] - ms[i];   // one edge per (v, e)
+    }
+    __syncthreads();
+    // block-wide exclusive scan, in place: warp w scans its contiguous
+    // segment of keys 32 at a time (conflict-free, coalesced), then the warp
+    // totals are scanned and added back; offs (global) gets a copy
+    {
+        const int nw = blockDim.x >> 5;
+        const int seg = ((NK + nw - 1) / nw + 31) & ~31;
+        const int s0 = min(NK, warp * seg), s1 = min(NK, s0 + seg);
+        int carry = 0;
+        for (int kb = s0; kb < s1; kb += 32) {
+            const int key = kb + lane;
+            const int x0 = key < s1 ? osz[key] : 0;
+            int x = x0;
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+                const int y = __shfl_up_sync(kFull, x, off);
+                if (lane >= off) x += y;
             }
+            if (key < s1) osz[key] = carry + x - x0;
+            carry += __shfl_sync(kFull, x, 31);
         }
-        return s;
-    };
-    int local = 0;
-    for (int key = k0; key < k1; ++key) local += bucket(key);
-    int incl = local;
+        if (lane == 0) wsum[warp] = carry;
+        __syncthreads();
+        if (warp == 0) {
+            const int c = lane < nw ? wsum[lane] : 0;
+            int x = c;
 #pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-        const int y = __shfl_up_sync(kFull, incl, off);
-        if (lane >= off) incl += y;
-    }
-    if (lane == 31) wsum[warp] = incl;
-    __syncthreads();
-    if (warp == 0) {
-        int x = lane < (blockDim.x >> 5) ? wsum[lane] : 0;
-#pragma unroll
-        for (int off = 1; off < 32; off <<= 1) {
-            const int y = __shfl_up_sync(kFull, x, off);
-            if (lane >= off) x += y;
+            for (int off = 1; off < 32; off <<= 1) {
+                const int y = __shfl_up_sync(kFull, x, off);
+                if (lane >= off) x += y;
+            }
+            if (lane < nw) wsum[lane] = x - c;   // exclusive per warp
+            if (lane == nw - 1) offs[NK] = x;
         }
-        if (lane < (blockDim.x >> 5)) wsum[lane] = x;   // inclusive per warp
+        __syncthreads();
+        const int add = wsum[warp];
+        for (int key = s0 + lane; key < s1; key += 32) {
+            const int o = osz[key] + add;
+            osz[key] = o;
+            offs[key] = o;
+        }
     }
     __syncthreads();
-    int run = (warp > 0 ? wsum[warp - 1] : 0) + incl - local;
-    for (int key = k0; key < k1; ++key) {
-        offs[key] = run;
-        run += bucket(key);
-    }
-    if (tid == blockDim.x - 1) offs[NK] = wsum[(blockDim.x >> 5) - 1];
-    __syncthreads();
+    LB_TICK(22);
 
-    // final base per (block g, expert e)
-    for (int key = tid; key < NK; key += blockDim.x) {
-        const int g = key / E, e = key - g * E;
+    // ---- base per (block g, expert e): thread per expert, g ascending with
+    // the running remote prefix q0 and a cursor into the expert's replica
+    // edges (ordered by ascending replica rank)
+    for (int e = tid; e < E; e += blockDim.x) {
         const int h = e / Eg;
-        const int q0 = base[key];
-        const int r0 = rep_ptr[e], r1 = rcnt[e] > 0 ? rep_ptr[e + 1] : r0;
-        int out;
-        if ((hold[e] >> g) & 1ull) {
-            int before = 0;
-            if (g == h) {
-                if (r1 == r0) {
-                    before = q0;
+        const uint64_t hm = hold[e];
+        const int r0 = rep_ptr[e], m = rcnt[e];
+        int j = r0;
+        int q0 = 0;
+        for (int g = 0; g < G; ++g) {
+            int out;
+            if ((hm >> g) & 1ull) {
+                int before = 0;
+                if (g == h) {
+                    if (m == 0) {
+                        before = q0;
+                    } else {
+                        for (int jj = r0; jj < r0 + m; ++jj) {
+                            const int i = rep_edge[jj];
+                            if (i >= 0 && i < ne) before += clampi(q0 - sq[i], 0, ms[i]);
+                        }
+                    }
                 } else {
-                    for (int j = r0; j < r1; ++j) {
+                    while (j < r0 + m && !(rep_edge[j] >= 0 && rep_edge[j] < ne && ev[rep_edge[j]] >= g)) ++j;
+                    if (j < r0 + m) {
                         const int i = rep_edge[j];
-                        if (i >= 0 && i < ne) before += clampi(q0 - seg_qoff[i], 0, mass[i]);
+                        if (ev[i] == g) before = clampi(q0 - sq[i] - ms[i], 0, tk[i] - ms[i]);
                     }
                 }
+                out = osz[g * E + e] + before;
+            } else if (m == 0) {
+                out = osz[h * E + e] + (h < g ? cnt_s[h * E + e] : 0) + q0;
             } else {
-                for (int j = r0; j < r1; ++j) {
-                    const int i = rep_edge[j];
-                    if (i >= 0 && i < ne && p_ev[i] == g)
-                        before = clampi(q0 - seg_qoff[i] - mass[i], 0, tok[i] - mass[i]);
-                }
+                out = q0;
             }
-            out = offs[key] + before;
-        } else if (r1 == r0) {
-            out = offs[h * E + e] + (h < g ? cnt[h * E + e] : 0) + q0;
-        } else {
-            out = q0;
+            base[g * E + e] = out;
+            if (!((hm >> g) & 1ull)) q0 += cnt_s[g * E + e];
         }
-        base[key] = out;
     }
     for (int i = tid; i < ne; i += blockDim.x) {
-        const int e = p_ee[i], v = p_ev[i];
-        seg_rep[i] = (e >= 0 && e < E && v >= 0 && v < G) ? offs[v * E + e] : 0;
+        const int e = ee[i], v = ev[i];
+        seg_qoff[i] = sq[i];
+        seg_cum[i] = sc[i];
+        seg_rep[i] = (e >= 0 && e < E && v >= 0 && v < G) ? osz[v * E + e] : 0;
     }
+    __syncthreads();
+    LB_TICK(23);
     if (tid == 0 && bad) flag(LB_DEV_BAD_SPLIT);
 }
 
 __global__ void __launch_bounds__(SC_THREADS) scatter_kernel(const Args a) {
     extern __shared__ __align__(16) uint8_t sm[];
     const int G = a.G, E = a.E, N = a.N, GN = G * N, NK = G * E, k = a.k;
+    const int EP = E + 1;   // padded row of the per-warp tables (no bank conflicts)
     uint64_t *hold = reinterpret_cast<uint64_t *>(sm);
     int32_t *rcnt = reinterpret_cast<int32_t *>(hold + E);
     int32_t *base_s = rcnt + E;
     int32_t *run = base_s + E;
-    int32_t *wcnt = run + E;                  // [SC_WARPS][E]
-    int32_t *pre = wcnt + SC_WARPS * E;       // [SC_WARPS][E]
+    int32_t *rep_ptr = run + E;          // [E+1]
+    int32_t *wcnt = rep_ptr + E + 1;     // [SC_WARPS][EP]
+    int32_t *pre = wcnt + SC_WARPS * EP; // [SC_WARPS][EP]
+    int32_t *s_qoff = pre + SC_WARPS * EP;   // per-expert CSR position j
+    int32_t *s_tok = s_qoff + GN;
+    int32_t *s_mass = s_tok + GN;
+    int32_t *s_home = s_mass + GN;
+    int32_t *s_rep = s_home + GN;
+    int32_t *s_v = s_rep + GN;
     __shared__ int bad;
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -235,9 +290,8 @@ __global__ void __launch_bounds__(SC_THREADS) scatter_kernel(const Args a) {
     const plan::Layout LY = plan::layout(G, E, N);
     const int32_t *hdr = reinterpret_cast<const int32_t *>(blob + LY.hdr);
     const int32_t *p_ev = reinterpret_cast<const int32_t *>(blob + LY.edge_v);
-    const int32_t *p_ee = reinterpret_cast<const int32_t *>(blob + LY.edge_e);
-    const int32_t *rep_ptr = reinterpret_cast<const int32_t *>(blob + LY.rep_ptr);
-    const int32_t *rep_edge = reinterpret_cast<const int32_t *>(blob + LY.rep_edge);
+    const int32_t *p_rep_ptr = reinterpret_cast<const int32_t *>(blob + LY.rep_ptr);
+    const int32_t *p_rep_edge = reinterpret_cast<const int32_t *>(blob + LY.rep_edge);
     const int32_t *tok = a.tok + static_cast<int64_t>(b) * GN;
     const int32_t *mass = a.mass + static_cast<int64_t>(b) * GN;
     const int32_t *offs = a.offs + static_cast<int64_t>(b) * (NK + 1);
@@ -256,24 +310,48 @@ __global__ void __launch_bounds__(SC_THREADS) scatter_kernel(const Args a) {
     int ne = hdr[0];
     if (ne < 0 || ne > GN) ne = 0;
 
+    // ---- stage: this block's bases, holder masks, replica segments
+    LB_TICK(10);
     if (tid == 0) bad = 0;
+    for (int e = tid; e <= E; e += blockDim.x) rep_ptr[e] = p_rep_ptr[e];
     for (int e = tid; e < E; e += blockDim.x) {
-        hold[e] = 1ull << (e / Eg);
-        const int r0 = rep_ptr[e], r1 = rep_ptr[e + 1];
-        rcnt[e] = (r0 < 0 || r1 > ne || r1 < r0) ? 0 : r1 - r0;
         base_s[e] = ws[g * E + e];
         run[e] = 0;
     }
     __syncthreads();
-    for (int i = tid; i < ne; i += blockDim.x) {
-        const int e = p_ee[i], v = p_ev[i];
-        if (e >= 0 && e < E && v >= 0 && v < G)
-            atomicOr(reinterpret_cast<unsigned long long *>(&hold[e]), 1ull << v);
+    for (int e = tid; e < E; e += blockDim.x) {
+        const int h = e / Eg;
+        int r0 = rep_ptr[e], r1 = rep_ptr[e + 1];
+        if (r0 < 0 || r1 > ne || r1 < r0) r0 = r1 = 0;
+        uint64_t hm = 1ull << h;
+        const int hb = offs[h * E + e] + (h < g ? cnt[h * E + e] : 0);
+        int mcount = 0;
+        for (int j = r0; j < r1; ++j) {
+            const int i = p_rep_edge[j];
+            const int v = (i >= 0 && i < ne) ? p_ev[i] : -1;
+            if (v < 0 || v >= G) {
+                s_tok[j] = 0;   // an empty segment: never matched
+                s_qoff[j] = 0;
+                continue;
+            }
+            hm |= 1ull << v;
+            s_qoff[j] = seg_qoff[i];
+            s_tok[j] = tok[i];
+            s_mass[j] = mass[i];
+            s_home[j] = hb + seg_cum[i];
+            s_rep[j] = seg_rep[i] + (v < g ? cnt[v * E + e] : 0);
+            s_v[j] = v;
+            ++mcount;
+        }
+        hold[e] = hm;
+        rcnt[e] = r1 - r0;
+        (void)mcount;
     }
     __syncthreads();
+    LB_TICK(11);
 
     constexpr int CH = SC_WARPS * 32 * SC_STEPS;
-    int32_t *wrow = wcnt + warp * E;
+    int32_t *wrow = wcnt + warp * EP;
     for (int cs = 0; cs < nitems; cs += CH) {
         for (int e = lane; e < E; e += 32) wrow[e] = 0;
         __syncwarp();
@@ -299,14 +377,19 @@ __global__ void __launch_bounds__(SC_THREADS) scatter_kernel(const Args a) {
             loc[s] = cur + rnk;
         }
         __syncthreads();
-        for (int e = tid; e < E; e += blockDim.x) {
-            int acc = run[e];
-            for (int w = 0; w < SC_WARPS; ++w) {
-                const int t = wcnt[w * E + e];
-                pre[w * E + e] = acc;
-                acc += t;
+        // per expert: exclusive scan of the warps' counts (warp order = f order)
+        for (int e = warp; e < E; e += SC_WARPS) {
+            const int c = wcnt[lane * EP + e];
+            int x = c;
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+                const int y = __shfl_up_sync(kFull, x, off);
+                if (lane >= off) x += y;
             }
-            run[e] = acc;
+            const int r = run[e];
+            pre[lane * EP + e] = r + x - c;
+            __syncwarp();
+            if (lane == 31) run[e] = r + x;
         }
         __syncthreads();
 #pragma unroll
@@ -314,36 +397,39 @@ __global__ void __launch_bounds__(SC_THREADS) scatter_kernel(const Args a) {
             const int e = es[s];
             if (e < 0) continue;
             const int i = cs + warp * 32 * SC_STEPS + s * 32 + lane;
-            const int rho = pre[warp * E + e] + loc[s];
-            const int h = e / Eg;
+            const int rho = pre[warp * EP + e] + loc[s];
             int d, p;
             if ((hold[e] >> g) & 1ull) {
                 d = g;
                 p = base_s[e] + rho;
             } else if (rcnt[e] == 0) {
-                d = h;
+                d = e / Eg;
                 p = base_s[e] + rho;
             } else {
                 const int q = base_s[e] + rho;
                 d = -1;
                 p = -1;
-                for (int j = rep_ptr[e]; j < rep_ptr[e] + rcnt[e]; ++j) {
-                    const int ei = rep_edge[j];
-                    if (ei < 0 || ei >= ne) break;
-                    const int qo = seg_qoff[ei];
-                    const int t = tok[ei];
-                    if (q < qo + t) {
-                        const int w = q - qo, mss = mass[ei];
+                // last segment starting at or before q (segment starts ascend)
+                int lo = rep_ptr[e], hi = lo + rcnt[e] - 1;
+                while (lo < hi) {
+                    const int mid = (lo + hi + 1) >> 1;
+                    if (s_qoff[mid] <= q) lo = mid; else hi = mid - 1;
+                }
+                // skip empty segments that start at q as well
+                while (lo < rep_ptr[e] + rcnt[e] - 1 && s_tok[lo] == 0 && s_qoff[lo + 1] <= q) ++lo;
+                {
+                    const int j = lo;
+                    const int qo = s_qoff[j];
+                    const int t = s_tok[j];
+                    if (rcnt[e] > 0 && q >= qo && q < qo + t) {
+                        const int w = q - qo, mss = s_mass[j];
                         if (w < mss) {
-                            d = h;
-                            p = offs[h * E + e] + (h < g ? cnt[h * E + e] : 0) + seg_cum[ei] + w;
+                            d = e / Eg;
+                            p = s_home[j] + w;
                         } else {
-                            const int v = p_ev[ei];
-                            if (v < 0 || v >= G) break;
-                            d = v;
-                            p = seg_rep[ei] + (v < g ? cnt[v * E + e] : 0) + (w - mss);
+                            d = s_v[j];
+                            p = s_rep[j] + (w - mss);
                         }
-                        break;
                     }
                 }
             }
@@ -355,8 +441,9 @@ __global__ void __launch_bounds__(SC_THREADS) scatter_kernel(const Args a) {
             dest[f] = d;
             perm[p] = static_cast<int32_t>(f);
         }
+        __syncthreads();   // pre/run are rewritten by the next chunk
     }
-    __syncthreads();
+    LB_TICK(12);
     if (tid == 0 && bad) flag(LB_DEV_BAD_SPLIT);
 }
 

@@ -17,6 +17,20 @@ __device__ int g_status;
 
 __device__ __forceinline__ void flag(int bits) { atomicOr(&g_status, bits); }
 
+// Phase timestamps of block 0 for latency analysis builds (-DLB_TIMING);
+// compiled out otherwise.
+#ifdef LB_TIMING
+__device__ long long g_ticks[64];
+#define LB_TICK(slot)                                                                          \
+    do {                                                                                       \
+        if (threadIdx.x == 0 && blockIdx.x == 0 && blockIdx.y == 0) lb::g_ticks[slot] = clock64(); \
+    } while (0)
+#else
+#define LB_TICK(slot) \
+    do {              \
+    } while (0)
+#endif
+
 // About one second at the B200's top SM clock: longer than any legitimate
 // wait inside one launch, short enough to keep a broken launch from hanging.
 constexpr long long kWaitCycles = 2000000000LL;
@@ -180,6 +194,40 @@ __device__ __forceinline__ float4 ld_cluster_f4(uint32_t addr) {
                  : "r"(addr)
                  : "memory");
     return v;
+}
+
+// ---------------------------------------------------------------- staging
+// Copy n int32 from global to shared memory with the whole CTA: 16-byte
+// loads when both sides are 16-byte aligned, four loads in flight per thread.
+__device__ __forceinline__ void stage_i32(int32_t *dst, const int32_t *__restrict__ src, int n) {
+    const int t = threadIdx.x, nt = blockDim.x;
+    if (((reinterpret_cast<uintptr_t>(dst) | reinterpret_cast<uintptr_t>(src)) & 15) == 0) {
+        const int n4 = n >> 2;
+        const int4 *s4 = reinterpret_cast<const int4 *>(src);
+        int4 *d4 = reinterpret_cast<int4 *>(dst);
+        int i = t;
+        for (; i + 3 * nt < n4; i += 4 * nt) {
+            const int4 a = __ldg(s4 + i), b = __ldg(s4 + i + nt), c = __ldg(s4 + i + 2 * nt),
+                       d = __ldg(s4 + i + 3 * nt);
+            d4[i] = a;
+            d4[i + nt] = b;
+            d4[i + 2 * nt] = c;
+            d4[i + 3 * nt] = d;
+        }
+        for (; i < n4; i += nt) d4[i] = __ldg(s4 + i);
+        for (int j = (n4 << 2) + t; j < n; j += nt) dst[j] = __ldg(src + j);
+    } else {
+        int i = t;
+        for (; i + 3 * nt < n; i += 4 * nt) {
+            const int a = __ldg(src + i), b = __ldg(src + i + nt), c = __ldg(src + i + 2 * nt),
+                      d = __ldg(src + i + 3 * nt);
+            dst[i] = a;
+            dst[i + nt] = b;
+            dst[i + 2 * nt] = c;
+            dst[i + 3 * nt] = d;
+        }
+        for (; i < n; i += nt) dst[i] = __ldg(src + i);
+    }
 }
 
 // ---------------------------------------------------------------- warp helpers

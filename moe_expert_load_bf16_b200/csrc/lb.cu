@@ -153,8 +153,9 @@ int launch_count_v(bool vec, const int32_t *ids, int nbatch, int T, int k, int E
 
 bool plan_shape_ok(int G, int E, int N, int L) {
     if (G < 1 || G > LB_MAX_G || E < 1 || E > LB_MAX_E || E % G != 0) return false;
-    if (static_cast<long long>(G) * E > 24576) return false;
     if (N < 0 || N > LB_MAX_N || N > E - E / G || L < 0 || L > N) return false;
+    // the planner stages the counts in shared memory; the split its tables
+    if (plan::smem_bytes(G, E, N) > 224 * 1024 || split::smem_bytes(G, E, N) > 224 * 1024) return false;
     return true;
 }
 
@@ -192,6 +193,14 @@ int lb_get_status(int32_t *flags, int clear) {
 }
 
 const char *lb_last_error(void) { return g_last_error; }
+
+#ifdef LB_TIMING
+int lb_debug_ticks(long long *out, int n) {
+    if (!out || n < 1 || n > 64) return LB_EINVAL;
+    if (cudaDeviceSynchronize() != cudaSuccess) return LB_ECUDA;
+    return cudaMemcpyFromSymbol(out, lb::g_ticks, sizeof(long long) * n) == cudaSuccess ? LB_OK : LB_ECUDA;
+}
+#endif
 
 int lb_gate_tuning(int stages, int split) {
     if (stages != 0 && (stages < 2 || stages > gate::MAX_STAGES)) return LB_EINVAL;
@@ -365,7 +374,8 @@ int lb_assign(const int32_t *ids, const int32_t *cnt, const void *plan, const in
     if (G * N > 0 && (!tok || !mass)) return LB_EINVAL;
     if (T > 0 && (!ids || !dest || !perm)) return LB_EINVAL;
     if (static_cast<long long>(T) * k * nbatch >= INT_MAX) return LB_EINVAL;
-    if (assign::scatter_smem_bytes(E) > 224 * 1024) return LB_EINVAL;
+    if (assign::scatter_smem_bytes(G, E, N) > 224 * 1024 || assign::prep_smem_bytes(G, E, N) > 224 * 1024)
+        return LB_EINVAL;
     if (workspace_bytes < lb_assign_workspace_bytes(nbatch, T, k, G, E, N)) return LB_ENOSPACE;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     assign::Args a;
@@ -385,7 +395,7 @@ int lb_assign(const int32_t *ids, const int32_t *cnt, const void *plan, const in
     a.offs = offs;
     a.ws = static_cast<int32_t *>(workspace);
     a.ws_stride = assign::ws_words(G, E, N);
-    const size_t sm1 = assign::prep_smem_bytes(E), sm2 = assign::scatter_smem_bytes(E);
+    const size_t sm1 = assign::prep_smem_bytes(G, E, N), sm2 = assign::scatter_smem_bytes(G, E, N);
     static SmemLimit lim1, lim2;
     if (!allow_smem(assign::prep_kernel, lim1, sm1, false) || !allow_smem(assign::scatter_kernel, lim2, sm2, false))
         return LB_ECUDA;
@@ -465,7 +475,8 @@ extern "C" int lb_assign_noalloc(const int32_t *ids, const int32_t *cnt, const v
     if (G * N > 0 && (!tok || !mass)) return LB_EINVAL;
     if (T > 0 && (!ids || !dest || !perm)) return LB_EINVAL;
     if (static_cast<long long>(T) * k * nbatch >= INT_MAX) return LB_EINVAL;
-    if (assign::scatter_smem_bytes(E) > 224 * 1024) return LB_EINVAL;
+    if (assign::scatter_smem_bytes(G, E, N) > 224 * 1024 || assign::prep_smem_bytes(G, E, N) > 224 * 1024)
+        return LB_EINVAL;
     const size_t need = lb_assign_workspace_bytes(nbatch, T, k, G, E, N);
     if (need > kNoAllocScratchBytes) {
         std::snprintf(g_last_error, sizeof g_last_error,
@@ -493,9 +504,9 @@ extern "C" int lb_assign_noalloc(const int32_t *ids, const int32_t *cnt, const v
     a.offs = offs;
     a.ws = scratch;
     a.ws_stride = assign::ws_words(G, E, N);
-    assign::prep_kernel<<<nbatch, assign::PREP_THREADS, assign::prep_smem_bytes(E), s>>>(a);
+    assign::prep_kernel<<<nbatch, assign::PREP_THREADS, assign::prep_smem_bytes(G, E, N), s>>>(a);
     if (launched("assign prep (noalloc)") != LB_OK) return LB_ECUDA;
     if (T == 0) return LB_OK;
-    assign::scatter_kernel<<<dim3(G, nbatch), assign::SC_THREADS, assign::scatter_smem_bytes(E), s>>>(a);
+    assign::scatter_kernel<<<dim3(G, nbatch), assign::SC_THREADS, assign::scatter_smem_bytes(G, E, N), s>>>(a);
     return launched("assign scatter (noalloc)");
 }

@@ -92,7 +92,8 @@ __global__ void __launch_bounds__(THREADS)
     const Layout LY = layout(G, E, N);
     const int Eg = E / G;
 
-    for (int i = tid; i < G * E; i += blockDim.x) cnt_s[i] = cnt[i];
+    LB_TICK(30);
+    stage_i32(cnt_s, cnt, G * E);
     for (int e = tid; e < E; e += blockDim.x) hold[e] = 1ull << (e / Eg);
     for (int i = tid; i < G * W; i += blockDim.x) busy[i] = 0ull;
     for (int i = tid; i < GN; i += blockDim.x) {
@@ -102,12 +103,13 @@ __global__ void __launch_bounds__(THREADS)
     if (tid < LB_MAX_G) used_s[tid] = 0;
     __syncthreads();
 
+    LB_TICK(31);
     // ---------------- phase 1: each rank imports its L most-requested foreign experts
     for (int g = warp; g < G; g += nwarps) {
         for (int pick = 0; pick < L; ++pick) {
             int bc = 0, be = 0x7fffffff;
             for (int e = lane; e < E; e += 32) {
-                if (e / Eg != g && !((hold[e] >> g) & 1ull)) {
+                if ((e < g * Eg || e >= (g + 1) * Eg) && !((hold[e] >> g) & 1ull)) {
                     const int c = cnt_s[g * E + e];
                     if (c > bc) {
                         bc = c;
@@ -129,6 +131,7 @@ __global__ void __launch_bounds__(THREADS)
     }
     __syncthreads();
 
+    LB_TICK(32);
     // ---------------- load model
     for (int e = tid; e < E; e += blockDim.x) {
         const uint64_t hm = hold[e];
@@ -140,15 +143,15 @@ __global__ void __launch_bounds__(THREADS)
     __syncthreads();
     for (int r = warp; r < G; r += nwarps) {
         int x = 0;
-        for (int e = lane; e < E; e += 32) {
+        for (int e = lane; e < E; e += 32)
             if ((hold[e] >> r) & 1ull) x += cnt_s[r * E + e];
-            if (e / Eg == r) x += m[e];
-        }
+        for (int e = r * Eg + lane; e < (r + 1) * Eg; e += 32) x += m[e];
         x = __reduce_add_sync(kFull, x);
         if (lane == 0) load_s[r] = x;
     }
     __syncthreads();
 
+    LB_TICK(33);
     // ---------------- phase 2: sequential greedy, one warp
     if (warp == 0) {
         const bool ha = lane < G, hb = lane + 32 < G;
@@ -164,42 +167,44 @@ __global__ void __launch_bounds__(THREADS)
             const uint64_t freem = static_cast<uint64_t>(__ballot_sync(kFull, ha && ua < N)) |
                                    (static_cast<uint64_t>(__ballot_sync(kFull, hb && ub < N)) << 32);
             int bm = 0, be = 0x7fffffff;
-            for (int e = u * Eg + lane; e < (u + 1) * Eg; e += 32) {
+            for (int q = lane; q < Eg; q += 32) {
+                const int e = u * Eg + q;
                 const int me = m[e];
-                if (me > bm && (~hold[e] & freem) != 0ull) {
-                    bm = me;
-                    be = e;
-                }
+                const bool ok = me > bm && (~hold[e] & freem) != 0ull;
+                bm = ok ? me : bm;
+                be = ok ? e : be;
             }
             const int mm = __reduce_max_sync(kFull, bm);
             if (mm <= 0) break;
             const int ce = __reduce_min_sync(kFull, bm == mm ? be : 0x7fffffff);
-            const uint64_t V = ~hold[ce] & freem;
+            const uint64_t hce = hold[ce];
+            const int mce = m[ce];
+            const uint64_t V = ~hce & freem;
             const bool ea = (V >> lane) & 1ull, eb = (V >> (lane + 32)) & 1ull;
             const int mn = __reduce_min_sync(kFull, min(ea ? la : INT_MAX, eb ? lb : INT_MAX));
             const unsigned bva = __ballot_sync(kFull, ea && la == mn);
             const unsigned bvb = __ballot_sync(kFull, eb && lb == mn);
             const int v = bva ? __ffs(bva) - 1 : 32 + __ffs(bvb) - 1;
             const int c = cnt_s[v * E + ce];
-            const int mr = m[ce] - c;
+            const int mr = mce - c;
             const int lu = mx - c, lv = mn + c;
             const int gap = lu - lv;
-            int d = gap > 0 ? (gap >> 1) : 0;
-            d = min(d, mr);
+            const int d = min(gap > 0 ? (gap >> 1) : 0, mr);
             if (c + d == 0) break;
             const int used_v = __shfl_sync(kFull, v < 32 ? ua : ub, v & 31);
             if (lane == 0) {
-                hold[ce] |= 1ull << v;
+                hold[ce] = hce | (1ull << v);
                 slots[v * N + used_v] = ce;
                 phase[v * N + used_v] = 2;
                 m[ce] = mr - d;
             }
-            if (lane == (u & 31)) {
-                if (u < 32) la = lu - d; else lb = lu - d;
-            }
-            if (lane == (v & 31)) {
-                if (v < 32) { la = lv + d; ua += 1; } else { lb = lv + d; ub += 1; }
-            }
+            const bool own_u = lane == (u & 31), own_v = lane == (v & 31);
+            la = (own_u && u < 32) ? lu - d : la;
+            lb = (own_u && u >= 32) ? lu - d : lb;
+            la = (own_v && v < 32) ? lv + d : la;
+            lb = (own_v && v >= 32) ? lv + d : lb;
+            ua += (own_v && v < 32) ? 1 : 0;
+            ub += (own_v && v >= 32) ? 1 : 0;
             ++np2;
             __syncwarp();
         }
@@ -209,6 +214,7 @@ __global__ void __launch_bounds__(THREADS)
     }
     __syncthreads();
 
+    LB_TICK(34);
     // ---------------- edges: expert ascending, replica rank ascending
     if (warp == 0) {
         int carry = 0;
@@ -245,8 +251,43 @@ __global__ void __launch_bounds__(THREADS)
     }
     __syncthreads();
 
-    // ---------------- greedy colouring and stable order by round (one thread)
-    if (tid == 0) {
+    LB_TICK(35);
+    // ---------------- greedy colouring, edge order: one warp, each rank's
+    // busy-round mask (rounds 0..127) in registers of lane (rank & 31)
+    __shared__ int overflow_s;
+    if (warp == 0) {
+        uint64_t a0 = 0, a1 = 0, b0 = 0, b1 = 0;   // ranks lane and lane+32
+        int nr = 0, overflow = 0;
+        for (int i = 0; i < ne; ++i) {
+            const int u = eu[i], v = ev[i];
+            const uint64_t mu0 = __shfl_sync(kFull, u < 32 ? a0 : b0, u & 31);
+            const uint64_t mu1 = __shfl_sync(kFull, u < 32 ? a1 : b1, u & 31);
+            const uint64_t mv0 = __shfl_sync(kFull, v < 32 ? a0 : b0, v & 31);
+            const uint64_t mv1 = __shfl_sync(kFull, v < 32 ? a1 : b1, v & 31);
+            const uint64_t f0 = ~(mu0 | mv0), f1 = ~(mu1 | mv1);
+            const int c = f0 ? __ffsll(static_cast<long long>(f0)) - 1
+                             : (f1 ? 64 + __ffsll(static_cast<long long>(f1)) - 1 : -1);
+            if (c < 0) {
+                overflow = 1;
+                break;
+            }
+            const uint64_t w0 = c < 64 ? (1ull << c) : 0ull, w1 = c >= 64 ? (1ull << (c - 64)) : 0ull;
+            const bool own_u = lane == (u & 31), own_v = lane == (v & 31);
+            a0 |= (own_u && u < 32) || (own_v && v < 32) ? w0 : 0ull;
+            a1 |= (own_u && u < 32) || (own_v && v < 32) ? w1 : 0ull;
+            b0 |= (own_u && u >= 32) || (own_v && v >= 32) ? w0 : 0ull;
+            b1 |= (own_u && u >= 32) || (own_v && v >= 32) ? w1 : 0ull;
+            if (lane == 0) er[i] = c;
+            nr = max(nr, c + 1);
+        }
+        if (lane == 0) {
+            n_rounds_s = nr;
+            overflow_s = overflow;
+        }
+    }
+    __syncthreads();
+    if (overflow_s && tid == 0) {
+        // more than 128 rounds: the same greedy colouring with W-word masks
         int nr = 0;
         for (int i = 0; i < ne; ++i) {
             const int u = eu[i], v = ev[i];
@@ -263,18 +304,45 @@ __global__ void __launch_bounds__(THREADS)
             er[i] = c;
             nr = max(nr, c + 1);
         }
-        for (int r = 0; r <= nr; ++r) rptr[r] = 0;
-        for (int i = 0; i < ne; ++i) rptr[er[i] + 1] += 1;
-        for (int r = 0; r < nr; ++r) {
-            rptr[r + 1] += rptr[r];
-            rfill[r] = rptr[r];
-        }
-        for (int i = 0; i < ne; ++i) pos[i] = rfill[er[i]]++;
         n_rounds_s = nr;
+    }
+    __syncthreads();
+    {
+        // stable order by round: position = start of the round + earlier
+        // edges (in edge order) of the same round
+        const int nrr = n_rounds_s;
+        for (int r = tid; r <= nrr; r += blockDim.x) rfill[r] = 0;
+        __syncthreads();
+        for (int i = tid; i < ne; i += blockDim.x) atomicAdd(&rfill[er[i]], 1);
+        __syncthreads();
+        if (warp == 0) {
+            int carry = 0;
+            for (int base = 0; base < nrr; base += 32) {
+                const int r = base + lane;
+                int x = r < nrr ? rfill[r] : 0;
+                const int own = x;
+#pragma unroll
+                for (int off = 1; off < 32; off <<= 1) {
+                    const int y = __shfl_up_sync(kFull, x, off);
+                    if (lane >= off) x += y;
+                }
+                if (r < nrr) rptr[r] = carry + x - own;
+                carry += __shfl_sync(kFull, x, 31);
+            }
+            if (lane == 0) rptr[nrr] = carry;
+        }
+        __syncthreads();
+        for (int i = tid; i < ne; i += blockDim.x) {
+            const int r = er[i];
+            int before = 0;
+            for (int j = 0; j < i; ++j) before += er[j] == r;
+            pos[i] = rptr[r] + before;
+        }
     }
     __syncthreads();
     const int nr = n_rounds_s;
 
+    LB_TICK(36);
     // ---------------- write the blob
     int32_t *hdr = reinterpret_cast<int32_t *>(blob + LY.hdr);
     if (tid == 0) {
@@ -327,13 +395,13 @@ __global__ void __launch_bounds__(THREADS)
     int32_t *o_rep_ptr = reinterpret_cast<int32_t *>(blob + LY.rep_ptr);
     for (int e = tid; e <= E; e += blockDim.x) o_rep_ptr[e] = eoff[e];
     uint8_t *o_holds = blob + LY.holds;
-    for (int i = tid; i < G * E; i += blockDim.x) {
-        const int g = i / E, e = i - g * E;
-        o_holds[i] = static_cast<uint8_t>((hold[e] >> g) & 1ull);
-    }
+    for (int g = warp; g < G; g += nwarps)
+        for (int e = lane; e < E; e += 32) o_holds[g * E + e] = static_cast<uint8_t>((hold[e] >> g) & 1ull);
     // padding to the blob's 256-byte size: written too, so a blob is fully
     // determined by its inputs
     for (size_t i = LY.holds + static_cast<size_t>(G) * E + tid; i < LY.total; i += blockDim.x) blob[i] = 0;
+    __syncthreads();
+    LB_TICK(37);
 }
 
 }  // namespace plan

@@ -1,15 +1,23 @@
 // Step 4: the per-step split (Relief, Methodology, Algorithm 1; The Per-Step
 // Optimum Problem for the edge/weight structure).
 //
-// One CTA per problem.  Setup is parallel (remote mass per expert, rank
-// loads by warp reductions, equal integer partition of each replicated
-// expert's remote mass over its edges).  The passes run in one warp: a round
-// is rank-disjoint, so with G <= 64 it has at most 32 transfers, one per
-// lane; the load table lives in shared memory, every transfer of a round
-// reads and writes its two entries with no atomics, and __syncwarp commits
-// the round so the next one reads what it wrote (Gauss-Seidel).  A pass that
-// moves nothing is a fixpoint, so the loop stops there with identical
-// results.
+// One CTA per problem.  Everything the split reads (counts, replica edges,
+// round schedule, per-expert edge lists) is first staged into shared memory
+// with coalesced loads, so no loop ever waits on L2.  Setup is one thread per
+// expert (holder mask, remote mass, equal integer partition of the remote
+// mass over the expert's edges) and one warp per rank (starting loads).
+//
+// The passes run in one warp with the load table in registers: lane j owns
+// ranks j and j+32.  A round of the schedule is rank-disjoint, so every rank
+// has at most one partner per round; a per-(round, rank) table built once
+// names it.  Both owners of a transfer fetch the other's load with one
+// shuffle and compute the same delta from the same (L[u], L[v], tok, mass),
+// so a round costs a shuffle and a few integer operations, with no shared
+// memory round trip on the dependency chain.  Each side keeps its own copy
+// of the edge's mass, so no two lanes write the same word.  A pass that moves
+// nothing is a fixpoint, so the loop stops there with identical results.
+// Schedules too long for the table fall back to one lane per transfer with
+// the loads in shared memory and __syncwarp between rounds.
 #pragma once
 #include "common.cuh"
 #include "plan.cuh"
@@ -17,159 +25,333 @@
 namespace lb {
 namespace split {
 
-constexpr int THREADS = 256;
+constexpr int THREADS = 512;
+
+// Rounds the per-(round, rank) transfer table holds (at most 96 KB of it,
+// 16 bytes per slot).
+__host__ __device__ inline int table_rounds(int G, int N) {
+    const int cap = (96 * 1024) / (16 * G);
+    return G * N < cap ? G * N : cap;
+}
+
+// Shared-memory carve-up of one problem's split.
+struct View {
+    uint64_t *hold;     // [E]   holder ranks of each expert (bit g)
+    int32_t *cnt;       // [G*E]
+    int32_t *R;         // [E]   remote mass
+    int32_t *rep_ptr;   // [E+1]
+    int32_t *rep_edge;  // [GN]
+    int32_t *eu, *ev, *ee;  // [GN] schedule order
+    int32_t *rptr;      // [GN+1]
+    int32_t *tk, *mu, *mv;  // [GN] tok, mass (home side), mass (replica side)
+    int4 *tab;          // [RC*G] (round, rank) slots: {code, tok, own-side mass, 0}
+    int32_t *Ls;        // [64]
+};
 
 __host__ __device__ inline size_t smem_bytes(int G, int E, int N) {
     const size_t GN = static_cast<size_t>(G) * N;
-    return static_cast<size_t>(E) * 8 + static_cast<size_t>(E) * 4 + GN * 4 * 4 + (GN + 1) * 4;
+    return static_cast<size_t>(E) * 8 + static_cast<size_t>(G) * E * 4 + static_cast<size_t>(E) * 4 +
+           (static_cast<size_t>(E) + 1) * 4 + GN * 4 * 7 + (GN + 1) * 4 +
+           static_cast<size_t>(table_rounds(G, N)) * G * 16 + 64 * 4 + 64;
 }
 
-__global__ void __launch_bounds__(THREADS)
-    split_kernel(const int32_t *__restrict__ cnt_all, const uint8_t *__restrict__ plan_all,
-                 size_t stride, int G, int E, int N, int passes, int32_t *__restrict__ tok_all,
-                 int32_t *__restrict__ mass_all, int32_t *__restrict__ loads_all,
-                 int32_t *__restrict__ passes_run_all) {
-    extern __shared__ __align__(16) uint8_t sm[];
+__device__ inline View carve(uint8_t *sm, int G, int E, int N) {
     const int GN = G * N;
-    uint64_t *hold = reinterpret_cast<uint64_t *>(sm);
-    int32_t *R = reinterpret_cast<int32_t *>(hold + E);
-    int32_t *eu = R + E;
-    int32_t *ev = eu + GN;
-    int32_t *tk = ev + GN;
-    int32_t *ms = tk + GN;
-    int32_t *rptr = ms + GN;
-    __shared__ int Ls[LB_MAX_G];
-    __shared__ int bad;
+    View v;
+    v.hold = reinterpret_cast<uint64_t *>(sm);
+    v.cnt = reinterpret_cast<int32_t *>(v.hold + E);
+    v.R = v.cnt + G * E;
+    v.rep_ptr = v.R + E;
+    v.rep_edge = v.rep_ptr + E + 1;
+    v.eu = v.rep_edge + GN;
+    v.ev = v.eu + GN;
+    v.ee = v.ev + GN;
+    v.rptr = v.ee + GN;
+    v.tk = v.rptr + GN + 1;
+    v.mu = v.tk + GN;
+    v.mv = v.mu + GN;
+    // 16-byte aligned table after the int32 arrays
+    uintptr_t t = reinterpret_cast<uintptr_t>(v.mv + GN);
+    t = (t + 15) & ~static_cast<uintptr_t>(15);
+    v.tab = reinterpret_cast<int4 *>(t);
+    v.Ls = reinterpret_cast<int32_t *>(v.tab + table_rounds(G, N) * G);
+    return v;
+}
 
+// Slot (round r, rank x) of the table, seen from x: code = partner lane
+// (bits 0-4), partner is rank lane+32 (bit 5), x is the transfer's home rank
+// (bit 6), edge index (bits 8-23); tok; the mass on x's side (home side: the
+// edge's mass; replica side: tok - mass).  An idle slot names x itself as
+// partner with tok = mass = 0, so it computes a zero move with no branch.
+__device__ __forceinline__ int slot_code(int partner, bool home, int edge) {
+    return (partner & 31) | ((partner >> 5) << 5) | (home ? 64 : 0) | (edge << 8);
+}
+
+// Relief passes (Algorithm 1), symmetric form.  For a transfer between x and
+// its partner y in a round: diff = L[x] - L[y]; the heavier side sends
+// min(|diff| >> 1, mass on its side), the lighter side receives the same
+// amount, limited by the partner's side (tok - own).  Both sides compute the
+// same delta, so this is exactly gap/limit/update of Algorithm 1 seen from u
+// and from v.  Lane j owns ranks j and (TWO) j+32; one full warp calls it.
+template <bool TWO>
+__device__ int relax_passes_regs(int G, int nr, int passes, const View &v) {
+    const int lane = threadIdx.x & 31;
+    const bool ha = lane < G, hb = TWO && lane + 32 < G;
+    int La = ha ? v.Ls[lane] : 0;
+    int Lb = hb ? v.Ls[lane + 32] : 0;
+    const int4 idle_a = make_int4(slot_code(lane, false, 0), 0, 0, 0);
+    const int4 idle_b = make_int4(slot_code(lane + 32, false, 0), 0, 0, 0);
+    int pr = 0;
+    for (int p = 1; p <= passes; ++p) {
+        bool moved = false;
+        int4 A = (nr > 0 && ha) ? v.tab[lane] : idle_a;
+        int4 B = (nr > 0 && hb) ? v.tab[lane + 32] : idle_b;
+        for (int r = 0; r < nr; ++r) {
+            const int4 a = A, b = B;
+            if (r + 1 < nr) {
+                A = ha ? v.tab[(r + 1) * G + lane] : idle_a;
+                if (TWO) B = hb ? v.tab[(r + 1) * G + lane + 32] : idle_b;
+            }
+            // every shuffle before any update: a lane may own both ends
+            int xa = __shfl_sync(kFull, La, a.x & 31);
+            int xb = 0;
+            if (TWO) {
+                const int ya = __shfl_sync(kFull, Lb, a.x & 31);
+                xa = (a.x & 32) ? ya : xa;
+                const int xl = __shfl_sync(kFull, La, b.x & 31);
+                const int xh = __shfl_sync(kFull, Lb, b.x & 31);
+                xb = (b.x & 32) ? xh : xl;
+            }
+            {
+                const int diff = La - xa;
+                const int d = min((diff < 0 ? -diff : diff) >> 1, diff > 0 ? a.z : a.y - a.z);
+                const int delta = diff > 0 ? -d : d;
+                La += delta;
+                if (delta != 0) {
+                    v.tab[r * G + lane].z = a.z + delta;
+                    moved = true;
+                }
+            }
+            if (TWO) {
+                const int diff = Lb - xb;
+                const int d = min((diff < 0 ? -diff : diff) >> 1, diff > 0 ? b.z : b.y - b.z);
+                const int delta = diff > 0 ? -d : d;
+                Lb += delta;
+                if (delta != 0) {
+                    v.tab[r * G + lane + 32].z = b.z + delta;
+                    moved = true;
+                }
+            }
+        }
+        pr = p;
+        if (!__any_sync(kFull, moved)) break;
+    }
+    if (ha) v.Ls[lane] = La;
+    if (hb) v.Ls[lane + 32] = Lb;
+    __syncwarp();
+    return pr;
+}
+
+// Fallback for schedules longer than the table: one lane per transfer of a
+// round, loads in shared memory.  Returns passes run; sets *bad on a round of
+// more than 32 transfers (impossible for a valid plan with G <= 64).
+__device__ int relax_passes_smem(int ne, int nr, int passes, const View &v, int *bad) {
+    const int lane = threadIdx.x & 31;
+    int pr = 0;
+    for (int p = 1; p <= passes; ++p) {
+        int moved = 0;
+        for (int r = 0; r < nr; ++r) {
+            const int a = v.rptr[r], n = v.rptr[r + 1] - a;
+            if (n > 32 || n < 0 || a < 0 || a + n > ne) {
+                if (lane == 0) *bad = 1;
+                continue;
+            }
+            if (lane < n) {
+                const int i = a + lane;
+                const int u = v.eu[i], w = v.ev[i];
+                const int Lu = v.Ls[u], Lw = v.Ls[w];
+                const int gap = Lu - Lw;
+                int d = (gap < 0 ? -gap : gap) >> 1;
+                d = min(d, gap > 0 ? v.mu[i] : v.tk[i] - v.mu[i]);
+                if (d > 0) {
+                    const int sd = gap > 0 ? d : -d;
+                    v.Ls[u] = Lu - sd;
+                    v.Ls[w] = Lw + sd;
+                    v.mu[i] -= sd;
+                    moved = 1;
+                }
+            }
+            __syncwarp();
+        }
+        pr = p;
+        if (!__any_sync(kFull, moved)) break;
+    }
+    return pr;
+}
+
+// The whole split of one problem by one CTA.  Inputs: the problem's counts
+// (global) and plan blob (global).  Leaves tok in v.tk, mass in v.mu, loads in
+// v.Ls, and returns passes run.  All threads of the CTA must call it.
+__device__ int split_problem(const int32_t *__restrict__ cnt, const uint8_t *__restrict__ blob, int G, int E,
+                             int N, int passes, const View &v, int &ne_out, int *bad) {
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, nwarps = blockDim.x >> 5;
-    const int b = blockIdx.x;
-    const int32_t *cnt = cnt_all + static_cast<int64_t>(b) * G * E;
-    const uint8_t *blob = plan_all + static_cast<size_t>(b) * stride;
+    const int GN = G * N, Eg = E / G;
     const plan::Layout LY = plan::layout(G, E, N);
     const int32_t *hdr = reinterpret_cast<const int32_t *>(blob + LY.hdr);
-    const int32_t *p_eu = reinterpret_cast<const int32_t *>(blob + LY.edge_u);
-    const int32_t *p_ev = reinterpret_cast<const int32_t *>(blob + LY.edge_v);
-    const int32_t *p_ee = reinterpret_cast<const int32_t *>(blob + LY.edge_e);
-    const int32_t *p_rptr = reinterpret_cast<const int32_t *>(blob + LY.round_ptr);
-    const int32_t *p_rep_ptr = reinterpret_cast<const int32_t *>(blob + LY.rep_ptr);
-    const int32_t *p_rep_edge = reinterpret_cast<const int32_t *>(blob + LY.rep_edge);
-    int32_t *tok = tok_all + static_cast<int64_t>(b) * GN;
-    int32_t *mass = mass_all + static_cast<int64_t>(b) * GN;
-    const int Eg = E / G;
-
     int ne = hdr[0], nr = hdr[1];
-    if (tid == 0) bad = 0;
     if (ne < 0 || ne > GN || nr < 0 || nr > GN) {
-        if (tid == 0) flag(LB_DEV_BAD_PLAN);
+        *bad = 1;
         ne = 0;
         nr = 0;
     }
-    for (int e = tid; e < E; e += blockDim.x) hold[e] = 1ull << (e / Eg);
-    for (int i = tid; i < ne; i += blockDim.x) {
-        eu[i] = p_eu[i];
-        ev[i] = p_ev[i];
-    }
-    for (int r = tid; r <= nr; r += blockDim.x) rptr[r] = p_rptr[r];
-    __syncthreads();
-    for (int i = tid; i < ne; i += blockDim.x) {
-        const int e = p_ee[i], v = ev[i];
-        if (e < 0 || e >= E || v < 0 || v >= G || eu[i] != e / Eg) {
-            bad = 1;
-            eu[i] = 0;   // neutralise: a self-loop never moves anything
-            ev[i] = 0;
-            continue;
-        }
-        atomicOr(reinterpret_cast<unsigned long long *>(&hold[e]), 1ull << v);
-    }
-    for (int i = tid; i < ne; i += blockDim.x) {
-        tk[i] = 0;
-        ms[i] = 0;
-    }
-    __syncthreads();
+    const int RC = table_rounds(G, N);
+    const bool use_table = nr <= RC;
+    LB_TICK(0);
 
-    // remote mass per expert
-    for (int e = tid; e < E; e += blockDim.x) {
-        const uint64_t hm = hold[e];
-        int s = 0;
-        for (int g = 0; g < G; ++g)
-            if (!((hm >> g) & 1ull)) s += cnt[g * E + e];
-        R[e] = s;
+    // ---- stage inputs (coalesced)
+    stage_i32(v.cnt, cnt, G * E);
+    {
+        const int32_t *p_eu = reinterpret_cast<const int32_t *>(blob + LY.edge_u);
+        const int32_t *p_ev = reinterpret_cast<const int32_t *>(blob + LY.edge_v);
+        const int32_t *p_ee = reinterpret_cast<const int32_t *>(blob + LY.edge_e);
+        const int32_t *p_rep_edge = reinterpret_cast<const int32_t *>(blob + LY.rep_edge);
+        for (int i = tid; i < ne; i += blockDim.x) {
+            v.eu[i] = p_eu[i];
+            v.ev[i] = p_ev[i];
+            v.ee[i] = p_ee[i];
+            v.rep_edge[i] = p_rep_edge[i];
+            v.tk[i] = 0;
+            v.mu[i] = 0;
+            v.mv[i] = 0;
+        }
+        const int32_t *p_rptr = reinterpret_cast<const int32_t *>(blob + LY.round_ptr);
+        for (int r = tid; r <= nr; r += blockDim.x) v.rptr[r] = p_rptr[r];
+        const int32_t *p_rep_ptr = reinterpret_cast<const int32_t *>(blob + LY.rep_ptr);
+        for (int e = tid; e <= E; e += blockDim.x) v.rep_ptr[e] = p_rep_ptr[e];
+        if (use_table)
+            for (int x = tid; x < nr * G; x += blockDim.x) {
+                const int rank = x % G;
+                v.tab[x] = make_int4(slot_code(rank, false, 0), 0, 0, 0);
+            }
     }
     __syncthreads();
-    // starting loads: own tokens of held experts + remote mass of home experts
+    LB_TICK(1);
+
+    // ---- per expert: holders, remote mass, equal partition over its edges
+    for (int e = tid; e < E; e += blockDim.x) {
+        const int h = e / Eg;
+        uint64_t hm = 1ull << h;
+        int a = v.rep_ptr[e], z = v.rep_ptr[e + 1];
+        if (a < 0 || z > ne || z < a) {
+            *bad = 1;
+            a = z = 0;
+        }
+        for (int j = a; j < z; ++j) {
+            const int i = v.rep_edge[j];
+            if (i < 0 || i >= ne || v.ee[i] != e || v.eu[i] != h || v.ev[i] < 0 || v.ev[i] >= G) {
+                *bad = 1;
+                continue;
+            }
+            hm |= 1ull << v.ev[i];
+        }
+        int R = 0;
+        for (int g = 0; g < G; ++g)
+            if (!((hm >> g) & 1ull)) R += v.cnt[g * E + e];
+        v.hold[e] = hm;
+        v.R[e] = R;
+        const int m = z - a;
+        if (m > 0) {
+            const int q = R / m, rem = R % m;
+            for (int j = 0; j < m; ++j) {
+                const int i = v.rep_edge[a + j];
+                if (i < 0 || i >= ne) continue;
+                const int t = q + (j < rem ? 1 : 0);
+                v.tk[i] = t;
+                v.mu[i] = t;
+                v.mv[i] = t;
+            }
+        }
+    }
+    __syncthreads();
+    LB_TICK(2);
+
+    // ---- starting loads (warp per rank) and the round table
     for (int r = warp; r < G; r += nwarps) {
         int x = 0;
         for (int e = lane; e < E; e += 32) {
-            if ((hold[e] >> r) & 1ull) x += cnt[r * E + e];
-            if (e / Eg == r) x += R[e];
+            if ((v.hold[e] >> r) & 1ull) x += v.cnt[r * E + e];
         }
+        for (int e = r * Eg + lane; e < (r + 1) * Eg; e += 32) x += v.R[e];
         x = __reduce_add_sync(kFull, x);
-        if (lane == 0) Ls[r] = x;
+        if (lane == 0) v.Ls[r] = x;
     }
-    // equal integer partition over each expert's edges (ascending replica rank)
-    for (int e = tid; e < E; e += blockDim.x) {
-        const int a = p_rep_ptr[e], z = p_rep_ptr[e + 1];
-        const int mcount = z - a;
-        if (a < 0 || z > ne || mcount < 0) {
-            bad = 1;
-            continue;
-        }
-        if (mcount == 0) continue;
-        const int q = R[e] / mcount, rem = R[e] % mcount;
-        for (int j = 0; j < mcount; ++j) {
-            const int i = p_rep_edge[a + j];
-            if (i < 0 || i >= ne) {
-                bad = 1;
+    if (use_table) {
+        for (int r = tid; r < nr; r += blockDim.x) {
+            const int a = v.rptr[r], z = v.rptr[r + 1];
+            if (a < 0 || z > ne || z < a) {
+                *bad = 1;
                 continue;
             }
-            const int t = q + (j < rem ? 1 : 0);
-            tk[i] = t;
-            ms[i] = t;
-        }
-    }
-    __syncthreads();
-
-    // passes: one warp
-    if (warp == 0) {
-        int pr = 0;
-        for (int p = 1; p <= passes; ++p) {
-            int moved = 0;
-            for (int r = 0; r < nr; ++r) {
-                const int a = rptr[r], n = rptr[r + 1] - a;
-                if (n > 32 || n < 0 || a < 0 || a + n > ne) {
-                    if (lane == 0) bad = 1;
-                    continue;
-                }
-                if (lane < n) {
-                    const int i = a + lane;
-                    const int u = eu[i], v = ev[i];
-                    const int Lu = Ls[u], Lv = Ls[v];
-                    const int gap = Lu - Lv;
-                    int d = (gap < 0 ? -gap : gap) >> 1;
-                    const int lim = gap > 0 ? ms[i] : tk[i] - ms[i];
-                    d = min(d, lim);
-                    if (d > 0) {
-                        const int sd = gap > 0 ? d : -d;
-                        Ls[u] = Lu - sd;
-                        Ls[v] = Lv + sd;
-                        ms[i] -= sd;
-                        moved = 1;
-                    }
-                }
-                __syncwarp();
+            for (int i = a; i < z; ++i) {
+                const int u = v.eu[i], w = v.ev[i];
+                if (u < 0 || u >= G || w < 0 || w >= G || u == w) continue;
+                const int t = v.tk[i];
+                v.tab[r * G + u] = make_int4(slot_code(w, true, i), t, t, 0);
+                v.tab[r * G + w] = make_int4(slot_code(u, false, i), t, 0, 0);
             }
-            pr = p;
-            if (!__any_sync(kFull, moved)) break;
         }
-        if (lane == 0) passes_run_all[b] = pr;
     }
     __syncthreads();
-    for (int i = tid; i < GN; i += blockDim.x) {
-        tok[i] = i < ne ? tk[i] : 0;
-        mass[i] = i < ne ? ms[i] : 0;
+    LB_TICK(3);
+
+    // ---- passes: one warp
+    __shared__ int pr_s;
+    if (warp == 0) {
+        int pr;
+        if (use_table)
+            pr = (G > 32) ? relax_passes_regs<true>(G, nr, passes, v) : relax_passes_regs<false>(G, nr, passes, v);
+        else
+            pr = relax_passes_smem(ne, nr, passes, v, bad);
+        if (lane == 0) pr_s = pr;
     }
-    for (int r = tid; r < G; r += blockDim.x) loads_all[static_cast<int64_t>(b) * G + r] = Ls[r];
-    if (tid == 0 && bad) flag(LB_DEV_BAD_PLAN);
+    __syncthreads();
+    if (use_table) {
+        // the edge's mass is the mass on its home side
+        for (int x = tid; x < nr * G; x += blockDim.x) {
+            const int4 c = v.tab[x];
+            if (c.x & 64) v.mu[(c.x >> 8) & 0xffff] = c.z;
+        }
+        __syncthreads();
+    }
+    LB_TICK(4);
+    ne_out = ne;
+    return pr_s;
+}
+
+__global__ void __launch_bounds__(THREADS)
+    split_kernel(const int32_t *__restrict__ cnt_all, const uint8_t *__restrict__ plan_all, size_t stride, int G,
+                 int E, int N, int passes, int32_t *__restrict__ tok_all, int32_t *__restrict__ mass_all,
+                 int32_t *__restrict__ loads_all, int32_t *__restrict__ passes_run_all) {
+    extern __shared__ __align__(16) uint8_t sm[];
+    __shared__ int bad;
+    const int tid = threadIdx.x, b = blockIdx.x, GN = G * N;
+    if (tid == 0) bad = 0;
+    __syncthreads();
+    const View v = carve(sm, G, E, N);
+    int ne = 0;
+    const int pr = split_problem(cnt_all + static_cast<int64_t>(b) * G * E, plan_all + static_cast<size_t>(b) * stride,
+                                 G, E, N, passes, v, ne, &bad);
+    int32_t *tok = tok_all + static_cast<int64_t>(b) * GN;
+    int32_t *mass = mass_all + static_cast<int64_t>(b) * GN;
+    for (int i = tid; i < GN; i += blockDim.x) {
+        tok[i] = i < ne ? v.tk[i] : 0;
+        mass[i] = i < ne ? v.mu[i] : 0;
+    }
+    for (int r = tid; r < G; r += blockDim.x) loads_all[static_cast<int64_t>(b) * G + r] = v.Ls[r];
+    if (tid == 0) {
+        passes_run_all[b] = pr;
+        if (bad) flag(LB_DEV_BAD_PLAN);
+    }
 }
 
 }  // namespace split

@@ -291,3 +291,23 @@ def test_batched_equals_unbatched():
     for l in range(3):
         assert torch.equal(cnt_b[l], _lib.lb_count(ids_b[l], w.G, w.E))
         assert torch.equal(plan_b[l], _lib.lb_plan_replicas(cnt_b[l], w.N, w.L)[0])
+
+
+def test_split_long_schedule_falls_back():
+    """A schedule longer than the per-(round, rank) table (every token asks
+    for rank 0's experts, so rank 0 gets hundreds of replica edges): the
+    shared-memory pass loop runs instead, with the same results."""
+    G, E, k, N, L = 64, 320, 5, 16, 8
+    T = G * 16
+    ids = torch.arange(k, dtype=torch.int32, device=DEV).repeat(T, 1)
+    path = DecisionPath(1, T, 8, E, k, G, N, L, device=DEV)
+    path.ids_pred.copy_(ids)
+    path.ids.copy_(ids)
+    _lib.lb_count(path.ids_pred, G, E, cnt=path.cnt_pred)
+    _lib.lb_plan_replicas(path.cnt_pred, N, L, plan=path.plan)
+    path.solve()
+    torch.cuda.synchronize()
+    assert _lib.lb_get_status() == 0
+    dec = _lib.decode_plan(path.plan[0], G, E, N)[0]
+    assert dec["n_rounds"] > 256
+    parity.check_path(path, 0, 12)
