@@ -86,10 +86,16 @@ int lb_predict_topk(const void *h, const void *w, const float *bias,
                     int32_t *ids, float *logits, void *stream);
 
 /* Tuning knobs of lb_predict_topk (process-wide; 0 = automatic choice):
- * pipeline stages per CTA (2..8) and split of H across a CTA cluster
- * (1, 2, 4, 8 or 16).  Results do not depend on them beyond fp32 rounding
- * of the split-H partial sums.  Returns LB_EINVAL for values out of range. */
-int lb_gate_tuning(int stages, int split);
+ * pipeline stages per CTA (2..8); split of H across a CTA cluster (1, 2, 4,
+ * 8 or 16); persistent kernel (1, 2 or 4 = that many CTAs per SM walking the
+ * tiles with a double-buffered TMEM accumulator; -1 = one CTA per tile);
+ * 64-column boxes per pipeline stage of the persistent kernel (1, 2 or 4).
+ * Automatic: with at least two token tiles per SM and E <= 128, persistent
+ * with two CTAs per SM; otherwise one CTA per tile, H split across a cluster
+ * until the GPU is filled when the tiles alone do not fill it.  Results do
+ * not depend on the knobs beyond fp32 rounding of split-H partial sums.
+ * LB_EINVAL for values out of range. */
+int lb_gate_tuning(int stages, int split, int persistent, int kbox);
 
 /* ------------------------------------------------------------------------
  * Step 2 -- per-rank histograms   [FB sec. 3.2 eq. 5; Algorithm 1,

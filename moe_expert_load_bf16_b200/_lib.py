@@ -45,7 +45,7 @@ def _load():
     lib = ctypes.CDLL(LIB_PATH)
     P, I, SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
     lib.lb_predict_topk.argtypes = [P, P, P, I, I, I, I, I, P, P, P]
-    lib.lb_gate_tuning.argtypes = [I, I]
+    lib.lb_gate_tuning.argtypes = [I, I, I, I]
     lib.lb_count.argtypes = [P, I, I, I, I, I, P, P]
     lib.lb_plan_bytes.argtypes = [I, I, I]
     lib.lb_plan_bytes.restype = SZ
@@ -125,8 +125,8 @@ def lb_predict_topk(h, w, bias, k, want_logits=False, ids=None, logits=None):
     return (ids, logits) if want_logits else ids
 
 
-def lb_gate_tuning(stages=0, split=0):
-    _check("lb_gate_tuning", _load().lb_gate_tuning(stages, split))
+def lb_gate_tuning(stages=0, split=0, persistent=0, kbox=0):
+    _check("lb_gate_tuning", _load().lb_gate_tuning(stages, split, persistent, kbox))
 
 
 # ------------------------------------------------------------------ step 2

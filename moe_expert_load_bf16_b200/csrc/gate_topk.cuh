@@ -36,6 +36,7 @@ struct Params {
     int32_t *ids;        // [B,T,k]
     float *logits;       // [B,T,E] or null
     int T, H, E, Epad, k, nkb, split, stages;
+    int kbox;            // persistent kernel: 64-column boxes per pipeline stage
     uint32_t tmem_cols;
 };
 
@@ -298,6 +299,201 @@ __global__ void __launch_bounds__(THREADS, 1)
                 if (j < p.k) out[j] = oi[j];
         }
         cluster_sync();   // keep this CTA's partials alive until all readers are done
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, p.tmem_cols);
+    }
+}
+
+
+// ---------------------------------------------------------------------------
+// Persistent variant, for when the token tiles fill the GPU.  One CTA per SM
+// walks the tiles blockIdx.x, blockIdx.x + gridDim.x, ... of all problems.
+// Warp 0 (one lane) keeps the TMA ring full across tile boundaries, warp 1
+// (one lane) issues the MMAs, and warps 2..5 run the epilogue.  The TMEM
+// accumulator is double-buffered (2 x Epad columns), so the top-k of tile i
+// overlaps the loads and MMAs of tile i+1.  h is streamed once (L2
+// evict-first); W is re-read by every tile of its problem (L2 evict-last).
+constexpr int P_THREADS = 192;
+
+template <int KMAX>
+__global__ void __launch_bounds__(P_THREADS, 1)
+    gate_topk_persistent(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                         const Params p, int mtiles, int ntiles) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                                ~static_cast<uintptr_t>(1023));
+    __shared__ __align__(8) uint64_t full_bar[MAX_STAGES];
+    __shared__ __align__(8) uint64_t empty_bar[MAX_STAGES];
+    __shared__ __align__(8) uint64_t acc_full[2];
+    __shared__ __align__(8) uint64_t acc_empty[2];
+    __shared__ __align__(8) uint64_t drain_bar;
+    __shared__ uint32_t tmem_slot;
+    __shared__ int aborted;
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const uint32_t a_box = BM * 128u, b_box = static_cast<uint32_t>(p.Epad) * 128u;
+    const int kbox = p.kbox;
+    const uint32_t a_bytes = a_box * kbox;              // A boxes first, then B boxes
+    const uint32_t stage_bytes = (a_box + b_box) * kbox;
+    const int stages = p.stages;
+    const int nks = (p.nkb + kbox - 1) / kbox;          // stages per tile (boxes past H read zeros)
+    const uint32_t half = p.tmem_cols >> 1;   // column offset of accumulator buffer 1
+
+    if (tid == 0) {
+        for (int s = 0; s < stages; ++s) {
+            mbar_init(&full_bar[s], 1);
+            mbar_init(&empty_bar[s], 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&acc_full[i], 1);
+            mbar_init(&acc_empty[i], 128);
+        }
+        mbar_init(&drain_bar, 1);
+        aborted = 0;
+        fence_mbar_init();
+        tma_prefetch_desc(&tmA);
+        tma_prefetch_desc(&tmB);
+    }
+    if (warp == 1) {
+        tmem_alloc(&tmem_slot, p.tmem_cols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = tmem_slot;
+    volatile int *abort_flag = &aborted;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            // ---------------- TMA producer
+            const uint64_t pol_a = l2_policy_evict_first(), pol_b = l2_policy_evict_last();
+            int it = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
+                const int b = tile / mtiles, m0 = (tile - b * mtiles) * BM;
+                for (int ks = 0; ks < nks; ++ks, ++it) {
+                    const int s = it % stages;
+                    const uint32_t ph = (it / stages) & 1;
+                    if (!mbar_wait(&empty_bar[s], ph ^ 1) || *abort_flag) {
+                        atomicExch(&aborted, 1);
+                        flag(LB_DEV_TIMEOUT);
+                        ok = false;
+                        break;
+                    }
+                    uint8_t *sa = smem + static_cast<size_t>(s) * stage_bytes;
+                    mbar_arrive_expect_tx(&full_bar[s], stage_bytes);
+                    for (int j = 0; j < kbox; ++j)
+                        tma_load_3d_hint(&tmA, sa + j * a_box, &full_bar[s], (ks * kbox + j) * BK, m0, b, pol_a);
+                    for (int j = 0; j < kbox; ++j)
+                        tma_load_3d_hint(&tmB, sa + a_bytes + j * b_box, &full_bar[s], (ks * kbox + j) * BK, 0, b,
+                                         pol_b);
+                }
+            }
+            // no copies left in flight into this CTA's shared memory
+            for (int s = 0; s < stages && s < it; ++s) {
+                const int last = s + ((it - 1 - s) / stages) * stages;
+                if (!mbar_wait(&full_bar[s], (last / stages) & 1)) flag(LB_DEV_TIMEOUT);
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            // ---------------- MMA issuer
+            const uint32_t idesc = umma_idesc_bf16(BM, p.Epad);
+            int it = 0, tl = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x, ++tl) {
+                const int buf = tl & 1;
+                const uint32_t use = static_cast<uint32_t>(tl >> 1);
+                if (!mbar_wait(&acc_empty[buf], (use & 1) ^ 1) || *abort_flag) {
+                    atomicExch(&aborted, 1);
+                    flag(LB_DEV_TIMEOUT);
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t d = tmem + buf * half;
+                for (int ks = 0; ks < nks; ++ks, ++it) {
+                    const int s = it % stages;
+                    const uint32_t ph = (it / stages) & 1;
+                    if (!mbar_wait(&full_bar[s], ph)) {
+                        atomicExch(&aborted, 1);
+                        flag(LB_DEV_TIMEOUT);
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t st = smem_u32(smem + static_cast<size_t>(s) * stage_bytes);
+                    for (int j = 0; j < kbox; ++j) {
+                        const uint32_t sa = st + j * a_box, sb = st + a_bytes + j * b_box;
+#pragma unroll
+                        for (int kk = 0; kk < BK / UK; ++kk)
+                            umma_bf16(d, sw128_kmajor_desc(sa + kk * UK * 2), sw128_kmajor_desc(sb + kk * UK * 2),
+                                      idesc, (ks > 0 || j > 0 || kk > 0) ? 1u : 0u);
+                    }
+                    umma_commit(&empty_bar[s]);
+                }
+                umma_commit(&acc_full[buf]);
+            }
+            // every MMA this CTA issued has finished before TMEM is freed
+            umma_commit(&drain_bar);
+            if (!mbar_wait(&drain_bar, 0)) flag(LB_DEV_TIMEOUT);
+        }
+    } else {
+        // ---------------- epilogue: warps 2..5, TMEM lane quadrant = warp % 4
+        const int q = warp & 3;
+        const int rloc = q * 32 + lane;
+        int tl = 0;
+        for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++tl) {
+            const int buf = tl & 1;
+            const uint32_t use = static_cast<uint32_t>(tl >> 1);
+            bool ok = mbar_wait(&acc_full[buf], use & 1) && !*abort_flag;
+            ok = __all_sync(kFull, ok);
+            if (!ok) {
+                if (lane == 0) {
+                    atomicExch(&aborted, 1);
+                    flag(LB_DEV_TIMEOUT);
+                }
+                break;
+            }
+            tc_fence_after();
+            const int b = tile / mtiles, m0 = (tile - b * mtiles) * BM;
+            const int row = m0 + rloc;
+            const bool valid = row < p.T;
+            const int64_t grow = static_cast<int64_t>(b) * p.T + row;
+            const float *bias = p.bias != nullptr ? p.bias + static_cast<int64_t>(b) * p.E : nullptr;
+            float *lrow = (p.logits != nullptr && valid) ? p.logits + grow * p.E : nullptr;
+            TopK<KMAX> tk;
+            tk.init();
+            const uint32_t tl_addr = tmem + buf * half + (static_cast<uint32_t>(q * 32) << 16);
+            for (int c0 = 0; c0 < p.Epad; c0 += 16) {
+                uint32_t r[16];
+                tmem_ld16(tl_addr + c0, r);
+                tmem_wait_ld();
+#pragma unroll
+                for (int j = 0; j < 16; ++j) {
+                    const int c = c0 + j;
+                    if (c < p.E) {
+                        const float x = __uint_as_float(r[j]) + (bias != nullptr ? __ldg(bias + c) : 0.f);
+                        tk.push(x, c);
+                        if (lrow) lrow[c] = x;
+                    }
+                }
+            }
+            // the accumulator buffer may be overwritten from here
+            tc_fence_before();
+            mbar_arrive(&acc_empty[buf]);
+            if (valid) {
+                int32_t *out = p.ids + grow * p.k;
+#pragma unroll
+                for (int j = 0; j < KMAX; ++j)
+                    if (j < p.k) out[j] = tk.i[j];
+            }
+        }
     }
 
     tc_fence_before();

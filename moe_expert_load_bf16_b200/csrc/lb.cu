@@ -21,6 +21,8 @@ using namespace lb;
 
 int g_tune_stages = 0;
 int g_tune_split = 0;
+int g_tune_persistent = 0;   // 0 automatic, 1/2/4 = persistent with that many CTAs per SM, -1 never
+int g_tune_kbox = 0;         // boxes per stage of the persistent kernel (0 automatic)
 
 inline bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
@@ -129,6 +131,24 @@ int launch_gate(const CUtensorMap &ma, const CUtensorMap &mb, const gate::Params
     return launched("gate_topk");
 }
 
+template <int KMAX>
+int launch_gate_persistent(const CUtensorMap &ma, const CUtensorMap &mb, const gate::Params &p, int mtiles,
+                           int ntiles, int grid, size_t smem, cudaStream_t s) {
+    auto kern = gate::gate_topk_persistent<KMAX>;
+    static SmemLimit lim;
+    if (!allow_smem(kern, lim, smem, false)) return LB_ECUDA;
+    kern<<<grid, gate::P_THREADS, smem, s>>>(ma, mb, p, mtiles, ntiles);
+    return launched("gate_topk_persistent");
+}
+
+int launch_gate_persistent_k(int k, const CUtensorMap &ma, const CUtensorMap &mb, const gate::Params &p,
+                             int mtiles, int ntiles, int grid, size_t smem, cudaStream_t s) {
+    if (k <= 2) return launch_gate_persistent<2>(ma, mb, p, mtiles, ntiles, grid, smem, s);
+    if (k <= 4) return launch_gate_persistent<4>(ma, mb, p, mtiles, ntiles, grid, smem, s);
+    if (k <= 8) return launch_gate_persistent<8>(ma, mb, p, mtiles, ntiles, grid, smem, s);
+    return launch_gate_persistent<16>(ma, mb, p, mtiles, ntiles, grid, smem, s);
+}
+
 template <bool SPLITK>
 int launch_gate_k(int k, const CUtensorMap &ma, const CUtensorMap &mb, const gate::Params &p, int mtiles,
                   int nbatch, size_t smem, cudaStream_t s) {
@@ -202,11 +222,16 @@ int lb_debug_ticks(long long *out, int n) {
 }
 #endif
 
-int lb_gate_tuning(int stages, int split) {
+int lb_gate_tuning(int stages, int split, int persistent, int kbox) {
+    if (kbox != 0 && kbox != 1 && kbox != 2 && kbox != 4) return LB_EINVAL;
     if (stages != 0 && (stages < 2 || stages > gate::MAX_STAGES)) return LB_EINVAL;
     if (split != 0 && split != 1 && split != 2 && split != 4 && split != 8 && split != 16) return LB_EINVAL;
+    if (persistent != -1 && persistent != 0 && persistent != 1 && persistent != 2 && persistent != 4)
+        return LB_EINVAL;
     g_tune_stages = stages;
     g_tune_split = split;
+    g_tune_persistent = persistent;
+    g_tune_kbox = kbox;
     return LB_OK;
 }
 
@@ -232,17 +257,57 @@ int lb_predict_topk(const void *h, const void *w, const float *bias, int nbatch,
     p.Epad = (E + 15) / 16 * 16;
     p.k = k;
     p.nkb = (H + gate::BK - 1) / gate::BK;
+    p.kbox = 1;
     uint32_t cols = 32;
     while (cols < static_cast<uint32_t>(p.Epad)) cols <<= 1;
     p.tmem_cols = cols;
     const int mtiles = (T + gate::BM - 1) / gate::BM;
+    const int sms = device_sms();
+    const long long ntiles = static_cast<long long>(mtiles) * nbatch;
+
+    // enough tiles for every SM: the persistent kernel (one CTA per SM)
+    // Automatic choice (measured on the benchmark shapes): with at least two
+    // tiles per SM, a persistent kernel with two CTAs per SM while two
+    // double-buffered accumulators fit in TMEM (E <= 128); otherwise one CTA
+    // per tile.
+    int per_sm = g_tune_persistent;
+    if (per_sm == 0 && g_tune_split <= 1 && ntiles >= 2LL * sms && p.Epad <= 128) per_sm = 2;
+    const bool persistent = per_sm > 0;
+    if (persistent) {
+        uint32_t pcols = 32;
+        while (pcols < 2u * static_cast<uint32_t>(p.Epad)) pcols <<= 1;
+        if (pcols > 512) return LB_EINVAL;
+        p.tmem_cols = pcols;
+        p.split = 1;
+        p.kbox = g_tune_kbox ? g_tune_kbox : (p.Epad <= 64 ? 2 : 1);
+        const size_t stage_bytes = (16384 + static_cast<size_t>(p.Epad) * 128) * p.kbox;
+        if (static_cast<uint32_t>(per_sm) * pcols > 512) return LB_EINVAL;
+        int stages = g_tune_stages;
+        if (!stages)
+            stages = static_cast<int>(
+                std::max<size_t>(2, std::min<size_t>(gate::MAX_STAGES, (100 * 1024 * 2 / per_sm) / stage_bytes)));
+        if (stages < 2) return LB_EINVAL;
+        size_t smem = stages * stage_bytes + 1024;
+        smem = std::max(smem, static_cast<size_t>(228 * 1024) / (per_sm + 1) + 1);   // at most per_sm CTAs per SM
+        if (smem > 224 * 1024) return LB_EINVAL;
+        p.stages = stages;
+        CUtensorMap ma, mb;
+        if (!make_map(&ma, h, static_cast<uint64_t>(H), static_cast<uint64_t>(T), static_cast<uint64_t>(nbatch),
+                      gate::BM) ||
+            !make_map(&mb, w, static_cast<uint64_t>(H), static_cast<uint64_t>(E), static_cast<uint64_t>(nbatch),
+                      static_cast<uint32_t>(p.Epad))) {
+            std::snprintf(g_last_error, sizeof g_last_error, "cuTensorMapEncodeTiled failed");
+            return LB_ECUDA;
+        }
+        const int grid = static_cast<int>(std::min<long long>(ntiles, static_cast<long long>(sms) * per_sm));
+        return launch_gate_persistent_k(k, ma, mb, p, mtiles, static_cast<int>(ntiles), grid, smem, s);
+    }
 
     // split of H across a cluster when the token tiles alone underfill the GPU
     int S = 1;
     if (g_tune_split) {
         S = g_tune_split;
     } else {
-        const int sms = device_sms();
         while (static_cast<long long>(mtiles) * nbatch * S < sms && S * 2 <= 16 && S * 2 <= p.nkb / 2 &&
                p.Epad % (4 * S * 2) == 0)
             S *= 2;
@@ -254,7 +319,10 @@ int lb_predict_topk(const void *h, const void *w, const float *bias, int nbatch,
 
     const size_t stage_bytes = 16384 + static_cast<size_t>(p.Epad) * 128;
     int stages = g_tune_stages;
-    if (!stages) stages = static_cast<int>(std::min<size_t>(8, std::max<size_t>(2, (110 * 1024 - 1024) / stage_bytes)));
+    if (!stages)
+        stages = (ntiles * S >= sms)
+                     ? 2
+                     : static_cast<int>(std::min<size_t>(8, std::max<size_t>(2, (110 * 1024 - 1024) / stage_bytes)));
     size_t smem = stages * stage_bytes + 1024;
     if (S > 1) smem = std::max(smem, static_cast<size_t>(gate::BM) * (p.Epad + 4) * 4 + 1024);
     if (smem > 224 * 1024) {

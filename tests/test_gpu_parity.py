@@ -17,10 +17,10 @@ DEV = "cuda"
 def _clean_status():
     if not torch.cuda.is_available():
         pytest.skip("needs a CUDA device")
-    _lib.lb_gate_tuning(0, 0)
+    _lib.lb_gate_tuning()
     _lib.lb_get_status(clear=True)
     yield
-    _lib.lb_gate_tuning(0, 0)
+    _lib.lb_gate_tuning()
 
 
 def run_model(w, layers, passes=12, T=None, sample_rows=None):
@@ -117,15 +117,18 @@ def test_decode_gate(T):
 
 @pytest.mark.parametrize("T,H,E,k", [(200, 72, 60, 5), (1, 8, 16, 1), (333, 128, 256, 16), (130, 64, 17, 3),
                                      (4096, 256, 128, 8), (96, 2048, 32, 2)])
-@pytest.mark.parametrize("split", [0, 1, 2, 4])
+@pytest.mark.parametrize("split", [0, 1, 2, 4, "persistent"])
 def test_gate_shapes(T, H, E, k, split):
     """Ragged token tails, E not a multiple of 16, H not a multiple of 64,
-    tiny and maximum k, every split of H."""
+    tiny and maximum k, every split of H, and the persistent kernel."""
     nkb = (H + 63) // 64
     Epad = (E + 15) // 16 * 16
-    if split > nkb or (split and Epad % (4 * split) != 0):
-        pytest.skip("split not valid for this shape")
-    _lib.lb_gate_tuning(0, split)
+    if split == "persistent":
+        _lib.lb_gate_tuning(0, 0, 1)
+    else:
+        if split > nkb or (split and Epad % (4 * split) != 0):
+            pytest.skip("split not valid for this shape")
+        _lib.lb_gate_tuning(0, split, -1)
     g = torch.Generator(device=DEV).manual_seed(T * 7 + H + E + k)
     h = torch.randn(T, H, generator=g, device=DEV).to(torch.bfloat16)
     W = (torch.randn(E, H, generator=g, device=DEV) / H ** 0.5).to(torch.bfloat16)
@@ -139,7 +142,7 @@ def test_gate_shapes(T, H, E, k, split):
 @pytest.mark.parametrize("split", [2, 4, 8, 16])
 def test_gate_split_cluster(split):
     """Forced split of H across clusters of 2..16 CTAs."""
-    _lib.lb_gate_tuning(0, split)
+    _lib.lb_gate_tuning(0, split, -1)
     T, H, E, k = 300, 4096, 256, 8
     g = torch.Generator(device=DEV).manual_seed(split)
     h = torch.randn(T, H, generator=g, device=DEV).to(torch.bfloat16)
@@ -148,9 +151,10 @@ def test_gate_split_cluster(split):
     parity.gate_check(h, W, None, k, ids, logits)
 
 
+@pytest.mark.parametrize("persistent", [-1, 1])
 @pytest.mark.parametrize("stages", [2, 3, 5, 8])
-def test_gate_stages(stages):
-    _lib.lb_gate_tuning(stages, 1)
+def test_gate_stages(stages, persistent):
+    _lib.lb_gate_tuning(stages, 1 if persistent < 0 else 0, persistent, 1)
     T, H, E, k = 512, 1024, 64, 8
     g = torch.Generator(device=DEV).manual_seed(stages)
     h = torch.randn(T, H, generator=g, device=DEV).to(torch.bfloat16)
@@ -311,3 +315,21 @@ def test_split_long_schedule_falls_back():
     dec = _lib.decode_plan(path.plan[0], G, E, N)[0]
     assert dec["n_rounds"] > 256
     parity.check_path(path, 0, 12)
+
+
+@pytest.mark.parametrize("persistent,kbox", [(-1, 0), (1, 1), (2, 1), (2, 2), (4, 1), (2, 4)])
+def test_gate_persistent_many_tiles_batched(persistent, kbox):
+    """Many tiles over several problems (more tiles than SMs, ragged last
+    tile per problem): persistent and one-CTA-per-tile kernels both match
+    the oracle on sampled rows of every problem."""
+    _lib.lb_gate_tuning(0, 0, persistent, kbox)
+    B, T, H, E, k = 5, 4000, 576, 64, 8   # H: 9 boxes, so a stage of 2 or 4 boxes runs past H
+    g = torch.Generator(device=DEV).manual_seed(11)
+    h = torch.randn(B, T, H, generator=g, device=DEV).to(torch.bfloat16)
+    W = (torch.randn(B, E, H, generator=g, device=DEV) / H ** 0.5).to(torch.bfloat16)
+    bias = torch.randn(B, E, generator=g, device=DEV)
+    ids, logits = _lib.lb_predict_topk(h, W, bias, k, want_logits=True)
+    rng = np.random.default_rng(4)
+    for b in range(B):
+        rows = np.concatenate([rng.choice(T, 64, replace=False), [0, 127, 128, T - 1]])
+        parity.gate_check(h[b], W[b], bias[b], k, ids[b], logits[b], rows=rows)
