@@ -122,15 +122,20 @@ class ClockSampler:
                 "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons), "samples": len(self.samples)}
 
 
-def dist_setup(n_gpus):
+def dist_setup(backend=None):
+    """One process per GPU (torchrun env); NCCL on GPUs, gloo on CPU-only hosts."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
-    if world > 1:
+    if world > 1 and not torch.distributed.is_initialized():
         import datetime
-        torch.cuda.set_device(local)
-        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                             device_id=torch.device("cuda", local))
+        backend = backend or ("nccl" if torch.cuda.is_available() else "gloo")
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+            torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                                 device_id=torch.device("cuda", local))
+        else:
+            torch.distributed.init_process_group("gloo", timeout=datetime.timedelta(seconds=120))
     return world, rank, local
 
 
@@ -140,11 +145,23 @@ def barrier(world):
 
 
 def max_over_ranks(x, world):
+    """The slowest rank's time (whole-job timing is the max over ranks)."""
     if world == 1:
         return x
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if torch.distributed.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
     return float(t.item())
+
+
+def rank_workload(wl, rank):
+    """Each rank decides its own independent problems (weak scaling): same
+    shapes, seeds offset by rank."""
+    return wl if rank == 0 else wl.with_(seed=wl.seed + 1000 * rank)
+
+
+def whole_job_rate(units_per_step_per_rank, world, ms_per_step):
+    return units_per_step_per_rank * world / (ms_per_step * 1e-3)
 
 
 # ----------------------------------------------------------------------------- GPU arm
@@ -153,9 +170,7 @@ def run_ours(args, world, rank, local):
     from moe_expert_load_bf16_b200.pipeline import DecisionPath
 
     build.build()
-    wl = workloads.WORKLOADS[args.config]
-    if rank:
-        wl = wl.with_(seed=wl.seed + 1000 * rank)     # independent problems per rank
+    wl = rank_workload(workloads.WORKLOADS[args.config], rank)
     Lyr, T, H, E, k, G, N, L = wl.layers, wl.T, wl.H, wl.E, wl.k, wl.G, wl.N, wl.L
     dev = torch.device("cuda", local)
     stream = torch.cuda.current_stream()
@@ -198,7 +213,7 @@ def run_ours(args, world, rank, local):
     ms_total = max_over_ranks(ev0.elapsed_time(ev1), world)
     ms_step = ms_total / args.steps
     assign_per_step = Lyr * T * k
-    value = assign_per_step * world / (ms_step * 1e-3)
+    value = whole_job_rate(assign_per_step, world, ms_step)
     if args.lean:
         return {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
                 "warmup": args.warmup, "ms_per_step": ms_step, "lean": True,
@@ -342,6 +357,82 @@ def end_to_end(args, wl, hid, W, bias, path, dev, world):
             "d2h_bytes_per_step": int(d2h), "ms_per_step": ms, "steps": n}
 
 
+
+# ----------------------------------------------------------------------------- decode sweep
+def run_decode(args, world, rank, local):
+    """Decode-step split sweep: E=256, top-8, G=64 ranks x 4 experts, N=2.
+    The plan is made once from step 0's counts (placement changes minutes
+    apart); each decode step then runs the fused count + split + assign on
+    its own ids.  Per T: T_solve of one step, T_split, the throughput of 64
+    steps in one launch, and the gate at the decode shape (H=7168)."""
+    from moe_expert_load_bf16_b200 import _lib, build, workloads
+    from moe_expert_load_bf16_b200.pipeline import DecisionPath
+    build.build()
+    wl = rank_workload(workloads.WORKLOADS["decode"], rank)
+    dev = torch.device("cuda", local)
+    B = 64
+
+    def timed(fn, reps):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            fn()
+        g.replay()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier(world)
+        a.record()
+        for _ in range(reps):
+            g.replay()
+        b.record()
+        torch.cuda.synchronize()
+        return max_over_ranks(a.elapsed_time(b) * 1e3 / reps, world)
+
+    per_T = {}
+    total_assign, total_us = 0, 0.0
+    for T in wl.decode_T:
+        ids = workloads.decode_ids(wl.with_(T=T), T, range(B + 1), device=dev)
+        path = DecisionPath(B, T, wl.H, wl.E, wl.k, wl.G, wl.N, wl.L, device=dev)
+        path.ids.copy_(ids[1:])
+        path.ids_pred.copy_(ids[0:1].expand(B, -1, -1))
+        _lib.lb_count(path.ids_pred[0:1], wl.G, wl.E, cnt=path.cnt_pred[0:1])
+        _lib.lb_plan_replicas(path.cnt_pred[0:1], wl.N, wl.L, plan=path.plan[0:1])
+        path.plan[1:].copy_(path.plan[0:1].expand(B - 1, -1))
+        one = DecisionPath(1, T, wl.H, wl.E, wl.k, wl.G, wl.N, wl.L, device=dev)
+        one.ids.copy_(ids[1:2])
+        one.plan.copy_(path.plan[0:1])
+        for _ in range(args.warmup):
+            path.solve()
+            one.solve()
+        torch.cuda.synchronize()
+        reps = max(20, args.steps)
+        t_solve = timed(one.solve, reps)
+        t_split = timed(lambda: _lib.lb_split(one.cnt, one.plan, wl.N, 12,
+                                              out=(one.tok, one.mass, one.loads, one.passes_run)), reps)
+        t_batch = timed(path.solve, max(5, reps // 4))
+        h = workloads.hidden_chain(wl, 1, device=dev, T=T)[0]
+        W = workloads.gate_weights(wl, 1, device=dev)[0]
+        bias = workloads.biases(wl, 1)[0].to(dev)
+        gate_ids = torch.empty(T, wl.k, dtype=torch.int32, device=dev)
+        t_gate = timed(lambda: _lib.lb_predict_topk(h, W, bias, wl.k, ids=gate_ids), reps)
+        gate_bytes = 2 * T * wl.H + 2 * wl.H * wl.E + 4 * wl.E + 4 * T * wl.k
+        per_T[str(T)] = {"t_solve_us": t_solve, "t_split_us": t_split,
+                         "batch64_us": t_batch, "batch64_assignments_per_s": B * T * wl.k / (t_batch * 1e-6),
+                         "gate_us": t_gate, "gate_gbs": gate_bytes / (t_gate * 1e-6) / 1e9}
+        total_assign += B * T * wl.k
+        total_us += t_batch
+        del ids, path, one, h, W
+        torch.cuda.empty_cache()
+    if _lib.lb_get_status():
+        raise RuntimeError("device status flagged")
+    value = total_assign * world / (total_us * 1e-6)
+    return {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": total_us / 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "int32", "data": "synthetic",
+            "config": {"workload": "decode-step split sweep: E=256, top-8, G=64 ranks x 4 experts, N=2 (L=1); "
+                                   "64 steps per T in one fused launch; plan from step 0",
+                       "T": list(wl.decode_T), "steps_per_launch": B},
+            "per_T": per_T}
+
 # ----------------------------------------------------------------------------- CPU oracle
 def cpu_baseline(wl, budget_s=15.0):
     """The oracle, as it stands, on this host's cores, over whole layers of
@@ -405,7 +496,7 @@ def run_reference(args, world, rank):
         return None
     for _ in range(min(args.warmup, 1)):
         cpu_baseline(wl, budget_s=1.0)
-    per = max(2.0, min(20.0, 120.0 / max(1, args.steps)))
+    per = args.cpu_budget if args.cpu_budget_set else max(2.0, min(20.0, 120.0 / max(1, args.steps)))
     t0 = time.perf_counter()
     vals = [cpu_baseline(wl, budget_s=per) for _ in range(args.steps)]
     wall = time.perf_counter() - t0
@@ -436,6 +527,7 @@ def main():
                     help="time the steps only (no gate-only loop, per-layer latencies, end-to-end or CPU "
                          "baseline): the command used for ncu launch lists")
     args = ap.parse_args()
+    args.cpu_budget_set = "--cpu-budget" in sys.argv
     if args.warmup < 3:
         args.warmup = 3
     if args.impl == "reference":
@@ -445,9 +537,9 @@ def main():
         if out is not None:
             print(json.dumps(out), flush=True)
         return
-    world, rank, local = dist_setup(args.gpus)
+    world, rank, local = dist_setup()
     try:
-        out = run_ours(args, world, rank, local)
+        out = run_decode(args, world, rank, local) if args.config == "decode" else run_ours(args, world, rank, local)
         if rank == 0:
             print(json.dumps(out), flush=True)
     finally:

@@ -210,6 +210,28 @@ int lb_assign(const int32_t *ids, const int32_t *cnt, const void *plan,
               void *workspace, size_t workspace_bytes, void *stream);
 
 /* ------------------------------------------------------------------------
+ * Steps 2, 4 and 5 fused -- the per-step decision on the actual ids in one
+ * launch   [FB sec. 3.2 eq. 5; Relief, Algorithm 1; Libra, Key Ideas]
+ * Computes exactly what lb_count, then lb_split, then lb_assign compute
+ * (same outputs, same layouts, bit for bit), with one thread-block cluster
+ * per problem: its CTAs count slices of the tokens, CTA 0 combines the counts
+ * over distributed shared memory and runs the split and the permutation
+ * tables, then every CTA scatters its slice.
+ *   ids, plan, passes: as lb_count / lb_split
+ *   cnt [nbatch,G,E], tok, mass [nbatch,G*N], loads [nbatch,G],
+ *   passes_run [nbatch], dest [nbatch,T,k], perm [nbatch,T*k],
+ *   offs [nbatch,G*E+1]: outputs
+ *   workspace: >= lb_assign_workspace_bytes(...) bytes, 256-byte aligned
+ * Limits: those of lb_count, lb_split and lb_assign together.  Shapes whose
+ * cluster tables do not fit one SM's shared memory run as the three separate
+ * launches, with the same results.
+ * ------------------------------------------------------------------------ */
+int lb_solve(const int32_t *ids, const void *plan, int nbatch, int T, int k, int G, int E,
+             int N, int passes, int32_t *cnt, int32_t *tok, int32_t *mass, int32_t *loads,
+             int32_t *passes_run, int32_t *dest, int32_t *perm, int32_t *offs,
+             void *workspace, size_t workspace_bytes, void *stream);
+
+/* ------------------------------------------------------------------------
  * lb_assign without a caller workspace (the pages have no counterpart; this
  * is a convenience of this library).
  * For callers that cannot provide device scratch memory: a runtime whose

@@ -56,13 +56,14 @@ def _load():
     lib.lb_assign_workspace_bytes.restype = SZ
     lib.lb_assign.argtypes = [P, P, P, P, P, I, I, I, I, I, I, P, P, P, P, SZ, P]
     lib.lb_assign_noalloc.argtypes = [P, P, P, P, P, I, I, I, I, I, I, P, P, P, P]
+    lib.lb_solve.argtypes = [P, P, I, I, I, I, I, I, I, P, P, P, P, P, P, P, P, P, SZ, P]
     lib.lb_get_status.argtypes = [ctypes.POINTER(ctypes.c_int32), I]
     lib.lb_strerror.argtypes = [I]
     lib.lb_strerror.restype = ctypes.c_char_p
     lib.lb_last_error.argtypes = []
     lib.lb_last_error.restype = ctypes.c_char_p
     for f in ("lb_predict_topk", "lb_gate_tuning", "lb_count", "lb_plan_layout_of", "lb_plan_replicas",
-              "lb_split", "lb_assign", "lb_assign_noalloc", "lb_get_status", "lb_version"):
+              "lb_split", "lb_assign", "lb_assign_noalloc", "lb_solve", "lb_get_status", "lb_version"):
         getattr(lib, f).restype = ctypes.c_int
     _lib = lib
     return lib
@@ -238,6 +239,29 @@ def lb_assign(ids, cnt, plan, tok, mass, N, out=None, workspace=None):
     return dest, perm, offs
 
 
+def lb_solve(ids, plan, G, E, N, passes=12, out=None, workspace=None):
+    """Count + split + assign in one launch.  out = (cnt, tok, mass, loads,
+    passes_run, dest, perm, offs) preallocated, or None."""
+    lib = _load()
+    ids = _batched(ids, 3)
+    _need(ids, torch.int32, "ids")
+    B, T, k = ids.shape
+    dev = ids.device
+    if out is None:
+        i32 = dict(dtype=torch.int32, device=dev)
+        out = (torch.empty(B, G, E, **i32), torch.empty(B, G * N, **i32), torch.empty(B, G * N, **i32),
+               torch.empty(B, G, **i32), torch.empty(B, **i32), torch.empty(B, T, k, **i32),
+               torch.empty(B, T * k, **i32), torch.empty(B, G * E + 1, **i32))
+    cnt, tok, mass, loads, pr, dest, perm, offs = out
+    nbytes = lb_assign_workspace_bytes(B, T, k, G, E, N)
+    if workspace is None:
+        workspace = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=dev)
+    _check("lb_solve", lib.lb_solve(_p(ids), _p(plan), B, T, k, G, E, N, passes, _p(cnt), _p(tok), _p(mass),
+                                    _p(loads), _p(pr), _p(dest), _p(perm), _p(offs), _p(workspace),
+                                    workspace.numel(), _stream()))
+    return out
+
+
 def lb_assign_noalloc(ids, cnt, plan, tok, mass, N, out=None):
     """lb_assign for callers that cannot provide device scratch memory: the
     library uses its own fixed device array instead (see include/lb.h).
@@ -274,6 +298,6 @@ def lb_version():
 
 
 EXPORTS = ("lb_predict_topk", "lb_gate_tuning", "lb_count", "lb_plan_bytes", "lb_plan_layout_of",
-           "lb_plan_replicas", "lb_split", "lb_assign_workspace_bytes", "lb_assign", "lb_assign_noalloc",
+           "lb_plan_replicas", "lb_split", "lb_assign_workspace_bytes", "lb_assign", "lb_assign_noalloc", "lb_solve",
            "lb_get_status",
            "lb_strerror", "lb_last_error", "lb_version")

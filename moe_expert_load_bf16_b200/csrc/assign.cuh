@@ -46,11 +46,18 @@ __host__ __device__ inline size_t prep_smem_bytes(int G, int E, int N) {
            (static_cast<size_t>(E) + 1) * 4 + GN * 4 * 7 + 64;
 }
 
+// Shared memory of the scatter: per-expert tables (holders, replica count,
+// CSR start, home count), the per-(CTA or warp) block bases and running
+// counts, the per-warp counter tables, and the replica segments.
 __host__ __device__ inline size_t scatter_smem_bytes(int G, int E, int N) {
-    const size_t GN = static_cast<size_t>(G) * N;
+    const size_t GN = static_cast<size_t>(G) * N, EP = static_cast<size_t>(E) + 1;
     return static_cast<size_t>(E) * 8 + static_cast<size_t>(E) * 4 * 3 + (static_cast<size_t>(E) + 1) * 4 +
-           static_cast<size_t>(SC_WARPS) * (E + 1) * 4 * 2 + GN * 4 * 6 + 64;
+           static_cast<size_t>(SC_WARPS) * EP * 4 * 3 + GN * 4 * 7 + 64;
 }
+
+// Source blocks of at most this many assignments are scattered one block per
+// warp (no block-wide barrier); larger ones by the whole CTA.
+constexpr int WARP_BLOCK_MAX = 2048;
 
 struct Args {
     const int32_t *ids, *cnt, *tok, *mass;
@@ -63,8 +70,9 @@ struct Args {
 
 __device__ __forceinline__ int clampi(int x, int lo, int hi) { return min(max(x, lo), hi); }
 
-__global__ void __launch_bounds__(PREP_THREADS) prep_kernel(const Args a) {
-    extern __shared__ __align__(16) uint8_t sm[];
+// Tables of problem b for its scatter: offs, base[g,e], replica segments.
+// All threads of the CTA call it; `sm` holds prep_smem_bytes(G,E,N) bytes.
+__device__ void prep_problem(const Args &a, int b, uint8_t *sm) {
     const int G = a.G, E = a.E, N = a.N, GN = G * N, NK = G * E;
     uint64_t *hold = reinterpret_cast<uint64_t *>(sm);
     int32_t *cnt_s = reinterpret_cast<int32_t *>(hold + E);
@@ -80,11 +88,10 @@ __global__ void __launch_bounds__(PREP_THREADS) prep_kernel(const Args a) {
     int32_t *sq = ms + GN;           // segment start in q
     int32_t *sc = sq + GN;           // mass of earlier segments
     int32_t *osz = sc + GN;          // [NK] bucket sizes, then their exclusive scan
-    __shared__ int wsum[PREP_THREADS / 32];
+    __shared__ int wsum[32];
     __shared__ int bad;
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int b = blockIdx.x;
     const int32_t *cnt = a.cnt + static_cast<int64_t>(b) * NK;
     const uint8_t *blob = a.plan + static_cast<size_t>(b) * a.plan_stride;
     const plan::Layout LY = plan::layout(G, E, N);
@@ -262,29 +269,69 @@ __global__ void __launch_bounds__(PREP_THREADS) prep_kernel(const Args a) {
     __syncthreads();
     LB_TICK(23);
     if (tid == 0 && bad) flag(LB_DEV_BAD_SPLIT);
+    __syncthreads();
 }
 
-__global__ void __launch_bounds__(SC_THREADS) scatter_kernel(const Args a) {
+__global__ void __launch_bounds__(PREP_THREADS) prep_kernel(const Args a) {
     extern __shared__ __align__(16) uint8_t sm[];
-    const int G = a.G, E = a.E, N = a.N, GN = G * N, NK = G * E, k = a.k;
-    const int EP = E + 1;   // padded row of the per-warp tables (no bank conflicts)
-    uint64_t *hold = reinterpret_cast<uint64_t *>(sm);
-    int32_t *rcnt = reinterpret_cast<int32_t *>(hold + E);
-    int32_t *base_s = rcnt + E;
-    int32_t *run = base_s + E;
-    int32_t *rep_ptr = run + E;          // [E+1]
-    int32_t *wcnt = rep_ptr + E + 1;     // [SC_WARPS][EP]
-    int32_t *pre = wcnt + SC_WARPS * EP; // [SC_WARPS][EP]
-    int32_t *s_qoff = pre + SC_WARPS * EP;   // per-expert CSR position j
-    int32_t *s_tok = s_qoff + GN;
-    int32_t *s_mass = s_tok + GN;
-    int32_t *s_home = s_mass + GN;
-    int32_t *s_rep = s_home + GN;
-    int32_t *s_v = s_rep + GN;
-    __shared__ int bad;
+    prep_problem(a, blockIdx.x, sm);
+}
 
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int g = blockIdx.x, b = blockIdx.y;
+// ---- scatter ---------------------------------------------------------------
+// Peers of this lane's expert id among the warp's lanes (bit-by-bit ballots:
+// a fixed log2(E) collectives, where __match_any_sync serialises over the
+// distinct values in the warp).  Lanes with e < 0 are excluded.
+__device__ __forceinline__ unsigned warp_peers(int e, int nbits) {
+    unsigned m = __ballot_sync(kFull, e >= 0);
+    for (int bit = 0; bit < nbits; ++bit) {
+        const bool on = (e >> bit) & 1;
+        const unsigned bb = __ballot_sync(kFull, on);
+        m &= on ? bb : ~bb;
+    }
+    return m;
+}
+
+struct ScatterView {
+    uint64_t *hold;     // [E]
+    int32_t *rcnt;      // [E] replica edges of e
+    int32_t *rep0;      // [E+1] first CSR position of e
+    int32_t *homecnt;   // [E] cnt[home(e), e]
+    int32_t *homeoff;   // [E] offs[home(e)*E + e]
+    int32_t *base;      // [SC_WARPS][EP] block bases (row 0 only in CTA mode)
+    int32_t *wcnt;      // [SC_WARPS][EP]
+    int32_t *pre;       // [SC_WARPS][EP] (CTA mode) / unused
+    int32_t *s_qoff, *s_tok, *s_mass, *s_cum, *s_rep, *s_v, *s_vcnt;   // [GN] per CSR position
+};
+
+__device__ inline ScatterView scatter_carve(uint8_t *sm, int G, int E, int N) {
+    const int GN = G * N, EP = E + 1;
+    ScatterView v;
+    v.hold = reinterpret_cast<uint64_t *>(sm);
+    v.rcnt = reinterpret_cast<int32_t *>(v.hold + E);
+    v.rep0 = v.rcnt + E;
+    v.homecnt = v.rep0 + E + 1;
+    v.homeoff = v.homecnt + E;
+    v.base = v.homeoff + E;
+    v.wcnt = v.base + SC_WARPS * EP;
+    v.pre = v.wcnt + SC_WARPS * EP;
+    v.s_qoff = v.pre + SC_WARPS * EP;
+    v.s_tok = v.s_qoff + GN;
+    v.s_mass = v.s_tok + GN;
+    v.s_cum = v.s_mass + GN;
+    v.s_rep = v.s_cum + GN;
+    v.s_v = v.s_rep + GN;
+    v.s_vcnt = v.s_v + GN;
+    return v;
+}
+
+// Per-problem tables every block shares (built once per CTA): holder masks,
+// replica segments in per-expert CSR order (start in q, tok, mass, mass of
+// earlier segments, bucket start on the replica rank, replica rank, the
+// replica rank's own count of e), and per expert its home bucket start and
+// home count.  The per-block terms are added per assignment.
+__device__ void scatter_setup(const Args &a, int b, const ScatterView &v) {
+    const int G = a.G, E = a.E, N = a.N, GN = G * N, NK = G * E;
+    const int tid = threadIdx.x;
     const int32_t *cnt = a.cnt + static_cast<int64_t>(b) * NK;
     const uint8_t *blob = a.plan + static_cast<size_t>(b) * a.plan_stride;
     const plan::Layout LY = plan::layout(G, E, N);
@@ -300,74 +347,183 @@ __global__ void __launch_bounds__(SC_THREADS) scatter_kernel(const Args a) {
     const int32_t *seg_cum = seg_qoff + GN;
     const int32_t *seg_rep = seg_cum + GN;
     const int Eg = E / G;
-    const int Tg = a.T / G;
-    const int nitems = Tg * k;
-    const int64_t f0 = static_cast<int64_t>(g) * nitems;         // problem-local flat index
+    int ne = hdr[0];
+    if (ne < 0 || ne > GN) ne = 0;
+    for (int e = tid; e <= E; e += blockDim.x) v.rep0[e] = p_rep_ptr[e];
+    // per CSR position j (parallel): segment data
+    for (int j = tid; j < ne; j += blockDim.x) {
+        const int i = p_rep_edge[j];
+        const bool ok = i >= 0 && i < ne;
+        const int w = ok ? p_ev[i] : -1;
+        if (!ok || w < 0 || w >= G) {
+            v.s_tok[j] = 0;   // an empty segment: never matched
+            v.s_qoff[j] = 0x7fffffff;
+            v.s_v[j] = 0;
+            continue;
+        }
+        v.s_qoff[j] = seg_qoff[i];
+        v.s_tok[j] = tok[i];
+        v.s_mass[j] = mass[i];
+        v.s_cum[j] = seg_cum[i];
+        v.s_rep[j] = seg_rep[i];
+        v.s_v[j] = w;
+    }
+    __syncthreads();
+    for (int j = tid; j < ne; j += blockDim.x) {
+        // the expert of CSR position j: last e with rep0[e] <= j
+        int lo = 0, hi = E - 1;
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (v.rep0[mid] <= j) lo = mid; else hi = mid - 1;
+        }
+        v.s_vcnt[j] = cnt[v.s_v[j] * E + lo];
+    }
+    for (int e = tid; e < E; e += blockDim.x) {
+        const int h = e / Eg;
+        int r0 = v.rep0[e], r1 = v.rep0[e + 1];
+        if (r0 < 0 || r1 > ne || r1 < r0) r0 = r1 = 0;
+        uint64_t hm = 1ull << h;
+        for (int j = r0; j < r1; ++j)
+            if (v.s_tok[j] > 0 || v.s_qoff[j] != 0x7fffffff) hm |= 1ull << v.s_v[j];
+        v.hold[e] = hm;
+        v.rcnt[e] = r1 - r0;
+        v.homecnt[e] = cnt[h * E + e];
+        v.homeoff[e] = offs[h * E + e];
+    }
+    __syncthreads();
+}
+
+// Destination rank and permutation slot of an assignment of expert e from
+// source block g whose rank among the block's earlier assignments of e is
+// rho; bse = base[g, e].  Returns false if the tables do not place it.
+__device__ __forceinline__ bool place(const ScatterView &v, int Eg, int g, int e, int bse, int rho, int &d, int &p) {
+    const uint64_t hm = v.hold[e];
+    if ((hm >> g) & 1ull) {
+        d = g;
+        p = bse + rho;
+        return true;
+    }
+    const int h = e / Eg;
+    const int m = v.rcnt[e];
+    if (m == 0) {
+        d = h;
+        p = bse + rho;
+        return true;
+    }
+    const int q = bse + rho;
+    // last segment starting at or before q (starts ascend along the CSR)
+    int lo = v.rep0[e], hi = lo + m - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (v.s_qoff[mid] <= q) lo = mid; else hi = mid - 1;
+    }
+    const int qo = v.s_qoff[lo], t = v.s_tok[lo];
+    if (!(q >= qo && q < qo + t)) return false;
+    const int w = q - qo, mss = v.s_mass[lo];
+    if (w < mss) {
+        d = h;
+        p = v.homeoff[e] + (h < g ? v.homecnt[e] : 0) + v.s_cum[lo] + w;
+    } else {
+        const int r = v.s_v[lo];
+        d = r;
+        p = v.s_rep[lo] + (r < g ? v.s_vcnt[lo] : 0) + (w - mss);
+    }
+    return true;
+}
+
+// Whole blocks, one per warp (blocks g0, g0 + SC_WARPS, ... below g1): the
+// warp walks the block's assignments 32 at a time in order, ranking each
+// among the earlier ones of its expert with bit-ballot peers and a per-warp
+// running count in shared memory.  No block-wide barrier.
+__device__ void scatter_blocks_warp(const Args &a, int b, int g0, int g1, const ScatterView &v, int *bad) {
+    const int G = a.G, E = a.E, k = a.k, EP = E + 1;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int Eg = E / G, Tg = a.T / G, nitems = Tg * k, nf = a.T * k;
+    const int nbits = E > 1 ? 32 - __clz(E - 1) : 1;
     const int32_t *ids = a.ids + static_cast<int64_t>(b) * a.T * k;
     int32_t *dest = a.dest + static_cast<int64_t>(b) * a.T * k;
     int32_t *perm = a.perm + static_cast<int64_t>(b) * a.T * k;
-    const int nf = a.T * k;
-    int ne = hdr[0];
-    if (ne < 0 || ne > GN) ne = 0;
-
-    // ---- stage: this block's bases, holder masks, replica segments
-    LB_TICK(10);
-    if (tid == 0) bad = 0;
-    for (int e = tid; e <= E; e += blockDim.x) rep_ptr[e] = p_rep_ptr[e];
-    for (int e = tid; e < E; e += blockDim.x) {
-        base_s[e] = ws[g * E + e];
-        run[e] = 0;
-    }
-    __syncthreads();
-    for (int e = tid; e < E; e += blockDim.x) {
-        const int h = e / Eg;
-        int r0 = rep_ptr[e], r1 = rep_ptr[e + 1];
-        if (r0 < 0 || r1 > ne || r1 < r0) r0 = r1 = 0;
-        uint64_t hm = 1ull << h;
-        const int hb = offs[h * E + e] + (h < g ? cnt[h * E + e] : 0);
-        int mcount = 0;
-        for (int j = r0; j < r1; ++j) {
-            const int i = p_rep_edge[j];
-            const int v = (i >= 0 && i < ne) ? p_ev[i] : -1;
-            if (v < 0 || v >= G) {
-                s_tok[j] = 0;   // an empty segment: never matched
-                s_qoff[j] = 0;
-                continue;
-            }
-            hm |= 1ull << v;
-            s_qoff[j] = seg_qoff[i];
-            s_tok[j] = tok[i];
-            s_mass[j] = mass[i];
-            s_home[j] = hb + seg_cum[i];
-            s_rep[j] = seg_rep[i] + (v < g ? cnt[v * E + e] : 0);
-            s_v[j] = v;
-            ++mcount;
+    const int32_t *wsb = a.ws + static_cast<size_t>(b) * a.ws_stride;
+    int32_t *cntw = v.wcnt + warp * EP;
+    int32_t *basew = v.base + warp * EP;
+    for (int g = g0 + warp; g < g1; g += SC_WARPS) {
+        for (int e = lane; e < E; e += 32) {
+            cntw[e] = 0;
+            basew[e] = wsb[g * E + e];
         }
-        hold[e] = hm;
-        rcnt[e] = r1 - r0;
-        (void)mcount;
+        __syncwarp();
+        const int64_t f0 = static_cast<int64_t>(g) * nitems;
+        for (int i0 = 0; i0 < nitems; i0 += 32) {
+            const int i = i0 + lane;
+            int e = -1;
+            if (i < nitems) {
+                e = __ldg(ids + f0 + i);
+                if (e < 0 || e >= E) {
+                    *bad = 1;
+                    e = -1;
+                }
+            }
+            const unsigned peers = warp_peers(e, nbits);
+            const int rnk = __popc(peers & lanemask_lt());
+            const int cur = e >= 0 ? cntw[e] : 0;
+            __syncwarp();
+            if (e >= 0 && lane == 31 - __clz(peers)) cntw[e] = cur + __popc(peers);
+            if (e >= 0) {
+                int d, pp;
+                if (place(v, Eg, g, e, basew[e], cur + rnk, d, pp) && pp >= 0 && pp < nf) {
+                    dest[f0 + i] = d;
+                    perm[pp] = static_cast<int32_t>(f0 + i);
+                } else {
+                    *bad = 1;
+                }
+            }
+            __syncwarp();
+        }
+    }
+}
+
+// Assignments [i0, i1) of one block by the whole CTA (large blocks): warps
+// take consecutive 32-assignment steps, then a shuffle scan across warps
+// turns per-warp counts into block-order ranks.  `prefix` (shared memory,
+// E entries) holds each expert's assignments in the block before i0, or is
+// null when i0 == 0.
+__device__ void scatter_block_cta(const Args &a, int b, int g, int i0, int i1, const int32_t *prefix,
+                                  const ScatterView &v, int *bad) {
+    const int G = a.G, E = a.E, k = a.k, EP = E + 1;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int Eg = E / G, Tg = a.T / G, nitems = Tg * k, nf = a.T * k;
+    const int nbits = E > 1 ? 32 - __clz(E - 1) : 1;
+    const int64_t f0 = static_cast<int64_t>(g) * nitems;
+    const int32_t *ids = a.ids + static_cast<int64_t>(b) * a.T * k;
+    int32_t *dest = a.dest + static_cast<int64_t>(b) * a.T * k;
+    int32_t *perm = a.perm + static_cast<int64_t>(b) * a.T * k;
+    const int32_t *wsb = a.ws + static_cast<size_t>(b) * a.ws_stride;
+    int32_t *run = v.base + EP;   // row 1 of the base table: running counts
+    for (int e = tid; e < E; e += blockDim.x) {
+        v.base[e] = wsb[g * E + e];
+        run[e] = prefix != nullptr ? prefix[e] : 0;
     }
     __syncthreads();
-    LB_TICK(11);
-
     constexpr int CH = SC_WARPS * 32 * SC_STEPS;
-    int32_t *wrow = wcnt + warp * EP;
-    for (int cs = 0; cs < nitems; cs += CH) {
+    int32_t *wrow = v.wcnt + warp * EP;
+    const int iend = min(i1, nitems);
+    for (int cs = i0; cs < iend; cs += CH) {
         for (int e = lane; e < E; e += 32) wrow[e] = 0;
         __syncwarp();
         int es[SC_STEPS], loc[SC_STEPS];
 #pragma unroll
         for (int s = 0; s < SC_STEPS; ++s) {
             const int i = cs + warp * 32 * SC_STEPS + s * 32 + lane;
-            int e = -1;
-            if (i < nitems) {
-                e = __ldg(ids + f0 + i);
-                if (e < 0 || e >= E) {
-                    bad = 1;
-                    e = -1;
-                }
+            es[s] = i < iend ? __ldg(ids + f0 + i) : -1;
+        }
+#pragma unroll
+        for (int s = 0; s < SC_STEPS; ++s) {
+            int e = es[s];
+            if (e >= E || e < -1 || (e == -1 && cs + warp * 32 * SC_STEPS + s * 32 + lane < iend)) {
+                *bad = 1;
+                e = -1;
             }
-            const unsigned peers = __match_any_sync(kFull, e);
+            const unsigned peers = warp_peers(e, nbits);
             const int rnk = __popc(peers & lanemask_lt());
             const int cur = e >= 0 ? wrow[e] : 0;
             __syncwarp();
@@ -377,9 +533,8 @@ __global__ void __launch_bounds__(SC_THREADS) scatter_kernel(const Args a) {
             loc[s] = cur + rnk;
         }
         __syncthreads();
-        // per expert: exclusive scan of the warps' counts (warp order = f order)
         for (int e = warp; e < E; e += SC_WARPS) {
-            const int c = wcnt[lane * EP + e];
+            const int c = v.wcnt[lane * EP + e];
             int x = c;
 #pragma unroll
             for (int off = 1; off < 32; off <<= 1) {
@@ -387,7 +542,7 @@ __global__ void __launch_bounds__(SC_THREADS) scatter_kernel(const Args a) {
                 if (lane >= off) x += y;
             }
             const int r = run[e];
-            pre[lane * EP + e] = r + x - c;
+            v.pre[lane * EP + e] = r + x - c;
             __syncwarp();
             if (lane == 31) run[e] = r + x;
         }
@@ -397,54 +552,40 @@ __global__ void __launch_bounds__(SC_THREADS) scatter_kernel(const Args a) {
             const int e = es[s];
             if (e < 0) continue;
             const int i = cs + warp * 32 * SC_STEPS + s * 32 + lane;
-            const int rho = pre[warp * EP + e] + loc[s];
-            int d, p;
-            if ((hold[e] >> g) & 1ull) {
-                d = g;
-                p = base_s[e] + rho;
-            } else if (rcnt[e] == 0) {
-                d = e / Eg;
-                p = base_s[e] + rho;
+            int d, pp;
+            if (place(v, Eg, g, e, v.base[e], v.pre[warp * EP + e] + loc[s], d, pp) && pp >= 0 && pp < nf) {
+                dest[f0 + i] = d;
+                perm[pp] = static_cast<int32_t>(f0 + i);
             } else {
-                const int q = base_s[e] + rho;
-                d = -1;
-                p = -1;
-                // last segment starting at or before q (segment starts ascend)
-                int lo = rep_ptr[e], hi = lo + rcnt[e] - 1;
-                while (lo < hi) {
-                    const int mid = (lo + hi + 1) >> 1;
-                    if (s_qoff[mid] <= q) lo = mid; else hi = mid - 1;
-                }
-                // skip empty segments that start at q as well
-                while (lo < rep_ptr[e] + rcnt[e] - 1 && s_tok[lo] == 0 && s_qoff[lo + 1] <= q) ++lo;
-                {
-                    const int j = lo;
-                    const int qo = s_qoff[j];
-                    const int t = s_tok[j];
-                    if (rcnt[e] > 0 && q >= qo && q < qo + t) {
-                        const int w = q - qo, mss = s_mass[j];
-                        if (w < mss) {
-                            d = e / Eg;
-                            p = s_home[j] + w;
-                        } else {
-                            d = s_v[j];
-                            p = s_rep[j] + (w - mss);
-                        }
-                    }
-                }
+                *bad = 1;
             }
-            const int64_t f = f0 + i;
-            if (d < 0 || p < 0 || p >= nf) {
-                bad = 1;
-                continue;
-            }
-            dest[f] = d;
-            perm[p] = static_cast<int32_t>(f);
         }
         __syncthreads();   // pre/run are rewritten by the next chunk
     }
+    __syncthreads();
+}
+
+// Scatter kernel: CTA (x, problem y).  Small blocks: CTA x takes blocks
+// [x*SC_WARPS, (x+1)*SC_WARPS), one per warp.  Large blocks: CTA x takes
+// block x.
+__global__ void __launch_bounds__(SC_THREADS) scatter_kernel(const Args a) {
+    extern __shared__ __align__(16) uint8_t sm[];
+    __shared__ int bad;
+    if (threadIdx.x == 0) bad = 0;
+    const ScatterView v = scatter_carve(sm, a.G, a.E, a.N);
+    LB_TICK(10);
+    scatter_setup(a, blockIdx.y, v);
+    LB_TICK(11);
+    const int nitems = (a.T / a.G) * a.k;
+    if (nitems <= WARP_BLOCK_MAX) {
+        const int g0 = blockIdx.x * SC_WARPS;
+        scatter_blocks_warp(a, blockIdx.y, g0, min(a.G, g0 + SC_WARPS), v, &bad);
+        __syncthreads();
+    } else {
+        scatter_block_cta(a, blockIdx.y, blockIdx.x, 0, nitems, nullptr, v, &bad);
+    }
     LB_TICK(12);
-    if (tid == 0 && bad) flag(LB_DEV_BAD_SPLIT);
+    if (threadIdx.x == 0 && bad) flag(LB_DEV_BAD_SPLIT);
 }
 
 }  // namespace assign

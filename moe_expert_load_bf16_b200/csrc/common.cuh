@@ -211,6 +211,11 @@ __device__ __forceinline__ uint32_t mapa_shared(uint32_t saddr, uint32_t rank) {
     asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
     return r;
 }
+__device__ __forceinline__ int ld_cluster_i32(uint32_t addr) {
+    int v;
+    asm volatile("ld.shared::cluster.s32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+    return v;
+}
 __device__ __forceinline__ float4 ld_cluster_f4(uint32_t addr) {
     float4 v;
     asm volatile("ld.shared::cluster.v4.f32 {%0,%1,%2,%3}, [%4];"
@@ -223,7 +228,9 @@ __device__ __forceinline__ float4 ld_cluster_f4(uint32_t addr) {
 // ---------------------------------------------------------------- staging
 // Copy n int32 from global to shared memory with the whole CTA: 16-byte
 // loads when both sides are 16-byte aligned, four loads in flight per thread.
-__device__ __forceinline__ void stage_i32(int32_t *dst, const int32_t *__restrict__ src, int n) {
+// Plain (coherent) loads: the source may have been written earlier in the
+// same kernel by this CTA.
+__device__ __forceinline__ void stage_i32(int32_t *dst, const int32_t *src, int n) {
     const int t = threadIdx.x, nt = blockDim.x;
     if (((reinterpret_cast<uintptr_t>(dst) | reinterpret_cast<uintptr_t>(src)) & 15) == 0) {
         const int n4 = n >> 2;
@@ -231,26 +238,26 @@ __device__ __forceinline__ void stage_i32(int32_t *dst, const int32_t *__restric
         int4 *d4 = reinterpret_cast<int4 *>(dst);
         int i = t;
         for (; i + 3 * nt < n4; i += 4 * nt) {
-            const int4 a = __ldg(s4 + i), b = __ldg(s4 + i + nt), c = __ldg(s4 + i + 2 * nt),
-                       d = __ldg(s4 + i + 3 * nt);
+            const int4 a = s4[i], b = s4[i + nt], c = s4[i + 2 * nt],
+                       d = s4[i + 3 * nt];
             d4[i] = a;
             d4[i + nt] = b;
             d4[i + 2 * nt] = c;
             d4[i + 3 * nt] = d;
         }
-        for (; i < n4; i += nt) d4[i] = __ldg(s4 + i);
-        for (int j = (n4 << 2) + t; j < n; j += nt) dst[j] = __ldg(src + j);
+        for (; i < n4; i += nt) d4[i] = s4[i];
+        for (int j = (n4 << 2) + t; j < n; j += nt) dst[j] = src[j];
     } else {
         int i = t;
         for (; i + 3 * nt < n; i += 4 * nt) {
-            const int a = __ldg(src + i), b = __ldg(src + i + nt), c = __ldg(src + i + 2 * nt),
-                      d = __ldg(src + i + 3 * nt);
+            const int a = src[i], b = src[i + nt], c = src[i + 2 * nt],
+                      d = src[i + 3 * nt];
             dst[i] = a;
             dst[i + nt] = b;
             dst[i + 2 * nt] = c;
             dst[i + 3 * nt] = d;
         }
-        for (; i < n; i += nt) dst[i] = __ldg(src + i);
+        for (; i < n; i += nt) dst[i] = src[i];
     }
 }
 

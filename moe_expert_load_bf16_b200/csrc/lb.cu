@@ -13,6 +13,7 @@
 #include "count.cuh"
 #include "gate_topk.cuh"
 #include "plan.cuh"
+#include "solve.cuh"
 #include "split.cuh"
 
 namespace {
@@ -169,6 +170,13 @@ int launch_count_v(bool vec, const int32_t *ids, int nbatch, int T, int k, int E
                    cudaStream_t s) {
     return vec ? launch_count<K, true>(ids, nbatch, T, k, E, G, cnt, s)
                : launch_count<K, false>(ids, nbatch, T, k, E, G, cnt, s);
+}
+
+// Scatter CTAs per problem: one per source block, or one per SC_WARPS small
+// blocks (one block per warp).
+int scatter_grid_x(int T, int k, int G) {
+    const long long nitems = static_cast<long long>(T / G) * k;
+    return nitems <= assign::WARP_BLOCK_MAX ? (G + assign::SC_WARPS - 1) / assign::SC_WARPS : G;
 }
 
 bool plan_shape_ok(int G, int E, int N, int L) {
@@ -470,11 +478,92 @@ int lb_assign(const int32_t *ids, const int32_t *cnt, const void *plan, const in
     assign::prep_kernel<<<nbatch, assign::PREP_THREADS, sm1, s>>>(a);
     if (launched("assign prep") != LB_OK) return LB_ECUDA;
     if (T == 0) return LB_OK;
-    assign::scatter_kernel<<<dim3(G, nbatch), assign::SC_THREADS, sm2, s>>>(a);
+    assign::scatter_kernel<<<dim3(scatter_grid_x(T, k, G), nbatch), assign::SC_THREADS, sm2, s>>>(a);
     return launched("assign scatter");
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Fused count + split + assign (one cluster launch per batch of problems).
+namespace {
+
+// CTAs per problem: about one per 4096 assignments, a power of two up to 16
+// that divides G or that G divides (so slices are whole blocks or equal parts
+// of one), and 1 when nothing fits.
+int solve_cluster(int T, int k, int G, int sms, int nbatch) {
+    long long items = static_cast<long long>(T) * k;
+    int C = 1;
+    while (C < 16 && items / (2LL * C) >= 4096 && static_cast<long long>(nbatch) * C * 2 <= 2LL * sms) C *= 2;
+    while (C > 1 && !((C <= G && G % C == 0) || (C > G && C % G == 0))) C >>= 1;
+    return C;
+}
+
+}  // namespace
+
+extern "C" int lb_solve(const int32_t *ids, const void *plan, int nbatch, int T, int k, int G, int E, int N,
+                        int passes, int32_t *cnt, int32_t *tok, int32_t *mass, int32_t *loads,
+                        int32_t *passes_run, int32_t *dest, int32_t *perm, int32_t *offs, void *workspace,
+                        size_t workspace_bytes, void *stream) {
+    if (nbatch < 1 || nbatch > 65535 || T < 0 || T % G != 0 || k < 1 || k > LB_MAX_K || !plan_shape_ok(G, E, N, 0) ||
+        passes < 0 || passes > 4096)
+        return LB_EINVAL;
+    if (!plan || !cnt || !offs || !loads || !passes_run || !workspace || !aligned(plan, 256) ||
+        !aligned(workspace, 256))
+        return LB_EINVAL;
+    if (G * N > 0 && (!tok || !mass)) return LB_EINVAL;
+    if (T > 0 && (!ids || !dest || !perm)) return LB_EINVAL;
+    if (static_cast<long long>(T) * k * nbatch >= INT_MAX) return LB_EINVAL;
+    if (workspace_bytes < lb_assign_workspace_bytes(nbatch, T, k, G, E, N)) return LB_ENOSPACE;
+    int C = solve_cluster(T, k, G, device_sms(), nbatch);
+    // a larger cluster keeps fewer source blocks' counts per CTA
+    while (solve::smem_bytes(G, E, N, C) > 224 * 1024 && C < 16 && G % (2 * C) == 0) C *= 2;
+    const size_t smem = solve::smem_bytes(G, E, N, C);
+    if (smem > 224 * 1024) {
+        // does not fit one SM: the same work as three launches
+        int rc = lb_count(ids, nbatch, T, k, E, G, cnt, stream);
+        if (rc == LB_OK) rc = lb_split(cnt, plan, nbatch, G, E, N, passes, tok, mass, loads, passes_run, stream);
+        if (rc == LB_OK)
+            rc = lb_assign(ids, cnt, plan, tok, mass, nbatch, T, k, G, E, N, dest, perm, offs, workspace,
+                           workspace_bytes, stream);
+        return rc;
+    }
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    assign::Args a;
+    a.ids = ids;
+    a.cnt = cnt;
+    a.tok = tok;
+    a.mass = mass;
+    a.plan = static_cast<const uint8_t *>(plan);
+    a.plan_stride = plan::layout(G, E, N).total;
+    a.T = T;
+    a.k = k;
+    a.G = G;
+    a.E = E;
+    a.N = N;
+    a.dest = dest;
+    a.perm = perm;
+    a.offs = offs;
+    a.ws = static_cast<int32_t *>(workspace);
+    a.ws_stride = assign::ws_words(G, E, N);
+    static SmemLimit lim;
+    if (!allow_smem(solve::solve_kernel, lim, smem, true)) return LB_ECUDA;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(C, nbatch, 1);
+    cfg.blockDim = dim3(solve::THREADS, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = C;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, solve::solve_kernel, a, passes, loads, passes_run);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaLaunchKernelEx(solve)");
+    return launched("solve");
+}
 
 // ---------------------------------------------------------------------------
 // Allocation-free variant of lb_assign.
@@ -575,6 +664,7 @@ extern "C" int lb_assign_noalloc(const int32_t *ids, const int32_t *cnt, const v
     assign::prep_kernel<<<nbatch, assign::PREP_THREADS, assign::prep_smem_bytes(G, E, N), s>>>(a);
     if (launched("assign prep (noalloc)") != LB_OK) return LB_ECUDA;
     if (T == 0) return LB_OK;
-    assign::scatter_kernel<<<dim3(G, nbatch), assign::SC_THREADS, assign::scatter_smem_bytes(G, E, N), s>>>(a);
+    assign::scatter_kernel<<<dim3(scatter_grid_x(T, k, G), nbatch), assign::SC_THREADS,
+                             assign::scatter_smem_bytes(G, E, N), s>>>(a);
     return launched("assign scatter (noalloc)");
 }

@@ -47,8 +47,15 @@ class DecisionPath:
     def route(self, h_cur, w, bias):
         _lib.lb_predict_topk(h_cur, w, bias, self.k, ids=self.ids)
 
-    # the per-step decision on actual ids (T_solve)
+    # the per-step decision on actual ids (T_solve): one fused launch
     def solve(self, ids=None):
+        ids = self.ids if ids is None else ids
+        _lib.lb_solve(ids, self.plan, self.G, self.E, self.N, self.passes,
+                      out=(self.cnt, self.tok, self.mass, self.loads, self.passes_run, self.dest, self.perm,
+                           self.offs), workspace=self.ws)
+
+    # the same decision as three separate calls (lb_count, lb_split, lb_assign)
+    def solve_separate(self, ids=None):
         ids = self.ids if ids is None else ids
         _lib.lb_count(ids, self.G, self.E, cnt=self.cnt)
         _lib.lb_split(self.cnt, self.plan, self.N, self.passes,
@@ -61,4 +68,4 @@ class DecisionPath:
         self.route(h_cur, w, bias)
         self.solve()
 
-    LAUNCHES_PER_RUN = 8   # 2 gate, 2 count, plan, split, assign prep + scatter
+    LAUNCHES_PER_RUN = 5   # 2 gate, count, plan (lookahead); fused count + split + assign

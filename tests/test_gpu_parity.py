@@ -333,3 +333,31 @@ def test_gate_persistent_many_tiles_batched(persistent, kbox):
     for b in range(B):
         rows = np.concatenate([rng.choice(T, 64, replace=False), [0, 127, 128, T - 1]])
         parity.gate_check(h[b], W[b], bias[b], k, ids[b], logits[b], rows=rows)
+
+
+@pytest.mark.parametrize("name,T,B", [("olmoe", 4096, 2), ("qwen3-235b", 32768, 1), ("qwen3-30b", 16384, 1),
+                                      ("decode", 8192, 2), ("decode", 1024, 2), ("decode", 64, 3),
+                                      ("tiny-p1", 256, 2), ("tiny", 0, 1)])
+def test_solve_fused_equals_separate_calls(name, T, B):
+    """lb_solve (one cluster launch: counts, split, permutation) gives the
+    same bytes as lb_count + lb_split + lb_assign, whatever the cluster layout
+    (several source blocks per CTA, parts of one block per CTA, one CTA)."""
+    w = workloads.WORKLOADS[name]
+    steps = list(range(B + 1))
+    ids = workloads.decode_ids(w.with_(T=max(T, 1)), max(T, 1), steps).to(DEV)[:, :T]
+    path = DecisionPath(B, T, 8, w.E, w.k, w.G, w.N, w.L, device=DEV)
+    path.ids_pred.copy_(ids[0:1].expand(B, -1, -1))
+    path.ids.copy_(ids[1:])
+    _lib.lb_count(path.ids_pred, w.G, w.E, cnt=path.cnt_pred)
+    _lib.lb_plan_replicas(path.cnt_pred, w.N, w.L, plan=path.plan)
+    path.solve()
+    fused = [t.clone() for t in (path.cnt, path.tok, path.mass, path.loads, path.passes_run, path.dest, path.perm,
+                                 path.offs)]
+    path.solve_separate()
+    torch.cuda.synchronize()
+    assert _lib.lb_get_status() == 0
+    for f, s in zip(fused, (path.cnt, path.tok, path.mass, path.loads, path.passes_run, path.dest, path.perm,
+                            path.offs)):
+        assert torch.equal(f, s)
+    for b in range(B):
+        parity.check_path(path, b, 12)
