@@ -182,9 +182,10 @@ def run_ours(args, world, rank, local):
     W = workloads.gate_weights(wl, Lyr, device=dev)
     bias = workloads.biases(wl, Lyr).to(dev)
     path = DecisionPath(Lyr, T, H, E, k, G, N, L, device=dev)
+    side = torch.cuda.Stream(device=dev)
 
     def step():
-        path.run(hid[:-1], hid[1:], W, bias)
+        path.run(hid[:-1], hid[1:], W, bias, side_stream=side)
 
     # warm-up (also loads the library, sets kernel attributes, builds maps)
     for _ in range(args.warmup):
@@ -258,10 +259,11 @@ def run_ours(args, world, rank, local):
         "config": {"workload": f"{wl.name}: {Lyr} layers x T={T} tokens, H={H}, E={E}, top-{k}, "
                                f"G={G} ranks, N={N} replica slots (L={L})",
                    "layers": Lyr, "T": T, "H": H, "E": E, "k": k, "G": G, "N": N, "L": L, "passes": 12,
-                   "batching": "all layers of a step in one launch per kernel, CUDA-graph replay",
+                   "batching": "all layers of a step in one launch per kernel, CUDA-graph replay; lookahead "
+                               "counts + plan on a second stream beside the normal-router gate",
                    "l2": "inputs larger than L2 (hidden states %.0f MB per step)" % (2 * Lyr * T * H * 2 / 1e6),
                    "parallelism": f"{world} independent replicas"},
-        "t_solve_us": lat["solve"], "t_split_us": lat["split"], "t_lookahead_us": lat["lookahead"],
+        "t_solve_us": lat["solve"], "t_solve_fused_us": lat["solve_fused"], "t_split_us": lat["split"], "t_lookahead_us": lat["lookahead"],
         "per_kernel_us": lat["kernels"],
         "roofline": {"kernel": "gate_topk", "bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
                      "frac": achieved / hbm, "traffic": traffic, "peak_kind": peak_kind,
@@ -303,6 +305,7 @@ def per_layer_latency(wl, hid, W, bias, dev, reps):
 
     res = {
         "solve": timed(p1.solve),
+        "solve_fused": timed(p1.solve_fused),
         "split": timed(lambda: _lib.lb_split(p1.cnt, p1.plan, N, 12,
                                              out=(p1.tok, p1.mass, p1.loads, p1.passes_run))),
         "lookahead": timed(lambda: (p1.lookahead(hid[0:1], W[0:1], bias[0:1]), p1.route(hid[1:2], W[0:1],
@@ -362,9 +365,11 @@ def end_to_end(args, wl, hid, W, bias, path, dev, world):
 def run_decode(args, world, rank, local):
     """Decode-step split sweep: E=256, top-8, G=64 ranks x 4 experts, N=2.
     The plan is made once from step 0's counts (placement changes minutes
-    apart); each decode step then runs the fused count + split + assign on
-    its own ids.  Per T: T_solve of one step, T_split, the throughput of 64
-    steps in one launch, and the gate at the decode shape (H=7168)."""
+    apart); each decode step then runs count + split + assign on its own ids,
+    as separate launches and as the fused lb_solve.  Per T: T_solve of one
+    step, T_split, the throughput of 64 steps per launch, and the gate at the
+    decode shape (H=7168).  The line's value takes, per T, the faster of the
+    two batched forms."""
     from moe_expert_load_bf16_b200 import _lib, build, workloads
     from moe_expert_load_bf16_b200.pipeline import DecisionPath
     build.build()
@@ -403,20 +408,26 @@ def run_decode(args, world, rank, local):
         for _ in range(args.warmup):
             path.solve()
             one.solve()
+            path.solve_fused()
+            one.solve_fused()
         torch.cuda.synchronize()
         reps = max(20, args.steps)
         t_solve = timed(one.solve, reps)
+        t_fused = timed(one.solve_fused, reps)
         t_split = timed(lambda: _lib.lb_split(one.cnt, one.plan, wl.N, 12,
                                               out=(one.tok, one.mass, one.loads, one.passes_run)), reps)
-        t_batch = timed(path.solve, max(5, reps // 4))
+        t_batch_sep = timed(path.solve, max(5, reps // 4))
+        t_batch_fused = timed(path.solve_fused, max(5, reps // 4))
+        t_batch = min(t_batch_sep, t_batch_fused)
         h = workloads.hidden_chain(wl, 1, device=dev, T=T)[0]
         W = workloads.gate_weights(wl, 1, device=dev)[0]
         bias = workloads.biases(wl, 1)[0].to(dev)
         gate_ids = torch.empty(T, wl.k, dtype=torch.int32, device=dev)
         t_gate = timed(lambda: _lib.lb_predict_topk(h, W, bias, wl.k, ids=gate_ids), reps)
         gate_bytes = 2 * T * wl.H + 2 * wl.H * wl.E + 4 * wl.E + 4 * T * wl.k
-        per_T[str(T)] = {"t_solve_us": t_solve, "t_split_us": t_split,
-                         "batch64_us": t_batch, "batch64_assignments_per_s": B * T * wl.k / (t_batch * 1e-6),
+        per_T[str(T)] = {"t_solve_us": t_solve, "t_solve_fused_us": t_fused, "t_split_us": t_split,
+                         "batch64_us": t_batch_sep, "batch64_fused_us": t_batch_fused,
+                         "batch64_assignments_per_s": B * T * wl.k / (t_batch * 1e-6),
                          "gate_us": t_gate, "gate_gbs": gate_bytes / (t_gate * 1e-6) / 1e9}
         total_assign += B * T * wl.k
         total_us += t_batch
@@ -429,7 +440,7 @@ def run_decode(args, world, rank, local):
             "warmup": args.warmup, "ms_per_step": total_us / 1e3, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "int32", "data": "synthetic",
             "config": {"workload": "decode-step split sweep: E=256, top-8, G=64 ranks x 4 experts, N=2 (L=1); "
-                                   "64 steps per T in one fused launch; plan from step 0",
+                                   "64 steps per T per launch (separate or fused, the faster); plan from step 0",
                        "T": list(wl.decode_T), "steps_per_launch": B},
             "per_T": per_T}
 

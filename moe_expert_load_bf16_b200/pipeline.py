@@ -47,15 +47,10 @@ class DecisionPath:
     def route(self, h_cur, w, bias):
         _lib.lb_predict_topk(h_cur, w, bias, self.k, ids=self.ids)
 
-    # the per-step decision on actual ids (T_solve): one fused launch
+    # the per-step decision on actual ids (T_solve): lb_count, lb_split,
+    # lb_assign (on the benchmark shapes these three launches are faster than
+    # the fused lb_solve, whose single CTA 0 runs split and tables in series)
     def solve(self, ids=None):
-        ids = self.ids if ids is None else ids
-        _lib.lb_solve(ids, self.plan, self.G, self.E, self.N, self.passes,
-                      out=(self.cnt, self.tok, self.mass, self.loads, self.passes_run, self.dest, self.perm,
-                           self.offs), workspace=self.ws)
-
-    # the same decision as three separate calls (lb_count, lb_split, lb_assign)
-    def solve_separate(self, ids=None):
         ids = self.ids if ids is None else ids
         _lib.lb_count(ids, self.G, self.E, cnt=self.cnt)
         _lib.lb_split(self.cnt, self.plan, self.N, self.passes,
@@ -63,9 +58,30 @@ class DecisionPath:
         _lib.lb_assign(ids, self.cnt, self.plan, self.tok, self.mass, self.N,
                        out=(self.dest, self.perm, self.offs), workspace=self.ws)
 
-    def run(self, h_prev, h_cur, w, bias):
-        self.lookahead(h_prev, w, bias)
+    # the same decision as one fused launch (lb_solve)
+    def solve_fused(self, ids=None):
+        ids = self.ids if ids is None else ids
+        _lib.lb_solve(ids, self.plan, self.G, self.E, self.N, self.passes,
+                      out=(self.cnt, self.tok, self.mass, self.loads, self.passes_run, self.dest, self.perm,
+                           self.offs), workspace=self.ws)
+
+    def run(self, h_prev, h_cur, w, bias, side_stream=None):
+        """One pass.  With `side_stream`, the lookahead's counts and plan run
+        on it concurrently with the normal-router gate (they only meet at the
+        solve); both streams join before the solve."""
+        if side_stream is None:
+            self.lookahead(h_prev, w, bias)
+            self.route(h_cur, w, bias)
+            self.solve()
+            return
+        main = torch.cuda.current_stream()
+        _lib.lb_predict_topk(h_prev, w, bias, self.k, ids=self.ids_pred)
+        side_stream.wait_stream(main)
+        with torch.cuda.stream(side_stream):
+            _lib.lb_count(self.ids_pred, self.G, self.E, cnt=self.cnt_pred)
+            _lib.lb_plan_replicas(self.cnt_pred, self.N, self.L, plan=self.plan)
         self.route(h_cur, w, bias)
+        main.wait_stream(side_stream)
         self.solve()
 
-    LAUNCHES_PER_RUN = 5   # 2 gate, count, plan (lookahead); fused count + split + assign
+    LAUNCHES_PER_RUN = 8   # 2 gate, 2 count, plan, split, assign prep + scatter

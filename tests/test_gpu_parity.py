@@ -47,9 +47,23 @@ def test_small_full_path(name):
 
 def test_olmoe_all_layers_as_benchmarked():
     """The benchmark's launch configuration: all 16 OLMoE-shaped layers in one
-    batched pass; gate on sampled rows of every layer, integer stages exact."""
+    batched pass, lookahead counts and plan on a side stream, captured in a
+    CUDA graph and replayed; gate on sampled rows of every layer, integer
+    stages exact."""
     w = workloads.WORKLOADS["olmoe"]
-    hid, W, bias, path = run_model(w, w.layers)
+    hid, W, bias = parity.model_inputs(w, w.layers, DEV)
+    path = DecisionPath(w.layers, w.T, w.H, w.E, w.k, w.G, w.N, w.L, device=DEV)
+    side = torch.cuda.Stream()
+    path.run(hid[:-1], hid[1:], W, bias, side_stream=side)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        path.run(hid[:-1], hid[1:], W, bias, side_stream=side)
+    path.dest.fill_(-1)
+    path.perm.fill_(-1)
+    g.replay()
+    torch.cuda.synchronize()
+    assert _lib.lb_get_status() == 0
     rng = np.random.default_rng(0)
     for l in range(w.layers):
         rows = np.concatenate([rng.choice(w.T, 48, replace=False), [0, w.T - 1]])
@@ -350,10 +364,10 @@ def test_solve_fused_equals_separate_calls(name, T, B):
     path.ids.copy_(ids[1:])
     _lib.lb_count(path.ids_pred, w.G, w.E, cnt=path.cnt_pred)
     _lib.lb_plan_replicas(path.cnt_pred, w.N, w.L, plan=path.plan)
-    path.solve()
+    path.solve_fused()
     fused = [t.clone() for t in (path.cnt, path.tok, path.mass, path.loads, path.passes_run, path.dest, path.perm,
                                  path.offs)]
-    path.solve_separate()
+    path.solve()
     torch.cuda.synchronize()
     assert _lib.lb_get_status() == 0
     for f, s in zip(fused, (path.cnt, path.tok, path.mass, path.loads, path.passes_run, path.dest, path.perm,
