@@ -183,9 +183,14 @@ def run_ours(args, world, rank, local):
     bias = workloads.biases(wl, Lyr).to(dev)
     path = DecisionPath(Lyr, T, H, E, k, G, N, L, device=dev)
     side = torch.cuda.Stream(device=dev)
+    chain = args.gate == "chain"
 
     def step():
-        path.run(hid[:-1], hid[1:], W, bias, side_stream=side)
+        if chain:
+            path.run_chain(hid, W, bias)
+        else:
+            path.run(hid[:-1], hid[1:], W, bias, side_stream=side)
+    launches = path.LAUNCHES_PER_CHAIN if chain else path.LAUNCHES_PER_RUN
 
     # warm-up (also loads the library, sets kernel attributes, builds maps)
     for _ in range(args.warmup):
@@ -218,13 +223,17 @@ def run_ours(args, world, rank, local):
     if args.lean:
         return {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
                 "warmup": args.warmup, "ms_per_step": ms_step, "lean": True,
-                "gpu_launches": path.LAUNCHES_PER_RUN * args.steps, "clocks": clk.summary()}
+                "gpu_launches": launches * args.steps, "clocks": clk.summary()}
 
-    # ---------------- dominant kernel: the gate (two launches per step)
+    # ---------------- dominant kernel: the gate (one chain launch per step,
+    # or two launches in the two-pass form)
     g_gate = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g_gate):
-        _lib.lb_predict_topk(hid[:-1], W, bias, k, ids=path.ids_pred)
-        _lib.lb_predict_topk(hid[1:], W, bias, k, ids=path.ids)
+        if chain:
+            _lib.lb_predict_topk_chain(hid, W, bias, k, ids_pred=path.ids_pred, ids_act=path.ids)
+        else:
+            _lib.lb_predict_topk(hid[:-1], W, bias, k, ids=path.ids_pred)
+            _lib.lb_predict_topk(hid[1:], W, bias, k, ids=path.ids)
     g_gate.replay()
     torch.cuda.synchronize()
     barrier(world)
@@ -233,19 +242,28 @@ def run_ours(args, world, rank, local):
         g_gate.replay()
     ev1.record(stream)
     torch.cuda.synchronize()
-    gate_ms = ev0.elapsed_time(ev1) / (2 * args.steps)
-    gate_bytes = Lyr * (2 * T * H + 2 * H * E + 4 * E + 4 * T * k)
-    gate_flops = Lyr * 2.0 * T * H * E
+    if chain:
+        gate_ms = ev0.elapsed_time(ev1) / args.steps
+        gate_bytes = (Lyr + 1) * 2 * T * H + Lyr * (2 * H * E + 4 * E + 2 * 4 * T * k)
+        gate_flops = Lyr * 2 * 2.0 * T * H * E
+        tag = "gate_chain_olmoe16"
+    else:
+        gate_ms = ev0.elapsed_time(ev1) / (2 * args.steps)
+        gate_bytes = Lyr * (2 * T * H + 2 * H * E + 4 * E + 4 * T * k)
+        gate_flops = Lyr * 2.0 * T * H * E
+        tag = "gate_topk_olmoe16"
     hbm, tflops, peak_kind = peaks()
     achieved = gate_bytes / (gate_ms * 1e-3) / 1e9
-    traffic = profile_traffic("gate_topk_olmoe16", ["moe_expert_load_bf16_b200/csrc/gate_topk.cuh",
-                                                    "moe_expert_load_bf16_b200/csrc/common.cuh"])
+    traffic = profile_traffic(tag, ["moe_expert_load_bf16_b200/csrc/gate_topk.cuh",
+                                    "moe_expert_load_bf16_b200/csrc/common.cuh"])
+    if args.config != "olmoe":
+        traffic = None   # the committed captures are of the OLMoE-shaped launch
 
     # ---------------- per-layer latencies (single problem, graph replays)
     lat = per_layer_latency(wl, hid, W, bias, dev, reps=max(50, args.steps))
 
     # ---------------- end to end through the C ABI with host buffers
-    e2e = end_to_end(args, wl, hid, W, bias, path, dev, world)
+    e2e = end_to_end(args, wl, hid, W, bias, path, dev, world, chain)
 
     torch.cuda.synchronize()
     flags = _lib.lb_get_status()
@@ -259,18 +277,23 @@ def run_ours(args, world, rank, local):
         "config": {"workload": f"{wl.name}: {Lyr} layers x T={T} tokens, H={H}, E={E}, top-{k}, "
                                f"G={G} ranks, N={N} replica slots (L={L})",
                    "layers": Lyr, "T": T, "H": H, "E": E, "k": k, "G": G, "N": N, "L": L, "passes": 12,
-                   "batching": "all layers of a step in one launch per kernel, CUDA-graph replay; lookahead "
-                               "counts + plan on a second stream beside the normal-router gate",
-                   "l2": "inputs larger than L2 (hidden states %.0f MB per step)" % (2 * Lyr * T * H * 2 / 1e6),
+                   "batching": "all layers of a step in one launch per kernel, CUDA-graph replay",
+                   "gate": ("chain: one pass per hidden state evaluates the normal router of the layer before "
+                            "it and the lookahead of the layer after it" if chain else
+                            "two passes (lookahead, normal router); lookahead counts + plan on a second stream"),
+                   "l2": "inputs larger than L2 (hidden states %.0f MB read per step)" % (
+                       (Lyr + 1 if chain else 2 * Lyr) * T * H * 2 / 1e6),
                    "parallelism": f"{world} independent replicas"},
-        "t_solve_us": lat["solve"], "t_solve_fused_us": lat["solve_fused"], "t_split_us": lat["split"], "t_lookahead_us": lat["lookahead"],
+        "t_solve_us": lat["solve"], "t_solve_fused_us": lat["solve_fused"], "t_split_us": lat["split"],
+        "t_lookahead_us": lat["lookahead"],
         "per_kernel_us": lat["kernels"],
-        "roofline": {"kernel": "gate_topk", "bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
+        "roofline": {"kernel": "gate_topk_persistent (chain)" if chain else "gate_topk", "bound": "hbm",
+                     "achieved": achieved, "peak": hbm, "unit": "GB/s",
                      "frac": achieved / hbm, "traffic": traffic, "peak_kind": peak_kind,
                      "algorithmic_bytes_per_launch": gate_bytes, "launch_us": gate_ms * 1e3,
                      "tensor_frac": gate_flops / (gate_ms * 1e-3) / (tflops * 1e12)},
         "e2e": e2e,
-        "gpu_launches": path.LAUNCHES_PER_RUN * args.steps,
+        "gpu_launches": launches * args.steps,
         "clocks": clk.summary(),
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -322,7 +345,7 @@ def per_layer_latency(wl, hid, W, bias, dev, reps):
     return res
 
 
-def end_to_end(args, wl, hid, W, bias, path, dev, world):
+def end_to_end(args, wl, hid, W, bias, path, dev, world, chain=True):
     """Same metric through the public API with host buffers: every step
     copies its inputs from pinned host memory and reads its results back."""
     Lyr, T, k = wl.layers, wl.T, wl.k
@@ -338,7 +361,10 @@ def end_to_end(args, wl, hid, W, bias, path, dev, world):
         hid.copy_(h_host, non_blocking=True)
         W.copy_(w_host, non_blocking=True)
         bias.copy_(b_host, non_blocking=True)
-        path.run(hid[:-1], hid[1:], W, bias)
+        if chain:
+            path.run_chain(hid, W, bias)
+        else:
+            path.run(hid[:-1], hid[1:], W, bias)
         for o, oh in zip(outs, o_host):
             oh.copy_(o, non_blocking=True)
 
@@ -447,8 +473,8 @@ def run_decode(args, world, rank, local):
 # ----------------------------------------------------------------------------- CPU oracle
 def cpu_baseline(wl, budget_s=15.0):
     """The oracle, as it stands, on this host's cores, over whole layers of
-    the workload (both gate calls, count, plan, count, split, assign) until
-    the time budget is spent.  If one layer's gate would not fit the budget,
+    the workload (both gate calls, count, plan, count, split, assign),
+    repeated on one layer's inputs until the time budget is spent.  If one layer's gate would not fit the budget,
     the gate runs on evenly spaced sampled rows and its time is scaled to the
     full layer (the integer stages always run on the whole layer)."""
     import oracle
@@ -471,7 +497,7 @@ def cpu_baseline(wl, budget_s=15.0):
         ids_pred_full = o.gate(hb[0], wb, b, k)[1]
         ids_full = o.gate(hb[1], wb, b, k)[1]
     total, layers, t_start = 0.0, 0, time.perf_counter()
-    while layers == 0 or (time.perf_counter() - t_start < budget_s and layers < wl.layers):
+    while layers == 0 or time.perf_counter() - t_start < budget_s:
         t0 = time.perf_counter()
         _, ids_pred = o.gate(hb[0][sel], wb, b, k)
         t_gate = time.perf_counter() - t0
@@ -492,8 +518,8 @@ def cpu_baseline(wl, budget_s=15.0):
         t_int += time.perf_counter() - t1
         total += t_gate * T / rows + t_int
         layers += 1
-    sample = (f"{layers} full layer(s) of {wl.name} (T={T}, H={H}, E={E}, top-{k}): both gate calls, "
-              f"count, plan, count, split, assign")
+    sample = (f"{layers} full layer pass(es) of {wl.name} (T={T}, H={H}, E={E}, top-{k}) on one layer's "
+              f"inputs: both gate calls, count, plan, count, split, assign")
     if rows < T:
         sample += f"; gate on {rows} of {T} rows per call, time scaled to the full layer"
     return {"value": layers * T * k / total, "unit": UNIT, "cores": o.threads(), "kind": "oracle",
@@ -533,6 +559,9 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--config", default=DEFAULT_WORKLOAD)
     ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--gate", choices=("chain", "two-pass"), default="chain",
+                    help="chain: one gate pass per hidden state for both gates that read it; two-pass: "
+                         "lookahead and normal router as separate passes")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--lean", action="store_true",
                     help="time the steps only (no gate-only loop, per-layer latencies, end-to-end or CPU "

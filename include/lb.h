@@ -85,6 +85,35 @@ int lb_predict_topk(const void *h, const void *w, const float *bias,
                     int nbatch, int T, int H, int E, int k,
                     int32_t *ids, float *logits, void *stream);
 
+/* ------------------------------------------------------------------------
+ * Step 1 over a chain of layers -- both gates that read one hidden state,
+ * in one pass   [FB sec. 3.2 eq. 2-5: layer l's routing is predicted from
+ * the hidden state that precedes it, with layer l's own gate]
+ * Hidden state h_j (j = 0..L) is the input of layer j-1's normal router and
+ * of layer j's lookahead, so one read of h_j serves both:
+ *   ids_pred[l] = top-k(h[l]   . w[l]^T + bias[l])   l = 0..L-1  (lookahead)
+ *   ids_act[l]  = top-k(h[l+1] . w[l]^T + bias[l])   l = 0..L-1  (normal)
+ * Layer 0's lookahead reads h_0, the state before layer 0.  Each row's
+ * ranking is that of lb_predict_topk (descending, ties to the lower id),
+ * and the logits equal lb_predict_topk's up to fp32 summation order.
+ *   h            bf16 [L+1, T, H] row-major, 16-byte aligned
+ *   w            bf16 [L, E, H], 16-byte aligned (gates of consecutive
+ *                layers adjacent in memory)
+ *   bias         fp32 [L, E] or NULL
+ *   ids_pred     int32 [L, T, k]                          (output)
+ *   ids_act      int32 [L, T, k]                          (output)
+ *   logits_pred, logits_act   fp32 [L, T, E] or NULL       (optional outputs)
+ * Limits: 16 <= E <= 128 with E % 16 == 0 (the two gates form one MMA tile
+ * of N = 2E <= 256 columns), 1 <= k <= min(E, LB_MAX_K_GATE), H >= 8 and
+ * H % 8 == 0, 1 <= L <= 65534, T >= 0.  Other shapes: LB_EINVAL (call
+ * lb_predict_topk twice instead).  Tuning knobs of lb_gate_tuning that apply
+ * to the persistent kernel (stages, CTAs per SM, boxes per stage) apply here.
+ * ------------------------------------------------------------------------ */
+int lb_predict_topk_chain(const void *h, const void *w, const float *bias,
+                          int L, int T, int H, int E, int k,
+                          int32_t *ids_pred, int32_t *ids_act,
+                          float *logits_pred, float *logits_act, void *stream);
+
 /* Tuning knobs of lb_predict_topk (process-wide; 0 = automatic choice):
  * pipeline stages per CTA (2..8); split of H across a CTA cluster (1, 2, 4,
  * 8 or 16); persistent kernel (1, 2 or 4 = that many CTAs per SM walking the

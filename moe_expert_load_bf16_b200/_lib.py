@@ -45,6 +45,7 @@ def _load():
     lib = ctypes.CDLL(LIB_PATH)
     P, I, SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
     lib.lb_predict_topk.argtypes = [P, P, P, I, I, I, I, I, P, P, P]
+    lib.lb_predict_topk_chain.argtypes = [P, P, P, I, I, I, I, I, P, P, P, P, P]
     lib.lb_gate_tuning.argtypes = [I, I, I, I]
     lib.lb_count.argtypes = [P, I, I, I, I, I, P, P]
     lib.lb_plan_bytes.argtypes = [I, I, I]
@@ -124,6 +125,43 @@ def lb_predict_topk(h, w, bias, k, want_logits=False, ids=None, logits=None):
         ids = ids[0]
         logits = logits[0] if want_logits else None
     return (ids, logits) if want_logits else ids
+
+
+def lb_predict_topk_chain(h, w, bias, k, want_logits=False, ids_pred=None, ids_act=None, logits_pred=None,
+                          logits_act=None):
+    """Both gates that read each hidden state of a chain, in one pass.
+    h bf16 [L+1,T,H], w bf16 [L,E,H], bias f32 [L,E] or None.
+    ids_pred[l] = top-k(h[l] w[l]^T + b[l]) (lookahead of layer l),
+    ids_act[l] = top-k(h[l+1] w[l]^T + b[l]) (normal router of layer l).
+    Returns (ids_pred, ids_act) int32 [L,T,k], plus (logits_pred, logits_act)
+    f32 [L,T,E] when want_logits."""
+    lib = _load()
+    _need(h, torch.bfloat16, "h")
+    _need(w, torch.bfloat16, "w")
+    if h.dim() != 3 or w.dim() != 3:
+        raise ValueError("h must be [L+1,T,H] and w [L,E,H]")
+    L1, T, H = h.shape
+    L, E = w.shape[0], w.shape[1]
+    if L1 != L + 1 or w.shape[2] != H:
+        raise ValueError("h must be [L+1,T,H] for w [L,E,H]")
+    if bias is not None:
+        _need(bias, torch.float32, "bias")
+        if bias.shape != (L, E):
+            raise ValueError("bias must be [L,E]")
+    outs = []
+    for t in (ids_pred, ids_act):
+        t = torch.empty(L, T, k, dtype=torch.int32, device=h.device) if t is None else t
+        _need(t, torch.int32, "ids")
+        if t.shape != (L, T, k):
+            raise ValueError("ids outputs must be [L,T,k]")
+        outs.append(t)
+    lg = [None, None]
+    if want_logits:
+        lg = [torch.empty(L, T, E, dtype=torch.float32, device=h.device) if t is None else t
+              for t in (logits_pred, logits_act)]
+    _check("lb_predict_topk_chain", lib.lb_predict_topk_chain(_p(h), _p(w), _p(bias), L, T, H, E, k, _p(outs[0]),
+                                                              _p(outs[1]), _p(lg[0]), _p(lg[1]), _stream()))
+    return (outs[0], outs[1], lg[0], lg[1]) if want_logits else (outs[0], outs[1])
 
 
 def lb_gate_tuning(stages=0, split=0, persistent=0, kbox=0):
@@ -297,7 +335,7 @@ def lb_version():
     return int(_load().lb_version())
 
 
-EXPORTS = ("lb_predict_topk", "lb_gate_tuning", "lb_count", "lb_plan_bytes", "lb_plan_layout_of",
+EXPORTS = ("lb_predict_topk", "lb_predict_topk_chain", "lb_gate_tuning", "lb_count", "lb_plan_bytes", "lb_plan_layout_of",
            "lb_plan_replicas", "lb_split", "lb_assign_workspace_bytes", "lb_assign", "lb_assign_noalloc", "lb_solve",
            "lb_get_status",
            "lb_strerror", "lb_last_error", "lb_version")

@@ -38,6 +38,14 @@ struct Params {
     int T, H, E, Epad, k, nkb, split, stages;
     int kbox;            // persistent kernel: 64-column boxes per pipeline stage
     uint32_t tmem_cols;
+    // Chain mode (persistent kernel only): problem b = 0..L is hidden state
+    // h_b, and its B tile is rows [(b-1)E, (b+1)E) of the [L*E, H] stack of
+    // gates, i.e. W_{b-1} then W_b (rows outside the stack read as zeros).
+    // Columns [0,E) rank into ids/logits of layer b-1 (its normal router),
+    // columns [E,2E) into ids2/logits2 of layer b (its lookahead).
+    int chain, L;
+    int32_t *ids2;       // [L,T,k]
+    float *logits2;      // [L,T,E] or null
 };
 
 template <int KMAX>
@@ -318,6 +326,14 @@ __global__ void __launch_bounds__(THREADS, 1)
 // accumulator is double-buffered (2 x Epad columns), so the top-k of tile i
 // overlaps the loads and MMAs of tile i+1.  h is streamed once (L2
 // evict-first); W is re-read by every tile of its problem (L2 evict-last).
+//
+// In chain mode (see Params) the kernel evaluates both gates that read one
+// hidden state: h_b feeds the normal router of layer b-1 (gate W_{b-1}) and
+// the lookahead of layer b (gate W_b, FreeBalance sec. 3.2, predicted
+// routing from the previous layer's hidden state).  The two gates are
+// adjacent rows of the stacked [L*E, H] weights, so one N = 2E MMA tile per
+// k-block covers both, and each hidden state crosses HBM once instead of
+// twice.
 constexpr int P_THREADS = 192;
 
 template <int KMAX>
@@ -390,8 +406,9 @@ __global__ void __launch_bounds__(P_THREADS, 1)
                     mbar_arrive_expect_tx(&full_bar[s], stage_bytes);
                     for (int j = 0; j < kbox; ++j)
                         tma_load_3d_hint(&tmA, sa + j * a_box, &full_bar[s], (ks * kbox + j) * BK, m0, b, pol_a);
+                    const int by = p.chain ? (b - 1) * p.E : 0, bz = p.chain ? 0 : b;
                     for (int j = 0; j < kbox; ++j)
-                        tma_load_3d_hint(&tmB, sa + a_bytes + j * b_box, &full_bar[s], (ks * kbox + j) * BK, 0, b,
+                        tma_load_3d_hint(&tmB, sa + a_bytes + j * b_box, &full_bar[s], (ks * kbox + j) * BK, by, bz,
                                          pol_b);
                 }
             }
@@ -464,35 +481,47 @@ __global__ void __launch_bounds__(P_THREADS, 1)
             const int b = tile / mtiles, m0 = (tile - b * mtiles) * BM;
             const int row = m0 + rloc;
             const bool valid = row < p.T;
-            const int64_t grow = static_cast<int64_t>(b) * p.T + row;
-            const float *bias = p.bias != nullptr ? p.bias + static_cast<int64_t>(b) * p.E : nullptr;
-            float *lrow = (p.logits != nullptr && valid) ? p.logits + grow * p.E : nullptr;
-            TopK<KMAX> tk;
-            tk.init();
             const uint32_t tl_addr = tmem + buf * half + (static_cast<uint32_t>(q * 32) << 16);
-            for (int c0 = 0; c0 < p.Epad; c0 += 16) {
-                uint32_t r[16];
-                tmem_ld16(tl_addr + c0, r);
-                tmem_wait_ld();
+            // One output (normal mode) or two column halves (chain mode); the
+            // layer of each is uniform across the tile, so a skipped half
+            // skips its warp-collective TMEM loads in every lane alike.
+            const int nhalf = p.chain ? 2 : 1;
+            for (int hh = 0; hh < nhalf; ++hh) {
+                const int layer = p.chain ? b - 1 + hh : b;
+                if (layer < 0 || (p.chain && layer >= p.L)) continue;
+                int32_t *ids_out = (p.chain && hh == 1) ? p.ids2 : p.ids;
+                float *lg_out = (p.chain && hh == 1) ? p.logits2 : p.logits;
+                const int64_t grow = static_cast<int64_t>(layer) * p.T + row;
+                const float *bias = p.bias != nullptr ? p.bias + static_cast<int64_t>(layer) * p.E : nullptr;
+                float *lrow = (lg_out != nullptr && valid) ? lg_out + grow * p.E : nullptr;
+                const int cols = p.chain ? p.E : p.Epad;
+                const uint32_t col0 = p.chain ? static_cast<uint32_t>(hh * p.E) : 0u;
+                TopK<KMAX> tk;
+                tk.init();
+                for (int c0 = 0; c0 < cols; c0 += 16) {
+                    uint32_t r[16];
+                    tmem_ld16(tl_addr + col0 + c0, r);
+                    tmem_wait_ld();
 #pragma unroll
-                for (int j = 0; j < 16; ++j) {
-                    const int c = c0 + j;
-                    if (c < p.E) {
-                        const float x = __uint_as_float(r[j]) + (bias != nullptr ? __ldg(bias + c) : 0.f);
-                        tk.push(x, c);
-                        if (lrow) lrow[c] = x;
+                    for (int j = 0; j < 16; ++j) {
+                        const int c = c0 + j;
+                        if (c < p.E) {
+                            const float x = __uint_as_float(r[j]) + (bias != nullptr ? __ldg(bias + c) : 0.f);
+                            tk.push(x, c);
+                            if (lrow) lrow[c] = x;
+                        }
                     }
+                }
+                if (valid) {
+                    int32_t *out = ids_out + grow * p.k;
+#pragma unroll
+                    for (int j = 0; j < KMAX; ++j)
+                        if (j < p.k) out[j] = tk.i[j];
                 }
             }
             // the accumulator buffer may be overwritten from here
             tc_fence_before();
             mbar_arrive(&acc_empty[buf]);
-            if (valid) {
-                int32_t *out = p.ids + grow * p.k;
-#pragma unroll
-                for (int j = 0; j < KMAX; ++j)
-                    if (j < p.k) out[j] = tk.i[j];
-            }
         }
     }
 

@@ -150,6 +150,38 @@ int launch_gate_persistent_k(int k, const CUtensorMap &ma, const CUtensorMap &mb
     return launch_gate_persistent<16>(ma, mb, p, mtiles, ntiles, grid, smem, s);
 }
 
+// Persistent gate launch shared by lb_predict_topk and lb_predict_topk_chain:
+// TMEM columns for two accumulators of p.Epad, boxes per stage, stages, and
+// shared memory padded so that at most per_sm CTAs share an SM.  The h map
+// covers nprob problems of [T, H].
+int run_persistent(gate::Params &p, const void *h, int nprob, const CUtensorMap &mb, int per_sm, int mtiles,
+                   long long ntiles, int sms, cudaStream_t s) {
+    uint32_t pcols = 32;
+    while (pcols < 2u * static_cast<uint32_t>(p.Epad)) pcols <<= 1;
+    if (pcols > 512 || static_cast<uint32_t>(per_sm) * pcols > 512) return LB_EINVAL;
+    p.tmem_cols = pcols;
+    p.split = 1;
+    p.kbox = g_tune_kbox ? g_tune_kbox : (p.Epad <= 64 ? 2 : 1);
+    const size_t stage_bytes = (16384 + static_cast<size_t>(p.Epad) * 128) * p.kbox;
+    int stages = g_tune_stages;
+    if (!stages)
+        stages = static_cast<int>(
+            std::max<size_t>(2, std::min<size_t>(gate::MAX_STAGES, (100 * 1024 * 2 / per_sm) / stage_bytes)));
+    if (stages < 2) return LB_EINVAL;
+    size_t smem = stages * stage_bytes + 1024;
+    smem = std::max(smem, static_cast<size_t>(228 * 1024) / (per_sm + 1) + 1);   // at most per_sm CTAs per SM
+    if (smem > 224 * 1024) return LB_EINVAL;
+    p.stages = stages;
+    CUtensorMap ma;
+    if (!make_map(&ma, h, static_cast<uint64_t>(p.H), static_cast<uint64_t>(p.T), static_cast<uint64_t>(nprob),
+                  gate::BM)) {
+        std::snprintf(g_last_error, sizeof g_last_error, "cuTensorMapEncodeTiled failed for h");
+        return LB_ECUDA;
+    }
+    const int grid = static_cast<int>(std::min<long long>(ntiles, static_cast<long long>(sms) * per_sm));
+    return launch_gate_persistent_k(p.k, ma, mb, p, mtiles, static_cast<int>(ntiles), grid, smem, s);
+}
+
 template <bool SPLITK>
 int launch_gate_k(int k, const CUtensorMap &ma, const CUtensorMap &mb, const gate::Params &p, int mtiles,
                   int nbatch, size_t smem, cudaStream_t s) {
@@ -255,7 +287,7 @@ int lb_predict_topk(const void *h, const void *w, const float *bias, int nbatch,
     if (T == 0) return LB_OK;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
 
-    gate::Params p;
+    gate::Params p{};
     p.bias = bias;
     p.ids = ids;
     p.logits = logits;
@@ -280,35 +312,14 @@ int lb_predict_topk(const void *h, const void *w, const float *bias, int nbatch,
     // per tile.
     int per_sm = g_tune_persistent;
     if (per_sm == 0 && g_tune_split <= 1 && ntiles >= 2LL * sms && p.Epad <= 128) per_sm = 2;
-    const bool persistent = per_sm > 0;
-    if (persistent) {
-        uint32_t pcols = 32;
-        while (pcols < 2u * static_cast<uint32_t>(p.Epad)) pcols <<= 1;
-        if (pcols > 512) return LB_EINVAL;
-        p.tmem_cols = pcols;
-        p.split = 1;
-        p.kbox = g_tune_kbox ? g_tune_kbox : (p.Epad <= 64 ? 2 : 1);
-        const size_t stage_bytes = (16384 + static_cast<size_t>(p.Epad) * 128) * p.kbox;
-        if (static_cast<uint32_t>(per_sm) * pcols > 512) return LB_EINVAL;
-        int stages = g_tune_stages;
-        if (!stages)
-            stages = static_cast<int>(
-                std::max<size_t>(2, std::min<size_t>(gate::MAX_STAGES, (100 * 1024 * 2 / per_sm) / stage_bytes)));
-        if (stages < 2) return LB_EINVAL;
-        size_t smem = stages * stage_bytes + 1024;
-        smem = std::max(smem, static_cast<size_t>(228 * 1024) / (per_sm + 1) + 1);   // at most per_sm CTAs per SM
-        if (smem > 224 * 1024) return LB_EINVAL;
-        p.stages = stages;
-        CUtensorMap ma, mb;
-        if (!make_map(&ma, h, static_cast<uint64_t>(H), static_cast<uint64_t>(T), static_cast<uint64_t>(nbatch),
-                      gate::BM) ||
-            !make_map(&mb, w, static_cast<uint64_t>(H), static_cast<uint64_t>(E), static_cast<uint64_t>(nbatch),
+    if (per_sm > 0) {
+        CUtensorMap mb;
+        if (!make_map(&mb, w, static_cast<uint64_t>(H), static_cast<uint64_t>(E), static_cast<uint64_t>(nbatch),
                       static_cast<uint32_t>(p.Epad))) {
-            std::snprintf(g_last_error, sizeof g_last_error, "cuTensorMapEncodeTiled failed");
+            std::snprintf(g_last_error, sizeof g_last_error, "cuTensorMapEncodeTiled failed for w");
             return LB_ECUDA;
         }
-        const int grid = static_cast<int>(std::min<long long>(ntiles, static_cast<long long>(sms) * per_sm));
-        return launch_gate_persistent_k(k, ma, mb, p, mtiles, static_cast<int>(ntiles), grid, smem, s);
+        return run_persistent(p, h, nbatch, mb, per_sm, mtiles, ntiles, sms, s);
     }
 
     // split of H across a cluster when the token tiles alone underfill the GPU
@@ -364,6 +375,54 @@ int lb_predict_topk(const void *h, const void *w, const float *bias, int nbatch,
     }
     return S > 1 ? launch_gate_k<true>(k, ma, mb, p, mtiles, nbatch, smem, s)
                  : launch_gate_k<false>(k, ma, mb, p, mtiles, nbatch, smem, s);
+}
+
+int lb_predict_topk_chain(const void *h, const void *w, const float *bias, int L, int T, int H, int E, int k,
+                          int32_t *ids_pred, int32_t *ids_act, float *logits_pred, float *logits_act,
+                          void *stream) {
+    if (L < 1 || L > 65534 || T < 0 || H < 8 || H % 8 != 0 || E < 16 || E % 16 != 0 || 2 * E > 256 || k < 1 ||
+        k > E || k > LB_MAX_K_GATE)
+        return LB_EINVAL;
+    if (!h || !w || !ids_pred || !ids_act || !aligned(h, 16) || !aligned(w, 16) || !aligned(ids_pred, 4) ||
+        !aligned(ids_act, 4))
+        return LB_EINVAL;
+    if ((bias && !aligned(bias, 4)) || (logits_pred && !aligned(logits_pred, 4)) ||
+        (logits_act && !aligned(logits_act, 4)))
+        return LB_EINVAL;
+    if (static_cast<long long>(T) * (L + 1) * std::max(k, E) >= INT_MAX ||
+        static_cast<long long>(L) * E * H * 2 >= (1LL << 40))
+        return LB_EINVAL;
+    if (T == 0) return LB_OK;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+
+    gate::Params p{};
+    p.bias = bias;
+    p.ids = ids_act;
+    p.logits = logits_act;
+    p.ids2 = ids_pred;
+    p.logits2 = logits_pred;
+    p.chain = 1;
+    p.L = L;
+    p.T = T;
+    p.H = H;
+    p.E = E;
+    p.Epad = 2 * E;   // the MMA's N: W_{b-1} and W_b side by side
+    p.k = k;
+    p.nkb = (H + gate::BK - 1) / gate::BK;
+    const int mtiles = (T + gate::BM - 1) / gate::BM;
+    const int sms = device_sms();
+    const long long ntiles = static_cast<long long>(mtiles) * (L + 1);
+    uint32_t pcols = 32;
+    while (pcols < 4u * static_cast<uint32_t>(E)) pcols <<= 1;
+    int per_sm = g_tune_persistent > 0 ? g_tune_persistent : std::max(1, std::min(2, static_cast<int>(512 / pcols)));
+    // the stack of gates as one [L*E, H] matrix; a box of 2E rows starting
+    // at row (b-1)E (negative for b = 0, past the end for b = L: zeros)
+    CUtensorMap mb;
+    if (!make_map(&mb, w, static_cast<uint64_t>(H), static_cast<uint64_t>(L) * E, 1, static_cast<uint32_t>(2 * E))) {
+        std::snprintf(g_last_error, sizeof g_last_error, "cuTensorMapEncodeTiled failed for w");
+        return LB_ECUDA;
+    }
+    return run_persistent(p, h, L + 1, mb, per_sm, mtiles, ntiles, sms, s);
 }
 
 int lb_count(const int32_t *ids, int nbatch, int T, int k, int E, int G, int32_t *cnt, void *stream) {

@@ -3,7 +3,8 @@ steps or micro-batches of identical shape), with every buffer preallocated so
 the pass can be captured in a CUDA graph.
 
 Per problem (Libra README, Key Ideas; FreeBalance sec. 3.2, Algorithm 1;
-Relief, Algorithm 1):
+Relief, Algorithm 1); over a chain of consecutive layers, `run_chain` runs
+both gates that read one hidden state in a single pass over it:
   ids_pred = top-k(gate(h_prev))           lookahead        lb_predict_topk
   cnt_pred = counts(ids_pred)                               lb_count
   plan     = replica plan(cnt_pred)                         lb_plan_replicas
@@ -23,11 +24,13 @@ class DecisionPath:
         self.passes = passes
         dev = torch.device(device)
         i32 = dict(dtype=torch.int32, device=dev)
-        self.ids_pred = torch.empty(B, T, k, **i32)
-        self.cnt_pred = torch.empty(B, G, E, **i32)
+        # predicted and actual ids (and counts) side by side, so one launch
+        # can fill or count both
+        self.ids_both = torch.empty(2, B, T, k, **i32)
+        self.cnt_both = torch.empty(2, B, G, E, **i32)
+        self.ids_pred, self.ids = self.ids_both[0], self.ids_both[1]
+        self.cnt_pred, self.cnt = self.cnt_both[0], self.cnt_both[1]
         self.plan = torch.empty(B, _lib.lb_plan_bytes(G, E, N), dtype=torch.uint8, device=dev)
-        self.ids = torch.empty(B, T, k, **i32)
-        self.cnt = torch.empty(B, G, E, **i32)
         self.tok = torch.empty(B, G * N, **i32)
         self.mass = torch.empty(B, G * N, **i32)
         self.loads = torch.empty(B, G, **i32)
@@ -50,9 +53,10 @@ class DecisionPath:
     # the per-step decision on actual ids (T_solve): lb_count, lb_split,
     # lb_assign (on the benchmark shapes these three launches are faster than
     # the fused lb_solve, whose single CTA 0 runs split and tables in series)
-    def solve(self, ids=None):
+    def solve(self, ids=None, counted=False):
         ids = self.ids if ids is None else ids
-        _lib.lb_count(ids, self.G, self.E, cnt=self.cnt)
+        if not counted:
+            _lib.lb_count(ids, self.G, self.E, cnt=self.cnt)
         _lib.lb_split(self.cnt, self.plan, self.N, self.passes,
                       out=(self.tok, self.mass, self.loads, self.passes_run))
         _lib.lb_assign(ids, self.cnt, self.plan, self.tok, self.mass, self.N,
@@ -85,3 +89,19 @@ class DecisionPath:
         self.solve()
 
     LAUNCHES_PER_RUN = 8   # 2 gate, 2 count, plan, split, assign prep + scatter
+
+    def run_chain(self, hid, w, bias):
+        """One pass over a chain of B consecutive layers whose hidden states
+        are hid [B+1, T, H]: layer l predicts from hid[l] and routes hid[l+1]
+        (the same problems as run(hid[:-1], hid[1:], w, bias)).  Both gates
+        that read one hidden state run in one pass over it
+        (lb_predict_topk_chain); predicted and actual ids are counted in one
+        launch."""
+        B = self.B
+        _lib.lb_predict_topk_chain(hid, w, bias, self.k, ids_pred=self.ids_pred, ids_act=self.ids)
+        _lib.lb_count(self.ids_both.view(2 * B, self.T, self.k), self.G, self.E,
+                      cnt=self.cnt_both.view(2 * B, self.G, self.E))
+        _lib.lb_plan_replicas(self.cnt_pred, self.N, self.L, plan=self.plan)
+        self.solve(counted=True)
+
+    LAUNCHES_PER_CHAIN = 6   # chain gate, count (both), plan, split, assign prep + scatter

@@ -56,6 +56,10 @@ def test_arguments_rejected_before_any_launch(lib):
     assert lib.lb_predict_topk(P(16), P(16), None, 1, 128, 64, 300, 2, P(16), None, s) == _lib.LB_EINVAL
     assert lib.lb_predict_topk(P(16), P(16), None, 1, 128, 64, 4, 5, P(16), None, s) == _lib.LB_EINVAL
     assert lib.lb_predict_topk(P(16), P(16), None, 1, 128, 60, 16, 2, P(16), None, s) == _lib.LB_EINVAL
+    # chain gate: E = 256 (N = 2E > 256), E % 16, L = 0, k > E
+    for L, E, k in ((2, 256, 2), (2, 24, 2), (0, 64, 2), (2, 16, 17)):
+        assert lib.lb_predict_topk_chain(P(16), P(16), None, L, 128, 64, E, k, P(16), P(16), None, None,
+                                         s) == _lib.LB_EINVAL
     assert lib.lb_count(P(16), 1, 10, 2, 16, 4, P(16), s) == _lib.LB_EINVAL          # T % G
     assert lib.lb_plan_replicas(P(256), 1, 3, 16, 1, 0, P(256), s) == _lib.LB_EINVAL  # E % G
     assert lib.lb_plan_replicas(P(256), 1, 4, 16, 20, 0, P(256), s) == _lib.LB_EINVAL  # N > E - E/G

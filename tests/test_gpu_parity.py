@@ -375,3 +375,60 @@ def test_solve_fused_equals_separate_calls(name, T, B):
         assert torch.equal(f, s)
     for b in range(B):
         parity.check_path(path, b, 12)
+
+
+@pytest.mark.parametrize("L,T,H,E,k,bias_on", [(3, 200, 128, 16, 2, True), (1, 256, 64, 16, 4, True),
+                                               (4, 4096, 2048, 64, 8, True), (2, 1100, 2048, 128, 8, True),
+                                               (5, 3000, 576, 64, 8, False), (2, 130, 8, 32, 16, True)])
+def test_gate_chain(L, T, H, E, k, bias_on):
+    """lb_predict_topk_chain: for every layer l, the lookahead ids from
+    hid[l] and the normal-router ids from hid[l+1] (with gate W_l) pass the
+    oracle check and agree with lb_predict_topk on the same rows.  Distinct
+    hidden states, so reading the wrong one (or the wrong layer's gate) fails.
+    Shapes: ragged last tile, one layer (both boundary states), E = 128 (one
+    CTA per SM), a stage of boxes past H, no bias, H = 8."""
+    g = torch.Generator(device=DEV).manual_seed(100 + L * 7 + E)
+    hid = torch.randn(L + 1, T, H, generator=g, device=DEV).to(torch.bfloat16)
+    W = (torch.randn(L, E, H, generator=g, device=DEV) / H ** 0.5).to(torch.bfloat16)
+    bias = torch.randn(L, E, generator=g, device=DEV) if bias_on else None
+    ip, ia, lp, la = _lib.lb_predict_topk_chain(hid, W, bias, k, want_logits=True)
+    torch.cuda.synchronize()
+    assert _lib.lb_get_status() == 0
+    rng = np.random.default_rng(L + T)
+    rows = None if T <= 256 else np.unique(np.concatenate([rng.choice(T, 96, replace=False),
+                                                           [0, 127, 128, T - 1]]))
+    for l in range(L):
+        bl = None if bias is None else bias[l]
+        for src, ids, lg in ((hid[l], ip[l], lp[l]), (hid[l + 1], ia[l], la[l])):
+            parity.gate_check(src, W[l], bl, k, ids, lg, rows=rows)
+            ids1, lg1 = _lib.lb_predict_topk(src, W[l], bl, k, want_logits=True)
+            assert torch.allclose(lg, lg1, rtol=1e-5, atol=1e-5)
+            assert (ids == ids1).all(dim=1).float().mean().item() > 0.999
+
+
+def test_gate_chain_drives_the_path():
+    """DecisionPath.run_chain (one gate pass per hidden state, both id sets
+    counted in one launch) gives the same bytes downstream as run() on the
+    same hidden chain, when the gates agree."""
+    w = workloads.WORKLOADS["olmoe"]
+    hid, W, bias = parity.model_inputs(w, 4, DEV)
+    hid[0].copy_((hid[0].float() * 0.9).to(torch.bfloat16))   # a distinct h_0
+    a = DecisionPath(4, w.T, w.H, w.E, w.k, w.G, w.N, w.L, device=DEV)
+    b = DecisionPath(4, w.T, w.H, w.E, w.k, w.G, w.N, w.L, device=DEV)
+    a.run_chain(hid, W, bias)
+    b.run(hid[:-1], hid[1:], W, bias)
+    torch.cuda.synchronize()
+    assert _lib.lb_get_status() == 0
+    if torch.equal(a.ids_both, b.ids_both):
+        for f in ("cnt_both", "plan", "tok", "mass", "loads", "passes_run", "dest", "perm", "offs"):
+            assert torch.equal(getattr(a, f), getattr(b, f)), f
+    for l in range(4):
+        parity.check_path(a, l, 12)
+
+
+@pytest.mark.parametrize("E,L", [(256, 2), (24, 2), (64, 0)])
+def test_gate_chain_rejects_unsupported_shapes(E, L):
+    hid = torch.zeros(L + 1, 128, 64, dtype=torch.bfloat16, device=DEV)
+    W = torch.zeros(max(L, 1), E, 64, dtype=torch.bfloat16, device=DEV)[:L]
+    with pytest.raises((_lib.LBError, ValueError)):
+        _lib.lb_predict_topk_chain(hid, W, None, 2)
