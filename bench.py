@@ -262,6 +262,9 @@ def run_ours(args, world, rank, local):
     # ---------------- per-layer latencies (single problem, graph replays)
     lat = per_layer_latency(wl, hid, W, bias, dev, reps=max(50, args.steps))
 
+    # ---------------- count / split / assign as throughput kernels
+    ints = integer_kernels_at_throughput(dev, world)
+
     # ---------------- end to end through the C ABI with host buffers
     e2e = end_to_end(args, wl, hid, W, bias, path, dev, world, chain)
 
@@ -292,6 +295,7 @@ def run_ours(args, world, rank, local):
                      "frac": achieved / hbm, "traffic": traffic, "peak_kind": peak_kind,
                      "algorithmic_bytes_per_launch": gate_bytes, "launch_us": gate_ms * 1e3,
                      "tensor_frac": gate_flops / (gate_ms * 1e-3) / (tflops * 1e12)},
+        "integer_kernels": ints,
         "e2e": e2e,
         "gpu_launches": launches * args.steps,
         "clocks": clk.summary(),
@@ -343,6 +347,66 @@ def per_layer_latency(wl, hid, W, bias, dev, reps):
                                                out=(p1.dest, p1.perm, p1.offs), workspace=p1.ws)),
     }
     return res
+
+
+def integer_kernels_at_throughput(dev, world, nbatch=128, reps=20):
+    """Count, split and assign (prep + scatter) as throughput kernels: one
+    launch over `nbatch` independent Qwen3-235B-shaped problems (T=32768,
+    top-8, E=128, G=8, N=4), ids larger than L2 in total.  Each kernel group
+    is graph-replayed alone; achieved = algorithmic bytes / mean time."""
+    from moe_expert_load_bf16_b200 import _lib, workloads
+    from moe_expert_load_bf16_b200.pipeline import DecisionPath
+    wl = workloads.WORKLOADS["qwen3-235b"]
+    T, E, k, G, N, L = wl.T, wl.E, wl.k, wl.G, wl.N, wl.L
+    ids = torch.empty(nbatch, T, k, dtype=torch.int32, device=dev)
+    for c0 in range(0, nbatch, 16):
+        ids[c0:c0 + 16].copy_(workloads.decode_ids(wl, T, range(c0, min(nbatch, c0 + 16)), device=dev))
+    path = DecisionPath(nbatch, T, 8, E, k, G, N, L, device=dev)
+    path.ids.copy_(ids)
+    del ids
+    _lib.lb_count(path.ids, G, E, cnt=path.cnt)
+    _lib.lb_plan_replicas(path.cnt, N, L, plan=path.plan)   # any valid plan serves the throughput run
+    path.solve()
+    torch.cuda.synchronize()
+
+    def timed(fn):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            fn()
+        g.replay()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier(world)
+        a.record()
+        for _ in range(reps):
+            g.replay()
+        b.record()
+        torch.cuda.synchronize()
+        return max_over_ranks(a.elapsed_time(b) / reps, world) * 1e3
+
+    n_edges = sum(int(d["n_edges"]) for d in _lib.decode_plan(path.plan, G, E, N)) / nbatch
+    t_count = timed(lambda: _lib.lb_count(path.ids, G, E, cnt=path.cnt))
+    t_split = timed(lambda: _lib.lb_split(path.cnt, path.plan, N, 12,
+                                          out=(path.tok, path.mass, path.loads, path.passes_run)))
+    t_assign = timed(lambda: _lib.lb_assign(path.ids, path.cnt, path.plan, path.tok, path.mass, N,
+                                            out=(path.dest, path.perm, path.offs), workspace=path.ws))
+    if _lib.lb_get_status():
+        raise RuntimeError("device status flagged in the integer-kernel run")
+    hbm, _, _ = peaks()
+    tk = T * k
+    by = {"count": nbatch * (4 * tk + 4 * G * E),
+          "split": int(nbatch * (4 * G * E + 12 * n_edges + 16 * G * N + 4 * G)),
+          "assign": nbatch * (3 * 4 * tk + 4 * (G * E + 1) + 4 * G * E + 8 * G * N)}
+    out = {"workload": f"{nbatch} problems x (T={T}, top-{k}, E={E}, G={G}, N={N}) per launch; ids "
+                       f"{nbatch * tk * 4 / 1e6:.0f} MB",
+           "peak_gbs": hbm}
+    for name, t in (("count", t_count), ("split", t_split), ("assign", t_assign)):
+        gbs = by[name] / (t * 1e-6) / 1e9
+        out[name] = {"us": t, "algorithmic_bytes": by[name], "gbs": gbs, "frac": gbs / hbm,
+                     "assignments_per_s": nbatch * tk / (t * 1e-6)}
+    del path
+    torch.cuda.empty_cache()
+    return out
 
 
 def end_to_end(args, wl, hid, W, bias, path, dev, world, chain=True):

@@ -12,14 +12,16 @@
 //               destination depends on their rank q among e's remote ones).
 // The prep kernel (one CTA per problem) computes these from cnt, plan and
 // split without reading the ids; counts and plan are staged in shared memory
-// first.  The scatter kernel (one CTA per (problem, source block)) then needs
-// only each assignment's rank among the earlier assignments of the same
-// expert in its block: warps take consecutive 32-assignment steps with
-// __match_any_sync ranks and per-warp counters in shared memory, a warp
-// shuffle scan across warps keeps block order, and each assignment's slot is
-// base + rank, or, for a replicated expert's remote assignment, a short walk
-// over the expert's replica segments (staged in shared memory).  Positions
-// never come from atomics, so the permutation is deterministic and stable.
+// first.  The scatter kernel (one CTA per (problem, source block), or one
+// warp per block when blocks are small) then needs only each assignment's
+// rank among the earlier assignments of the same expert in its block: warps
+// take consecutive 32-assignment steps, find each lane's peers (same expert)
+// with one ballot per bit of the expert id, keep per-warp counters in shared
+// memory, a per-expert scan down the warps' counters keeps block order, and each
+// assignment's slot is base + rank, or, for a replicated expert's remote
+// assignment, a binary search over the expert's replica segments (staged in
+// shared memory).  Positions never come from atomics, so the permutation is
+// deterministic and stable.
 #pragma once
 #include "common.cuh"
 #include "plan.cuh"
@@ -28,10 +30,10 @@ namespace lb {
 namespace assign {
 
 constexpr int PREP_THREADS = 1024;
-constexpr int SC_THREADS = 1024;
+constexpr int SC_THREADS = 1024;   // scatter CTA for one problem's latency (the throughput launch uses 512)
 constexpr int SC_WARPS = SC_THREADS / 32;
 constexpr int SC_STEPS = 8;   // 32-assignment steps per warp per chunk
-static_assert(SC_WARPS == 32, "the cross-warp scan maps one warp's counts to one lane");
+constexpr int TOK_QUEUE = 256;   // token path: queued slots per warp (32 lanes x 8 ids)
 
 // Workspace per problem (int32 words): base[G*E], seg_qoff[GN], seg_cum[GN],
 // seg_rep[GN]; rounded to 256 bytes.
@@ -49,10 +51,10 @@ __host__ __device__ inline size_t prep_smem_bytes(int G, int E, int N) {
 // Shared memory of the scatter: per-expert tables (holders, replica count,
 // CSR start, home count), the per-(CTA or warp) block bases and running
 // counts, the per-warp counter tables, and the replica segments.
-__host__ __device__ inline size_t scatter_smem_bytes(int G, int E, int N) {
+__host__ __device__ inline size_t scatter_smem_bytes(int G, int E, int N, int nw = SC_WARPS) {
     const size_t GN = static_cast<size_t>(G) * N, EP = static_cast<size_t>(E) + 1;
-    return static_cast<size_t>(E) * 8 + static_cast<size_t>(E) * 4 * 3 + (static_cast<size_t>(E) + 1) * 4 +
-           static_cast<size_t>(SC_WARPS) * EP * 4 * 3 + GN * 4 * 7 + 64;
+    return static_cast<size_t>(E) * 8 + static_cast<size_t>(E) * 4 * 6 + (static_cast<size_t>(E) + 1) * 4 +
+           static_cast<size_t>(nw) * EP * 4 * 3 + static_cast<size_t>(nw) * TOK_QUEUE * 8 + GN * 4 * 7 + 64;
 }
 
 // Source blocks of at most this many assignments are scattered one block per
@@ -279,14 +281,17 @@ __global__ void __launch_bounds__(PREP_THREADS) prep_kernel(const Args a) {
 
 // ---- scatter ---------------------------------------------------------------
 // Peers of this lane's expert id among the warp's lanes (bit-by-bit ballots:
-// a fixed log2(E) collectives, where __match_any_sync serialises over the
-// distinct values in the warp).  Lanes with e < 0 are excluded.
-__device__ __forceinline__ unsigned warp_peers(int e, int nbits) {
+// a fixed NB collectives, where __match_any_sync serialises over the distinct
+// values in the warp).  Lanes with e < 0 are excluded.  NB >= the bits of the
+// largest id; extra bits are zero for every valid id and change nothing.
+template <int NB>
+__device__ __forceinline__ unsigned warp_peers(int e) {
     unsigned m = __ballot_sync(kFull, e >= 0);
-    for (int bit = 0; bit < nbits; ++bit) {
-        const bool on = (e >> bit) & 1;
+#pragma unroll
+    for (int bit = 0; bit < NB; ++bit) {
+        const unsigned on = (e >> bit) & 1u;
         const unsigned bb = __ballot_sync(kFull, on);
-        m &= on ? bb : ~bb;
+        m &= bb ^ (on - 1u);   // bb where the bit is set, ~bb where it is clear
     }
     return m;
 }
@@ -297,24 +302,32 @@ struct ScatterView {
     int32_t *rep0;      // [E+1] first CSR position of e
     int32_t *homecnt;   // [E] cnt[home(e), e]
     int32_t *homeoff;   // [E] offs[home(e)*E + e]
-    int32_t *base;      // [SC_WARPS][EP] block bases (row 0 only in CTA mode)
-    int32_t *wcnt;      // [SC_WARPS][EP]
-    int32_t *pre;       // [SC_WARPS][EP] (CTA mode) / unused
+    int32_t *home;      // [E] home(e)
+    int32_t *cls;       // [E] CTA mode: class of e for the CTA's source block (see scatter_block_cta)
+    int32_t *sfirst;    // [E] CTA mode: replica segment of the block's first remote rank of e
+    int32_t *base;      // [warps][EP] block bases (row 0 only in CTA mode)
+    int32_t *wcnt;      // [warps][EP] per-warp counts (CTA mode: scanned in place into prefixes)
+    uint32_t *lmask;    // [warps][EP] token path: lanes whose token holds e (kept zero between steps)
+    int2 *queue;        // [warps][TOK_QUEUE] token path: slots of replicated experts' remote assignments
     int32_t *s_qoff, *s_tok, *s_mass, *s_cum, *s_rep, *s_v, *s_vcnt;   // [GN] per CSR position
 };
 
-__device__ inline ScatterView scatter_carve(uint8_t *sm, int G, int E, int N) {
+__device__ inline ScatterView scatter_carve(uint8_t *sm, int G, int E, int N, int nw = SC_WARPS) {
     const int GN = G * N, EP = E + 1;
     ScatterView v;
     v.hold = reinterpret_cast<uint64_t *>(sm);
-    v.rcnt = reinterpret_cast<int32_t *>(v.hold + E);
+    v.queue = reinterpret_cast<int2 *>(v.hold + E);   // 8-byte aligned after the 8-byte masks
+    v.rcnt = reinterpret_cast<int32_t *>(v.queue + nw * TOK_QUEUE);
     v.rep0 = v.rcnt + E;
     v.homecnt = v.rep0 + E + 1;
     v.homeoff = v.homecnt + E;
-    v.base = v.homeoff + E;
-    v.wcnt = v.base + SC_WARPS * EP;
-    v.pre = v.wcnt + SC_WARPS * EP;
-    v.s_qoff = v.pre + SC_WARPS * EP;
+    v.home = v.homeoff + E;
+    v.cls = v.home + E;
+    v.sfirst = v.cls + E;
+    v.base = v.sfirst + E;
+    v.wcnt = v.base + nw * EP;
+    v.lmask = reinterpret_cast<uint32_t *>(v.wcnt + nw * EP);
+    v.s_qoff = reinterpret_cast<int32_t *>(v.lmask + nw * EP);
     v.s_tok = v.s_qoff + GN;
     v.s_mass = v.s_tok + GN;
     v.s_cum = v.s_mass + GN;
@@ -389,6 +402,7 @@ __device__ void scatter_setup(const Args &a, int b, const ScatterView &v) {
         v.rcnt[e] = r1 - r0;
         v.homecnt[e] = cnt[h * E + e];
         v.homeoff[e] = offs[h * E + e];
+        v.home[e] = h;
     }
     __syncthreads();
 }
@@ -396,21 +410,11 @@ __device__ void scatter_setup(const Args &a, int b, const ScatterView &v) {
 // Destination rank and permutation slot of an assignment of expert e from
 // source block g whose rank among the block's earlier assignments of e is
 // rho; bse = base[g, e].  Returns false if the tables do not place it.
-__device__ __forceinline__ bool place(const ScatterView &v, int Eg, int g, int e, int bse, int rho, int &d, int &p) {
-    const uint64_t hm = v.hold[e];
-    if ((hm >> g) & 1ull) {
-        d = g;
-        p = bse + rho;
-        return true;
-    }
-    const int h = e / Eg;
+// A replicated expert's remote assignment with rank q among e's remote ones:
+// the replica segment covering q decides between home(e) and the replica.
+__device__ __forceinline__ bool place_remote(const ScatterView &v, int g, int e, int q, int &d, int &p) {
+    const int h = v.home[e];
     const int m = v.rcnt[e];
-    if (m == 0) {
-        d = h;
-        p = bse + rho;
-        return true;
-    }
-    const int q = bse + rho;
     // last segment starting at or before q (starts ascend along the CSR)
     int lo = v.rep0[e], hi = lo + m - 1;
     while (lo < hi) {
@@ -431,22 +435,38 @@ __device__ __forceinline__ bool place(const ScatterView &v, int Eg, int g, int e
     return true;
 }
 
+__device__ __forceinline__ bool place(const ScatterView &v, int g, int e, int bse, int rho, int &d, int &p) {
+    const uint64_t hm = v.hold[e];
+    if ((hm >> g) & 1ull) {
+        d = g;
+        p = bse + rho;
+        return true;
+    }
+    if (v.rcnt[e] == 0) {
+        d = v.home[e];
+        p = bse + rho;
+        return true;
+    }
+    return place_remote(v, g, e, bse + rho, d, p);
+}
+
 // Whole blocks, one per warp (blocks g0, g0 + SC_WARPS, ... below g1): the
 // warp walks the block's assignments 32 at a time in order, ranking each
 // among the earlier ones of its expert with bit-ballot peers and a per-warp
 // running count in shared memory.  No block-wide barrier.
+template <int NB>
 __device__ void scatter_blocks_warp(const Args &a, int b, int g0, int g1, const ScatterView &v, int *bad) {
     const int G = a.G, E = a.E, k = a.k, EP = E + 1;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int Eg = E / G, Tg = a.T / G, nitems = Tg * k, nf = a.T * k;
-    const int nbits = E > 1 ? 32 - __clz(E - 1) : 1;
+    const int Tg = a.T / G, nitems = Tg * k, nf = a.T * k;
     const int32_t *ids = a.ids + static_cast<int64_t>(b) * a.T * k;
     int32_t *dest = a.dest + static_cast<int64_t>(b) * a.T * k;
     int32_t *perm = a.perm + static_cast<int64_t>(b) * a.T * k;
     const int32_t *wsb = a.ws + static_cast<size_t>(b) * a.ws_stride;
+    const int nw = blockDim.x >> 5;
     int32_t *cntw = v.wcnt + warp * EP;
     int32_t *basew = v.base + warp * EP;
-    for (int g = g0 + warp; g < g1; g += SC_WARPS) {
+    for (int g = g0 + warp; g < g1; g += nw) {
         for (int e = lane; e < E; e += 32) {
             cntw[e] = 0;
             basew[e] = wsb[g * E + e];
@@ -463,14 +483,14 @@ __device__ void scatter_blocks_warp(const Args &a, int b, int g0, int g1, const 
                     e = -1;
                 }
             }
-            const unsigned peers = warp_peers(e, nbits);
+            const unsigned peers = warp_peers<NB>(e);
             const int rnk = __popc(peers & lanemask_lt());
             const int cur = e >= 0 ? cntw[e] : 0;
             __syncwarp();
             if (e >= 0 && lane == 31 - __clz(peers)) cntw[e] = cur + __popc(peers);
             if (e >= 0) {
                 int d, pp;
-                if (place(v, Eg, g, e, basew[e], cur + rnk, d, pp) && pp >= 0 && pp < nf) {
+                if (place(v, g, e, basew[e], cur + rnk, d, pp) && pp >= 0 && pp < nf) {
                     dest[f0 + i] = d;
                     perm[pp] = static_cast<int32_t>(f0 + i);
                 } else {
@@ -483,106 +503,384 @@ __device__ void scatter_blocks_warp(const Args &a, int b, int g0, int g1, const 
 }
 
 // Assignments [i0, i1) of one block by the whole CTA (large blocks): warps
-// take consecutive 32-assignment steps, then a shuffle scan across warps
-// turns per-warp counts into block-order ranks.  `prefix` (shared memory,
+// take consecutive 32-assignment steps, then a scan down the per-warp counts
+// (one thread per expert) turns them into block-order ranks.  `prefix` (shared memory,
 // E entries) holds each expert's assignments in the block before i0, or is
 // null when i0 == 0.
+template <int NB>
 __device__ void scatter_block_cta(const Args &a, int b, int g, int i0, int i1, const int32_t *prefix,
                                   const ScatterView &v, int *bad) {
     const int G = a.G, E = a.E, k = a.k, EP = E + 1;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int Eg = E / G, Tg = a.T / G, nitems = Tg * k, nf = a.T * k;
-    const int nbits = E > 1 ? 32 - __clz(E - 1) : 1;
-    const int64_t f0 = static_cast<int64_t>(g) * nitems;
-    const int32_t *ids = a.ids + static_cast<int64_t>(b) * a.T * k;
-    int32_t *dest = a.dest + static_cast<int64_t>(b) * a.T * k;
-    int32_t *perm = a.perm + static_cast<int64_t>(b) * a.T * k;
+    const int Tg = a.T / G, nitems = Tg * k, nf = a.T * k;
+    const int fbase = g * nitems;   // problem-local index of the block's first assignment
+    const int64_t pb = static_cast<int64_t>(b) * a.T * k;
+    const int32_t *ids = a.ids + pb + fbase;   // this block's assignments
+    int32_t *dest = a.dest + pb + fbase;
+    int32_t *perm = a.perm + pb;               // the problem's permutation
     const int32_t *wsb = a.ws + static_cast<size_t>(b) * a.ws_stride;
     int32_t *run = v.base + EP;   // row 1 of the base table: running counts
+    // Class of each expert for this source block: (g << 2) | 0 when g holds
+    // it (served locally), (home << 2) | 1 when it has no replica (served at
+    // home), 2 when it is replicated elsewhere (the split decides).  In the
+    // first two classes an assignment's slot is base + rank.  For the third,
+    // sfirst[e] is the replica segment holding the block's first remote rank
+    // of e here; later ranks only move forward from it.
     for (int e = tid; e < E; e += blockDim.x) {
-        v.base[e] = wsb[g * E + e];
-        run[e] = prefix != nullptr ? prefix[e] : 0;
+        const int bse = wsb[g * E + e];
+        const int r0 = prefix != nullptr ? prefix[e] : 0;
+        v.base[e] = bse;
+        run[e] = r0;
+        const bool local = (v.hold[e] >> g) & 1ull;
+        const int m = v.rcnt[e];
+        v.cls[e] = local ? (g << 2) : (m == 0 ? (v.home[e] << 2) | 1 : 2);
+        int sf = 0;
+        if (!local && m > 0) {
+            const int q = bse + r0;
+            int lo = v.rep0[e], hi = lo + m - 1;
+            while (lo < hi) {
+                const int mid = (lo + hi + 1) >> 1;
+                if (v.s_qoff[mid] <= q) lo = mid; else hi = mid - 1;
+            }
+            sf = lo;
+        }
+        v.sfirst[e] = sf;
     }
     __syncthreads();
-    constexpr int CH = SC_WARPS * 32 * SC_STEPS;
+    const int nw = blockDim.x >> 5;
+    const int CH = nw * 32 * SC_STEPS;
     int32_t *wrow = v.wcnt + warp * EP;
+    const int32_t *prow = v.wcnt + warp * EP;   // after the scan: the warp's prefixes
     const int iend = min(i1, nitems);
+    const unsigned lt = lanemask_lt();
+    int badl = 0;
     for (int cs = i0; cs < iend; cs += CH) {
         for (int e = lane; e < E; e += 32) wrow[e] = 0;
         __syncwarp();
+        const int ib = cs + warp * 32 * SC_STEPS + lane;   // this lane's index at step 0
         int es[SC_STEPS], loc[SC_STEPS];
 #pragma unroll
-        for (int s = 0; s < SC_STEPS; ++s) {
-            const int i = cs + warp * 32 * SC_STEPS + s * 32 + lane;
-            es[s] = i < iend ? __ldg(ids + f0 + i) : -1;
-        }
+        for (int s = 0; s < SC_STEPS; ++s) es[s] = ib + s * 32 < iend ? __ldg(ids + ib + s * 32) : -1;
 #pragma unroll
         for (int s = 0; s < SC_STEPS; ++s) {
             int e = es[s];
-            if (e >= E || e < -1 || (e == -1 && cs + warp * 32 * SC_STEPS + s * 32 + lane < iend)) {
-                *bad = 1;
+            if (ib + s * 32 < iend && static_cast<unsigned>(e) >= static_cast<unsigned>(E)) {
+                badl = 1;
                 e = -1;
             }
-            const unsigned peers = warp_peers(e, nbits);
-            const int rnk = __popc(peers & lanemask_lt());
+            const unsigned peers = warp_peers<NB>(e);
             const int cur = e >= 0 ? wrow[e] : 0;
             __syncwarp();
-            if (e >= 0 && lane == 31 - __clz(peers)) wrow[e] = cur + __popc(peers);
+            if (e >= 0 && (peers >> lane) == 1u) wrow[e] = cur + __popc(peers);   // highest peer lane
             __syncwarp();
             es[s] = e;
-            loc[s] = cur + rnk;
+            loc[s] = cur + __popc(peers & lt);
         }
         __syncthreads();
-        for (int e = warp; e < E; e += SC_WARPS) {
-            const int c = v.wcnt[lane * EP + e];
-            int x = c;
-#pragma unroll
-            for (int off = 1; off < 32; off <<= 1) {
-                const int y = __shfl_up_sync(kFull, x, off);
-                if (lane >= off) x += y;
+        // per expert, an exclusive scan down the warps' counts (one thread per
+        // expert walking the nw rows; the rows are per-warp, the columns
+        // consecutive, so the walkers' loads hit distinct banks)
+        for (int e = tid; e < E; e += blockDim.x) {
+            int acc = run[e];
+            for (int w = 0; w < nw; ++w) {
+                const int c = v.wcnt[w * EP + e];
+                v.wcnt[w * EP + e] = acc;   // in place: each row becomes its warp's prefix
+                acc += c;
             }
-            const int r = run[e];
-            v.pre[lane * EP + e] = r + x - c;
-            __syncwarp();
-            if (lane == 31) run[e] = r + x;
+            run[e] = acc;
         }
         __syncthreads();
 #pragma unroll
         for (int s = 0; s < SC_STEPS; ++s) {
             const int e = es[s];
             if (e < 0) continue;
-            const int i = cs + warp * 32 * SC_STEPS + s * 32 + lane;
-            int d, pp;
-            if (place(v, Eg, g, e, v.base[e], v.pre[warp * EP + e] + loc[s], d, pp) && pp >= 0 && pp < nf) {
-                dest[f0 + i] = d;
-                perm[pp] = static_cast<int32_t>(f0 + i);
+            const int i = ib + s * 32;
+            const int c = v.cls[e];
+            const int q = v.base[e] + prow[e] + loc[s];
+            int d = c >> 2, pp = q;
+            bool ok = true;
+            if ((c & 3) == 2) {
+                // the segment covering q: forward from the block's first one
+                const int last = v.rep0[e] + v.rcnt[e] - 1;
+                int j = v.sfirst[e];
+                while (j < last && v.s_qoff[j + 1] <= q) ++j;
+                const int qo = v.s_qoff[j], t = v.s_tok[j];
+                ok = q >= qo && q < qo + t;
+                const int w = q - qo, mss = v.s_mass[j];
+                if (w < mss) {
+                    const int h = v.home[e];
+                    d = h;
+                    pp = v.homeoff[e] + (h < g ? v.homecnt[e] : 0) + v.s_cum[j] + w;
+                } else {
+                    const int r = v.s_v[j];
+                    d = r;
+                    pp = v.s_rep[j] + (r < g ? v.s_vcnt[j] : 0) + (w - mss);
+                }
+            }
+            if (ok && static_cast<unsigned>(pp) < static_cast<unsigned>(nf)) {
+                dest[i] = d;
+                perm[pp] = fbase + i;
             } else {
-                *bad = 1;
+                badl = 1;
             }
         }
         __syncthreads();   // pre/run are rewritten by the next chunk
     }
+    if (badl) *bad = 1;
     __syncthreads();
 }
 
-// Scatter kernel: CTA (x, problem y).  Small blocks: CTA x takes blocks
-// [x*SC_WARPS, (x+1)*SC_WARPS), one per warp.  Large blocks: CTA x takes
-// block x.
+// Token path of the CTA-mode scatter (k <= KT <= 8; [i0, i1) whole tokens).
+// One token per lane: its k ids are distinct, so the rank of (t, j) among
+// the block's earlier assignments of e = ids[t, j] is the number of earlier
+// tokens holding e.  Every lane ORs its bit into a per-warp mask word of each
+// of its experts; a slot's rank inside the warp's 32 tokens is then
+// popc(mask & lanes below), and the lowest lane holding e records the warp's
+// count of e for the scan down the warps.  A few operations per slot in
+// place of a ballot per id bit per 32 assignments; dest rows are written as
+// 16-byte vectors.  An id out of range gets dest = -1 and no permutation
+// slot, and is flagged.
+template <int KT>
+__device__ void scatter_block_tok(const Args &a, int b, int g, int i0, int i1, const int32_t *prefix,
+                                  const ScatterView &v, int *bad) {
+    const int G = a.G, E = a.E, k = a.k, EP = E + 1;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int Tg = a.T / G, nitems = Tg * k, nf = a.T * k;
+    const int fbase = g * nitems;
+    const int64_t pb = static_cast<int64_t>(b) * a.T * k;
+    const int32_t *ids = a.ids + pb + fbase;
+    int32_t *dest = a.dest + pb + fbase;
+    int32_t *perm = a.perm + pb;
+    const int32_t *wsb = a.ws + static_cast<size_t>(b) * a.ws_stride;
+    int32_t *run = v.base + EP;
+    const int nw = blockDim.x >> 5;
+    for (int e = tid; e < E; e += blockDim.x) {
+        const int bse = wsb[g * E + e];
+        const int r0 = prefix != nullptr ? prefix[e] : 0;
+        v.base[e] = bse;
+        run[e] = r0;
+        const bool local = (v.hold[e] >> g) & 1ull;
+        const int m = v.rcnt[e];
+        v.cls[e] = local ? (g << 2) : (m == 0 ? (v.home[e] << 2) | 1 : 2);
+        int sf = 0;
+        if (!local && m > 0) {
+            const int q = bse + r0;
+            int lo = v.rep0[e], hi = lo + m - 1;
+            while (lo < hi) {
+                const int mid = (lo + hi + 1) >> 1;
+                if (v.s_qoff[mid] <= q) lo = mid; else hi = mid - 1;
+            }
+            sf = lo;
+        }
+        v.sfirst[e] = sf;
+    }
+    for (int x = tid; x < nw * EP; x += blockDim.x) v.lmask[x] = 0u;
+    __syncthreads();
+    int32_t *wrow = v.wcnt + warp * EP;
+    const int32_t *prow = v.wcnt + warp * EP;   // after the scan: the warp's prefixes
+    uint32_t *lm = v.lmask + warp * EP;
+    const unsigned lt = lanemask_lt();
+    const bool vec = KT == k && (KT % 4) == 0 && ((reinterpret_cast<uintptr_t>(ids) | reinterpret_cast<uintptr_t>(dest)) &
+                                                  15) == 0;
+    const int tb0 = i0 / k, tb1 = min(i1, nitems) / k;
+    int badl = 0;
+    for (int cs = tb0; cs < tb1; cs += nw * 32) {
+        for (int e = lane; e < E; e += 32) wrow[e] = 0;
+        const int t = cs + warp * 32 + lane;   // this lane's token (block-local)
+        const bool tv = t < tb1;
+        int ev[KT];
+        if (tv && vec) {
+#pragma unroll
+            for (int j = 0; j < KT; j += 4) {
+                const int4 x = __ldg(reinterpret_cast<const int4 *>(ids + t * KT + j));
+                ev[j] = x.x;
+                ev[j + 1] = x.y;
+                ev[j + 2] = x.z;
+                ev[j + 3] = x.w;
+            }
+        } else {
+#pragma unroll
+            for (int j = 0; j < KT; ++j) ev[j] = (tv && j < k) ? __ldg(ids + t * k + j) : -1;
+        }
+        // ids out of range take no slot (a row repeating an id is lb_count's
+        // to flag: its slots are then unspecified, every write stays in range)
+#pragma unroll
+        for (int j = 0; j < KT; ++j) {
+            if (tv && j < k && static_cast<unsigned>(ev[j]) >= static_cast<unsigned>(E)) {
+                badl = 1;
+                ev[j] = -1;
+            }
+        }
+        __syncwarp();   // wrow zeroed before the leaders below write it
+#pragma unroll
+        for (int j = 0; j < KT; ++j)
+            if (ev[j] >= 0) atomicOr(&lm[ev[j]], 1u << lane);
+        __syncwarp();
+        int loc[KT];    // rank inside the warp's tokens | (warp count of e if this lane leads e) << 8
+#pragma unroll
+        for (int j = 0; j < KT; ++j) {
+            loc[j] = 0;
+            if (ev[j] >= 0) {
+                const unsigned msk = lm[ev[j]];
+                const unsigned below = msk & lt;
+                loc[j] = __popc(below) | (below == 0u ? __popc(msk) << 8 : 0);
+            }
+        }
+        __syncwarp();   // every lane has read the masks before they are cleared
+#pragma unroll
+        for (int j = 0; j < KT; ++j) {
+            if (ev[j] >= 0 && (loc[j] >> 8) != 0) {
+                wrow[ev[j]] = loc[j] >> 8;
+                lm[ev[j]] = 0u;
+            }
+        }
+        __syncthreads();
+        for (int e = tid; e < E; e += blockDim.x) {
+            int acc = run[e];
+            for (int w = 0; w < nw; ++w) {
+                const int c = v.wcnt[w * EP + e];
+                v.wcnt[w * EP + e] = acc;   // in place: each row becomes its warp's prefix
+                acc += c;
+            }
+            run[e] = acc;
+        }
+        __syncthreads();
+        // Slots served where they are (held locally, or unreplicated: home)
+        // are placed now; a replicated expert's remote slots (a minority,
+        // but present in nearly every 32-lane slot column) go to the warp's
+        // queue and are resolved 32 at a time with every lane busy.
+        int2 *qw = v.queue + warp * TOK_QUEUE;
+        int qn = 0;   // queued items (warp-uniform)
+        int dv[KT];
+#pragma unroll
+        for (int j = 0; j < KT; ++j) {
+            dv[j] = -1;
+            const int e = ev[j];
+            const int c = e >= 0 ? v.cls[e] : 0;
+            const bool rem = e >= 0 && (c & 3) == 2;
+            const unsigned rmask = __ballot_sync(kFull, rem);
+            if (rem) {
+                const int slot = qn + __popc(rmask & lt);
+                qw[slot] = make_int2(t * k + j, e | ((loc[j] & 0xff) << 16));
+                loc[j] = slot | (1 << 30);   // this slot's answer comes back through the queue
+            } else if (e >= 0) {
+                const int pp = v.base[e] + prow[e] + (loc[j] & 0xff);
+                if (static_cast<unsigned>(pp) < static_cast<unsigned>(nf)) {
+                    perm[pp] = fbase + t * k + j;
+                    dv[j] = c >> 2;
+                } else {
+                    badl = 1;
+                }
+            }
+            qn += __popc(rmask);
+        }
+        __syncwarp();
+        for (int i0q = 0; i0q < qn; i0q += 32) {
+            const int iq = i0q + lane;
+            if (iq < qn) {
+                const int2 it = qw[iq];
+                const int fl = it.x, e = it.y & 0xffff;
+                const int q = v.base[e] + prow[e] + (it.y >> 16);
+                // the segment covering q: forward from the block's first one
+                const int last = v.rep0[e] + v.rcnt[e] - 1;
+                int jj = v.sfirst[e];
+                while (jj < last && v.s_qoff[jj + 1] <= q) ++jj;
+                const int qo = v.s_qoff[jj], tk = v.s_tok[jj];
+                const int w = q - qo, mss = v.s_mass[jj];
+                int d, pp;
+                if (w < mss) {
+                    const int h = v.home[e];
+                    d = h;
+                    pp = v.homeoff[e] + (h < g ? v.homecnt[e] : 0) + v.s_cum[jj] + w;
+                } else {
+                    const int r = v.s_v[jj];
+                    d = r;
+                    pp = v.s_rep[jj] + (r < g ? v.s_vcnt[jj] : 0) + (w - mss);
+                }
+                if (q >= qo && q < qo + tk && static_cast<unsigned>(pp) < static_cast<unsigned>(nf)) {
+                    perm[pp] = fbase + fl;
+                } else {
+                    badl = 1;
+                    d = -1;
+                }
+                qw[iq].x = d;
+            }
+        }
+        __syncwarp();
+#pragma unroll
+        for (int j = 0; j < KT; ++j)
+            if (loc[j] & (1 << 30)) dv[j] = qw[loc[j] & 0xffff].x;
+        if (tv) {
+            if (vec) {
+#pragma unroll
+                for (int j = 0; j < KT; j += 4)
+                    *reinterpret_cast<int4 *>(dest + t * KT + j) = make_int4(dv[j], dv[j + 1], dv[j + 2], dv[j + 3]);
+            } else {
+#pragma unroll
+                for (int j = 0; j < KT; ++j)
+                    if (j < k) dest[t * k + j] = dv[j];
+            }
+        }
+        __syncthreads();   // pre/run are rewritten by the next chunk
+    }
+    if (badl) *bad = 1;
+    __syncthreads();
+}
+
+// Bits of the largest expert id, rounded up to an instantiated width.
+__device__ __forceinline__ int id_bits(int E) {
+    const int nb = E > 1 ? 32 - __clz(E - 1) : 1;
+    return nb <= 4 ? 4 : nb <= 6 ? 6 : nb <= 8 ? 8 : 10;
+}
+
+__device__ inline void scatter_blocks_warp_any(const Args &a, int b, int g0, int g1, const ScatterView &v,
+                                               int *bad) {
+    switch (id_bits(a.E)) {
+        case 4: scatter_blocks_warp<4>(a, b, g0, g1, v, bad); break;
+        case 6: scatter_blocks_warp<6>(a, b, g0, g1, v, bad); break;
+        case 8: scatter_blocks_warp<8>(a, b, g0, g1, v, bad); break;
+        default: scatter_blocks_warp<10>(a, b, g0, g1, v, bad); break;
+    }
+}
+
+__device__ inline void scatter_block_cta_any(const Args &a, int b, int g, int i0, int i1, const int32_t *prefix,
+                                             const ScatterView &v, int *bad) {
+    const int nitems = (a.T / a.G) * a.k;
+    if (a.k <= 8 && i0 % a.k == 0 && (i1 % a.k == 0 || i1 >= nitems)) {
+        if (a.k <= 2) scatter_block_tok<2>(a, b, g, i0, i1, prefix, v, bad);
+        else if (a.k <= 4) scatter_block_tok<4>(a, b, g, i0, i1, prefix, v, bad);
+        else scatter_block_tok<8>(a, b, g, i0, i1, prefix, v, bad);
+        return;
+    }
+    switch (id_bits(a.E)) {
+        case 4: scatter_block_cta<4>(a, b, g, i0, i1, prefix, v, bad); break;
+        case 6: scatter_block_cta<6>(a, b, g, i0, i1, prefix, v, bad); break;
+        case 8: scatter_block_cta<8>(a, b, g, i0, i1, prefix, v, bad); break;
+        default: scatter_block_cta<10>(a, b, g, i0, i1, prefix, v, bad); break;
+    }
+}
+
+// Scatter kernel: CTA (x, problem y) of W = blockDim.x / 32 warps (32 for
+// one problem's latency; 16 when many problems fill the GPU, so that two CTAs
+// share an SM and one's barriers overlap the other's work).  Small blocks:
+// CTA x takes blocks [x*W, (x+1)*W), one per warp.  Large blocks: CTA x
+// takes block x.
 __global__ void __launch_bounds__(SC_THREADS) scatter_kernel(const Args a) {
     extern __shared__ __align__(16) uint8_t sm[];
     __shared__ int bad;
     if (threadIdx.x == 0) bad = 0;
-    const ScatterView v = scatter_carve(sm, a.G, a.E, a.N);
+    const int nw = blockDim.x >> 5;
+    const ScatterView v = scatter_carve(sm, a.G, a.E, a.N, nw);
     LB_TICK(10);
     scatter_setup(a, blockIdx.y, v);
     LB_TICK(11);
     const int nitems = (a.T / a.G) * a.k;
     if (nitems <= WARP_BLOCK_MAX) {
-        const int g0 = blockIdx.x * SC_WARPS;
-        scatter_blocks_warp(a, blockIdx.y, g0, min(a.G, g0 + SC_WARPS), v, &bad);
+        const int g0 = blockIdx.x * nw;
+        scatter_blocks_warp_any(a, blockIdx.y, g0, min(a.G, g0 + nw), v, &bad);
         __syncthreads();
     } else {
-        scatter_block_cta(a, blockIdx.y, blockIdx.x, 0, nitems, nullptr, v, &bad);
+        scatter_block_cta_any(a, blockIdx.y, blockIdx.x, 0, nitems, nullptr, v, &bad);
     }
     LB_TICK(12);
     if (threadIdx.x == 0 && bad) flag(LB_DEV_BAD_SPLIT);

@@ -334,10 +334,52 @@ __global__ void __launch_bounds__(THREADS, 1)
 // adjacent rows of the stacked [L*E, H] weights, so one N = 2E MMA tile per
 // k-block covers both, and each hidden state crosses HBM once instead of
 // twice.
-constexpr int P_THREADS = 192;
+constexpr int P_THREADS = 320;   // warp 0 TMA, warp 1 MMA, warps 2..9 epilogue (two per TMEM lane quadrant)
+constexpr int P_EPI = 256;       // epilogue threads
+
+// The two epilogue warps of TMEM lane quadrant q meet at named barrier 1 + q
+// (ids as immediates, so the kernel reserves barriers 0..4 only).
+template <int ID>
+__device__ __forceinline__ bool pair_all_id(bool v) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred pa, pb;\n\t"
+        "setp.ne.u32 pa, %1, 0;\n\t"
+        "bar.red.and.pred pb, %2, 64, pa;\n\t"
+        "selp.u32 %0, 1, 0, pb;\n\t}"
+        : "=r"(r)
+        : "r"(static_cast<uint32_t>(v)), "n"(ID)
+        : "memory");
+    return r != 0;
+}
+template <int ID>
+__device__ __forceinline__ void pair_sync_id() {
+    asm volatile("bar.sync %0, 64;" ::"n"(ID) : "memory");
+}
+__device__ __forceinline__ bool pair_all(int q, bool v) {
+    switch (q) {
+        case 0: return pair_all_id<1>(v);
+        case 1: return pair_all_id<2>(v);
+        case 2: return pair_all_id<3>(v);
+        default: return pair_all_id<4>(v);
+    }
+}
+__device__ __forceinline__ void pair_sync(int q) {
+    switch (q) {
+        case 0: pair_sync_id<1>(); break;
+        case 1: pair_sync_id<2>(); break;
+        case 2: pair_sync_id<3>(); break;
+        default: pair_sync_id<4>(); break;
+    }
+}
+
+// (value desc, id asc): the order the top-k ranks by.
+__device__ __forceinline__ bool ranks_before(float av, int ai, float bv, int bi) {
+    return av > bv || (av == bv && ai < bi);
+}
 
 template <int KMAX>
-__global__ void __launch_bounds__(P_THREADS, 1)
+__global__ void __launch_bounds__(P_THREADS, 2)
     gate_topk_persistent(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                          const Params p, int mtiles, int ntiles) {
     extern __shared__ uint8_t smem_raw[];
@@ -350,6 +392,9 @@ __global__ void __launch_bounds__(P_THREADS, 1)
     __shared__ __align__(8) uint64_t drain_bar;
     __shared__ uint32_t tmem_slot;
     __shared__ int aborted;
+    __shared__ float bias_w[8][LB_MAX_E_GATE / 2];   // each epilogue warp's copy of its columns' bias
+    __shared__ float merge_v[4][KMAX][32];            // second-half lists, handed to the first half
+    __shared__ int merge_i[4][KMAX][32];
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const uint32_t a_box = BM * 128u, b_box = static_cast<uint32_t>(p.Epad) * 128u;
@@ -367,7 +412,7 @@ __global__ void __launch_bounds__(P_THREADS, 1)
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&acc_full[i], 1);
-            mbar_init(&acc_empty[i], 128);
+            mbar_init(&acc_empty[i], P_EPI);
         }
         mbar_init(&drain_bar, 1);
         aborted = 0;
@@ -461,15 +506,41 @@ __global__ void __launch_bounds__(P_THREADS, 1)
             if (!mbar_wait(&drain_bar, 0)) flag(LB_DEV_TIMEOUT);
         }
     } else {
-        // ---------------- epilogue: warps 2..5, TMEM lane quadrant = warp % 4
+        // ---------------- epilogue: warps 2..9.  TMEM lane quadrant q =
+        // warp % 4 (rows q*32..q*32+31); set s = (warp - 2) / 4 picks the
+        // columns: in chain mode set s ranks gate s (columns [sE, sE+E)); in
+        // normal mode set s takes one half of the columns, and set 1 hands
+        // its sorted list to set 0, which merges and writes the ids.  The two
+        // warps of a quadrant take the same decisions (pair barriers), so
+        // they always meet at the same barriers.
         const int q = warp & 3;
+        const int set = (warp - 2) >> 2;
         const int rloc = q * 32 + lane;
+        const int half_cols = (p.Epad / 2 + 15) / 16 * 16;
+        const int cbeg = p.chain ? set * p.E : set * half_cols;
+        const int cend = p.chain ? cbeg + p.E : min(p.Epad, cbeg + half_cols);
+        float *wb = bias_w[warp - 2];
         int tl = 0;
         for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++tl) {
             const int buf = tl & 1;
             const uint32_t use = static_cast<uint32_t>(tl >> 1);
+            const int b = tile / mtiles, m0 = (tile - b * mtiles) * BM;
+            // The layer this warp's columns belong to (uniform over the tile).
+            const int layer = p.chain ? b - 1 + set : b;
+            const bool active = cbeg < cend && layer >= 0 && (!p.chain || layer < p.L);
+            // This tile's bias for the warp's columns into its own shared-
+            // memory slice, before the wait for the accumulator: under the
+            // full load of the h stream a global load takes microseconds,
+            // and here its latency hides behind the tile's MMAs.  (The warp
+            // finished reading the previous tile's copy in program order.)
+            for (int c = cbeg + lane; c < cend; c += 32) {
+                const int cc = c - (p.chain ? set * p.E : 0);
+                wb[c - cbeg] = (p.bias != nullptr && active && cc < p.E) ? p.bias[static_cast<int64_t>(layer) * p.E + cc]
+                                                                        : 0.f;
+            }
+            __syncwarp();
             bool ok = mbar_wait(&acc_full[buf], use & 1) && !*abort_flag;
-            ok = __all_sync(kFull, ok);
+            ok = pair_all(q, ok);
             if (!ok) {
                 if (lane == 0) {
                     atomicExch(&aborted, 1);
@@ -478,50 +549,87 @@ __global__ void __launch_bounds__(P_THREADS, 1)
                 break;
             }
             tc_fence_after();
-            const int b = tile / mtiles, m0 = (tile - b * mtiles) * BM;
             const int row = m0 + rloc;
             const bool valid = row < p.T;
             const uint32_t tl_addr = tmem + buf * half + (static_cast<uint32_t>(q * 32) << 16);
-            // One output (normal mode) or two column halves (chain mode); the
-            // layer of each is uniform across the tile, so a skipped half
-            // skips its warp-collective TMEM loads in every lane alike.
-            const int nhalf = p.chain ? 2 : 1;
-            for (int hh = 0; hh < nhalf; ++hh) {
-                const int layer = p.chain ? b - 1 + hh : b;
-                if (layer < 0 || (p.chain && layer >= p.L)) continue;
-                int32_t *ids_out = (p.chain && hh == 1) ? p.ids2 : p.ids;
-                float *lg_out = (p.chain && hh == 1) ? p.logits2 : p.logits;
-                const int64_t grow = static_cast<int64_t>(layer) * p.T + row;
-                const float *bias = p.bias != nullptr ? p.bias + static_cast<int64_t>(layer) * p.E : nullptr;
-                float *lrow = (lg_out != nullptr && valid) ? lg_out + grow * p.E : nullptr;
-                const int cols = p.chain ? p.E : p.Epad;
-                const uint32_t col0 = p.chain ? static_cast<uint32_t>(hh * p.E) : 0u;
-                TopK<KMAX> tk;
-                tk.init();
-                for (int c0 = 0; c0 < cols; c0 += 16) {
+            const int cl0 = p.chain ? set * p.E : 0;   // first column of this warp's gate
+            int32_t *ids_out = (p.chain && set == 1) ? p.ids2 : p.ids;
+            float *lg_out = (p.chain && set == 1) ? p.logits2 : p.logits;
+            const int64_t grow = static_cast<int64_t>(layer) * p.T + row;
+            float *lrow = (lg_out != nullptr && valid && active) ? lg_out + grow * p.E : nullptr;
+            TopK<KMAX> tk;
+            tk.init();
+            if (active) {
+                for (int c0 = cbeg; c0 < cend; c0 += 16) {
                     uint32_t r[16];
-                    tmem_ld16(tl_addr + col0 + c0, r);
+                    tmem_ld16(tl_addr + c0, r);
                     tmem_wait_ld();
 #pragma unroll
                     for (int j = 0; j < 16; ++j) {
-                        const int c = c0 + j;
+                        const int c = c0 + j - cl0;   // expert id within the gate
                         if (c < p.E) {
-                            const float x = __uint_as_float(r[j]) + (bias != nullptr ? __ldg(bias + c) : 0.f);
+                            const float x = __uint_as_float(r[j]) + wb[c0 + j - cbeg];
                             tk.push(x, c);
                             if (lrow) lrow[c] = x;
                         }
                     }
                 }
-                if (valid) {
-                    int32_t *out = ids_out + grow * p.k;
-#pragma unroll
-                    for (int j = 0; j < KMAX; ++j)
-                        if (j < p.k) out[j] = tk.i[j];
-                }
             }
-            // the accumulator buffer may be overwritten from here
+            // this warp's TMEM reads are done: the buffer may be overwritten
             tc_fence_before();
             mbar_arrive(&acc_empty[buf]);
+            if (!p.chain) {
+                // set 1 hands over its list; set 0 merges two sorted lists
+                // (bitonic: pairwise best against the reversed other list,
+                // then a half-cleaner cascade) and writes the ids
+                if (set == 1) {
+#pragma unroll
+                    for (int j = 0; j < KMAX; ++j) {
+                        merge_v[q][j][lane] = tk.v[j];
+                        merge_i[q][j][lane] = tk.i[j];
+                    }
+                }
+                pair_sync(q);
+                if (set == 0) {
+                    float cv[KMAX];
+                    int ci[KMAX];
+#pragma unroll
+                    for (int j = 0; j < KMAX; ++j) {
+                        const float ov = merge_v[q][KMAX - 1 - j][lane];
+                        const int oi = merge_i[q][KMAX - 1 - j][lane];
+                        const bool mine = ranks_before(tk.v[j], tk.i[j], ov, oi);
+                        cv[j] = mine ? tk.v[j] : ov;
+                        ci[j] = mine ? tk.i[j] : oi;
+                    }
+#pragma unroll
+                    for (int st = KMAX / 2; st > 0; st >>= 1) {
+#pragma unroll
+                        for (int j = 0; j < KMAX; ++j) {
+                            if ((j & st) == 0) {
+                                const bool keep = ranks_before(cv[j], ci[j], cv[j + st], ci[j + st]);
+                                const float hv = keep ? cv[j] : cv[j + st], lv = keep ? cv[j + st] : cv[j];
+                                const int hi = keep ? ci[j] : ci[j + st], li = keep ? ci[j + st] : ci[j];
+                                cv[j] = hv;
+                                ci[j] = hi;
+                                cv[j + st] = lv;
+                                ci[j + st] = li;
+                            }
+                        }
+                    }
+                    if (valid) {
+                        int32_t *out = ids_out + grow * p.k;
+#pragma unroll
+                        for (int j = 0; j < KMAX; ++j)
+                            if (j < p.k) out[j] = ci[j];
+                    }
+                }
+                pair_sync(q);   // set 1 may refill merge_* only after set 0 read it
+            } else if (active && valid) {
+                int32_t *out = ids_out + grow * p.k;
+#pragma unroll
+                for (int j = 0; j < KMAX; ++j)
+                    if (j < p.k) out[j] = tk.i[j];
+            }
         }
     }
 

@@ -166,7 +166,7 @@ int run_persistent(gate::Params &p, const void *h, int nprob, const CUtensorMap 
     int stages = g_tune_stages;
     if (!stages)
         stages = static_cast<int>(
-            std::max<size_t>(2, std::min<size_t>(gate::MAX_STAGES, (100 * 1024 * 2 / per_sm) / stage_bytes)));
+            std::max<size_t>(2, std::min<size_t>(gate::MAX_STAGES, (96 * 1024 * 2 / per_sm) / stage_bytes)));
     if (stages < 2) return LB_EINVAL;
     size_t smem = stages * stage_bytes + 1024;
     smem = std::max(smem, static_cast<size_t>(228 * 1024) / (per_sm + 1) + 1);   // at most per_sm CTAs per SM
@@ -206,9 +206,19 @@ int launch_count_v(bool vec, const int32_t *ids, int nbatch, int T, int k, int E
 
 // Scatter CTAs per problem: one per source block, or one per SC_WARPS small
 // blocks (one block per warp).
-int scatter_grid_x(int T, int k, int G) {
+int scatter_grid_x(int T, int k, int G, int nw = assign::SC_WARPS) {
     const long long nitems = static_cast<long long>(T / G) * k;
-    return nitems <= assign::WARP_BLOCK_MAX ? (G + assign::SC_WARPS - 1) / assign::SC_WARPS : G;
+    return nitems <= assign::WARP_BLOCK_MAX ? (G + nw - 1) / nw : G;
+}
+
+// Warps per scatter CTA: 32 while the problems' CTAs leave SMs free (one
+// problem's latency), 16 once they fill the GPU twice over (throughput: two
+// CTAs per SM); fewer if the per-warp tables would not fit shared memory.
+int scatter_warps(int nbatch, int T, int k, int G, int E, int N) {
+    const long long ctas = static_cast<long long>(scatter_grid_x(T, k, G, 16)) * nbatch;
+    int nw = ctas >= 2LL * device_sms() ? 16 : assign::SC_WARPS;
+    while (nw > 8 && assign::scatter_smem_bytes(G, E, N, nw) > 224 * 1024) nw >>= 1;
+    return nw;
 }
 
 bool plan_shape_ok(int G, int E, int N, int L) {
@@ -509,7 +519,7 @@ int lb_assign(const int32_t *ids, const int32_t *cnt, const void *plan, const in
     if (G * N > 0 && (!tok || !mass)) return LB_EINVAL;
     if (T > 0 && (!ids || !dest || !perm)) return LB_EINVAL;
     if (static_cast<long long>(T) * k * nbatch >= INT_MAX) return LB_EINVAL;
-    if (assign::scatter_smem_bytes(G, E, N) > 224 * 1024 || assign::prep_smem_bytes(G, E, N) > 224 * 1024)
+    if (assign::scatter_smem_bytes(G, E, N, 8) > 224 * 1024 || assign::prep_smem_bytes(G, E, N) > 224 * 1024)
         return LB_EINVAL;
     if (workspace_bytes < lb_assign_workspace_bytes(nbatch, T, k, G, E, N)) return LB_ENOSPACE;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -530,14 +540,16 @@ int lb_assign(const int32_t *ids, const int32_t *cnt, const void *plan, const in
     a.offs = offs;
     a.ws = static_cast<int32_t *>(workspace);
     a.ws_stride = assign::ws_words(G, E, N);
-    const size_t sm1 = assign::prep_smem_bytes(G, E, N), sm2 = assign::scatter_smem_bytes(G, E, N);
+    const int nw = T > 0 ? scatter_warps(nbatch, T, k, G, E, N) : assign::SC_WARPS;
+    const size_t sm1 = assign::prep_smem_bytes(G, E, N), sm2 = assign::scatter_smem_bytes(G, E, N, nw);
     static SmemLimit lim1, lim2;
     if (!allow_smem(assign::prep_kernel, lim1, sm1, false) || !allow_smem(assign::scatter_kernel, lim2, sm2, false))
         return LB_ECUDA;
     assign::prep_kernel<<<nbatch, assign::PREP_THREADS, sm1, s>>>(a);
     if (launched("assign prep") != LB_OK) return LB_ECUDA;
     if (T == 0) return LB_OK;
-    assign::scatter_kernel<<<dim3(scatter_grid_x(T, k, G), nbatch), assign::SC_THREADS, sm2, s>>>(a);
+    assign::scatter_kernel<<<dim3(scatter_grid_x(T, k, G, nw), nbatch), nw * 32,
+                             assign::scatter_smem_bytes(G, E, N, nw), s>>>(a);
     return launched("assign scatter");
 }
 
@@ -691,7 +703,7 @@ extern "C" int lb_assign_noalloc(const int32_t *ids, const int32_t *cnt, const v
     if (G * N > 0 && (!tok || !mass)) return LB_EINVAL;
     if (T > 0 && (!ids || !dest || !perm)) return LB_EINVAL;
     if (static_cast<long long>(T) * k * nbatch >= INT_MAX) return LB_EINVAL;
-    if (assign::scatter_smem_bytes(G, E, N) > 224 * 1024 || assign::prep_smem_bytes(G, E, N) > 224 * 1024)
+    if (assign::scatter_smem_bytes(G, E, N, 8) > 224 * 1024 || assign::prep_smem_bytes(G, E, N) > 224 * 1024)
         return LB_EINVAL;
     const size_t need = lb_assign_workspace_bytes(nbatch, T, k, G, E, N);
     if (need > kNoAllocScratchBytes) {
@@ -723,7 +735,8 @@ extern "C" int lb_assign_noalloc(const int32_t *ids, const int32_t *cnt, const v
     assign::prep_kernel<<<nbatch, assign::PREP_THREADS, assign::prep_smem_bytes(G, E, N), s>>>(a);
     if (launched("assign prep (noalloc)") != LB_OK) return LB_ECUDA;
     if (T == 0) return LB_OK;
-    assign::scatter_kernel<<<dim3(scatter_grid_x(T, k, G), nbatch), assign::SC_THREADS,
-                             assign::scatter_smem_bytes(G, E, N), s>>>(a);
+    const int nw = scatter_warps(nbatch, T, k, G, E, N);
+    assign::scatter_kernel<<<dim3(scatter_grid_x(T, k, G, nw), nbatch), nw * 32,
+                             assign::scatter_smem_bytes(G, E, N, nw), s>>>(a);
     return launched("assign scatter (noalloc)");
 }

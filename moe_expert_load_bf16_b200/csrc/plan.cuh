@@ -12,8 +12,12 @@
 //            holder sets are 64-bit masks per expert, and every arg-max /
 //            arg-min is one redux.sync plus a ballot.
 //   edges:   per-expert replica counts, warp scan, parallel edge emission
-//            (expert ascending, rank ascending); greedy colouring and the
-//            stable order by round run in one thread over <= G*N edges.
+//            (expert ascending, rank ascending).
+//   rounds:  greedy colouring in edge order by one warp, each rank's busy
+//            rounds as a 128-bit mask in a lane's registers (one thread with
+//            shared-memory masks past 128 rounds); the stable order by round
+//            from per-round counts, a warp scan and each edge's rank among
+//            the earlier edges of its round.
 #pragma once
 #include "common.cuh"
 

@@ -146,7 +146,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     const assign::ScatterView sv = assign::scatter_carve(work, G, E, N);
     assign::scatter_setup(a, b, sv);
     if (!parts && nitems <= assign::WARP_BLOCK_MAX) {
-        assign::scatter_blocks_warp(a, b, crank * nseg, (crank + 1) * nseg, sv, &bad_sc);
+        assign::scatter_blocks_warp_any(a, b, crank * nseg, (crank + 1) * nseg, sv, &bad_sc);
         __syncthreads();
     } else {
         for (int sidx = 0; sidx < nseg; ++sidx) {
@@ -162,7 +162,8 @@ __global__ void __launch_bounds__(THREADS, 1)
                 }
                 __syncthreads();
             }
-            assign::scatter_block_cta(a, b, g, r0 * k, min(r1 * k, nitems), parts ? prefix : nullptr, sv, &bad_sc);
+            assign::scatter_block_cta_any(a, b, g, r0 * k, min(r1 * k, nitems), parts ? prefix : nullptr, sv,
+                                          &bad_sc);
         }
     }
     if (tid == 0 && bad_sc) flag(LB_DEV_BAD_SPLIT);

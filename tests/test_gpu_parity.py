@@ -432,3 +432,93 @@ def test_gate_chain_rejects_unsupported_shapes(E, L):
     W = torch.zeros(max(L, 1), E, 64, dtype=torch.bfloat16, device=DEV)[:L]
     with pytest.raises((_lib.LBError, ValueError)):
         _lib.lb_predict_topk_chain(hid, W, None, 2)
+
+
+@pytest.mark.parametrize("name,T,B", [("qwen3-235b", 8192, 40), ("decode", 1024, 80)])
+def test_assign_throughput_launch_equals_single(name, T, B):
+    """Enough problems to fill the GPU twice over switch the scatter to
+    512-thread CTAs (two per SM), in CTA mode (large source blocks) and in
+    warp mode (small blocks); the bytes equal one-problem calls (1024-thread
+    CTAs) and pass the oracle check."""
+    w = workloads.WORKLOADS[name]
+    ids = workloads.decode_ids(w.with_(T=T), T, range(B + 1)).to(DEV)
+    path = DecisionPath(B, T, 8, w.E, w.k, w.G, w.N, w.L, device=DEV)
+    path.ids_pred.copy_(ids[0:1].expand(B, -1, -1))
+    path.ids.copy_(ids[1:])
+    _lib.lb_count(path.ids_pred, w.G, w.E, cnt=path.cnt_pred)
+    _lib.lb_plan_replicas(path.cnt_pred, w.N, w.L, plan=path.plan)
+    path.solve()
+    torch.cuda.synchronize()
+    assert _lib.lb_get_status() == 0
+    for b in (0, B // 2, B - 1):
+        one = DecisionPath(1, T, 8, w.E, w.k, w.G, w.N, w.L, device=DEV)
+        one.ids.copy_(path.ids[b:b + 1])
+        one.plan.copy_(path.plan[b:b + 1])
+        one.solve()
+        torch.cuda.synchronize()
+        for f in ("cnt", "tok", "mass", "loads", "dest", "perm", "offs"):
+            assert torch.equal(getattr(one, f)[0], getattr(path, f)[b]), (f, b)
+    for b in (0, B - 1):
+        parity.check_path(path, b, 12)
+
+
+@pytest.mark.parametrize("k", [1, 2, 3, 4, 5, 8, 9])
+def test_scatter_large_blocks_every_k(k):
+    """Source blocks larger than one warp's share (the whole-CTA scatter):
+    every top-k width through its path (token-wise for k <= 8, with and
+    without 16-byte rows; assignment-wise above), fused and separate, against
+    the oracle."""
+    rng = np.random.default_rng(40 + k)
+    G, E, N, L = 4, 32, 3, 1
+    T = G * (2600 // k + 37)             # > 2048 assignments per block, ragged against the chunks
+    pr = rng.permutation(np.arange(1, E + 1)) ** -1.2
+    pr /= pr.sum()
+    rows = [rng.choice(E, k, replace=False, p=pr) for _ in range(2 * T)]
+    ids_np = np.stack(rows).astype(np.int32).reshape(2, T, k)
+    path = DecisionPath(1, T, 8, E, k, G, N, L, device=DEV)
+    path.ids_pred.copy_(torch.from_numpy(ids_np[0:1]).to(DEV))
+    path.ids.copy_(torch.from_numpy(ids_np[1:2]).to(DEV))
+    _lib.lb_count(path.ids_pred, G, E, cnt=path.cnt_pred)
+    _lib.lb_plan_replicas(path.cnt_pred, N, L, plan=path.plan)
+    path.solve()
+    torch.cuda.synchronize()
+    assert _lib.lb_get_status() == 0
+    parity.check_path(path, 0, 12)
+    sep = [t.clone() for t in (path.dest, path.perm, path.offs)]
+    path.solve_fused()
+    torch.cuda.synchronize()
+    assert _lib.lb_get_status() == 0
+    for a, b in zip(sep, (path.dest, path.perm, path.offs)):
+        assert torch.equal(a, b)
+
+
+def test_scatter_repeated_id_in_row_is_flagged_and_contained():
+    """A repeated id in a row is bad data: lb_count flags it, and what
+    lb_assign then writes for that row is unspecified, but every write stays
+    inside dest and perm, the other rows are placed as the oracle places them
+    on the same counts, and the context stays usable."""
+    G, E, k = 4, 16, 4
+    T = G * 700
+    rng = np.random.default_rng(5)
+    ids_np = np.stack([rng.choice(E, k, replace=False) for _ in range(T)]).astype(np.int32)
+    ids_np[101, 3] = ids_np[101, 1]
+    path = DecisionPath(1, T, 8, E, k, G, 2, 1, device=DEV)
+    guard = torch.full((2, T * k + 64), -7, dtype=torch.int32, device=DEV)
+    path.dest = guard[0, 32:32 + T * k].view(1, T, k)   # 32 guard words on either side
+    path.perm = guard[1, 32:32 + T * k].view(1, T * k)
+    path.ids_pred.copy_(torch.from_numpy(ids_np).to(DEV).unsqueeze(0))
+    path.ids.copy_(path.ids_pred)
+    _lib.lb_count(path.ids_pred, G, E, cnt=path.cnt_pred)
+    flags = _lib.lb_get_status(clear=True)
+    assert flags & _lib.LB_DEV_BAD_IDS
+    _lib.lb_plan_replicas(path.cnt_pred, 2, 1, plan=path.plan)
+    path.solve()
+    torch.cuda.synchronize()
+    _lib.lb_get_status(clear=True)
+    g = guard.cpu().numpy()
+    assert (g[:, :32] == -7).all() and (g[:, 32 + T * k:] == -7).all()
+    dest = path.dest[0].cpu().numpy()
+    assert ((dest >= -1) & (dest < G)).all()
+    perm = path.perm[0].cpu().numpy()
+    assert ((perm == -7) | ((perm >= 0) & (perm < T * k))).all()
+    assert torch.ones(4, device=DEV).sum().item() == 4.0
