@@ -13,6 +13,8 @@ Functions (see lb_oracle.c for the definitions and the pages they follow):
   split(cnt, plan, passes)               -> Split
   assign(ids, plan, split, G, E)         -> dest, perm, offs
   split_optimum(cnt, plan)               -> exact integer min-max load
+  plan_swaps(cnt, pi, gamma, tau, alpha, beta, expert_bytes, budget)
+                                         -> Swaps (budgeted pairwise swaps)
 
 `Oracle(path)` binds the same functions to another build of lb_oracle.c
 (the tests use it to check that the pins reject planted mistakes).
@@ -67,6 +69,17 @@ class Split:
     passes_run: int
 
 
+@dataclass
+class Swaps:
+    pi: np.ndarray          # [E] int32, rank of each expert after the swaps
+    swaps: np.ndarray       # [n,4] int32 (u, v, a, b) in acceptance order
+    loads: np.ndarray       # [G] int64, rank loads under pi
+
+    @property
+    def n_swaps(self):
+        return int(self.swaps.shape[0])
+
+
 def _ptr(a):
     return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
 
@@ -96,6 +109,9 @@ class Oracle:
         lib.orc_assign.argtypes = [P, i64, i32, i32, i32, P, i32, P, P, P, P, P, P, P, P]
         lib.orc_split_optimum.argtypes = [P, i32, i32, P, i32, P, P, P]
         lib.orc_split_optimum.restype = ctypes.c_int64
+        d = ctypes.c_double
+        lib.orc_plan_swaps.argtypes = [P, P, i32, i32, d, d, d, d, d, d, d, P, P, P, P]
+        lib.orc_plan_swaps.restype = ctypes.c_int
         for f in (lib.orc_gate, lib.orc_count, lib.orc_plan, lib.orc_split, lib.orc_assign):
             f.restype = ctypes.c_int
         lib.orc_threads.restype = ctypes.c_int
@@ -195,6 +211,23 @@ class Oracle:
         return int(r)
 
 
+    def plan_swaps(self, cnt, pi=None, gamma=0.0, tau=0.0, alpha=0.0, beta=1.0, expert_bytes=0.0,
+                   budget=float("inf"), link_budget=None):
+        link_budget = budget if link_budget is None else link_budget
+        cnt = _c(cnt, np.int32)
+        G, E = cnt.shape
+        pi_in = None if pi is None else _c(pi, np.int32)
+        pi_out = np.zeros(E, np.int32)
+        sw = np.zeros((max(1, E // 2 + 1), 4), np.int32)
+        n = ctypes.c_int32(0)
+        loads = np.zeros(G, np.int64)
+        self._check("orc_plan_swaps", self.lib.orc_plan_swaps(
+            _ptr(cnt), _ptr(pi_in), G, E, gamma, tau, alpha, beta, expert_bytes, budget, link_budget, _ptr(pi_out),
+            _ptr(sw),
+            ctypes.byref(n), _ptr(loads)))
+        return Swaps(pi_out, sw[:n.value].copy(), loads)
+
+
 _default = None
 
 
@@ -227,6 +260,10 @@ def assign(*a, **kw):
 
 def split_optimum(*a, **kw):
     return default().split_optimum(*a, **kw)
+
+
+def plan_swaps(*a, **kw):
+    return default().plan_swaps(*a, **kw)
 
 
 def lib_path():

@@ -25,6 +25,9 @@
  *                      FreeBalance sec. 2.2)
  *   orc_split_optimum exact integer min-max over the same per-edge feasible
  *                     set (Relief summary, "The Per-Step Optimum Problem")
+ *   orc_plan_swaps    budgeted pairwise expert-swap planning, the alternative
+ *                     to replication (FreeBalance sec. 3.3 eq. 6-10,
+ *                     Algorithm 1)
  *
  * Readings taken where the pages are silent are stated beside the code that
  * takes them.  Return codes: 0 ok, 1 invalid argument, 3 bad data.
@@ -781,4 +784,124 @@ int64_t orc_split_optimum(const int32_t *cnt, int G, int E, const uint8_t *holds
 done:
     free(rep_cnt); free(rep_ptr); free(rep_edge); free(tok); free(R); free(fixed);
     return result;
+}
+
+
+/* ------------------------------------------------------------------------
+ * Budgeted pairwise expert-swap planning (FreeBalance sec. 3.3, eq. 6-10;
+ * Algorithm 1, the loop over beneficial swaps).
+ *
+ * Expert workloads: nhat[e] = sum_g cnt[g, e] (the predicted counts).
+ * Rank loads under the placement pi: L[r] = sum_{e: pi[e] = r} nhat[e].
+ * Exchanging expert a on rank u with expert b on rank v changes only
+ *   L'[u] = L[u] - nhat[a] + nhat[b],   L'[v] = L[v] - nhat[b] + nhat[a]   (eq. 6-7).
+ * Objective Phi(L) = max_r L[r] + gamma * sum_r (L[r] - Lbar)^2 (eq. 8);
+ * benefit Delta = Phi(L) - Phi(L').  Lbar does not change under a swap, so
+ * the change of the squared term is the integer
+ *   (L[u]^2 + L[v]^2) - (L'[u]^2 + L'[v]^2)
+ * and Delta = (max L - max L') + gamma * that, evaluated in double as one
+ * product then one sum (reading: the pages fix no precision).
+ * Cost of a swap C = alpha + (S(a) + S(b)) / beta with S(e) = expert_bytes
+ * for every expert (eq. 9); budgets (eq. 10 gives their value): every rank
+ * may spend at most `budget`, every rank pair at most `link_budget`.
+ * Loop (Algorithm 1 with the frontier of sec. 3.3):
+ *   u = most-loaded rank, v = least-loaded rank (lowest id on ties);
+ *   stop when L[u] - L[v] <= tau;
+ *   candidates: a on u, b on v, neither moved yet in this plan, Delta > 0,
+ *   C within the residual budgets of u, v and the pair (u, v);
+ *   take the largest Delta / C (Delta alone when C = 0); ties by (u, v,
+ *   a, b) ascending (u, v are fixed here, so by a then b);
+ *   no candidate: stop; else swap, update loads and budgets, repeat.
+ * Outputs: pi_out[E], swaps[4 * n] (u, v, a, b) in acceptance order, the
+ * swap count, final loads[G].  pi_in NULL = the even placement e / (E/G).
+ * ------------------------------------------------------------------------ */
+int orc_plan_swaps(const int32_t *cnt, const int32_t *pi_in, int G, int E, double gamma, double tau,
+                   double alpha, double beta, double expert_bytes, double budget, double link_budget,
+                   int32_t *pi_out, int32_t *swaps, int32_t *n_swaps, int64_t *loads)
+{
+    if (G < 1 || E < 1 || E % G != 0 || !cnt || !pi_out || !swaps || !n_swaps || !loads || !(beta > 0.0) ||
+        !(gamma >= 0.0) || !(alpha >= 0.0) || !(expert_bytes >= 0.0) || !(tau >= 0.0) || !(budget >= 0.0) ||
+        !(link_budget >= 0.0))
+        return 1;
+    int64_t *nhat = calloc((size_t)E, sizeof(int64_t));
+    double *res_rank = calloc((size_t)G, sizeof(double));
+    double *res_link = calloc((size_t)G * G, sizeof(double));
+    uint8_t *moved = calloc((size_t)E, 1);
+    if (!nhat || !res_rank || !res_link || !moved) {
+        free(nhat); free(res_rank); free(res_link); free(moved);
+        return 1;
+    }
+    for (int g = 0; g < G; ++g)
+        for (int e = 0; e < E; ++e) nhat[e] += cnt[(int64_t)g * E + e];
+    for (int e = 0; e < E; ++e) {
+        const int r = pi_in ? pi_in[e] : e / (E / G);
+        if (r < 0 || r >= G) {
+            free(nhat); free(res_rank); free(res_link); free(moved);
+            return 3;
+        }
+        pi_out[e] = r;
+    }
+    for (int r = 0; r < G; ++r) loads[r] = 0;
+    for (int e = 0; e < E; ++e) loads[pi_out[e]] += nhat[e];
+    for (int r = 0; r < G; ++r) res_rank[r] = budget;
+    for (int i = 0; i < G * G; ++i) res_link[i] = link_budget;
+    const double cost = alpha + (expert_bytes + expert_bytes) / beta;
+
+    int n = 0;
+    for (;;) {
+        int u = 0, v = 0;
+        for (int r = 1; r < G; ++r) {
+            if (loads[r] > loads[u]) u = r;
+            if (loads[r] < loads[v]) v = r;
+        }
+        if ((double)(loads[u] - loads[v]) <= tau) break;
+        /* the largest load over the ranks the swap leaves alone */
+        int64_t rest = INT64_MIN;
+        for (int r = 0; r < G; ++r)
+            if (r != u && r != v && loads[r] > rest) rest = loads[r];
+        int best_a = -1, best_b = -1;
+        double best_ratio = 0.0;
+        const int feasible = res_rank[u] >= cost && res_rank[v] >= cost && res_link[u * G + v] >= cost;
+        for (int a = 0; a < E && feasible; ++a) {
+            if (pi_out[a] != u || moved[a]) continue;
+            for (int b = 0; b < E; ++b) {
+                if (pi_out[b] != v || moved[b]) continue;
+                const int64_t lu = loads[u] - nhat[a] + nhat[b];
+                const int64_t lv = loads[v] - nhat[b] + nhat[a];
+                int64_t mx = lu > lv ? lu : lv;
+                if (rest > mx) mx = rest;
+                const int64_t dsq = (loads[u] * loads[u] + loads[v] * loads[v]) - (lu * lu + lv * lv);
+                const double prod = gamma * (double)dsq;
+                const double delta = (double)(loads[u] - mx) + prod;
+                if (!(delta > 0.0)) continue;
+                /* a free swap (cost 0) ranks by its benefit alone */
+                const double ratio = cost > 0.0 ? delta / cost : delta;
+                /* a ascending, then b ascending: a strict '>' keeps the first */
+                if (best_a < 0 || ratio > best_ratio) {
+                    best_a = a;
+                    best_b = b;
+                    best_ratio = ratio;
+                }
+            }
+        }
+        if (best_a < 0) break;
+        const int a = best_a, b = best_b;
+        pi_out[a] = v;
+        pi_out[b] = u;
+        moved[a] = moved[b] = 1;
+        loads[u] = loads[u] - nhat[a] + nhat[b];
+        loads[v] = loads[v] - nhat[b] + nhat[a];
+        res_rank[u] -= cost;
+        res_rank[v] -= cost;
+        res_link[u * G + v] -= cost;
+        res_link[v * G + u] -= cost;
+        swaps[4 * n + 0] = u;
+        swaps[4 * n + 1] = v;
+        swaps[4 * n + 2] = a;
+        swaps[4 * n + 3] = b;
+        ++n;
+    }
+    *n_swaps = n;
+    free(nhat); free(res_rank); free(res_link); free(moved);
+    return 0;
 }

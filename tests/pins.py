@@ -409,10 +409,130 @@ def check_assign_invariants_random(o):
         assign_invariants(ids, cnt, p, s, dest, perm, offs)
 
 
+# ----------------------------------------------------------------------------- swaps (FreeBalance sec. 3.3)
+
+def check_swaps_golden(o):
+    for name in ("swaps_gamma_budget_tau.json", "swaps_two_ranks.json"):
+        d = golden(name)
+        for c in d["cases"]:
+            r = o.plan_swaps(np.array(d[c.get("cnt", "cnt")]), pi=c.get("pi_in"), gamma=c["gamma"], tau=c["tau"],
+                             alpha=c["alpha"], beta=c["beta"], expert_bytes=c["expert_bytes"], budget=c["budget"],
+                             link_budget=c.get("link_budget"))
+            assert r.swaps.tolist() == c["swaps"], (name, c, r.swaps.tolist())
+            assert r.pi.tolist() == c["pi"], (name, c)
+            assert r.loads.tolist() == c["loads"], (name, c)
+
+
+def phi_exact(L, gamma):
+    """eq. 8 of FreeBalance sec. 3.3, in exact rational arithmetic, over every
+    rank (the definition, not the two-rank update the planner uses)."""
+    Lf = [Fraction(int(x)) for x in L]
+    mean = sum(Lf) / len(Lf)
+    return max(Lf) + Fraction(gamma) * sum((x - mean) ** 2 for x in Lf)
+
+
+def swaps_invariants(cnt, pi_in, prm, r):
+    """Replay a swap plan with exact arithmetic: each accepted swap is between
+    the then most- and least-loaded ranks (lowest id on ties), while their
+    gap exceeds tau; it lowers Phi; it is the best feasible candidate of that
+    frontier by benefit / cost with ties by (a, b); no expert moves twice;
+    budgets per rank and per pair hold; the plan stops only when the gap is
+    within tau or the frontier has no feasible beneficial candidate; the
+    final loads and placement are those the swaps produce."""
+    G, E = cnt.shape
+    nh = cnt.sum(axis=0).astype(np.int64)
+    pi = list(pi_in) if pi_in is not None else [e // (E // G) for e in range(E)]
+    gamma, tau = prm["gamma"], Fraction(prm["tau"])
+    cost = Fraction(prm["alpha"]) + Fraction(2 * prm["expert_bytes"]) / Fraction(prm["beta"])
+    budget = Fraction(prm["budget"])
+    link_budget = Fraction(prm.get("link_budget", prm["budget"]))
+    spent_rank = [Fraction(0)] * G
+    spent_link = {}
+    moved = set()
+
+    def loads():
+        L = [0] * G
+        for e in range(E):
+            L[pi[e]] += int(nh[e])
+        return L
+
+    def frontier():
+        L = loads()
+        u = min(range(G), key=lambda x: (-L[x], x))
+        v = min(range(G), key=lambda x: (L[x], x))
+        return L, u, v
+
+    def candidates(L, u, v):
+        out = []
+        if not (spent_rank[u] + cost <= budget and spent_rank[v] + cost <= budget and
+                spent_link.get((min(u, v), max(u, v)), Fraction(0)) + cost <= link_budget):
+            return out
+        for a in range(E):
+            if pi[a] != u or a in moved:
+                continue
+            for b in range(E):
+                if pi[b] != v or b in moved:
+                    continue
+                L2 = list(L)
+                L2[u] += int(nh[b]) - int(nh[a])
+                L2[v] += int(nh[a]) - int(nh[b])
+                delta = phi_exact(L, gamma) - phi_exact(L2, gamma)
+                if delta > 0:
+                    out.append((delta / cost if cost > 0 else delta, a, b))
+        return out
+
+    for (u_, v_, a, b) in r.swaps.tolist():
+        L, u, v = frontier()
+        assert (u_, v_) == (u, v), "swap not on the most/least loaded pair"
+        assert Fraction(L[u] - L[v]) > tau, "swap taken although the gap is within tau"
+        cands = candidates(L, u, v)
+        assert cands, "swap taken with no feasible beneficial candidate"
+        best = max(x[0] for x in cands)
+        first = min((x for x in cands if x[0] == best), key=lambda x: (x[1], x[2]))
+        assert (a, b) == (first[1], first[2]), f"not the best candidate: {(a, b)} vs {first[1:]}"
+        assert a not in moved and b not in moved
+        pi[a], pi[b] = v, u
+        moved.update((a, b))
+        spent_rank[u] += cost
+        spent_rank[v] += cost
+        key = (min(u, v), max(u, v))
+        spent_link[key] = spent_link.get(key, Fraction(0)) + cost
+    assert all(x <= budget for x in spent_rank) and all(x <= link_budget for x in spent_link.values())
+    L, u, v = frontier()
+    assert Fraction(L[u] - L[v]) <= tau or not candidates(L, u, v), "planner stopped early"
+    assert r.pi.tolist() == pi and r.loads.tolist() == L
+    # swaps keep every rank's expert count
+    assert np.array_equal(np.bincount(r.pi, minlength=G),
+                          np.bincount(np.array(pi_in if pi_in is not None else [e // (E // G) for e in range(E)]),
+                                      minlength=G))
+
+
+def check_swaps_invariants_random(o):
+    rng = np.random.default_rng(21)
+    for G, E, T, k, prm in ((4, 16, 64, 2, dict(gamma=0.0, tau=0.0, alpha=0.0, beta=1.0, expert_bytes=0.0,
+                                                 budget=1e300)),
+                            (8, 64, 512, 8, dict(gamma=0.001, tau=0.0, alpha=5.0, beta=2.0, expert_bytes=9.0,
+                                                 budget=200.0)),
+                            (3, 12, 90, 3, dict(gamma=0.5, tau=4.0, alpha=1.0, beta=1.0, expert_bytes=1.0,
+                                                budget=6.0)),
+                            (2, 8, 40, 2, dict(gamma=0.25, tau=0.0, alpha=0.0, beta=1.0, expert_bytes=0.0,
+                                               budget=1e300)),
+                            (16, 128, 1024, 8, dict(gamma=1e-4, tau=2.0, alpha=2.0, beta=4.0, expert_bytes=8.0,
+                                                    budget=40.0)),
+                            (4, 32, 256, 4, dict(gamma=0.0, tau=0.0, alpha=1.0, beta=1.0, expert_bytes=0.0,
+                                                 budget=6.0, link_budget=1.0))):
+        for trial in range(3):
+            cnt = o.count(zipf_counts(rng, G, E, T, k), G, E)
+            pi_in = None if trial == 0 else rng.permutation(np.arange(E) // (E // G)).astype(np.int32)
+            r = o.plan_swaps(cnt, pi=pi_in, **prm)
+            swaps_invariants(cnt, pi_in, prm, r)
+
+
 ALL_CHECKS = [
     check_gate_exact_tiny, check_gate_matches_numpy, check_gate_ties, check_gate_cancellation,
     check_count, check_count_rejects,
     check_plan_golden, check_plan_phase1_ties, check_plan_invariants_random,
     check_split_golden, check_split_invariants_random, check_optimum_brute_force,
     check_assign_golden, check_assign_invariants_random,
+    check_swaps_golden, check_swaps_invariants_random,
 ]

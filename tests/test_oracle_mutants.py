@@ -37,6 +37,16 @@ MUTANTS = {
                               "{ int64_t at = fill[key]++; perm[(int64_t)offs[key + 1] - 1 - (at - offs[key])] = (int32_t)f; }"),
     "assign_remote_ignores_locality": ("if (holds[(int64_t)s * E + e]) {\n            d = s;",
                                        "if (0) {\n            d = s;"),
+    "swaps_drops_gamma": ("const double prod = gamma * (double)dsq;", "const double prod = 0.0 * (double)dsq;"),
+    "swaps_squared_term_sign": ("const double delta = (double)(loads[u] - mx) + prod;",
+                                "const double delta = (double)(loads[u] - mx) - prod;"),
+    "swaps_tie_to_last_pair": ("if (best_a < 0 || ratio > best_ratio)", "if (best_a < 0 || ratio >= best_ratio)"),
+    "swaps_expert_moves_twice": ("moved[a] = moved[b] = 1;", "(void)moved;"),
+    "swaps_link_budget_unspent": ("res_link[u * G + v] -= cost;\n        res_link[v * G + u] -= cost;", ";"),
+    "swaps_tau_strict": ("if ((double)(loads[u] - loads[v]) <= tau) break;",
+                         "if ((double)(loads[u] - loads[v]) < tau) break;"),
+    "swaps_frontier_tie_to_higher_rank": ("if (loads[r] > loads[u]) u = r;", "if (loads[r] >= loads[u]) u = r;"),
+    "swaps_ignores_untouched_ranks": ("if (rest > mx) mx = rest;", ";"),
     "optimum_ignores_fixed": ("orc_flow_add(&f, n_edges + r, snk, z - fixed[r]);",
                               "orc_flow_add(&f, n_edges + r, snk, z);"),
 }
