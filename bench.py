@@ -264,6 +264,7 @@ def run_ours(args, world, rank, local):
 
     # ---------------- count / split / assign as throughput kernels
     ints = integer_kernels_at_throughput(dev, world)
+    swp = swap_planner(wl, path, world)
 
     # ---------------- end to end through the C ABI with host buffers
     e2e = end_to_end(args, wl, hid, W, bias, path, dev, world, chain)
@@ -296,6 +297,7 @@ def run_ours(args, world, rank, local):
                      "algorithmic_bytes_per_launch": gate_bytes, "launch_us": gate_ms * 1e3,
                      "tensor_frac": gate_flops / (gate_ms * 1e-3) / (tflops * 1e12)},
         "integer_kernels": ints,
+        "swap_planner": swp,
         "e2e": e2e,
         "gpu_launches": launches * args.steps,
         "clocks": clk.summary(),
@@ -347,6 +349,60 @@ def per_layer_latency(wl, hid, W, bias, dev, reps):
                                                out=(p1.dest, p1.perm, p1.offs), workspace=p1.ws)),
     }
     return res
+
+
+def swap_planner(wl, path, world, reps=50):
+    """FreeBalance's budgeted pairwise-swap planner (lb_plan_swaps) as the
+    alternative to replication, on the step's predicted counts of every
+    layer: latency (one layer; all layers in one launch) and the max-to-mean
+    rank load before and after the swaps, on the predicted counts and on the
+    actual counts under the new placement.  Cost model (illustrative, stated):
+    alpha = 10 us per swap, beta = 770 GB/s (this machine's measured peer copy),
+    S = one expert's three bf16 matrices (3*H*I, I = 1024 for the OLMoE
+    shape), budget 200 us per rank and per link; gamma = 1 / (T*k)."""
+    from moe_expert_load_bf16_b200 import _lib
+    G, E = wl.G, wl.E
+    prm = dict(gamma=1.0 / (wl.T * wl.k), tau=0.0, alpha=10.0, beta=770e3, expert_bytes=3.0 * wl.H * 1024 * 2,
+               budget=200.0)
+    cp = path.cnt_pred.contiguous()
+    out = _lib.lb_plan_swaps(cp, **prm)
+    one = _lib.lb_plan_swaps(cp[0:1], **prm)
+    torch.cuda.synchronize()
+
+    def timed(fn):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            fn()
+        g.replay()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier(world)
+        a.record()
+        for _ in range(reps):
+            g.replay()
+        b.record()
+        torch.cuda.synchronize()
+        return max_over_ranks(a.elapsed_time(b) * 1e3 / reps, world)
+
+    t_all = timed(lambda: _lib.lb_plan_swaps(cp, out=out, **prm))
+    t_one = timed(lambda: _lib.lb_plan_swaps(cp[0:1], out=one, **prm))
+    # quality (reporting only): rank loads under the even and the new placement
+    even = (torch.arange(E, device=cp.device) // (E // G)).long()
+    pi = out[0].long()
+
+    def max_to_mean(n_e, placement):
+        loads = torch.zeros(n_e.shape[0], G, dtype=torch.float64, device=n_e.device)
+        loads.scatter_add_(1, placement.expand(n_e.shape[0], -1) if placement.dim() == 1 else placement,
+                           n_e.double())
+        return (loads.max(dim=1).values / loads.mean(dim=1)).mean().item()
+
+    n_pred = path.cnt_pred.sum(dim=1)
+    n_act = path.cnt.sum(dim=1)
+    return {"t_one_layer_us": t_one, "t_all_layers_us": t_all, "layers": int(cp.shape[0]),
+            "swaps_per_layer": out[2].double().mean().item(),
+            "max_to_mean_predicted": {"even": max_to_mean(n_pred, even), "swapped": max_to_mean(n_pred, pi)},
+            "max_to_mean_actual": {"even": max_to_mean(n_act, even), "swapped": max_to_mean(n_act, pi)},
+            "params": prm}
 
 
 def integer_kernels_at_throughput(dev, world, nbatch=128, reps=20):

@@ -192,6 +192,46 @@ typedef struct {
 int lb_plan_layout_of(int G, int E, int N, lb_plan_layout *out);
 
 /* ------------------------------------------------------------------------
+ * Step 3, alternative -- budgeted pairwise expert swaps   [FreeBalance sec.
+ * 3.3 eq. 6-10; Algorithm 1]
+ * Instead of replicating experts, exchange pairs of experts between ranks
+ * (every rank keeps its expert count; no replica, no split).
+ *   nhat[e] = sum_g cnt[b,g,e];  L[r] = sum_{e: pi[e]=r} nhat[e]
+ *   loop: u = most-loaded rank, v = least-loaded rank (lowest id on ties);
+ *     stop if L[u] - L[v] <= tau;
+ *     candidates: a on u, b on v, neither moved yet; their swap gives
+ *       L'[u] = L[u] - nhat[a] + nhat[b], L'[v] = L[v] - nhat[b] + nhat[a]
+ *       (eq. 6-7) and benefit Delta = Phi(L) - Phi(L') with
+ *       Phi(L) = max_r L[r] + gamma * sum_r (L[r] - mean)^2 (eq. 8),
+ *       evaluated in double as (L[u] - max L') + gamma * (integer change of
+ *       the squared term), one rounded product and one rounded sum;
+ *     cost C = alpha + 2 * expert_bytes / beta (eq. 9, every expert the same
+ *       size); a candidate needs Delta > 0 and C within the residual budgets
+ *       of u, of v (`budget` each) and of the pair (u, v) (`link_budget`);
+ *     take the largest Delta / C (Delta when C = 0), ties to the smaller
+ *       (a, b); swap; update loads and residual budgets; no candidate: stop.
+ *   cnt            int32 [nbatch, G, E] predicted counts (lb_count)
+ *   placement      int32 [nbatch, E] owner rank of each expert, or NULL for
+ *                  the even placement e / (E/G)
+ *   gamma, tau >= 0; alpha >= 0 (per-swap overhead), beta > 0 (bandwidth),
+ *   expert_bytes >= 0, budget and link_budget >= 0 (+inf allowed), in the
+ *   units of C
+ *   placement_out  int32 [nbatch, E]                       (output)
+ *   swaps_out      int32 [nbatch, lb_swaps_capacity(E), 4]: (u, v, a, b)
+ *                  in acceptance order                      (output)
+ *   n_swaps        int32 [nbatch]                          (output)
+ *   loads          int32 [nbatch, G] rank loads under placement_out (output)
+ * Limits: G <= LB_MAX_G, E <= LB_MAX_E, E % G == 0.  A placement entry
+ * outside [0, G) sets LB_DEV_BAD_PLAN and that problem gets n_swaps = 0
+ * (its other outputs unspecified).
+ * ------------------------------------------------------------------------ */
+int lb_swaps_capacity(int E);   /* rows of swaps_out per problem: E / 2 (at least 1) */
+int lb_plan_swaps(const int32_t *cnt, const int32_t *placement, int nbatch, int G, int E,
+                  double gamma, double tau, double alpha, double beta, double expert_bytes,
+                  double budget, double link_budget, int32_t *placement_out,
+                  int32_t *swaps_out, int32_t *n_swaps, int32_t *loads, void *stream);
+
+/* ------------------------------------------------------------------------
  * Step 4 -- Relief split   [Relief, Methodology, Algorithm 1; The Per-Step
  * Optimum Problem]
  * Remote mass of expert e: R_e = tokens of e whose source does not hold e.

@@ -47,6 +47,9 @@ def _load():
     lib.lb_predict_topk.argtypes = [P, P, P, I, I, I, I, I, P, P, P]
     lib.lb_predict_topk_chain.argtypes = [P, P, P, I, I, I, I, I, P, P, P, P, P]
     lib.lb_gate_tuning.argtypes = [I, I, I, I]
+    D = ctypes.c_double
+    lib.lb_swaps_capacity.argtypes = [I]
+    lib.lb_plan_swaps.argtypes = [P, P, I, I, I, D, D, D, D, D, D, D, P, P, P, P, P]
     lib.lb_count.argtypes = [P, I, I, I, I, I, P, P]
     lib.lb_plan_bytes.argtypes = [I, I, I]
     lib.lb_plan_bytes.restype = SZ
@@ -63,7 +66,8 @@ def _load():
     lib.lb_strerror.restype = ctypes.c_char_p
     lib.lb_last_error.argtypes = []
     lib.lb_last_error.restype = ctypes.c_char_p
-    for f in ("lb_predict_topk", "lb_gate_tuning", "lb_count", "lb_plan_layout_of", "lb_plan_replicas",
+    for f in ("lb_predict_topk", "lb_predict_topk_chain", "lb_plan_swaps", "lb_swaps_capacity", "lb_gate_tuning",
+              "lb_count", "lb_plan_layout_of", "lb_plan_replicas",
               "lb_split", "lb_assign", "lb_assign_noalloc", "lb_solve", "lb_get_status", "lb_version"):
         getattr(lib, f).restype = ctypes.c_int
     _lib = lib
@@ -162,6 +166,35 @@ def lb_predict_topk_chain(h, w, bias, k, want_logits=False, ids_pred=None, ids_a
     _check("lb_predict_topk_chain", lib.lb_predict_topk_chain(_p(h), _p(w), _p(bias), L, T, H, E, k, _p(outs[0]),
                                                               _p(outs[1]), _p(lg[0]), _p(lg[1]), _stream()))
     return (outs[0], outs[1], lg[0], lg[1]) if want_logits else (outs[0], outs[1])
+
+
+def lb_plan_swaps(cnt, placement=None, gamma=0.0, tau=0.0, alpha=0.0, beta=1.0, expert_bytes=0.0,
+                  budget=float("inf"), link_budget=None, out=None):
+    """Budgeted pairwise expert swaps (FreeBalance sec. 3.3).  cnt int32
+    [B,G,E] (or [G,E]); placement int32 [B,E] or None (even).  Returns
+    (placement_out [B,E], swaps [B,E//2,4], n_swaps [B], loads [B,G])."""
+    lib = _load()
+    squeeze = cnt.dim() == 2
+    cnt = _batched(cnt, 3)
+    _need(cnt, torch.int32, "cnt")
+    B, G, E = cnt.shape
+    if placement is not None:
+        placement = _batched(placement, 2)
+        _need(placement, torch.int32, "placement")
+        if placement.shape != (B, E):
+            raise ValueError("placement must be [B,E]")
+    cap = int(lib.lb_swaps_capacity(E))
+    if out is None:
+        dev = cnt.device
+        out = (torch.empty(B, E, dtype=torch.int32, device=dev), torch.empty(B, cap, 4, dtype=torch.int32, device=dev),
+               torch.empty(B, dtype=torch.int32, device=dev), torch.empty(B, G, dtype=torch.int32, device=dev))
+    pi_out, sw, ns, lo = out
+    link_budget = budget if link_budget is None else link_budget
+    _check("lb_plan_swaps", lib.lb_plan_swaps(_p(cnt), _p(placement), B, G, E, gamma, tau, alpha, beta, expert_bytes,
+                                              budget, link_budget, _p(pi_out), _p(sw), _p(ns), _p(lo), _stream()))
+    if squeeze:
+        return pi_out[0], sw[0], ns[0], lo[0]
+    return pi_out, sw, ns, lo
 
 
 def lb_gate_tuning(stages=0, split=0, persistent=0, kbox=0):
@@ -335,7 +368,7 @@ def lb_version():
     return int(_load().lb_version())
 
 
-EXPORTS = ("lb_predict_topk", "lb_predict_topk_chain", "lb_gate_tuning", "lb_count", "lb_plan_bytes", "lb_plan_layout_of",
+EXPORTS = ("lb_predict_topk", "lb_predict_topk_chain", "lb_gate_tuning", "lb_plan_swaps", "lb_swaps_capacity", "lb_count", "lb_plan_bytes", "lb_plan_layout_of",
            "lb_plan_replicas", "lb_split", "lb_assign_workspace_bytes", "lb_assign", "lb_assign_noalloc", "lb_solve",
            "lb_get_status",
            "lb_strerror", "lb_last_error", "lb_version")

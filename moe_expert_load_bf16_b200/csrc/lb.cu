@@ -5,6 +5,7 @@
 
 #include <algorithm>
 #include <climits>
+#include <cmath>
 #include <cstdio>
 #include <mutex>
 
@@ -14,6 +15,7 @@
 #include "gate_topk.cuh"
 #include "plan.cuh"
 #include "solve.cuh"
+#include "swaps.cuh"
 #include "split.cuh"
 
 namespace {
@@ -235,6 +237,8 @@ extern "C" {
 
 int lb_version(void) { return 100; }
 
+int lb_swaps_capacity(int E) { return E < 2 ? 1 : E / 2; }
+
 const char *lb_strerror(int code) {
     switch (code) {
         case LB_OK: return "ok";
@@ -433,6 +437,43 @@ int lb_predict_topk_chain(const void *h, const void *w, const float *bias, int L
         return LB_ECUDA;
     }
     return run_persistent(p, h, L + 1, mb, per_sm, mtiles, ntiles, sms, s);
+}
+
+int lb_plan_swaps(const int32_t *cnt, const int32_t *placement, int nbatch, int G, int E, double gamma, double tau,
+                  double alpha, double beta, double expert_bytes, double budget, double link_budget,
+                  int32_t *placement_out, int32_t *swaps_out, int32_t *n_swaps, int32_t *loads, void *stream) {
+    if (nbatch < 1 || nbatch > 65535 || G < 1 || G > LB_MAX_G || E < 1 || E > LB_MAX_E || E % G != 0)
+        return LB_EINVAL;
+    if (!cnt || !placement_out || !swaps_out || !n_swaps || !loads) return LB_EINVAL;
+    if (!aligned(cnt, 4) || !aligned(placement_out, 4) || !aligned(swaps_out, 4) || !aligned(n_swaps, 4) ||
+        !aligned(loads, 4) || (placement && !aligned(placement, 4)))
+        return LB_EINVAL;
+    // finite or +inf parameters in range (NaN fails every comparison)
+    if (!(gamma >= 0.0) || !(tau >= 0.0) || !(alpha >= 0.0) || !(beta > 0.0) || !(expert_bytes >= 0.0) ||
+        !(budget >= 0.0) || !(link_budget >= 0.0) || !(gamma < HUGE_VAL) || !(alpha < HUGE_VAL) ||
+        !(expert_bytes < HUGE_VAL))
+        return LB_EINVAL;
+    const size_t smem = swaps::smem_bytes(G, E);
+    if (smem > 224 * 1024) return LB_EINVAL;
+    swaps::Params p;
+    p.cnt = cnt;
+    p.pi_in = placement;
+    p.G = G;
+    p.E = E;
+    p.gamma = gamma;
+    p.tau = tau;
+    p.cost = alpha + (expert_bytes + expert_bytes) / beta;   // eq. 9 with S(e) = expert_bytes for every expert
+    p.budget = budget;
+    p.link_budget = link_budget;
+    p.pi_out = placement_out;
+    p.swaps = swaps_out;
+    p.n_swaps = n_swaps;
+    p.loads = loads;
+    p.max_swaps = lb_swaps_capacity(E);
+    static SmemLimit lim;
+    if (!allow_smem(swaps::swaps_kernel, lim, smem, false)) return LB_ECUDA;
+    swaps::swaps_kernel<<<nbatch, swaps::THREADS, smem, static_cast<cudaStream_t>(stream)>>>(p);
+    return launched("plan swaps");
 }
 
 int lb_count(const int32_t *ids, int nbatch, int T, int k, int E, int G, int32_t *cnt, void *stream) {

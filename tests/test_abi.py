@@ -60,6 +60,13 @@ def test_arguments_rejected_before_any_launch(lib):
     for L, E, k in ((2, 256, 2), (2, 24, 2), (0, 64, 2), (2, 16, 17)):
         assert lib.lb_predict_topk_chain(P(16), P(16), None, L, 128, 64, E, k, P(16), P(16), None, None,
                                          s) == _lib.LB_EINVAL
+    # swap planner: beta = 0, NaN gamma, E % G, G > 64, negative budget
+    D = ctypes.c_double
+    for G, E, gamma, beta, budget in ((4, 16, 0.0, 0.0, 1.0), (4, 16, float("nan"), 1.0, 1.0), (3, 16, 0.0, 1.0, 1.0),
+                                      (128, 128, 0.0, 1.0, 1.0), (4, 16, 0.0, 1.0, -1.0)):
+        assert lib.lb_plan_swaps(P(16), None, 1, G, E, D(gamma), D(0), D(0), D(beta), D(0), D(budget), D(budget),
+                                 P(16), P(16), P(16), P(16), s) == _lib.LB_EINVAL
+    assert lib.lb_swaps_capacity(16) == 8 and lib.lb_swaps_capacity(1) == 1
     assert lib.lb_count(P(16), 1, 10, 2, 16, 4, P(16), s) == _lib.LB_EINVAL          # T % G
     assert lib.lb_plan_replicas(P(256), 1, 3, 16, 1, 0, P(256), s) == _lib.LB_EINVAL  # E % G
     assert lib.lb_plan_replicas(P(256), 1, 4, 16, 20, 0, P(256), s) == _lib.LB_EINVAL  # N > E - E/G

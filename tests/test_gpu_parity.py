@@ -522,3 +522,69 @@ def test_scatter_repeated_id_in_row_is_flagged_and_contained():
     perm = path.perm[0].cpu().numpy()
     assert ((perm == -7) | ((perm >= 0) & (perm < T * k))).all()
     assert torch.ones(4, device=DEV).sum().item() == 4.0
+
+
+# ----------------------------------------------------------------------------- swap planner (FreeBalance sec. 3.3)
+def _swaps_check(cnt_np, pi_np, prm, gpu):
+    r = oracle.plan_swaps(cnt_np, pi=pi_np, **prm)
+    pi_out, sw, ns, lo = (t.cpu().numpy() for t in gpu)
+    n = int(ns)
+    assert n == r.n_swaps, (n, r.n_swaps)
+    assert np.array_equal(sw[:n], r.swaps), (sw[:n], r.swaps)
+    assert np.array_equal(pi_out, r.pi)
+    assert np.array_equal(lo.astype(np.int64), r.loads)
+
+
+def test_swaps_golden_cases():
+    import pins
+    for name in ("swaps_gamma_budget_tau.json", "swaps_two_ranks.json"):
+        d = pins.golden(name)
+        for c in d["cases"]:
+            cnt = np.array(d[c.get("cnt", "cnt")], np.int32)
+            prm = dict(gamma=c["gamma"], tau=c["tau"], alpha=c["alpha"], beta=c["beta"],
+                       expert_bytes=c["expert_bytes"], budget=c["budget"], link_budget=c.get("link_budget"))
+            pl = None if c.get("pi_in") is None else torch.tensor(c["pi_in"], dtype=torch.int32, device=DEV)
+            out = _lib.lb_plan_swaps(torch.from_numpy(cnt).to(DEV), pl, **prm)
+            torch.cuda.synchronize()
+            assert out[1][:int(out[2])].cpu().tolist() == c["swaps"]
+            assert out[0].cpu().tolist() == c["pi"] and out[3].cpu().tolist() == c["loads"]
+
+
+@pytest.mark.parametrize("G,E,B,prm", [
+    (8, 64, 16, dict(gamma=0.0)),
+    (8, 64, 16, dict(gamma=1e-3, alpha=5.0, beta=2.0, expert_bytes=9.0, budget=200.0)),
+    (16, 128, 8, dict(gamma=1e-4, tau=2.0, alpha=2.0, beta=4.0, expert_bytes=8.0, budget=40.0, link_budget=12.0)),
+    (64, 256, 4, dict(gamma=1e-5, alpha=1.0, beta=1.0, expert_bytes=1.0, budget=9.0)),
+    (2, 8, 6, dict(gamma=0.25)),
+    (3, 12, 6, dict(gamma=0.5, tau=4.0, alpha=1.0, beta=1.0, expert_bytes=1.0, budget=6.0)),
+    (40, 1000, 2, dict(gamma=0.0, alpha=1.0, beta=1.0, expert_bytes=0.0, budget=7.0)),
+    (1, 4, 2, dict(gamma=1.0)),
+])
+def test_swaps_match_oracle(G, E, B, prm):
+    """Batched problems with skewed predicted counts, even and shuffled
+    placements: swaps, placement and loads bit-exact with the oracle."""
+    rng = np.random.default_rng(G * 1000 + E)
+    cnts, pis = [], []
+    for b in range(B):
+        pr = rng.permutation(np.arange(1, E + 1)) ** -1.2
+        pr /= pr.sum()
+        cnts.append(rng.multinomial(G * 400, pr, size=G).astype(np.int32))
+        pis.append(rng.permutation(np.arange(E) // (E // G)).astype(np.int32))
+    cnt = np.stack(cnts)
+    for use_pi in (False, True):
+        pl = torch.from_numpy(np.stack(pis)).to(DEV) if use_pi else None
+        out = _lib.lb_plan_swaps(torch.from_numpy(cnt).to(DEV), pl, **prm)
+        torch.cuda.synchronize()
+        assert _lib.lb_get_status() == 0
+        for b in range(B):
+            _swaps_check(cnt[b], pis[b] if use_pi else None, prm, tuple(t[b] for t in out))
+
+
+def test_swaps_bad_placement_flagged():
+    cnt = torch.ones(2, 4, 16, dtype=torch.int32, device=DEV)
+    pl = (torch.arange(16, dtype=torch.int32, device=DEV) // 4).repeat(2, 1)
+    pl[1, 3] = 9
+    out = _lib.lb_plan_swaps(cnt, pl)
+    torch.cuda.synchronize()
+    assert _lib.lb_get_status(clear=True) & _lib.LB_DEV_BAD_PLAN
+    assert int(out[2][1]) == 0
