@@ -15,6 +15,8 @@ Functions (see lb_oracle.c for the definitions and the pages they follow):
   split_optimum(cnt, plan)               -> exact integer min-max load
   plan_swaps(cnt, pi, gamma, tau, alpha, beta, expert_bytes, budget)
                                          -> Swaps (budgeted pairwise swaps)
+  split_variant(cnt, plan, passes, variant)
+                                         -> Split (Relief's ablation variants)
 
 `Oracle(path)` binds the same functions to another build of lb_oracle.c
 (the tests use it to check that the pins reject planted mistakes).
@@ -112,6 +114,8 @@ class Oracle:
         d = ctypes.c_double
         lib.orc_plan_swaps.argtypes = [P, P, i32, i32, d, d, d, d, d, d, d, P, P, P, P]
         lib.orc_plan_swaps.restype = ctypes.c_int
+        lib.orc_split_variant.argtypes = [P, i32, i32, P, i32, P, P, P, i32, P, i32, i32, P, P, P, P]
+        lib.orc_split_variant.restype = ctypes.c_int
         for f in (lib.orc_gate, lib.orc_count, lib.orc_plan, lib.orc_split, lib.orc_assign):
             f.restype = ctypes.c_int
         lib.orc_threads.restype = ctypes.c_int
@@ -197,6 +201,24 @@ class Oracle:
             _ptr(tok), _ptr(mass), _ptr(dest), _ptr(perm), _ptr(offs)))
         return dest, perm, offs
 
+    # variants of Relief's ablation (see orc_split_variant for the readings)
+    SPLIT_VARIANTS = ("relief", "no_reverse", "jacobi", "hash", "water", "proportional", "fp32", "q1120")
+
+    def split_variant(self, cnt, p, passes=12, variant="relief"):
+        v = self.SPLIT_VARIANTS.index(variant) if isinstance(variant, str) else int(variant)
+        cnt = _c(cnt, np.int32)
+        G, E = cnt.shape
+        holds, eu, ev, ee, rp = self._plan_arrays(p)
+        ne = eu.shape[0]
+        tok = np.zeros(max(ne, 1), np.int32)
+        mass = np.zeros(max(ne, 1), np.int32)
+        loads = np.zeros(G, np.int64)
+        pr = ctypes.c_int32(0)
+        self._check("orc_split_variant", self.lib.orc_split_variant(
+            _ptr(cnt), G, E, _ptr(holds), ne, _ptr(eu), _ptr(ev), _ptr(ee), rp.shape[0] - 1, _ptr(rp), passes, v,
+            _ptr(tok), _ptr(mass), _ptr(loads), ctypes.byref(pr)))
+        return Split(tok[:ne].copy(), mass[:ne].copy(), loads, int(pr.value))
+
     def threads(self):
         return int(self.lib.orc_threads())
 
@@ -264,6 +286,10 @@ def split_optimum(*a, **kw):
 
 def plan_swaps(*a, **kw):
     return default().plan_swaps(*a, **kw)
+
+
+def split_variant(*a, **kw):
+    return default().split_variant(*a, **kw)
 
 
 def lib_path():

@@ -16,7 +16,7 @@ def build(force: bool = False, src: str = SRC, out: str = LIB) -> str:
     if not force and os.path.exists(out) and os.path.getmtime(out) >= os.path.getmtime(src):
         return out
     cmd = ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-fopenmp",
-           "-Wall", "-Wextra", "-Wno-unused-parameter", src, "-o", out]
+           "-Wall", "-Wextra", "-Wno-unused-parameter", src, "-o", out, "-lm"]
     subprocess.run(cmd, check=True)
     return out
 

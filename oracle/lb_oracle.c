@@ -28,6 +28,8 @@
  *   orc_plan_swaps    budgeted pairwise expert-swap planning, the alternative
  *                     to replication (FreeBalance sec. 3.3 eq. 6-10,
  *                     Algorithm 1)
+ *   orc_split_variant the split variants of Relief's ablation (Relief,
+ *                     Ablation Results, Table III; Key Properties, Q11.20)
  *
  * Readings taken where the pages are silent are stated beside the code that
  * takes them.  Return codes: 0 ok, 1 invalid argument, 3 bad data.
@@ -39,6 +41,7 @@
 #include <stdint.h>
 #include <stdlib.h>
 #include <string.h>
+#include <math.h>
 #ifdef _OPENMP
 #include <omp.h>
 #endif
@@ -904,4 +907,307 @@ int orc_plan_swaps(const int32_t *cnt, const int32_t *pi_in, int G, int E, doubl
     *n_swaps = n;
     free(nhat); free(res_rank); free(res_link); free(moved);
     return 0;
+}
+
+
+/* ------------------------------------------------------------------------
+ * Split variants (Relief, Ablation Results, Table III; The Relief Algorithm,
+ * key properties: all-integer Q11.20).  Same edges, schedule and starting
+ * point as orc_split (remote mass partitioned equally over a replicated
+ * expert's edges, all of it at home).  Readings of the variants, which the
+ * pages name without spelling out:
+ *   0 RELIEF      the reference (orc_split).
+ *   1 NO_REVERSE  Relief without the reverse move: a transfer only moves
+ *                 tokens from home to the replica (limit = 0 when the
+ *                 replica is the heavier end).
+ *   2 JACOBI      snapshot loads, damped: every transfer of a pass reads the
+ *                 loads of the pass start and moves |gap| >> 2 (a quarter in
+ *                 place of a half), capped as in Relief; all moves of the
+ *                 pass are applied together.
+ *   3 HASH        the load-oblivious split of a hash router: a replicated
+ *                 expert's remote tokens are divided equally over its holders
+ *                 (home first, then replicas by rank; remainders to the
+ *                 first holders).  No passes.
+ *   4 WATER       water-filling relaxation: each pass visits the replicated
+ *                 experts in ascending id; an expert's remote tokens are
+ *                 taken off its holders and poured back from the lowest load
+ *                 up (integer levels; the tokens left over at the last level
+ *                 go to the holders at that level in holder order), a
+ *                 replica never receiving more than its edge's tokens.
+ *   5 PROPORTIONAL each pass, each replicated expert (ascending id) divides
+ *                 its remote tokens over its holders in proportion to
+ *                 (max base load - base load + 1) (largest remainders, ties
+ *                 in holder order); a replica's excess over its edge's tokens
+ *                 stays at home.
+ *   6 FP32        Relief in single precision: loads and masses in fp32, the
+ *                 gap halved exactly (no truncation); at the end every mass
+ *                 is rounded to the nearest token (ties to even) and the
+ *                 loads recomputed.
+ *   7 Q1120       Relief in the engine's Q11.20 fixed point: quantities in
+ *                 units of 2^-f tokens, f = 20 - s with s the smallest shift
+ *                 that keeps the total load below 2^11 (11 integer bits);
+ *                 truncating halves at that resolution; at the end every mass
+ *                 is rounded to the nearest token (ties up) and the loads
+ *                 recomputed.
+ * Passes end early after a pass that changed nothing (variants 0-2, 4-7).
+ * ------------------------------------------------------------------------ */
+enum { ORC_SV_RELIEF = 0, ORC_SV_NO_REVERSE, ORC_SV_JACOBI, ORC_SV_HASH, ORC_SV_WATER, ORC_SV_PROPORTIONAL,
+       ORC_SV_FP32, ORC_SV_Q1120, ORC_SV_COUNT };
+
+/* Integer water-filling of R tokens over n holders with base loads B and
+ * capacities cap: the largest level lam with sum min(cap, max(0, lam - B)) <= R,
+ * then one more token to each holder still below its cap at that level, in
+ * holder order, until R is used up. */
+static void orc_water_fill(int n, const int64_t *B, const int64_t *cap, int64_t R, int64_t *a)
+{
+    int64_t lo = B[0], hi = B[0];
+    for (int h = 1; h < n; ++h) {
+        if (B[h] < lo) lo = B[h];
+        if (B[h] > hi) hi = B[h];
+    }
+    hi += R + 1;
+    /* f(lam) is non-decreasing; find the largest lam in [lo, hi] with f <= R */
+    while (lo < hi) {
+        int64_t mid = lo + (hi - lo + 1) / 2, f = 0;
+        for (int h = 0; h < n; ++h) {
+            int64_t x = mid - B[h];
+            if (x < 0) x = 0;
+            if (x > cap[h]) x = cap[h];
+            f += x;
+        }
+        if (f <= R) lo = mid; else hi = mid - 1;
+    }
+    int64_t used = 0;
+    for (int h = 0; h < n; ++h) {
+        int64_t x = lo - B[h];
+        if (x < 0) x = 0;
+        if (x > cap[h]) x = cap[h];
+        a[h] = x;
+        used += x;
+    }
+    for (int h = 0; h < n && used < R; ++h)
+        if (B[h] + a[h] <= lo && a[h] < cap[h]) { a[h] += 1; used += 1; }
+}
+
+int orc_split_variant(const int32_t *cnt, int G, int E, const uint8_t *holds, int n_edges, const int32_t *edge_u,
+                      const int32_t *edge_v, const int32_t *edge_e, int n_rounds, const int32_t *round_ptr,
+                      int passes, int variant, int32_t *tok, int32_t *mass, int64_t *loads, int32_t *passes_run)
+{
+    if (variant < 0 || variant >= ORC_SV_COUNT)
+        return ORC_EINVAL;
+    if (variant == ORC_SV_RELIEF)
+        return orc_split(cnt, G, E, holds, n_edges, edge_u, edge_v, edge_e, n_rounds, round_ptr, passes, tok, mass,
+                         loads, passes_run);
+    if (G <= 0 || E <= 0 || E % G != 0 || n_edges < 0 || n_rounds < 0 || passes < 0)
+        return ORC_EINVAL;
+    if (round_ptr[0] != 0 || round_ptr[n_rounds] != n_edges)
+        return ORC_EDATA;
+    int32_t *rep_cnt = malloc(sizeof(int32_t) * (size_t)E);
+    int32_t *rep_ptr = malloc(sizeof(int32_t) * (size_t)(E + 1));
+    int32_t *rep_edge = malloc(sizeof(int32_t) * (size_t)(n_edges + 1));
+    int64_t *R = malloc(sizeof(int64_t) * (size_t)E);
+    int64_t *fixed = malloc(sizeof(int64_t) * (size_t)G);
+    int64_t *snap = malloc(sizeof(int64_t) * (size_t)G);
+    int64_t *B = malloc(sizeof(int64_t) * (size_t)(G + 1));
+    int64_t *cap = malloc(sizeof(int64_t) * (size_t)(G + 1));
+    int64_t *a = malloc(sizeof(int64_t) * (size_t)(G + 1));
+    int64_t *wt = malloc(sizeof(int64_t) * (size_t)(G + 1));
+    int64_t *rm = malloc(sizeof(int64_t) * (size_t)(G + 1));
+    float *Lf = malloc(sizeof(float) * (size_t)G);
+    float *mf = malloc(sizeof(float) * (size_t)(n_edges + 1));
+    int64_t *Lq = malloc(sizeof(int64_t) * (size_t)G);
+    int64_t *mq = malloc(sizeof(int64_t) * (size_t)(n_edges + 1));
+    int rc = ORC_OK;
+    if (!rep_cnt || !rep_ptr || !rep_edge || !R || !fixed || !snap || !B || !cap || !a || !wt || !rm || !Lf ||
+        !mf || !Lq || !mq) {
+        rc = ORC_EINVAL;
+        goto done;
+    }
+    for (int r = 0; r < n_rounds; ++r) {
+        if (round_ptr[r + 1] < round_ptr[r]) { rc = ORC_EDATA; goto done; }
+        for (int i = round_ptr[r]; i < round_ptr[r + 1]; ++i)
+            for (int i2 = round_ptr[r]; i2 < i; ++i2)
+                if (edge_u[i] == edge_u[i2] || edge_u[i] == edge_v[i2] || edge_v[i] == edge_u[i2] ||
+                    edge_v[i] == edge_v[i2]) { rc = ORC_EDATA; goto done; }
+    }
+    rc = orc_edges_by_expert(G, E, holds, n_edges, edge_u, edge_v, edge_e, rep_cnt, rep_ptr, rep_edge);
+    if (rc != ORC_OK)
+        goto done;
+    orc_split_start(cnt, G, E, holds, rep_cnt, rep_ptr, rep_edge, R, fixed, tok);
+    for (int i = 0; i < G; ++i)
+        loads[i] = fixed[i];
+    for (int i = 0; i < n_edges; ++i) {
+        mass[i] = tok[i];
+        loads[edge_u[i]] += tok[i];
+    }
+    *passes_run = 0;
+
+    if (variant == ORC_SV_NO_REVERSE || variant == ORC_SV_JACOBI) {
+        for (int p = 1; p <= passes; ++p) {
+            int moved = 0;
+            if (variant == ORC_SV_JACOBI)
+                for (int i = 0; i < G; ++i) snap[i] = loads[i];
+            for (int r = 0; r < n_rounds; ++r)
+                for (int i = round_ptr[r]; i < round_ptr[r + 1]; ++i) {
+                    const int u = edge_u[i], v = edge_v[i];
+                    const int64_t gap = variant == ORC_SV_JACOBI ? snap[u] - snap[v] : loads[u] - loads[v];
+                    int64_t delta = (gap < 0 ? -gap : gap) >> (variant == ORC_SV_JACOBI ? 2 : 1);
+                    int64_t limit = gap > 0 ? (int64_t)mass[i]
+                                            : (variant == ORC_SV_NO_REVERSE ? 0 : (int64_t)(tok[i] - mass[i]));
+                    if (delta > limit) delta = limit;
+                    if (delta > 0) {
+                        const int64_t sd = gap > 0 ? delta : -delta;
+                        loads[u] -= sd;
+                        loads[v] += sd;
+                        mass[i] -= (int32_t)sd;
+                        moved = 1;
+                    }
+                }
+            *passes_run = p;
+            if (!moved) break;
+        }
+    } else if (variant == ORC_SV_HASH) {
+        for (int e = 0; e < E; ++e) {
+            const int m = rep_cnt[e];
+            if (m == 0) continue;
+            const int64_t q = R[e] / (m + 1), rem = R[e] % (m + 1);
+            const int home = e / (E / G);
+            for (int j = 0; j < m; ++j) {
+                const int i = rep_edge[rep_ptr[e] + j];
+                int64_t share = q + (j + 1 < rem ? 1 : 0);   /* holder j + 1; holder 0 is home */
+                if (share > tok[i]) share = tok[i];
+                mass[i] = (int32_t)(tok[i] - share);
+                loads[home] -= share;
+                loads[edge_v[i]] += share;
+            }
+        }
+    } else if (variant == ORC_SV_WATER || variant == ORC_SV_PROPORTIONAL) {
+        for (int p = 1; p <= passes; ++p) {
+            int changed = 0;
+            for (int e = 0; e < E; ++e) {
+                const int m = rep_cnt[e];
+                if (m == 0) continue;
+                const int home = e / (E / G);
+                /* holders: 0 = home, j + 1 = replica of edge j; base loads without e's remote tokens */
+                int64_t at_home = 0;
+                for (int j = 0; j < m; ++j) at_home += mass[rep_edge[rep_ptr[e] + j]];
+                B[0] = loads[home] - at_home;
+                cap[0] = R[e];
+                for (int j = 0; j < m; ++j) {
+                    const int i = rep_edge[rep_ptr[e] + j];
+                    B[j + 1] = loads[edge_v[i]] - (tok[i] - mass[i]);
+                    cap[j + 1] = tok[i];
+                }
+                const int n = m + 1;
+                if (variant == ORC_SV_WATER) {
+                    orc_water_fill(n, B, cap, R[e], a);
+                } else {
+                    int64_t M = B[0], W = 0, used = 0;
+                    for (int h = 1; h < n; ++h) if (B[h] > M) M = B[h];
+                    for (int h = 0; h < n; ++h) { wt[h] = M - B[h] + 1; W += wt[h]; }
+                    for (int h = 0; h < n; ++h) {
+                        a[h] = (R[e] * wt[h]) / W;
+                        rm[h] = (R[e] * wt[h]) % W;
+                        used += a[h];
+                    }
+                    /* largest remainders, ties in holder order */
+                    while (used < R[e]) {
+                        int best = 0;
+                        for (int h = 1; h < n; ++h) if (rm[h] > rm[best]) best = h;
+                        a[best] += 1;
+                        rm[best] = -1;
+                        used += 1;
+                    }
+                    for (int h = 1; h < n; ++h)
+                        if (a[h] > cap[h]) { a[0] += a[h] - cap[h]; a[h] = cap[h]; }
+                }
+                loads[home] = B[0] + a[0];
+                for (int j = 0; j < m; ++j) {
+                    const int i = rep_edge[rep_ptr[e] + j];
+                    const int32_t nm = (int32_t)(tok[i] - a[j + 1]);
+                    if (nm != mass[i]) changed = 1;
+                    mass[i] = nm;
+                    loads[edge_v[i]] = B[j + 1] + a[j + 1];
+                }
+            }
+            *passes_run = p;
+            if (!changed) break;
+        }
+    } else if (variant == ORC_SV_FP32) {
+        for (int i = 0; i < G; ++i) Lf[i] = (float)fixed[i];
+        for (int i = 0; i < n_edges; ++i) {
+            mf[i] = (float)tok[i];
+            Lf[edge_u[i]] += (float)tok[i];   /* in edge order, one rounded sum at a time */
+        }
+        for (int p = 1; p <= passes; ++p) {
+            int moved = 0;
+            for (int r = 0; r < n_rounds; ++r)
+                for (int i = round_ptr[r]; i < round_ptr[r + 1]; ++i) {
+                    const int u = edge_u[i], v = edge_v[i];
+                    const float gap = Lf[u] - Lf[v];
+                    float delta = (gap < 0.0f ? -gap : gap) * 0.5f;
+                    const float limit = gap > 0.0f ? mf[i] : (float)tok[i] - mf[i];
+                    if (delta > limit) delta = limit;
+                    if (delta > 0.0f) {
+                        const float sd = gap > 0.0f ? delta : -delta;
+                        Lf[u] -= sd;
+                        Lf[v] += sd;
+                        mf[i] -= sd;
+                        moved = 1;
+                    }
+                }
+            *passes_run = p;
+            if (!moved) break;
+        }
+        for (int i = 0; i < G; ++i) loads[i] = fixed[i];
+        for (int i = 0; i < n_edges; ++i) {
+            float x = rintf(mf[i]);   /* nearest, ties to even (default rounding mode) */
+            if (x < 0.0f) x = 0.0f;
+            if (x > (float)tok[i]) x = (float)tok[i];
+            mass[i] = (int32_t)x;
+            loads[edge_u[i]] += mass[i];
+            loads[edge_v[i]] += tok[i] - mass[i];
+        }
+    } else { /* ORC_SV_Q1120 */
+        int64_t total = 0;
+        for (int i = 0; i < G; ++i) total += loads[i];
+        int s = 0;
+        while ((total >> s) >= 2048) ++s;
+        const int f = 20 - s;   /* fractional bits at this scale (total < 2^31 so s <= 20) */
+        for (int i = 0; i < G; ++i) Lq[i] = loads[i] << f;
+        for (int i = 0; i < n_edges; ++i) mq[i] = (int64_t)tok[i] << f;
+        for (int p = 1; p <= passes; ++p) {
+            int moved = 0;
+            for (int r = 0; r < n_rounds; ++r)
+                for (int i = round_ptr[r]; i < round_ptr[r + 1]; ++i) {
+                    const int u = edge_u[i], v = edge_v[i];
+                    const int64_t gap = Lq[u] - Lq[v];
+                    int64_t delta = (gap < 0 ? -gap : gap) >> 1;
+                    const int64_t limit = gap > 0 ? mq[i] : ((int64_t)tok[i] << f) - mq[i];
+                    if (delta > limit) delta = limit;
+                    if (delta > 0) {
+                        const int64_t sd = gap > 0 ? delta : -delta;
+                        Lq[u] -= sd;
+                        Lq[v] += sd;
+                        mq[i] -= sd;
+                        moved = 1;
+                    }
+                }
+            *passes_run = p;
+            if (!moved) break;
+        }
+        for (int i = 0; i < G; ++i) loads[i] = fixed[i];
+        for (int i = 0; i < n_edges; ++i) {
+            int64_t x = f > 0 ? (mq[i] + ((int64_t)1 << (f - 1))) >> f : mq[i];
+            if (x < 0) x = 0;
+            if (x > tok[i]) x = tok[i];
+            mass[i] = (int32_t)x;
+            loads[edge_u[i]] += mass[i];
+            loads[edge_v[i]] += tok[i] - mass[i];
+        }
+    }
+done:
+    free(rep_cnt); free(rep_ptr); free(rep_edge); free(R); free(fixed); free(snap); free(B); free(cap); free(a);
+    free(wt); free(rm); free(Lf); free(mf); free(Lq); free(mq);
+    return rc;
 }

@@ -409,6 +409,68 @@ def check_assign_invariants_random(o):
         assign_invariants(ids, cnt, p, s, dest, perm, offs)
 
 
+# ----------------------------------------------------------------------------- split variants (Relief Table III)
+
+def check_split_variants_golden(o):
+    d = golden("split_variants.json")
+    for variant, rows in d["expect"].items():
+        for fx, (mass, loads, passes_run) in zip(d["fixtures"], rows):
+            f = golden(fx)
+            s = o.split_variant(np.array(f["cnt"], np.int32), golden_plan(o, f), f["passes"], variant)
+            assert s.mass.tolist() == mass, (variant, fx, s.mass.tolist())
+            assert s.loads.tolist() == loads, (variant, fx, s.loads.tolist())
+            assert s.passes_run == passes_run, (variant, fx, s.passes_run)
+            assert s.tok.tolist() == f["tok"], (variant, fx)
+
+
+def check_split_variants_invariants_random(o):
+    """Every variant: the same starting partition as Relief, 0 <= mass <= tok,
+    the loads equal the fixed loads plus the masses at home and the rest at
+    the replicas, the total is T*k, and max L >= the exact optimum.
+    Water-filling with one replicated expert reaches the exact optimum (the
+    flow computation, a different method)."""
+    rng = np.random.default_rng(17)
+    for G, E, N, L, T, k in ((4, 16, 1, 0, 64, 2), (8, 64, 2, 1, 256, 8), (3, 9, 3, 2, 60, 3),
+                             (16, 128, 2, 1, 1024, 8)):
+        ids = zipf_counts(rng, G, E, T, k)
+        cnt = o.count(ids, G, E)
+        p = o.plan(cnt, N, L)
+        ref = o.split(cnt, p)
+        opt = o.split_optimum(cnt, p)
+        for variant in o.SPLIT_VARIANTS:
+            for passes in (0, 1, 12):
+                s = o.split_variant(cnt, p, passes, variant)
+                assert np.array_equal(s.tok, ref.tok)
+                assert ((s.mass >= 0) & (s.mass <= s.tok)).all()
+                loads = np.zeros(G, np.int64)
+                for i in range(p.n_edges):
+                    loads[p.edge_u[i]] += s.mass[i]
+                    loads[p.edge_v[i]] += s.tok[i] - s.mass[i]
+                fixed = ref.loads.copy()
+                for i in range(p.n_edges):
+                    fixed[p.edge_u[i]] -= ref.mass[i]
+                    fixed[p.edge_v[i]] -= ref.tok[i] - ref.mass[i]
+                assert np.array_equal(loads + fixed, s.loads), (variant, passes)
+                assert s.loads.sum() == T * k
+                assert s.loads.max() >= opt
+    # single replicated expert: water-filling is optimal
+    for trial in range(6):
+        G, E = 6, 12
+        cnt = rng.integers(0, 30, (G, E)).astype(np.int32)
+        e0 = int(rng.integers(E))
+        h = e0 // (E // G)
+        reps = sorted(rng.choice([r for r in range(G) if r != h], size=int(rng.integers(1, 4)), replace=False))
+        holds = np.zeros((G, E), np.uint8)
+        for e in range(E):
+            holds[e // (E // G), e] = 1
+        for r in reps:
+            holds[r, e0] = 1
+        pl = __import__("oracle").plan_from_arrays(G, E, len(reps), 0, holds, [h] * len(reps), list(reps),
+                                                   [e0] * len(reps), list(range(len(reps) + 1)))
+        s = o.split_variant(cnt, pl, 4, "water")
+        assert int(s.loads.max()) == o.split_optimum(cnt, pl), trial
+
+
 # ----------------------------------------------------------------------------- swaps (FreeBalance sec. 3.3)
 
 def check_swaps_golden(o):
@@ -535,4 +597,5 @@ ALL_CHECKS = [
     check_split_golden, check_split_invariants_random, check_optimum_brute_force,
     check_assign_golden, check_assign_invariants_random,
     check_swaps_golden, check_swaps_invariants_random,
+    check_split_variants_golden, check_split_variants_invariants_random,
 ]

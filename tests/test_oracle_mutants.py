@@ -47,6 +47,18 @@ MUTANTS = {
                          "if ((double)(loads[u] - loads[v]) < tau) break;"),
     "swaps_frontier_tie_to_higher_rank": ("if (loads[r] > loads[u]) u = r;", "if (loads[r] >= loads[u]) u = r;"),
     "swaps_ignores_untouched_ranks": ("if (rest > mx) mx = rest;", ";"),
+    "variant_no_reverse_allows_reverse": ("(variant == ORC_SV_NO_REVERSE ? 0 : (int64_t)(tok[i] - mass[i]))",
+                                          "(int64_t)(tok[i] - mass[i])"),
+    "variant_jacobi_not_damped": ("(gap < 0 ? -gap : gap) >> (variant == ORC_SV_JACOBI ? 2 : 1)",
+                                  "(gap < 0 ? -gap : gap) >> 1"),
+    "variant_jacobi_no_snapshot": ("for (int i = 0; i < G; ++i) snap[i] = loads[i];",
+                                   "for (int i = 0; i < G && p == 1; ++i) snap[i] = loads[i];"),
+    "variant_hash_remainder_shifted": ("int64_t share = q + (j + 1 < rem ? 1 : 0);", "int64_t share = q + (j < rem ? 1 : 0);"),
+    "variant_water_leftover_last": ("for (int h = 0; h < n && used < R; ++h)", "for (int h = n - 1; h >= 0 && used < R; --h)"),
+    "variant_proportional_equal_weights": ("wt[h] = M - B[h] + 1;", "wt[h] = 1;"),
+    "variant_fp32_truncates": ("float delta = (gap < 0.0f ? -gap : gap) * 0.5f;",
+                               "float delta = floorf((gap < 0.0f ? -gap : gap) * 0.5f);"),
+    "variant_q1120_no_fraction": ("const int f = 20 - s;", "const int f = 0 * s;"),
     "optimum_ignores_fixed": ("orc_flow_add(&f, n_edges + r, snk, z - fixed[r]);",
                               "orc_flow_add(&f, n_edges + r, snk, z);"),
 }
