@@ -255,6 +255,32 @@ int lb_split(const int32_t *cnt, const void *plan, int nbatch, int G, int E, int
              int32_t *passes_run, void *stream);
 
 /* ------------------------------------------------------------------------
+ * Step 4, ablation variants   [Relief, Ablation Results, Table III; The
+ * Relief Algorithm, key properties (Q11.20)]
+ * The same inputs, starting point and outputs as lb_split, with the pass
+ * replaced by variant:
+ *   0 Relief (as lb_split)      1 no reverse move (home -> replica only)
+ *   2 Jacobi: loads snapshotted per pass, moves of |gap| >> 2
+ *   3 hash split: remote tokens divided equally over home and replicas
+ *     (home first, remainders to the first holders); no passes
+ *   4 water-filling: experts in ascending id, each poured over its holders
+ *     from the lowest load up (integer levels, leftovers in holder order,
+ *     replicas capped at their edge's tokens)
+ *   5 proportional: experts in ascending id, remote tokens divided in
+ *     proportion to (max base load - base load + 1), largest remainders,
+ *     a replica's excess over its edge's tokens kept at home
+ *   6 fp32 Relief (exact halving; masses rounded to nearest, ties to even)
+ *   7 Q11.20 Relief (units of 2^-f tokens, f = 20 - s, s the smallest shift
+ *     keeping the total load below 2^11; masses rounded to nearest, ties up)
+ * Passes end after a pass that changes nothing (all but 3).
+ * Limits: as lb_split, G <= 64; rounds of at most 32 transfers.  A plan
+ * whose header or round table is inconsistent sets LB_DEV_BAD_PLAN.
+ * ------------------------------------------------------------------------ */
+int lb_split_variant(const int32_t *cnt, const void *plan, int nbatch, int G, int E, int N,
+                     int passes, int variant, int32_t *tok, int32_t *mass, int32_t *loads,
+                     int32_t *passes_run, void *stream);
+
+/* ------------------------------------------------------------------------
  * Step 5 -- destinations + stable permutation   [Libra, Key Ideas,
  * two-stage locality-aware execution and token sharding; FB sec. 2.2]
  * For assignment f = t*k + j (e = ids[t,j], s = src(t)):

@@ -50,6 +50,7 @@ def _load():
     D = ctypes.c_double
     lib.lb_swaps_capacity.argtypes = [I]
     lib.lb_plan_swaps.argtypes = [P, P, I, I, I, D, D, D, D, D, D, D, P, P, P, P, P]
+    lib.lb_split_variant.argtypes = [P, P, I, I, I, I, I, I, P, P, P, P, P]
     lib.lb_count.argtypes = [P, I, I, I, I, I, P, P]
     lib.lb_plan_bytes.argtypes = [I, I, I]
     lib.lb_plan_bytes.restype = SZ
@@ -66,7 +67,8 @@ def _load():
     lib.lb_strerror.restype = ctypes.c_char_p
     lib.lb_last_error.argtypes = []
     lib.lb_last_error.restype = ctypes.c_char_p
-    for f in ("lb_predict_topk", "lb_predict_topk_chain", "lb_plan_swaps", "lb_swaps_capacity", "lb_gate_tuning",
+    for f in ("lb_predict_topk", "lb_predict_topk_chain", "lb_plan_swaps", "lb_swaps_capacity", "lb_split_variant",
+              "lb_gate_tuning",
               "lb_count", "lb_plan_layout_of", "lb_plan_replicas",
               "lb_split", "lb_assign", "lb_assign_noalloc", "lb_solve", "lb_get_status", "lb_version"):
         getattr(lib, f).restype = ctypes.c_int
@@ -195,6 +197,29 @@ def lb_plan_swaps(cnt, placement=None, gamma=0.0, tau=0.0, alpha=0.0, beta=1.0, 
     if squeeze:
         return pi_out[0], sw[0], ns[0], lo[0]
     return pi_out, sw, ns, lo
+
+
+SPLIT_VARIANTS = ("relief", "no_reverse", "jacobi", "hash", "water", "proportional", "fp32", "q1120")
+
+
+def lb_split_variant(cnt, plan, N, passes=12, variant="relief", out=None):
+    """Relief's ablation variants (see include/lb.h); same shapes as lb_split."""
+    lib = _load()
+    v = SPLIT_VARIANTS.index(variant) if isinstance(variant, str) else int(variant)
+    squeeze = cnt.dim() == 2
+    cnt = _batched(cnt, 3)
+    plan = _batched(plan, 2)
+    _need(cnt, torch.int32, "cnt")
+    B, G, E = cnt.shape
+    if out is None:
+        dev = cnt.device
+        out = tuple(torch.zeros(*sh, dtype=torch.int32, device=dev) for sh in ((B, G * N), (B, G * N), (B, G), (B,)))
+    tok, mass, loads, pr = out
+    _check("lb_split_variant", lib.lb_split_variant(_p(cnt), _p(plan), B, G, E, N, passes, v, _p(tok), _p(mass),
+                                                    _p(loads), _p(pr), _stream()))
+    if squeeze:
+        return tok[0], mass[0], loads[0], pr[0]
+    return tok, mass, loads, pr
 
 
 def lb_gate_tuning(stages=0, split=0, persistent=0, kbox=0):
@@ -368,7 +393,8 @@ def lb_version():
     return int(_load().lb_version())
 
 
-EXPORTS = ("lb_predict_topk", "lb_predict_topk_chain", "lb_gate_tuning", "lb_plan_swaps", "lb_swaps_capacity", "lb_count", "lb_plan_bytes", "lb_plan_layout_of",
+EXPORTS = ("lb_predict_topk", "lb_predict_topk_chain", "lb_gate_tuning", "lb_plan_swaps", "lb_swaps_capacity",
+           "lb_split_variant", "lb_count", "lb_plan_bytes", "lb_plan_layout_of",
            "lb_plan_replicas", "lb_split", "lb_assign_workspace_bytes", "lb_assign", "lb_assign_noalloc", "lb_solve",
            "lb_get_status",
            "lb_strerror", "lb_last_error", "lb_version")

@@ -16,6 +16,7 @@
 #include "plan.cuh"
 #include "solve.cuh"
 #include "swaps.cuh"
+#include "split_variants.cuh"
 #include "split.cuh"
 
 namespace {
@@ -474,6 +475,36 @@ int lb_plan_swaps(const int32_t *cnt, const int32_t *placement, int nbatch, int 
     if (!allow_smem(swaps::swaps_kernel, lim, smem, false)) return LB_ECUDA;
     swaps::swaps_kernel<<<nbatch, swaps::THREADS, smem, static_cast<cudaStream_t>(stream)>>>(p);
     return launched("plan swaps");
+}
+
+int lb_split_variant(const int32_t *cnt, const void *plan, int nbatch, int G, int E, int N, int passes, int variant,
+                     int32_t *tok, int32_t *mass, int32_t *loads, int32_t *passes_run, void *stream) {
+    if (nbatch < 1 || nbatch > 65535 || !plan_shape_ok(G, E, N, 0) || passes < 0 || passes > 4096 || variant < 0 ||
+        variant >= splitv::COUNT)
+        return LB_EINVAL;
+    if (!cnt || !plan || !loads || !passes_run || !aligned(cnt, 4) || !aligned(plan, 256) || !aligned(loads, 4) ||
+        !aligned(passes_run, 4))
+        return LB_EINVAL;
+    if (G * N > 0 && (!tok || !mass || !aligned(tok, 4) || !aligned(mass, 4))) return LB_EINVAL;
+    const size_t smem = splitv::smem_bytes(G, E, N);
+    if (smem > 224 * 1024) return LB_EINVAL;
+    splitv::Params p;
+    p.cnt = cnt;
+    p.plan = static_cast<const uint8_t *>(plan);
+    p.plan_stride = plan::layout(G, E, N).total;
+    p.G = G;
+    p.E = E;
+    p.N = N;
+    p.passes = passes;
+    p.variant = variant;
+    p.tok = tok;
+    p.mass = mass;
+    p.loads = loads;
+    p.passes_run = passes_run;
+    static SmemLimit lim;
+    if (!allow_smem(splitv::split_variant_kernel, lim, smem, false)) return LB_ECUDA;
+    splitv::split_variant_kernel<<<nbatch, splitv::THREADS, smem, static_cast<cudaStream_t>(stream)>>>(p);
+    return launched("split variant");
 }
 
 int lb_count(const int32_t *ids, int nbatch, int T, int k, int E, int G, int32_t *cnt, void *stream) {

@@ -67,6 +67,9 @@ def test_arguments_rejected_before_any_launch(lib):
         assert lib.lb_plan_swaps(P(16), None, 1, G, E, D(gamma), D(0), D(0), D(beta), D(0), D(budget), D(budget),
                                  P(16), P(16), P(16), P(16), s) == _lib.LB_EINVAL
     assert lib.lb_swaps_capacity(16) == 8 and lib.lb_swaps_capacity(1) == 1
+    # split variants: unknown variant, negative passes
+    assert lib.lb_split_variant(P(256), P(256), 1, 4, 16, 1, 12, 8, P(16), P(16), P(16), P(16), s) == _lib.LB_EINVAL
+    assert lib.lb_split_variant(P(256), P(256), 1, 4, 16, 1, -1, 0, P(16), P(16), P(16), P(16), s) == _lib.LB_EINVAL
     assert lib.lb_count(P(16), 1, 10, 2, 16, 4, P(16), s) == _lib.LB_EINVAL          # T % G
     assert lib.lb_plan_replicas(P(256), 1, 3, 16, 1, 0, P(256), s) == _lib.LB_EINVAL  # E % G
     assert lib.lb_plan_replicas(P(256), 1, 4, 16, 20, 0, P(256), s) == _lib.LB_EINVAL  # N > E - E/G

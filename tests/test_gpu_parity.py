@@ -588,3 +588,44 @@ def test_swaps_bad_placement_flagged():
     torch.cuda.synchronize()
     assert _lib.lb_get_status(clear=True) & _lib.LB_DEV_BAD_PLAN
     assert int(out[2][1]) == 0
+
+
+# ----------------------------------------------------------------------------- split variants (Relief Table III)
+@pytest.mark.parametrize("variant", _lib.SPLIT_VARIANTS)
+@pytest.mark.parametrize("G,E,N,L,T,k,passes", [(8, 64, 2, 1, 4096, 8, 12), (16, 128, 2, 1, 2048, 8, 12),
+                                                (64, 256, 2, 1, 1024, 8, 12), (4, 16, 3, 2, 400, 2, 3),
+                                                (3, 9, 2, 1, 90, 3, 0), (64, 256, 2, 1, 8192, 8, 40)])
+def test_split_variants_match_oracle(variant, G, E, N, L, T, k, passes):
+    """Each ablation variant on batched problems (plans from the predicted
+    counts, split of the actual counts): tok, mass, loads and passes_run
+    bit-exact with the oracle."""
+    B = 3
+    rng = np.random.default_rng(G + E + T + passes)
+    pr = rng.permutation(np.arange(1, E + 1)) ** -1.2
+    pr /= pr.sum()
+    ids_np = np.stack([np.stack([rng.choice(E, k, replace=False, p=pr) for _ in range(T)]) for _ in range(2 * B)])
+    ids = torch.from_numpy(ids_np.astype(np.int32)).to(DEV)
+    cnt_pred = _lib.lb_count(ids[:B], G, E)
+    cnt = _lib.lb_count(ids[B:], G, E)
+    plan = torch.empty(B, _lib.lb_plan_bytes(G, E, N), dtype=torch.uint8, device=DEV)
+    _lib.lb_plan_replicas(cnt_pred, N, L, plan=plan)
+    tok, mass, loads, prun = _lib.lb_split_variant(cnt, plan, N, passes, variant)
+    torch.cuda.synchronize()
+    assert _lib.lb_get_status() == 0
+    for b in range(B):
+        p = oracle.plan(cnt_pred[b].cpu().numpy(), N, L)
+        s = oracle.split_variant(cnt[b].cpu().numpy(), p, passes, variant)
+        ne = p.n_edges
+        assert np.array_equal(tok[b].cpu().numpy()[:ne], s.tok), (variant, b)
+        assert np.array_equal(mass[b].cpu().numpy()[:ne], s.mass), (variant, b)
+        assert np.array_equal(loads[b].cpu().numpy().astype(np.int64), s.loads), (variant, b)
+        assert int(prun[b]) == s.passes_run, (variant, b)
+
+
+def test_split_variant_relief_equals_lb_split():
+    w = workloads.WORKLOADS["qwen3-30b"]
+    hid, W, bias, path = run_model(w, 1, T=4096)
+    out = _lib.lb_split_variant(path.cnt, path.plan, w.N, 12, "relief")
+    torch.cuda.synchronize()
+    for a, b in zip(out, (path.tok, path.mass, path.loads, path.passes_run)):
+        assert torch.equal(a, b)
