@@ -684,24 +684,34 @@ __device__ void scatter_block_tok(const Args &a, int b, int g, int i0, int i1, c
                                                   15) == 0;
     const int tb0 = i0 / k, tb1 = min(i1, nitems) / k;
     int badl = 0;
+    // The next chunk's ids are loaded one chunk ahead (registers), so no
+    // chunk waits on a global load.
+    int nx[KT];
+    auto load_ids = [&](int tt) {
+        const bool ok = tt < tb1;
+        if (ok && vec) {
+#pragma unroll
+            for (int j = 0; j < KT; j += 4) {
+                const int4 x = __ldg(reinterpret_cast<const int4 *>(ids + tt * KT + j));
+                nx[j] = x.x;
+                nx[j + 1] = x.y;
+                nx[j + 2] = x.z;
+                nx[j + 3] = x.w;
+            }
+        } else {
+#pragma unroll
+            for (int j = 0; j < KT; ++j) nx[j] = (ok && j < k) ? __ldg(ids + tt * k + j) : -1;
+        }
+    };
+    load_ids(tb0 + warp * 32 + lane);
     for (int cs = tb0; cs < tb1; cs += nw * 32) {
         for (int e = lane; e < E; e += 32) wrow[e] = 0;
         const int t = cs + warp * 32 + lane;   // this lane's token (block-local)
         const bool tv = t < tb1;
         int ev[KT];
-        if (tv && vec) {
 #pragma unroll
-            for (int j = 0; j < KT; j += 4) {
-                const int4 x = __ldg(reinterpret_cast<const int4 *>(ids + t * KT + j));
-                ev[j] = x.x;
-                ev[j + 1] = x.y;
-                ev[j + 2] = x.z;
-                ev[j + 3] = x.w;
-            }
-        } else {
-#pragma unroll
-            for (int j = 0; j < KT; ++j) ev[j] = (tv && j < k) ? __ldg(ids + t * k + j) : -1;
-        }
+        for (int j = 0; j < KT; ++j) ev[j] = nx[j];
+        load_ids(t + nw * 32);
         // ids out of range take no slot (a row repeating an id is lb_count's
         // to flag: its slots are then unspecified, every write stays in range)
 #pragma unroll
