@@ -114,17 +114,22 @@ int lb_predict_topk_chain(const void *h, const void *w, const float *bias,
                           int32_t *ids_pred, int32_t *ids_act,
                           float *logits_pred, float *logits_act, void *stream);
 
-/* Tuning knobs of lb_predict_topk (process-wide; 0 = automatic choice):
- * pipeline stages per CTA (2..8); split of H across a CTA cluster (1, 2, 4,
- * 8 or 16); persistent kernel (1, 2 or 4 = that many CTAs per SM walking the
- * tiles with a double-buffered TMEM accumulator; -1 = one CTA per tile);
- * 64-column boxes per pipeline stage of the persistent kernel (1, 2 or 4).
+/* Tuning knobs of lb_predict_topk and lb_predict_topk_chain (process-wide;
+ * 0 = automatic choice): pipeline stages per CTA (2..8, clamped to what the
+ * CTA's shared memory holds); split of H across a
+ * CTA cluster (1, 2, 4, 8 or 16); persistent kernel (1, 2 or 4 = that many
+ * CTAs per SM walking the token tiles with a TMEM accumulator, double-
+ * buffered where TMEM allows; -1 = one CTA per tile); 64-column boxes per
+ * pipeline stage of the persistent kernel (1, 2 or 4); token tiles per work
+ * unit of the persistent kernel (1 or 2: two tiles share every W box, each
+ * with its own accumulator, halving W's L2 traffic).
  * Automatic: with at least two token tiles per SM and E <= 128, persistent
- * with two CTAs per SM; otherwise one CTA per tile, H split across a cluster
- * until the GPU is filled when the tiles alone do not fill it.  Results do
- * not depend on the knobs beyond fp32 rounding of split-H partial sums.
- * LB_EINVAL for values out of range. */
-int lb_gate_tuning(int stages, int split, int persistent, int kbox);
+ * with two CTAs per SM (one when two double-buffered accumulators of the
+ * MMA's N do not fit TMEM twice) and one tile per unit; otherwise one CTA
+ * per tile, H split across a cluster until the GPU is filled when the tiles
+ * alone do not fill it.  Results do not depend on the knobs beyond fp32 rounding of
+ * split-H partial sums.  LB_EINVAL for values out of range. */
+int lb_gate_tuning(int stages, int split, int persistent, int kbox, int tiles_per_unit);
 
 /* ------------------------------------------------------------------------
  * Step 2 -- per-rank histograms   [FB sec. 3.2 eq. 5; Algorithm 1,

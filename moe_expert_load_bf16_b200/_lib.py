@@ -46,7 +46,7 @@ def _load():
     P, I, SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
     lib.lb_predict_topk.argtypes = [P, P, P, I, I, I, I, I, P, P, P]
     lib.lb_predict_topk_chain.argtypes = [P, P, P, I, I, I, I, I, P, P, P, P, P]
-    lib.lb_gate_tuning.argtypes = [I, I, I, I]
+    lib.lb_gate_tuning.argtypes = [I, I, I, I, I]
     D = ctypes.c_double
     lib.lb_swaps_capacity.argtypes = [I]
     lib.lb_plan_swaps.argtypes = [P, P, I, I, I, D, D, D, D, D, D, D, P, P, P, P, P]
@@ -222,8 +222,8 @@ def lb_split_variant(cnt, plan, N, passes=12, variant="relief", out=None):
     return tok, mass, loads, pr
 
 
-def lb_gate_tuning(stages=0, split=0, persistent=0, kbox=0):
-    _check("lb_gate_tuning", _load().lb_gate_tuning(stages, split, persistent, kbox))
+def lb_gate_tuning(stages=0, split=0, persistent=0, kbox=0, tiles_per_unit=0):
+    _check("lb_gate_tuning", _load().lb_gate_tuning(stages, split, persistent, kbox, tiles_per_unit))
 
 
 # ------------------------------------------------------------------ step 2

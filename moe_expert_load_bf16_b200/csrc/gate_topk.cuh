@@ -46,6 +46,7 @@ struct Params {
     int chain, L;
     int32_t *ids2;       // [L,T,k]
     float *logits2;      // [L,T,E] or null
+    int nbuf;            // persistent kernel: TMEM accumulator buffers (2 = double-buffered, 1)
 };
 
 template <int KMAX>
@@ -319,10 +320,13 @@ __global__ void __launch_bounds__(THREADS, 1)
 
 
 // ---------------------------------------------------------------------------
-// Persistent variant, for when the token tiles fill the GPU.  One CTA per SM
-// walks the tiles blockIdx.x, blockIdx.x + gridDim.x, ... of all problems.
-// Warp 0 (one lane) keeps the TMA ring full across tile boundaries, warp 1
-// (one lane) issues the MMAs, and warps 2..5 run the epilogue.  The TMEM
+// Persistent variant, for when the token tiles fill the GPU.  One or two CTAs
+// per SM walk the work units blockIdx.x, blockIdx.x + gridDim.x, ... of all
+// problems; a unit is MP consecutive 128-token tiles that share every W box
+// (one MMA per tile and k-block into its own accumulator), so W crosses
+// from L2 once per MP tiles.  Warp 0 (one lane) keeps the TMA ring full across tile
+// boundaries, warp 1 (one lane) issues the MMAs, and 8 or 16 warps run the
+// epilogue.  The TMEM
 // accumulator is double-buffered (2 x Epad columns), so the top-k of tile i
 // overlaps the loads and MMAs of tile i+1.  h is streamed once (L2
 // evict-first); W is re-read by every tile of its problem (L2 evict-last).
@@ -334,42 +338,50 @@ __global__ void __launch_bounds__(THREADS, 1)
 // adjacent rows of the stacked [L*E, H] weights, so one N = 2E MMA tile per
 // k-block covers both, and each hidden state crosses HBM once instead of
 // twice.
-constexpr int P_THREADS = 320;   // warp 0 TMA, warp 1 MMA, warps 2..9 epilogue (two per TMEM lane quadrant)
-constexpr int P_EPI = 256;       // epilogue threads
+// Epilogue warp sets: ES = 2 (eight epilogue warps, two per TMEM lane
+// quadrant) or ES = 4 (sixteen; used at one CTA per SM, where the registers
+// allow it and the wide tiles need the top-k throughput).
+template <int ES>
+struct Shape {
+    static constexpr int THREADS = 64 + 128 * ES;   // warp 0 TMA, warp 1 MMA, 4 * ES epilogue warps
+    static constexpr int EPI = 128 * ES;            // epilogue threads
+};
 
-// The two epilogue warps of TMEM lane quadrant q meet at named barrier 1 + q
-// (ids as immediates, so the kernel reserves barriers 0..4 only).
-template <int ID>
-__device__ __forceinline__ bool pair_all_id(bool v) {
+// The ES epilogue warps of TMEM lane quadrant q meet at named barrier 1 + q
+// (ids and thread counts as immediates, so the kernel reserves barriers 0..4).
+template <int ID, int CNT>
+__device__ __forceinline__ bool quad_all_id(bool v) {
     uint32_t r;
     asm volatile(
         "{\n\t.reg .pred pa, pb;\n\t"
         "setp.ne.u32 pa, %1, 0;\n\t"
-        "bar.red.and.pred pb, %2, 64, pa;\n\t"
+        "bar.red.and.pred pb, %2, %3, pa;\n\t"
         "selp.u32 %0, 1, 0, pb;\n\t}"
         : "=r"(r)
-        : "r"(static_cast<uint32_t>(v)), "n"(ID)
+        : "r"(static_cast<uint32_t>(v)), "n"(ID), "n"(CNT)
         : "memory");
     return r != 0;
 }
-template <int ID>
-__device__ __forceinline__ void pair_sync_id() {
-    asm volatile("bar.sync %0, 64;" ::"n"(ID) : "memory");
+template <int ID, int CNT>
+__device__ __forceinline__ void quad_sync_id() {
+    asm volatile("bar.sync %0, %1;" ::"n"(ID), "n"(CNT) : "memory");
 }
-__device__ __forceinline__ bool pair_all(int q, bool v) {
+template <int CNT>
+__device__ __forceinline__ bool quad_all(int q, bool v) {
     switch (q) {
-        case 0: return pair_all_id<1>(v);
-        case 1: return pair_all_id<2>(v);
-        case 2: return pair_all_id<3>(v);
-        default: return pair_all_id<4>(v);
+        case 0: return quad_all_id<1, CNT>(v);
+        case 1: return quad_all_id<2, CNT>(v);
+        case 2: return quad_all_id<3, CNT>(v);
+        default: return quad_all_id<4, CNT>(v);
     }
 }
-__device__ __forceinline__ void pair_sync(int q) {
+template <int CNT>
+__device__ __forceinline__ void quad_sync(int q) {
     switch (q) {
-        case 0: pair_sync_id<1>(); break;
-        case 1: pair_sync_id<2>(); break;
-        case 2: pair_sync_id<3>(); break;
-        default: pair_sync_id<4>(); break;
+        case 0: quad_sync_id<1, CNT>(); break;
+        case 1: quad_sync_id<2, CNT>(); break;
+        case 2: quad_sync_id<3, CNT>(); break;
+        default: quad_sync_id<4, CNT>(); break;
     }
 }
 
@@ -378,8 +390,39 @@ __device__ __forceinline__ bool ranks_before(float av, int ai, float bv, int bi)
     return av > bv || (av == bv && ai < bi);
 }
 
+// Merge a sorted list (v, i) with another sorted list read back from shared
+// memory (ov[j * 32], oi[j * 32] for this lane): pairwise best against the
+// reversed other list, then a half-cleaner cascade (bitonic); the result is
+// the best KMAX of both, sorted, in (v, i).
 template <int KMAX>
-__global__ void __launch_bounds__(P_THREADS, 2)
+__device__ __forceinline__ void merge_sorted(float (&v)[KMAX], int (&i)[KMAX], const float *ov, const int *oi) {
+#pragma unroll
+    for (int j = 0; j < KMAX; ++j) {
+        const float x = ov[(KMAX - 1 - j) * 32];
+        const int xi = oi[(KMAX - 1 - j) * 32];
+        const bool mine = ranks_before(v[j], i[j], x, xi);
+        v[j] = mine ? v[j] : x;
+        i[j] = mine ? i[j] : xi;
+    }
+#pragma unroll
+    for (int st = KMAX / 2; st > 0; st >>= 1) {
+#pragma unroll
+        for (int j = 0; j < KMAX; ++j) {
+            if ((j & st) == 0) {
+                const bool keep = ranks_before(v[j], i[j], v[j + st], i[j + st]);
+                const float hv = keep ? v[j] : v[j + st], lv = keep ? v[j + st] : v[j];
+                const int hi = keep ? i[j] : i[j + st], li = keep ? i[j + st] : i[j];
+                v[j] = hv;
+                i[j] = hi;
+                v[j + st] = lv;
+                i[j + st] = li;
+            }
+        }
+    }
+}
+
+template <int KMAX, int ES, int MP>
+__global__ void __launch_bounds__(Shape<ES>::THREADS, ES == 2 ? 2 : 1)
     gate_topk_persistent(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                          const Params p, int mtiles, int ntiles) {
     extern __shared__ uint8_t smem_raw[];
@@ -392,18 +435,26 @@ __global__ void __launch_bounds__(P_THREADS, 2)
     __shared__ __align__(8) uint64_t drain_bar;
     __shared__ uint32_t tmem_slot;
     __shared__ int aborted;
-    __shared__ float bias_w[8][LB_MAX_E_GATE / 2];   // each epilogue warp's copy of its columns' bias
-    __shared__ float merge_v[4][KMAX][32];            // second-half lists, handed to the first half
-    __shared__ int merge_i[4][KMAX][32];
+    // each epilogue warp's copy of its columns' bias; lists handed over for
+    // merging: per quadrant, the lists of every part but the first of each
+    // gate (chain: 2 gates x (ES/2 - 1) parts; normal: 1 gate x (ES - 1))
+    constexpr int MLISTS = ES - MP > 1 ? ES - MP : 1;
+    // (a warp ranks a whole gate only with 8 epilogue warps and two tiles per
+    // unit; every other layout splits a gate of at most 256 columns in two)
+    constexpr int BW = (ES == 2 && MP == 2) ? LB_MAX_E_GATE : LB_MAX_E_GATE / 2;
+    __shared__ float bias_w[4 * ES][BW];
+    __shared__ float merge_v[4][MLISTS][KMAX][32];
+    __shared__ int merge_i[4][MLISTS][KMAX][32];
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const uint32_t a_box = BM * 128u, b_box = static_cast<uint32_t>(p.Epad) * 128u;
     const int kbox = p.kbox;
-    const uint32_t a_bytes = a_box * kbox;              // A boxes first, then B boxes
-    const uint32_t stage_bytes = (a_box + b_box) * kbox;
+    const uint32_t a_bytes = a_box * kbox * MP;         // A boxes first (M-tile by M-tile), then B boxes
+    const uint32_t stage_bytes = (a_box * MP + b_box) * kbox;
     const int stages = p.stages;
-    const int nks = (p.nkb + kbox - 1) / kbox;          // stages per tile (boxes past H read zeros)
-    const uint32_t half = p.tmem_cols >> 1;   // column offset of accumulator buffer 1
+    const int nks = (p.nkb + kbox - 1) / kbox;          // stages per work unit (boxes past H read zeros)
+    const int nbuf = p.nbuf;
+    const uint32_t bufcols = p.tmem_cols / nbuf;        // TMEM columns of one accumulator buffer (MP tiles)
 
     if (tid == 0) {
         for (int s = 0; s < stages; ++s) {
@@ -412,7 +463,7 @@ __global__ void __launch_bounds__(P_THREADS, 2)
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&acc_full[i], 1);
-            mbar_init(&acc_empty[i], P_EPI);
+            mbar_init(&acc_empty[i], Shape<ES>::EPI);
         }
         mbar_init(&drain_bar, 1);
         aborted = 0;
@@ -437,7 +488,7 @@ __global__ void __launch_bounds__(P_THREADS, 2)
             int it = 0;
             bool ok = true;
             for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
-                const int b = tile / mtiles, m0 = (tile - b * mtiles) * BM;
+                const int b = tile / mtiles, m0 = (tile - b * mtiles) * BM * MP;
                 for (int ks = 0; ks < nks; ++ks, ++it) {
                     const int s = it % stages;
                     const uint32_t ph = (it / stages) & 1;
@@ -449,8 +500,11 @@ __global__ void __launch_bounds__(P_THREADS, 2)
                     }
                     uint8_t *sa = smem + static_cast<size_t>(s) * stage_bytes;
                     mbar_arrive_expect_tx(&full_bar[s], stage_bytes);
-                    for (int j = 0; j < kbox; ++j)
-                        tma_load_3d_hint(&tmA, sa + j * a_box, &full_bar[s], (ks * kbox + j) * BK, m0, b, pol_a);
+#pragma unroll
+                    for (int mt = 0; mt < MP; ++mt)
+                        for (int j = 0; j < kbox; ++j)
+                            tma_load_3d_hint(&tmA, sa + (mt * kbox + j) * a_box, &full_bar[s], (ks * kbox + j) * BK,
+                                             m0 + mt * BM, b, pol_a);
                     const int by = p.chain ? (b - 1) * p.E : 0, bz = p.chain ? 0 : b;
                     for (int j = 0; j < kbox; ++j)
                         tma_load_3d_hint(&tmB, sa + a_bytes + j * b_box, &full_bar[s], (ks * kbox + j) * BK, by, bz,
@@ -470,15 +524,15 @@ __global__ void __launch_bounds__(P_THREADS, 2)
             int it = 0, tl = 0;
             bool ok = true;
             for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x, ++tl) {
-                const int buf = tl & 1;
-                const uint32_t use = static_cast<uint32_t>(tl >> 1);
+                const int buf = tl % nbuf;
+                const uint32_t use = static_cast<uint32_t>(tl / nbuf);
                 if (!mbar_wait(&acc_empty[buf], (use & 1) ^ 1) || *abort_flag) {
                     atomicExch(&aborted, 1);
                     flag(LB_DEV_TIMEOUT);
                     break;
                 }
                 tc_fence_after();
-                const uint32_t d = tmem + buf * half;
+                const uint32_t d = tmem + buf * bufcols;   // M-tile mt accumulates at d + mt * Epad
                 for (int ks = 0; ks < nks; ++ks, ++it) {
                     const int s = it % stages;
                     const uint32_t ph = (it / stages) & 1;
@@ -491,11 +545,16 @@ __global__ void __launch_bounds__(P_THREADS, 2)
                     tc_fence_after();
                     const uint32_t st = smem_u32(smem + static_cast<size_t>(s) * stage_bytes);
                     for (int j = 0; j < kbox; ++j) {
-                        const uint32_t sa = st + j * a_box, sb = st + a_bytes + j * b_box;
+                        const uint32_t sb = st + a_bytes + j * b_box;
 #pragma unroll
-                        for (int kk = 0; kk < BK / UK; ++kk)
-                            umma_bf16(d, sw128_kmajor_desc(sa + kk * UK * 2), sw128_kmajor_desc(sb + kk * UK * 2),
-                                      idesc, (ks > 0 || j > 0 || kk > 0) ? 1u : 0u);
+                        for (int mt = 0; mt < MP; ++mt) {
+                            const uint32_t sa = st + (mt * kbox + j) * a_box;
+#pragma unroll
+                            for (int kk = 0; kk < BK / UK; ++kk)
+                                umma_bf16(d + mt * static_cast<uint32_t>(p.Epad), sw128_kmajor_desc(sa + kk * UK * 2),
+                                          sw128_kmajor_desc(sb + kk * UK * 2), idesc,
+                                          (ks > 0 || j > 0 || kk > 0) ? 1u : 0u);
+                        }
                     }
                     umma_commit(&empty_bar[s]);
                 }
@@ -506,41 +565,56 @@ __global__ void __launch_bounds__(P_THREADS, 2)
             if (!mbar_wait(&drain_bar, 0)) flag(LB_DEV_TIMEOUT);
         }
     } else {
-        // ---------------- epilogue: warps 2..9.  TMEM lane quadrant q =
-        // warp % 4 (rows q*32..q*32+31); set s = (warp - 2) / 4 picks the
-        // columns: in chain mode set s ranks gate s (columns [sE, sE+E)); in
-        // normal mode set s takes one half of the columns, and set 1 hands
-        // its sorted list to set 0, which merges and writes the ids.  The two
-        // warps of a quadrant take the same decisions (pair barriers), so
-        // they always meet at the same barriers.
+        // ---------------- epilogue: warps 2 .. 2 + 4 ES - 1.  TMEM lane
+        // quadrant q = warp % 4 (rows q*32..q*32+31); set s = (warp - 2) / 4
+        // picks a gate and a part of its columns: chain mode has 2 gates of
+        // ES/2 parts, normal mode 1 gate of ES parts.  Each warp ranks its
+        // part; the first part's warp of each gate merges the other parts'
+        // lists (handed over in shared memory) and writes the ids.  The ES
+        // warps of a quadrant take the same decisions (quadrant barriers),
+        // so they always meet at the same barriers.
+        constexpr int QCNT = 32 * ES;
+        constexpr int RS = ES / MP;                    // sets per M-tile of the work unit
         const int q = warp & 3;
         const int set = (warp - 2) >> 2;
+        const int mt = set % MP;                       // the M-tile this warp ranks
+        const int rr = set / MP;
+        const int GP = p.chain ? RS / 2 : RS;          // parts per gate
+        const int NG = p.chain ? 2 : 1;                // gates
+        const int gate_id = rr / GP, part = rr - gate_id * GP;
+        const int width = p.chain ? p.E : p.Epad;
+        const int pw = ((width + GP - 1) / GP + 15) / 16 * 16;
+        const int gbase = p.chain ? gate_id * p.E : 0;  // first column of this warp's gate
+        const int cbeg = gbase + part * pw;
+        const int cend = min(gbase + width, cbeg + pw);
         const int rloc = q * 32 + lane;
-        const int half_cols = (p.Epad / 2 + 15) / 16 * 16;
-        const int cbeg = p.chain ? set * p.E : set * half_cols;
-        const int cend = p.chain ? cbeg + p.E : min(p.Epad, cbeg + half_cols);
         float *wb = bias_w[warp - 2];
+        float *mv = &merge_v[q][0][0][0];
+        int *mi = &merge_i[q][0][0][0];
+        const int mbase = (mt * NG + gate_id) * (GP - 1);  // this (M-tile, gate)'s hand-over lists
+        const int mslot = mbase + part - 1;                 // this warp's list (part > 0)
         int tl = 0;
         for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++tl) {
-            const int buf = tl & 1;
-            const uint32_t use = static_cast<uint32_t>(tl >> 1);
-            const int b = tile / mtiles, m0 = (tile - b * mtiles) * BM;
+            const int buf = tl % nbuf;
+            const uint32_t use = static_cast<uint32_t>(tl / nbuf);
+            const int b = tile / mtiles, m0 = (tile - b * mtiles) * BM * MP + mt * BM;
             // The layer this warp's columns belong to (uniform over the tile).
-            const int layer = p.chain ? b - 1 + set : b;
-            const bool active = cbeg < cend && layer >= 0 && (!p.chain || layer < p.L);
+            const int layer = p.chain ? b - 1 + gate_id : b;
+            const bool live = layer >= 0 && (!p.chain || layer < p.L);   // the gate has a layer here
+            const bool active = live && cbeg < cend;
             // This tile's bias for the warp's columns into its own shared-
             // memory slice, before the wait for the accumulator: under the
             // full load of the h stream a global load takes microseconds,
             // and here its latency hides behind the tile's MMAs.  (The warp
             // finished reading the previous tile's copy in program order.)
             for (int c = cbeg + lane; c < cend; c += 32) {
-                const int cc = c - (p.chain ? set * p.E : 0);
+                const int cc = c - gbase;
                 wb[c - cbeg] = (p.bias != nullptr && active && cc < p.E) ? p.bias[static_cast<int64_t>(layer) * p.E + cc]
                                                                         : 0.f;
             }
             __syncwarp();
             bool ok = mbar_wait(&acc_full[buf], use & 1) && !*abort_flag;
-            ok = pair_all(q, ok);
+            ok = quad_all<QCNT>(q, ok);
             if (!ok) {
                 if (lane == 0) {
                     atomicExch(&aborted, 1);
@@ -551,10 +625,10 @@ __global__ void __launch_bounds__(P_THREADS, 2)
             tc_fence_after();
             const int row = m0 + rloc;
             const bool valid = row < p.T;
-            const uint32_t tl_addr = tmem + buf * half + (static_cast<uint32_t>(q * 32) << 16);
-            const int cl0 = p.chain ? set * p.E : 0;   // first column of this warp's gate
-            int32_t *ids_out = (p.chain && set == 1) ? p.ids2 : p.ids;
-            float *lg_out = (p.chain && set == 1) ? p.logits2 : p.logits;
+            const uint32_t tl_addr =
+                tmem + buf * bufcols + mt * static_cast<uint32_t>(p.Epad) + (static_cast<uint32_t>(q * 32) << 16);
+            int32_t *ids_out = (p.chain && gate_id == 1) ? p.ids2 : p.ids;
+            float *lg_out = (p.chain && gate_id == 1) ? p.logits2 : p.logits;
             const int64_t grow = static_cast<int64_t>(layer) * p.T + row;
             float *lrow = (lg_out != nullptr && valid && active) ? lg_out + grow * p.E : nullptr;
             TopK<KMAX> tk;
@@ -566,7 +640,7 @@ __global__ void __launch_bounds__(P_THREADS, 2)
                     tmem_wait_ld();
 #pragma unroll
                     for (int j = 0; j < 16; ++j) {
-                        const int c = c0 + j - cl0;   // expert id within the gate
+                        const int c = c0 + j - gbase;   // expert id within the gate
                         if (c < p.E) {
                             const float x = __uint_as_float(r[j]) + wb[c0 + j - cbeg];
                             tk.push(x, c);
@@ -578,53 +652,24 @@ __global__ void __launch_bounds__(P_THREADS, 2)
             // this warp's TMEM reads are done: the buffer may be overwritten
             tc_fence_before();
             mbar_arrive(&acc_empty[buf]);
-            if (!p.chain) {
-                // set 1 hands over its list; set 0 merges two sorted lists
-                // (bitonic: pairwise best against the reversed other list,
-                // then a half-cleaner cascade) and writes the ids
-                if (set == 1) {
+            if (GP > 1) {
+                if (part > 0) {
 #pragma unroll
                     for (int j = 0; j < KMAX; ++j) {
-                        merge_v[q][j][lane] = tk.v[j];
-                        merge_i[q][j][lane] = tk.i[j];
+                        mv[(mslot * KMAX + j) * 32 + lane] = tk.v[j];
+                        mi[(mslot * KMAX + j) * 32 + lane] = tk.i[j];
                     }
                 }
-                pair_sync(q);
-                if (set == 0) {
-                    float cv[KMAX];
-                    int ci[KMAX];
-#pragma unroll
-                    for (int j = 0; j < KMAX; ++j) {
-                        const float ov = merge_v[q][KMAX - 1 - j][lane];
-                        const int oi = merge_i[q][KMAX - 1 - j][lane];
-                        const bool mine = ranks_before(tk.v[j], tk.i[j], ov, oi);
-                        cv[j] = mine ? tk.v[j] : ov;
-                        ci[j] = mine ? tk.i[j] : oi;
-                    }
-#pragma unroll
-                    for (int st = KMAX / 2; st > 0; st >>= 1) {
-#pragma unroll
-                        for (int j = 0; j < KMAX; ++j) {
-                            if ((j & st) == 0) {
-                                const bool keep = ranks_before(cv[j], ci[j], cv[j + st], ci[j + st]);
-                                const float hv = keep ? cv[j] : cv[j + st], lv = keep ? cv[j + st] : cv[j];
-                                const int hi = keep ? ci[j] : ci[j + st], li = keep ? ci[j + st] : ci[j];
-                                cv[j] = hv;
-                                ci[j] = hi;
-                                cv[j + st] = lv;
-                                ci[j + st] = li;
-                            }
-                        }
-                    }
-                    if (valid) {
-                        int32_t *out = ids_out + grow * p.k;
-#pragma unroll
-                        for (int j = 0; j < KMAX; ++j)
-                            if (j < p.k) out[j] = ci[j];
+                quad_sync<QCNT>(q);
+                if (part == 0) {
+                    for (int o = 1; o < GP; ++o) {
+                        const int sl = mbase + o - 1;
+                        merge_sorted<KMAX>(tk.v, tk.i, mv + sl * KMAX * 32 + lane, mi + sl * KMAX * 32 + lane);
                     }
                 }
-                pair_sync(q);   // set 1 may refill merge_* only after set 0 read it
-            } else if (active && valid) {
+                quad_sync<QCNT>(q);   // the lists may be refilled only after the merges read them
+            }
+            if (part == 0 && live && valid) {
                 int32_t *out = ids_out + grow * p.k;
 #pragma unroll
                 for (int j = 0; j < KMAX; ++j)

@@ -27,6 +27,7 @@ int g_tune_stages = 0;
 int g_tune_split = 0;
 int g_tune_persistent = 0;   // 0 automatic, 1/2/4 = persistent with that many CTAs per SM, -1 never
 int g_tune_kbox = 0;         // boxes per stage of the persistent kernel (0 automatic)
+int g_tune_mp = 0;           // token tiles per work unit of the persistent kernel (0 automatic, 1 or 2)
 
 inline bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
@@ -135,22 +136,48 @@ int launch_gate(const CUtensorMap &ma, const CUtensorMap &mb, const gate::Params
     return launched("gate_topk");
 }
 
-template <int KMAX>
-int launch_gate_persistent(const CUtensorMap &ma, const CUtensorMap &mb, const gate::Params &p, int mtiles,
-                           int ntiles, int grid, size_t smem, cudaStream_t s) {
-    auto kern = gate::gate_topk_persistent<KMAX>;
+template <int KMAX, int ES, int MP>
+int launch_gate_persistent(const CUtensorMap &ma, const CUtensorMap &mb, const gate::Params &p, int units,
+                           int nunits, int grid, size_t smem, cudaStream_t s) {
+    auto kern = gate::gate_topk_persistent<KMAX, ES, MP>;
     static SmemLimit lim;
     if (!allow_smem(kern, lim, smem, false)) return LB_ECUDA;
-    kern<<<grid, gate::P_THREADS, smem, s>>>(ma, mb, p, mtiles, ntiles);
+    kern<<<grid, gate::Shape<ES>::THREADS, smem, s>>>(ma, mb, p, units, nunits);
     return launched("gate_topk_persistent");
 }
 
-int launch_gate_persistent_k(int k, const CUtensorMap &ma, const CUtensorMap &mb, const gate::Params &p,
-                             int mtiles, int ntiles, int grid, size_t smem, cudaStream_t s) {
-    if (k <= 2) return launch_gate_persistent<2>(ma, mb, p, mtiles, ntiles, grid, smem, s);
-    if (k <= 4) return launch_gate_persistent<4>(ma, mb, p, mtiles, ntiles, grid, smem, s);
-    if (k <= 8) return launch_gate_persistent<8>(ma, mb, p, mtiles, ntiles, grid, smem, s);
-    return launch_gate_persistent<16>(ma, mb, p, mtiles, ntiles, grid, smem, s);
+// (sixteen epilogue warps only for k <= 8: the hand-over lists of k <= 16
+// would not fit the static shared memory)
+template <int ES, int MP>
+int launch_gate_persistent_es(int k, const CUtensorMap &ma, const CUtensorMap &mb, const gate::Params &p,
+                              int units, int nunits, int grid, size_t smem, cudaStream_t s) {
+    if (k <= 2) return launch_gate_persistent<2, ES, MP>(ma, mb, p, units, nunits, grid, smem, s);
+    if (k <= 4) return launch_gate_persistent<4, ES, MP>(ma, mb, p, units, nunits, grid, smem, s);
+    if (k <= 8) return launch_gate_persistent<8, ES, MP>(ma, mb, p, units, nunits, grid, smem, s);
+    if constexpr (ES == 2) return launch_gate_persistent<16, 2, MP>(ma, mb, p, units, nunits, grid, smem, s);
+    return LB_EINVAL;
+}
+
+template <int KMAX, int ES, int MP>
+size_t static_smem_of() {
+    cudaFuncAttributes a{};
+    return cudaFuncGetAttributes(&a, gate::gate_topk_persistent<KMAX, ES, MP>) == cudaSuccess ? a.sharedSizeBytes
+                                                                                             : 64 * 1024;
+}
+
+// Static shared memory of the persistent kernel instance a launch will use.
+template <int ES, int MP>
+size_t persistent_static_smem(int k) {
+    if (k <= 2) return static_smem_of<2, ES, MP>();
+    if (k <= 4) return static_smem_of<4, ES, MP>();
+    if (k <= 8) return static_smem_of<8, ES, MP>();
+    if constexpr (ES == 2) return static_smem_of<16, 2, MP>();
+    return 64 * 1024;
+}
+
+size_t persistent_static_smem(int k, int es, int mp) {
+    if (es == 4) return mp == 2 ? persistent_static_smem<4, 2>(k) : persistent_static_smem<4, 1>(k);
+    return mp == 2 ? persistent_static_smem<2, 2>(k) : persistent_static_smem<2, 1>(k);
 }
 
 // Persistent gate launch shared by lb_predict_topk and lb_predict_topk_chain:
@@ -159,21 +186,54 @@ int launch_gate_persistent_k(int k, const CUtensorMap &ma, const CUtensorMap &mb
 // covers nprob problems of [T, H].
 int run_persistent(gate::Params &p, const void *h, int nprob, const CUtensorMap &mb, int per_sm, int mtiles,
                    long long ntiles, int sms, cudaStream_t s) {
+    // Work units of MP tiles sharing every W box: two when the MMA's N makes
+    // W's L2 traffic comparable to h's (N >= 128) or when asked.
+    int mp = g_tune_mp ? g_tune_mp : 1;   // measured: two tiles per unit gained nothing on the benchmark shapes
+    if (mp == 2 && mtiles < 2) mp = 1;
+    // epilogue sets: 16 warps at one CTA per SM (k <= 8), else 8; chain mode
+    // with two tiles per unit needs the 16
+    int es = (per_sm == 1 && p.k <= 8) ? 4 : 2;
+    if (p.chain && mp == 2) {
+        if (p.k > 8) mp = 1;
+        else {
+            es = 4;
+            per_sm = 1;
+        }
+    }
+    if (es == 4 && per_sm > 1) per_sm = 1;
+    // TMEM: MP accumulators of Epad columns, double-buffered when they fit
+    int nbuf = 2;
+    uint32_t need = 2u * mp * static_cast<uint32_t>(p.Epad);
+    if (need > 512u / per_sm) {
+        nbuf = 1;
+        need = static_cast<uint32_t>(mp) * static_cast<uint32_t>(p.Epad);
+    }
     uint32_t pcols = 32;
-    while (pcols < 2u * static_cast<uint32_t>(p.Epad)) pcols <<= 1;
+    while (pcols < need) pcols <<= 1;
     if (pcols > 512 || static_cast<uint32_t>(per_sm) * pcols > 512) return LB_EINVAL;
     p.tmem_cols = pcols;
+    p.nbuf = nbuf;
     p.split = 1;
-    p.kbox = g_tune_kbox ? g_tune_kbox : (p.Epad <= 64 ? 2 : 1);
-    const size_t stage_bytes = (16384 + static_cast<size_t>(p.Epad) * 128) * p.kbox;
-    int stages = g_tune_stages;
-    if (!stages)
-        stages = static_cast<int>(
-            std::max<size_t>(2, std::min<size_t>(gate::MAX_STAGES, (96 * 1024 * 2 / per_sm) / stage_bytes)));
+    // boxes per stage (measured): two for N <= 64 and for N >= 256, one between
+    p.kbox = g_tune_kbox ? g_tune_kbox : ((p.Epad <= 64 || p.Epad >= 256) ? 2 : 1);
+    const size_t stage_bytes = (16384 * static_cast<size_t>(mp) + static_cast<size_t>(p.Epad) * 128) * p.kbox;
+    const size_t stat = persistent_static_smem(p.k, es, mp);
+    const size_t room = 227 * 1024 - stat - 2048;   // dynamic shared memory the CTA can still take
+    // per CTA when per_sm CTAs share the SM's 228 KB (static memory and the
+    // 1 KB the driver reserves per CTA included)
+    const size_t share = 228 * 1024 / per_sm - stat - 3 * 1024;
+    // a requested stage count is clamped to what the CTA's shared memory holds
+    const size_t fit = std::min<size_t>(224 * 1024 - 1024, room) / stage_bytes;
+    int stages = g_tune_stages ? static_cast<int>(std::min<size_t>(g_tune_stages, fit))
+                               : static_cast<int>(std::max<size_t>(
+                                     2, std::min<size_t>(gate::MAX_STAGES,
+                                                         std::min<size_t>(std::min<size_t>(96 * 1024 * 2 / per_sm,
+                                                                                           share), room) /
+                                                             stage_bytes)));
     if (stages < 2) return LB_EINVAL;
     size_t smem = stages * stage_bytes + 1024;
     smem = std::max(smem, static_cast<size_t>(228 * 1024) / (per_sm + 1) + 1);   // at most per_sm CTAs per SM
-    if (smem > 224 * 1024) return LB_EINVAL;
+    if (smem > std::min<size_t>(224 * 1024, room + 1024)) return LB_EINVAL;
     p.stages = stages;
     CUtensorMap ma;
     if (!make_map(&ma, h, static_cast<uint64_t>(p.H), static_cast<uint64_t>(p.T), static_cast<uint64_t>(nprob),
@@ -181,8 +241,14 @@ int run_persistent(gate::Params &p, const void *h, int nprob, const CUtensorMap 
         std::snprintf(g_last_error, sizeof g_last_error, "cuTensorMapEncodeTiled failed for h");
         return LB_ECUDA;
     }
-    const int grid = static_cast<int>(std::min<long long>(ntiles, static_cast<long long>(sms) * per_sm));
-    return launch_gate_persistent_k(p.k, ma, mb, p, mtiles, static_cast<int>(ntiles), grid, smem, s);
+    const int units = (mtiles + mp - 1) / mp;
+    const long long nunits = static_cast<long long>(units) * nprob;
+    const int grid = static_cast<int>(std::min<long long>(nunits, static_cast<long long>(sms) * per_sm));
+    if (es == 4)
+        return mp == 2 ? launch_gate_persistent_es<4, 2>(p.k, ma, mb, p, units, static_cast<int>(nunits), grid, smem, s)
+                       : launch_gate_persistent_es<4, 1>(p.k, ma, mb, p, units, static_cast<int>(nunits), grid, smem, s);
+    return mp == 2 ? launch_gate_persistent_es<2, 2>(p.k, ma, mb, p, units, static_cast<int>(nunits), grid, smem, s)
+                   : launch_gate_persistent_es<2, 1>(p.k, ma, mb, p, units, static_cast<int>(nunits), grid, smem, s);
 }
 
 template <bool SPLITK>
@@ -277,7 +343,8 @@ int lb_debug_ticks(long long *out, int n) {
 }
 #endif
 
-int lb_gate_tuning(int stages, int split, int persistent, int kbox) {
+int lb_gate_tuning(int stages, int split, int persistent, int kbox, int tiles_per_unit) {
+    if (tiles_per_unit != 0 && tiles_per_unit != 1 && tiles_per_unit != 2) return LB_EINVAL;
     if (kbox != 0 && kbox != 1 && kbox != 2 && kbox != 4) return LB_EINVAL;
     if (stages != 0 && (stages < 2 || stages > gate::MAX_STAGES)) return LB_EINVAL;
     if (split != 0 && split != 1 && split != 2 && split != 4 && split != 8 && split != 16) return LB_EINVAL;
@@ -287,6 +354,7 @@ int lb_gate_tuning(int stages, int split, int persistent, int kbox) {
     g_tune_split = split;
     g_tune_persistent = persistent;
     g_tune_kbox = kbox;
+    g_tune_mp = tiles_per_unit;
     return LB_OK;
 }
 

@@ -629,3 +629,36 @@ def test_split_variant_relief_equals_lb_split():
     torch.cuda.synchronize()
     for a, b in zip(out, (path.tok, path.mass, path.loads, path.passes_run)):
         assert torch.equal(a, b)
+
+
+@pytest.mark.parametrize("chain", [False, True])
+@pytest.mark.parametrize("tpu,persistent,E", [(2, 0, 64), (2, 1, 64), (2, 2, 32), (1, 1, 64), (2, 0, 128), (2, 1, 16)])
+def test_gate_two_tiles_per_unit(chain, tpu, persistent, E):
+    """Work units of two token tiles sharing every W box (and one tile per
+    unit for contrast), with an odd tile count per problem (the last unit's
+    second tile lies past T): ids and logits pass the oracle check on sampled
+    rows of every problem, and equal the per-tile kernel's ids."""
+    if chain and E > 128:
+        pytest.skip("chain needs 2E <= 256")
+    _lib.lb_gate_tuning(0, 0, persistent, 0, tpu)
+    B, T, H, k = 3, 2900, 576, 8   # 23 tiles per problem
+    g = torch.Generator(device=DEV).manual_seed(7 + E + tpu)
+    h = torch.randn(B + (1 if chain else 0), T, H, generator=g, device=DEV).to(torch.bfloat16)
+    W = (torch.randn(B, E, H, generator=g, device=DEV) / H ** 0.5).to(torch.bfloat16)
+    bias = torch.randn(B, E, generator=g, device=DEV)
+    rng = np.random.default_rng(E)
+    rows = np.unique(np.concatenate([rng.choice(T, 48, replace=False), [0, 127, 128, 255, 256, T - 1]]))
+    if chain:
+        ip, ia, lp, la = _lib.lb_predict_topk_chain(h, W, bias, k, want_logits=True)
+        pairs = [(h[l], W[l], bias[l], ip[l], lp[l]) for l in range(B)] + \
+                [(h[l + 1], W[l], bias[l], ia[l], la[l]) for l in range(B)]
+    else:
+        ids, lg = _lib.lb_predict_topk(h, W, bias, k, want_logits=True)
+        pairs = [(h[b], W[b], bias[b], ids[b], lg[b]) for b in range(B)]
+    torch.cuda.synchronize()
+    assert _lib.lb_get_status() == 0
+    _lib.lb_gate_tuning(0, 0, -1)
+    for src, w_, b_, ids_, lg_ in pairs:
+        parity.gate_check(src, w_, b_, k, ids_, lg_, rows=rows)
+        ref = _lib.lb_predict_topk(src, w_, b_, k)
+        assert (ref == ids_).all(dim=1).float().mean().item() > 0.999
