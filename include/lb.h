@@ -71,7 +71,10 @@ enum {
  * Key Ideas, lookahead predictor]
  *   logit[b,t,e] = sum_h h[b,t,h] * w[b,e,h] + bias[b,e]   (fp32 accumulate)
  *   ids[b,t,0..k-1] = the k largest logits of row t, in descending order,
- *                     equal logits ordered by ascending expert id.
+ *                     equal logits ordered by ascending expert id.  The
+ *                     ranking compares fp32 logits with their ceil(log2 E)
+ *                     lowest bits dropped: logits closer than a relative
+ *                     2^(ceil(log2 E) - 23) order like equal ones.
  * The same call is the "normal" router when given the layer's own input.
  *   h       bf16 [nbatch, T, H] row-major, 16-byte aligned
  *   w       bf16 [nbatch, E, H] (row e = expert e's gate weights), 16-byte aligned

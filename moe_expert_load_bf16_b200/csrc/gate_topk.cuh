@@ -49,61 +49,55 @@ struct Params {
     int nbuf;            // persistent kernel: TMEM accumulator buffers (2 = double-buffered, 1)
 };
 
+// Ranking keys.  A logit x and its expert id c (c <= mask, mask = 2^ib - 1)
+// pack into one 32-bit key whose unsigned order is the ranking order: the
+// bits of x mapped to an order-preserving unsigned integer (negative values
+// complemented, the sign bit set on the others), with its ib low bits
+// replaced by mask - c.  Larger keys rank first.  Logits that agree in all
+// but their ib lowest bits (a relative difference below 2^(ib-23), far under
+// the resolution of bf16 inputs) rank by ascending id, exactly like equal
+// logits.  One key per candidate turns the sorted insertion into a chain of
+// min/max operations with no branches, whatever the lanes of a warp hold.
+__device__ __forceinline__ uint32_t id_mask(int E) {
+    return E > 1 ? 0xffffffffu >> __clz(E - 1) : 0u;
+}
+__device__ __forceinline__ uint32_t rank_key(float x, int c, uint32_t mask) {
+    const uint32_t u = __float_as_uint(x);
+    const uint32_t o = u ^ (static_cast<uint32_t>(static_cast<int32_t>(u) >> 31) | 0x80000000u);
+    return (o & ~mask) | (mask - static_cast<uint32_t>(c));
+}
+__device__ __forceinline__ int key_id(uint32_t key, uint32_t mask) {
+    return static_cast<int>(mask - (key & mask));
+}
+
 template <int KMAX>
 struct TopK {
-    float v[KMAX];
-    int i[KMAX];
+    uint32_t key[KMAX];   // descending
     __device__ __forceinline__ void init() {
 #pragma unroll
-        for (int j = 0; j < KMAX; ++j) {
-            v[j] = -INFINITY;
-            i[j] = 0x7fffffff;
-        }
+        for (int j = 0; j < KMAX; ++j) key[j] = 0u;   // below every real key
     }
-    // Candidates must arrive in ascending id order.
-    __device__ __forceinline__ void push(float x, int id) {
-        if (!(x > v[KMAX - 1])) return;
+    __device__ __forceinline__ void push(uint32_t x) {
 #pragma unroll
-        for (int j = KMAX - 1; j > 0; --j) {
-            const bool up = x > v[j - 1];          // x goes above slot j-1
-            const bool here = !up && x > v[j];     // x lands exactly in slot j
-            const float nv = up ? v[j - 1] : (here ? x : v[j]);
-            const int ni = up ? i[j - 1] : (here ? id : i[j]);
-            v[j] = nv;
-            i[j] = ni;
-        }
-        if (x > v[0]) {
-            v[0] = x;
-            i[0] = id;
+        for (int j = 0; j < KMAX; ++j) {
+            const uint32_t hi = max(key[j], x);
+            x = min(key[j], x);
+            key[j] = hi;
         }
     }
     // Merge the lists of `width` adjacent lanes (width a power of two <= 32);
-    // every lane of the group ends up with the merged list in `out`.
-    __device__ __forceinline__ void merge(int width, float (&ov)[KMAX], int (&oi)[KMAX]) {
+    // every lane of the group ends up with the merged list in `out`.  Keys
+    // of different lanes differ (their ids do), so exactly one lane pops.
+    __device__ __forceinline__ void merge(int width, uint32_t (&out)[KMAX]) {
 #pragma unroll
         for (int j = 0; j < KMAX; ++j) {
-            float hv = v[0];
-            int hi = i[0];
-            for (int off = width >> 1; off > 0; off >>= 1) {
-                const float xv = __shfl_xor_sync(kFull, hv, off);
-                const int xi = __shfl_xor_sync(kFull, hi, off);
-                if (xv > hv || (xv == hv && xi < hi)) {
-                    hv = xv;
-                    hi = xi;
-                }
-            }
-            ov[j] = hv;
-            oi[j] = hi;
-            const bool pop = (i[0] == hi);
+            uint32_t h = key[0];
+            for (int off = width >> 1; off > 0; off >>= 1) h = max(h, __shfl_xor_sync(kFull, h, off));
+            out[j] = h;
+            const bool pop = (key[0] == h);
 #pragma unroll
-            for (int q = 0; q < KMAX - 1; ++q) {
-                v[q] = pop ? v[q + 1] : v[q];
-                i[q] = pop ? i[q + 1] : i[q];
-            }
-            if (pop) {
-                v[KMAX - 1] = -INFINITY;
-                i[KMAX - 1] = 0x7fffffff;
-            }
+            for (int q = 0; q < KMAX - 1; ++q) key[q] = pop ? key[q + 1] : key[q];
+            if (pop) key[KMAX - 1] = 0u;
         }
     }
 };
@@ -222,6 +216,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     if constexpr (!SPLITK) {
         const int row = m0 + tid;
         const bool valid = ok && row < p.T;
+        const uint32_t kmask = id_mask(p.E);
         TopK<KMAX> tk;
         tk.init();
         float *lrow = (p.logits != nullptr && valid) ? p.logits + (rowbase + row) * p.E : nullptr;
@@ -233,11 +228,9 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
                 for (int q = 0; q < 16; ++q) {
                     const int c = c0 + q;
-                    if (c < p.E) {
-                        const float x = __uint_as_float(r[q]) + bias_s[c];
-                        tk.push(x, c);
-                        if (lrow) lrow[c] = x;
-                    }
+                    const float x = __uint_as_float(r[q]) + bias_s[c];
+                    tk.push(c < p.E ? rank_key(x, c, kmask) : 0u);
+                    if (lrow && c < p.E) lrow[c] = x;
                 }
             }
         }
@@ -245,7 +238,7 @@ __global__ void __launch_bounds__(THREADS, 1)
             int32_t *out = p.ids + (rowbase + row) * p.k;
 #pragma unroll
             for (int j = 0; j < KMAX; ++j)
-                if (j < p.k) out[j] = tk.i[j];
+                if (j < p.k) out[j] = key_id(tk.key[j], kmask);
         }
     } else {
         // Stage the partial tile in this CTA's shared memory (pipeline buffers
@@ -273,6 +266,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         const int trow = crank * R + rl;
         const int row = m0 + trow;
         const int C = p.Epad / S;      // columns per thread (multiple of 4)
+        const uint32_t kmask = id_mask(p.E);
         TopK<KMAX> tk;
         tk.init();
         const bool valid = row < p.T;
@@ -293,19 +287,18 @@ __global__ void __launch_bounds__(THREADS, 1)
                 const int cc = c + q;
                 if (cc < p.E) {
                     const float x = xs[q] + bias_s[cc];
-                    tk.push(x, cc);
+                    tk.push(rank_key(x, cc, kmask));
                     if (lrow) lrow[cc] = x;
                 }
             }
         }
-        float ov[KMAX];
-        int oi[KMAX];
-        tk.merge(S, ov, oi);
+        uint32_t best[KMAX];
+        tk.merge(S, best);
         if (valid && pp == 0) {
             int32_t *out = p.ids + (rowbase + row) * p.k;
 #pragma unroll
             for (int j = 0; j < KMAX; ++j)
-                if (j < p.k) out[j] = oi[j];
+                if (j < p.k) out[j] = key_id(best[j], kmask);
         }
         cluster_sync();   // keep this CTA's partials alive until all readers are done
     }
@@ -385,37 +378,22 @@ __device__ __forceinline__ void quad_sync(int q) {
     }
 }
 
-// (value desc, id asc): the order the top-k ranks by.
-__device__ __forceinline__ bool ranks_before(float av, int ai, float bv, int bi) {
-    return av > bv || (av == bv && ai < bi);
-}
-
-// Merge a sorted list (v, i) with another sorted list read back from shared
-// memory (ov[j * 32], oi[j * 32] for this lane): pairwise best against the
-// reversed other list, then a half-cleaner cascade (bitonic); the result is
-// the best KMAX of both, sorted, in (v, i).
+// Merge a sorted key list with another sorted list read back from shared
+// memory (ok[j * 32] for this lane): pairwise best against the reversed
+// other list, then a half-cleaner cascade (bitonic); the result is the best
+// KMAX of both, sorted.
 template <int KMAX>
-__device__ __forceinline__ void merge_sorted(float (&v)[KMAX], int (&i)[KMAX], const float *ov, const int *oi) {
+__device__ __forceinline__ void merge_sorted(uint32_t (&key)[KMAX], const uint32_t *ok) {
 #pragma unroll
-    for (int j = 0; j < KMAX; ++j) {
-        const float x = ov[(KMAX - 1 - j) * 32];
-        const int xi = oi[(KMAX - 1 - j) * 32];
-        const bool mine = ranks_before(v[j], i[j], x, xi);
-        v[j] = mine ? v[j] : x;
-        i[j] = mine ? i[j] : xi;
-    }
+    for (int j = 0; j < KMAX; ++j) key[j] = max(key[j], ok[(KMAX - 1 - j) * 32]);
 #pragma unroll
     for (int st = KMAX / 2; st > 0; st >>= 1) {
 #pragma unroll
         for (int j = 0; j < KMAX; ++j) {
             if ((j & st) == 0) {
-                const bool keep = ranks_before(v[j], i[j], v[j + st], i[j + st]);
-                const float hv = keep ? v[j] : v[j + st], lv = keep ? v[j + st] : v[j];
-                const int hi = keep ? i[j] : i[j + st], li = keep ? i[j + st] : i[j];
-                v[j] = hv;
-                i[j] = hi;
-                v[j + st] = lv;
-                i[j + st] = li;
+                const uint32_t hi = max(key[j], key[j + st]), lo = min(key[j], key[j + st]);
+                key[j] = hi;
+                key[j + st] = lo;
             }
         }
     }
@@ -442,9 +420,8 @@ __global__ void __launch_bounds__(Shape<ES>::THREADS, ES == 2 ? 2 : 1)
     // (a warp ranks a whole gate only with 8 epilogue warps and two tiles per
     // unit; every other layout splits a gate of at most 256 columns in two)
     constexpr int BW = (ES == 2 && MP == 2) ? LB_MAX_E_GATE : LB_MAX_E_GATE / 2;
-    __shared__ float bias_w[4 * ES][BW];
-    __shared__ float merge_v[4][MLISTS][KMAX][32];
-    __shared__ int merge_i[4][MLISTS][KMAX][32];
+    __shared__ __align__(16) float bias_w[4 * ES][BW];
+    __shared__ uint32_t merge_k[4][MLISTS][KMAX][32];
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const uint32_t a_box = BM * 128u, b_box = static_cast<uint32_t>(p.Epad) * 128u;
@@ -589,8 +566,8 @@ __global__ void __launch_bounds__(Shape<ES>::THREADS, ES == 2 ? 2 : 1)
         const int cend = min(gbase + width, cbeg + pw);
         const int rloc = q * 32 + lane;
         float *wb = bias_w[warp - 2];
-        float *mv = &merge_v[q][0][0][0];
-        int *mi = &merge_i[q][0][0][0];
+        uint32_t *mk = &merge_k[q][0][0][0];
+        const uint32_t kmask = id_mask(p.E);
         const int mbase = (mt * NG + gate_id) * (GP - 1);  // this (M-tile, gate)'s hand-over lists
         const int mslot = mbase + part - 1;                 // this warp's list (part > 0)
         int tl = 0;
@@ -634,17 +611,29 @@ __global__ void __launch_bounds__(Shape<ES>::THREADS, ES == 2 ? 2 : 1)
             TopK<KMAX> tk;
             tk.init();
             if (active) {
-                for (int c0 = cbeg; c0 < cend; c0 += 16) {
-                    uint32_t r[16];
-                    tmem_ld16(tl_addr + c0, r);
+                // 32 columns per TMEM load and wait (16 for a part's last
+                // odd block); the bias as 16-byte shared-memory reads
+                for (int c0 = cbeg; c0 < cend; c0 += 32) {
+                    uint32_t r[32];
+                    const bool full = c0 + 32 <= cend;   // warp-uniform
+                    if (full)
+                        tmem_ld32(tl_addr + c0, r);
+                    else
+                        tmem_ld16(tl_addr + c0, *reinterpret_cast<uint32_t(*)[16]>(r));
                     tmem_wait_ld();
+                    const float4 *b4 = reinterpret_cast<const float4 *>(wb + (c0 - cbeg));
 #pragma unroll
-                    for (int j = 0; j < 16; ++j) {
-                        const int c = c0 + j - gbase;   // expert id within the gate
-                        if (c < p.E) {
-                            const float x = __uint_as_float(r[j]) + wb[c0 + j - cbeg];
-                            tk.push(x, c);
-                            if (lrow) lrow[c] = x;
+                    for (int j4 = 0; j4 < 8; ++j4) {
+                        if (j4 < 4 || full) {
+                            const float4 bb = b4[j4];
+                            const float bj[4] = {bb.x, bb.y, bb.z, bb.w};
+#pragma unroll
+                            for (int u = 0; u < 4; ++u) {
+                                const int c = c0 + 4 * j4 + u - gbase;   // expert id within the gate
+                                const float x = __uint_as_float(r[4 * j4 + u]) + bj[u];
+                                tk.push(c < p.E ? rank_key(x, c, kmask) : 0u);
+                                if (lrow && c < p.E) lrow[c] = x;
+                            }
                         }
                     }
                 }
@@ -656,15 +645,14 @@ __global__ void __launch_bounds__(Shape<ES>::THREADS, ES == 2 ? 2 : 1)
                 if (part > 0) {
 #pragma unroll
                     for (int j = 0; j < KMAX; ++j) {
-                        mv[(mslot * KMAX + j) * 32 + lane] = tk.v[j];
-                        mi[(mslot * KMAX + j) * 32 + lane] = tk.i[j];
+                        mk[(mslot * KMAX + j) * 32 + lane] = tk.key[j];
                     }
                 }
                 quad_sync<QCNT>(q);
                 if (part == 0) {
                     for (int o = 1; o < GP; ++o) {
                         const int sl = mbase + o - 1;
-                        merge_sorted<KMAX>(tk.v, tk.i, mv + sl * KMAX * 32 + lane, mi + sl * KMAX * 32 + lane);
+                        merge_sorted<KMAX>(tk.key, mk + sl * KMAX * 32 + lane);
                     }
                 }
                 quad_sync<QCNT>(q);   // the lists may be refilled only after the merges read them
@@ -673,7 +661,7 @@ __global__ void __launch_bounds__(Shape<ES>::THREADS, ES == 2 ? 2 : 1)
                 int32_t *out = ids_out + grow * p.k;
 #pragma unroll
                 for (int j = 0; j < KMAX; ++j)
-                    if (j < p.k) out[j] = tk.i[j];
+                    if (j < p.k) out[j] = key_id(tk.key[j], kmask);
             }
         }
     }

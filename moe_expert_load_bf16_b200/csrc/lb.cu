@@ -215,10 +215,14 @@ int run_persistent(gate::Params &p, const void *h, int nprob, const CUtensorMap 
     p.nbuf = nbuf;
     p.split = 1;
     // boxes per stage (measured): two for N <= 64 and for N >= 256, one between
-    p.kbox = g_tune_kbox ? g_tune_kbox : ((p.Epad <= 64 || p.Epad >= 256) ? 2 : 1);
-    const size_t stage_bytes = (16384 * static_cast<size_t>(mp) + static_cast<size_t>(p.Epad) * 128) * p.kbox;
     const size_t stat = persistent_static_smem(p.k, es, mp);
     const size_t room = 227 * 1024 - stat - 2048;   // dynamic shared memory the CTA can still take
+    const size_t box_bytes = 16384 * static_cast<size_t>(mp) + static_cast<size_t>(p.Epad) * 128;
+    p.kbox = g_tune_kbox ? g_tune_kbox : ((p.Epad <= 64 || p.Epad >= 256) ? 2 : 1);
+    // (automatic choice: back to one box per stage when two stages of two
+    // boxes would not fit, e.g. two tiles per unit at N = 256)
+    if (!g_tune_kbox && p.kbox == 2 && 4 * box_bytes + 1024 > std::min<size_t>(224 * 1024, room + 1024)) p.kbox = 1;
+    const size_t stage_bytes = box_bytes * p.kbox;
     // per CTA when per_sm CTAs share the SM's 228 KB (static memory and the
     // 1 KB the driver reserves per CTA included)
     const size_t share = 228 * 1024 / per_sm - stat - 3 * 1024;
