@@ -167,7 +167,7 @@ def whole_job_rate(units_per_step_per_rank, world, ms_per_step):
 # ----------------------------------------------------------------------------- GPU arm
 def run_ours(args, world, rank, local):
     from moe_expert_load_bf16_b200 import _lib, build, workloads
-    from moe_expert_load_bf16_b200.pipeline import DecisionPath
+    from moe_expert_load_bf16_b200.pipeline import DecisionPath, StepPipeline
 
     build.build()
     wl = rank_workload(workloads.WORKLOADS[args.config], rank)
@@ -181,9 +181,14 @@ def run_ours(args, world, rank, local):
     hid[0].copy_(hid[1])
     W = workloads.gate_weights(wl, Lyr, device=dev)
     bias = workloads.biases(wl, Lyr).to(dev)
-    path = DecisionPath(Lyr, T, H, E, k, G, N, L, device=dev)
-    side = torch.cuda.Stream(device=dev)
     chain = args.gate == "chain"
+    pipe = StepPipeline(Lyr, T, H, E, k, G, N, L, device=dev) if chain and args.in_flight == 2 else None
+    if pipe:
+        # integer blocks of at most 512 threads, so that one fits beside a
+        # gate CTA on an SM the gate's grid leaves half free
+        _lib.lb_launch_options(1, 512)
+    path = pipe.paths[0] if pipe else DecisionPath(Lyr, T, H, E, k, G, N, L, device=dev)
+    side = torch.cuda.Stream(device=dev)
 
     def step():
         if chain:
@@ -193,37 +198,61 @@ def run_ours(args, world, rank, local):
     launches = path.LAUNCHES_PER_CHAIN if chain else path.LAUNCHES_PER_RUN
 
     # warm-up (also loads the library, sets kernel attributes, builds maps)
-    for _ in range(args.warmup):
-        step()
+    if pipe:
+        pipe.run(args.warmup, hid, W, bias)
+    else:
+        for _ in range(args.warmup):
+            step()
     torch.cuda.synchronize()
     if _lib.lb_get_status():
         raise RuntimeError("device status flagged during warm-up")
 
+    # one step alone (its latency), and the K timed steps: one step per
+    # graph replay, or with two steps in flight the K steps as one graph
     g_step = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g_step):
         step()
     g_step.replay()
+    if pipe:
+        g_steps = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g_steps):
+            pipe.run(args.steps, hid, W, bias)
+        g_steps.replay()
     torch.cuda.synchronize()
 
-    # ---------------- timed region: K graph replays
+    # ---------------- timed region: K steps
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(local) as clk:
         barrier(world)
         torch.cuda.synchronize()
         ev0.record(stream)
-        for _ in range(args.steps):
-            g_step.replay()
+        if pipe:
+            g_steps.replay()
+        else:
+            for _ in range(args.steps):
+                g_step.replay()
         ev1.record(stream)
         torch.cuda.synchronize()
         barrier(world)
     ms_total = max_over_ranks(ev0.elapsed_time(ev1), world)
     ms_step = ms_total / args.steps
+    if pipe:
+        del g_steps
     assign_per_step = Lyr * T * k
     value = whole_job_rate(assign_per_step, world, ms_step)
     if args.lean:
         return {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
                 "warmup": args.warmup, "ms_per_step": ms_step, "lean": True,
                 "gpu_launches": launches * args.steps, "clocks": clk.summary()}
+
+    # ---------------- one step alone: its latency (graph replays, one at a time)
+    barrier(world)
+    ev0.record(stream)
+    for _ in range(args.steps):
+        g_step.replay()
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    step_latency_us = max_over_ranks(ev0.elapsed_time(ev1), world) / args.steps * 1e3
 
     # ---------------- dominant kernel: the gate (one chain launch per step,
     # or two launches in the two-pass form)
@@ -282,12 +311,18 @@ def run_ours(args, world, rank, local):
                                f"G={G} ranks, N={N} replica slots (L={L})",
                    "layers": Lyr, "T": T, "H": H, "E": E, "k": k, "G": G, "N": N, "L": L, "passes": 12,
                    "batching": "all layers of a step in one launch per kernel, CUDA-graph replay",
+                   "steps_in_flight": (2 if pipe else 1),
+                   "integer_block_threads_max": (512 if pipe else 1024),
+                   "overlap": ("two steps in flight: the gate of step i+1 on one stream beside the integer "
+                               "stages of step i on a second, higher-priority stream (two buffer sets); "
+                               "the K timed steps are one CUDA graph" if pipe else "none: one step after another"),
                    "gate": ("chain: one pass per hidden state evaluates the normal router of the layer before "
                             "it and the lookahead of the layer after it" if chain else
                             "two passes (lookahead, normal router); lookahead counts + plan on a second stream"),
                    "l2": "inputs larger than L2 (hidden states %.0f MB read per step)" % (
                        (Lyr + 1 if chain else 2 * Lyr) * T * H * 2 / 1e6),
                    "parallelism": f"{world} independent replicas"},
+        "step_latency_us": step_latency_us,
         "t_solve_us": lat["solve"], "t_solve_fused_us": lat["solve_fused"], "t_split_us": lat["split"],
         "t_lookahead_us": lat["lookahead"],
         "per_kernel_us": lat["kernels"],
@@ -679,6 +714,9 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--config", default=DEFAULT_WORKLOAD)
     ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--in-flight", type=int, choices=(1, 2), default=2,
+                    help="steps in flight in the chain form (2: the gate of one step beside the integer "
+                         "stages of the previous one, on two streams)")
     ap.add_argument("--gate", choices=("chain", "two-pass"), default="chain",
                     help="chain: one gate pass per hidden state for both gates that read it; two-pass: "
                          "lookahead and normal router as separate passes")

@@ -125,14 +125,33 @@ int lb_predict_topk_chain(const void *h, const void *w, const float *bias,
  * buffered where TMEM allows; -1 = one CTA per tile); 64-column boxes per
  * pipeline stage of the persistent kernel (1, 2 or 4); token tiles per work
  * unit of the persistent kernel (1 or 2: two tiles share every W box, each
- * with its own accumulator, halving W's L2 traffic).
+ * with its own accumulator, halving W's L2 traffic); at most max_ctas CTAs
+ * in the persistent kernel's grid (0 = its CTAs per SM on every SM; fewer
+ * leave SMs to kernels that run beside it on other streams).
  * Automatic: with at least two token tiles per SM and E <= 128, persistent
  * with two CTAs per SM (one when two double-buffered accumulators of the
  * MMA's N do not fit TMEM twice) and one tile per unit; otherwise one CTA
  * per tile, H split across a cluster until the GPU is filled when the tiles
  * alone do not fill it.  Results do not depend on the knobs beyond fp32 rounding of
  * split-H partial sums.  LB_EINVAL for values out of range. */
-int lb_gate_tuning(int stages, int split, int persistent, int kbox, int tiles_per_unit);
+int lb_gate_tuning(int stages, int split, int persistent, int kbox, int tiles_per_unit,
+                   int max_ctas);
+
+/* Launch options (process-wide; results are identical under every option).
+ * programmatic_dependent_launch = 1 (the default): every kernel without a
+ * thread-block cluster is launched with programmatic stream serialization,
+ * so its launch is processed while the previous kernel on the stream runs;
+ * each kernel waits for its predecessor's completion (and the visibility of
+ * its writes) before it touches global memory.  0 = plain stream order.
+ * max_block_threads (0 = 1024, or 256, 512, 1024): the largest thread block
+ * the integer kernels use (lb_assign's prep and scatter take up to 1024
+ * threads; count, plan and split 512).  512 lets a block of every integer
+ * kernel share an SM with one CTA of the persistent gate, so that the
+ * integer stages of one batch can run on a second stream beside the gate
+ * of the next (with lb_gate_tuning's max_ctas leaving one gate CTA on some
+ * SMs).  lb_solve's cluster launch is not affected.  LB_EINVAL for other
+ * values. */
+int lb_launch_options(int programmatic_dependent_launch, int max_block_threads);
 
 /* ------------------------------------------------------------------------
  * Step 2 -- per-rank histograms   [FB sec. 3.2 eq. 5; Algorithm 1,

@@ -46,7 +46,8 @@ def _load():
     P, I, SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
     lib.lb_predict_topk.argtypes = [P, P, P, I, I, I, I, I, P, P, P]
     lib.lb_predict_topk_chain.argtypes = [P, P, P, I, I, I, I, I, P, P, P, P, P]
-    lib.lb_gate_tuning.argtypes = [I, I, I, I, I]
+    lib.lb_gate_tuning.argtypes = [I, I, I, I, I, I]
+    lib.lb_launch_options.argtypes = [I, I]
     D = ctypes.c_double
     lib.lb_swaps_capacity.argtypes = [I]
     lib.lb_plan_swaps.argtypes = [P, P, I, I, I, D, D, D, D, D, D, D, P, P, P, P, P]
@@ -68,7 +69,7 @@ def _load():
     lib.lb_last_error.argtypes = []
     lib.lb_last_error.restype = ctypes.c_char_p
     for f in ("lb_predict_topk", "lb_predict_topk_chain", "lb_plan_swaps", "lb_swaps_capacity", "lb_split_variant",
-              "lb_gate_tuning",
+              "lb_gate_tuning", "lb_launch_options",
               "lb_count", "lb_plan_layout_of", "lb_plan_replicas",
               "lb_split", "lb_assign", "lb_assign_noalloc", "lb_solve", "lb_get_status", "lb_version"):
         getattr(lib, f).restype = ctypes.c_int
@@ -222,8 +223,12 @@ def lb_split_variant(cnt, plan, N, passes=12, variant="relief", out=None):
     return tok, mass, loads, pr
 
 
-def lb_gate_tuning(stages=0, split=0, persistent=0, kbox=0, tiles_per_unit=0):
-    _check("lb_gate_tuning", _load().lb_gate_tuning(stages, split, persistent, kbox, tiles_per_unit))
+def lb_gate_tuning(stages=0, split=0, persistent=0, kbox=0, tiles_per_unit=0, max_ctas=0):
+    _check("lb_gate_tuning", _load().lb_gate_tuning(stages, split, persistent, kbox, tiles_per_unit, max_ctas))
+
+
+def lb_launch_options(programmatic_dependent_launch=1, max_block_threads=0):
+    _check("lb_launch_options", _load().lb_launch_options(int(programmatic_dependent_launch), int(max_block_threads)))
 
 
 # ------------------------------------------------------------------ step 2
@@ -393,7 +398,7 @@ def lb_version():
     return int(_load().lb_version())
 
 
-EXPORTS = ("lb_predict_topk", "lb_predict_topk_chain", "lb_gate_tuning", "lb_plan_swaps", "lb_swaps_capacity",
+EXPORTS = ("lb_predict_topk", "lb_predict_topk_chain", "lb_gate_tuning", "lb_launch_options", "lb_plan_swaps", "lb_swaps_capacity",
            "lb_split_variant", "lb_count", "lb_plan_bytes", "lb_plan_layout_of",
            "lb_plan_replicas", "lb_split", "lb_assign_workspace_bytes", "lb_assign", "lb_assign_noalloc", "lb_solve",
            "lb_get_status",

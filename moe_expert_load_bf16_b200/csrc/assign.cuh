@@ -276,6 +276,7 @@ __device__ void prep_problem(const Args &a, int b, uint8_t *sm) {
 
 __global__ void __launch_bounds__(PREP_THREADS) prep_kernel(const Args a) {
     extern __shared__ __align__(16) uint8_t sm[];
+    pdl_begin();
     prep_problem(a, blockIdx.x, sm);
 }
 
@@ -877,6 +878,7 @@ __device__ inline void scatter_block_cta_any(const Args &a, int b, int g, int i0
 // takes block x.
 __global__ void __launch_bounds__(SC_THREADS) scatter_kernel(const Args a) {
     extern __shared__ __align__(16) uint8_t sm[];
+    pdl_begin();
     __shared__ int bad;
     if (threadIdx.x == 0) bad = 0;
     const int nw = blockDim.x >> 5;

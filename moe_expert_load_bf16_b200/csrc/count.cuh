@@ -37,6 +37,7 @@ __global__ void __launch_bounds__(THREADS)
     count_kernel(const int32_t *__restrict__ ids, int T, int k, int E, int G,
                  int32_t *__restrict__ cnt) {
     extern __shared__ int hist[];
+    pdl_begin();
     __shared__ int bad;
     const int g = blockIdx.x, b = blockIdx.y;
     for (int e = threadIdx.x; e < E; e += blockDim.x) hist[e] = 0;

@@ -107,6 +107,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     gate_topk_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                      const Params p) {
     extern __shared__ uint8_t smem_raw[];
+    pdl_begin();
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                 ~static_cast<uintptr_t>(1023));
     __shared__ __align__(8) uint64_t full_bar[MAX_STAGES];
@@ -404,6 +405,7 @@ __global__ void __launch_bounds__(Shape<ES>::THREADS, ES == 2 ? 2 : 1)
     gate_topk_persistent(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                          const Params p, int mtiles, int ntiles) {
     extern __shared__ uint8_t smem_raw[];
+    pdl_begin();
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                 ~static_cast<uintptr_t>(1023));
     __shared__ __align__(8) uint64_t full_bar[MAX_STAGES];

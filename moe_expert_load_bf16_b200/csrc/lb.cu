@@ -28,6 +28,7 @@ int g_tune_split = 0;
 int g_tune_persistent = 0;   // 0 automatic, 1/2/4 = persistent with that many CTAs per SM, -1 never
 int g_tune_kbox = 0;         // boxes per stage of the persistent kernel (0 automatic)
 int g_tune_mp = 0;           // token tiles per work unit of the persistent kernel (0 automatic, 1 or 2)
+int g_tune_max_ctas = 0;     // cap on the persistent kernel's grid (0: every SM's share)
 
 inline bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
@@ -43,6 +44,33 @@ inline int cuda_fail(cudaError_t e, const char *where) {
 inline int launched(const char *where = "launch") {
     const cudaError_t e = cudaGetLastError();
     return e == cudaSuccess ? LB_OK : cuda_fail(e, where);
+}
+
+// Launch options (lb_launch_options): programmatic dependent launch, on by
+// default; the largest block of the integer kernels (prep and scatter pick
+// up to 1024 threads).
+int g_pdl = 1;
+int g_max_threads = 1024;
+
+// Launch of a kernel without clusters, with programmatic stream
+// serialization when enabled: the kernel may be scheduled while the previous
+// kernel on the stream is still running, and waits for it in pdl_begin().
+template <typename... KArgs, typename... Args>
+int launch_kernel(const char *where, void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                  Args &&...args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = g_pdl ? 1 : 0;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+    if (e != cudaSuccess) return cuda_fail(e, where);
+    return launched(where);
 }
 
 int device_sms() {
@@ -128,9 +156,13 @@ int launch_gate(const CUtensorMap &ma, const CUtensorMap &mb, const gate::Params
         attr[0].val.clusterDim.x = p.split;
         attr[0].val.clusterDim.y = 1;
         attr[0].val.clusterDim.z = 1;
-        cfg.attrs = attr;
-        cfg.numAttrs = 1;
+    } else {
+        // (programmatic dependent launch only for launches without clusters)
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = g_pdl ? 1 : 0;
     }
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
     const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, ma, mb, p);
     if (e != cudaSuccess) return cuda_fail(e, "cudaLaunchKernelEx(gate_topk)");
     return launched("gate_topk");
@@ -142,8 +174,8 @@ int launch_gate_persistent(const CUtensorMap &ma, const CUtensorMap &mb, const g
     auto kern = gate::gate_topk_persistent<KMAX, ES, MP>;
     static SmemLimit lim;
     if (!allow_smem(kern, lim, smem, false)) return LB_ECUDA;
-    kern<<<grid, gate::Shape<ES>::THREADS, smem, s>>>(ma, mb, p, units, nunits);
-    return launched("gate_topk_persistent");
+    return launch_kernel("gate_topk_persistent", kern, dim3(grid), dim3(gate::Shape<ES>::THREADS), smem, s, ma, mb, p,
+                         units, nunits);
 }
 
 // (sixteen epilogue warps only for k <= 8: the hand-over lists of k <= 16
@@ -247,7 +279,14 @@ int run_persistent(gate::Params &p, const void *h, int nprob, const CUtensorMap 
     }
     const int units = (mtiles + mp - 1) / mp;
     const long long nunits = static_cast<long long>(units) * nprob;
-    const int grid = static_cast<int>(std::min<long long>(nunits, static_cast<long long>(sms) * per_sm));
+    long long cap = static_cast<long long>(sms) * per_sm;
+    if (g_tune_max_ctas > 0) cap = std::min<long long>(cap, g_tune_max_ctas);
+    if (nunits < 1 || cap < 1) return LB_EINVAL;
+    // the fewest CTAs that take the units in the same number of rounds: no
+    // CTA does more units than with the full grid, and the slots left over
+    // stay free for kernels on other streams
+    const long long rounds = (nunits + cap - 1) / cap;
+    const int grid = static_cast<int>((nunits + rounds - 1) / rounds);
     if (es == 4)
         return mp == 2 ? launch_gate_persistent_es<4, 2>(p.k, ma, mb, p, units, static_cast<int>(nunits), grid, smem, s)
                        : launch_gate_persistent_es<4, 1>(p.k, ma, mb, p, units, static_cast<int>(nunits), grid, smem, s);
@@ -266,8 +305,8 @@ int launch_gate_k(int k, const CUtensorMap &ma, const CUtensorMap &mb, const gat
 
 template <int K, bool VEC>
 int launch_count(const int32_t *ids, int nbatch, int T, int k, int E, int G, int32_t *cnt, cudaStream_t s) {
-    count::count_kernel<K, VEC><<<dim3(G, nbatch), count::THREADS, E * sizeof(int), s>>>(ids, T, k, E, G, cnt);
-    return launched("count");
+    return launch_kernel("count", count::count_kernel<K, VEC>, dim3(G, nbatch), dim3(count::THREADS),
+                         E * sizeof(int), s, ids, T, k, E, G, cnt);
 }
 
 template <int K>
@@ -290,6 +329,7 @@ int scatter_grid_x(int T, int k, int G, int nw = assign::SC_WARPS) {
 int scatter_warps(int nbatch, int T, int k, int G, int E, int N) {
     const long long ctas = static_cast<long long>(scatter_grid_x(T, k, G, 16)) * nbatch;
     int nw = ctas >= 2LL * device_sms() ? 16 : assign::SC_WARPS;
+    nw = std::min(nw, g_max_threads / 32);
     while (nw > 8 && assign::scatter_smem_bytes(G, E, N, nw) > 224 * 1024) nw >>= 1;
     return nw;
 }
@@ -347,8 +387,18 @@ int lb_debug_ticks(long long *out, int n) {
 }
 #endif
 
-int lb_gate_tuning(int stages, int split, int persistent, int kbox, int tiles_per_unit) {
+int lb_launch_options(int programmatic_dependent_launch, int max_block_threads) {
+    if (programmatic_dependent_launch != 0 && programmatic_dependent_launch != 1) return LB_EINVAL;
+    if (max_block_threads != 0 && max_block_threads != 256 && max_block_threads != 512 && max_block_threads != 1024)
+        return LB_EINVAL;
+    g_pdl = programmatic_dependent_launch;
+    g_max_threads = max_block_threads ? max_block_threads : 1024;
+    return LB_OK;
+}
+
+int lb_gate_tuning(int stages, int split, int persistent, int kbox, int tiles_per_unit, int max_ctas) {
     if (tiles_per_unit != 0 && tiles_per_unit != 1 && tiles_per_unit != 2) return LB_EINVAL;
+    if (max_ctas < 0) return LB_EINVAL;
     if (kbox != 0 && kbox != 1 && kbox != 2 && kbox != 4) return LB_EINVAL;
     if (stages != 0 && (stages < 2 || stages > gate::MAX_STAGES)) return LB_EINVAL;
     if (split != 0 && split != 1 && split != 2 && split != 4 && split != 8 && split != 16) return LB_EINVAL;
@@ -359,6 +409,7 @@ int lb_gate_tuning(int stages, int split, int persistent, int kbox, int tiles_pe
     g_tune_persistent = persistent;
     g_tune_kbox = kbox;
     g_tune_mp = tiles_per_unit;
+    g_tune_max_ctas = max_ctas;
     return LB_OK;
 }
 
@@ -545,8 +596,8 @@ int lb_plan_swaps(const int32_t *cnt, const int32_t *placement, int nbatch, int 
     p.max_swaps = lb_swaps_capacity(E);
     static SmemLimit lim;
     if (!allow_smem(swaps::swaps_kernel, lim, smem, false)) return LB_ECUDA;
-    swaps::swaps_kernel<<<nbatch, swaps::THREADS, smem, static_cast<cudaStream_t>(stream)>>>(p);
-    return launched("plan swaps");
+    return launch_kernel("plan swaps", swaps::swaps_kernel, dim3(nbatch), dim3(swaps::THREADS), smem,
+                         static_cast<cudaStream_t>(stream), p);
 }
 
 int lb_split_variant(const int32_t *cnt, const void *plan, int nbatch, int G, int E, int N, int passes, int variant,
@@ -575,8 +626,8 @@ int lb_split_variant(const int32_t *cnt, const void *plan, int nbatch, int G, in
     p.passes_run = passes_run;
     static SmemLimit lim;
     if (!allow_smem(splitv::split_variant_kernel, lim, smem, false)) return LB_ECUDA;
-    splitv::split_variant_kernel<<<nbatch, splitv::THREADS, smem, static_cast<cudaStream_t>(stream)>>>(p);
-    return launched("split variant");
+    return launch_kernel("split variant", splitv::split_variant_kernel, dim3(nbatch), dim3(splitv::THREADS), smem,
+                         static_cast<cudaStream_t>(stream), p);
 }
 
 int lb_count(const int32_t *ids, int nbatch, int T, int k, int E, int G, int32_t *cnt, void *stream) {
@@ -627,9 +678,8 @@ int lb_plan_replicas(const int32_t *cnt, int nbatch, int G, int E, int N, int L,
     if (smem > 224 * 1024) return LB_EINVAL;
     static SmemLimit lim;
     if (!allow_smem(plan::plan_kernel, lim, smem, false)) return LB_ECUDA;
-    plan::plan_kernel<<<nbatch, plan::THREADS, smem, s>>>(cnt, G, E, N, L, static_cast<uint8_t *>(plan),
-                                                            plan::layout(G, E, N).total);
-    return launched("plan");
+    return launch_kernel("plan", plan::plan_kernel, dim3(nbatch), dim3(plan::THREADS), smem, s, cnt, G, E, N, L,
+                         static_cast<uint8_t *>(plan), plan::layout(G, E, N).total);
 }
 
 int lb_split(const int32_t *cnt, const void *plan, int nbatch, int G, int E, int N, int passes, int32_t *tok,
@@ -641,10 +691,9 @@ int lb_split(const int32_t *cnt, const void *plan, int nbatch, int G, int E, int
     const size_t smem = split::smem_bytes(G, E, N);
     static SmemLimit lim;
     if (!allow_smem(split::split_kernel, lim, smem, false)) return LB_ECUDA;
-    split::split_kernel<<<nbatch, split::THREADS, smem, s>>>(cnt, static_cast<const uint8_t *>(plan),
-                                                              plan::layout(G, E, N).total, G, E, N, passes, tok,
-                                                              mass, loads, passes_run);
-    return launched("split");
+    return launch_kernel("split", split::split_kernel, dim3(nbatch), dim3(split::THREADS), smem, s, cnt,
+                         static_cast<const uint8_t *>(plan), plan::layout(G, E, N).total, G, E, N, passes, tok, mass,
+                         loads, passes_run);
 }
 
 size_t lb_assign_workspace_bytes(int nbatch, int T, int k, int G, int E, int N) {
@@ -689,12 +738,12 @@ int lb_assign(const int32_t *ids, const int32_t *cnt, const void *plan, const in
     static SmemLimit lim1, lim2;
     if (!allow_smem(assign::prep_kernel, lim1, sm1, false) || !allow_smem(assign::scatter_kernel, lim2, sm2, false))
         return LB_ECUDA;
-    assign::prep_kernel<<<nbatch, assign::PREP_THREADS, sm1, s>>>(a);
-    if (launched("assign prep") != LB_OK) return LB_ECUDA;
+    if (launch_kernel("assign prep", assign::prep_kernel, dim3(nbatch), dim3(std::min(assign::PREP_THREADS, g_max_threads)),
+                      sm1, s, a) != LB_OK)
+        return LB_ECUDA;
     if (T == 0) return LB_OK;
-    assign::scatter_kernel<<<dim3(scatter_grid_x(T, k, G, nw), nbatch), nw * 32,
-                             assign::scatter_smem_bytes(G, E, N, nw), s>>>(a);
-    return launched("assign scatter");
+    return launch_kernel("assign scatter", assign::scatter_kernel, dim3(scatter_grid_x(T, k, G, nw), nbatch),
+                         dim3(nw * 32), assign::scatter_smem_bytes(G, E, N, nw), s, a);
 }
 
 }  // extern "C"
@@ -876,11 +925,12 @@ extern "C" int lb_assign_noalloc(const int32_t *ids, const int32_t *cnt, const v
     a.offs = offs;
     a.ws = scratch;
     a.ws_stride = assign::ws_words(G, E, N);
-    assign::prep_kernel<<<nbatch, assign::PREP_THREADS, assign::prep_smem_bytes(G, E, N), s>>>(a);
-    if (launched("assign prep (noalloc)") != LB_OK) return LB_ECUDA;
+    if (launch_kernel("assign prep (noalloc)", assign::prep_kernel, dim3(nbatch),
+                      dim3(std::min(assign::PREP_THREADS, g_max_threads)),
+                      assign::prep_smem_bytes(G, E, N), s, a) != LB_OK)
+        return LB_ECUDA;
     if (T == 0) return LB_OK;
     const int nw = scatter_warps(nbatch, T, k, G, E, N);
-    assign::scatter_kernel<<<dim3(scatter_grid_x(T, k, G, nw), nbatch), nw * 32,
-                             assign::scatter_smem_bytes(G, E, N, nw), s>>>(a);
-    return launched("assign scatter (noalloc)");
+    return launch_kernel("assign scatter (noalloc)", assign::scatter_kernel, dim3(scatter_grid_x(T, k, G, nw), nbatch),
+                         dim3(nw * 32), assign::scatter_smem_bytes(G, E, N, nw), s, a);
 }

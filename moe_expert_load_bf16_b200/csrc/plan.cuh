@@ -70,6 +70,7 @@ __global__ void __launch_bounds__(THREADS)
     plan_kernel(const int32_t *__restrict__ cnt_all, int G, int E, int N, int L,
                 uint8_t *__restrict__ plan_all, size_t stride) {
     extern __shared__ __align__(16) uint8_t sm[];
+    pdl_begin();
     const int GN = G * N;
     const int W = (GN + 63) / 64 + 1;
     uint64_t *hold = reinterpret_cast<uint64_t *>(sm);

@@ -45,6 +45,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     solve_kernel(const assign::Args a, int passes, int32_t *__restrict__ loads_out,
                  int32_t *__restrict__ passes_run_out) {
     extern __shared__ __align__(16) uint8_t sm[];
+    pdl_begin();
     __shared__ int bad_ids, bad_plan;
     const int G = a.G, E = a.E, N = a.N, k = a.k, T = a.T, GN = G * N;
     const int tid = threadIdx.x;

@@ -333,6 +333,7 @@ __global__ void __launch_bounds__(THREADS)
                  int E, int N, int passes, int32_t *__restrict__ tok_all, int32_t *__restrict__ mass_all,
                  int32_t *__restrict__ loads_all, int32_t *__restrict__ passes_run_all) {
     extern __shared__ __align__(16) uint8_t sm[];
+    pdl_begin();
     __shared__ int bad;
     const int tid = threadIdx.x, b = blockIdx.x, GN = G * N;
     if (tid == 0) bad = 0;

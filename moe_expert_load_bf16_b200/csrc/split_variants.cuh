@@ -74,6 +74,7 @@ __device__ __forceinline__ long long warp_max_ll(long long x) {
 
 __global__ void __launch_bounds__(THREADS) split_variant_kernel(const Params p) {
     extern __shared__ __align__(16) uint8_t sm[];
+    pdl_begin();
     const int G = p.G, E = p.E, N = p.N, GN = G * N, b = blockIdx.x;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     long long *L = reinterpret_cast<long long *>(sm);

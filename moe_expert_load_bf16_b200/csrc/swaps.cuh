@@ -65,6 +65,7 @@ __device__ __forceinline__ bool better(double r1, int a1, int b1, double r2, int
 
 __global__ void __launch_bounds__(THREADS) swaps_kernel(const Params p) {
     extern __shared__ __align__(16) uint8_t sm[];
+    pdl_begin();
     const int G = p.G, E = p.E, b = blockIdx.x;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     double *res_link = reinterpret_cast<double *>(sm);

@@ -97,11 +97,66 @@ class DecisionPath:
         that read one hidden state run in one pass over it
         (lb_predict_topk_chain); predicted and actual ids are counted in one
         launch."""
-        B = self.B
+        self.gate_chain(hid, w, bias)
+        self.decide_chain()
+
+    def gate_chain(self, hid, w, bias):
+        """The gate half of run_chain: predicted and actual ids."""
         _lib.lb_predict_topk_chain(hid, w, bias, self.k, ids_pred=self.ids_pred, ids_act=self.ids)
+
+    def decide_chain(self):
+        """The integer half of run_chain, from the ids in this path's
+        buffers: both counts in one launch, plan, split, assign."""
+        B = self.B
         _lib.lb_count(self.ids_both.view(2 * B, self.T, self.k), self.G, self.E,
                       cnt=self.cnt_both.view(2 * B, self.G, self.E))
         _lib.lb_plan_replicas(self.cnt_pred, self.N, self.L, plan=self.plan)
         self.solve(counted=True)
 
     LAUNCHES_PER_CHAIN = 6   # chain gate, count (both), plan, split, assign prep + scatter
+
+
+class StepPipeline:
+    """Consecutive steps of the chained path with two batches in flight.
+
+    The gate of a step streams the hidden states at full HBM bandwidth on
+    every SM; the integer stages that follow it (count, plan, split, assign)
+    are latency-bound chains with one block per problem.  Here the gate of
+    step i+1 runs on one stream while the integer stages of step i run on a
+    second stream of higher priority, so the integer chain takes SM slots
+    as the gate frees them and overlaps it.  Two DecisionPath buffers
+    alternate between steps; an event per buffer keeps a step's gate from
+    overwriting ids that the integer stages of the step two before it still
+    read.  Every step computes the whole path over its batch: step i's
+    results are in paths[i % 2] once run() returns (in stream order).
+    run() forks from and joins back to the current stream, so a sequence of
+    steps can be captured in a CUDA graph."""
+
+    def __init__(self, B, T, H, E, k, G, N, L, passes=12, device="cuda"):
+        dev = torch.device(device)
+        self.paths = [DecisionPath(B, T, H, E, k, G, N, L, passes=passes, device=dev) for _ in range(2)]
+        self.gate_stream = torch.cuda.Stream(device=dev)
+        self.int_stream = torch.cuda.Stream(device=dev, priority=-1)
+        self.gate_done = [torch.cuda.Event() for _ in range(2)]
+        self.int_done = [torch.cuda.Event() for _ in range(2)]
+
+    def run(self, steps, hid, w, bias):
+        cur = torch.cuda.current_stream()
+        self.gate_stream.wait_stream(cur)
+        self.int_stream.wait_stream(cur)
+        for i in range(steps):
+            b = i % 2
+            p = self.paths[b]
+            with torch.cuda.stream(self.gate_stream):
+                if i >= 2:
+                    self.gate_stream.wait_event(self.int_done[b])
+                p.gate_chain(hid, w, bias)
+                self.gate_done[b].record(self.gate_stream)
+            with torch.cuda.stream(self.int_stream):
+                self.int_stream.wait_event(self.gate_done[b])
+                p.decide_chain()
+                self.int_done[b].record(self.int_stream)
+        cur.wait_stream(self.gate_stream)
+        cur.wait_stream(self.int_stream)
+
+    LAUNCHES_PER_STEP = DecisionPath.LAUNCHES_PER_CHAIN

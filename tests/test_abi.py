@@ -78,11 +78,18 @@ def test_arguments_rejected_before_any_launch(lib):
     assert lib.lb_split(P(256), P(256), 1, 4, 16, 1, -1, P(16), P(16), P(16), P(16), s) == _lib.LB_EINVAL
     assert lib.lb_assign(P(16), P(16), P(256), P(16), P(16), 1, 8, 2, 4, 16, 1, P(16), P(16), P(16), P(256),
                          1, s) == _lib.LB_ENOSPACE
-    assert lib.lb_gate_tuning(3, 5, 0, 0, 0) == _lib.LB_EINVAL
-    assert lib.lb_gate_tuning(3, 2, 3, 0, 0) == _lib.LB_EINVAL
-    assert lib.lb_gate_tuning(3, 2, 1, 3, 0) == _lib.LB_EINVAL
-    assert lib.lb_gate_tuning(0, 0, 0, 0, 3) == _lib.LB_EINVAL
-    assert lib.lb_gate_tuning(0, 0, 0, 0, 0) == _lib.LB_OK
+    assert lib.lb_gate_tuning(3, 5, 0, 0, 0, 0) == _lib.LB_EINVAL
+    assert lib.lb_gate_tuning(3, 2, 3, 0, 0, 0) == _lib.LB_EINVAL
+    assert lib.lb_gate_tuning(3, 2, 1, 3, 0, 0) == _lib.LB_EINVAL
+    assert lib.lb_gate_tuning(0, 0, 0, 0, 3, 0) == _lib.LB_EINVAL
+    assert lib.lb_gate_tuning(0, 0, 0, 0, 0, -1) == _lib.LB_EINVAL
+    assert lib.lb_gate_tuning(0, 0, 0, 0, 0, 0) == _lib.LB_OK
+    assert lib.lb_launch_options(2, 0) == _lib.LB_EINVAL
+    assert lib.lb_launch_options(-1, 0) == _lib.LB_EINVAL
+    assert lib.lb_launch_options(1, 384) == _lib.LB_EINVAL
+    assert lib.lb_launch_options(1, 2048) == _lib.LB_EINVAL
+    assert lib.lb_launch_options(1, 512) == _lib.LB_OK
+    assert lib.lb_launch_options(1, 0) == _lib.LB_OK
 
 
 def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
