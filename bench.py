@@ -183,10 +183,6 @@ def run_ours(args, world, rank, local):
     bias = workloads.biases(wl, Lyr).to(dev)
     chain = args.gate == "chain"
     pipe = StepPipeline(Lyr, T, H, E, k, G, N, L, device=dev) if chain and args.in_flight == 2 else None
-    if pipe:
-        # integer blocks of at most 512 threads, so that one fits beside a
-        # gate CTA on an SM the gate's grid leaves half free
-        _lib.lb_launch_options(1, 512)
     path = pipe.paths[0] if pipe else DecisionPath(Lyr, T, H, E, k, G, N, L, device=dev)
     side = torch.cuda.Stream(device=dev)
 
@@ -312,10 +308,10 @@ def run_ours(args, world, rank, local):
                    "layers": Lyr, "T": T, "H": H, "E": E, "k": k, "G": G, "N": N, "L": L, "passes": 12,
                    "batching": "all layers of a step in one launch per kernel, CUDA-graph replay",
                    "steps_in_flight": (2 if pipe else 1),
-                   "integer_block_threads_max": (512 if pipe else 1024),
-                   "overlap": ("two steps in flight: the gate of step i+1 on one stream beside the integer "
-                               "stages of step i on a second, higher-priority stream (two buffer sets); "
-                               "the K timed steps are one CUDA graph" if pipe else "none: one step after another"),
+                   "overlap": ("two steps in flight: the integer stages of step i on a second, higher-priority "
+                               "stream; the gate of step i+1 starts after step i's count and runs beside its "
+                               "plan, split and assign (two buffer sets); the K timed steps are one CUDA graph"
+                               if pipe else "none: one step after another"),
                    "gate": ("chain: one pass per hidden state evaluates the normal router of the layer before "
                             "it and the lookahead of the layer after it" if chain else
                             "two passes (lookahead, normal router); lookahead counts + plan on a second stream"),
