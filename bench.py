@@ -308,9 +308,10 @@ def run_ours(args, world, rank, local):
                    "layers": Lyr, "T": T, "H": H, "E": E, "k": k, "G": G, "N": N, "L": L, "passes": 12,
                    "batching": "all layers of a step in one launch per kernel, CUDA-graph replay",
                    "steps_in_flight": (2 if pipe else 1),
-                   "overlap": ("two steps in flight: the integer stages of step i on a second, higher-priority "
-                               "stream; the gate of step i+1 starts after step i's count and runs beside its "
-                               "plan, split and assign (two buffer sets); the K timed steps are one CUDA graph"
+                   "overlap": ("two steps in flight: gate and count of each step on one stream, plan, split "
+                               "and assign on a second, higher-priority stream, so the gate of step i+1 runs "
+                               "beside the plan, split and assign of step i (two buffer sets); the K timed "
+                               "steps are one CUDA graph"
                                if pipe else "none: one step after another"),
                    "gate": ("chain: one pass per hidden state evaluates the normal router of the layer before "
                             "it and the lookahead of the layer after it" if chain else

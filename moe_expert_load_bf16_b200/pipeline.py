@@ -104,15 +104,20 @@ class DecisionPath:
         """The gate half of run_chain: predicted and actual ids."""
         _lib.lb_predict_topk_chain(hid, w, bias, self.k, ids_pred=self.ids_pred, ids_act=self.ids)
 
-    def decide_chain(self, counted=None):
+    def decide_chain(self):
         """The integer half of run_chain, from the ids in this path's
-        buffers: both counts in one launch, plan, split, assign.  `counted`,
-        an event, is recorded once the counts are enqueued."""
+        buffers: both counts in one launch, plan, split, assign."""
+        self.count_chain()
+        self.finish_chain()
+
+    def count_chain(self):
+        """Predicted and actual ids counted in one launch."""
         B = self.B
         _lib.lb_count(self.ids_both.view(2 * B, self.T, self.k), self.G, self.E,
                       cnt=self.cnt_both.view(2 * B, self.G, self.E))
-        if counted is not None:
-            counted.record()
+
+    def finish_chain(self):
+        """Plan, split and assign from this path's counts."""
         _lib.lb_plan_replicas(self.cnt_pred, self.N, self.L, plan=self.plan)
         self.solve(counted=True)
 
@@ -125,25 +130,24 @@ class StepPipeline:
     The gate of a step streams the hidden states at full HBM bandwidth on
     every SM; of the integer stages that follow it, count spreads over many
     blocks, while plan, split and assign are latency-bound chains with one
-    block (or a few) per problem.  Here the integer stages of step i run on
-    a second stream of higher priority; the gate of step i+1 starts once
-    step i's counts are done and runs beside step i's plan, split and
-    assign, which take the SM slots the gate's grid leaves free.  (Starting
-    the next gate at once was slower: its blocks, launched early, took the
-    SMs before the count's.)  Two DecisionPath buffers alternate between
-    steps; an event per buffer keeps a step's gate from overwriting ids that
-    the integer stages of the step two before it still read.  Every step
-    computes the whole path over its batch: step i's results are in
-    paths[i % 2] once run() returns (in stream order).  run() forks from and
-    joins back to the current stream, so a sequence of steps can be captured
-    in a CUDA graph."""
+    block (or a few) per problem.  Here gate and count of each step run on
+    one stream, and plan, split and assign on a second stream of higher
+    priority: the gate of step i+1 follows step i's count and runs beside
+    step i's plan, split and assign, which take the SM slots the gate's
+    grid leaves free.  (Starting the next gate before the count was slower:
+    its blocks, launched early, took the SMs before the count's.)  Two
+    DecisionPath buffers alternate between steps; an event per buffer keeps
+    a step's gate from overwriting ids that the integer stages of the step
+    two before it still read.  Every step computes the whole path over its
+    batch: step i's results are in paths[i % 2] once run() returns (in
+    stream order).  run() forks from and joins back to the current stream,
+    so a sequence of steps can be captured in a CUDA graph."""
 
     def __init__(self, B, T, H, E, k, G, N, L, passes=12, device="cuda"):
         dev = torch.device(device)
         self.paths = [DecisionPath(B, T, H, E, k, G, N, L, passes=passes, device=dev) for _ in range(2)]
         self.gate_stream = torch.cuda.Stream(device=dev)
         self.int_stream = torch.cuda.Stream(device=dev, priority=-1)
-        self.gate_done = [torch.cuda.Event() for _ in range(2)]
         self.counted = [torch.cuda.Event() for _ in range(2)]
         self.int_done = [torch.cuda.Event() for _ in range(2)]
 
@@ -157,13 +161,12 @@ class StepPipeline:
             with torch.cuda.stream(self.gate_stream):
                 if i >= 2:
                     self.gate_stream.wait_event(self.int_done[b])
-                if i >= 1:
-                    self.gate_stream.wait_event(self.counted[1 - b])
                 p.gate_chain(hid, w, bias)
-                self.gate_done[b].record(self.gate_stream)
+                p.count_chain()
+                self.counted[b].record(self.gate_stream)
             with torch.cuda.stream(self.int_stream):
-                self.int_stream.wait_event(self.gate_done[b])
-                p.decide_chain(counted=self.counted[b])
+                self.int_stream.wait_event(self.counted[b])
+                p.finish_chain()
                 self.int_done[b].record(self.int_stream)
         cur.wait_stream(self.gate_stream)
         cur.wait_stream(self.int_stream)
