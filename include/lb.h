@@ -332,6 +332,27 @@ int lb_assign(const int32_t *ids, const int32_t *cnt, const void *plan,
               void *workspace, size_t workspace_bytes, void *stream);
 
 /* ------------------------------------------------------------------------
+ * Steps 3-5 in two launches -- plan (optional), split, assign   [Libra, Key
+ * Ideas; Relief, Algorithm 1; FB sec. 2.2]
+ * The same bytes as, in order,
+ *   lb_plan_replicas(cnt_pred, nbatch, G, E, N, L, plan)   (if cnt_pred)
+ *   lb_split(cnt, plan, nbatch, G, E, N, passes, tok, mass, loads, passes_run)
+ *   lb_assign(ids, cnt, plan, tok, mass, nbatch, T, k, G, E, N, dest, perm,
+ *             offs, workspace, workspace_bytes)
+ * with the plan, the split and the assign's tables of each problem made by
+ * one block in series (one launch) and the scatter as a second launch.
+ *   cnt_pred   int32 [nbatch, G, E] or NULL.  NULL: plan is an input (a blob
+ *              of lb_plan_replicas) and L is ignored; else plan is written.
+ *   other arguments, limits and errors: as the three calls (L, N: as
+ *   lb_plan_replicas when cnt_pred is given).
+ * ------------------------------------------------------------------------ */
+int lb_decide(const int32_t *cnt_pred, const int32_t *cnt, const int32_t *ids,
+              void *plan, int nbatch, int T, int k, int G, int E, int N, int L,
+              int passes, int32_t *tok, int32_t *mass, int32_t *loads,
+              int32_t *passes_run, int32_t *dest, int32_t *perm, int32_t *offs,
+              void *workspace, size_t workspace_bytes, void *stream);
+
+/* ------------------------------------------------------------------------
  * Steps 2, 4 and 5 fused -- the per-step decision on the actual ids in one
  * launch   [FB sec. 3.2 eq. 5; Relief, Algorithm 1; Libra, Key Ideas]
  * Computes exactly what lb_count, then lb_split, then lb_assign compute

@@ -61,6 +61,7 @@ def _load():
     lib.lb_assign_workspace_bytes.argtypes = [I, I, I, I, I, I]
     lib.lb_assign_workspace_bytes.restype = SZ
     lib.lb_assign.argtypes = [P, P, P, P, P, I, I, I, I, I, I, P, P, P, P, SZ, P]
+    lib.lb_decide.argtypes = [P, P, P, P, I, I, I, I, I, I, I, I, P, P, P, P, P, P, P, P, SZ, P]
     lib.lb_assign_noalloc.argtypes = [P, P, P, P, P, I, I, I, I, I, I, P, P, P, P]
     lib.lb_solve.argtypes = [P, P, I, I, I, I, I, I, I, P, P, P, P, P, P, P, P, P, SZ, P]
     lib.lb_get_status.argtypes = [ctypes.POINTER(ctypes.c_int32), I]
@@ -71,7 +72,7 @@ def _load():
     for f in ("lb_predict_topk", "lb_predict_topk_chain", "lb_plan_swaps", "lb_swaps_capacity", "lb_split_variant",
               "lb_gate_tuning", "lb_launch_options",
               "lb_count", "lb_plan_layout_of", "lb_plan_replicas",
-              "lb_split", "lb_assign", "lb_assign_noalloc", "lb_solve", "lb_get_status", "lb_version"):
+              "lb_split", "lb_assign", "lb_assign_noalloc", "lb_decide", "lb_solve", "lb_get_status", "lb_version"):
         getattr(lib, f).restype = ctypes.c_int
     _lib = lib
     return lib
@@ -340,6 +341,35 @@ def lb_assign(ids, cnt, plan, tok, mass, N, out=None, workspace=None):
     return dest, perm, offs
 
 
+def lb_decide(cnt, ids, plan, N, passes=12, cnt_pred=None, L=0, out=None, workspace=None):
+    """Plan (from cnt_pred, when given; else plan is an input), split and
+    assign in two launches.  Returns (tok, mass, loads, passes_run, dest,
+    perm, offs); out preallocates them."""
+    lib = _load()
+    ids, cnt = _batched(ids, 3), _batched(cnt, 3)
+    _need(ids, torch.int32, "ids")
+    _need(cnt, torch.int32, "cnt")
+    if cnt_pred is not None:
+        cnt_pred = _batched(cnt_pred, 3)
+        _need(cnt_pred, torch.int32, "cnt_pred")
+    B, T, k = ids.shape
+    _, G, E = cnt.shape
+    dev = ids.device
+    if out is None:
+        i32 = dict(dtype=torch.int32, device=dev)
+        out = (torch.empty(B, G * N, **i32), torch.empty(B, G * N, **i32), torch.empty(B, G, **i32),
+               torch.empty(B, **i32), torch.empty(B, T, k, **i32), torch.empty(B, T * k, **i32),
+               torch.empty(B, G * E + 1, **i32))
+    tok, mass, loads, passes_run, dest, perm, offs = out
+    nbytes = lb_assign_workspace_bytes(B, T, k, G, E, N)
+    if workspace is None:
+        workspace = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=dev)
+    _check("lb_decide", lib.lb_decide(_p(cnt_pred), _p(cnt), _p(ids), _p(plan), B, T, k, G, E, N, L, passes,
+                                      _p(tok), _p(mass), _p(loads), _p(passes_run), _p(dest), _p(perm), _p(offs),
+                                      _p(workspace), workspace.numel(), _stream()))
+    return out
+
+
 def lb_solve(ids, plan, G, E, N, passes=12, out=None, workspace=None):
     """Count + split + assign in one launch.  out = (cnt, tok, mass, loads,
     passes_run, dest, perm, offs) preallocated, or None."""
@@ -400,6 +430,7 @@ def lb_version():
 
 EXPORTS = ("lb_predict_topk", "lb_predict_topk_chain", "lb_gate_tuning", "lb_launch_options", "lb_plan_swaps", "lb_swaps_capacity",
            "lb_split_variant", "lb_count", "lb_plan_bytes", "lb_plan_layout_of",
-           "lb_plan_replicas", "lb_split", "lb_assign_workspace_bytes", "lb_assign", "lb_assign_noalloc", "lb_solve",
+           "lb_plan_replicas", "lb_split", "lb_assign_workspace_bytes", "lb_assign", "lb_assign_noalloc", "lb_decide",
+           "lb_solve",
            "lb_get_status",
            "lb_strerror", "lb_last_error", "lb_version")

@@ -12,6 +12,7 @@
 #include "assign.cuh"
 #include "common.cuh"
 #include "count.cuh"
+#include "decide.cuh"
 #include "gate_topk.cuh"
 #include "plan.cuh"
 #include "solve.cuh"
@@ -138,6 +139,9 @@ bool allow_smem(F *kernel, SmemLimit &lim, size_t bytes, bool cluster16) {
     }
     return true;
 }
+
+// One limit record per kernel that several entry points launch.
+SmemLimit g_lim_prep, g_lim_scatter;
 
 template <int KMAX, bool SPLITK>
 int launch_gate(const CUtensorMap &ma, const CUtensorMap &mb, const gate::Params &p, int mtiles, int nbatch,
@@ -735,8 +739,8 @@ int lb_assign(const int32_t *ids, const int32_t *cnt, const void *plan, const in
     a.ws_stride = assign::ws_words(G, E, N);
     const int nw = T > 0 ? scatter_warps(nbatch, T, k, G, E, N) : assign::SC_WARPS;
     const size_t sm1 = assign::prep_smem_bytes(G, E, N), sm2 = assign::scatter_smem_bytes(G, E, N, nw);
-    static SmemLimit lim1, lim2;
-    if (!allow_smem(assign::prep_kernel, lim1, sm1, false) || !allow_smem(assign::scatter_kernel, lim2, sm2, false))
+    if (!allow_smem(assign::prep_kernel, g_lim_prep, sm1, false) ||
+        !allow_smem(assign::scatter_kernel, g_lim_scatter, sm2, false))
         return LB_ECUDA;
     if (launch_kernel("assign prep", assign::prep_kernel, dim3(nbatch), dim3(std::min(assign::PREP_THREADS, g_max_threads)),
                       sm1, s, a) != LB_OK)
@@ -744,6 +748,60 @@ int lb_assign(const int32_t *ids, const int32_t *cnt, const void *plan, const in
     if (T == 0) return LB_OK;
     return launch_kernel("assign scatter", assign::scatter_kernel, dim3(scatter_grid_x(T, k, G, nw), nbatch),
                          dim3(nw * 32), assign::scatter_smem_bytes(G, E, N, nw), s, a);
+}
+
+int lb_decide(const int32_t *cnt_pred, const int32_t *cnt, const int32_t *ids, void *plan, int nbatch, int T,
+              int k, int G, int E, int N, int L, int passes, int32_t *tok, int32_t *mass, int32_t *loads,
+              int32_t *passes_run, int32_t *dest, int32_t *perm, int32_t *offs, void *workspace,
+              size_t workspace_bytes, void *stream) {
+    const bool with_plan = cnt_pred != nullptr;
+    if (nbatch < 1 || nbatch > 65535 || T < 0 || T % G != 0 || k < 1 || k > LB_MAX_K ||
+        !plan_shape_ok(G, E, N, with_plan ? L : 0) || passes < 0 || passes > 4096)
+        return LB_EINVAL;
+    if (!cnt || !plan || !loads || !passes_run || !offs || !workspace || !aligned(plan, 256) ||
+        !aligned(workspace, 256) || (with_plan && !aligned(cnt_pred, 4)))
+        return LB_EINVAL;
+    if (G * N > 0 && (!tok || !mass)) return LB_EINVAL;
+    if (T > 0 && (!ids || !dest || !perm)) return LB_EINVAL;
+    if (static_cast<long long>(T) * k * nbatch >= INT_MAX) return LB_EINVAL;
+    const size_t sm1 = decide::smem_bytes(G, E, N, with_plan);
+    if (assign::scatter_smem_bytes(G, E, N, 8) > 224 * 1024 || sm1 > 224 * 1024) return LB_EINVAL;
+    if (workspace_bytes < lb_assign_workspace_bytes(nbatch, T, k, G, E, N)) return LB_ENOSPACE;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    assign::Args a;
+    a.ids = ids;
+    a.cnt = cnt;
+    a.tok = tok;
+    a.mass = mass;
+    a.plan = static_cast<const uint8_t *>(plan);
+    a.plan_stride = plan::layout(G, E, N).total;
+    a.T = T;
+    a.k = k;
+    a.G = G;
+    a.E = E;
+    a.N = N;
+    a.dest = dest;
+    a.perm = perm;
+    a.offs = offs;
+    a.ws = static_cast<int32_t *>(workspace);
+    a.ws_stride = assign::ws_words(G, E, N);
+    const int nw = T > 0 ? scatter_warps(nbatch, T, k, G, E, N) : assign::SC_WARPS;
+    const size_t sm2 = assign::scatter_smem_bytes(G, E, N, nw);
+    static SmemLimit lim0, lim1;
+    if (!allow_smem(assign::scatter_kernel, g_lim_scatter, sm2, false)) return LB_ECUDA;
+    int rc;
+    if (with_plan) {
+        if (!allow_smem(decide::decide_kernel<true>, lim1, sm1, false)) return LB_ECUDA;
+        rc = launch_kernel("decide (plan, split, tables)", decide::decide_kernel<true>, dim3(nbatch),
+                           dim3(decide::THREADS), sm1, s, cnt_pred, L, a, passes, loads, passes_run);
+    } else {
+        if (!allow_smem(decide::decide_kernel<false>, lim0, sm1, false)) return LB_ECUDA;
+        rc = launch_kernel("decide (split, tables)", decide::decide_kernel<false>, dim3(nbatch),
+                           dim3(decide::THREADS), sm1, s, cnt_pred, L, a, passes, loads, passes_run);
+    }
+    if (rc != LB_OK || T == 0) return rc;
+    return launch_kernel("assign scatter", assign::scatter_kernel, dim3(scatter_grid_x(T, k, G, nw), nbatch),
+                         dim3(nw * 32), sm2, s, a);
 }
 
 }  // extern "C"
@@ -925,12 +983,15 @@ extern "C" int lb_assign_noalloc(const int32_t *ids, const int32_t *cnt, const v
     a.offs = offs;
     a.ws = scratch;
     a.ws_stride = assign::ws_words(G, E, N);
+    const int nw = T > 0 ? scatter_warps(nbatch, T, k, G, E, N) : assign::SC_WARPS;
+    if (!allow_smem(assign::prep_kernel, g_lim_prep, assign::prep_smem_bytes(G, E, N), false) ||
+        !allow_smem(assign::scatter_kernel, g_lim_scatter, assign::scatter_smem_bytes(G, E, N, nw), false))
+        return LB_ECUDA;
     if (launch_kernel("assign prep (noalloc)", assign::prep_kernel, dim3(nbatch),
                       dim3(std::min(assign::PREP_THREADS, g_max_threads)),
                       assign::prep_smem_bytes(G, E, N), s, a) != LB_OK)
         return LB_ECUDA;
     if (T == 0) return LB_OK;
-    const int nw = scatter_warps(nbatch, T, k, G, E, N);
     return launch_kernel("assign scatter (noalloc)", assign::scatter_kernel, dim3(scatter_grid_x(T, k, G, nw), nbatch),
                          dim3(nw * 32), assign::scatter_smem_bytes(G, E, N, nw), s, a);
 }

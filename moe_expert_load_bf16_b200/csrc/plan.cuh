@@ -66,11 +66,11 @@ __host__ __device__ inline size_t smem_bytes(int G, int E, int N) {
            + (GN + 1) * 4 * 2;                   // round ptr, round fill
 }
 
-__global__ void __launch_bounds__(THREADS)
-    plan_kernel(const int32_t *__restrict__ cnt_all, int G, int E, int N, int L,
-                uint8_t *__restrict__ plan_all, size_t stride) {
-    extern __shared__ __align__(16) uint8_t sm[];
-    pdl_begin();
+// The whole plan of one problem by one CTA: counts cnt [G, E] (global) in,
+// the blob (global) out; `sm` holds smem_bytes(G, E, N) bytes.  All threads
+// of the CTA call it; it ends with a block barrier.
+__device__ void plan_problem(const int32_t *__restrict__ cnt, int G, int E, int N, int L, uint8_t *__restrict__ blob,
+                             uint8_t *sm) {
     const int GN = G * N;
     const int W = (GN + 63) / 64 + 1;
     uint64_t *hold = reinterpret_cast<uint64_t *>(sm);
@@ -91,9 +91,6 @@ __global__ void __launch_bounds__(THREADS)
     __shared__ int n_edges_s, n_rounds_s, n_p2_s;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, nwarps = blockDim.x >> 5;
-    const int b = blockIdx.x;
-    const int32_t *cnt = cnt_all + static_cast<int64_t>(b) * G * E;
-    uint8_t *blob = plan_all + static_cast<size_t>(b) * stride;
     const Layout LY = layout(G, E, N);
     const int Eg = E / G;
 
@@ -407,6 +404,16 @@ __global__ void __launch_bounds__(THREADS)
     for (size_t i = LY.holds + static_cast<size_t>(G) * E + tid; i < LY.total; i += blockDim.x) blob[i] = 0;
     __syncthreads();
     LB_TICK(37);
+}
+
+__global__ void __launch_bounds__(THREADS)
+    plan_kernel(const int32_t *__restrict__ cnt_all, int G, int E, int N, int L,
+                uint8_t *__restrict__ plan_all, size_t stride) {
+    extern __shared__ __align__(16) uint8_t sm[];
+    pdl_begin();
+    const int b = blockIdx.x;
+    plan_problem(cnt_all + static_cast<int64_t>(b) * G * E, G, E, N, L, plan_all + static_cast<size_t>(b) * stride,
+                 sm);
 }
 
 }  // namespace plan

@@ -12,6 +12,8 @@ both gates that read one hidden state in a single pass over it:
   cnt      = counts(ids)                                    lb_count
   tok, mass, loads = split(cnt, plan)                       lb_split
   dest, perm, offs = assign(ids, cnt, plan, split)          lb_assign
+(`solve` runs split and assign as lb_decide: split and the assign's tables
+in one launch per problem, the scatter in a second.)
 """
 import torch
 
@@ -50,10 +52,17 @@ class DecisionPath:
     def route(self, h_cur, w, bias):
         _lib.lb_predict_topk(h_cur, w, bias, self.k, ids=self.ids)
 
-    # the per-step decision on actual ids (T_solve): lb_count, lb_split,
-    # lb_assign (on the benchmark shapes these three launches are faster than
-    # the fused lb_solve, whose single CTA 0 runs split and tables in series)
+    # the per-step decision on actual ids (T_solve): lb_count, then split and
+    # assign by lb_decide (split and the assign's tables in one launch per
+    # problem, the scatter in a second); solve_separate makes the same bytes
+    # with lb_split and lb_assign
     def solve(self, ids=None, counted=False):
+        ids = self.ids if ids is None else ids
+        if not counted:
+            _lib.lb_count(ids, self.G, self.E, cnt=self.cnt)
+        self.decide(ids)
+
+    def solve_separate(self, ids=None, counted=False):
         ids = self.ids if ids is None else ids
         if not counted:
             _lib.lb_count(ids, self.G, self.E, cnt=self.cnt)
@@ -61,6 +70,15 @@ class DecisionPath:
                       out=(self.tok, self.mass, self.loads, self.passes_run))
         _lib.lb_assign(ids, self.cnt, self.plan, self.tok, self.mass, self.N,
                        out=(self.dest, self.perm, self.offs), workspace=self.ws)
+
+    def decide(self, ids=None, with_plan=False):
+        """lb_decide on this path's buffers: the plan from cnt_pred first when
+        with_plan, then split and assign of cnt."""
+        ids = self.ids if ids is None else ids
+        cnt_pred = self.cnt_pred if with_plan else None
+        _lib.lb_decide(self.cnt, ids, self.plan, self.N, self.passes, cnt_pred=cnt_pred, L=self.L,
+                       out=(self.tok, self.mass, self.loads, self.passes_run, self.dest, self.perm, self.offs),
+                       workspace=self.ws)
 
     # the same decision as one fused launch (lb_solve)
     def solve_fused(self, ids=None):
@@ -88,7 +106,7 @@ class DecisionPath:
         main.wait_stream(side_stream)
         self.solve()
 
-    LAUNCHES_PER_RUN = 8   # 2 gate, 2 count, plan, split, assign prep + scatter
+    LAUNCHES_PER_RUN = 7   # 2 gate, 2 count, plan, split + tables, scatter
 
     def run_chain(self, hid, w, bias):
         """One pass over a chain of B consecutive layers whose hidden states
@@ -117,9 +135,12 @@ class DecisionPath:
                       cnt=self.cnt_both.view(2 * B, self.G, self.E))
 
     def finish_chain(self):
-        """Plan, split and assign from this path's counts."""
+        """Plan, split and assign from this path's counts, as separate
+        launches (measured: beside the next step's gate in StepPipeline,
+        lb_decide's single plan + split + tables launch per problem made
+        the pipelined step slower, 76.6 against 63.4 us)."""
         _lib.lb_plan_replicas(self.cnt_pred, self.N, self.L, plan=self.plan)
-        self.solve(counted=True)
+        self.solve_separate(counted=True)
 
     LAUNCHES_PER_CHAIN = 6   # chain gate, count (both), plan, split, assign prep + scatter
 

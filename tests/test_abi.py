@@ -78,6 +78,15 @@ def test_arguments_rejected_before_any_launch(lib):
     assert lib.lb_split(P(256), P(256), 1, 4, 16, 1, -1, P(16), P(16), P(16), P(16), s) == _lib.LB_EINVAL
     assert lib.lb_assign(P(16), P(16), P(256), P(16), P(16), 1, 8, 2, 4, 16, 1, P(16), P(16), P(16), P(256),
                          1, s) == _lib.LB_ENOSPACE
+    # lb_decide: L > N with predicted counts, negative passes, T % G, unaligned plan
+    #   (cnt_pred, cnt, ids, plan, nbatch, T, k, G, E, N, L, passes, tok, mass, loads, passes_run,
+    #    dest, perm, offs, workspace, workspace_bytes, stream)
+    for cp, T, L, passes, plan in ((P(256), 16, 3, 12, P(256)), (None, 16, 0, -1, P(256)),
+                                   (None, 10, 0, 12, P(256)), (None, 16, 0, 12, P(16))):
+        assert lib.lb_decide(cp, P(256), P(256), plan, 1, T, 2, 4, 16, 2, L, passes, P(16), P(16), P(16), P(16),
+                             P(16), P(16), P(16), P(256), 1 << 20, s) == _lib.LB_EINVAL
+    assert lib.lb_decide(None, P(256), P(256), P(256), 1, 16, 2, 4, 16, 2, 0, 12, P(16), P(16), P(16), P(16),
+                         P(16), P(16), P(16), P(256), 1, s) == _lib.LB_ENOSPACE
     assert lib.lb_gate_tuning(3, 5, 0, 0, 0, 0) == _lib.LB_EINVAL
     assert lib.lb_gate_tuning(3, 2, 3, 0, 0, 0) == _lib.LB_EINVAL
     assert lib.lb_gate_tuning(3, 2, 1, 3, 0, 0) == _lib.LB_EINVAL

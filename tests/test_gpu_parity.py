@@ -379,6 +379,45 @@ def test_solve_fused_equals_separate_calls(name, T, B):
         parity.check_path(path, b, 12)
 
 
+@pytest.mark.parametrize("name,T,B", [("tiny", 256, 3), ("olmoe", 4096, 4), ("qwen3-235b", 8192, 3),
+                                      ("decode", 1024, 5), ("decode", 64, 2), ("olmoe", 0, 2), ("decode", 0, 1)])
+def test_decide_equals_separate_calls(name, T, B):
+    """lb_decide (plan, split and the assign's tables in one launch per
+    problem, then the scatter) gives the bytes of lb_plan_replicas + lb_split
+    + lb_assign, with the plan computed from predicted counts and with the
+    plan given; the result passes the oracle check.  Distinct predicted
+    counts per problem, so a plan read from the wrong problem fails."""
+    w = workloads.WORKLOADS[name]
+    Tg = max(T, w.G)
+    ids = workloads.decode_ids(w.with_(T=Tg), Tg, range(2 * B)).to(DEV)[:, :T]
+    a = DecisionPath(B, T, 8, w.E, w.k, w.G, w.N, w.L, device=DEV)
+    b = DecisionPath(B, T, 8, w.E, w.k, w.G, w.N, w.L, device=DEV)
+    for p in (a, b):
+        p.ids_pred.copy_(ids[:B])
+        p.ids.copy_(ids[B:])
+        p.count_chain()
+    # separate calls
+    _lib.lb_plan_replicas(a.cnt_pred, w.N, w.L, plan=a.plan)
+    a.solve_separate(counted=True)
+    # plan + split + tables in one launch
+    b.plan.fill_(0x5a)
+    b.decide(with_plan=True)
+    torch.cuda.synchronize()
+    assert _lib.lb_get_status() == 0
+    for f in ("plan", "tok", "mass", "loads", "passes_run", "dest", "perm", "offs"):
+        assert torch.equal(getattr(a, f), getattr(b, f)), f
+    # plan given
+    for t in (b.tok, b.mass, b.loads, b.passes_run, b.dest, b.perm, b.offs):
+        t.fill_(-7)
+    b.solve(counted=True)
+    torch.cuda.synchronize()
+    assert _lib.lb_get_status() == 0
+    for f in ("plan", "tok", "mass", "loads", "passes_run", "dest", "perm", "offs"):
+        assert torch.equal(getattr(a, f), getattr(b, f)), f
+    for i in range(B):
+        parity.check_path(b, i, 12)
+
+
 @pytest.mark.parametrize("L,T,H,E,k,bias_on", [(3, 200, 128, 16, 2, True), (1, 256, 64, 16, 4, True),
                                                (4, 4096, 2048, 64, 8, True), (2, 1100, 2048, 128, 8, True),
                                                (5, 3000, 576, 64, 8, False), (2, 130, 8, 32, 16, True)])
