@@ -339,8 +339,10 @@ int lb_assign(const int32_t *ids, const int32_t *cnt, const void *plan,
  *   lb_split(cnt, plan, nbatch, G, E, N, passes, tok, mass, loads, passes_run)
  *   lb_assign(ids, cnt, plan, tok, mass, nbatch, T, k, G, E, N, dest, perm,
  *             offs, workspace, workspace_bytes)
- * with the plan, the split and the assign's tables of each problem made by
- * one block in series (one launch) and the scatter as a second launch.
+ * For count tables of fewer than 4096 keys (G*E) the plan, the split and
+ * the assign's tables of each problem are made by one block in series (one
+ * launch) and the scatter is a second launch; for larger tables, where the
+ * separate launches measured faster, the four run as separate launches.
  *   cnt_pred   int32 [nbatch, G, E] or NULL.  NULL: plan is an input (a blob
  *              of lb_plan_replicas) and L is ignored; else plan is written.
  *   other arguments, limits and errors: as the three calls (L, N: as

@@ -141,7 +141,7 @@ bool allow_smem(F *kernel, SmemLimit &lim, size_t bytes, bool cluster16) {
 }
 
 // One limit record per kernel that several entry points launch.
-SmemLimit g_lim_prep, g_lim_scatter;
+SmemLimit g_lim_plan, g_lim_split, g_lim_prep, g_lim_scatter;
 
 template <int KMAX, bool SPLITK>
 int launch_gate(const CUtensorMap &ma, const CUtensorMap &mb, const gate::Params &p, int mtiles, int nbatch,
@@ -680,8 +680,7 @@ int lb_plan_replicas(const int32_t *cnt, int nbatch, int G, int E, int N, int L,
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const size_t smem = plan::smem_bytes(G, E, N);
     if (smem > 224 * 1024) return LB_EINVAL;
-    static SmemLimit lim;
-    if (!allow_smem(plan::plan_kernel, lim, smem, false)) return LB_ECUDA;
+    if (!allow_smem(plan::plan_kernel, g_lim_plan, smem, false)) return LB_ECUDA;
     return launch_kernel("plan", plan::plan_kernel, dim3(nbatch), dim3(plan::THREADS), smem, s, cnt, G, E, N, L,
                          static_cast<uint8_t *>(plan), plan::layout(G, E, N).total);
 }
@@ -693,8 +692,7 @@ int lb_split(const int32_t *cnt, const void *plan, int nbatch, int G, int E, int
     if (G * N > 0 && (!tok || !mass)) return LB_EINVAL;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const size_t smem = split::smem_bytes(G, E, N);
-    static SmemLimit lim;
-    if (!allow_smem(split::split_kernel, lim, smem, false)) return LB_ECUDA;
+    if (!allow_smem(split::split_kernel, g_lim_split, smem, false)) return LB_ECUDA;
     return launch_kernel("split", split::split_kernel, dim3(nbatch), dim3(split::THREADS), smem, s, cnt,
                          static_cast<const uint8_t *>(plan), plan::layout(G, E, N).total, G, E, N, passes, tok, mass,
                          loads, passes_run);
@@ -790,14 +788,36 @@ int lb_decide(const int32_t *cnt_pred, const int32_t *cnt, const int32_t *ids, v
     static SmemLimit lim0, lim1;
     if (!allow_smem(assign::scatter_kernel, g_lim_scatter, sm2, false)) return LB_ECUDA;
     int rc;
-    if (with_plan) {
-        if (!allow_smem(decide::decide_kernel<true>, lim1, sm1, false)) return LB_ECUDA;
-        rc = launch_kernel("decide (plan, split, tables)", decide::decide_kernel<true>, dim3(nbatch),
-                           dim3(decide::THREADS), sm1, s, cnt_pred, L, a, passes, loads, passes_run);
+    if (decide::fused_for(G, E)) {
+        if (with_plan) {
+            if (!allow_smem(decide::decide_kernel<true>, lim1, sm1, false)) return LB_ECUDA;
+            rc = launch_kernel("decide (plan, split, tables)", decide::decide_kernel<true>, dim3(nbatch),
+                               dim3(decide::THREADS), sm1, s, cnt_pred, L, a, passes, loads, passes_run);
+        } else {
+            if (!allow_smem(decide::decide_kernel<false>, lim0, sm1, false)) return LB_ECUDA;
+            rc = launch_kernel("decide (split, tables)", decide::decide_kernel<false>, dim3(nbatch),
+                               dim3(decide::THREADS), sm1, s, cnt_pred, L, a, passes, loads, passes_run);
+        }
     } else {
-        if (!allow_smem(decide::decide_kernel<false>, lim0, sm1, false)) return LB_ECUDA;
-        rc = launch_kernel("decide (split, tables)", decide::decide_kernel<false>, dim3(nbatch),
-                           dim3(decide::THREADS), sm1, s, cnt_pred, L, a, passes, loads, passes_run);
+        // large count tables: plan, split and tables as separate launches
+        const size_t stride = plan::layout(G, E, N).total;
+        const size_t smp = plan::smem_bytes(G, E, N), sms = split::smem_bytes(G, E, N),
+                     smt = assign::prep_smem_bytes(G, E, N);
+        if ((with_plan && !allow_smem(plan::plan_kernel, g_lim_plan, smp, false)) ||
+            !allow_smem(split::split_kernel, g_lim_split, sms, false) ||
+            !allow_smem(assign::prep_kernel, g_lim_prep, smt, false))
+            return LB_ECUDA;
+        rc = LB_OK;
+        if (with_plan)
+            rc = launch_kernel("plan", plan::plan_kernel, dim3(nbatch), dim3(plan::THREADS), smp, s, cnt_pred, G, E,
+                               N, L, static_cast<uint8_t *>(plan), stride);
+        if (rc == LB_OK)
+            rc = launch_kernel("split", split::split_kernel, dim3(nbatch), dim3(split::THREADS), sms, s, cnt,
+                               static_cast<const uint8_t *>(plan), stride, G, E, N, passes, tok, mass, loads,
+                               passes_run);
+        if (rc == LB_OK)
+            rc = launch_kernel("assign prep", assign::prep_kernel, dim3(nbatch),
+                               dim3(std::min(assign::PREP_THREADS, g_max_threads)), smt, s, a);
     }
     if (rc != LB_OK || T == 0) return rc;
     return launch_kernel("assign scatter", assign::scatter_kernel, dim3(scatter_grid_x(T, k, G, nw), nbatch),
