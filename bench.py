@@ -71,7 +71,7 @@ def profile_traffic(kernel_tag, source_files):
 class ClockSampler:
     """Samples SM clock and throttle reasons with NVML in a background thread."""
 
-    def __init__(self, index, period=0.005):
+    def __init__(self, index, period=0.001):
         self.index, self.period = index, period
         self.samples, self.reasons, self.max_mhz = [], set(), None
         self._stop = threading.Event()
