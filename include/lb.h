@@ -390,9 +390,10 @@ int lb_solve(const int32_t *ids, const void *plan, int nbatch, int T, int k, int
  *     use lb_assign for those.
  *   - It allocates nothing: no cudaMalloc, no cudaFree, no allocating
  *     library routine.
- *   - The first call on a device looks up the array's device address and
- *     raises two kernels' shared-memory limits (once per device); make that
- *     first call before any stream capture.
+ *   - The first call on a device looks up the array's device address (once
+ *     per device, with that device current) and, like the first call of any
+ *     entry point, raises its kernels' shared-memory limits on that device;
+ *     make that first call before any stream capture.
  *   - All calls share the one array: calls that overlap on the GPU (for
  *     example on two streams) race and give wrong results.  The scratch keeps
  *     the last call's contents; every call fully rewrites what it reads, so

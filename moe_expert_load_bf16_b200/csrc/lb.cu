@@ -108,34 +108,54 @@ bool make_map(CUtensorMap *map, const void *base, uint64_t d0, uint64_t d1, uint
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+constexpr int kMaxDevices = 256;
+
+// Ordinal of the current device, or -1 (with the error recorded).
+int current_device() {
+    int dev = 0;
+    const cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) {
+        cuda_fail(e, "cudaGetDevice");
+        return -1;
+    }
+    if (dev < 0 || dev >= kMaxDevices) {
+        std::snprintf(g_last_error, sizeof g_last_error, "device ordinal %d out of range", dev);
+        return -1;
+    }
+    return dev;
+}
+
 // Raise a kernel's dynamic shared-memory limit to at least `bytes` (the
 // limit plus the kernel's static shared memory must stay within the
-// per-block opt-in maximum, so it is raised only as far as needed).
+// per-block opt-in maximum, so it is raised only as far as needed).  Kernel
+// attributes belong to a device, so the record is kept per device ordinal.
 struct SmemLimit {
     std::mutex mu;
-    size_t current = 0;
-    bool cluster_set = false;
+    size_t current[kMaxDevices] = {};
+    bool cluster_set[kMaxDevices] = {};
 };
 
 template <typename F>
 bool allow_smem(F *kernel, SmemLimit &lim, size_t bytes, bool cluster16) {
+    const int dev = current_device();
+    if (dev < 0) return false;
     std::lock_guard<std::mutex> lock(lim.mu);
-    if (bytes > lim.current) {
+    if (bytes > lim.current[dev]) {
         const cudaError_t e =
             cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(bytes));
         if (e != cudaSuccess) {
             cuda_fail(e, "cudaFuncSetAttribute(max dynamic shared memory)");
             return false;
         }
-        lim.current = bytes;
+        lim.current[dev] = bytes;
     }
-    if (cluster16 && !lim.cluster_set) {
+    if (cluster16 && !lim.cluster_set[dev]) {
         const cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
         if (e != cudaSuccess) {
             cuda_fail(e, "cudaFuncSetAttribute(non-portable cluster size)");
             return false;
         }
-        lim.cluster_set = true;
+        lim.cluster_set[dev] = true;
     }
     return true;
 }
@@ -708,7 +728,8 @@ size_t lb_assign_workspace_bytes(int nbatch, int T, int k, int G, int E, int N) 
 int lb_assign(const int32_t *ids, const int32_t *cnt, const void *plan, const int32_t *tok, const int32_t *mass,
               int nbatch, int T, int k, int G, int E, int N, int32_t *dest, int32_t *perm, int32_t *offs,
               void *workspace, size_t workspace_bytes, void *stream) {
-    if (nbatch < 1 || nbatch > 65535 || T < 0 || T % G != 0 || k < 1 || k > LB_MAX_K || !plan_shape_ok(G, E, N, 0))
+    // (G is range-checked by plan_shape_ok before T % G is taken)
+    if (nbatch < 1 || nbatch > 65535 || T < 0 || k < 1 || k > LB_MAX_K || !plan_shape_ok(G, E, N, 0) || T % G != 0)
         return LB_EINVAL;
     if (!cnt || !plan || !offs || !workspace || !aligned(plan, 256) || !aligned(workspace, 256)) return LB_EINVAL;
     if (G * N > 0 && (!tok || !mass)) return LB_EINVAL;
@@ -753,8 +774,8 @@ int lb_decide(const int32_t *cnt_pred, const int32_t *cnt, const int32_t *ids, v
               int32_t *passes_run, int32_t *dest, int32_t *perm, int32_t *offs, void *workspace,
               size_t workspace_bytes, void *stream) {
     const bool with_plan = cnt_pred != nullptr;
-    if (nbatch < 1 || nbatch > 65535 || T < 0 || T % G != 0 || k < 1 || k > LB_MAX_K ||
-        !plan_shape_ok(G, E, N, with_plan ? L : 0) || passes < 0 || passes > 4096)
+    if (nbatch < 1 || nbatch > 65535 || T < 0 || k < 1 || k > LB_MAX_K ||
+        !plan_shape_ok(G, E, N, with_plan ? L : 0) || T % G != 0 || passes < 0 || passes > 4096)
         return LB_EINVAL;
     if (!cnt || !plan || !loads || !passes_run || !offs || !workspace || !aligned(plan, 256) ||
         !aligned(workspace, 256) || (with_plan && !aligned(cnt_pred, 4)))
@@ -847,8 +868,8 @@ extern "C" int lb_solve(const int32_t *ids, const void *plan, int nbatch, int T,
                         int passes, int32_t *cnt, int32_t *tok, int32_t *mass, int32_t *loads,
                         int32_t *passes_run, int32_t *dest, int32_t *perm, int32_t *offs, void *workspace,
                         size_t workspace_bytes, void *stream) {
-    if (nbatch < 1 || nbatch > 65535 || T < 0 || T % G != 0 || k < 1 || k > LB_MAX_K || !plan_shape_ok(G, E, N, 0) ||
-        passes < 0 || passes > 4096)
+    if (nbatch < 1 || nbatch > 65535 || T < 0 || k < 1 || k > LB_MAX_K || !plan_shape_ok(G, E, N, 0) ||
+        T % G != 0 || passes < 0 || passes > 4096)
         return LB_EINVAL;
     if (!plan || !cnt || !offs || !loads || !passes_run || !workspace || !aligned(plan, 256) ||
         !aligned(workspace, 256))
@@ -922,40 +943,21 @@ namespace {
 constexpr size_t kNoAllocScratchBytes = LB_NOALLOC_SCRATCH_BYTES;
 static __device__ __align__(256) int32_t g_noalloc_scratch[kNoAllocScratchBytes / sizeof(int32_t)];
 
-constexpr int kMaxDevices = 256;
 std::mutex g_noalloc_mu;
 int32_t *g_noalloc_ptr[kMaxDevices] = {};
 
 // Device address of the scratch array on the current device (the array's
 // name in host code is only a host-side stand-in).  Looked up once per
-// device, together with the kernels' shared-memory limits.
+// device, with that device current.
 int32_t *noalloc_scratch() {
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) {
-        cuda_fail(e, "cudaGetDevice");
-        return nullptr;
-    }
-    if (dev < 0 || dev >= kMaxDevices) {
-        std::snprintf(g_last_error, sizeof g_last_error, "device ordinal %d out of range", dev);
-        return nullptr;
-    }
+    const int dev = current_device();
+    if (dev < 0) return nullptr;
     std::lock_guard<std::mutex> lock(g_noalloc_mu);
     if (g_noalloc_ptr[dev] == nullptr) {
         void *p = nullptr;
-        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
         if (e != cudaSuccess) {
             cuda_fail(e, "cudaGetSymbolAddress(scratch)");
-            return nullptr;
-        }
-        // Raise the limits to the largest shared-memory size these kernels
-        // accept, so this never lowers a limit another entry point relies on.
-        e = cudaFuncSetAttribute(assign::prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 224 * 1024);
-        if (e == cudaSuccess)
-            e = cudaFuncSetAttribute(assign::scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     224 * 1024);
-        if (e != cudaSuccess) {
-            cuda_fail(e, "cudaFuncSetAttribute(noalloc)");
             return nullptr;
         }
         g_noalloc_ptr[dev] = static_cast<int32_t *>(p);
@@ -968,7 +970,8 @@ int32_t *noalloc_scratch() {
 extern "C" int lb_assign_noalloc(const int32_t *ids, const int32_t *cnt, const void *plan, const int32_t *tok,
                                  const int32_t *mass, int nbatch, int T, int k, int G, int E, int N,
                                  int32_t *dest, int32_t *perm, int32_t *offs, void *stream) {
-    if (nbatch < 1 || nbatch > 65535 || T < 0 || T % G != 0 || k < 1 || k > LB_MAX_K || !plan_shape_ok(G, E, N, 0))
+    // (G is range-checked by plan_shape_ok before T % G is taken)
+    if (nbatch < 1 || nbatch > 65535 || T < 0 || k < 1 || k > LB_MAX_K || !plan_shape_ok(G, E, N, 0) || T % G != 0)
         return LB_EINVAL;
     if (!cnt || !plan || !offs || !aligned(plan, 256)) return LB_EINVAL;
     if (G * N > 0 && (!tok || !mass)) return LB_EINVAL;

@@ -101,6 +101,40 @@ def test_arguments_rejected_before_any_launch(lib):
     assert lib.lb_launch_options(1, 0) == _lib.LB_OK
 
 
+BAD_SHAPES = [(0, 16, 2), (-1, 16, 2), (65, 130, 2), (4, 0, 2), (4, 16, 0)]   # (G, E, k)
+
+
+@pytest.mark.parametrize("G,E,k", BAD_SHAPES)
+def test_bad_rank_expert_or_k_counts_return_einval(lib, G, E, k):
+    """Every compute entry point that takes G, E or k rejects G <= 0, G beyond
+    the maximum, E = 0 and k = 0 with LB_EINVAL before it divides by any of them
+    or launches anything (a divide by G = 0 in the caller's process would end it
+    with SIGFPE).  Each call is made only with a tuple that is invalid for that
+    entry point, so no call can reach a launch."""
+    P, D = ctypes.c_void_p, ctypes.c_double
+    s, T, N, L, a = P(0), 16, 1, 0, P(256)
+    EINVAL = _lib.LB_EINVAL
+    # entry points that take G, E and k
+    assert lib.lb_count(a, 1, T, k, E, G, a, s) == EINVAL
+    assert lib.lb_assign(a, a, a, a, a, 1, T, k, G, E, N, a, a, a, a, 1 << 20, s) == EINVAL
+    assert lib.lb_assign_noalloc(a, a, a, a, a, 1, T, k, G, E, N, a, a, a, s) == EINVAL
+    assert lib.lb_decide(None, a, a, a, 1, T, k, G, E, N, L, 12, a, a, a, a, a, a, a, a, 1 << 20, s) == EINVAL
+    assert lib.lb_decide(a, a, a, a, 1, T, k, G, E, N, L, 12, a, a, a, a, a, a, a, a, 1 << 20, s) == EINVAL
+    assert lib.lb_solve(a, a, 1, T, k, G, E, N, 12, a, a, a, a, a, a, a, a, a, 1 << 20, s) == EINVAL
+    if k > 0:   # entry points that take G and E but no k: the tuple is bad in G or E
+        assert lib.lb_plan_replicas(a, 1, G, E, N, L, a, s) == EINVAL
+        assert lib.lb_split(a, a, 1, G, E, N, 12, a, a, a, a, s) == EINVAL
+        assert lib.lb_plan_swaps(a, None, 1, G, E, D(0), D(0), D(0), D(1), D(0), D(1), D(1), a, a, a, a,
+                                 s) == EINVAL
+        assert lib.lb_split_variant(a, a, 1, G, E, N, 12, 0, a, a, a, a, s) == EINVAL
+    if E == 0 or k == 0:   # the gates take E and k but no G
+        assert lib.lb_predict_topk(a, a, None, 1, T, 64, E, k, a, None, s) == EINVAL
+        assert lib.lb_predict_topk_chain(a, a, None, 2, T, 64, E, k, a, a, None, None, s) == EINVAL
+    if G <= 0 or E <= 0:   # sizes of shapes that cannot exist are zero
+        assert lib.lb_plan_bytes(G, E, N) == 0
+        assert lib.lb_assign_workspace_bytes(1, T, k, G, E, N) == 0
+
+
 def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(_lib, "_lib", None)
     monkeypatch.setattr(_lib, "LIB_PATH", str(tmp_path / "missing.so"))
