@@ -7,8 +7,9 @@ per-rank counts, replica plan, normal gate + top-k, counts, Relief split,
 destinations + stable permutation) over every layer of the workload's model,
 all layers batched into one launch per kernel, replayed from a CUDA graph.
 Inputs (hidden states, gate weights, biases) are resident in HBM before the
-timed region; the per-step hidden-state stream (285 MB for the default
-workload) is larger than the 126 MB L2, so no L2 flush is needed.
+timed region; the per-step hidden-state stream (25.5 GB for the default
+Qwen3-235B-shaped workload, 94 layers) is far larger than the 126 MB L2, so
+no L2 flush is needed.
 
 One JSON line is printed by rank 0.  `value` is whole-job routed
 token-assignments per second (all ranks; each rank runs its own independent
@@ -34,38 +35,57 @@ if ROOT not in sys.path:
 
 METRIC = "routed token-assignments/s and per-layer T_solve (µs); % of HBM roofline"
 UNIT = "token-assignments/s"
-DEFAULT_WORKLOAD = "olmoe"
+DEFAULT_WORKLOAD = "qwen3-235b"
 
 
 def peaks():
+    """(HBM GB/s, bf16 TFLOP/s burst, bf16 TFLOP/s sustained, kind): the
+    pool's measured copy bandwidth and cuBLAS throughput, else the fallback
+    figures measured earlier on this machine."""
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
         with open(path) as f:
             d = json.load(f)
-        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), "measured"
+        burst = float(d["bf16_tflops"])
+        return float(d["hbm_gbs"]), burst, float(d.get("bf16_tflops_sustained", burst)), "measured"
     except Exception:
-        return 6650.0, 1590.0, "fallback"
+        return 6650.0, 1590.0, 1400.0, "fallback"
 
 
-def profile_traffic(kernel_tag, source_files):
-    """Per-launch DRAM bytes from a committed ncu summary, if the kernel's
-    source has not changed since the capture (else None)."""
+GATE_SOURCES = ["moe_expert_load_bf16_b200/csrc/gate_topk.cuh", "moe_expert_load_bf16_b200/csrc/common.cuh"]
+
+
+def source_sha(source_files):
     import hashlib
-    path = os.path.join(ROOT, "profiles", f"{kernel_tag}.md")
-    if not os.path.exists(path):
-        return None
     h = hashlib.sha256()
     for f in source_files:
         with open(os.path.join(ROOT, f), "rb") as fh:
             h.update(fh.read())
-    want = h.hexdigest()[:16]
-    got, traffic = None, None
+    return h.hexdigest()[:16]
+
+
+def profile_traffic(kernel_tag, source_files, units=None):
+    """DRAM bytes of one launch from a committed ncu summary, if the
+    kernel's source has not changed since the capture (else None).  A
+    summary gives either `traffic_bytes_per_launch` (a capture of the same
+    launch) or `traffic_bytes_per_unit` (a capture of a smaller launch of
+    the same kernel, scaled here by the `units` this launch processes)."""
+    path = os.path.join(ROOT, "profiles", f"{kernel_tag}.md")
+    if not os.path.exists(path):
+        return None
+    got, per_launch, per_unit = None, None, None
     for line in open(path):
         if line.startswith("source_sha:"):
             got = line.split(":", 1)[1].strip()
         if line.startswith("traffic_bytes_per_launch:"):
-            traffic = float(line.split(":", 1)[1].strip())
-    return traffic if got == want else None
+            per_launch = float(line.split(":", 1)[1].strip())
+        if line.startswith("traffic_bytes_per_unit:"):
+            per_unit = float(line.split(":", 1)[1].strip())
+    if got != source_sha(source_files):
+        return None
+    if per_unit is not None and units is not None:
+        return per_unit * units
+    return per_launch
 
 
 class ClockSampler:
@@ -271,21 +291,25 @@ def run_ours(args, world, rank, local):
         gate_ms = ev0.elapsed_time(ev1) / args.steps
         gate_bytes = (Lyr + 1) * 2 * T * H + Lyr * (2 * H * E + 4 * E + 2 * 4 * T * k)
         gate_flops = Lyr * 2 * 2.0 * T * H * E
-        tag = "gate_chain_olmoe16"
+        gate_units = Lyr + 1          # hidden states streamed by one launch
+        tag = f"gate_chain_{wl.name}"
     else:
         gate_ms = ev0.elapsed_time(ev1) / (2 * args.steps)
         gate_bytes = Lyr * (2 * T * H + 2 * H * E + 4 * E + 4 * T * k)
         gate_flops = Lyr * 2.0 * T * H * E
-        tag = "gate_topk_olmoe16"
-    hbm, tflops, peak_kind = peaks()
-    achieved = gate_bytes / (gate_ms * 1e-3) / 1e9
-    traffic = profile_traffic(tag, ["moe_expert_load_bf16_b200/csrc/gate_topk.cuh",
-                                    "moe_expert_load_bf16_b200/csrc/common.cuh"])
-    if args.config != "olmoe":
-        traffic = None   # the committed captures are of the OLMoE-shaped launch
+        gate_units = Lyr
+        tag = f"gate_topk_{wl.name}"
+    gate_ms = max_over_ranks(gate_ms, world)
+    hbm, tflops, tflops_sus, peak_kind = peaks()
+    roofline = gate_roofline(gate_bytes, gate_flops, gate_ms, hbm, tflops, tflops_sus, peak_kind,
+                             profile_traffic(tag, GATE_SOURCES, units=gate_units))
+    roofline["kernel"] = "gate_topk_persistent (chain)" if chain else "gate_topk"
 
-    # ---------------- per-layer latencies (single problem, graph replays)
+    # ---------------- per-layer latencies (single problem, graph replays),
+    # this workload's and every other configuration's
     lat = per_layer_latency(wl, hid, W, bias, dev, reps=max(50, args.steps))
+    per_config = per_config_latency(dev, world, wl, lat, reps=max(50, args.steps),
+                                    decode_steps=args.decode_steps)
 
     # ---------------- count / split / assign as throughput kernels
     ints = integer_kernels_at_throughput(dev, world)
@@ -320,14 +344,11 @@ def run_ours(args, world, rank, local):
                        (Lyr + 1 if chain else 2 * Lyr) * T * H * 2 / 1e6),
                    "parallelism": f"{world} independent replicas"},
         "step_latency_us": step_latency_us,
-        "t_solve_us": lat["solve"], "t_solve_fused_us": lat["solve_fused"], "t_split_us": lat["split"],
-        "t_lookahead_us": lat["lookahead"],
+        "t_solve_us": max_over_ranks(lat["solve"], world), "t_solve_fused_us": lat["solve_fused"],
+        "t_split_us": max_over_ranks(lat["split"], world), "t_lookahead_us": lat["lookahead"],
         "per_kernel_us": lat["kernels"],
-        "roofline": {"kernel": "gate_topk_persistent (chain)" if chain else "gate_topk", "bound": "hbm",
-                     "achieved": achieved, "peak": hbm, "unit": "GB/s",
-                     "frac": achieved / hbm, "traffic": traffic, "peak_kind": peak_kind,
-                     "algorithmic_bytes_per_launch": gate_bytes, "launch_us": gate_ms * 1e3,
-                     "tensor_frac": gate_flops / (gate_ms * 1e-3) / (tflops * 1e12)},
+        "roofline": roofline,
+        "per_config": per_config,
         "integer_kernels": ints,
         "swap_planner": swp,
         "e2e": e2e,
@@ -337,6 +358,120 @@ def run_ours(args, world, rank, local):
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline(wl, budget_s=args.cpu_budget)
     return out
+
+
+def gate_roofline(nbytes, flops, ms, hbm, tflops, tflops_sus, peak_kind, traffic):
+    """Roofline of one gate launch: its algorithmic bytes and flops against
+    the measured HBM copy and bf16 tensor peaks.  The bound is the larger of
+    the two minimum times (bytes / HBM peak, flops / tensor peak; burst
+    figures, the launch being timed alone); both fractions are reported,
+    and the tensor fraction against the sustained (power-capped) peak too."""
+    s = ms * 1e-3
+    t_hbm, t_tensor = nbytes / (hbm * 1e9), flops / (tflops * 1e12)
+    out = {"bound": "tensor" if t_tensor > t_hbm else "hbm"}
+    if t_tensor > t_hbm:
+        out.update(achieved=flops / s / 1e12, peak=tflops, unit="TFLOP/s")
+    else:
+        out.update(achieved=nbytes / s / 1e9, peak=hbm, unit="GB/s")
+    out.update(frac=max(t_hbm, t_tensor) / s, traffic=traffic, peak_kind=peak_kind,
+               algorithmic_bytes_per_launch=nbytes, algorithmic_flops_per_launch=flops, launch_us=ms * 1e3,
+               hbm_gbs=nbytes / s / 1e9, hbm_frac=t_hbm / s, tensor_tflops=flops / s / 1e12,
+               tensor_frac=t_tensor / s, tensor_frac_of_sustained=flops / (tflops_sus * 1e12) / s,
+               sustained_tflops=tflops_sus,
+               traffic_over_algorithmic=(traffic / nbytes if traffic else None))
+    return out
+
+
+def per_config_latency(dev, world, main_wl, main_lat, reps, decode_steps=1000):
+    """T_solve, T_split and T_lookahead of one layer of every prefill
+    configuration (the gate applied to that configuration's synthetic hidden
+    states gives the ids), and the decode sweep per step."""
+    from moe_expert_load_bf16_b200 import workloads
+    out = {}
+    for name in ("olmoe", "qwen3-30b", "qwen3-235b"):
+        wl = workloads.WORKLOADS[name]
+        if name == main_wl.name:
+            lat = main_lat
+        else:
+            hid = workloads.hidden_chain(wl, 2, device=dev)
+            W = workloads.gate_weights(wl, 1, device=dev)
+            bias = workloads.biases(wl, 1).to(dev)
+            lat = per_layer_latency(wl, hid, W, bias, dev, reps)
+            del hid, W, bias
+        out[name] = {"shape": f"T={wl.T}, H={wl.H}, E={wl.E}, top-{wl.k}, G={wl.G}, N={wl.N} (L={wl.L})",
+                     "t_solve_us": max_over_ranks(lat["solve"], world),
+                     "t_split_us": max_over_ranks(lat["split"], world),
+                     "t_lookahead_us": max_over_ranks(lat["lookahead"], world),
+                     "per_kernel_us": lat["kernels"]}
+    torch.cuda.empty_cache()
+    out["decode"] = decode_per_step(dev, world, decode_steps)
+    return out
+
+
+def decode_per_step(dev, world, nsteps=1000, chunk=100):
+    """Decode-step sweep: E=256, top-8, G=64 ranks x 4 experts, N=2, T per
+    step in {64, 256, 1024, 4096, 8192}.  `nsteps` consecutive steps with
+    their own synthetic ids (per-step Zipf bias re-drawn with correlation
+    0.5, so the counts shift every step); the plan is made once from step
+    0's counts.  Every step's count + split + assign (lb_count + lb_decide)
+    runs on its own ids, one step after another (graphs of `chunk` steps);
+    T_solve and T_split are the mean per step.  The same steps as one
+    batched launch give the throughput form."""
+    from moe_expert_load_bf16_b200 import _lib, workloads
+    from moe_expert_load_bf16_b200.pipeline import DecisionPath
+    wl = workloads.WORKLOADS["decode"]
+    G, E, N, L, k = wl.G, wl.E, wl.N, wl.L, wl.k
+    res = {"shape": f"E={E}, top-{k}, G={G} ranks x {E // G} experts, N={N} (L={L}); plan from step 0",
+           "steps": nsteps}
+
+    def graphs_of(fns):
+        gs = []
+        for c0 in range(0, len(fns), chunk):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                for f in fns[c0:c0 + chunk]:
+                    f()
+            gs.append(g)
+        return gs
+
+    def run_timed(gs, reps=1):
+        for g in gs:
+            g.replay()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier(world)
+        a.record()
+        for _ in range(reps):
+            for g in gs:
+                g.replay()
+        b.record()
+        torch.cuda.synchronize()
+        return max_over_ranks(a.elapsed_time(b) * 1e3 / reps, world)
+
+    for T in wl.decode_T:
+        path = DecisionPath(nsteps, T, wl.H, E, k, G, N, L, device=dev)
+        for c0 in range(0, nsteps, 100):
+            path.ids[c0:c0 + 100].copy_(workloads.decode_ids(wl.with_(T=T), T, range(c0, min(nsteps, c0 + 100)),
+                                                             device=dev))
+        _lib.lb_count(path.ids[0:1], G, E, cnt=path.cnt_pred[0:1])
+        _lib.lb_plan_replicas(path.cnt_pred[0:1], N, L, plan=path.plan[0:1])
+        path.plan[1:].copy_(path.plan[0:1].expand(nsteps - 1, -1))
+        solve = graphs_of([(lambda b=b: path.solve_one(b)) for b in range(nsteps)])
+        split = graphs_of([(lambda b=b: path.solve_one(b, split_only=True)) for b in range(nsteps)])
+        t_solve = run_timed(solve) / nsteps
+        t_split = run_timed(split) / nsteps
+        gb = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gb):
+            path.solve()
+        t_batch = run_timed([gb], reps=5)
+        if _lib.lb_get_status():
+            raise RuntimeError("device status flagged in the decode sweep")
+        res[str(T)] = {"t_solve_us": t_solve, "t_split_us": t_split,
+                       "assignments_per_s_step_by_step": T * k / (t_solve * 1e-6),
+                       "batched_us": t_batch, "assignments_per_s_batched": nsteps * T * k / (t_batch * 1e-6)}
+        del solve, split, gb, path
+        torch.cuda.empty_cache()
+    return res
 
 
 def per_layer_latency(wl, hid, W, bias, dev, reps):
@@ -501,9 +636,15 @@ def end_to_end(args, wl, hid, W, bias, path, dev, world, chain=True):
     """Same metric through the public API with host buffers: every step
     copies its inputs from pinned host memory and reads its results back."""
     Lyr, T, k = wl.layers, wl.T, wl.k
-    h_host = hid.cpu().pin_memory()
-    w_host = W.cpu().pin_memory()
-    b_host = bias.cpu().pin_memory()
+
+    def pinned_copy(t):
+        # allocated pinned directly (no pageable staging copy of a 25 GB input)
+        hst = torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
+        hst.copy_(t)
+        return hst
+    h_host = pinned_copy(hid)
+    w_host = pinned_copy(W)
+    b_host = pinned_copy(bias)
     outs = (path.dest, path.perm, path.offs, path.loads)
     o_host = [torch.empty(o.shape, dtype=o.dtype).pin_memory() for o in outs]
     h2d = h_host.numel() * 2 + w_host.numel() * 2 + b_host.numel() * 4
@@ -520,10 +661,13 @@ def end_to_end(args, wl, hid, W, bias, path, dev, world, chain=True):
         for o, oh in zip(outs, o_host):
             oh.copy_(o, non_blocking=True)
 
+    t0 = time.perf_counter()
     for _ in range(max(1, args.warmup)):
         step()
     torch.cuda.synchronize()
-    n = max(3, min(args.steps, 20))
+    per = (time.perf_counter() - t0) / max(1, args.warmup)
+    # at least 3 steps, at most 20, about 6 s of copies in all
+    n = max(3, min(args.steps, 20, int(6.0 / max(per, 1e-6))))
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier(world)
     torch.cuda.synchronize()
@@ -534,6 +678,7 @@ def end_to_end(args, wl, hid, W, bias, path, dev, world, chain=True):
     torch.cuda.synchronize()
     barrier(world)
     ms = max_over_ranks(a.elapsed_time(b), world) / n
+    del h_host, w_host, b_host, o_host
     return {"value": Lyr * T * k * world / (ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": int(h2d),
             "d2h_bytes_per_step": int(d2h), "ms_per_step": ms, "steps": n}
 
@@ -623,6 +768,21 @@ def run_decode(args, world, rank, local):
             "per_T": per_T}
 
 # ----------------------------------------------------------------------------- CPU oracle
+_CPU_INPUTS = {}
+
+
+def _cpu_inputs(wl):
+    """One layer's host inputs (two hidden states, its gate and bias as bit
+    patterns), made once per workload."""
+    from moe_expert_load_bf16_b200 import workloads
+    if wl.name not in _CPU_INPUTS:
+        hid = workloads.hidden_chain(wl, 2)
+        hb = [workloads.bf16_bits(hid[0]), workloads.bf16_bits(hid[1])]
+        wb = workloads.bf16_bits(workloads.gate_weights(wl, 1)[0])
+        _CPU_INPUTS[wl.name] = (hb, wb, workloads.biases(wl, 1)[0].numpy())
+    return _CPU_INPUTS[wl.name]
+
+
 def cpu_baseline(wl, budget_s=15.0):
     """The oracle, as it stands, on this host's cores, over whole layers of
     the workload (both gate calls, count, plan, count, split, assign),
@@ -630,13 +790,9 @@ def cpu_baseline(wl, budget_s=15.0):
     the gate runs on evenly spaced sampled rows and its time is scaled to the
     full layer (the integer stages always run on the whole layer)."""
     import oracle
-    from moe_expert_load_bf16_b200 import workloads
     o = oracle.default()
     T, H, E, k, G, N, L = wl.T, wl.H, wl.E, wl.k, wl.G, wl.N, wl.L
-    hid = workloads.hidden_chain(wl, 2)
-    hb = [workloads.bf16_bits(hid[0]), workloads.bf16_bits(hid[1])]
-    wb = workloads.bf16_bits(workloads.gate_weights(wl, 1)[0])
-    b = workloads.biases(wl, 1)[0].numpy()
+    hb, wb, b = _cpu_inputs(wl)
     probe = np.arange(min(T, 64))
     t0 = time.perf_counter()
     o.gate(hb[1][probe], wb, b, k)
@@ -718,6 +874,8 @@ def main():
                     help="chain: one gate pass per hidden state for both gates that read it; two-pass: "
                          "lookahead and normal router as separate passes")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--decode-steps", type=int, default=1000,
+                    help="decode steps per T in the per-step decode sweep of the extra keys")
     ap.add_argument("--lean", action="store_true",
                     help="time the steps only (no gate-only loop, per-layer latencies, end-to-end or CPU "
                          "baseline): the command used for ncu launch lists")

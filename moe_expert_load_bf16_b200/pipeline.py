@@ -80,6 +80,23 @@ class DecisionPath:
                        out=(self.tok, self.mass, self.loads, self.passes_run, self.dest, self.perm, self.offs),
                        workspace=self.ws)
 
+    def solve_one(self, b, split_only=False):
+        """The per-step decision of problem b alone, on views of this path's
+        buffers (its plan must be in place): count + split + assign as
+        lb_count and lb_decide, or the split alone (lb_split, on counts
+        already made)."""
+        s = slice(b, b + 1)
+        if split_only:
+            _lib.lb_split(self.cnt[s], self.plan[s], self.N, self.passes,
+                          out=(self.tok[s], self.mass[s], self.loads[s], self.passes_run[s]))
+            return
+        _lib.lb_count(self.ids[s], self.G, self.E, cnt=self.cnt[s])
+        wsb = _lib.lb_assign_workspace_bytes(1, self.T, self.k, self.G, self.E, self.N)
+        _lib.lb_decide(self.cnt[s], self.ids[s], self.plan[s], self.N, self.passes,
+                       out=(self.tok[s], self.mass[s], self.loads[s], self.passes_run[s], self.dest[s],
+                            self.perm[s], self.offs[s]),
+                       workspace=self.ws[b * wsb:(b + 1) * wsb])
+
     # the same decision as one fused launch (lb_solve)
     def solve_fused(self, ids=None):
         ids = self.ids if ids is None else ids

@@ -1058,7 +1058,7 @@ int orc_split_variant(const int32_t *cnt, int G, int E, const uint8_t *holds, in
                     if (delta > 0) {
                         const int64_t sd = gap > 0 ? delta : -delta;
                         loads[u] -= sd;
-                        loads[v] = loads[v] + sd;
+                        loads[v] += sd;
                         mass[i] -= (int32_t)sd;
                         moved = 1;
                     }
@@ -1182,7 +1182,7 @@ int orc_split_variant(const int32_t *cnt, int G, int E, const uint8_t *holds, in
                 for (int i = round_ptr[r]; i < round_ptr[r + 1]; ++i) {
                     const int u = edge_u[i], v = edge_v[i];
                     const int64_t gap = Lq[u] - Lq[v];
-                    int64_t delta = (gap > 0 ? gap : -gap) >> 1;   /* truncating halve at 2^-f */
+                    int64_t delta = (gap < 0 ? -gap : gap) >> 1;   /* truncating halve at 2^-f */
                     const int64_t limit = gap > 0 ? mq[i] : ((int64_t)tok[i] << f) - mq[i];
                     if (delta > limit) delta = limit;
                     if (delta > 0) {

@@ -22,6 +22,11 @@ import oracle
 from moe_expert_load_bf16_b200 import _lib, workloads
 
 TOL = 1e-2
+# The error the kernel actually shows (fp32 accumulation of exact bf16
+# products, |logit| ~ 1-3) is of order 1e-6; this second, tighter bound makes
+# a regression of the kernel's arithmetic visible long before it reaches the
+# contract above.  It is a regression guard, not the method's tolerance.
+TIGHT = 1e-4
 
 
 def gate_check(h, w, bias, k, ids_gpu, logits_gpu=None, rows=None):
@@ -40,6 +45,7 @@ def gate_check(h, w, bias, k, ids_gpu, logits_gpu=None, rows=None):
         err = np.abs(g_logits.astype(np.float64) - o_logits) / np.maximum(np.abs(o_logits), 1.0)
         max_err = float(err.max()) if err.size else 0.0
         assert max_err <= TOL, f"logit error {max_err}"
+        assert max_err <= TIGHT, f"logit error {max_err}: within the contract, far above the kernel's usual error"
     mism = 0
     for r in range(len(rows)):
         if np.array_equal(g_ids[r], o_ids[r]):

@@ -98,7 +98,7 @@ def test_large_configs(name, layers):
         parity.check_path(path, l, 12)
 
 
-@pytest.mark.parametrize("T", [64, 1024, 8192])
+@pytest.mark.parametrize("T", [64, 256, 1024, 4096, 8192])
 def test_decode_steps(T):
     """Decode sweep shape: plan from step 0, split + assign for several steps."""
     w = workloads.WORKLOADS["decode"]
@@ -188,15 +188,26 @@ def test_gate_ties_lower_id():
     W[7] = W[3]
     W[20] = W[3]
     W[9] = W[1]
-    ids = _lib.lb_predict_topk(h, W, None, k)
+    ids, logits = _lib.lb_predict_topk(h, W, None, k, want_logits=True)
+    # every row within the logit tolerance (ids differ only between near-ties)
+    parity.gate_check(h, W, None, k, ids, logits)
     _, o_ids = oracle.gate(workloads.bf16_bits(h), workloads.bf16_bits(W), None, k)
     got = ids.cpu().numpy()
+    lg = logits.cpu().numpy()
     for r in range(T):
         row = list(got[r])
+        # duplicated rows give bit-identical logits: the lower id ranks first
         for lo, hi in ((3, 7), (3, 20), (7, 20), (1, 9)):
+            assert lg[r, lo] == lg[r, hi]
             if lo in row and hi in row:
                 assert row.index(lo) < row.index(hi)
-    assert (got == o_ids).mean() > 0.99
+            if hi in row:
+                assert lo in row
+        # rows without a near-tie among the kept ids equal the oracle's exactly
+        kth = np.sort(lg[r])[::-1]
+        gaps = np.abs(np.diff(kth[:k + 1]))
+        if (gaps[gaps > 0] > 1e-3 * max(abs(kth[k - 1]), 1.0)).all():
+            assert np.array_equal(got[r], o_ids[r]), r
 
 
 def test_integer_stages_random_shapes():

@@ -1,17 +1,162 @@
-"""CPU checks of the host-side arithmetic of the measurement studies."""
+"""The measurement studies (moe_expert_load_bf16_b200.studies): their host
+arithmetic on hand cases (CPU), and on the GPU the statistics they compute
+from the library's kernels against the same statistics computed from the
+oracle on the same inputs.
+
+Run as a script, this module prints the full Relief ablation table (study 3
+with the oracle's exact optimum):  python tests/test_studies.py [--steps S]
+"""
 import os
 import sys
 
 import numpy as np
+import pytest
+import torch
 
+sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
 sys.path.insert(0, os.path.dirname(os.path.abspath(__file__)))
-import lookahead_study  # noqa: E402
+
+import oracle  # noqa: E402
+import parity  # noqa: E402
+from moe_expert_load_bf16_b200 import studies, workloads  # noqa: E402
 
 
 def test_stale_split_loads_by_hand():
     # fixed [5, 0, 2]; edge 0 (0 -> 1) had kept 30 % at home, edge 1 (2 -> 1) 50 %;
     # the later step's edges carry 10 and 7 tokens: home keeps 3 and 4 (3.5 rounds to even)
-    loads = lookahead_study.stale_loads(np.array([5, 0, 2]), np.array([0, 2]), np.array([1, 1]),
-                                        np.array([10, 7]), np.array([0.3, 0.5]))
+    loads = studies.stale_loads(np.array([5, 0, 2]), np.array([0, 2]), np.array([1, 1]),
+                                np.array([10, 7]), np.array([0.3, 0.5]))
     assert loads.tolist() == [5 + 3, 7 + 3, 2 + 4]
     assert loads.sum() == 5 + 2 + 10 + 7
+
+
+def test_forfeited_share_by_hand():
+    # two ranks, one edge 0 -> 1; three steps.  Without balancing rank 0 carries
+    # fixed + tok; the fresh split levels the two ranks.
+    fixed = np.array([[2, 0], [4, 0], [0, 0]])
+    tok = np.array([[8], [6], [10]])
+    mass = np.array([[3], [1], [5]])            # home keeps 3/8, 1/6, 5/10
+    loads0 = fixed + np.stack([tok[:, 0], 0 * tok[:, 0]], axis=1)   # [10,0], [10,0], [10,0]
+    loads = np.array([[5, 5], [5, 5], [5, 5]])
+    eu, ev = np.array([0]), np.array([1])
+    got = studies.forfeited(loads0, loads, fixed, tok, mass, eu, ev, lags=(1, 2))
+    # lag 1, s=0 -> t=1: home share 3/8 of 6 = 2.25 -> 2: loads [6, 4], gain 4 of 5 -> 0.2 forfeited
+    #        s=1 -> t=2: share 1/6 of 10 = 1.67 -> 2: loads [2, 8], gain 2 of 5 -> 0.6 forfeited
+    # lag 2, s=0 -> t=2: share 3/8 of 10 = 3.75 -> 4: loads [4, 6], gain 4 of 5 -> 0.2 forfeited
+    assert np.allclose(got[1], [0.2, 0.6]) and np.allclose(got[2], [0.2])
+
+
+@pytest.mark.gpu
+def test_lookahead_quality_against_oracle():
+    """Hit rate, logit cosine and rank max-to-mean of the lookahead study
+    against the same statistics from the oracle's gate on the same hidden
+    states (FreeBalance sec. 4, Table 2)."""
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    layers, T = 3, 512
+    w = workloads.WORKLOADS["olmoe"]
+    res = studies.lookahead_quality("olmoe", layers, T=T)
+    t = res["tensors"]
+    wb = [workloads.bf16_bits(t["W"][l]) for l in range(layers)]
+    for l in range(layers):
+        b = t["bias"][l].cpu().numpy()
+        olp, oip = oracle.gate(workloads.bf16_bits(t["hid"][l]), wb[l], b, w.k)
+        ola, oia = oracle.gate(workloads.bf16_bits(t["hid"][l + 1]), wb[l], b, w.k)
+        # the kernel's ids and logits pass the parity check on every row
+        parity.gate_check(t["hid"][l], t["W"][l], t["bias"][l], w.k, t["ids_pred"][l], t["logits_pred"][l])
+        parity.gate_check(t["hid"][l + 1], t["W"][l], t["bias"][l], w.k, t["ids_act"][l], t["logits_act"][l])
+        gip, gia = t["ids_pred"][l].cpu().numpy(), t["ids_act"][l].cpu().numpy()
+        # the study's hit equals a plain recount of the kernel's ids
+        inter = [len(set(gip[r]) & set(gia[r])) for r in range(T)]
+        assert res["per_layer_hit"][l] == pytest.approx(np.mean(inter) / w.k, abs=1e-12)
+        # against the oracle's ids: rows whose ids differ from the oracle's
+        # (near-ties only) can move the hit by the size of the difference
+        o_inter = [len(set(oip[r]) & set(oia[r])) for r in range(T)]
+        slack = sum(len(set(gip[r]) ^ set(oip[r])) // 2 + len(set(gia[r]) ^ set(oia[r])) // 2 for r in range(T))
+        assert abs(np.mean(inter) - np.mean(o_inter)) * T <= slack
+        # cosine of the logits: the oracle's in double vs the study's
+        num = (olp * ola).sum(1)
+        den = np.linalg.norm(olp, axis=1) * np.linalg.norm(ola, axis=1)
+        assert res["per_layer_cosine"][l] == pytest.approx(float(np.mean(num / den)), abs=1e-6)
+        # rank max-to-mean of the predicted counts (even placement)
+        cnt = oracle.count(gip, w.G, w.E).sum(axis=0).reshape(w.G, -1).sum(axis=1)
+        assert studies.rank_max_to_mean(t["cnt_pred"][l], w.G) == pytest.approx(cnt.max() / cnt.mean(), rel=1e-12)
+    assert 0.0 < res["hit_min"] <= res["hit_mean"] <= 1.0
+    assert 0.9 < res["cosine_min"] <= res["cosine_mean"] <= 1.0
+
+
+@pytest.mark.gpu
+def test_decision_frequency_against_oracle_split():
+    """The stale-split study (Relief, Failure of Existing Approaches): the
+    per-step loads without balancing and with the fresh split, and every
+    forfeited share, recomputed from the oracle's count, plan and split of the
+    same decode steps plus the host re-split."""
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    G, E, N, steps, T = 16, 128, 8, 6, 512
+    lags = (1, 2, 4)
+    res = studies.decision_frequency(G, E, N, steps=steps, T=T, lags=lags)
+    raw = res["raw"]
+    ids = raw["ids"].cpu().numpy()
+    p = oracle.plan(oracle.count(ids[0], G, E), N, raw["L"])
+    ne = p.n_edges
+    eu, ev = p.edge_u[:ne], p.edge_v[:ne]
+    tok, mass, loads, loads0, fixed = [], [], [], [], []
+    for s in range(1, steps + 1):
+        c = oracle.count(ids[s], G, E)
+        sp, s0 = oracle.split(c, p, 12), oracle.split(c, p, 0)
+        tok.append(sp.tok[:ne])
+        mass.append(sp.mass[:ne])
+        loads.append(sp.loads)
+        loads0.append(s0.loads)
+        f = s0.loads.astype(np.int64).copy()
+        np.subtract.at(f, eu, sp.tok[:ne])
+        fixed.append(f)
+    assert np.array_equal(np.array(loads), raw["loads"].astype(np.int64))
+    assert np.array_equal(np.array(loads0), raw["loads0"].astype(np.int64))
+    want = studies.forfeited(np.array(loads0), np.array(loads), np.array(fixed), np.array(tok), np.array(mass),
+                             eu, ev, lags)
+    for r in lags:
+        assert np.allclose(raw["values"][r], want[r], rtol=0, atol=0), r
+
+
+@pytest.mark.gpu
+def test_ablation_against_exact_optimum():
+    """Relief's ablation at a small size: no variant's max load is below the
+    exact per-step optimum (attainment <= 1), Relief with 12 passes reaches
+    the pages' software figure (93 % of the optimum), and its attainment
+    never falls as passes are added (a move never raises the larger of its
+    two loads)."""
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    G, E, N, steps = 16, 128, 8, 3
+
+    def optimum(c0, cs):
+        return oracle.split_optimum(cs, oracle.plan(c0, N, N // 2))
+    res = studies.ablation("qwen3-30b-shaped", G, E, steps, optimum, T=1024, N=N, max_passes=12, timing=False)
+    for v, row in res["variants"].items():
+        assert row["attainment"] <= 1.0 + 1e-12, v
+        assert all(m >= o for m, o in zip(row["max_load"], res["optimum"])), v
+    assert res["variants"]["relief"]["attainment"] >= 0.93
+    curve = res["relief_attainment_by_passes"]
+    assert all(b >= a - 1e-12 for a, b in zip(curve, curve[1:]))
+    assert curve[12] == pytest.approx(res["variants"]["relief"]["attainment"], abs=1e-12)
+
+
+def _ablation_table(steps):
+    import json
+
+    def opt_for(N, L):
+        return lambda c0, cs: oracle.split_optimum(cs, oracle.plan(c0, N, L))
+    res = {}
+    for N in (2, 8):
+        res[f"G16_N{N}"] = studies.ablation("qwen3-30b-shaped", 16, 128, steps, opt_for(N, N // 2), N=N)
+        res[f"G64_N{N}"] = studies.ablation("decode-shaped", 64, 256, steps, opt_for(N, N // 2), N=N)
+    print(json.dumps(res, indent=1))
+
+
+if __name__ == "__main__":
+    import argparse
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--steps", type=int, default=8)
+    _ablation_table(ap.parse_args().steps)
