@@ -615,7 +615,7 @@ def integer_kernels_at_throughput(dev, world, nbatch=128, reps=20):
                                             out=(path.dest, path.perm, path.offs), workspace=path.ws))
     if _lib.lb_get_status():
         raise RuntimeError("device status flagged in the integer-kernel run")
-    hbm, _, _ = peaks()
+    hbm = peaks()[0]
     tk = T * k
     by = {"count": nbatch * (4 * tk + 4 * G * E),
           "split": int(nbatch * (4 * G * E + 12 * n_edges + 16 * G * N + 4 * G)),
