@@ -122,15 +122,20 @@ int lb_predict_topk_chain(const void *h, const void *w, const float *bias,
  * CTA's shared memory holds); split of H across a
  * CTA cluster (1, 2, 4, 8 or 16); persistent kernel (1, 2 or 4 = that many
  * CTAs per SM walking the token tiles with a TMEM accumulator, double-
- * buffered where TMEM allows; -1 = one CTA per tile); 64-column boxes per
+ * buffered where TMEM allows; 3 = CTA pairs: clusters of two CTAs, one per
+ * SM, sharing one MMA of M = 256 over 256-token work units, each CTA
+ * loading its 128 tokens and half of the MMA's N weight rows, k <= 8;
+ * -1 = one CTA per tile); 64-column boxes per
  * pipeline stage of the persistent kernel (1, 2 or 4); token tiles per work
  * unit of the persistent kernel (1 or 2: two tiles share every W box, each
  * with its own accumulator, halving W's L2 traffic); at most max_ctas CTAs
  * in the persistent kernel's grid (0 = its CTAs per SM on every SM; fewer
  * leave SMs to kernels that run beside it on other streams).
- * Automatic: with at least two token tiles per SM and E <= 128, persistent
- * with two CTAs per SM (one when two double-buffered accumulators of the
- * MMA's N do not fit TMEM twice) and one tile per unit; otherwise one CTA
+ * Automatic: lb_predict_topk_chain with E = 128 (N = 256) and k <= 8 runs
+ * CTA pairs; otherwise, with at least two token tiles per SM and E <= 128,
+ * persistent with two CTAs per SM (one when two double-buffered
+ * accumulators of the MMA's N do not fit TMEM twice) and one tile per unit;
+ * otherwise one CTA
  * per tile, H split across a cluster until the GPU is filled when the tiles
  * alone do not fill it.  Results do not depend on the knobs beyond fp32 rounding of
  * split-H partial sums.  LB_EINVAL for values out of range. */

@@ -400,10 +400,21 @@ __device__ __forceinline__ void merge_sorted(uint32_t (&key)[KMAX], const uint32
     }
 }
 
-template <int KMAX, int ES, int MP>
+// PAIR: the CTAs of each cluster of two share one MMA of M = 256 (see the
+// CTA-pair helpers in common.cuh).  A work unit is then two consecutive
+// 128-token tiles, one per CTA; each CTA loads its own h rows and half of
+// the unit's B rows (chain mode: CTA 0 the gate W_{b-1}, CTA 1 the gate W_b),
+// so every W byte crosses into one SM per unit instead of two.  Rank 0's
+// producer expects the bytes of both CTAs' loads on its own full barrier
+// (rank 1's loads complete there), rank 0's MMA warp issues every MMA and
+// commits to the stage-free and accumulator-full barriers of both CTAs, and
+// the epilogue warps of both CTAs release an accumulator buffer on rank 0's
+// empty barrier.  Each CTA ranks its own 128 rows.  (MP = 1, ES = 4.)
+template <int KMAX, int ES, int MP, bool PAIR = false>
 __global__ void __launch_bounds__(Shape<ES>::THREADS, ES == 2 ? 2 : 1)
     gate_topk_persistent(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                          const Params p, int mtiles, int ntiles) {
+    static_assert(!PAIR || (MP == 1 && ES == 4), "CTA pairs: one tile per CTA and sixteen epilogue warps");
     extern __shared__ uint8_t smem_raw[];
     pdl_begin();
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -426,8 +437,12 @@ __global__ void __launch_bounds__(Shape<ES>::THREADS, ES == 2 ? 2 : 1)
     __shared__ uint32_t merge_k[4][MLISTS][KMAX][32];
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const uint32_t a_box = BM * 128u, b_box = static_cast<uint32_t>(p.Epad) * 128u;
+    const uint32_t a_box = BM * 128u, b_box = static_cast<uint32_t>(PAIR ? p.Epad / 2 : p.Epad) * 128u;
     const int kbox = p.kbox;
+    // work units: PAIR walks units of two tiles per cluster, else one per CTA
+    const int crank = PAIR ? static_cast<int>(cluster_ctarank()) : 0;
+    const int ufirst = PAIR ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
+    const int ustep = PAIR ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
     const uint32_t a_bytes = a_box * kbox * MP;         // A boxes first (M-tile by M-tile), then B boxes
     const uint32_t stage_bytes = (a_box * MP + b_box) * kbox;
     const int stages = p.stages;
@@ -442,7 +457,8 @@ __global__ void __launch_bounds__(Shape<ES>::THREADS, ES == 2 ? 2 : 1)
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&acc_full[i], 1);
-            mbar_init(&acc_empty[i], Shape<ES>::EPI);
+            // PAIR: one arrival per epilogue warp of both CTAs (on rank 0's)
+            mbar_init(&acc_empty[i], PAIR ? 2 * (Shape<ES>::EPI / 32) : Shape<ES>::EPI);
         }
         mbar_init(&drain_bar, 1);
         aborted = 0;
@@ -451,14 +467,25 @@ __global__ void __launch_bounds__(Shape<ES>::THREADS, ES == 2 ? 2 : 1)
         tma_prefetch_desc(&tmB);
     }
     if (warp == 1) {
-        tmem_alloc(&tmem_slot, p.tmem_cols);
-        tmem_relinquish();
+        if constexpr (PAIR) {
+            tmem_alloc_pair(&tmem_slot, p.tmem_cols);
+            tmem_relinquish_pair();
+        } else {
+            tmem_alloc(&tmem_slot, p.tmem_cols);
+            tmem_relinquish();
+        }
     }
     tc_fence_before();
     __syncthreads();
+    // PAIR: both CTAs' barriers are initialized and their TMEM allocated
+    // before either signals the other
+    if constexpr (PAIR) cluster_sync();
     tc_fence_after();
     const uint32_t tmem = tmem_slot;
     volatile int *abort_flag = &aborted;
+    // rank 0's copies of the barriers every CTA of the pair signals
+    const uint32_t full0 = PAIR ? mapa_shared(smem_u32(&full_bar[0]), 0) : smem_u32(&full_bar[0]);
+    const uint32_t accempty0 = PAIR ? mapa_shared(smem_u32(&acc_empty[0]), 0) : smem_u32(&acc_empty[0]);
 
     if (warp == 0) {
         if (lane == 0) {
@@ -466,8 +493,9 @@ __global__ void __launch_bounds__(Shape<ES>::THREADS, ES == 2 ? 2 : 1)
             const uint64_t pol_a = l2_policy_evict_first(), pol_b = l2_policy_evict_last();
             int it = 0;
             bool ok = true;
-            for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
-                const int b = tile / mtiles, m0 = (tile - b * mtiles) * BM * MP;
+            for (int tile = ufirst; tile < ntiles && ok; tile += ustep) {
+                const int b = tile / mtiles;
+                const int m0 = PAIR ? (tile - b * mtiles) * 2 * BM + crank * BM : (tile - b * mtiles) * BM * MP;
                 for (int ks = 0; ks < nks; ++ks, ++it) {
                     const int s = it % stages;
                     const uint32_t ph = (it / stages) & 1;
@@ -478,31 +506,48 @@ __global__ void __launch_bounds__(Shape<ES>::THREADS, ES == 2 ? 2 : 1)
                         break;
                     }
                     uint8_t *sa = smem + static_cast<size_t>(s) * stage_bytes;
-                    mbar_arrive_expect_tx(&full_bar[s], stage_bytes);
-#pragma unroll
-                    for (int mt = 0; mt < MP; ++mt)
+                    if constexpr (PAIR) {
+                        // rank 0 expects both CTAs' bytes; each CTA loads its
+                        // own h rows and its half of the B rows
+                        if (crank == 0) mbar_arrive_expect_tx(&full_bar[s], 2 * stage_bytes);
+                        const uint32_t fb = full0 + static_cast<uint32_t>(s) * 8u;
                         for (int j = 0; j < kbox; ++j)
-                            tma_load_3d_hint(&tmA, sa + (mt * kbox + j) * a_box, &full_bar[s], (ks * kbox + j) * BK,
-                                             m0 + mt * BM, b, pol_a);
-                    const int by = p.chain ? (b - 1) * p.E : 0, bz = p.chain ? 0 : b;
-                    for (int j = 0; j < kbox; ++j)
-                        tma_load_3d_hint(&tmB, sa + a_bytes + j * b_box, &full_bar[s], (ks * kbox + j) * BK, by, bz,
-                                         pol_b);
+                            tma_load_3d_pair(&tmA, sa + j * a_box, fb, (ks * kbox + j) * BK, m0, b, pol_a);
+                        const int half = p.Epad / 2;
+                        const int by = (p.chain ? (b - 1) * p.E : 0) + crank * half, bz = p.chain ? 0 : b;
+                        for (int j = 0; j < kbox; ++j)
+                            tma_load_3d_pair(&tmB, sa + a_bytes + j * b_box, fb, (ks * kbox + j) * BK, by, bz, pol_b);
+                    } else {
+                        mbar_arrive_expect_tx(&full_bar[s], stage_bytes);
+#pragma unroll
+                        for (int mt = 0; mt < MP; ++mt)
+                            for (int j = 0; j < kbox; ++j)
+                                tma_load_3d_hint(&tmA, sa + (mt * kbox + j) * a_box, &full_bar[s],
+                                                 (ks * kbox + j) * BK, m0 + mt * BM, b, pol_a);
+                        const int by = p.chain ? (b - 1) * p.E : 0, bz = p.chain ? 0 : b;
+                        for (int j = 0; j < kbox; ++j)
+                            tma_load_3d_hint(&tmB, sa + a_bytes + j * b_box, &full_bar[s], (ks * kbox + j) * BK, by,
+                                             bz, pol_b);
+                    }
                 }
             }
-            // no copies left in flight into this CTA's shared memory
-            for (int s = 0; s < stages && s < it; ++s) {
-                const int last = s + ((it - 1 - s) / stages) * stages;
-                if (!mbar_wait(&full_bar[s], (last / stages) & 1)) flag(LB_DEV_TIMEOUT);
+            // no copies left in flight into this CTA's shared memory (PAIR:
+            // rank 0's full barriers count both CTAs' copies; rank 1 is held
+            // at the closing cluster barrier until rank 0 has seen them land)
+            if (!PAIR || crank == 0) {
+                for (int s = 0; s < stages && s < it; ++s) {
+                    const int last = s + ((it - 1 - s) / stages) * stages;
+                    if (!mbar_wait(&full_bar[s], (last / stages) & 1)) flag(LB_DEV_TIMEOUT);
+                }
             }
         }
     } else if (warp == 1) {
-        if (lane == 0) {
-            // ---------------- MMA issuer
-            const uint32_t idesc = umma_idesc_bf16(BM, p.Epad);
+        if (lane == 0 && (!PAIR || crank == 0)) {
+            // ---------------- MMA issuer (PAIR: rank 0 only)
+            const uint32_t idesc = umma_idesc_bf16(PAIR ? 2 * BM : BM, p.Epad);
             int it = 0, tl = 0;
             bool ok = true;
-            for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x, ++tl) {
+            for (int tile = ufirst; tile < ntiles && ok; tile += ustep, ++tl) {
                 const int buf = tl % nbuf;
                 const uint32_t use = static_cast<uint32_t>(tl / nbuf);
                 if (!mbar_wait(&acc_empty[buf], (use & 1) ^ 1) || *abort_flag) {
@@ -529,18 +574,26 @@ __global__ void __launch_bounds__(Shape<ES>::THREADS, ES == 2 ? 2 : 1)
                         for (int mt = 0; mt < MP; ++mt) {
                             const uint32_t sa = st + (mt * kbox + j) * a_box;
 #pragma unroll
-                            for (int kk = 0; kk < BK / UK; ++kk)
-                                umma_bf16(d + mt * static_cast<uint32_t>(p.Epad), sw128_kmajor_desc(sa + kk * UK * 2),
-                                          sw128_kmajor_desc(sb + kk * UK * 2), idesc,
-                                          (ks > 0 || j > 0 || kk > 0) ? 1u : 0u);
+                            for (int kk = 0; kk < BK / UK; ++kk) {
+                                const uint32_t acc = (ks > 0 || j > 0 || kk > 0) ? 1u : 0u;
+                                if constexpr (PAIR)
+                                    umma_bf16_pair(d, sw128_kmajor_desc(sa + kk * UK * 2),
+                                                   sw128_kmajor_desc(sb + kk * UK * 2), idesc, acc);
+                                else
+                                    umma_bf16(d + mt * static_cast<uint32_t>(p.Epad), sw128_kmajor_desc(sa + kk * UK * 2),
+                                              sw128_kmajor_desc(sb + kk * UK * 2), idesc, acc);
+                            }
                         }
                     }
-                    umma_commit(&empty_bar[s]);
+                    if constexpr (PAIR) umma_commit_pair(&empty_bar[s], 3);
+                    else umma_commit(&empty_bar[s]);
                 }
-                umma_commit(&acc_full[buf]);
+                if constexpr (PAIR) umma_commit_pair(&acc_full[buf], 3);
+                else umma_commit(&acc_full[buf]);
             }
             // every MMA this CTA issued has finished before TMEM is freed
-            umma_commit(&drain_bar);
+            if constexpr (PAIR) umma_commit_pair(&drain_bar, 1);
+            else umma_commit(&drain_bar);
             if (!mbar_wait(&drain_bar, 0)) flag(LB_DEV_TIMEOUT);
         }
     } else {
@@ -573,10 +626,11 @@ __global__ void __launch_bounds__(Shape<ES>::THREADS, ES == 2 ? 2 : 1)
         const int mbase = (mt * NG + gate_id) * (GP - 1);  // this (M-tile, gate)'s hand-over lists
         const int mslot = mbase + part - 1;                 // this warp's list (part > 0)
         int tl = 0;
-        for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++tl) {
+        for (int tile = ufirst; tile < ntiles; tile += ustep, ++tl) {
             const int buf = tl % nbuf;
             const uint32_t use = static_cast<uint32_t>(tl / nbuf);
-            const int b = tile / mtiles, m0 = (tile - b * mtiles) * BM * MP + mt * BM;
+            const int b = tile / mtiles;
+            const int m0 = PAIR ? (tile - b * mtiles) * 2 * BM + crank * BM : (tile - b * mtiles) * BM * MP + mt * BM;
             // The layer this warp's columns belong to (uniform over the tile).
             const int layer = p.chain ? b - 1 + gate_id : b;
             const bool live = layer >= 0 && (!p.chain || layer < p.L);   // the gate has a layer here
@@ -642,7 +696,12 @@ __global__ void __launch_bounds__(Shape<ES>::THREADS, ES == 2 ? 2 : 1)
             }
             // this warp's TMEM reads are done: the buffer may be overwritten
             tc_fence_before();
-            mbar_arrive(&acc_empty[buf]);
+            if constexpr (PAIR) {
+                __syncwarp();
+                if (lane == 0) mbar_arrive_cluster(accempty0 + static_cast<uint32_t>(buf) * 8u);
+            } else {
+                mbar_arrive(&acc_empty[buf]);
+            }
             if (GP > 1) {
                 if (part > 0) {
 #pragma unroll
@@ -670,9 +729,13 @@ __global__ void __launch_bounds__(Shape<ES>::THREADS, ES == 2 ? 2 : 1)
 
     tc_fence_before();
     __syncthreads();
+    // PAIR: neither CTA leaves (or frees TMEM) while the other may still
+    // signal its barriers, read its TMEM or be written by its copies
+    if constexpr (PAIR) cluster_sync();
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem, p.tmem_cols);
+        if constexpr (PAIR) tmem_dealloc_pair(tmem, p.tmem_cols);
+        else tmem_dealloc(tmem, p.tmem_cols);
     }
 }
 

@@ -231,9 +231,92 @@ size_t persistent_static_smem(int k) {
     return 64 * 1024;
 }
 
+template <int KMAX>
+size_t static_smem_pair_of() {
+    cudaFuncAttributes a{};
+    return cudaFuncGetAttributes(&a, gate::gate_topk_persistent<KMAX, 4, 1, true>) == cudaSuccess ? a.sharedSizeBytes
+                                                                                                 : 64 * 1024;
+}
+
+size_t persistent_static_smem_pair(int k) {
+    if (k <= 2) return static_smem_pair_of<2>();
+    if (k <= 4) return static_smem_pair_of<4>();
+    return static_smem_pair_of<8>();
+}
+
 size_t persistent_static_smem(int k, int es, int mp) {
     if (es == 4) return mp == 2 ? persistent_static_smem<4, 2>(k) : persistent_static_smem<4, 1>(k);
     return mp == 2 ? persistent_static_smem<2, 2>(k) : persistent_static_smem<2, 1>(k);
+}
+
+// CTA-pair launch of the persistent gate (clusters of two CTAs sharing one
+// MMA of M = 256; sixteen epilogue warps, k <= 8).
+template <int KMAX>
+int launch_gate_pair(const CUtensorMap &ma, const CUtensorMap &mb, const gate::Params &p, int units, int nunits,
+                     int grid, size_t smem, cudaStream_t s) {
+    auto kern = gate::gate_topk_persistent<KMAX, 4, 1, true>;
+    static SmemLimit lim;
+    if (!allow_smem(kern, lim, smem, false)) return LB_ECUDA;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid, 1, 1);
+    cfg.blockDim = dim3(gate::Shape<4>::THREADS, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, ma, mb, p, units, nunits);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaLaunchKernelEx(gate_topk pair)");
+    return launched("gate_topk pair");
+}
+
+// Persistent gate over CTA pairs: work units of 256 tokens (one 128-token
+// tile per CTA), each CTA loading half of the N = Epad B rows, so the map
+// `mb` has boxes of Epad/2 rows.  One CTA per SM; TMEM holds two
+// accumulators of Epad columns.
+int run_pair(gate::Params &p, const void *h, int nprob, const CUtensorMap &mb, int sms, cudaStream_t s) {
+    if (p.k > 8 || p.Epad % 16 != 0 || p.Epad < 16 || p.Epad > 256) return LB_EINVAL;
+    uint32_t pcols = 32;
+    while (pcols < 2u * static_cast<uint32_t>(p.Epad)) pcols <<= 1;
+    if (pcols > 512) return LB_EINVAL;
+    p.tmem_cols = pcols;
+    p.nbuf = 2;
+    p.split = 1;
+    const size_t stat = persistent_static_smem_pair(p.k);
+    const size_t room = 227 * 1024 - stat - 2048;
+    const size_t box_bytes = 16384 + static_cast<size_t>(p.Epad / 2) * 128;
+    p.kbox = g_tune_kbox ? g_tune_kbox : 2;
+    if (p.kbox * box_bytes * 2 + 1024 > std::min<size_t>(224 * 1024, room + 1024)) p.kbox = 1;
+    const size_t stage_bytes = box_bytes * p.kbox;
+    const size_t fit = std::min<size_t>(224 * 1024 - 1024, room) / stage_bytes;
+    int stages = static_cast<int>(std::min<size_t>(gate::MAX_STAGES, fit));
+    if (g_tune_stages) stages = std::min(stages, g_tune_stages);
+    if (stages < 2) return LB_EINVAL;
+    // at least half the SM's shared memory: one CTA per SM (TMEM)
+    size_t smem = std::max(stages * stage_bytes + 1024, static_cast<size_t>(115 * 1024));
+    if (smem > std::min<size_t>(224 * 1024, room + 1024)) return LB_EINVAL;
+    p.stages = stages;
+    CUtensorMap ma;
+    if (!make_map(&ma, h, static_cast<uint64_t>(p.H), static_cast<uint64_t>(p.T), static_cast<uint64_t>(nprob),
+                  gate::BM)) {
+        std::snprintf(g_last_error, sizeof g_last_error, "cuTensorMapEncodeTiled failed for h");
+        return LB_ECUDA;
+    }
+    const int units = (p.T + 2 * gate::BM - 1) / (2 * gate::BM);
+    const long long nunits = static_cast<long long>(units) * nprob;
+    long long cap = sms / 2;
+    if (g_tune_max_ctas > 0) cap = std::min<long long>(cap, g_tune_max_ctas / 2);
+    if (nunits < 1 || cap < 1 || nunits > INT_MAX) return LB_EINVAL;
+    const long long rounds = (nunits + cap - 1) / cap;
+    const int grid = 2 * static_cast<int>((nunits + rounds - 1) / rounds);
+    const int nu = static_cast<int>(nunits);
+    if (p.k <= 2) return launch_gate_pair<2>(ma, mb, p, units, nu, grid, smem, s);
+    if (p.k <= 4) return launch_gate_pair<4>(ma, mb, p, units, nu, grid, smem, s);
+    return launch_gate_pair<8>(ma, mb, p, units, nu, grid, smem, s);
 }
 
 // Persistent gate launch shared by lb_predict_topk and lb_predict_topk_chain:
@@ -426,7 +509,8 @@ int lb_gate_tuning(int stages, int split, int persistent, int kbox, int tiles_pe
     if (kbox != 0 && kbox != 1 && kbox != 2 && kbox != 4) return LB_EINVAL;
     if (stages != 0 && (stages < 2 || stages > gate::MAX_STAGES)) return LB_EINVAL;
     if (split != 0 && split != 1 && split != 2 && split != 4 && split != 8 && split != 16) return LB_EINVAL;
-    if (persistent != -1 && persistent != 0 && persistent != 1 && persistent != 2 && persistent != 4)
+    if (persistent != -1 && persistent != 0 && persistent != 1 && persistent != 2 && persistent != 3 &&
+        persistent != 4)
         return LB_EINVAL;
     g_tune_stages = stages;
     g_tune_split = split;
@@ -474,6 +558,16 @@ int lb_predict_topk(const void *h, const void *w, const float *bias, int nbatch,
     // per tile.
     int per_sm = g_tune_persistent;
     if (per_sm == 0 && g_tune_split <= 1 && ntiles >= 2LL * sms && p.Epad <= 128) per_sm = 2;
+    if (per_sm == 3) {
+        CUtensorMap mb;
+        if (p.Epad % 16 != 0 ||
+            !make_map(&mb, w, static_cast<uint64_t>(H), static_cast<uint64_t>(E), static_cast<uint64_t>(nbatch),
+                      static_cast<uint32_t>(p.Epad / 2))) {
+            std::snprintf(g_last_error, sizeof g_last_error, "cuTensorMapEncodeTiled failed for w");
+            return LB_ECUDA;
+        }
+        return run_pair(p, h, nbatch, mb, sms, s);
+    }
     if (per_sm > 0) {
         CUtensorMap mb;
         if (!make_map(&mb, w, static_cast<uint64_t>(H), static_cast<uint64_t>(E), static_cast<uint64_t>(nbatch),
@@ -577,6 +671,22 @@ int lb_predict_topk_chain(const void *h, const void *w, const float *bias, int L
     uint32_t pcols = 32;
     while (pcols < 4u * static_cast<uint32_t>(E)) pcols <<= 1;
     int per_sm = g_tune_persistent > 0 ? g_tune_persistent : std::max(1, std::min(2, static_cast<int>(512 / pcols)));
+    // Automatic: CTA pairs when the two gates fill the MMA's N = 256 (E = 128;
+    // measured: Qwen3-235B-shaped chain 964 against 1124 us for 16 layers,
+    // Qwen3-30B-shaped 293 against 332 us), where one CTA would stream a
+    // weight box twice the size of its h box; one CTA per tile below that
+    // (OLMoE-shaped, N = 128: 62 against 72 us).
+    if (g_tune_persistent == 0 && 2 * E >= 256 && k <= 8) per_sm = 3;
+    if (per_sm == 3) {
+        // CTA pairs: each CTA loads one gate, a box of E rows starting at row
+        // (b-1)E (CTA 0) or bE (CTA 1)
+        CUtensorMap mb;
+        if (!make_map(&mb, w, static_cast<uint64_t>(H), static_cast<uint64_t>(L) * E, 1, static_cast<uint32_t>(E))) {
+            std::snprintf(g_last_error, sizeof g_last_error, "cuTensorMapEncodeTiled failed for w");
+            return LB_ECUDA;
+        }
+        return run_pair(p, h, L + 1, mb, sms, s);
+    }
     // the stack of gates as one [L*E, H] matrix; a box of 2E rows starting
     // at row (b-1)E (negative for b = 0, past the end for b = L: zeros)
     CUtensorMap mb;

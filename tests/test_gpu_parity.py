@@ -792,3 +792,55 @@ def test_gate_two_tiles_per_unit(chain, tpu, persistent, E):
         parity.gate_check(src, w_, b_, k, ids_, lg_, rows=rows)
         ref = _lib.lb_predict_topk(src, w_, b_, k)
         assert (ref == ids_).all(dim=1).float().mean().item() > 0.999
+
+
+@pytest.mark.parametrize("chain", [True, False])
+@pytest.mark.parametrize("T,H,E,k,B,bias_on", [(4096, 2048, 128, 8, 3, True), (1100, 576, 64, 8, 2, True),
+                                               (300, 128, 16, 2, 2, False), (2900, 4096, 128, 4, 1, True),
+                                               (130, 64, 48, 8, 3, True)])
+def test_gate_cta_pairs(chain, T, H, E, k, B, bias_on):
+    """CTA pairs (clusters of two CTAs sharing one MMA of M = 256, each CTA
+    loading its 128 tokens and half of the weight rows): ids and logits of
+    every problem pass the oracle check on sampled rows (all rows of short
+    problems), and agree with the one-CTA persistent kernel.  Shapes: an odd
+    number of 128-token tiles (the last unit's second tile lies past T), a
+    ragged tail, H past the last full stage of boxes, E = 16 (N = 32 chain),
+    E = 48 (N = 48 per gate), no bias."""
+    if not chain and E % 16:
+        pytest.skip("pairs need E % 16 == 0 in the per-layer gate")
+    g = torch.Generator(device=DEV).manual_seed(T + H + E + k + B)
+    nh = B + 1 if chain else B
+    h = torch.randn(nh, T, H, generator=g, device=DEV).to(torch.bfloat16)
+    W = (torch.randn(B, E, H, generator=g, device=DEV) / H ** 0.5).to(torch.bfloat16)
+    bias = torch.randn(B, E, generator=g, device=DEV) if bias_on else None
+    _lib.lb_gate_tuning(0, 0, 3)
+    if chain:
+        out = _lib.lb_predict_topk_chain(h, W, bias, k, want_logits=True)
+    else:
+        out = _lib.lb_predict_topk(h, W, bias, k, want_logits=True)
+    torch.cuda.synchronize()
+    assert _lib.lb_get_status() == 0
+    _lib.lb_gate_tuning(0, 0, 1)
+    ref = (_lib.lb_predict_topk_chain(h, W, bias, k, want_logits=True) if chain else
+           _lib.lb_predict_topk(h, W, bias, k, want_logits=True))
+    torch.cuda.synchronize()
+    _lib.lb_gate_tuning()
+    rng = np.random.default_rng(T + E)
+    rows = None if T <= 512 else np.unique(np.concatenate([rng.choice(T, 64, replace=False),
+                                                           [0, 127, 128, 255, 256, T - 1]]))
+    if chain:
+        ip, ia, lp, la = out
+        pairs = [(h[l], W[l], None if bias is None else bias[l], ip[l], lp[l]) for l in range(B)] + \
+                [(h[l + 1], W[l], None if bias is None else bias[l], ia[l], la[l]) for l in range(B)]
+        for a_, r_ in zip(out, ref):
+            if a_.dtype == torch.int32:
+                assert (a_ == r_).all(dim=-1).float().mean().item() > 0.999
+            else:
+                assert torch.allclose(a_, r_, rtol=1e-5, atol=1e-5)
+    else:
+        ids, lg = out
+        pairs = [(h[b], W[b], None if bias is None else bias[b], ids[b], lg[b]) for b in range(B)]
+        assert (ids == ref[0]).all(dim=-1).float().mean().item() > 0.999
+        assert torch.allclose(lg, ref[1], rtol=1e-5, atol=1e-5)
+    for src, w_, b_, ids_, lg_ in pairs:
+        parity.gate_check(src, w_, b_, k, ids_, lg_, rows=rows)
