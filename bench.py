@@ -767,6 +767,83 @@ def run_decode(args, world, rank, local):
                        "T": list(wl.decode_T), "steps_per_launch": B},
             "per_T": per_T}
 
+# ----------------------------------------------------------------------------- one kernel
+def run_kernel(args, local):
+    """One kernel of the path alone, for timing and for ncu: `--launches`
+    plain launches (a profiler picks one with -k/-s/-c), then the mean of 20
+    graph replays.  gate: the chain gate over `--problems` layers of the
+    workload (its default: all); count, plan, split, assign: one launch over
+    `--problems` independent problems of the workload's shape (T, k, E, G, N)
+    with decode-style synthetic ids (`--problems` default 128)."""
+    from moe_expert_load_bf16_b200 import _lib, build, workloads
+    from moe_expert_load_bf16_b200.pipeline import DecisionPath
+    build.build()
+    wl = workloads.WORKLOADS[args.config]
+    dev = torch.device("cuda", local)
+    T, H, E, k, G, N, L = wl.T, wl.H, wl.E, wl.k, wl.G, wl.N, wl.L
+    hbm, tflops, _, peak_kind = peaks()
+    if args.kernel == "gate":
+        nl = args.problems or wl.layers
+        hid = torch.empty(nl + 1, T, H, dtype=torch.bfloat16, device=dev)
+        workloads.hidden_chain(wl, nl, out=hid[1:])
+        hid[0].copy_(hid[1])
+        W = workloads.gate_weights(wl, nl, device=dev)
+        bias = workloads.biases(wl, nl).to(dev)
+        ip = torch.empty(nl, T, k, dtype=torch.int32, device=dev)
+        ia = torch.empty_like(ip)
+
+        def fn():
+            _lib.lb_predict_topk_chain(hid, W, bias, k, ids_pred=ip, ids_act=ia)
+        nbytes = (nl + 1) * 2 * T * H + nl * (2 * H * E + 4 * E + 8 * T * k)
+        flops = nl * 4.0 * T * H * E
+        work = f"chain gate, {nl} layers ({nl + 1} hidden states) of {wl.name}"
+    else:
+        nb = args.problems or 128
+        path = DecisionPath(nb, T, 8, E, k, G, N, L, device=dev)
+        for c0 in range(0, nb, 16):
+            path.ids[c0:c0 + 16].copy_(workloads.decode_ids(wl, T, range(c0, min(nb, c0 + 16)), device=dev))
+        _lib.lb_count(path.ids, G, E, cnt=path.cnt)
+        _lib.lb_plan_replicas(path.cnt, N, L, plan=path.plan)
+        _lib.lb_split(path.cnt, path.plan, N, 12, out=(path.tok, path.mass, path.loads, path.passes_run))
+        tk = T * k
+        n_edges = sum(int(d["n_edges"]) for d in _lib.decode_plan(path.plan, G, E, N)) / nb
+        fns = {
+            "count": (lambda: _lib.lb_count(path.ids, G, E, cnt=path.cnt), nb * (4 * tk + 4 * G * E)),
+            "plan": (lambda: _lib.lb_plan_replicas(path.cnt, N, L, plan=path.plan), nb * 4 * G * E),
+            "split": (lambda: _lib.lb_split(path.cnt, path.plan, N, 12,
+                                            out=(path.tok, path.mass, path.loads, path.passes_run)),
+                      int(nb * (4 * G * E + 12 * n_edges + 16 * G * N + 4 * G))),
+            "assign": (lambda: _lib.lb_assign(path.ids, path.cnt, path.plan, path.tok, path.mass, N,
+                                              out=(path.dest, path.perm, path.offs), workspace=path.ws),
+                       nb * (3 * 4 * tk + 4 * (G * E + 1) + 4 * G * E + 8 * G * N)),
+        }
+        fn, nbytes = fns[args.kernel]
+        flops = 0.0
+        work = f"{args.kernel}, {nb} problems of {wl.name} (T={T}, top-{k}, E={E}, G={G}, N={N}), decode-style ids"
+    for _ in range(args.launches):
+        fn()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        fn()
+    g.replay()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(20):
+        g.replay()
+    b.record()
+    torch.cuda.synchronize()
+    us = a.elapsed_time(b) * 1e3 / 20
+    if _lib.lb_get_status():
+        raise RuntimeError("device status flagged")
+    out = {"kernel": args.kernel, "work": work, "us": us, "algorithmic_bytes": nbytes,
+           "gbs": nbytes / us / 1e3, "hbm_frac": nbytes / us / 1e3 / hbm, "peak_kind": peak_kind}
+    if flops:
+        out.update(tflops=flops / us / 1e6, tensor_frac=flops / us / 1e6 / tflops)
+    return out
+
+
 # ----------------------------------------------------------------------------- CPU oracle
 _CPU_INPUTS = {}
 
@@ -874,6 +951,11 @@ def main():
                     help="chain: one gate pass per hidden state for both gates that read it; two-pass: "
                          "lookahead and normal router as separate passes")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--kernel", choices=("gate", "count", "plan", "split", "assign"), default=None,
+                    help="time one kernel alone (with --problems, --launches) instead of the step")
+    ap.add_argument("--problems", type=int, default=0,
+                    help="--kernel: layers of the chain gate, or problems per integer-kernel launch")
+    ap.add_argument("--launches", type=int, default=3, help="--kernel: plain launches before the timed replays")
     ap.add_argument("--decode-steps", type=int, default=1000,
                     help="decode steps per T in the per-step decode sweep of the extra keys")
     ap.add_argument("--lean", action="store_true",
@@ -889,6 +971,10 @@ def main():
         out = run_reference(args, world, rank)
         if out is not None:
             print(json.dumps(out), flush=True)
+        return
+    if args.kernel:
+        local = int(os.environ.get("LOCAL_RANK", "0"))
+        print(json.dumps(run_kernel(args, local)), flush=True)
         return
     world, rank, local = dist_setup()
     try:

@@ -31,16 +31,19 @@ def sources():
                   [os.path.join(INCLUDE, "lb.h")])
 
 
-def build(force: bool = False, verbose: bool = False, extra=()) -> str:
+def build(force: bool = False, verbose: bool = False, extra=(), out: str = LIB) -> str:
+    """Compile lb.cu into `out` (the product library by default) unless it is
+    newer than every source.  `extra` adds nvcc flags (e.g. -DLB_TIMING for
+    the phase-timing build, which goes to its own file)."""
     newest = max(os.path.getmtime(s) for s in sources())
-    if not force and os.path.exists(LIB) and os.path.getmtime(LIB) >= newest:
-        return LIB
+    if not force and os.path.exists(out) and os.path.getmtime(out) >= newest:
+        return out
     cmd = [nvcc(), *NVCC_FLAGS, *extra, "-I", INCLUDE, "-I", CSRC,
-           os.path.join(CSRC, "lb.cu"), "-o", LIB]
+           os.path.join(CSRC, "lb.cu"), "-o", out]
     if verbose:
         print(" ".join(cmd))
     subprocess.run(cmd, check=True)
-    return LIB
+    return out
 
 
 if __name__ == "__main__":

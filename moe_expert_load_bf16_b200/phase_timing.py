@@ -1,0 +1,87 @@
+"""Phase timing of the latency-bound kernels (plan, split, assign prep and
+scatter) on one problem, from a separate build of the library with
+-DLB_TIMING: block 0 of each kernel stamps clock64() at its phase boundaries
+into a device array, read back with lb_debug_ticks.  The product library is
+untouched (the timing build goes to liblb_timing.so and is loaded in place of
+liblb.so by this process only).
+
+    python -m moe_expert_load_bf16_b200.phase_timing [--config decode] [--T 8192] [--reps 20]
+
+Prints, per kernel, the cycles (and microseconds at the maximum SM clock)
+between consecutive stamps, the median over --reps launches.
+"""
+import argparse
+import ctypes
+import json
+import os
+import statistics
+
+import torch
+
+from . import _lib, build, workloads
+
+TIMING_LIB = os.path.join(os.path.dirname(os.path.abspath(__file__)), "liblb_timing.so")
+
+PHASES = {
+    "plan": (30, ["stage counts", "phase 1 (locality imports)", "load model", "phase 2 (greedy moves)",
+                  "edges", "round colouring + order", "write blob"]),
+    "split": (0, ["stage inputs", "per-expert setup", "start loads + round table", "passes + masses"]),
+    "assign prep": (20, ["stage inputs + per-expert segments", "bucket sizes + scan", "block bases"]),
+    "assign scatter": (10, ["per-problem tables", "scatter"]),
+}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--config", default="decode")
+    ap.add_argument("--T", type=int, default=0, help="tokens per problem (default: the workload's)")
+    ap.add_argument("--reps", type=int, default=20)
+    args = ap.parse_args()
+    build.build(extra=["-DLB_TIMING"], out=TIMING_LIB)
+    _lib.LIB_PATH = TIMING_LIB
+    lib = _lib._load()
+    lib.lb_debug_ticks.argtypes = [ctypes.POINTER(ctypes.c_longlong), ctypes.c_int]
+    lib.lb_debug_ticks.restype = ctypes.c_int
+    wl = workloads.WORKLOADS[args.config]
+    T = args.T or wl.T
+    G, E, k, N, L = wl.G, wl.E, wl.k, wl.N, wl.L
+    dev = torch.device("cuda", 0)
+    ids = workloads.decode_ids(wl.with_(T=T), T, [0, 1], device=dev)
+    cnt_pred = _lib.lb_count(ids[0:1], G, E)
+    cnt = _lib.lb_count(ids[1:2], G, E)
+    plan = _lib.lb_plan_replicas(cnt_pred, N, L)
+    tok, mass, loads, pr = _lib.lb_split(cnt, plan, N, 12)
+    ws = torch.empty(max(256, _lib.lb_assign_workspace_bytes(1, T, k, G, E, N)), dtype=torch.uint8, device=dev)
+    launches = {
+        "plan": lambda: _lib.lb_plan_replicas(cnt_pred, N, L, plan=plan),
+        "split": lambda: _lib.lb_split(cnt, plan, N, 12, out=(tok, mass, loads, pr)),
+        "assign": lambda: _lib.lb_assign(ids[1:2], cnt, plan, tok, mass, N, workspace=ws),
+    }
+    try:   # clock64 counts SM cycles; microseconds below are at the maximum SM clock
+        import pynvml
+        pynvml.nvmlInit()
+        khz = 1000 * pynvml.nvmlDeviceGetMaxClockInfo(pynvml.nvmlDeviceGetHandleByIndex(0), pynvml.NVML_CLOCK_SM)
+    except Exception:
+        khz = 1965000
+    ticks = (ctypes.c_longlong * 64)()
+    res = {"workload": f"{wl.name}: T={T}, E={E}, top-{k}, G={G}, N={N} (L={L}), one problem",
+           "passes_run": int(pr.item()), "clock_khz": khz}
+    samples = {}
+    for name, fn in launches.items():
+        for _ in range(args.reps):
+            fn()
+            if lib.lb_debug_ticks(ticks, 64) != 0:
+                raise RuntimeError("lb_debug_ticks failed")
+            kernels = [name] if name != "assign" else ["assign prep", "assign scatter"]
+            for kn in kernels:
+                first, labels = PHASES[kn]
+                for i, lab in enumerate(labels):
+                    samples.setdefault(kn, {}).setdefault(lab, []).append(ticks[first + i + 1] - ticks[first + i])
+    for kn, d in samples.items():
+        res[kn] = {lab: {"cycles": statistics.median(v), "us": statistics.median(v) / (khz * 1e-3)}
+                   for lab, v in d.items()}
+    print(json.dumps(res, indent=1))
+
+
+if __name__ == "__main__":
+    main()
