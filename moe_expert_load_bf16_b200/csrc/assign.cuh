@@ -474,16 +474,23 @@ __device__ void scatter_blocks_warp(const Args &a, int b, int g0, int g1, const 
         }
         __syncwarp();
         const int64_t f0 = static_cast<int64_t>(g) * nitems;
+        // ids of the next PF steps in flight (a ring of registers), so no step
+        // waits on its own global load
+        constexpr int PF = 4;
+        int ring[PF];
+#pragma unroll
+        for (int q = 0; q < PF; ++q) ring[q] = (q * 32 + lane < nitems) ? __ldg(ids + f0 + q * 32 + lane) : -1;
         for (int i0 = 0; i0 < nitems; i0 += 32) {
             const int i = i0 + lane;
-            int e = -1;
-            if (i < nitems) {
-                e = __ldg(ids + f0 + i);
-                if (e < 0 || e >= E) {
-                    *bad = 1;
-                    e = -1;
-                }
+            int e = ring[0];
+#pragma unroll
+            for (int q = 0; q + 1 < PF; ++q) ring[q] = ring[q + 1];
+            ring[PF - 1] = (i + PF * 32 < nitems) ? __ldg(ids + f0 + i + PF * 32) : -1;
+            if (i < nitems && (e < 0 || e >= E)) {
+                *bad = 1;
+                e = -1;
             }
+            if (i >= nitems) e = -1;
             const unsigned peers = warp_peers<NB>(e);
             const int rnk = __popc(peers & lanemask_lt());
             const int cur = e >= 0 ? cntw[e] : 0;

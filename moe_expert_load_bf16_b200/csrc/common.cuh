@@ -21,9 +21,16 @@ __device__ __forceinline__ void flag(int bits) { atomicOr(&g_status, bits); }
 // compiled out otherwise.
 #ifdef LB_TIMING
 __device__ long long g_ticks[64];
+// (the clock read carries a memory clobber, so it stays between the memory
+// operations and barriers around it)
+__device__ __forceinline__ long long lb_clock() {
+    long long t;
+    asm volatile("mov.u64 %0, %%clock64;" : "=l"(t)::"memory");
+    return t;
+}
 #define LB_TICK(slot)                                                                          \
     do {                                                                                       \
-        if (threadIdx.x == 0 && blockIdx.x == 0 && blockIdx.y == 0) lb::g_ticks[slot] = clock64(); \
+        if (threadIdx.x == 0 && blockIdx.x == 0 && blockIdx.y == 0) lb::g_ticks[slot] = lb::lb_clock(); \
     } while (0)
 #else
 #define LB_TICK(slot) \

@@ -134,28 +134,101 @@ __device__ void plan_problem(const int32_t *__restrict__ cnt, int G, int E, int 
     __syncthreads();
 
     LB_TICK(32);
-    // ---------------- load model
+    // ---------------- load model: per expert, its remote mass m[e] (tokens of
+    // sources that do not hold it) stays at home; every holder serves its own
+    // tokens.  Rank loads are integer sums, so their order is immaterial.
+    if (tid < LB_MAX_G) load_s[tid] = 0;
+    __syncthreads();
     for (int e = tid; e < E; e += blockDim.x) {
         const uint64_t hm = hold[e];
         int s = 0;
         for (int g = 0; g < G; ++g)
             if (!((hm >> g) & 1ull)) s += cnt_s[g * E + e];
         m[e] = s;
-    }
-    __syncthreads();
-    for (int r = warp; r < G; r += nwarps) {
-        int x = 0;
-        for (int e = lane; e < E; e += 32)
-            if ((hold[e] >> r) & 1ull) x += cnt_s[r * E + e];
-        for (int e = r * Eg + lane; e < (r + 1) * Eg; e += 32) x += m[e];
-        x = __reduce_add_sync(kFull, x);
-        if (lane == 0) load_s[r] = x;
+        for (uint64_t mk = hm; mk; mk &= mk - 1) {
+            const int g = __ffsll(static_cast<long long>(mk)) - 1;
+            atomicAdd(&load_s[g], cnt_s[g * E + e]);
+        }
+        atomicAdd(&load_s[e / Eg], s);
     }
     __syncthreads();
 
     LB_TICK(33);
     // ---------------- phase 2: sequential greedy, one warp
+    __shared__ int total_s;
     if (warp == 0) {
+        int x = 0;
+        for (int r = lane; r < G; r += 32) x += load_s[r];
+        x = __reduce_add_sync(kFull, x);
+        if (lane == 0) total_s = x;
+    }
+    __syncthreads();
+    if (warp == 0 && total_s < (1 << 21)) {
+        // Every load and remote mass is below 2^21, so each arg-reduction is
+        // one redux over a packed 32-bit key: (load, 63 - rank) + 1 for the
+        // most-loaded rank (lowest rank on ties), (mass, 1023 - position) for
+        // the candidate expert (lowest id on ties), (load, rank) for the
+        // least-loaded eligible rank.  Same choices as the general loop below.
+        const bool ha = lane < G, hb = lane + 32 < G;
+        int la = ha ? load_s[lane] : 0, lb = hb ? load_s[lane + 32] : 0;
+        int ua = ha ? used_s[lane] : N, ub = hb ? used_s[lane + 32] : N;
+        const int iters = __reduce_add_sync(kFull, (ha ? N - ua : 0) + (hb ? N - ub : 0));
+        uint64_t freem = static_cast<uint64_t>(__ballot_sync(kFull, ha && ua < N)) |
+                         (static_cast<uint64_t>(__ballot_sync(kFull, hb && ub < N)) << 32);
+        int np2 = 0;
+        for (int it = 0; it < iters; ++it) {
+            const unsigned ka = ha ? ((static_cast<unsigned>(la) << 6) | static_cast<unsigned>(63 - lane)) + 1u : 0u;
+            const unsigned kb = hb ? ((static_cast<unsigned>(lb) << 6) | static_cast<unsigned>(31 - lane)) + 1u : 0u;
+            const unsigned ku = __reduce_max_sync(kFull, max(ka, kb));
+            const int u = 63 - static_cast<int>((ku - 1u) & 63u);
+            const int mx = static_cast<int>((ku - 1u) >> 6);
+            unsigned kc = 0u;
+            for (int q = lane; q < Eg; q += 32) {
+                const int e = u * Eg + q;
+                const int me = m[e];
+                if (me > 0 && (~hold[e] & freem) != 0ull)
+                    kc = max(kc, (static_cast<unsigned>(me) << 10) | static_cast<unsigned>(1023 - q));
+            }
+            kc = __reduce_max_sync(kFull, kc);
+            if (kc == 0u) break;
+            const int ce = u * Eg + (1023 - static_cast<int>(kc & 1023u));
+            const uint64_t hce = hold[ce];
+            const int mce = static_cast<int>(kc >> 10);
+            const uint64_t V = ~hce & freem;
+            const bool ea = (V >> lane) & 1ull, eb = (V >> (lane + 32)) & 1ull;
+            const unsigned kva = ea ? (static_cast<unsigned>(la) << 6) | static_cast<unsigned>(lane) : 0xffffffffu;
+            const unsigned kvb = eb ? (static_cast<unsigned>(lb) << 6) | static_cast<unsigned>(lane + 32) : 0xffffffffu;
+            const unsigned kv = __reduce_min_sync(kFull, min(kva, kvb));
+            const int v = static_cast<int>(kv & 63u);
+            const int mn = static_cast<int>(kv >> 6);
+            const int c = cnt_s[v * E + ce];
+            const int mr = mce - c;
+            const int lu = mx - c, lv = mn + c;
+            const int gap = lu - lv;
+            const int d = min(gap > 0 ? (gap >> 1) : 0, mr);
+            if (c + d == 0) break;
+            const int used_v = __shfl_sync(kFull, v < 32 ? ua : ub, v & 31);
+            if (lane == 0) {
+                hold[ce] = hce | (1ull << v);
+                slots[v * N + used_v] = ce;
+                phase[v * N + used_v] = 2;
+                m[ce] = mr - d;
+            }
+            if (used_v + 1 >= N) freem &= ~(1ull << v);
+            const bool own_u = lane == (u & 31), own_v = lane == (v & 31);
+            la = (own_u && u < 32) ? lu - d : la;
+            lb = (own_u && u >= 32) ? lu - d : lb;
+            la = (own_v && v < 32) ? lv + d : la;
+            lb = (own_v && v >= 32) ? lv + d : lb;
+            ua += (own_v && v < 32) ? 1 : 0;
+            ub += (own_v && v >= 32) ? 1 : 0;
+            ++np2;
+            __syncwarp();
+        }
+        if (ha) { load_s[lane] = la; used_s[lane] = ua; }
+        if (hb) { load_s[lane + 32] = lb; used_s[lane + 32] = ub; }
+        if (lane == 0) n_p2_s = np2;
+    } else if (warp == 0) {
         const bool ha = lane < G, hb = lane + 32 < G;
         int la = ha ? load_s[lane] : INT_MIN, lb = hb ? load_s[lane + 32] : INT_MIN;
         int ua = ha ? used_s[lane] : N, ub = hb ? used_s[lane + 32] : N;
@@ -309,6 +382,7 @@ __device__ void plan_problem(const int32_t *__restrict__ cnt, int G, int E, int 
         n_rounds_s = nr;
     }
     __syncthreads();
+    LB_TICK(38);
     {
         // stable order by round: position = start of the round + earlier
         // edges (in edge order) of the same round

@@ -44,7 +44,7 @@ struct View {
     int32_t *eu, *ev, *ee;  // [GN] schedule order
     int32_t *rptr;      // [GN+1]
     int32_t *tk, *mu, *mv;  // [GN] tok, mass (home side), mass (replica side)
-    int4 *tab;          // [RC*G] (round, rank) slots: {code, tok, own-side mass, 0}
+    int4 *tab;          // [(RC+1)*G] (round, rank) slots: {code, tok, own-side mass, 0}; row nr idle
     int32_t *Ls;        // [64]
 };
 
@@ -52,7 +52,7 @@ __host__ __device__ inline size_t smem_bytes(int G, int E, int N) {
     const size_t GN = static_cast<size_t>(G) * N;
     return static_cast<size_t>(E) * 8 + static_cast<size_t>(G) * E * 4 + static_cast<size_t>(E) * 4 +
            (static_cast<size_t>(E) + 1) * 4 + GN * 4 * 7 + (GN + 1) * 4 +
-           static_cast<size_t>(table_rounds(G, N)) * G * 16 + 64 * 4 + 64;
+           (static_cast<size_t>(table_rounds(G, N)) + 1) * G * 16 + 64 * 4 + 64;
 }
 
 __device__ inline View carve(uint8_t *sm, int G, int E, int N) {
@@ -74,7 +74,7 @@ __device__ inline View carve(uint8_t *sm, int G, int E, int N) {
     uintptr_t t = reinterpret_cast<uintptr_t>(v.mv + GN);
     t = (t + 15) & ~static_cast<uintptr_t>(15);
     v.tab = reinterpret_cast<int4 *>(t);
-    v.Ls = reinterpret_cast<int32_t *>(v.tab + table_rounds(G, N) * G);
+    v.Ls = reinterpret_cast<int32_t *>(v.tab + (table_rounds(G, N) + 1) * G);   // one idle row past the rounds
     return v;
 }
 
@@ -97,29 +97,33 @@ template <bool TWO>
 __device__ int relax_passes_regs(int G, int nr, int passes, const View &v) {
     const int lane = threadIdx.x & 31;
     const bool ha = lane < G, hb = TWO && lane + 32 < G;
+    // lanes that own no rank read column 0 and compute throw-away moves:
+    // nobody shuffles from them and they store nothing
+    const int ca = ha ? lane : 0, cb = hb ? lane + 32 : 0;
     int La = ha ? v.Ls[lane] : 0;
     int Lb = hb ? v.Ls[lane + 32] : 0;
-    const int4 idle_a = make_int4(slot_code(lane, false, 0), 0, 0, 0);
-    const int4 idle_b = make_int4(slot_code(lane + 32, false, 0), 0, 0, 0);
     int pr = 0;
     for (int p = 1; p <= passes; ++p) {
-        bool moved = false;
-        int4 A = (nr > 0 && ha) ? v.tab[lane] : idle_a;
-        int4 B = (nr > 0 && hb) ? v.tab[lane + 32] : idle_b;
+        // a move changes the loads at both its ends, so a pass moved something
+        // exactly when some load differs from its value at the pass's start
+        const int La0 = La, Lb0 = Lb;
+        int4 A = v.tab[ca];
+        int4 B = TWO ? v.tab[cb] : make_int4(0, 0, 0, 0);
         for (int r = 0; r < nr; ++r) {
             const int4 a = A, b = B;
-            if (r + 1 < nr) {
-                A = ha ? v.tab[(r + 1) * G + lane] : idle_a;
-                if (TWO) B = hb ? v.tab[(r + 1) * G + lane + 32] : idle_b;
-            }
+            // next round's slots (row nr is an idle row, so no bound check)
+            A = v.tab[(r + 1) * G + ca];
+            if (TWO) B = v.tab[(r + 1) * G + cb];
             // every shuffle before any update: a lane may own both ends
-            int xa = __shfl_sync(kFull, La, a.x & 31);
+            const int pa = a.x & 31;
+            int xa = __shfl_sync(kFull, La, pa);
             int xb = 0;
             if (TWO) {
-                const int ya = __shfl_sync(kFull, Lb, a.x & 31);
+                const int ya = __shfl_sync(kFull, Lb, pa);
+                const int pb = b.x & 31;
+                const int xl = __shfl_sync(kFull, La, pb);
+                const int xh = __shfl_sync(kFull, Lb, pb);
                 xa = (a.x & 32) ? ya : xa;
-                const int xl = __shfl_sync(kFull, La, b.x & 31);
-                const int xh = __shfl_sync(kFull, Lb, b.x & 31);
                 xb = (b.x & 32) ? xh : xl;
             }
             {
@@ -127,24 +131,18 @@ __device__ int relax_passes_regs(int G, int nr, int passes, const View &v) {
                 const int d = min((diff < 0 ? -diff : diff) >> 1, diff > 0 ? a.z : a.y - a.z);
                 const int delta = diff > 0 ? -d : d;
                 La += delta;
-                if (delta != 0) {
-                    v.tab[r * G + lane].z = a.z + delta;
-                    moved = true;
-                }
+                if (ha) v.tab[r * G + lane].z = a.z + delta;   // unchanged value when delta is 0
             }
             if (TWO) {
                 const int diff = Lb - xb;
                 const int d = min((diff < 0 ? -diff : diff) >> 1, diff > 0 ? b.z : b.y - b.z);
                 const int delta = diff > 0 ? -d : d;
                 Lb += delta;
-                if (delta != 0) {
-                    v.tab[r * G + lane + 32].z = b.z + delta;
-                    moved = true;
-                }
+                if (hb) v.tab[r * G + lane + 32].z = b.z + delta;
             }
         }
         pr = p;
-        if (!__any_sync(kFull, moved)) break;
+        if (!__any_sync(kFull, (ha && La != La0) || (hb && Lb != Lb0))) break;
     }
     if (ha) v.Ls[lane] = La;
     if (hb) v.Ls[lane + 32] = Lb;
@@ -194,7 +192,7 @@ __device__ int relax_passes_smem(int ne, int nr, int passes, const View &v, int 
 // v.Ls, and returns passes run.  All threads of the CTA must call it.
 __device__ int split_problem(const int32_t *__restrict__ cnt, const uint8_t *__restrict__ blob, int G, int E,
                              int N, int passes, const View &v, int &ne_out, int *bad) {
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, nwarps = blockDim.x >> 5;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int GN = G * N, Eg = E / G;
     const plan::Layout LY = plan::layout(G, E, N);
     const int32_t *hdr = reinterpret_cast<const int32_t *>(blob + LY.hdr);
@@ -224,12 +222,13 @@ __device__ int split_problem(const int32_t *__restrict__ cnt, const uint8_t *__r
             v.mu[i] = 0;
             v.mv[i] = 0;
         }
+        for (int r = tid; r < G; r += blockDim.x) v.Ls[r] = 0;
         const int32_t *p_rptr = reinterpret_cast<const int32_t *>(blob + LY.round_ptr);
         for (int r = tid; r <= nr; r += blockDim.x) v.rptr[r] = p_rptr[r];
         const int32_t *p_rep_ptr = reinterpret_cast<const int32_t *>(blob + LY.rep_ptr);
         for (int e = tid; e <= E; e += blockDim.x) v.rep_ptr[e] = p_rep_ptr[e];
         if (use_table)
-            for (int x = tid; x < nr * G; x += blockDim.x) {
+            for (int x = tid; x < (nr + 1) * G; x += blockDim.x) {
                 const int rank = x % G;
                 v.tab[x] = make_int4(slot_code(rank, false, 0), 0, 0, 0);
             }
@@ -259,6 +258,13 @@ __device__ int split_problem(const int32_t *__restrict__ cnt, const uint8_t *__r
             if (!((hm >> g) & 1ull)) R += v.cnt[g * E + e];
         v.hold[e] = hm;
         v.R[e] = R;
+        // starting loads: every holder serves its own tokens of e, and all the
+        // remote mass R starts at home (integer sums: the order is immaterial)
+        for (uint64_t mk = hm; mk; mk &= mk - 1) {
+            const int g = __ffsll(static_cast<long long>(mk)) - 1;
+            atomicAdd(&v.Ls[g], v.cnt[g * E + e]);
+        }
+        atomicAdd(&v.Ls[h], R);
         const int m = z - a;
         if (m > 0) {
             const int q = R / m, rem = R % m;
@@ -272,33 +278,26 @@ __device__ int split_problem(const int32_t *__restrict__ cnt, const uint8_t *__r
             }
         }
     }
+    LB_TICK(7);
     __syncthreads();
     LB_TICK(2);
 
-    // ---- starting loads (warp per rank) and the round table
-    for (int r = warp; r < G; r += nwarps) {
-        int x = 0;
-        for (int e = lane; e < E; e += 32) {
-            if ((v.hold[e] >> r) & 1ull) x += v.cnt[r * E + e];
-        }
-        for (int e = r * Eg + lane; e < (r + 1) * Eg; e += 32) x += v.R[e];
-        x = __reduce_add_sync(kFull, x);
-        if (lane == 0) v.Ls[r] = x;
-    }
+    // ---- the round table: one thread per edge, at the (round, rank) slots of
+    // both its ends (the plan blob gives each edge's round)
+    LB_TICK(5);
     if (use_table) {
-        for (int r = tid; r < nr; r += blockDim.x) {
-            const int a = v.rptr[r], z = v.rptr[r + 1];
-            if (a < 0 || z > ne || z < a) {
+        const int32_t *p_er = reinterpret_cast<const int32_t *>(blob + LY.edge_round);
+        for (int i = tid; i < ne; i += blockDim.x) {
+            const int r = p_er[i];
+            const int u = v.eu[i], w = v.ev[i];
+            if (r < 0 || r >= nr || i < v.rptr[r] || i >= v.rptr[r + 1]) {
                 *bad = 1;
                 continue;
             }
-            for (int i = a; i < z; ++i) {
-                const int u = v.eu[i], w = v.ev[i];
-                if (u < 0 || u >= G || w < 0 || w >= G || u == w) continue;
-                const int t = v.tk[i];
-                v.tab[r * G + u] = make_int4(slot_code(w, true, i), t, t, 0);
-                v.tab[r * G + w] = make_int4(slot_code(u, false, i), t, 0, 0);
-            }
+            if (u < 0 || u >= G || w < 0 || w >= G || u == w) continue;
+            const int t = v.tk[i];
+            v.tab[r * G + u] = make_int4(slot_code(w, true, i), t, t, 0);
+            v.tab[r * G + w] = make_int4(slot_code(u, false, i), t, 0, 0);
         }
     }
     __syncthreads();
@@ -313,6 +312,7 @@ __device__ int split_problem(const int32_t *__restrict__ cnt, const uint8_t *__r
         else
             pr = relax_passes_smem(ne, nr, passes, v, bad);
         if (lane == 0) pr_s = pr;
+        LB_TICK(6);
     }
     __syncthreads();
     if (use_table) {

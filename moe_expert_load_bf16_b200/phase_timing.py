@@ -25,7 +25,10 @@ TIMING_LIB = os.path.join(os.path.dirname(os.path.abspath(__file__)), "liblb_tim
 PHASES = {
     "plan": (30, ["stage counts", "phase 1 (locality imports)", "load model", "phase 2 (greedy moves)",
                   "edges", "round colouring + order", "write blob"]),
-    "split": (0, ["stage inputs", "per-expert setup", "start loads + round table", "passes + masses"]),
+    "split": (0, ["stage inputs", "per-expert setup and start loads", "round table", "passes + masses"]),
+    "plan detail": (None, [(35, 38, "round colouring"), (38, 36, "order by round")]),
+    "split detail": (None, [(1, 7, "per-expert setup (thread 0)"), (7, 2, "wait for the other experts"),
+                            (2, 3, "round table"), (3, 6, "passes"), (6, 4, "masses")]),
     "assign prep": (20, ["stage inputs + per-expert segments", "bucket sizes + scan", "block bases"]),
     "assign scatter": (10, ["per-problem tables", "scatter"]),
 }
@@ -73,10 +76,19 @@ def main():
             if lib.lb_debug_ticks(ticks, 64) != 0:
                 raise RuntimeError("lb_debug_ticks failed")
             kernels = [name] if name != "assign" else ["assign prep", "assign scatter"]
+            if name == "split":
+                kernels = kernels + ["split detail"]
+            if name == "plan":
+                kernels = kernels + ["plan detail"]
             for kn in kernels:
                 first, labels = PHASES[kn]
                 for i, lab in enumerate(labels):
-                    samples.setdefault(kn, {}).setdefault(lab, []).append(ticks[first + i + 1] - ticks[first + i])
+                    if first is None:   # (from stamp, to stamp, label)
+                        a, b, lab = lab
+                        dt = ticks[b] - ticks[a]
+                    else:
+                        dt = ticks[first + i + 1] - ticks[first + i]
+                    samples.setdefault(kn, {}).setdefault(lab, []).append(dt)
     for kn, d in samples.items():
         res[kn] = {lab: {"cycles": statistics.median(v), "us": statistics.median(v) / (khz * 1e-3)}
                    for lab, v in d.items()}
