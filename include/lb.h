@@ -120,7 +120,9 @@ int lb_predict_topk_chain(const void *h, const void *w, const float *bias,
 /* Tuning knobs of lb_predict_topk and lb_predict_topk_chain (process-wide;
  * 0 = automatic choice): pipeline stages per CTA (2..8, clamped to what the
  * CTA's shared memory holds); split of H across a
- * CTA cluster (1, 2, 4, 8 or 16); persistent kernel (1, 2 or 4 = that many
+ * CTA cluster (1, 2, 4, 8 or 16), or of N (-2, -4, -8: the S CTAs of a
+ * cluster share a token tile, each ranking Epad/S experts, their lists
+ * merged over distributed shared memory); persistent kernel (1, 2 or 4 = that many
  * CTAs per SM walking the token tiles with a TMEM accumulator, double-
  * buffered where TMEM allows; 3 = CTA pairs: clusters of two CTAs, one per
  * SM, sharing one MMA of M = 256 over 256-token work units, each CTA
@@ -136,8 +138,9 @@ int lb_predict_topk_chain(const void *h, const void *w, const float *bias,
  * persistent with two CTAs per SM (one when two double-buffered
  * accumulators of the MMA's N do not fit TMEM twice) and one tile per unit;
  * otherwise one CTA
- * per tile, H split across a cluster until the GPU is filled when the tiles
- * alone do not fill it.  Results do not depend on the knobs beyond fp32 rounding of
+ * per tile; when the tiles alone do not fill the GPU, H split across the
+ * largest cluster that keeps one wave (at most 8, 16 for one or two tiles),
+ * or N split in two where that cluster would be two or fewer.  Results do not depend on the knobs beyond fp32 rounding of
  * split-H partial sums.  LB_EINVAL for values out of range. */
 int lb_gate_tuning(int stages, int split, int persistent, int kbox, int tiles_per_unit,
                    int max_ctas);

@@ -102,10 +102,19 @@ struct TopK {
     }
 };
 
-template <int KMAX, bool SPLITK>
+// Split of N across a cluster (SPLITN): the S CTAs of a cluster share one
+// token tile; CTA r loads the tile's h rows and rows [r Nc, (r+1) Nc) of W
+// (Nc = Epad / S; the B map's box is Nc rows), accumulates the tile's logits
+// for those experts over all of H, ranks them per row, and leaves its sorted
+// key list of each row in shared memory.  After a cluster barrier, CTA r
+// merges rows [r BM/S, (r+1) BM/S) over the S lists (distributed shared
+// memory reads) and writes their ids.  Keys carry the global expert id, so
+// the merge is a plain top-k of the S lists: the same ranking as one CTA.
+template <int KMAX, bool SPLITK, bool SPLITN = false>
 __global__ void __launch_bounds__(THREADS, 1)
     gate_topk_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                      const Params p) {
+    static_assert(!(SPLITK && SPLITN), "one split at a time");
     extern __shared__ uint8_t smem_raw[];
     pdl_begin();
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -119,15 +128,17 @@ __global__ void __launch_bounds__(THREADS, 1)
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int b = blockIdx.y;
-    const int S = SPLITK ? p.split : 1;
-    const int crank = SPLITK ? static_cast<int>(cluster_ctarank()) : 0;
+    const int S = (SPLITK || SPLITN) ? p.split : 1;
+    const int crank = (SPLITK || SPLITN) ? static_cast<int>(cluster_ctarank()) : 0;
     const int mtile = blockIdx.x / S;
     const int m0 = mtile * BM;
-    const int kb_per = (p.nkb + S - 1) / S;
-    const int kb0 = crank * kb_per;
+    const int kb_per = SPLITN ? p.nkb : (p.nkb + S - 1) / S;
+    const int kb0 = SPLITN ? 0 : crank * kb_per;
     const int nk = max(0, min(p.nkb, kb0 + kb_per) - kb0);
+    const int Nc = SPLITN ? p.Epad / S : p.Epad;   // the MMA's N: this CTA's experts
+    const int c_off = SPLITN ? crank * Nc : 0;     // its first expert
     const uint32_t a_bytes = BM * 128u;
-    const uint32_t stage_bytes = a_bytes + static_cast<uint32_t>(p.Epad) * 128u;
+    const uint32_t stage_bytes = a_bytes + static_cast<uint32_t>(Nc) * 128u;
     const int stages = p.stages;
 
     for (int c = tid; c < p.Epad; c += THREADS)
@@ -168,7 +179,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                 uint8_t *sa = smem + static_cast<size_t>(s) * stage_bytes;
                 mbar_arrive_expect_tx(&full_bar[s], stage_bytes);
                 tma_load_3d(&tmA, sa, &full_bar[s], (kb0 + i) * BK, m0, b);
-                tma_load_3d(&tmB, sa + a_bytes, &full_bar[s], (kb0 + i) * BK, 0, b);
+                tma_load_3d(&tmB, sa + a_bytes, &full_bar[s], (kb0 + i) * BK, c_off, b);
                 ++issued;
             }
             // Never leave with copies in flight into this CTA's shared memory:
@@ -181,7 +192,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     } else if (warp == 1) {
         if (lane == 0) {
             // ---------------- MMA issuer
-            const uint32_t idesc = umma_idesc_bf16(BM, p.Epad);
+            const uint32_t idesc = umma_idesc_bf16(BM, Nc);
             for (int i = 0; i < nk; ++i) {
                 const int s = i % stages;
                 const uint32_t ph = (i / stages) & 1;
@@ -214,7 +225,54 @@ __global__ void __launch_bounds__(THREADS, 1)
     const int64_t rowbase = static_cast<int64_t>(b) * p.T;
     const uint32_t tl = tmem + (static_cast<uint32_t>(warp * 32) << 16);
 
-    if constexpr (!SPLITK) {
+    if constexpr (SPLITN) {
+        // rank this CTA's experts per row; hand the list over in shared
+        // memory (the pipeline buffers are free: acc_bar completed)
+        const int row = m0 + tid;
+        const bool valid = ok && row < p.T;
+        const uint32_t kmask = id_mask(p.E);
+        TopK<KMAX> tk;
+        tk.init();
+        float *lrow = (p.logits != nullptr && valid) ? p.logits + (rowbase + row) * p.E : nullptr;
+        if (ok) {
+            for (int c0 = 0; c0 < Nc; c0 += 16) {
+                uint32_t r[16];
+                tmem_ld16(tl + c0, r);
+                tmem_wait_ld();
+#pragma unroll
+                for (int q = 0; q < 16; ++q) {
+                    const int c = c_off + c0 + q;
+                    const float x = __uint_as_float(r[q]) + bias_s[c];
+                    tk.push(c < p.E ? rank_key(x, c, kmask) : 0u);
+                    if (lrow && c < p.E) lrow[c] = x;
+                }
+            }
+        }
+        uint32_t *lists = reinterpret_cast<uint32_t *>(smem);   // [BM][KMAX]
+#pragma unroll
+        for (int j = 0; j < KMAX; ++j) lists[tid * KMAX + j] = tk.key[j];
+        cluster_sync();   // every CTA of the cluster passes both barriers, always
+        const int R = BM / S;
+        if (tid < R) {
+            const int trow = crank * R + tid;
+            const int grow_ = m0 + trow;
+            TopK<KMAX> mg;
+            mg.init();
+            const uint32_t laddr = smem_u32(lists + trow * KMAX);
+            for (int s2 = 0; s2 < S; ++s2) {
+                const uint32_t ra = mapa_shared(laddr, s2);
+#pragma unroll
+                for (int j = 0; j < KMAX; ++j) mg.push(static_cast<uint32_t>(ld_cluster_i32(ra + 4 * j)));
+            }
+            if (grow_ < p.T) {
+                int32_t *out = p.ids + (rowbase + grow_) * p.k;
+#pragma unroll
+                for (int j = 0; j < KMAX; ++j)
+                    if (j < p.k) out[j] = key_id(mg.key[j], kmask);
+            }
+        }
+        cluster_sync();   // keep this CTA's lists alive until all readers are done
+    } else if constexpr (!SPLITK) {
         const int row = m0 + tid;
         const bool valid = ok && row < p.T;
         const uint32_t kmask = id_mask(p.E);

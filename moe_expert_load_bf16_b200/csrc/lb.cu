@@ -163,19 +163,19 @@ bool allow_smem(F *kernel, SmemLimit &lim, size_t bytes, bool cluster16) {
 // One limit record per kernel that several entry points launch.
 SmemLimit g_lim_plan, g_lim_split, g_lim_prep, g_lim_scatter;
 
-template <int KMAX, bool SPLITK>
+template <int KMAX, bool SPLITK, bool SPLITN = false>
 int launch_gate(const CUtensorMap &ma, const CUtensorMap &mb, const gate::Params &p, int mtiles, int nbatch,
                 size_t smem, cudaStream_t s) {
-    auto kern = gate::gate_topk_kernel<KMAX, SPLITK>;
+    auto kern = gate::gate_topk_kernel<KMAX, SPLITK, SPLITN>;
     static SmemLimit lim;
-    if (!allow_smem(kern, lim, smem, SPLITK)) return LB_ECUDA;
+    if (!allow_smem(kern, lim, smem, SPLITK || SPLITN)) return LB_ECUDA;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(mtiles * p.split, nbatch, 1);
     cfg.blockDim = dim3(gate::THREADS, 1, 1);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = s;
     cudaLaunchAttribute attr[1];
-    if (SPLITK) {
+    if (SPLITK || SPLITN) {
         attr[0].id = cudaLaunchAttributeClusterDimension;
         attr[0].val.clusterDim.x = p.split;
         attr[0].val.clusterDim.y = 1;
@@ -401,13 +401,55 @@ int run_persistent(gate::Params &p, const void *h, int nprob, const CUtensorMap 
                    : launch_gate_persistent_es<2, 1>(p.k, ma, mb, p, units, static_cast<int>(nunits), grid, smem, s);
 }
 
-template <bool SPLITK>
+template <bool SPLITK, bool SPLITN = false>
 int launch_gate_k(int k, const CUtensorMap &ma, const CUtensorMap &mb, const gate::Params &p, int mtiles,
                   int nbatch, size_t smem, cudaStream_t s) {
-    if (k <= 2) return launch_gate<2, SPLITK>(ma, mb, p, mtiles, nbatch, smem, s);
-    if (k <= 4) return launch_gate<4, SPLITK>(ma, mb, p, mtiles, nbatch, smem, s);
-    if (k <= 8) return launch_gate<8, SPLITK>(ma, mb, p, mtiles, nbatch, smem, s);
-    return launch_gate<16, SPLITK>(ma, mb, p, mtiles, nbatch, smem, s);
+    if (k <= 2) return launch_gate<2, SPLITK, SPLITN>(ma, mb, p, mtiles, nbatch, smem, s);
+    if (k <= 4) return launch_gate<4, SPLITK, SPLITN>(ma, mb, p, mtiles, nbatch, smem, s);
+    if (k <= 8) return launch_gate<8, SPLITK, SPLITN>(ma, mb, p, mtiles, nbatch, smem, s);
+    return launch_gate<16, SPLITK, SPLITN>(ma, mb, p, mtiles, nbatch, smem, s);
+}
+
+// Split of N across a cluster of S CTAs per token tile (each CTA Epad/S
+// experts of the tile, lists merged over distributed shared memory).
+int run_splitn(gate::Params &p, const void *h, const void *w, int nbatch, int mtiles, int S, cudaStream_t s) {
+    const int Nc = p.Epad / S;
+    if (S < 2 || S > 8 || p.Epad % (16 * S) != 0 || Nc < 16) return LB_EINVAL;
+    uint32_t cols = 32;
+    while (cols < static_cast<uint32_t>(Nc)) cols <<= 1;
+    p.tmem_cols = cols;
+    p.split = S;
+    const size_t stage_bytes = 16384 + static_cast<size_t>(Nc) * 128;
+    int stages = g_tune_stages ? g_tune_stages
+                               : static_cast<int>(std::min<size_t>(gate::MAX_STAGES, (200 * 1024) / stage_bytes));
+    size_t smem = stages * stage_bytes + 1024;
+    if (smem > 224 * 1024) {
+        stages = static_cast<int>((224 * 1024 - 1024) / stage_bytes);
+        smem = stages * stage_bytes + 1024;
+    }
+    if (stages < 2) return LB_EINVAL;
+    smem = std::max(smem, static_cast<size_t>(gate::BM) * LB_MAX_K_GATE * 4 + 1024);   // the hand-over lists
+    {
+        // no more CTAs per SM than TMEM serves (a cluster's CTA blocked in
+        // tcgen05.alloc behind a sibling waiting at the cluster barrier
+        // would never proceed)
+        const size_t max_ctas = 512 / p.tmem_cols;
+        smem = std::max(smem, static_cast<size_t>(228 * 1024) / (max_ctas + 1) + 1);
+        if (smem > 224 * 1024) return LB_EINVAL;
+    }
+    p.stages = stages;
+    CUtensorMap ma, mb;
+    if (!make_map(&ma, h, static_cast<uint64_t>(p.H), static_cast<uint64_t>(p.T), static_cast<uint64_t>(nbatch),
+                  gate::BM)) {
+        std::snprintf(g_last_error, sizeof g_last_error, "cuTensorMapEncodeTiled failed for h");
+        return LB_ECUDA;
+    }
+    if (!make_map(&mb, w, static_cast<uint64_t>(p.H), static_cast<uint64_t>(p.E), static_cast<uint64_t>(nbatch),
+                  static_cast<uint32_t>(Nc))) {
+        std::snprintf(g_last_error, sizeof g_last_error, "cuTensorMapEncodeTiled failed for w");
+        return LB_ECUDA;
+    }
+    return launch_gate_k<false, true>(p.k, ma, mb, p, mtiles, nbatch, smem, s);
 }
 
 template <int K, bool VEC>
@@ -508,7 +550,9 @@ int lb_gate_tuning(int stages, int split, int persistent, int kbox, int tiles_pe
     if (max_ctas < 0) return LB_EINVAL;
     if (kbox != 0 && kbox != 1 && kbox != 2 && kbox != 4) return LB_EINVAL;
     if (stages != 0 && (stages < 2 || stages > gate::MAX_STAGES)) return LB_EINVAL;
-    if (split != 0 && split != 1 && split != 2 && split != 4 && split != 8 && split != 16) return LB_EINVAL;
+    if (split != 0 && split != 1 && split != 2 && split != 4 && split != 8 && split != 16 && split != -2 &&
+        split != -4 && split != -8)
+        return LB_EINVAL;
     if (persistent != -1 && persistent != 0 && persistent != 1 && persistent != 2 && persistent != 3 &&
         persistent != 4)
         return LB_EINVAL;
@@ -578,14 +622,26 @@ int lb_predict_topk(const void *h, const void *w, const float *bias, int nbatch,
         return run_persistent(p, h, nbatch, mb, per_sm, mtiles, ntiles, sms, s);
     }
 
-    // split of H across a cluster when the token tiles alone underfill the GPU
+    // Split across a cluster when the token tiles alone underfill the GPU.
+    // Automatic (measured at H=7168, E=256; the CTAs stream their operands
+    // from L2, so the split that moves the fewest bytes per CTA within one
+    // wave wins): split H over the most CTAs per tile that still fit one wave
+    // (decode shape T=4096: 4 per tile, 35 us, against 80 us for 8 in two waves); where
+    // that is two or fewer, split N in two instead (T=8192: 57 us, against
+    // 67 us for H in two).  A negative tuning value splits N.
+    if (g_tune_split < 0) return run_splitn(p, h, w, nbatch, mtiles, -g_tune_split, s);
     int S = 1;
     if (g_tune_split) {
         S = g_tune_split;
     } else {
-        while (static_cast<long long>(mtiles) * nbatch * S < sms && S * 2 <= 16 && S * 2 <= p.nkb / 2 &&
+        // (sixteen only for one or two tiles: at T=1024, eight tiles, eight per
+        // tile took 26.7 us against 43.7 us for sixteen)
+        const int smax = ntiles <= 2 ? 16 : 8;
+        while (static_cast<long long>(mtiles) * nbatch * S * 2 <= sms && S * 2 <= smax && S * 2 <= p.nkb / 2 &&
                p.Epad % (4 * S * 2) == 0)
             S *= 2;
+        if (S <= 2 && ntiles * 2 <= sms && ntiles < sms && p.Epad % 32 == 0 && p.Epad / 2 >= 32)
+            return run_splitn(p, h, w, nbatch, mtiles, 2, s);
     }
     // each of the S CTAs of a cluster reduces Epad/S columns per row with
     // 16-byte shared-memory loads, so Epad/S must be a multiple of 4

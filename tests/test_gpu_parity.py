@@ -118,7 +118,7 @@ def test_decode_steps(T):
         parity.check_path(path, b, 12)
 
 
-@pytest.mark.parametrize("T", [64, 8192])
+@pytest.mark.parametrize("T", [64, 1024, 4096, 8192])
 def test_decode_gate(T):
     """Gate at the decode shape (H=7168, E=256): the cluster split of H is
     what runs at small T."""
@@ -133,17 +133,20 @@ def test_decode_gate(T):
 
 @pytest.mark.parametrize("T,H,E,k", [(200, 72, 60, 5), (1, 8, 16, 1), (333, 128, 256, 16), (130, 64, 17, 3),
                                      (4096, 256, 128, 8), (96, 2048, 32, 2)])
-@pytest.mark.parametrize("split", [0, 1, 2, 4, "persistent"])
+@pytest.mark.parametrize("split", [0, 1, 2, 4, -2, -4, -8, "persistent"])
 def test_gate_shapes(T, H, E, k, split):
     """Ragged token tails, E not a multiple of 16, H not a multiple of 64,
-    tiny and maximum k, every split of H, and the persistent kernel."""
+    tiny and maximum k, every split of H, every split of N across a cluster
+    (negative values), and the persistent kernel."""
     nkb = (H + 63) // 64
     Epad = (E + 15) // 16 * 16
     if split == "persistent":
         _lib.lb_gate_tuning(0, 0, 1)
     else:
-        if split > nkb or (split and Epad % (4 * split) != 0):
-            pytest.skip("split not valid for this shape")
+        if split > nkb or (split > 0 and Epad % (4 * split) != 0):
+            pytest.skip("split of H not valid for this shape")
+        if split < 0 and (Epad % (16 * -split) != 0 or Epad // -split < 16):
+            pytest.skip("split of N not valid for this shape")
         _lib.lb_gate_tuning(0, split, -1)
     g = torch.Generator(device=DEV).manual_seed(T * 7 + H + E + k)
     h = torch.randn(T, H, generator=g, device=DEV).to(torch.bfloat16)
