@@ -400,6 +400,7 @@ def per_config_latency(dev, world, main_wl, main_lat, reps, decode_steps=1000):
             del hid, W, bias
         out[name] = {"shape": f"T={wl.T}, H={wl.H}, E={wl.E}, top-{wl.k}, G={wl.G}, N={wl.N} (L={wl.L})",
                      "t_solve_us": max_over_ranks(lat["solve"], world),
+                     "t_solve_separate_us": lat["solve_separate"], "t_solve_fused_us": lat["solve_fused"],
                      "t_split_us": max_over_ranks(lat["split"], world),
                      "t_lookahead_us": max_over_ranks(lat["lookahead"], world),
                      "per_kernel_us": lat["kernels"]}
@@ -501,6 +502,7 @@ def per_layer_latency(wl, hid, W, bias, dev, reps):
 
     res = {
         "solve": timed(p1.solve),
+        "solve_separate": timed(p1.solve_separate),
         "solve_fused": timed(p1.solve_fused),
         "split": timed(lambda: _lib.lb_split(p1.cnt, p1.plan, N, 12,
                                              out=(p1.tok, p1.mass, p1.loads, p1.passes_run))),

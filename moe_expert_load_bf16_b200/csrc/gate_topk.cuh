@@ -467,12 +467,14 @@ __device__ __forceinline__ void merge_sorted(uint32_t (&key)[KMAX], const uint32
 // (rank 1's loads complete there), rank 0's MMA warp issues every MMA and
 // commits to the stage-free and accumulator-full barriers of both CTAs, and
 // the epilogue warps of both CTAs release an accumulator buffer on rank 0's
-// empty barrier.  Each CTA ranks its own 128 rows.  (MP = 1, ES = 4.)
+// empty barrier.  Each CTA ranks its own 128 rows of each M-tile.  With
+// MP = 2 a unit is two such pair tiles (512 tokens) sharing every W box,
+// each into its own accumulator (sixteen epilogue warps, ES = 4).
 template <int KMAX, int ES, int MP, bool PAIR = false>
 __global__ void __launch_bounds__(Shape<ES>::THREADS, ES == 2 ? 2 : 1)
     gate_topk_persistent(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                          const Params p, int mtiles, int ntiles) {
-    static_assert(!PAIR || (MP == 1 && ES == 4), "CTA pairs: one tile per CTA and sixteen epilogue warps");
+    static_assert(!PAIR || ES == 4, "CTA pairs: sixteen epilogue warps");
     extern __shared__ uint8_t smem_raw[];
     pdl_begin();
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -553,7 +555,9 @@ __global__ void __launch_bounds__(Shape<ES>::THREADS, ES == 2 ? 2 : 1)
             bool ok = true;
             for (int tile = ufirst; tile < ntiles && ok; tile += ustep) {
                 const int b = tile / mtiles;
-                const int m0 = PAIR ? (tile - b * mtiles) * 2 * BM + crank * BM : (tile - b * mtiles) * BM * MP;
+                // PAIR: M-tile mt of the unit is rows [mt 2BM, (mt+1) 2BM) of it,
+                // this CTA's half of them starting at m0 + mt 2BM
+                const int m0 = PAIR ? (tile - b * mtiles) * 2 * BM * MP + crank * BM : (tile - b * mtiles) * BM * MP;
                 for (int ks = 0; ks < nks; ++ks, ++it) {
                     const int s = it % stages;
                     const uint32_t ph = (it / stages) & 1;
@@ -569,8 +573,11 @@ __global__ void __launch_bounds__(Shape<ES>::THREADS, ES == 2 ? 2 : 1)
                         // own h rows and its half of the B rows
                         if (crank == 0) mbar_arrive_expect_tx(&full_bar[s], 2 * stage_bytes);
                         const uint32_t fb = full0 + static_cast<uint32_t>(s) * 8u;
-                        for (int j = 0; j < kbox; ++j)
-                            tma_load_3d_pair(&tmA, sa + j * a_box, fb, (ks * kbox + j) * BK, m0, b, pol_a);
+#pragma unroll
+                        for (int mt = 0; mt < MP; ++mt)
+                            for (int j = 0; j < kbox; ++j)
+                                tma_load_3d_pair(&tmA, sa + (mt * kbox + j) * a_box, fb, (ks * kbox + j) * BK,
+                                                 m0 + mt * 2 * BM, b, pol_a);
                         const int half = p.Epad / 2;
                         const int by = (p.chain ? (b - 1) * p.E : 0) + crank * half, bz = p.chain ? 0 : b;
                         for (int j = 0; j < kbox; ++j)
@@ -635,7 +642,8 @@ __global__ void __launch_bounds__(Shape<ES>::THREADS, ES == 2 ? 2 : 1)
                             for (int kk = 0; kk < BK / UK; ++kk) {
                                 const uint32_t acc = (ks > 0 || j > 0 || kk > 0) ? 1u : 0u;
                                 if constexpr (PAIR)
-                                    umma_bf16_pair(d, sw128_kmajor_desc(sa + kk * UK * 2),
+                                    umma_bf16_pair(d + mt * static_cast<uint32_t>(p.Epad),
+                                                   sw128_kmajor_desc(sa + kk * UK * 2),
                                                    sw128_kmajor_desc(sb + kk * UK * 2), idesc, acc);
                                 else
                                     umma_bf16(d + mt * static_cast<uint32_t>(p.Epad), sw128_kmajor_desc(sa + kk * UK * 2),
@@ -688,7 +696,8 @@ __global__ void __launch_bounds__(Shape<ES>::THREADS, ES == 2 ? 2 : 1)
             const int buf = tl % nbuf;
             const uint32_t use = static_cast<uint32_t>(tl / nbuf);
             const int b = tile / mtiles;
-            const int m0 = PAIR ? (tile - b * mtiles) * 2 * BM + crank * BM : (tile - b * mtiles) * BM * MP + mt * BM;
+            const int m0 = PAIR ? (tile - b * mtiles) * 2 * BM * MP + mt * 2 * BM + crank * BM
+                                : (tile - b * mtiles) * BM * MP + mt * BM;
             // The layer this warp's columns belong to (uniform over the tile).
             const int layer = p.chain ? b - 1 + gate_id : b;
             const bool live = layer >= 0 && (!p.chain || layer < p.L);   // the gate has a layer here

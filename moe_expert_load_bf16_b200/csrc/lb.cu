@@ -231,17 +231,23 @@ size_t persistent_static_smem(int k) {
     return 64 * 1024;
 }
 
-template <int KMAX>
+template <int KMAX, int MP>
 size_t static_smem_pair_of() {
     cudaFuncAttributes a{};
-    return cudaFuncGetAttributes(&a, gate::gate_topk_persistent<KMAX, 4, 1, true>) == cudaSuccess ? a.sharedSizeBytes
-                                                                                                 : 64 * 1024;
+    return cudaFuncGetAttributes(&a, gate::gate_topk_persistent<KMAX, 4, MP, true>) == cudaSuccess
+               ? a.sharedSizeBytes
+               : 64 * 1024;
 }
 
-size_t persistent_static_smem_pair(int k) {
-    if (k <= 2) return static_smem_pair_of<2>();
-    if (k <= 4) return static_smem_pair_of<4>();
-    return static_smem_pair_of<8>();
+size_t persistent_static_smem_pair(int k, int mp) {
+    if (mp == 2) {
+        if (k <= 2) return static_smem_pair_of<2, 2>();
+        if (k <= 4) return static_smem_pair_of<4, 2>();
+        return static_smem_pair_of<8, 2>();
+    }
+    if (k <= 2) return static_smem_pair_of<2, 1>();
+    if (k <= 4) return static_smem_pair_of<4, 1>();
+    return static_smem_pair_of<8, 1>();
 }
 
 size_t persistent_static_smem(int k, int es, int mp) {
@@ -251,10 +257,10 @@ size_t persistent_static_smem(int k, int es, int mp) {
 
 // CTA-pair launch of the persistent gate (clusters of two CTAs sharing one
 // MMA of M = 256; sixteen epilogue warps, k <= 8).
-template <int KMAX>
+template <int KMAX, int MP>
 int launch_gate_pair(const CUtensorMap &ma, const CUtensorMap &mb, const gate::Params &p, int units, int nunits,
                      int grid, size_t smem, cudaStream_t s) {
-    auto kern = gate::gate_topk_persistent<KMAX, 4, 1, true>;
+    auto kern = gate::gate_topk_persistent<KMAX, 4, MP, true>;
     static SmemLimit lim;
     if (!allow_smem(kern, lim, smem, false)) return LB_ECUDA;
     cudaLaunchConfig_t cfg = {};
@@ -280,16 +286,26 @@ int launch_gate_pair(const CUtensorMap &ma, const CUtensorMap &mb, const gate::P
 // accumulators of Epad columns.
 int run_pair(gate::Params &p, const void *h, int nprob, const CUtensorMap &mb, int sms, cudaStream_t s) {
     if (p.k > 8 || p.Epad % 16 != 0 || p.Epad < 16 || p.Epad > 256) return LB_EINVAL;
+    // work units of one pair tile (256 tokens), or two sharing every W box
+    // (tuning: two tiles per unit; single-buffered accumulator when two
+    // double-buffered pairs of accumulators would not fit TMEM)
+    const int mp = g_tune_mp == 2 ? 2 : 1;
+    int nbuf = 2;
+    uint32_t need = 2u * mp * static_cast<uint32_t>(p.Epad);
+    if (need > 512u) {
+        nbuf = 1;
+        need = static_cast<uint32_t>(mp) * static_cast<uint32_t>(p.Epad);
+    }
     uint32_t pcols = 32;
-    while (pcols < 2u * static_cast<uint32_t>(p.Epad)) pcols <<= 1;
+    while (pcols < need) pcols <<= 1;
     if (pcols > 512) return LB_EINVAL;
     p.tmem_cols = pcols;
-    p.nbuf = 2;
+    p.nbuf = nbuf;
     p.split = 1;
-    const size_t stat = persistent_static_smem_pair(p.k);
+    const size_t stat = persistent_static_smem_pair(p.k, mp);
     const size_t room = 227 * 1024 - stat - 2048;
-    const size_t box_bytes = 16384 + static_cast<size_t>(p.Epad / 2) * 128;
-    p.kbox = g_tune_kbox ? g_tune_kbox : 2;
+    const size_t box_bytes = 16384 * static_cast<size_t>(mp) + static_cast<size_t>(p.Epad / 2) * 128;
+    p.kbox = g_tune_kbox ? g_tune_kbox : (mp == 2 ? 1 : 2);
     if (p.kbox * box_bytes * 2 + 1024 > std::min<size_t>(224 * 1024, room + 1024)) p.kbox = 1;
     const size_t stage_bytes = box_bytes * p.kbox;
     const size_t fit = std::min<size_t>(224 * 1024 - 1024, room) / stage_bytes;
@@ -306,7 +322,7 @@ int run_pair(gate::Params &p, const void *h, int nprob, const CUtensorMap &mb, i
         std::snprintf(g_last_error, sizeof g_last_error, "cuTensorMapEncodeTiled failed for h");
         return LB_ECUDA;
     }
-    const int units = (p.T + 2 * gate::BM - 1) / (2 * gate::BM);
+    const int units = (p.T + 2 * gate::BM * mp - 1) / (2 * gate::BM * mp);
     const long long nunits = static_cast<long long>(units) * nprob;
     long long cap = sms / 2;
     if (g_tune_max_ctas > 0) cap = std::min<long long>(cap, g_tune_max_ctas / 2);
@@ -314,9 +330,14 @@ int run_pair(gate::Params &p, const void *h, int nprob, const CUtensorMap &mb, i
     const long long rounds = (nunits + cap - 1) / cap;
     const int grid = 2 * static_cast<int>((nunits + rounds - 1) / rounds);
     const int nu = static_cast<int>(nunits);
-    if (p.k <= 2) return launch_gate_pair<2>(ma, mb, p, units, nu, grid, smem, s);
-    if (p.k <= 4) return launch_gate_pair<4>(ma, mb, p, units, nu, grid, smem, s);
-    return launch_gate_pair<8>(ma, mb, p, units, nu, grid, smem, s);
+    if (mp == 2) {
+        if (p.k <= 2) return launch_gate_pair<2, 2>(ma, mb, p, units, nu, grid, smem, s);
+        if (p.k <= 4) return launch_gate_pair<4, 2>(ma, mb, p, units, nu, grid, smem, s);
+        return launch_gate_pair<8, 2>(ma, mb, p, units, nu, grid, smem, s);
+    }
+    if (p.k <= 2) return launch_gate_pair<2, 1>(ma, mb, p, units, nu, grid, smem, s);
+    if (p.k <= 4) return launch_gate_pair<4, 1>(ma, mb, p, units, nu, grid, smem, s);
+    return launch_gate_pair<8, 1>(ma, mb, p, units, nu, grid, smem, s);
 }
 
 // Persistent gate launch shared by lb_predict_topk and lb_predict_topk_chain:

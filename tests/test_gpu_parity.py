@@ -797,18 +797,20 @@ def test_gate_two_tiles_per_unit(chain, tpu, persistent, E):
         assert (ref == ids_).all(dim=1).float().mean().item() > 0.999
 
 
+@pytest.mark.parametrize("tpu", [1, 2])
 @pytest.mark.parametrize("chain", [True, False])
 @pytest.mark.parametrize("T,H,E,k,B,bias_on", [(4096, 2048, 128, 8, 3, True), (1100, 576, 64, 8, 2, True),
                                                (300, 128, 16, 2, 2, False), (2900, 4096, 128, 4, 1, True),
                                                (130, 64, 48, 8, 3, True)])
-def test_gate_cta_pairs(chain, T, H, E, k, B, bias_on):
+def test_gate_cta_pairs(chain, T, H, E, k, B, bias_on, tpu):
     """CTA pairs (clusters of two CTAs sharing one MMA of M = 256, each CTA
     loading its 128 tokens and half of the weight rows): ids and logits of
     every problem pass the oracle check on sampled rows (all rows of short
     problems), and agree with the one-CTA persistent kernel.  Shapes: an odd
     number of 128-token tiles (the last unit's second tile lies past T), a
     ragged tail, H past the last full stage of boxes, E = 16 (N = 32 chain),
-    E = 48 (N = 48 per gate), no bias."""
+    E = 48 (N = 48 per gate), no bias; one or two pair tiles per work unit
+    (the second sharing every weight box)."""
     if not chain and E % 16:
         pytest.skip("pairs need E % 16 == 0 in the per-layer gate")
     g = torch.Generator(device=DEV).manual_seed(T + H + E + k + B)
@@ -816,7 +818,7 @@ def test_gate_cta_pairs(chain, T, H, E, k, B, bias_on):
     h = torch.randn(nh, T, H, generator=g, device=DEV).to(torch.bfloat16)
     W = (torch.randn(B, E, H, generator=g, device=DEV) / H ** 0.5).to(torch.bfloat16)
     bias = torch.randn(B, E, generator=g, device=DEV) if bias_on else None
-    _lib.lb_gate_tuning(0, 0, 3)
+    _lib.lb_gate_tuning(0, 0, 3, 0, tpu)
     if chain:
         out = _lib.lb_predict_topk_chain(h, W, bias, k, want_logits=True)
     else:
