@@ -310,6 +310,7 @@ def run_ours(args, world, rank, local):
     lat = per_layer_latency(wl, hid, W, bias, dev, reps=max(50, args.steps))
     per_config = per_config_latency(dev, world, wl, lat, reps=max(50, args.steps),
                                     decode_steps=args.decode_steps)
+    gate_shapes = gate_fractions(dev, world)
 
     # ---------------- count / split / assign as throughput kernels
     ints = integer_kernels_at_throughput(dev, world)
@@ -349,6 +350,7 @@ def run_ours(args, world, rank, local):
         "per_kernel_us": lat["kernels"],
         "roofline": roofline,
         "per_config": per_config,
+        "gate_shapes": gate_shapes,
         "integer_kernels": ints,
         "swap_planner": swp,
         "e2e": e2e,
@@ -379,6 +381,62 @@ def gate_roofline(nbytes, flops, ms, hbm, tflops, tflops_sus, peak_kind, traffic
                tensor_frac=t_tensor / s, tensor_frac_of_sustained=flops / (tflops_sus * 1e12) / s,
                sustained_tflops=tflops_sus,
                traffic_over_algorithmic=(traffic / nbytes if traffic else None))
+    return out
+
+
+def gate_fractions(dev, world, reps=20):
+    """The gate on every configuration's shape, against its roofline
+    (max(bytes / HBM peak, flops / tensor peak) / time, burst peaks): the
+    chain gate over 16 layers of each prefill configuration, and the
+    per-layer gate of the decode shape (H=7168, E=256) at every T."""
+    from moe_expert_load_bf16_b200 import _lib, workloads
+    hbm, tflops, _, peak_kind = peaks()
+
+    def timed(fn):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            fn()
+        g.replay()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier(world)
+        a.record()
+        for _ in range(reps):
+            g.replay()
+        b.record()
+        torch.cuda.synchronize()
+        return max_over_ranks(a.elapsed_time(b) * 1e3 / reps, world)
+
+    def frac(nbytes, flops, us):
+        return {"us": us, "hbm_frac": nbytes / us / 1e3 / hbm, "tensor_frac": flops / us / 1e6 / tflops,
+                "roofline_frac": max(nbytes / (hbm * 1e3), flops / (tflops * 1e6)) / us}
+
+    out = {"peak_kind": peak_kind}
+    for name in ("olmoe", "qwen3-30b", "qwen3-235b"):
+        wl = workloads.WORKLOADS[name]
+        nl = min(16, wl.layers)
+        hid = torch.empty(nl + 1, wl.T, wl.H, dtype=torch.bfloat16, device=dev)
+        workloads.hidden_chain(wl, nl, out=hid[1:])
+        hid[0].copy_(hid[1])
+        W = workloads.gate_weights(wl, nl, device=dev)
+        bias = workloads.biases(wl, nl).to(dev)
+        ip = torch.empty(nl, wl.T, wl.k, dtype=torch.int32, device=dev)
+        ia = torch.empty_like(ip)
+        us = timed(lambda: _lib.lb_predict_topk_chain(hid, W, bias, wl.k, ids_pred=ip, ids_act=ia))
+        nbytes = (nl + 1) * 2 * wl.T * wl.H + nl * (2 * wl.H * wl.E + 4 * wl.E + 8 * wl.T * wl.k)
+        out[f"chain_{name}"] = dict(frac(nbytes, nl * 4.0 * wl.T * wl.H * wl.E, us), layers=nl)
+        del hid, W, bias, ip, ia
+    wl = workloads.WORKLOADS["decode"]
+    W = workloads.gate_weights(wl, 1, device=dev)[0]
+    bias = workloads.biases(wl, 1)[0].to(dev)
+    for T in wl.decode_T:
+        h = workloads.hidden_chain(wl, 1, device=dev, T=T)[0]
+        ids = torch.empty(T, wl.k, dtype=torch.int32, device=dev)
+        us = timed(lambda: _lib.lb_predict_topk(h, W, bias, wl.k, ids=ids))
+        nbytes = 2 * T * wl.H + 2 * wl.H * wl.E + 4 * wl.E + 4 * T * wl.k
+        out[f"decode_T{T}"] = frac(nbytes, 2.0 * T * wl.H * wl.E, us)
+        del h, ids
+    torch.cuda.empty_cache()
     return out
 
 

@@ -12,8 +12,9 @@ both gates that read one hidden state in a single pass over it:
   cnt      = counts(ids)                                    lb_count
   tok, mass, loads = split(cnt, plan)                       lb_split
   dest, perm, offs = assign(ids, cnt, plan, split)          lb_assign
-(`solve` runs split and assign as lb_decide: split and the assign's tables
-in one launch per problem, the scatter in a second.)
+(`solve` runs count, split and assign as lb_count + lb_decide: split and the
+assign's tables in one launch per problem, the scatter in a second; or, for
+problems of more than FUSED_ABOVE assignments, as one lb_solve launch.)
 """
 import torch
 
@@ -56,8 +57,18 @@ class DecisionPath:
     # assign by lb_decide (split and the assign's tables in one launch per
     # problem, the scatter in a second); solve_separate makes the same bytes
     # with lb_split and lb_assign
+    # Problems of more than this many assignments take the fused lb_solve
+    # (one cluster of up to 16 CTAs per problem spreads the scatter; measured
+    # per layer: Qwen3-235B-shaped 57.4 against 71.7 us); smaller ones
+    # lb_count + lb_decide (OLMoE-shaped 34.8 against 38.5 us, Qwen3-30B-shaped
+    # 51.2 against 55.3 us).  The outputs are identical either way.
+    FUSED_ABOVE = 131072
+
     def solve(self, ids=None, counted=False):
         ids = self.ids if ids is None else ids
+        if self.T * self.k > self.FUSED_ABOVE:
+            self.solve_fused(ids)
+            return
         if not counted:
             _lib.lb_count(ids, self.G, self.E, cnt=self.cnt)
         self.decide(ids)
