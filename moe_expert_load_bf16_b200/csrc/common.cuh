@@ -20,7 +20,9 @@ __device__ __forceinline__ void flag(int bits) { atomicOr(&g_status, bits); }
 // Phase timestamps of block 0 for latency analysis builds (-DLB_TIMING);
 // compiled out otherwise.
 #ifdef LB_TIMING
-__device__ long long g_ticks[64];
+// [0, 64): phase stamps of block 0; [64, 64 + 1024): start and end
+// (globaltimer, ns) of CTAs 0..511 of the kernels that record them
+__device__ long long g_ticks[64 + 1024];
 // (the clock read carries a memory clobber, so it stays between the memory
 // operations and barriers around it)
 __device__ __forceinline__ long long lb_clock() {
@@ -32,9 +34,29 @@ __device__ __forceinline__ long long lb_clock() {
     do {                                                                                       \
         if (threadIdx.x == 0 && blockIdx.x == 0 && blockIdx.y == 0) lb::g_ticks[slot] = lb::lb_clock(); \
     } while (0)
+#define LB_CTA_TIME(which)                                                                     \
+    do {                                                                                       \
+        const unsigned cta_ = blockIdx.x + blockIdx.y * gridDim.x;                             \
+        if (cta_ < 512u) {                                                                     \
+            long long t_;                                                                      \
+            asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t_)::"memory");                   \
+            lb::g_ticks[64 + 2 * cta_ + (which)] = t_;                                         \
+        }                                                                                      \
+    } while (0)
+// stamp by whichever thread of block 0 calls it (the caller picks the thread)
+#define LB_TICK_ANY(slot)                                                      \
+    do {                                                                       \
+        if (blockIdx.x == 0 && blockIdx.y == 0) lb::g_ticks[slot] = lb::lb_clock(); \
+    } while (0)
 #else
 #define LB_TICK(slot) \
     do {              \
+    } while (0)
+#define LB_TICK_ANY(slot) \
+    do {                  \
+    } while (0)
+#define LB_CTA_TIME(which) \
+    do {                   \
     } while (0)
 #endif
 
@@ -300,6 +322,19 @@ __device__ __forceinline__ int ld_cluster_i32(uint32_t addr) {
     int v;
     asm volatile("ld.shared::cluster.s32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
     return v;
+}
+// Bulk copy of `bytes` (a multiple of 16, both addresses 16-byte aligned)
+// from this CTA's shared memory into another CTA's of the cluster (dst and
+// bar are cluster addresses from mapa); completes on the receiver's mbarrier.
+__device__ __forceinline__ void bulk_copy_to_cta(uint32_t dst, uint32_t src, uint32_t bytes, uint32_t bar) {
+    asm volatile("cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+                 "r"(src), "r"(bytes), "r"(bar)
+                 : "memory");
+}
+// Order this thread's shared-memory writes before later async-proxy reads
+// of them (a bulk copy issued after a barrier).
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 __device__ __forceinline__ float4 ld_cluster_f4(uint32_t addr) {
     float4 v;

@@ -31,6 +31,24 @@ constexpr int UK = 16;         // UMMA K for bf16
 constexpr int THREADS = 128;   // 4 warps; warp 0 lane 0 = TMA, warp 1 lane 0 = MMA
 constexpr int MAX_STAGES = 8;
 
+// The TMA producers are whole warps.  One thread's tensor copies are served
+// one after another (measured on B200: one issuing thread feeds an SM at
+// about 38 GB/s from L2 however many copies it has in flight, each further
+// thread adds about as much, up to the SM's share of L2 bandwidth), so every
+// copy in flight gets its own lane: box j of stage slot s is issued by lane
+// (s * nbox + j) mod 32.
+__device__ __forceinline__ bool issues_box(int s, int nbox, int j, int lane) {
+    return ((s * nbox + j) & 31) == lane;
+}
+
+// Producer wait of a whole warp on a stage's empty barrier: lane 0 waits and
+// the warp learns the outcome (0 go on, 1 timed out, 2 aborted elsewhere).
+__device__ __forceinline__ int warp_wait_empty(uint64_t *bar, uint32_t parity, const int *abort_flag, int lane) {
+    int st = 0;
+    if (lane == 0) st = !mbar_wait(bar, parity) ? 1 : (*reinterpret_cast<const volatile int *>(abort_flag) ? 2 : 0);
+    return __shfl_sync(0xffffffffu, st, 0);
+}
+
 struct Params {
     const float *bias;   // [B,E] or null
     int32_t *ids;        // [B,T,k]
@@ -164,26 +182,27 @@ __global__ void __launch_bounds__(THREADS, 1)
     const uint32_t tmem = tmem_slot;
 
     if (warp == 0) {
-        if (lane == 0) {
-            // ---------------- TMA producer
-            int issued = 0;
-            for (int i = 0; i < nk; ++i) {
-                const int s = i % stages;
-                const uint32_t ph = (i / stages) & 1;
-                if (!mbar_wait(&empty_bar[s], ph ^ 1)) {
-                    atomicExch(&aborted, 1);
-                    flag(LB_DEV_TIMEOUT);
-                    break;
-                }
-                if (*reinterpret_cast<volatile int *>(&aborted)) break;
-                uint8_t *sa = smem + static_cast<size_t>(s) * stage_bytes;
-                mbar_arrive_expect_tx(&full_bar[s], stage_bytes);
-                tma_load_3d(&tmA, sa, &full_bar[s], (kb0 + i) * BK, m0, b);
-                tma_load_3d(&tmB, sa + a_bytes, &full_bar[s], (kb0 + i) * BK, c_off, b);
-                ++issued;
+        // ---------------- TMA producer (the whole warp, one lane per box)
+        int issued = 0;
+        for (int i = 0; i < nk; ++i) {
+            const int s = i % stages;
+            const uint32_t ph = (i / stages) & 1;
+            const int st = warp_wait_empty(&empty_bar[s], ph ^ 1, &aborted, lane);
+            if (st == 1 && lane == 0) {
+                atomicExch(&aborted, 1);
+                flag(LB_DEV_TIMEOUT);
             }
-            // Never leave with copies in flight into this CTA's shared memory:
-            // wait (bounded) for the latest phase of every stage used.
+            if (st != 0) break;
+            uint8_t *sa = smem + static_cast<size_t>(s) * stage_bytes;
+            if (lane == 0) mbar_arrive_expect_tx(&full_bar[s], stage_bytes);
+            __syncwarp();
+            if (issues_box(s, 2, 0, lane)) tma_load_3d(&tmA, sa, &full_bar[s], (kb0 + i) * BK, m0, b);
+            if (issues_box(s, 2, 1, lane)) tma_load_3d(&tmB, sa + a_bytes, &full_bar[s], (kb0 + i) * BK, c_off, b);
+            ++issued;
+        }
+        // Never leave with copies in flight into this CTA's shared memory:
+        // wait (bounded) for the latest phase of every stage used.
+        if (lane == 0) {
             for (int s = 0; s < stages && s < issued; ++s) {
                 const int last = s + ((issued - 1 - s) / stages) * stages;
                 if (!mbar_wait(&full_bar[s], (last / stages) & 1)) flag(LB_DEV_TIMEOUT);
@@ -548,62 +567,69 @@ __global__ void __launch_bounds__(Shape<ES>::THREADS, ES == 2 ? 2 : 1)
     const uint32_t accempty0 = PAIR ? mapa_shared(smem_u32(&acc_empty[0]), 0) : smem_u32(&acc_empty[0]);
 
     if (warp == 0) {
-        if (lane == 0) {
-            // ---------------- TMA producer
-            const uint64_t pol_a = l2_policy_evict_first(), pol_b = l2_policy_evict_last();
-            int it = 0;
-            bool ok = true;
-            for (int tile = ufirst; tile < ntiles && ok; tile += ustep) {
-                const int b = tile / mtiles;
-                // PAIR: M-tile mt of the unit is rows [mt 2BM, (mt+1) 2BM) of it,
-                // this CTA's half of them starting at m0 + mt 2BM
-                const int m0 = PAIR ? (tile - b * mtiles) * 2 * BM * MP + crank * BM : (tile - b * mtiles) * BM * MP;
-                for (int ks = 0; ks < nks; ++ks, ++it) {
-                    const int s = it % stages;
-                    const uint32_t ph = (it / stages) & 1;
-                    if (!mbar_wait(&empty_bar[s], ph ^ 1) || *abort_flag) {
+        // ---------------- TMA producer (the whole warp, one lane per box)
+        const uint64_t pol_a = l2_policy_evict_first(), pol_b = l2_policy_evict_last();
+        const int nbox = (MP + 1) * kbox;
+        int it = 0;
+        bool ok = true;
+        for (int tile = ufirst; tile < ntiles && ok; tile += ustep) {
+            const int b = tile / mtiles;
+            // PAIR: M-tile mt of the unit is rows [mt 2BM, (mt+1) 2BM) of it,
+            // this CTA's half of them starting at m0 + mt 2BM
+            const int m0 = PAIR ? (tile - b * mtiles) * 2 * BM * MP + crank * BM : (tile - b * mtiles) * BM * MP;
+            for (int ks = 0; ks < nks; ++ks, ++it) {
+                const int s = it % stages;
+                const uint32_t ph = (it / stages) & 1;
+                if (warp_wait_empty(&empty_bar[s], ph ^ 1, &aborted, lane) != 0) {
+                    if (lane == 0) {
                         atomicExch(&aborted, 1);
                         flag(LB_DEV_TIMEOUT);
-                        ok = false;
-                        break;
                     }
-                    uint8_t *sa = smem + static_cast<size_t>(s) * stage_bytes;
-                    if constexpr (PAIR) {
-                        // rank 0 expects both CTAs' bytes; each CTA loads its
-                        // own h rows and its half of the B rows
-                        if (crank == 0) mbar_arrive_expect_tx(&full_bar[s], 2 * stage_bytes);
-                        const uint32_t fb = full0 + static_cast<uint32_t>(s) * 8u;
+                    ok = false;
+                    break;
+                }
+                uint8_t *sa = smem + static_cast<size_t>(s) * stage_bytes;
+                if constexpr (PAIR) {
+                    // rank 0 expects both CTAs' bytes; each CTA loads its
+                    // own h rows and its half of the B rows
+                    if (crank == 0 && lane == 0) mbar_arrive_expect_tx(&full_bar[s], 2 * stage_bytes);
+                    __syncwarp();
+                    const uint32_t fb = full0 + static_cast<uint32_t>(s) * 8u;
 #pragma unroll
-                        for (int mt = 0; mt < MP; ++mt)
-                            for (int j = 0; j < kbox; ++j)
+                    for (int mt = 0; mt < MP; ++mt)
+                        for (int j = 0; j < kbox; ++j)
+                            if (issues_box(s, nbox, mt * kbox + j, lane))
                                 tma_load_3d_pair(&tmA, sa + (mt * kbox + j) * a_box, fb, (ks * kbox + j) * BK,
                                                  m0 + mt * 2 * BM, b, pol_a);
-                        const int half = p.Epad / 2;
-                        const int by = (p.chain ? (b - 1) * p.E : 0) + crank * half, bz = p.chain ? 0 : b;
-                        for (int j = 0; j < kbox; ++j)
+                    const int half = p.Epad / 2;
+                    const int by = (p.chain ? (b - 1) * p.E : 0) + crank * half, bz = p.chain ? 0 : b;
+                    for (int j = 0; j < kbox; ++j)
+                        if (issues_box(s, nbox, MP * kbox + j, lane))
                             tma_load_3d_pair(&tmB, sa + a_bytes + j * b_box, fb, (ks * kbox + j) * BK, by, bz, pol_b);
-                    } else {
-                        mbar_arrive_expect_tx(&full_bar[s], stage_bytes);
+                } else {
+                    if (lane == 0) mbar_arrive_expect_tx(&full_bar[s], stage_bytes);
+                    __syncwarp();
 #pragma unroll
-                        for (int mt = 0; mt < MP; ++mt)
-                            for (int j = 0; j < kbox; ++j)
+                    for (int mt = 0; mt < MP; ++mt)
+                        for (int j = 0; j < kbox; ++j)
+                            if (issues_box(s, nbox, mt * kbox + j, lane))
                                 tma_load_3d_hint(&tmA, sa + (mt * kbox + j) * a_box, &full_bar[s],
                                                  (ks * kbox + j) * BK, m0 + mt * BM, b, pol_a);
-                        const int by = p.chain ? (b - 1) * p.E : 0, bz = p.chain ? 0 : b;
-                        for (int j = 0; j < kbox; ++j)
+                    const int by = p.chain ? (b - 1) * p.E : 0, bz = p.chain ? 0 : b;
+                    for (int j = 0; j < kbox; ++j)
+                        if (issues_box(s, nbox, MP * kbox + j, lane))
                             tma_load_3d_hint(&tmB, sa + a_bytes + j * b_box, &full_bar[s], (ks * kbox + j) * BK, by,
                                              bz, pol_b);
-                    }
                 }
             }
-            // no copies left in flight into this CTA's shared memory (PAIR:
-            // rank 0's full barriers count both CTAs' copies; rank 1 is held
-            // at the closing cluster barrier until rank 0 has seen them land)
-            if (!PAIR || crank == 0) {
-                for (int s = 0; s < stages && s < it; ++s) {
-                    const int last = s + ((it - 1 - s) / stages) * stages;
-                    if (!mbar_wait(&full_bar[s], (last / stages) & 1)) flag(LB_DEV_TIMEOUT);
-                }
+        }
+        // no copies left in flight into this CTA's shared memory (PAIR:
+        // rank 0's full barriers count both CTAs' copies; rank 1 is held
+        // at the closing cluster barrier until rank 0 has seen them land)
+        if (lane == 0 && (!PAIR || crank == 0)) {
+            for (int s = 0; s < stages && s < it; ++s) {
+                const int last = s + ((it - 1 - s) / stages) * stages;
+                if (!mbar_wait(&full_bar[s], (last / stages) & 1)) flag(LB_DEV_TIMEOUT);
             }
         }
     } else if (warp == 1) {
@@ -803,6 +829,341 @@ __global__ void __launch_bounds__(Shape<ES>::THREADS, ES == 2 ? 2 : 1)
         tc_fence_after();
         if constexpr (PAIR) tmem_dealloc_pair(tmem, p.tmem_cols);
         else tmem_dealloc(tmem, p.tmem_cols);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Top KMAX of two descending key lists, into a (descending): the elementwise
+// maximum of a and b reversed holds the KMAX largest keys of both as a
+// bitonic sequence, which a half-cleaner network then sorts.
+template <int KMAX>
+__device__ __forceinline__ void merge_top(uint32_t (&a)[KMAX], const uint32_t (&b)[KMAX]) {
+#pragma unroll
+    for (int j = 0; j < KMAX; ++j) a[j] = max(a[j], b[KMAX - 1 - j]);
+#pragma unroll
+    for (int st = KMAX / 2; st >= 1; st >>= 1)
+#pragma unroll
+        for (int j = 0; j < KMAX; ++j)
+            if ((j & st) == 0) {
+                const uint32_t hi = max(a[j], a[j + st]), lo = min(a[j], a[j + st]);
+                a[j] = hi;
+                a[j + st] = lo;
+            }
+}
+
+// Four keys into a descending top-KMAX list: sort them (the optimal network
+// of five comparators), then merge as above with the four standing in for a
+// list padded with the smallest key.  About half the operations of four
+// separate insertions for KMAX = 8.
+__device__ __forceinline__ void cmp_swap_desc(uint32_t &x, uint32_t &y) {
+    const uint32_t hi = max(x, y), lo = min(x, y);
+    x = hi;
+    y = lo;
+}
+template <int KMAX>
+__device__ __forceinline__ void push4(uint32_t (&a)[KMAX], uint32_t k0, uint32_t k1, uint32_t k2, uint32_t k3) {
+    cmp_swap_desc(k0, k1);
+    cmp_swap_desc(k2, k3);
+    cmp_swap_desc(k0, k2);
+    cmp_swap_desc(k1, k3);
+    cmp_swap_desc(k1, k2);
+    const uint32_t bk[4] = {k0, k1, k2, k3};
+    constexpr int m = KMAX < 4 ? KMAX : 4;
+#pragma unroll
+    for (int j = KMAX - m; j < KMAX; ++j) a[j] = max(a[j], bk[KMAX - 1 - j]);
+#pragma unroll
+    for (int st = KMAX / 2; st >= 1; st >>= 1)
+#pragma unroll
+        for (int j = 0; j < KMAX; ++j)
+            if ((j & st) == 0) cmp_swap_desc(a[j], a[j + st]);
+}
+
+// CTA pairs with H split over KS pairs (per-tile, one 256-token unit per
+// cluster of 2 KS CTAs; the per-layer gate of wide shapes whose token tiles
+// underfill the GPU, such as the decode shape).  Ranks 2p and 2p+1 form pair
+// p; within a pair, as in the persistent kernel, the even rank issues one
+// tcgen05.mma of M = 256 for both, each CTA loading its own 128 tokens and
+// half of the N = Epad weight rows.  Pair p accumulates k-blocks
+// [p kper, (p+1) kper), kper = ceil(nkb / KS).
+//
+// The partial accumulators are summed by a reduce-scatter over distributed
+// shared memory.  Each CTA copies its partial (128 rows x Epad fp32) from
+// TMEM into its own shared memory (rows of SR = Epad rounded up to 32
+// floats, float4 group g of row r stored at g ^ (r mod 8), which keeps both
+// the row-per-lane writes and the row-major reads free of bank conflicts).
+// After a cluster barrier (every MMA of the cluster done, so every CTA's
+// pipeline buffers are free), it sends rows [p' R, (p'+1) R) (R = 128 / KS)
+// to the CTA of pair p' holding the same tokens, one bulk shared-to-shared
+// copy per pair, each completing on the receiver's mbarrier.  Each CTA then
+// ranks its own R rows: its partial plus the received ones in pair order
+// (deterministic) plus the bias, 512 / R threads per row over interleaved
+// float4 groups, their lists merged by shuffles.
+template <int KMAX, int KS>
+__global__ void __launch_bounds__(Shape<4>::THREADS, 1)
+    gate_topk_pairk(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                    const Params p) {
+    constexpr int R = BM / KS;                  // rows this CTA ranks
+    constexpr int TPR = Shape<4>::EPI / R;      // ranking threads per row
+    static_assert(KS == 2 || KS == 4, "two or four pairs");
+    static_assert(TPR <= 32 && 32 % TPR == 0, "a row's ranking threads share a warp");
+    extern __shared__ uint8_t smem_raw[];
+    pdl_begin();
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                                ~static_cast<uintptr_t>(1023));
+    __shared__ __align__(8) uint64_t full_bar[MAX_STAGES];
+    __shared__ __align__(8) uint64_t empty_bar[MAX_STAGES];
+    __shared__ __align__(8) uint64_t acc_full;
+    __shared__ __align__(8) uint64_t drain_bar;
+    __shared__ __align__(8) uint64_t recv_bar;
+    __shared__ uint32_t tmem_slot;
+    __shared__ int aborted;
+    __shared__ __align__(16) float bias_s[LB_MAX_E_GATE];
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int crank = static_cast<int>(cluster_ctarank());
+    const int pair = crank >> 1, half = crank & 1, lead = crank & ~1;
+    const int b = blockIdx.y;
+    const int unit = static_cast<int>(blockIdx.x) / (2 * KS);
+    const int m0 = unit * 2 * BM + half * BM;   // this CTA's 128 rows
+    const int kper = (p.nkb + KS - 1) / KS;
+    const int kb0 = pair * kper;
+    const int kend = min(p.nkb, kb0 + kper);
+    const int kbox = p.kbox;
+    const int nks = (max(0, kend - kb0) + kbox - 1) / kbox;   // stages of kbox boxes
+    const uint32_t a_box = BM * 128u, b_box = static_cast<uint32_t>(p.Epad / 2) * 128u;
+    const uint32_t a_bytes = a_box * kbox;
+    const uint32_t stage_bytes = (a_box + b_box) * kbox;
+    const int stages = p.stages;
+    const int SR = (p.Epad + 31) & ~31;                         // staged row stride (floats)
+    const uint32_t slice_bytes = static_cast<uint32_t>(R * SR) * 4u;
+    if (tid == 0) {
+        LB_TICK_ANY(40);
+        LB_CTA_TIME(0);
+    }
+
+    for (int c = tid; c < p.Epad; c += Shape<4>::THREADS)
+        bias_s[c] = (p.bias != nullptr && c < p.E) ? p.bias[static_cast<int64_t>(b) * p.E + c] : 0.f;
+    if (tid == 0) {
+        for (int s = 0; s < stages; ++s) {
+            mbar_init(&full_bar[s], 1);
+            mbar_init(&empty_bar[s], 1);
+        }
+        mbar_init(&acc_full, 1);
+        mbar_init(&drain_bar, 1);
+        mbar_init(&recv_bar, 1);
+        aborted = 0;
+        fence_mbar_init();
+        // the other pairs' slices of this CTA's rows land on recv_bar
+        mbar_arrive_expect_tx(&recv_bar, (KS - 1) * slice_bytes);
+        tma_prefetch_desc(&tmA);
+        tma_prefetch_desc(&tmB);
+    }
+    if (warp == 1) {
+        tmem_alloc_pair(&tmem_slot, p.tmem_cols);
+        tmem_relinquish_pair();
+    }
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync();   // every CTA's barriers and TMEM exist before any signal
+    tc_fence_after();
+    if (tid == 0) LB_TICK_ANY(41);
+    const uint32_t tmem = tmem_slot;
+    volatile int *abort_flag = &aborted;
+    const uint32_t full0 = mapa_shared(smem_u32(&full_bar[0]), static_cast<uint32_t>(lead));
+    const uint16_t pair_mask = static_cast<uint16_t>(3u << lead);
+
+    if (warp == 0) {
+        // ---------------- TMA producer (both CTAs of the pair; the whole
+        // warp, one lane per box)
+        const uint64_t pol_a = l2_policy_evict_first(), pol_b = l2_policy_evict_last();
+        const int nbox = 2 * kbox;
+        int it = 0;
+        for (int ks = 0; ks < nks; ++ks, ++it) {
+            const int s = it % stages;
+            const uint32_t ph = (it / stages) & 1;
+            if (warp_wait_empty(&empty_bar[s], ph ^ 1, &aborted, lane) != 0) {
+                if (lane == 0) {
+                    atomicExch(&aborted, 1);
+                    flag(LB_DEV_TIMEOUT);
+                }
+                break;
+            }
+            uint8_t *sa = smem + static_cast<size_t>(s) * stage_bytes;
+            if (half == 0 && lane == 0) mbar_arrive_expect_tx(&full_bar[s], 2 * stage_bytes);
+            __syncwarp();
+            const uint32_t fb = full0 + static_cast<uint32_t>(s) * 8u;
+            for (int j = 0; j < kbox; ++j) {
+                // boxes past this pair's share of H read real data (the next
+                // pair's, or zeros past H) but are never multiplied: the MMA
+                // stops at kend
+                const int kx = (kb0 + ks * kbox + j) * BK;
+                if (issues_box(s, nbox, j, lane)) tma_load_3d_pair(&tmA, sa + j * a_box, fb, kx, m0, b, pol_a);
+                if (issues_box(s, nbox, kbox + j, lane))
+                    tma_load_3d_pair(&tmB, sa + a_bytes + j * b_box, fb, kx, half * (p.Epad / 2), b, pol_b);
+            }
+        }
+        if (half == 0 && lane == 0) {
+            for (int s = 0; s < stages && s < it; ++s) {
+                const int last = s + ((it - 1 - s) / stages) * stages;
+                if (!mbar_wait(&full_bar[s], (last / stages) & 1)) flag(LB_DEV_TIMEOUT);
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0 && half == 0) {
+            // ---------------- MMA issuer (the pair's even rank)
+            const uint32_t idesc = umma_idesc_bf16(2 * BM, p.Epad);
+            int it = 0;
+            bool first = true;
+            for (int ks = 0; ks < nks; ++ks, ++it) {
+                const int s = it % stages;
+                const uint32_t ph = (it / stages) & 1;
+                if (!mbar_wait(&full_bar[s], ph) || *abort_flag) {
+                    atomicExch(&aborted, 1);
+                    flag(LB_DEV_TIMEOUT);
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t st = smem_u32(smem + static_cast<size_t>(s) * stage_bytes);
+                for (int j = 0; j < kbox; ++j) {
+                    if (kb0 + ks * kbox + j >= kend) break;   // this pair's share of H only
+                    const uint32_t sa = st + j * a_box, sb = st + a_bytes + j * b_box;
+#pragma unroll
+                    for (int kk = 0; kk < BK / UK; ++kk) {
+                        umma_bf16_pair(tmem, sw128_kmajor_desc(sa + kk * UK * 2), sw128_kmajor_desc(sb + kk * UK * 2),
+                                       idesc, first ? 0u : 1u);
+                        first = false;
+                    }
+                }
+                umma_commit_pair(&empty_bar[s], pair_mask);
+            }
+            LB_TICK_ANY(44);
+            umma_commit_pair(&acc_full, pair_mask);
+            umma_commit_pair(&drain_bar, static_cast<uint16_t>(1u << lead));
+            if (!mbar_wait(&drain_bar, 0)) flag(LB_DEV_TIMEOUT);
+        }
+    }
+    __syncwarp();
+
+    // ---------------- epilogue warps 2..17
+    const bool epi = warp >= 2;
+    const int ew = warp - 2;
+    float *stage_f = reinterpret_cast<float *>(smem);   // [128][SR], reusing the pipeline buffers
+    float *recv_f = stage_f + BM * SR;                   // [KS-1][R][SR]
+    bool ok = true;
+    if (epi) {
+        ok = mbar_wait(&acc_full, 0) && !*abort_flag;
+        if (!ok && lane == 0) flag(LB_DEV_TIMEOUT);
+        ok = __all_sync(kFull, ok);
+        tc_fence_after();
+        if (tid == 64) LB_TICK_ANY(47);
+        // TMEM lane quadrant q = warp % 4, a quarter of the columns per warp
+        const int q = warp & 3, part = ew >> 2;
+        const int pw = ((p.Epad + 3) / 4 + 15) / 16 * 16;
+        const int cbeg = part * pw, cend = min(p.Epad, cbeg + pw);
+        const int r = q * 32 + lane;
+        float *srow = stage_f + r * SR;
+        const uint32_t tl_addr = tmem + (static_cast<uint32_t>(q * 32) << 16);
+        for (int c0 = cbeg; c0 < cend; c0 += 32) {
+            // two loads of 16 columns per wait (cend - c0 is a multiple of 16)
+            uint32_t v[2][16];
+            const bool two = c0 + 16 < cend;
+            tmem_ld16(tl_addr + c0, v[0]);
+            if (two) tmem_ld16(tl_addr + c0 + 16, v[1]);
+            tmem_wait_ld();
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                if (u >= 4 && !two) break;
+                const int g = (c0 >> 2) + u;
+                const uint32_t *w = v[u >> 2] + 4 * (u & 3);
+                *reinterpret_cast<float4 *>(srow + ((g ^ (r & 7)) << 2)) =
+                    make_float4(__uint_as_float(w[0]), __uint_as_float(w[1]), __uint_as_float(w[2]),
+                                __uint_as_float(w[3]));
+            }
+        }
+        if (tid == 64) LB_TICK_ANY(54);
+        fence_proxy_async_smem();   // the staged rows, before the bulk copies read them
+    }
+    cluster_sync();   // every partial staged; every CTA's buffers free for the slices
+    if (epi && ew == 0) {
+        // chunks of 4 rows, one lane each (one thread's bulk copies are served
+        // one after another)
+        if (lane == 0) LB_TICK_ANY(48);
+        constexpr int CH = R / 4;   // chunks per slice
+        for (int j = lane; j < (KS - 1) * CH; j += 32) {
+            const int o = j / CH, ch = j - o * CH;
+            const int pp = o < pair ? o : o + 1;             // receiving pair
+            const uint32_t dst_rank = static_cast<uint32_t>(2 * pp + half);
+            const int slot = pair < pp ? pair : pair - 1;   // this pair's slot at the receiver
+            const int roff = ch * 4 * SR;
+            bulk_copy_to_cta(mapa_shared(smem_u32(recv_f + slot * R * SR + roff), dst_rank),
+                             smem_u32(stage_f + pp * R * SR + roff), slice_bytes / CH,
+                             mapa_shared(smem_u32(&recv_bar), dst_rank));
+        }
+    }
+    if (epi) {
+        const bool got = mbar_wait(&recv_bar, 0);
+        if (!got && lane == 0) flag(LB_DEV_TIMEOUT);
+        if (tid == 64) LB_TICK_ANY(52);
+        const int lr = ew * (32 / TPR) + lane / TPR;   // row within this CTA's slice
+        const int pt = lane % TPR;
+        const int r = pair * R + lr;                   // row within the CTA's 128
+        const int row = m0 + r;
+        const bool valid = ok && got && row < p.T;
+        const uint32_t kmask = id_mask(p.E);
+        const int64_t grow = static_cast<int64_t>(b) * p.T + row;
+        float *lrow = (p.logits != nullptr && valid) ? p.logits + grow * p.E : nullptr;
+        TopK<KMAX> tk;
+        tk.init();
+        const float *own = stage_f + r * SR;
+        for (int g = pt; g < (p.Epad >> 2); g += TPR) {
+            const int sg = (g ^ (r & 7)) << 2;
+            float4 x = *reinterpret_cast<const float4 *>(own + sg);
+#pragma unroll
+            for (int o = 0; o < KS - 1; ++o) {
+                const float4 y = *reinterpret_cast<const float4 *>(recv_f + (o * R + lr) * SR + sg);
+                x.x += y.x;
+                x.y += y.y;
+                x.z += y.z;
+                x.w += y.w;
+            }
+            const float4 bv = *reinterpret_cast<const float4 *>(bias_s + 4 * g);
+            const float xs[4] = {x.x + bv.x, x.y + bv.y, x.z + bv.z, x.w + bv.w};
+            uint32_t key[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int c = 4 * g + u;
+                key[u] = c < p.E ? rank_key(xs[u], c, kmask) : 0u;
+                if (lrow && c < p.E) lrow[c] = xs[u];
+            }
+            push4<KMAX>(tk.key, key[0], key[1], key[2], key[3]);
+        }
+        if (tid == 64) LB_TICK_ANY(53);
+#pragma unroll
+        for (int d = 1; d < TPR; d <<= 1) {
+            uint32_t o[KMAX];
+#pragma unroll
+            for (int j = 0; j < KMAX; ++j) o[j] = __shfl_xor_sync(kFull, tk.key[j], d);
+            merge_top<KMAX>(tk.key, o);
+        }
+        if (tid == 64) LB_TICK_ANY(49);
+        if (pt == 0 && valid) {
+            int32_t *out = p.ids + grow * p.k;
+#pragma unroll
+            for (int j = 0; j < KMAX; ++j)
+                if (j < p.k) out[j] = key_id(tk.key[j], kmask);
+        }
+    }
+    if (tid == 64) LB_TICK_ANY(50);
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync();   // no CTA leaves while a slice copy may still read its shared memory
+    if (tid == 0) {
+        LB_TICK_ANY(51);
+        LB_CTA_TIME(1);
+    }
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc_pair(tmem, p.tmem_cols);
     }
 }
 

@@ -340,6 +340,117 @@ int run_pair(gate::Params &p, const void *h, int nprob, const CUtensorMap &mb, i
     return launch_gate_pair<8, 1>(ma, mb, p, units, nu, grid, smem, s);
 }
 
+// CTA pairs with H split in two: one 256-token unit per cluster of four
+// (two pairs), the second pair's partial accumulators added by the first.
+// One shared-memory limit record per instantiation of the pair split-H
+// gate (its launch and the occupancy query below both raise the limit).
+template <int KMAX, int KS>
+SmemLimit &pairk_lim() {
+    static SmemLimit lim;
+    return lim;
+}
+
+// Clusters of 2 KS CTAs of the pair split-H gate (one CTA per SM) that are
+// resident on the current device at once; 0 if the query fails.  Cached per
+// device.
+template <int KS>
+int pairk_max_clusters() {
+    static int cached[kMaxDevices] = {};   // 0 not asked yet, -1 failed
+    const int dev = current_device();
+    if (dev < 0) return 0;
+    if (cached[dev] != 0) return std::max(cached[dev], 0);
+    auto kern = gate::gate_topk_pairk<8, KS>;
+    const size_t smem = 115 * 1024;   // one CTA per SM whatever the pipeline's size
+    int n = 0;
+    if (allow_smem(kern, pairk_lim<8, KS>(), smem, false)) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(2 * KS * 64, 1, 1);
+        cfg.blockDim = dim3(gate::Shape<4>::THREADS, 1, 1);
+        cfg.dynamicSmemBytes = smem;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = 2 * KS;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess) {
+            cudaGetLastError();
+            n = 0;
+        }
+    }
+    cached[dev] = n > 0 ? n : -1;
+    return std::max(n, 0);
+}
+
+template <int KMAX, int KS>
+int launch_gate_pairk(const CUtensorMap &ma, const CUtensorMap &mb, const gate::Params &p, int units, int nbatch,
+                      size_t smem, cudaStream_t s) {
+    auto kern = gate::gate_topk_pairk<KMAX, KS>;
+    if (!allow_smem(kern, pairk_lim<KMAX, KS>(), smem, false)) return LB_ECUDA;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * KS * units, nbatch, 1);
+    cfg.blockDim = dim3(gate::Shape<4>::THREADS, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2 * KS;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, ma, mb, p);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaLaunchKernelEx(gate_topk pair, split H)");
+    return launched("gate_topk pair, split H");
+}
+
+// CTA pairs with H split over ks pairs (2 or 4): TMEM columns, boxes per
+// stage, stages, and shared memory for the larger of the pipeline and the
+// epilogue's staged partial plus the slices it receives.
+int run_pairk(gate::Params &p, const void *h, const void *w, int nbatch, int ks, cudaStream_t s) {
+    if (p.k > 8 || p.Epad % 16 != 0 || p.Epad < 16 || p.Epad > 256) return LB_EINVAL;
+    if (ks != 2 && ks != 4) return LB_EINVAL;
+    // every pair needs at least one k-block of H
+    if ((ks - 1) * ((p.nkb + ks - 1) / ks) >= p.nkb) return LB_EINVAL;
+    uint32_t pcols = 32;
+    while (pcols < static_cast<uint32_t>(p.Epad)) pcols <<= 1;
+    p.tmem_cols = pcols;
+    p.nbuf = 1;
+    p.split = 1;
+    p.kbox = g_tune_kbox ? g_tune_kbox : 2;
+    const size_t box_bytes = 16384 + static_cast<size_t>(p.Epad / 2) * 128;
+    const size_t sr = static_cast<size_t>((p.Epad + 31) & ~31);
+    const size_t epi_bytes = (gate::BM + static_cast<size_t>(ks - 1) * (gate::BM / ks)) * sr * 4;
+    const size_t room = 200 * 1024;
+    if (2 * box_bytes * p.kbox > room) p.kbox = 1;
+    const size_t stage_bytes = box_bytes * p.kbox;
+    int stages = static_cast<int>(std::min<size_t>(gate::MAX_STAGES, room / stage_bytes));
+    if (g_tune_stages) stages = std::min(stages, g_tune_stages);
+    if (stages < 2) return LB_EINVAL;
+    // one CTA per SM (TMEM); the epilogue reuses the pipeline buffers
+    const size_t smem = std::max({stages * stage_bytes + 1024, epi_bytes + 1024, static_cast<size_t>(115 * 1024)});
+    if (smem > 225 * 1024) return LB_EINVAL;
+    p.stages = stages;
+    CUtensorMap ma, mb;
+    if (!make_map(&ma, h, static_cast<uint64_t>(p.H), static_cast<uint64_t>(p.T), static_cast<uint64_t>(nbatch),
+                  gate::BM) ||
+        !make_map(&mb, w, static_cast<uint64_t>(p.H), static_cast<uint64_t>(p.E), static_cast<uint64_t>(nbatch),
+                  static_cast<uint32_t>(p.Epad / 2))) {
+        std::snprintf(g_last_error, sizeof g_last_error, "cuTensorMapEncodeTiled failed");
+        return LB_ECUDA;
+    }
+    const int units = (p.T + 2 * gate::BM - 1) / (2 * gate::BM);
+    if (ks == 2) {
+        if (p.k <= 2) return launch_gate_pairk<2, 2>(ma, mb, p, units, nbatch, smem, s);
+        if (p.k <= 4) return launch_gate_pairk<4, 2>(ma, mb, p, units, nbatch, smem, s);
+        return launch_gate_pairk<8, 2>(ma, mb, p, units, nbatch, smem, s);
+    }
+    if (p.k <= 2) return launch_gate_pairk<2, 4>(ma, mb, p, units, nbatch, smem, s);
+    if (p.k <= 4) return launch_gate_pairk<4, 4>(ma, mb, p, units, nbatch, smem, s);
+    return launch_gate_pairk<8, 4>(ma, mb, p, units, nbatch, smem, s);
+}
+
 // Persistent gate launch shared by lb_predict_topk and lb_predict_topk_chain:
 // TMEM columns for two accumulators of p.Epad, boxes per stage, stages, and
 // shared memory padded so that at most per_sm CTAs share an SM.  The h map
@@ -551,7 +662,7 @@ const char *lb_last_error(void) { return g_last_error; }
 
 #ifdef LB_TIMING
 int lb_debug_ticks(long long *out, int n) {
-    if (!out || n < 1 || n > 64) return LB_EINVAL;
+    if (!out || n < 1 || n > 64 + 1024) return LB_EINVAL;
     if (cudaDeviceSynchronize() != cudaSuccess) return LB_ECUDA;
     return cudaMemcpyFromSymbol(out, lb::g_ticks, sizeof(long long) * n) == cudaSuccess ? LB_OK : LB_ECUDA;
 }
@@ -575,7 +686,7 @@ int lb_gate_tuning(int stages, int split, int persistent, int kbox, int tiles_pe
         split != -4 && split != -8)
         return LB_EINVAL;
     if (persistent != -1 && persistent != 0 && persistent != 1 && persistent != 2 && persistent != 3 &&
-        persistent != 4)
+        persistent != 4 && persistent != 5 && persistent != 6)
         return LB_EINVAL;
     g_tune_stages = stages;
     g_tune_split = split;
@@ -623,6 +734,24 @@ int lb_predict_topk(const void *h, const void *w, const float *bias, int nbatch,
     // per tile.
     int per_sm = g_tune_persistent;
     if (per_sm == 0 && g_tune_split <= 1 && ntiles >= 2LL * sms && p.Epad <= 128) per_sm = 2;
+    // CTA pairs with H split over two or four pairs, when their clusters
+    // (four or eight CTAs per 256-token unit) fit in one wave.  Measured
+    // (H=7168, E=256): T=2048 24.8 us with four pairs against 53.0 us for a
+    // cluster split of H per tile, T=8192 37.1 against 65.4 us with two; the
+    // same order at H=4096, E=128 and H=2048, E=64 from 2048 to 8192 tokens.
+    // Four pairs below 2048 tokens only at E > 128 (at E <= 128 no faster
+    // there); two pairs in two waves only at E > 128 (T=12288: 68 against
+    // 96 us at E=256; at E <= 128 slower than the split per tile); never
+    // when a pair would get fewer than eight k-blocks.
+    if (per_sm == 0 && g_tune_split == 0 && k <= 8 && p.Epad >= 64 && p.nkb >= 32) {
+        const long long units = static_cast<long long>((T + 2 * gate::BM - 1) / (2 * gate::BM)) * nbatch;
+        const long long c2 = pairk_max_clusters<2>();
+        if (units >= 16 && (units <= c2 || (p.Epad > 128 && units <= 2 * c2)))
+            per_sm = 5;
+        else if (units <= pairk_max_clusters<4>() && (units >= 8 || p.Epad > 128))
+            per_sm = 6;
+    }
+    if (per_sm == 5 || per_sm == 6) return run_pairk(p, h, w, nbatch, per_sm == 5 ? 2 : 4, s);
     if (per_sm == 3) {
         CUtensorMap mb;
         if (p.Epad % 16 != 0 ||
@@ -747,13 +876,15 @@ int lb_predict_topk_chain(const void *h, const void *w, const float *bias, int L
     const long long ntiles = static_cast<long long>(mtiles) * (L + 1);
     uint32_t pcols = 32;
     while (pcols < 4u * static_cast<uint32_t>(E)) pcols <<= 1;
-    int per_sm = g_tune_persistent > 0 ? g_tune_persistent : std::max(1, std::min(2, static_cast<int>(512 / pcols)));
+    // (the per-layer modes 5 and 6, pairs with a split of H, do not apply to the chain)
+    const int tune = g_tune_persistent >= 5 ? 0 : g_tune_persistent;
+    int per_sm = tune > 0 ? tune : std::max(1, std::min(2, static_cast<int>(512 / pcols)));
     // Automatic: CTA pairs when the two gates fill the MMA's N = 256 (E = 128;
     // measured: Qwen3-235B-shaped chain 964 against 1124 us for 16 layers,
     // Qwen3-30B-shaped 293 against 332 us), where one CTA would stream a
     // weight box twice the size of its h box; one CTA per tile below that
     // (OLMoE-shaped, N = 128: 62 against 72 us).
-    if (g_tune_persistent == 0 && 2 * E >= 256 && k <= 8) per_sm = 3;
+    if (tune == 0 && 2 * E >= 256 && k <= 8) per_sm = 3;
     if (per_sm == 3) {
         // CTA pairs: each CTA loads one gate, a box of E rows starting at row
         // (b-1)E (CTA 0) or bE (CTA 1)

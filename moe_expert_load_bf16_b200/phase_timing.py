@@ -1,5 +1,6 @@
 """Phase timing of the latency-bound kernels (plan, split, assign prep and
-scatter) on one problem, from a separate build of the library with
+scatter) and of the per-layer gate as CTA pairs with H split over two pairs
+on one problem, from a separate build of the library with
 -DLB_TIMING: block 0 of each kernel stamps clock64() at its phase boundaries
 into a device array, read back with lb_debug_ticks.  The product library is
 untouched (the timing build goes to liblb_timing.so and is loaded in place of
@@ -31,6 +32,11 @@ PHASES = {
                             (2, 3, "round table"), (3, 6, "passes"), (6, 4, "masses")]),
     "assign prep": (20, ["stage inputs + per-expert segments", "bucket sizes + scan", "block bases"]),
     "assign scatter": (10, ["per-problem tables", "scatter"]),
+    "gate (pairs, H split)": (None, [(40, 41, "prologue"), (41, 44, "loads + MMAs (MMA issuer)"),
+                                     (44, 47, "accumulator complete (epilogue)"),
+                                     (47, 54, "partial TMEM -> shared memory"), (54, 48, "cluster barrier"),
+                                     (48, 52, "other pairs' slices arrive"), (52, 53, "rank own rows"),
+                                     (53, 49, "merge lists"), (49, 50, "write ids"), (50, 51, "closing barrier")]),
 }
 
 
@@ -60,6 +66,21 @@ def main():
         "split": lambda: _lib.lb_split(cnt, plan, N, 12, out=(tok, mass, loads, pr)),
         "assign": lambda: _lib.lb_assign(ids[1:2], cnt, plan, tok, mass, N, workspace=ws),
     }
+    # the per-layer gate as CTA pairs with H split over two pairs, on the
+    # workload's hidden size and experts
+    hid = workloads.hidden_chain(wl, 1, device=dev, T=T)[0]
+    Wg = workloads.gate_weights(wl, 1, device=dev)[0]
+    bg = workloads.biases(wl, 1)[0].to(dev)
+    ids_g = torch.empty(T, k, dtype=torch.int32, device=dev)
+
+    def gate_pairs():
+        _lib.lb_gate_tuning(0, 0, 5)
+        try:
+            _lib.lb_predict_topk(hid, Wg, bg, k, ids=ids_g)
+        finally:
+            _lib.lb_gate_tuning()
+
+    launches["gate"] = gate_pairs
     try:   # clock64 counts SM cycles; microseconds below are at the maximum SM clock
         import pynvml
         pynvml.nvmlInit()
@@ -76,6 +97,8 @@ def main():
             if lib.lb_debug_ticks(ticks, 64) != 0:
                 raise RuntimeError("lb_debug_ticks failed")
             kernels = [name] if name != "assign" else ["assign prep", "assign scatter"]
+            if name == "gate":
+                kernels = ["gate (pairs, H split)"]
             if name == "split":
                 kernels = kernels + ["split detail"]
             if name == "plan":
