@@ -127,8 +127,8 @@ int lb_predict_topk_chain(const void *h, const void *w, const float *bias,
  * buffered where TMEM allows; 3 = CTA pairs: clusters of two CTAs, one per
  * SM, sharing one MMA of M = 256 over 256-token work units, each CTA
  * loading its 128 tokens and half of the MMA's N weight rows, k <= 8;
- * 5 or 6 = lb_predict_topk only: CTA pairs with H split over two or four
- * pairs, one cluster of four or eight CTAs per 256-token unit, the partial
+ * 5, 7 or 6 = lb_predict_topk only: CTA pairs with H split over two, three
+ * or four pairs, one cluster of 4, 6 or 8 CTAs per 256-token unit, the partial
  * accumulators summed by a reduce-scatter over distributed shared memory,
  * k <= 8 and every pair given at least one 64-column block of H;
  * -1 = one CTA per tile); 64-column boxes per
@@ -139,10 +139,10 @@ int lb_predict_topk_chain(const void *h, const void *w, const float *bias,
  * leave SMs to kernels that run beside it on other streams).
  * Automatic: lb_predict_topk_chain with E = 128 (N = 256) and k <= 8 runs
  * CTA pairs; lb_predict_topk with k <= 8, E > 48 and H >= 2048 runs CTA
- * pairs with H split over two pairs when there are at least 16 units of
- * 256 tokens and their clusters fit the device at once (twice over for
- * E > 128), over four pairs when fewer units fit at once with eight CTAs
- * each (from 8 units, or any number for E > 128); otherwise, with at least two token tiles per SM and E <= 128,
+ * pairs with H split over the most pairs whose clusters fit the device
+ * at once: four (from 8 units of 256 tokens, or any number for E > 128),
+ * else three (from 8 units), else two (from 16 units; up to twice what
+ * fits at once for E > 128); otherwise, with at least two token tiles per SM and E <= 128,
  * persistent with two CTAs per SM (one when two double-buffered
  * accumulators of the MMA's N do not fit TMEM twice) and one tile per unit;
  * otherwise one CTA

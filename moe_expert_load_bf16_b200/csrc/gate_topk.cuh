@@ -878,6 +878,14 @@ __device__ __forceinline__ void push4(uint32_t (&a)[KMAX], uint32_t k0, uint32_t
             if ((j & st) == 0) cmp_swap_desc(a[j], a[j + st]);
 }
 
+// First of the rows [row0(q), row0(q+1)) of its 128 that the CTA of pair q
+// ranks: q BM / KS rounded up to a multiple of 8 (slices of 64 for two pairs,
+// 48, 40, 40 for three, 32 for four).
+template <int KS>
+__device__ __forceinline__ int pair_slice_row0(int q) {
+    return ((q * BM) / KS + 7) & ~7;
+}
+
 // CTA pairs with H split over KS pairs (per-tile, one 256-token unit per
 // cluster of 2 KS CTAs; the per-layer gate of wide shapes whose token tiles
 // underfill the GPU, such as the decode shape).  Ranks 2p and 2p+1 form pair
@@ -892,19 +900,21 @@ __device__ __forceinline__ void push4(uint32_t (&a)[KMAX], uint32_t k0, uint32_t
 // floats, float4 group g of row r stored at g ^ (r mod 8), which keeps both
 // the row-per-lane writes and the row-major reads free of bank conflicts).
 // After a cluster barrier (every MMA of the cluster done, so every CTA's
-// pipeline buffers are free), it sends rows [p' R, (p'+1) R) (R = 128 / KS)
-// to the CTA of pair p' holding the same tokens, one bulk shared-to-shared
-// copy per pair, each completing on the receiver's mbarrier.  Each CTA then
-// ranks its own R rows: its partial plus the received ones in pair order
-// (deterministic) plus the bias, 512 / R threads per row over interleaved
-// float4 groups, their lists merged by shuffles.
+// pipeline buffers are free), it sends the rows that pair p' ranks (a
+// slice of about 128 / KS rows, see pair_slice_row0) to the CTA of pair p'
+// holding the same tokens, as bulk shared-to-shared copies of four rows,
+// each issued by its own lane and completing on the receiver's mbarrier.
+// Each CTA then ranks its own rows: its partial plus the received ones in
+// pair order (deterministic) plus the bias, 8 or 16 threads per row over
+// interleaved float4 groups, their lists merged by shuffles.
 template <int KMAX, int KS>
 __global__ void __launch_bounds__(Shape<4>::THREADS, 1)
     gate_topk_pairk(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                     const Params p) {
-    constexpr int R = BM / KS;                  // rows this CTA ranks
-    constexpr int TPR = Shape<4>::EPI / R;      // ranking threads per row
-    static_assert(KS == 2 || KS == 4, "two or four pairs");
+    constexpr int RMAX = ((BM + KS - 1) / KS + 7) & ~7;        // largest row slice
+    constexpr int TPR = Shape<4>::EPI / RMAX >= 16 ? 16 : 8;   // ranking threads per row
+    static_assert(KS >= 2 && KS <= 4, "two to four pairs");
+    static_assert(Shape<4>::EPI / TPR >= RMAX, "a ranking slot for every row of a slice");
     static_assert(TPR <= 32 && 32 % TPR == 0, "a row's ranking threads share a warp");
     extern __shared__ uint8_t smem_raw[];
     pdl_begin();
@@ -935,7 +945,7 @@ __global__ void __launch_bounds__(Shape<4>::THREADS, 1)
     const uint32_t stage_bytes = (a_box + b_box) * kbox;
     const int stages = p.stages;
     const int SR = (p.Epad + 31) & ~31;                         // staged row stride (floats)
-    const uint32_t slice_bytes = static_cast<uint32_t>(R * SR) * 4u;
+    const int R = pair_slice_row0<KS>(pair + 1) - pair_slice_row0<KS>(pair);   // rows this CTA ranks
     if (tid == 0) {
         LB_TICK_ANY(40);
         LB_CTA_TIME(0);
@@ -954,7 +964,7 @@ __global__ void __launch_bounds__(Shape<4>::THREADS, 1)
         aborted = 0;
         fence_mbar_init();
         // the other pairs' slices of this CTA's rows land on recv_bar
-        mbar_arrive_expect_tx(&recv_bar, (KS - 1) * slice_bytes);
+        mbar_arrive_expect_tx(&recv_bar, static_cast<uint32_t>((KS - 1) * R * SR) * 4u);
         tma_prefetch_desc(&tmA);
         tma_prefetch_desc(&tmB);
     }
@@ -1048,7 +1058,7 @@ __global__ void __launch_bounds__(Shape<4>::THREADS, 1)
     const bool epi = warp >= 2;
     const int ew = warp - 2;
     float *stage_f = reinterpret_cast<float *>(smem);   // [128][SR], reusing the pipeline buffers
-    float *recv_f = stage_f + BM * SR;                   // [KS-1][R][SR]
+    float *recv_f = stage_f + BM * SR;                   // [KS-1][RMAX][SR]
     bool ok = true;
     if (epi) {
         ok = mbar_wait(&acc_full, 0) && !*abort_flag;
@@ -1088,16 +1098,16 @@ __global__ void __launch_bounds__(Shape<4>::THREADS, 1)
         // chunks of 4 rows, one lane each (one thread's bulk copies are served
         // one after another)
         if (lane == 0) LB_TICK_ANY(48);
-        constexpr int CH = R / 4;   // chunks per slice
-        for (int j = lane; j < (KS - 1) * CH; j += 32) {
-            const int o = j / CH, ch = j - o * CH;
-            const int pp = o < pair ? o : o + 1;             // receiving pair
+        const int slot = pair;   // this pair's slot at every receiver of a higher pair (pair - 1 below)
+        for (int o = 0; o < KS - 1; ++o) {
+            const int pp = o < pair ? o : o + 1;   // receiving pair
             const uint32_t dst_rank = static_cast<uint32_t>(2 * pp + half);
-            const int slot = pair < pp ? pair : pair - 1;   // this pair's slot at the receiver
-            const int roff = ch * 4 * SR;
-            bulk_copy_to_cta(mapa_shared(smem_u32(recv_f + slot * R * SR + roff), dst_rank),
-                             smem_u32(stage_f + pp * R * SR + roff), slice_bytes / CH,
-                             mapa_shared(smem_u32(&recv_bar), dst_rank));
+            const int r0 = pair_slice_row0<KS>(pp), nch = (pair_slice_row0<KS>(pp + 1) - r0) / 4;
+            const int dslot = pair < pp ? slot : slot - 1;
+            for (int ch = lane; ch < nch; ch += 32)
+                bulk_copy_to_cta(mapa_shared(smem_u32(recv_f + (dslot * RMAX + ch * 4) * SR), dst_rank),
+                                 smem_u32(stage_f + (r0 + ch * 4) * SR), static_cast<uint32_t>(4 * SR) * 4u,
+                                 mapa_shared(smem_u32(&recv_bar), dst_rank));
         }
     }
     if (epi) {
@@ -1106,21 +1116,22 @@ __global__ void __launch_bounds__(Shape<4>::THREADS, 1)
         if (tid == 64) LB_TICK_ANY(52);
         const int lr = ew * (32 / TPR) + lane / TPR;   // row within this CTA's slice
         const int pt = lane % TPR;
-        const int r = pair * R + lr;                   // row within the CTA's 128
+        const bool active = lr < R;                    // (a slot per row; spare slots rank nothing)
+        const int r = pair_slice_row0<KS>(pair) + lr;  // row within the CTA's 128
         const int row = m0 + r;
-        const bool valid = ok && got && row < p.T;
+        const bool valid = ok && got && active && row < p.T;
         const uint32_t kmask = id_mask(p.E);
         const int64_t grow = static_cast<int64_t>(b) * p.T + row;
         float *lrow = (p.logits != nullptr && valid) ? p.logits + grow * p.E : nullptr;
         TopK<KMAX> tk;
         tk.init();
         const float *own = stage_f + r * SR;
-        for (int g = pt; g < (p.Epad >> 2); g += TPR) {
+        for (int g = pt; active && g < (p.Epad >> 2); g += TPR) {
             const int sg = (g ^ (r & 7)) << 2;
             float4 x = *reinterpret_cast<const float4 *>(own + sg);
 #pragma unroll
             for (int o = 0; o < KS - 1; ++o) {
-                const float4 y = *reinterpret_cast<const float4 *>(recv_f + (o * R + lr) * SR + sg);
+                const float4 y = *reinterpret_cast<const float4 *>(recv_f + (o * RMAX + lr) * SR + sg);
                 x.x += y.x;
                 x.y += y.y;
                 x.z += y.z;

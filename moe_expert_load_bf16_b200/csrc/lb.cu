@@ -405,12 +405,12 @@ int launch_gate_pairk(const CUtensorMap &ma, const CUtensorMap &mb, const gate::
     return launched("gate_topk pair, split H");
 }
 
-// CTA pairs with H split over ks pairs (2 or 4): TMEM columns, boxes per
+// CTA pairs with H split over ks pairs (2, 3 or 4): TMEM columns, boxes per
 // stage, stages, and shared memory for the larger of the pipeline and the
 // epilogue's staged partial plus the slices it receives.
 int run_pairk(gate::Params &p, const void *h, const void *w, int nbatch, int ks, cudaStream_t s) {
     if (p.k > 8 || p.Epad % 16 != 0 || p.Epad < 16 || p.Epad > 256) return LB_EINVAL;
-    if (ks != 2 && ks != 4) return LB_EINVAL;
+    if (ks < 2 || ks > 4) return LB_EINVAL;
     // every pair needs at least one k-block of H
     if ((ks - 1) * ((p.nkb + ks - 1) / ks) >= p.nkb) return LB_EINVAL;
     uint32_t pcols = 32;
@@ -421,7 +421,8 @@ int run_pairk(gate::Params &p, const void *h, const void *w, int nbatch, int ks,
     p.kbox = g_tune_kbox ? g_tune_kbox : 2;
     const size_t box_bytes = 16384 + static_cast<size_t>(p.Epad / 2) * 128;
     const size_t sr = static_cast<size_t>((p.Epad + 31) & ~31);
-    const size_t epi_bytes = (gate::BM + static_cast<size_t>(ks - 1) * (gate::BM / ks)) * sr * 4;
+    const size_t rmax = static_cast<size_t>(((gate::BM + ks - 1) / ks + 7) & ~7);   // largest row slice
+    const size_t epi_bytes = (gate::BM + static_cast<size_t>(ks - 1) * rmax) * sr * 4;
     const size_t room = 200 * 1024;
     if (2 * box_bytes * p.kbox > room) p.kbox = 1;
     const size_t stage_bytes = box_bytes * p.kbox;
@@ -445,6 +446,11 @@ int run_pairk(gate::Params &p, const void *h, const void *w, int nbatch, int ks,
         if (p.k <= 2) return launch_gate_pairk<2, 2>(ma, mb, p, units, nbatch, smem, s);
         if (p.k <= 4) return launch_gate_pairk<4, 2>(ma, mb, p, units, nbatch, smem, s);
         return launch_gate_pairk<8, 2>(ma, mb, p, units, nbatch, smem, s);
+    }
+    if (ks == 3) {
+        if (p.k <= 2) return launch_gate_pairk<2, 3>(ma, mb, p, units, nbatch, smem, s);
+        if (p.k <= 4) return launch_gate_pairk<4, 3>(ma, mb, p, units, nbatch, smem, s);
+        return launch_gate_pairk<8, 3>(ma, mb, p, units, nbatch, smem, s);
     }
     if (p.k <= 2) return launch_gate_pairk<2, 4>(ma, mb, p, units, nbatch, smem, s);
     if (p.k <= 4) return launch_gate_pairk<4, 4>(ma, mb, p, units, nbatch, smem, s);
@@ -686,7 +692,7 @@ int lb_gate_tuning(int stages, int split, int persistent, int kbox, int tiles_pe
         split != -4 && split != -8)
         return LB_EINVAL;
     if (persistent != -1 && persistent != 0 && persistent != 1 && persistent != 2 && persistent != 3 &&
-        persistent != 4 && persistent != 5 && persistent != 6)
+        persistent != 4 && persistent != 5 && persistent != 6 && persistent != 7)
         return LB_EINVAL;
     g_tune_stages = stages;
     g_tune_split = split;
@@ -734,11 +740,13 @@ int lb_predict_topk(const void *h, const void *w, const float *bias, int nbatch,
     // per tile.
     int per_sm = g_tune_persistent;
     if (per_sm == 0 && g_tune_split <= 1 && ntiles >= 2LL * sms && p.Epad <= 128) per_sm = 2;
-    // CTA pairs with H split over two or four pairs, when their clusters
-    // (four or eight CTAs per 256-token unit) fit in one wave.  Measured
-    // (H=7168, E=256): T=2048 24.8 us with four pairs against 53.0 us for a
-    // cluster split of H per tile, T=8192 37.1 against 65.4 us with two; the
-    // same order at H=4096, E=128 and H=2048, E=64 from 2048 to 8192 tokens.
+    // CTA pairs with H split over the most pairs (four, three, two) whose
+    // clusters (8, 6 or 4 CTAs per 256-token unit) fit in one wave.
+    // Measured (H=7168, E=256): T=2048 24.8 us with four pairs against
+    // 53.0 us for a cluster split of H per tile, T=4096 30.3 us with three
+    // (34.5 with two, 47.2 with four in two waves), T=8192 36.3 against
+    // 65.4 us with two; the same order at H=4096, E=128 and H=2048, E=64
+    // from 2048 to 8192 tokens.
     // Four pairs below 2048 tokens only at E > 128 (at E <= 128 no faster
     // there); two pairs in two waves only at E > 128 (T=12288: 68 against
     // 96 us at E=256; at E <= 128 slower than the split per tile); never
@@ -746,12 +754,14 @@ int lb_predict_topk(const void *h, const void *w, const float *bias, int nbatch,
     if (per_sm == 0 && g_tune_split == 0 && k <= 8 && p.Epad >= 64 && p.nkb >= 32) {
         const long long units = static_cast<long long>((T + 2 * gate::BM - 1) / (2 * gate::BM)) * nbatch;
         const long long c2 = pairk_max_clusters<2>();
-        if (units >= 16 && (units <= c2 || (p.Epad > 128 && units <= 2 * c2)))
-            per_sm = 5;
-        else if (units <= pairk_max_clusters<4>() && (units >= 8 || p.Epad > 128))
+        if (units <= pairk_max_clusters<4>() && (units >= 8 || p.Epad > 128))
             per_sm = 6;
+        else if (units >= 8 && units <= pairk_max_clusters<3>())
+            per_sm = 7;
+        else if (units >= 16 && (units <= c2 || (p.Epad > 128 && units <= 2 * c2)))
+            per_sm = 5;
     }
-    if (per_sm == 5 || per_sm == 6) return run_pairk(p, h, w, nbatch, per_sm == 5 ? 2 : 4, s);
+    if (per_sm >= 5) return run_pairk(p, h, w, nbatch, per_sm == 5 ? 2 : per_sm == 6 ? 4 : 3, s);
     if (per_sm == 3) {
         CUtensorMap mb;
         if (p.Epad % 16 != 0 ||
@@ -876,7 +886,7 @@ int lb_predict_topk_chain(const void *h, const void *w, const float *bias, int L
     const long long ntiles = static_cast<long long>(mtiles) * (L + 1);
     uint32_t pcols = 32;
     while (pcols < 4u * static_cast<uint32_t>(E)) pcols <<= 1;
-    // (the per-layer modes 5 and 6, pairs with a split of H, do not apply to the chain)
+    // (the per-layer modes 5 to 7, pairs with a split of H, do not apply to the chain)
     const int tune = g_tune_persistent >= 5 ? 0 : g_tune_persistent;
     int per_sm = tune > 0 ? tune : std::max(1, std::min(2, static_cast<int>(512 / pcols)));
     // Automatic: CTA pairs when the two gates fill the MMA's N = 256 (E = 128;

@@ -88,7 +88,7 @@ def test_arguments_rejected_before_any_launch(lib):
     assert lib.lb_decide(None, P(256), P(256), P(256), 1, 16, 2, 4, 16, 2, 0, 12, P(16), P(16), P(16), P(16),
                          P(16), P(16), P(16), P(256), 1, s) == _lib.LB_ENOSPACE
     assert lib.lb_gate_tuning(3, 5, 0, 0, 0, 0) == _lib.LB_EINVAL
-    assert lib.lb_gate_tuning(3, 2, 7, 0, 0, 0) == _lib.LB_EINVAL
+    assert lib.lb_gate_tuning(3, 2, 8, 0, 0, 0) == _lib.LB_EINVAL
     assert lib.lb_gate_tuning(3, 2, 1, 3, 0, 0) == _lib.LB_EINVAL
     assert lib.lb_gate_tuning(0, 0, 0, 0, 3, 0) == _lib.LB_EINVAL
     assert lib.lb_gate_tuning(0, 0, 0, 0, 0, -1) == _lib.LB_EINVAL

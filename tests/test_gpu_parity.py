@@ -11,6 +11,8 @@ from moe_expert_load_bf16_b200.pipeline import DecisionPath, StepPipeline
 pytestmark = pytest.mark.gpu
 
 DEV = "cuda"
+# lb_gate_tuning's persistent values for CTA pairs with H split over 2, 3, 4 pairs
+PAIRS_SPLIT_H = {"pairs_split_h2": 5, "pairs_split_h3": 7, "pairs_split_h4": 6}
 
 
 @pytest.fixture(autouse=True)
@@ -118,14 +120,14 @@ def test_decode_steps(T):
         parity.check_path(path, b, 12)
 
 
-@pytest.mark.parametrize("mode", ["auto", "pairs_split_h2", "pairs_split_h4"])
+@pytest.mark.parametrize("mode", ["auto", "pairs_split_h2", "pairs_split_h3", "pairs_split_h4"])
 @pytest.mark.parametrize("T", [64, 1024, 4096, 8192])
 def test_decode_gate(T, mode):
     """Gate at the decode shape (H=7168, E=256): the automatic choice, and
-    CTA pairs with H split over two or four pairs (partials summed by a
-    reduce-scatter over distributed shared memory)."""
+    CTA pairs with H split over two, three or four pairs (partials summed by
+    a reduce-scatter over distributed shared memory)."""
     if mode != "auto":
-        _lib.lb_gate_tuning(0, 0, 5 if mode == "pairs_split_h2" else 6)
+        _lib.lb_gate_tuning(0, 0, PAIRS_SPLIT_H[mode])
     w = workloads.WORKLOADS["decode"]
     h = workloads.hidden_chain(w, 1, device=DEV, T=T)[0]
     W = workloads.gate_weights(w, 1, device=DEV)[0]
@@ -137,7 +139,8 @@ def test_decode_gate(T, mode):
 
 @pytest.mark.parametrize("T,H,E,k", [(200, 72, 60, 5), (1, 8, 16, 1), (333, 128, 256, 16), (130, 64, 17, 3),
                                      (4096, 256, 128, 8), (96, 2048, 32, 2), (300, 320, 80, 4)])
-@pytest.mark.parametrize("split", [0, 1, 2, 4, -2, -4, -8, "persistent", "pairs_split_h2", "pairs_split_h4"])
+@pytest.mark.parametrize("split", [0, 1, 2, 4, -2, -4, -8, "persistent", "pairs_split_h2", "pairs_split_h3",
+                                   "pairs_split_h4"])
 def test_gate_shapes(T, H, E, k, split):
     """Ragged token tails, E not a multiple of 16, H not a multiple of 64,
     tiny and maximum k, every split of H, every split of N across a cluster
@@ -146,11 +149,11 @@ def test_gate_shapes(T, H, E, k, split):
     Epad = (E + 15) // 16 * 16
     if split == "persistent":
         _lib.lb_gate_tuning(0, 0, 1)
-    elif split in ("pairs_split_h2", "pairs_split_h4"):
-        ks = 2 if split == "pairs_split_h2" else 4
+    elif split in PAIRS_SPLIT_H:
+        ks = int(split[-1])
         if k > 8 or (ks - 1) * ((nkb + ks - 1) // ks) >= nkb:
             pytest.skip("CTA pairs with a split of H take k <= 8 and a k-block of H for every pair")
-        _lib.lb_gate_tuning(0, 0, 5 if ks == 2 else 6)
+        _lib.lb_gate_tuning(0, 0, PAIRS_SPLIT_H[split])
     else:
         if split > nkb or (split > 0 and Epad % (4 * split) != 0):
             pytest.skip("split of H not valid for this shape")
