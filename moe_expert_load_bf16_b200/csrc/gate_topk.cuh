@@ -31,12 +31,15 @@ constexpr int UK = 16;         // UMMA K for bf16
 constexpr int THREADS = 128;   // 4 warps; warp 0 lane 0 = TMA, warp 1 lane 0 = MMA
 constexpr int MAX_STAGES = 8;
 
-// The TMA producers are whole warps.  One thread's tensor copies are served
-// one after another (measured on B200: one issuing thread feeds an SM at
-// about 38 GB/s from L2 however many copies it has in flight, each further
-// thread adds about as much, up to the SM's share of L2 bandwidth), so every
-// copy in flight gets its own lane: box j of stage slot s is issued by lane
-// (s * nbox + j) mod 32.
+// One thread's tensor copies are served one after another (measured on
+// B200: one issuing thread feeds an SM at about 38 GB/s from L2 however many
+// copies it has in flight; each further issuing thread adds about as much,
+// up to the SM's share of L2 bandwidth).  The producer of the pair split-H
+// gate is therefore a whole warp, box j of stage slot s issued by lane
+// (s * nbox + j) mod 32.  (The persistent and per-tile gates keep one
+// issuing lane: their MMAs, not their loads, set the pace, and the same
+// change measured slower there, 1278 against 1084 us on the 16-layer
+// Qwen3-235B-shaped chain.)
 __device__ __forceinline__ bool issues_box(int s, int nbox, int j, int lane) {
     return ((s * nbox + j) & 31) == lane;
 }
@@ -182,27 +185,26 @@ __global__ void __launch_bounds__(THREADS, 1)
     const uint32_t tmem = tmem_slot;
 
     if (warp == 0) {
-        // ---------------- TMA producer (the whole warp, one lane per box)
-        int issued = 0;
-        for (int i = 0; i < nk; ++i) {
-            const int s = i % stages;
-            const uint32_t ph = (i / stages) & 1;
-            const int st = warp_wait_empty(&empty_bar[s], ph ^ 1, &aborted, lane);
-            if (st == 1 && lane == 0) {
-                atomicExch(&aborted, 1);
-                flag(LB_DEV_TIMEOUT);
-            }
-            if (st != 0) break;
-            uint8_t *sa = smem + static_cast<size_t>(s) * stage_bytes;
-            if (lane == 0) mbar_arrive_expect_tx(&full_bar[s], stage_bytes);
-            __syncwarp();
-            if (issues_box(s, 2, 0, lane)) tma_load_3d(&tmA, sa, &full_bar[s], (kb0 + i) * BK, m0, b);
-            if (issues_box(s, 2, 1, lane)) tma_load_3d(&tmB, sa + a_bytes, &full_bar[s], (kb0 + i) * BK, c_off, b);
-            ++issued;
-        }
-        // Never leave with copies in flight into this CTA's shared memory:
-        // wait (bounded) for the latest phase of every stage used.
         if (lane == 0) {
+            // ---------------- TMA producer
+            int issued = 0;
+            for (int i = 0; i < nk; ++i) {
+                const int s = i % stages;
+                const uint32_t ph = (i / stages) & 1;
+                if (!mbar_wait(&empty_bar[s], ph ^ 1)) {
+                    atomicExch(&aborted, 1);
+                    flag(LB_DEV_TIMEOUT);
+                    break;
+                }
+                if (*reinterpret_cast<volatile int *>(&aborted)) break;
+                uint8_t *sa = smem + static_cast<size_t>(s) * stage_bytes;
+                mbar_arrive_expect_tx(&full_bar[s], stage_bytes);
+                tma_load_3d(&tmA, sa, &full_bar[s], (kb0 + i) * BK, m0, b);
+                tma_load_3d(&tmB, sa + a_bytes, &full_bar[s], (kb0 + i) * BK, c_off, b);
+                ++issued;
+            }
+            // Never leave with copies in flight into this CTA's shared memory:
+            // wait (bounded) for the latest phase of every stage used.
             for (int s = 0; s < stages && s < issued; ++s) {
                 const int last = s + ((issued - 1 - s) / stages) * stages;
                 if (!mbar_wait(&full_bar[s], (last / stages) & 1)) flag(LB_DEV_TIMEOUT);
@@ -567,69 +569,62 @@ __global__ void __launch_bounds__(Shape<ES>::THREADS, ES == 2 ? 2 : 1)
     const uint32_t accempty0 = PAIR ? mapa_shared(smem_u32(&acc_empty[0]), 0) : smem_u32(&acc_empty[0]);
 
     if (warp == 0) {
-        // ---------------- TMA producer (the whole warp, one lane per box)
-        const uint64_t pol_a = l2_policy_evict_first(), pol_b = l2_policy_evict_last();
-        const int nbox = (MP + 1) * kbox;
-        int it = 0;
-        bool ok = true;
-        for (int tile = ufirst; tile < ntiles && ok; tile += ustep) {
-            const int b = tile / mtiles;
-            // PAIR: M-tile mt of the unit is rows [mt 2BM, (mt+1) 2BM) of it,
-            // this CTA's half of them starting at m0 + mt 2BM
-            const int m0 = PAIR ? (tile - b * mtiles) * 2 * BM * MP + crank * BM : (tile - b * mtiles) * BM * MP;
-            for (int ks = 0; ks < nks; ++ks, ++it) {
-                const int s = it % stages;
-                const uint32_t ph = (it / stages) & 1;
-                if (warp_wait_empty(&empty_bar[s], ph ^ 1, &aborted, lane) != 0) {
-                    if (lane == 0) {
+        if (lane == 0) {
+            // ---------------- TMA producer
+            const uint64_t pol_a = l2_policy_evict_first(), pol_b = l2_policy_evict_last();
+            int it = 0;
+            bool ok = true;
+            for (int tile = ufirst; tile < ntiles && ok; tile += ustep) {
+                const int b = tile / mtiles;
+                // PAIR: M-tile mt of the unit is rows [mt 2BM, (mt+1) 2BM) of it,
+                // this CTA's half of them starting at m0 + mt 2BM
+                const int m0 = PAIR ? (tile - b * mtiles) * 2 * BM * MP + crank * BM : (tile - b * mtiles) * BM * MP;
+                for (int ks = 0; ks < nks; ++ks, ++it) {
+                    const int s = it % stages;
+                    const uint32_t ph = (it / stages) & 1;
+                    if (!mbar_wait(&empty_bar[s], ph ^ 1) || *abort_flag) {
                         atomicExch(&aborted, 1);
                         flag(LB_DEV_TIMEOUT);
+                        ok = false;
+                        break;
                     }
-                    ok = false;
-                    break;
-                }
-                uint8_t *sa = smem + static_cast<size_t>(s) * stage_bytes;
-                if constexpr (PAIR) {
-                    // rank 0 expects both CTAs' bytes; each CTA loads its
-                    // own h rows and its half of the B rows
-                    if (crank == 0 && lane == 0) mbar_arrive_expect_tx(&full_bar[s], 2 * stage_bytes);
-                    __syncwarp();
-                    const uint32_t fb = full0 + static_cast<uint32_t>(s) * 8u;
+                    uint8_t *sa = smem + static_cast<size_t>(s) * stage_bytes;
+                    if constexpr (PAIR) {
+                        // rank 0 expects both CTAs' bytes; each CTA loads its
+                        // own h rows and its half of the B rows
+                        if (crank == 0) mbar_arrive_expect_tx(&full_bar[s], 2 * stage_bytes);
+                        const uint32_t fb = full0 + static_cast<uint32_t>(s) * 8u;
 #pragma unroll
-                    for (int mt = 0; mt < MP; ++mt)
-                        for (int j = 0; j < kbox; ++j)
-                            if (issues_box(s, nbox, mt * kbox + j, lane))
+                        for (int mt = 0; mt < MP; ++mt)
+                            for (int j = 0; j < kbox; ++j)
                                 tma_load_3d_pair(&tmA, sa + (mt * kbox + j) * a_box, fb, (ks * kbox + j) * BK,
                                                  m0 + mt * 2 * BM, b, pol_a);
-                    const int half = p.Epad / 2;
-                    const int by = (p.chain ? (b - 1) * p.E : 0) + crank * half, bz = p.chain ? 0 : b;
-                    for (int j = 0; j < kbox; ++j)
-                        if (issues_box(s, nbox, MP * kbox + j, lane))
-                            tma_load_3d_pair(&tmB, sa + a_bytes + j * b_box, fb, (ks * kbox + j) * BK, by, bz, pol_b);
-                } else {
-                    if (lane == 0) mbar_arrive_expect_tx(&full_bar[s], stage_bytes);
-                    __syncwarp();
-#pragma unroll
-                    for (int mt = 0; mt < MP; ++mt)
+                        const int half = p.Epad / 2;
+                        const int by = (p.chain ? (b - 1) * p.E : 0) + crank * half, bz = p.chain ? 0 : b;
                         for (int j = 0; j < kbox; ++j)
-                            if (issues_box(s, nbox, mt * kbox + j, lane))
+                            tma_load_3d_pair(&tmB, sa + a_bytes + j * b_box, fb, (ks * kbox + j) * BK, by, bz, pol_b);
+                    } else {
+                        mbar_arrive_expect_tx(&full_bar[s], stage_bytes);
+#pragma unroll
+                        for (int mt = 0; mt < MP; ++mt)
+                            for (int j = 0; j < kbox; ++j)
                                 tma_load_3d_hint(&tmA, sa + (mt * kbox + j) * a_box, &full_bar[s],
                                                  (ks * kbox + j) * BK, m0 + mt * BM, b, pol_a);
-                    const int by = p.chain ? (b - 1) * p.E : 0, bz = p.chain ? 0 : b;
-                    for (int j = 0; j < kbox; ++j)
-                        if (issues_box(s, nbox, MP * kbox + j, lane))
+                        const int by = p.chain ? (b - 1) * p.E : 0, bz = p.chain ? 0 : b;
+                        for (int j = 0; j < kbox; ++j)
                             tma_load_3d_hint(&tmB, sa + a_bytes + j * b_box, &full_bar[s], (ks * kbox + j) * BK, by,
                                              bz, pol_b);
+                    }
                 }
             }
-        }
-        // no copies left in flight into this CTA's shared memory (PAIR:
-        // rank 0's full barriers count both CTAs' copies; rank 1 is held
-        // at the closing cluster barrier until rank 0 has seen them land)
-        if (lane == 0 && (!PAIR || crank == 0)) {
-            for (int s = 0; s < stages && s < it; ++s) {
-                const int last = s + ((it - 1 - s) / stages) * stages;
-                if (!mbar_wait(&full_bar[s], (last / stages) & 1)) flag(LB_DEV_TIMEOUT);
+            // no copies left in flight into this CTA's shared memory (PAIR:
+            // rank 0's full barriers count both CTAs' copies; rank 1 is held
+            // at the closing cluster barrier until rank 0 has seen them land)
+            if (!PAIR || crank == 0) {
+                for (int s = 0; s < stages && s < it; ++s) {
+                    const int last = s + ((it - 1 - s) / stages) * stages;
+                    if (!mbar_wait(&full_bar[s], (last / stages) & 1)) flag(LB_DEV_TIMEOUT);
+                }
             }
         }
     } else if (warp == 1) {
