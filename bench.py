@@ -832,7 +832,8 @@ def run_kernel(args, local):
     """One kernel of the path alone, for timing and for ncu: `--launches`
     plain launches (a profiler picks one with -k/-s/-c), then the mean of 20
     graph replays.  gate: the chain gate over `--problems` layers of the
-    workload (its default: all); count, plan, split, assign: one launch over
+    workload (its default: all); gate1: one layer's gate (lb_predict_topk,
+    its automatic kernel choice) on `--tokens` tokens; count, plan, split, assign: one launch over
     `--problems` independent problems of the workload's shape (T, k, E, G, N)
     with decode-style synthetic ids (`--problems` default 128)."""
     from moe_expert_load_bf16_b200 import _lib, build, workloads
@@ -857,6 +858,18 @@ def run_kernel(args, local):
         nbytes = (nl + 1) * 2 * T * H + nl * (2 * H * E + 4 * E + 8 * T * k)
         flops = nl * 4.0 * T * H * E
         work = f"chain gate, {nl} layers ({nl + 1} hidden states) of {wl.name}"
+    elif args.kernel == "gate1":
+        T1 = args.tokens or T
+        h1 = workloads.hidden_chain(wl, 1, device=dev, T=T1)[0]
+        W1 = workloads.gate_weights(wl, 1, device=dev)[0]
+        b1 = workloads.biases(wl, 1)[0].to(dev)
+        ids1 = torch.empty(T1, k, dtype=torch.int32, device=dev)
+
+        def fn():
+            _lib.lb_predict_topk(h1, W1, b1, k, ids=ids1)
+        nbytes = 2 * T1 * H + 2 * H * E + 4 * E + 4 * T1 * k
+        flops = 2.0 * T1 * H * E
+        work = f"one layer's gate, T={T1} of {wl.name} (H={H}, E={E}, top-{k})"
     else:
         nb = args.problems or 128
         path = DecisionPath(nb, T, 8, E, k, G, N, L, device=dev)
@@ -1011,8 +1024,10 @@ def main():
                     help="chain: one gate pass per hidden state for both gates that read it; two-pass: "
                          "lookahead and normal router as separate passes")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--kernel", choices=("gate", "count", "plan", "split", "assign"), default=None,
+    ap.add_argument("--kernel", choices=("gate", "gate1", "count", "plan", "split", "assign"), default=None,
                     help="time one kernel alone (with --problems, --launches) instead of the step")
+    ap.add_argument("--tokens", type=int, default=0,
+                    help="--kernel gate1: tokens of the one layer (default: the workload's T)")
     ap.add_argument("--problems", type=int, default=0,
                     help="--kernel: layers of the chain gate, or problems per integer-kernel launch")
     ap.add_argument("--launches", type=int, default=3, help="--kernel: plain launches before the timed replays")

@@ -713,6 +713,8 @@ __device__ void scatter_block_tok(const Args &a, int b, int g, int i0, int i1, c
     };
     load_ids(tb0 + warp * 32 + lane);
     for (int cs = tb0; cs < tb1; cs += nw * 32) {
+        const bool first = cs == tb0;
+        if (first) LB_TICK(13);
         for (int e = lane; e < E; e += 32) wrow[e] = 0;
         const int t = cs + warp * 32 + lane;   // this lane's token (block-local)
         const bool tv = t < tb1;
@@ -752,6 +754,7 @@ __device__ void scatter_block_tok(const Args &a, int b, int g, int i0, int i1, c
                 lm[ev[j]] = 0u;
             }
         }
+        if (first) LB_TICK(14);
         __syncthreads();
         for (int e = tid; e < E; e += blockDim.x) {
             int acc = run[e];
@@ -767,6 +770,7 @@ __device__ void scatter_block_tok(const Args &a, int b, int g, int i0, int i1, c
         // are placed now; a replicated expert's remote slots (a minority,
         // but present in nearly every 32-lane slot column) go to the warp's
         // queue and are resolved 32 at a time with every lane busy.
+        if (first) LB_TICK(15);
         int2 *qw = v.queue + warp * TOK_QUEUE;
         int qn = 0;   // queued items (warp-uniform)
         int dv[KT];
@@ -792,6 +796,7 @@ __device__ void scatter_block_tok(const Args &a, int b, int g, int i0, int i1, c
             }
             qn += __popc(rmask);
         }
+        if (first) LB_TICK(16);
         __syncwarp();
         for (int i0q = 0; i0q < qn; i0q += 32) {
             const int iq = i0q + lane;
@@ -824,6 +829,7 @@ __device__ void scatter_block_tok(const Args &a, int b, int g, int i0, int i1, c
                 qw[iq].x = d;
             }
         }
+        if (first) LB_TICK(17);
         __syncwarp();
 #pragma unroll
         for (int j = 0; j < KT; ++j)
@@ -839,7 +845,9 @@ __device__ void scatter_block_tok(const Args &a, int b, int g, int i0, int i1, c
                     if (j < k) dest[t * k + j] = dv[j];
             }
         }
+        if (first) LB_TICK(18);
         __syncthreads();   // pre/run are rewritten by the next chunk
+        if (first) LB_TICK(19);
     }
     if (badl) *bad = 1;
     __syncthreads();

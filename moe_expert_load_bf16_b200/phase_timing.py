@@ -32,6 +32,10 @@ PHASES = {
                             (2, 3, "round table"), (3, 6, "passes"), (6, 4, "masses")]),
     "assign prep": (20, ["stage inputs + per-expert segments", "bucket sizes + scan", "block bases"]),
     "assign scatter": (10, ["per-problem tables", "scatter"]),
+    "assign scatter, first chunk (warp 0)": (None, [(13, 14, "ids, lane masks, in-warp ranks"), (14, 15, "scan down the warps (2 barriers)"),
+                                                    (15, 16, "local and home slots placed, replicated queued"),
+                                                    (16, 17, "replicated queue resolved"), (17, 18, "dest rows written"),
+                                                    (18, 19, "closing barrier")]),
     "gate (pairs, H split)": (None, [(40, 41, "prologue"), (41, 44, "loads + MMAs (MMA issuer)"),
                                      (44, 47, "accumulator complete (epilogue)"),
                                      (47, 54, "partial TMEM -> shared memory"), (54, 48, "cluster barrier"),
@@ -96,7 +100,8 @@ def main():
             fn()
             if lib.lb_debug_ticks(ticks, 64) != 0:
                 raise RuntimeError("lb_debug_ticks failed")
-            kernels = [name] if name != "assign" else ["assign prep", "assign scatter"]
+            kernels = [name] if name != "assign" else ["assign prep", "assign scatter",
+                                                       "assign scatter, first chunk (warp 0)"]
             if name == "gate":
                 kernels = ["gate (pairs, H split)"]
             if name == "split":
