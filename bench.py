@@ -164,6 +164,41 @@ def barrier(world):
         torch.distributed.barrier()
 
 
+def settle(seconds=0.5):
+    """Let the GPU idle before a latency measurement: after the power-capped
+    step loop the SM clock takes a while to climb back, and a kernel of a
+    few microseconds timed at once would be timed at the low clock."""
+    torch.cuda.synchronize()
+    time.sleep(seconds)
+
+
+def graph_us(fn, reps, world=1, rounds=2, inner=10):
+    """Microseconds per call of fn: `inner` calls captured in one CUDA graph
+    (so the host's launch rate never paces calls of a few microseconds),
+    about reps calls per round between CUDA events on the launching stream;
+    the faster of `rounds` rounds (a first round can run at a clock still
+    recovering from the power-capped work before it), max over ranks."""
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for _ in range(inner):
+            fn()
+    g.replay()
+    torch.cuda.synchronize()
+    replays = max(1, (reps + inner - 1) // inner)
+    best = None
+    for _ in range(rounds):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier(world)
+        a.record()
+        for _ in range(replays):
+            g.replay()
+        b.record()
+        torch.cuda.synchronize()
+        t = a.elapsed_time(b) * 1e3 / (replays * inner)
+        best = t if best is None else min(best, t)
+    return max_over_ranks(best, world)
+
+
 def max_over_ranks(x, world):
     """The slowest rank's time (whole-job timing is the max over ranks)."""
     if world == 1:
@@ -307,10 +342,13 @@ def run_ours(args, world, rank, local):
 
     # ---------------- per-layer latencies (single problem, graph replays),
     # this workload's and every other configuration's
+    settle()
     lat = per_layer_latency(wl, hid, W, bias, dev, reps=max(50, args.steps))
     per_config = per_config_latency(dev, world, wl, lat, reps=max(50, args.steps),
                                     decode_steps=args.decode_steps)
+    settle()
     gate_shapes = gate_fractions(dev, world)
+    settle()
 
     # ---------------- count / split / assign as throughput kernels
     ints = integer_kernels_at_throughput(dev, world)
@@ -393,19 +431,7 @@ def gate_fractions(dev, world, reps=20):
     hbm, tflops, _, peak_kind = peaks()
 
     def timed(fn):
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g):
-            fn()
-        g.replay()
-        torch.cuda.synchronize()
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        barrier(world)
-        a.record()
-        for _ in range(reps):
-            g.replay()
-        b.record()
-        torch.cuda.synchronize()
-        return max_over_ranks(a.elapsed_time(b) * 1e3 / reps, world)
+        return graph_us(fn, reps, world)
 
     def frac(nbytes, flops, us):
         return {"us": us, "hbm_frac": nbytes / us / 1e3 / hbm, "tensor_frac": flops / us / 1e6 / tflops,
@@ -429,6 +455,7 @@ def gate_fractions(dev, world, reps=20):
     wl = workloads.WORKLOADS["decode"]
     W = workloads.gate_weights(wl, 1, device=dev)[0]
     bias = workloads.biases(wl, 1)[0].to(dev)
+    settle()
     for T in wl.decode_T:
         h = workloads.hidden_chain(wl, 1, device=dev, T=T)[0]
         ids = torch.empty(T, wl.k, dtype=torch.int32, device=dev)
@@ -454,6 +481,7 @@ def per_config_latency(dev, world, main_wl, main_lat, reps, decode_steps=1000):
             hid = workloads.hidden_chain(wl, 2, device=dev)
             W = workloads.gate_weights(wl, 1, device=dev)
             bias = workloads.biases(wl, 1).to(dev)
+            settle()
             lat = per_layer_latency(wl, hid, W, bias, dev, reps)
             del hid, W, bias
         out[name] = {"shape": f"T={wl.T}, H={wl.H}, E={wl.E}, top-{wl.k}, G={wl.G}, N={wl.N} (L={wl.L})",
@@ -545,18 +573,7 @@ def per_layer_latency(wl, hid, W, bias, dev, reps):
     torch.cuda.synchronize()
 
     def timed(fn):
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g):
-            fn()
-        g.replay()
-        torch.cuda.synchronize()
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record()
-        for _ in range(reps):
-            g.replay()
-        b.record()
-        torch.cuda.synchronize()
-        return a.elapsed_time(b) * 1e3 / reps
+        return graph_us(fn, reps)
 
     res = {
         "solve": timed(p1.solve),
@@ -597,19 +614,7 @@ def swap_planner(wl, path, world, reps=50):
     torch.cuda.synchronize()
 
     def timed(fn):
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g):
-            fn()
-        g.replay()
-        torch.cuda.synchronize()
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        barrier(world)
-        a.record()
-        for _ in range(reps):
-            g.replay()
-        b.record()
-        torch.cuda.synchronize()
-        return max_over_ranks(a.elapsed_time(b) * 1e3 / reps, world)
+        return graph_us(fn, reps, world)
 
     t_all = timed(lambda: _lib.lb_plan_swaps(cp, out=out, **prm))
     t_one = timed(lambda: _lib.lb_plan_swaps(cp[0:1], out=one, **prm))
@@ -653,19 +658,7 @@ def integer_kernels_at_throughput(dev, world, nbatch=128, reps=20):
     torch.cuda.synchronize()
 
     def timed(fn):
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g):
-            fn()
-        g.replay()
-        torch.cuda.synchronize()
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        barrier(world)
-        a.record()
-        for _ in range(reps):
-            g.replay()
-        b.record()
-        torch.cuda.synchronize()
-        return max_over_ranks(a.elapsed_time(b) / reps, world) * 1e3
+        return graph_us(fn, reps, world)
 
     n_edges = sum(int(d["n_edges"]) for d in _lib.decode_plan(path.plan, G, E, N)) / nbatch
     t_count = timed(lambda: _lib.lb_count(path.ids, G, E, cnt=path.cnt))
@@ -761,19 +754,7 @@ def run_decode(args, world, rank, local):
     B = 64
 
     def timed(fn, reps):
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g):
-            fn()
-        g.replay()
-        torch.cuda.synchronize()
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        barrier(world)
-        a.record()
-        for _ in range(reps):
-            g.replay()
-        b.record()
-        torch.cuda.synchronize()
-        return max_over_ranks(a.elapsed_time(b) * 1e3 / reps, world)
+        return graph_us(fn, reps, world)
 
     per_T = {}
     total_assign, total_us = 0, 0.0
@@ -830,8 +811,8 @@ def run_decode(args, world, rank, local):
 # ----------------------------------------------------------------------------- one kernel
 def run_kernel(args, local):
     """One kernel of the path alone, for timing and for ncu: `--launches`
-    plain launches (a profiler picks one with -k/-s/-c), then the mean of 20
-    graph replays.  gate: the chain gate over `--problems` layers of the
+    plain launches (a profiler picks one with -k/-s/-c), then the mean over
+    20 calls replayed from a CUDA graph (graph_us).  gate: the chain gate over `--problems` layers of the
     workload (its default: all); gate1: one layer's gate (lb_predict_topk,
     its automatic kernel choice) on `--tokens` tokens; count, plan, split, assign: one launch over
     `--problems` independent problems of the workload's shape (T, k, E, G, N)
@@ -896,18 +877,7 @@ def run_kernel(args, local):
     for _ in range(args.launches):
         fn()
     torch.cuda.synchronize()
-    g = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g):
-        fn()
-    g.replay()
-    torch.cuda.synchronize()
-    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    a.record()
-    for _ in range(20):
-        g.replay()
-    b.record()
-    torch.cuda.synchronize()
-    us = a.elapsed_time(b) * 1e3 / 20
+    us = graph_us(fn, 20)
     if _lib.lb_get_status():
         raise RuntimeError("device status flagged")
     out = {"kernel": args.kernel, "work": work, "us": us, "algorithmic_bytes": nbytes,
