@@ -42,6 +42,7 @@ struct View {
     int32_t *rep_ptr;   // [E+1]
     int32_t *rep_edge;  // [GN]
     int32_t *eu, *ev, *ee;  // [GN] schedule order
+    int32_t *er;        // [GN]  each edge's round
     int32_t *rptr;      // [GN+1]
     int32_t *tk, *mu, *mv;  // [GN] tok, mass (home side), mass (replica side)
     int4 *tab;          // [(RC+1)*G] (round, rank) slots: {code, tok, own-side mass, 0}; row nr idle
@@ -51,7 +52,7 @@ struct View {
 __host__ __device__ inline size_t smem_bytes(int G, int E, int N) {
     const size_t GN = static_cast<size_t>(G) * N;
     return static_cast<size_t>(E) * 8 + static_cast<size_t>(G) * E * 4 + static_cast<size_t>(E) * 4 +
-           (static_cast<size_t>(E) + 1) * 4 + GN * 4 * 7 + (GN + 1) * 4 +
+           (static_cast<size_t>(E) + 1) * 4 + GN * 4 * 8 + (GN + 1) * 4 +
            (static_cast<size_t>(table_rounds(G, N)) + 1) * G * 16 + 64 * 4 + 64;
 }
 
@@ -66,7 +67,8 @@ __device__ inline View carve(uint8_t *sm, int G, int E, int N) {
     v.eu = v.rep_edge + GN;
     v.ev = v.eu + GN;
     v.ee = v.ev + GN;
-    v.rptr = v.ee + GN;
+    v.er = v.ee + GN;
+    v.rptr = v.er + GN;
     v.tk = v.rptr + GN + 1;
     v.mu = v.tk + GN;
     v.mv = v.mu + GN;
@@ -187,6 +189,19 @@ __device__ int relax_passes_smem(int ne, int nr, int passes, const View &v, int 
     return pr;
 }
 
+// The expert whose slice [rep_ptr[e], rep_ptr[e+1]) of the per-expert edge
+// lists holds position j: the largest e < E with rep_ptr[e] <= j (binary
+// search; every index stays in [0, E] whatever rep_ptr holds).
+__device__ __forceinline__ int list_expert(const int32_t *rep_ptr, int E, int j) {
+    int lo = 0, hi = E - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (rep_ptr[mid] <= j) lo = mid;
+        else hi = mid - 1;
+    }
+    return lo;
+}
+
 // The whole split of one problem by one CTA.  Inputs: the problem's counts
 // (global) and plan blob (global).  Leaves tok in v.tk, mass in v.mu, loads in
 // v.Ls, and returns passes run.  All threads of the CTA must call it.
@@ -213,7 +228,9 @@ __device__ int split_problem(const int32_t *__restrict__ cnt, const uint8_t *__r
         const int32_t *p_ev = reinterpret_cast<const int32_t *>(blob + LY.edge_v);
         const int32_t *p_ee = reinterpret_cast<const int32_t *>(blob + LY.edge_e);
         const int32_t *p_rep_edge = reinterpret_cast<const int32_t *>(blob + LY.rep_edge);
+        const int32_t *p_er = reinterpret_cast<const int32_t *>(blob + LY.edge_round);
         for (int i = tid; i < ne; i += blockDim.x) {
+            v.er[i] = p_er[i];
             v.eu[i] = p_eu[i];
             v.ev[i] = p_ev[i];
             v.ee[i] = p_ee[i];
@@ -236,46 +253,70 @@ __device__ int split_problem(const int32_t *__restrict__ cnt, const uint8_t *__r
     __syncthreads();
     LB_TICK(1);
 
-    // ---- per expert: holders, remote mass, equal partition over its edges
+    // ---- holders, remote mass, starting loads, equal partition.  Edge work
+    // is spread over the CTA by position in the per-expert edge lists (a hot
+    // expert can hold tens of replicas: one thread per expert walking its
+    // list left the whole CTA waiting on that one thread).
+    // (a) per expert: its home as first holder; an edge range that is not a
+    //     valid slice of the list is flagged and treated as empty (R = -1
+    //     marks it until (c)).
+    for (int e = tid; e < E; e += blockDim.x) {
+        const int a = v.rep_ptr[e], z = v.rep_ptr[e + 1];
+        const bool ok = !(a < 0 || z > ne || z < a);
+        if (!ok) *bad = 1;
+        v.hold[e] = 1ull << (e / Eg);
+        v.R[e] = ok ? 0 : -1;
+    }
+    __syncthreads();
+    // (b) per list position: validate the edge and add its replica rank to
+    //     the expert's holders
+    const int npos = max(0, min(v.rep_ptr[E], ne));
+    for (int j = tid; j < npos; j += blockDim.x) {
+        const int e = list_expert(v.rep_ptr, E, j);
+        if (v.R[e] < 0 || j < v.rep_ptr[e] || j >= v.rep_ptr[e + 1]) continue;
+        const int i = v.rep_edge[j];
+        if (i < 0 || i >= ne || v.ee[i] != e || v.eu[i] != e / Eg || v.ev[i] < 0 || v.ev[i] >= G) {
+            *bad = 1;
+            continue;
+        }
+        atomicOr(reinterpret_cast<unsigned long long *>(&v.hold[e]), 1ull << v.ev[i]);
+    }
+    __syncthreads();
+    // (c) per expert: remote mass R (tokens of ranks that hold no copy); the
+    //     home serves its own tokens of e and, at the start, all of R.  The
+    //     replica holders left in the mask are claimed in (d).
     for (int e = tid; e < E; e += blockDim.x) {
         const int h = e / Eg;
-        uint64_t hm = 1ull << h;
-        int a = v.rep_ptr[e], z = v.rep_ptr[e + 1];
-        if (a < 0 || z > ne || z < a) {
-            *bad = 1;
-            a = z = 0;
-        }
-        for (int j = a; j < z; ++j) {
-            const int i = v.rep_edge[j];
-            if (i < 0 || i >= ne || v.ee[i] != e || v.eu[i] != h || v.ev[i] < 0 || v.ev[i] >= G) {
-                *bad = 1;
-                continue;
-            }
-            hm |= 1ull << v.ev[i];
-        }
+        const uint64_t hm = v.hold[e];
         int R = 0;
         for (int g = 0; g < G; ++g)
             if (!((hm >> g) & 1ull)) R += v.cnt[g * E + e];
-        v.hold[e] = hm;
+        atomicAdd(&v.Ls[h], v.cnt[h * E + e] + R);
         v.R[e] = R;
-        // starting loads: every holder serves its own tokens of e, and all the
-        // remote mass R starts at home (integer sums: the order is immaterial)
-        for (uint64_t mk = hm; mk; mk &= mk - 1) {
-            const int g = __ffsll(static_cast<long long>(mk)) - 1;
-            atomicAdd(&v.Ls[g], v.cnt[g * E + e]);
-        }
-        atomicAdd(&v.Ls[h], R);
-        const int m = z - a;
-        if (m > 0) {
-            const int q = R / m, rem = R % m;
-            for (int j = 0; j < m; ++j) {
-                const int i = v.rep_edge[a + j];
-                if (i < 0 || i >= ne) continue;
-                const int t = q + (j < rem ? 1 : 0);
-                v.tk[i] = t;
-                v.mu[i] = t;
-                v.mv[i] = t;
-            }
+        v.hold[e] = hm & ~(1ull << h);
+    }
+    __syncthreads();
+    // (d) per list position: the equal integer partition of R over the
+    //     expert's edges (the first R mod m edges take one more), and the
+    //     starting load of the edge's replica rank: its own tokens of e, added
+    //     by whichever edge clears the rank's bit first (once per holder, as
+    //     the mask counts it; integer sums, so the order is immaterial)
+    for (int j = tid; j < npos; j += blockDim.x) {
+        const int e = list_expert(v.rep_ptr, E, j);
+        const int a = v.rep_ptr[e], z = v.rep_ptr[e + 1];
+        if (j < a || j >= z || a < 0 || z > ne || z < a) continue;
+        const int i = v.rep_edge[j];
+        if (i < 0 || i >= ne) continue;
+        const int m = z - a, R = v.R[e];
+        const int t = R / m + (j - a < R % m ? 1 : 0);
+        v.tk[i] = t;
+        v.mu[i] = t;
+        v.mv[i] = t;
+        const int w = v.ev[i];
+        if (v.ee[i] == e && v.eu[i] == e / Eg && w >= 0 && w < G) {
+            const unsigned long long bit = 1ull << w;
+            if (atomicAnd(reinterpret_cast<unsigned long long *>(&v.hold[e]), ~bit) & bit)
+                atomicAdd(&v.Ls[w], v.cnt[w * E + e]);
         }
     }
     LB_TICK(7);
@@ -286,9 +327,8 @@ __device__ int split_problem(const int32_t *__restrict__ cnt, const uint8_t *__r
     // both its ends (the plan blob gives each edge's round)
     LB_TICK(5);
     if (use_table) {
-        const int32_t *p_er = reinterpret_cast<const int32_t *>(blob + LY.edge_round);
         for (int i = tid; i < ne; i += blockDim.x) {
-            const int r = p_er[i];
+            const int r = v.er[i];
             const int u = v.eu[i], w = v.ev[i];
             if (r < 0 || r >= nr || i < v.rptr[r] || i >= v.rptr[r + 1]) {
                 *bad = 1;
@@ -300,6 +340,7 @@ __device__ int split_problem(const int32_t *__restrict__ cnt, const uint8_t *__r
             v.tab[r * G + w] = make_int4(slot_code(u, false, i), t, 0, 0);
         }
     }
+    LB_TICK(8);
     __syncthreads();
     LB_TICK(3);
 

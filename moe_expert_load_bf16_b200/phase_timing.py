@@ -29,7 +29,8 @@ PHASES = {
     "split": (0, ["stage inputs", "per-expert setup and start loads", "round table", "passes + masses"]),
     "plan detail": (None, [(35, 38, "round colouring"), (38, 36, "order by round")]),
     "split detail": (None, [(1, 7, "per-expert setup (thread 0)"), (7, 2, "wait for the other experts"),
-                            (2, 3, "round table"), (3, 6, "passes"), (6, 4, "masses")]),
+                            (2, 8, "round table (thread 0's edges)"), (8, 3, "round table (wait for the others)"),
+                            (3, 6, "passes"), (6, 4, "masses")]),
     "assign prep": (20, ["stage inputs + per-expert segments", "bucket sizes + scan", "block bases"]),
     "assign scatter": (10, ["per-problem tables", "scatter"]),
     "assign scatter, first chunk (warp 0)": (None, [(13, 14, "ids, lane masks, in-warp ranks"), (14, 15, "scan down the warps (2 barriers)"),
