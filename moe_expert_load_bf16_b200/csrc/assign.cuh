@@ -45,7 +45,7 @@ __host__ __device__ inline size_t ws_words(int G, int E, int N) {
 __host__ __device__ inline size_t prep_smem_bytes(int G, int E, int N) {
     const size_t GN = static_cast<size_t>(G) * N;
     return static_cast<size_t>(E) * 8 + static_cast<size_t>(G) * E * 4 * 2 + static_cast<size_t>(E) * 4 * 3 +
-           (static_cast<size_t>(E) + 1) * 4 + GN * 4 * 7 + 64;
+           (static_cast<size_t>(E) + 1) * 4 + GN * 4 * 7 + static_cast<size_t>(E) * 4 * 10 + 64;
 }
 
 // Shared memory of the scatter: per-expert tables (holders, replica count,
@@ -90,6 +90,9 @@ __device__ void prep_problem(const Args &a, int b, uint8_t *sm) {
     int32_t *sq = ms + GN;           // segment start in q
     int32_t *sc = sq + GN;           // mass of earlier segments
     int32_t *osz = sc + GN;          // [NK] bucket sizes, then their exclusive scan
+    int32_t *csum = osz + NK;        // [E][8] remote counts per chunk of 8 blocks
+    int32_t *qh = csum + E * 8;      // [E] remote assignments before the home block
+    int32_t *bh = qh + E;            // [E] the home block's share of the edges' segments
     __shared__ int wsum[32];
     __shared__ int bad;
 
@@ -223,44 +226,62 @@ __device__ void prep_problem(const Args &a, int b, uint8_t *sm) {
     __syncthreads();
     LB_TICK(22);
 
-    // ---- base per (block g, expert e): thread per expert, g ascending with
-    // the running remote prefix q0 and a cursor into the expert's replica
-    // edges (ordered by ascending replica rank)
-    for (int e = tid; e < E; e += blockDim.x) {
-        const int h = e / Eg;
+    // ---- base per (block g, expert e).  q0(g, e) = remote assignments of e
+    // in the blocks before g (blocks that hold no copy of e).  In four
+    // parallel steps (one thread per expert walking all blocks, with a hot
+    // expert's tens of edges at its home block, held the CTA on that thread):
+    // (1) remote counts per chunk of 8 blocks; (2) q0 of every block from the
+    // chunk prefixes, parked in base (global, read back by the same CTA after
+    // a barrier); (3) per edge, the home block's share of its segment and the
+    // replica holder's base; (4) every other (g, e).
+    const int nch = (G + 7) >> 3;
+    for (int x = tid; x < E * nch; x += blockDim.x) {
+        const int e = x % E, c = x / E;
         const uint64_t hm = hold[e];
-        const int r0 = rep_ptr[e], m = rcnt[e];
-        int j = r0;
+        int sum = 0;
+        for (int g = c * 8; g < min(G, c * 8 + 8); ++g)
+            if (!((hm >> g) & 1ull)) sum += cnt_s[g * E + e];
+        csum[e * 8 + c] = sum;
+    }
+    for (int e = tid; e < E; e += blockDim.x) bh[e] = 0;
+    __syncthreads();
+    for (int x = tid; x < E * nch; x += blockDim.x) {
+        const int e = x % E, c = x / E;
+        const uint64_t hm = hold[e];
+        const int h = e / Eg;
         int q0 = 0;
-        for (int g = 0; g < G; ++g) {
-            int out;
-            if ((hm >> g) & 1ull) {
-                int before = 0;
-                if (g == h) {
-                    if (m == 0) {
-                        before = q0;
-                    } else {
-                        for (int jj = r0; jj < r0 + m; ++jj) {
-                            const int i = rep_edge[jj];
-                            if (i >= 0 && i < ne) before += clampi(q0 - sq[i], 0, ms[i]);
-                        }
-                    }
-                } else {
-                    while (j < r0 + m && !(rep_edge[j] >= 0 && rep_edge[j] < ne && ev[rep_edge[j]] >= g)) ++j;
-                    if (j < r0 + m) {
-                        const int i = rep_edge[j];
-                        if (ev[i] == g) before = clampi(q0 - sq[i] - ms[i], 0, tk[i] - ms[i]);
-                    }
-                }
-                out = osz[g * E + e] + before;
-            } else if (m == 0) {
-                out = osz[h * E + e] + (h < g ? cnt_s[h * E + e] : 0) + q0;
-            } else {
-                out = q0;
-            }
-            base[g * E + e] = out;
+        for (int c2 = 0; c2 < c; ++c2) q0 += csum[e * 8 + c2];
+        for (int g = c * 8; g < min(G, c * 8 + 8); ++g) {
+            base[g * E + e] = q0;
+            if (g == h) qh[e] = q0;
             if (!((hm >> g) & 1ull)) q0 += cnt_s[g * E + e];
         }
+    }
+    __syncthreads();
+    for (int i = tid; i < ne; i += blockDim.x) {
+        // (in a plan every edge of e sits once in e's list; a list that does
+        // not match its edges was flagged above)
+        const int e = ee[i], v = ev[i];
+        if (e < 0 || e >= E || v < 0 || v >= G || rcnt[e] == 0) continue;
+        atomicAdd(&bh[e], clampi(qh[e] - sq[i], 0, ms[i]));
+        if (v != e / Eg && ((hold[e] >> v) & 1ull)) {
+            const int q0 = base[v * E + e];
+            base[v * E + e] = osz[v * E + e] + clampi(q0 - sq[i] - ms[i], 0, tk[i] - ms[i]);
+        }
+    }
+    __syncthreads();
+    for (int x = tid; x < NK; x += blockDim.x) {
+        const int g = x / E, e = x - g * E;
+        const int h = e / Eg;
+        const uint64_t hm = hold[e];
+        const bool held = (hm >> g) & 1ull;
+        if (held && g != h) continue;   // replica holders: set in (3)
+        const int m = rcnt[e], q0 = base[x];
+        int out;
+        if (held) out = osz[x] + (m == 0 ? q0 : bh[e]);
+        else if (m == 0) out = osz[h * E + e] + (h < g ? cnt_s[h * E + e] : 0) + q0;
+        else out = q0;
+        base[x] = out;
     }
     for (int i = tid; i < ne; i += blockDim.x) {
         const int e = ee[i], v = ev[i];

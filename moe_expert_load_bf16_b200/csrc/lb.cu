@@ -613,7 +613,14 @@ int scatter_grid_x(int T, int k, int G, int nw = assign::SC_WARPS) {
 // Warps per scatter CTA: 32 while the problems' CTAs leave SMs free (one
 // problem's latency), 16 once they fill the GPU twice over (throughput: two
 // CTAs per SM); fewer if the per-warp tables would not fit shared memory.
+// Small source blocks (one warp each) go in CTAs of 8 warps while those fit
+// one wave, so that one problem's blocks spread over more SMs (decode shape,
+// G=64, one problem: lb_assign 80.0 against 93.6 us at T=8192 and 69.6
+// against 77.5 us at T=4096 with 32 warps per CTA; 4, 2 or 1 were slower).
 int scatter_warps(int nbatch, int T, int k, int G, int E, int N) {
+    if (static_cast<long long>(T / G) * k <= assign::WARP_BLOCK_MAX &&
+        static_cast<long long>(scatter_grid_x(T, k, G, 8)) * nbatch <= device_sms())
+        return 8;
     const long long ctas = static_cast<long long>(scatter_grid_x(T, k, G, 16)) * nbatch;
     int nw = ctas >= 2LL * device_sms() ? 16 : assign::SC_WARPS;
     nw = std::min(nw, g_max_threads / 32);
