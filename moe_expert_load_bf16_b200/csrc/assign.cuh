@@ -779,9 +779,10 @@ __device__ void scatter_block_tok(const Args &a, int b, int g, int i0, int i1, c
         __syncthreads();
         for (int e = tid; e < E; e += blockDim.x) {
             int acc = run[e];
+            const int bse = v.base[e];
             for (int w = 0; w < nw; ++w) {
                 const int c = v.wcnt[w * EP + e];
-                v.wcnt[w * EP + e] = acc;   // in place: each row becomes its warp's prefix
+                v.wcnt[w * EP + e] = bse + acc;   // in place: each row becomes its warp's first slot of e
                 acc += c;
             }
             run[e] = acc;
@@ -807,7 +808,7 @@ __device__ void scatter_block_tok(const Args &a, int b, int g, int i0, int i1, c
                 qw[slot] = make_int2(t * k + j, e | ((loc[j] & 0xff) << 16));
                 loc[j] = slot | (1 << 30);   // this slot's answer comes back through the queue
             } else if (e >= 0) {
-                const int pp = v.base[e] + prow[e] + (loc[j] & 0xff);
+                const int pp = prow[e] + (loc[j] & 0xff);
                 if (static_cast<unsigned>(pp) < static_cast<unsigned>(nf)) {
                     perm[pp] = fbase + t * k + j;
                     dv[j] = c >> 2;
@@ -824,7 +825,7 @@ __device__ void scatter_block_tok(const Args &a, int b, int g, int i0, int i1, c
             if (iq < qn) {
                 const int2 it = qw[iq];
                 const int fl = it.x, e = it.y & 0xffff;
-                const int q = v.base[e] + prow[e] + (it.y >> 16);
+                const int q = prow[e] + (it.y >> 16);
                 // the segment covering q: forward from the block's first one
                 const int last = v.rep0[e] + v.rcnt[e] - 1;
                 int jj = v.sfirst[e];
