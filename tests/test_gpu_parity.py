@@ -137,6 +137,27 @@ def test_decode_gate(T, mode):
     parity.gate_check(h, W, bias, w.k, ids, logits, rows=rows)
 
 
+@pytest.mark.parametrize("mode", ["auto", "pairs_split_h2", "pairs_split_h3", "pairs_split_h4"])
+@pytest.mark.parametrize("T", [200, 1024, 4100])
+def test_gate_pairs_batched(T, mode):
+    """CTA pairs with a split of H on a batch of three independent problems
+    (the grid's second dimension; the automatic choice counts the units of
+    the whole batch), E=256, H=2048, a ragged last unit at T=200 and 4100,
+    every row against the oracle with logits."""
+    if mode != "auto":
+        _lib.lb_gate_tuning(0, 0, PAIRS_SPLIT_H[mode])
+    B, H, E, k = 3, 2048, 256, 8
+    g = torch.Generator(device=DEV).manual_seed(T + 17 * len(mode))
+    h = torch.randn(B, T, H, generator=g, device=DEV).to(torch.bfloat16)
+    W = (torch.randn(B, E, H, generator=g, device=DEV) / H ** 0.5).to(torch.bfloat16)
+    bias = 0.1 * torch.randn(B, E, generator=g, device=DEV)
+    ids, logits = _lib.lb_predict_topk(h, W, bias, k, want_logits=True)
+    assert _lib.lb_get_status() == 0
+    rows = np.arange(T) if T <= 1024 else np.random.default_rng(3).choice(T, 256, replace=False)
+    for b in range(B):
+        parity.gate_check(h[b], W[b], bias[b], k, ids[b], logits[b], rows=rows)
+
+
 @pytest.mark.parametrize("T,H,E,k", [(200, 72, 60, 5), (1, 8, 16, 1), (333, 128, 256, 16), (130, 64, 17, 3),
                                      (4096, 256, 128, 8), (96, 2048, 32, 2), (300, 320, 80, 4)])
 @pytest.mark.parametrize("split", [0, 1, 2, 4, -2, -4, -8, "persistent", "pairs_split_h2", "pairs_split_h3",
