@@ -68,6 +68,7 @@ struct Args {
     int T, k, G, E, N;
     int32_t *dest, *perm, *offs, *ws;
     size_t ws_stride;   // words per problem
+    int slices = 1;     // scatter CTAs per large source block (token-aligned slices)
 };
 
 __device__ __forceinline__ int clampi(int x, int lo, int hi) { return min(max(x, lo), hi); }
@@ -929,7 +930,44 @@ __global__ void __launch_bounds__(SC_THREADS) scatter_kernel(const Args a) {
         scatter_blocks_warp_any(a, blockIdx.y, g0, min(a.G, g0 + nw), v, &bad);
         __syncthreads();
     } else {
-        scatter_block_cta_any(a, blockIdx.y, blockIdx.x, 0, nitems, nullptr, v, &bad);
+        // CTA x scatters slice x mod S of source block x / S (S = a.slices
+        // token-aligned slices, so that one problem's few blocks spread over
+        // more SMs).  A slice's ranks continue the block's earlier slices:
+        // the CTA first counts each expert's valid ids there (the scatter's
+        // own ranking counts the same ones).
+        const int S = a.slices;
+        const int g = static_cast<int>(blockIdx.x) / S, sl = static_cast<int>(blockIdx.x) - g * S;
+        const int Tg = a.T / a.G, tps = (Tg + S - 1) / S;
+        const int t0 = min(Tg, sl * tps);
+        const int i0 = t0 * a.k, i1 = sl == S - 1 ? nitems : min(Tg, t0 + tps) * a.k;
+        const int32_t *prefix = nullptr;
+        if (S > 1) {
+            int32_t *pref = v.base + 2 * (a.E + 1);   // (rows 0 and 1 serve the block; nw >= 8 here)
+            for (int e = threadIdx.x; e < a.E; e += blockDim.x) pref[e] = 0;
+            __syncthreads();
+            const int32_t *ids = a.ids + static_cast<int64_t>(blockIdx.y) * a.T * a.k + static_cast<int64_t>(g) * nitems;
+            const unsigned E = static_cast<unsigned>(a.E);
+            int n4 = 0;
+            if ((reinterpret_cast<uintptr_t>(ids) & 15) == 0) {
+                n4 = i0 >> 2;
+                const int4 *ids4 = reinterpret_cast<const int4 *>(ids);
+#pragma unroll 4
+                for (int x = threadIdx.x; x < n4; x += blockDim.x) {
+                    const int4 q = __ldg(ids4 + x);
+                    if (static_cast<unsigned>(q.x) < E) atomicAdd(&pref[q.x], 1);
+                    if (static_cast<unsigned>(q.y) < E) atomicAdd(&pref[q.y], 1);
+                    if (static_cast<unsigned>(q.z) < E) atomicAdd(&pref[q.z], 1);
+                    if (static_cast<unsigned>(q.w) < E) atomicAdd(&pref[q.w], 1);
+                }
+            }
+            for (int x = 4 * n4 + threadIdx.x; x < i0; x += blockDim.x) {
+                const int e = __ldg(ids + x);
+                if (static_cast<unsigned>(e) < E) atomicAdd(&pref[e], 1);
+            }
+            __syncthreads();
+            prefix = pref;
+        }
+        scatter_block_cta_any(a, blockIdx.y, g, i0, i1, prefix, v, &bad);
     }
     LB_TICK(12);
     if (threadIdx.x == 0 && bad) flag(LB_DEV_BAD_SPLIT);

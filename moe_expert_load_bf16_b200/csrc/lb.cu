@@ -605,9 +605,33 @@ int launch_count_v(bool vec, const int32_t *ids, int nbatch, int T, int k, int E
 
 // Scatter CTAs per problem: one per source block, or one per SC_WARPS small
 // blocks (one block per warp).
-int scatter_grid_x(int T, int k, int G, int nw = assign::SC_WARPS) {
+int scatter_grid_x(int T, int k, int G, int nw = assign::SC_WARPS, int slices = 1) {
     const long long nitems = static_cast<long long>(T / G) * k;
-    return nitems <= assign::WARP_BLOCK_MAX ? (G + nw - 1) / nw : G;
+    return nitems <= assign::WARP_BLOCK_MAX ? (G + nw - 1) / nw : G * slices;
+}
+
+// Scatter CTAs per large source block: when one CTA per block leaves most
+// SMs idle (one problem's latency: G = 8 blocks of 4096 tokens take 8 SMs),
+// token-aligned slices of at least 256 tokens, as many as keep the CTAs
+// within one wave; each slice's CTA first counts its block's earlier slices.
+// (Qwen3-235B-shaped problem, one launch of lb_assign, T = 32768, G = 8.)
+int scatter_slices(int nbatch, int T, int k, int G) {
+    if (T <= 0 || static_cast<long long>(T / G) * k <= assign::WARP_BLOCK_MAX) return 1;
+    const long long ctas = static_cast<long long>(G) * nbatch;
+    const long long sms = device_sms();
+    int S = 1;
+    while (ctas * S * 2 <= sms && (T / G) / (S * 2) >= 256) S *= 2;
+    return S;
+}
+
+// Warps per scatter CTA for sliced blocks: one chunk of 32 tokens per warp
+// covers the slice (at least 8 warps: the prefix counts use a row of the
+// per-warp table).
+int slice_warps(int T, int G, int S) {
+    const int tps = (T / G + S - 1) / S;
+    int nw = 8;
+    while (nw < assign::SC_WARPS && nw * 32 < tps) nw <<= 1;
+    return nw;
 }
 
 // Warps per scatter CTA: 32 while the problems' CTAs leave SMs free (one
@@ -1091,7 +1115,10 @@ int lb_assign(const int32_t *ids, const int32_t *cnt, const void *plan, const in
     a.offs = offs;
     a.ws = static_cast<int32_t *>(workspace);
     a.ws_stride = assign::ws_words(G, E, N);
-    const int nw = T > 0 ? scatter_warps(nbatch, T, k, G, E, N) : assign::SC_WARPS;
+    a.slices = scatter_slices(nbatch, T, k, G);
+    const int nw = T == 0 ? assign::SC_WARPS
+                          : a.slices > 1 ? std::min(slice_warps(T, G, a.slices), g_max_threads / 32)
+                                         : scatter_warps(nbatch, T, k, G, E, N);
     const size_t sm1 = assign::prep_smem_bytes(G, E, N), sm2 = assign::scatter_smem_bytes(G, E, N, nw);
     if (!allow_smem(assign::prep_kernel, g_lim_prep, sm1, false) ||
         !allow_smem(assign::scatter_kernel, g_lim_scatter, sm2, false))
@@ -1100,7 +1127,7 @@ int lb_assign(const int32_t *ids, const int32_t *cnt, const void *plan, const in
                       sm1, s, a) != LB_OK)
         return LB_ECUDA;
     if (T == 0) return LB_OK;
-    return launch_kernel("assign scatter", assign::scatter_kernel, dim3(scatter_grid_x(T, k, G, nw), nbatch),
+    return launch_kernel("assign scatter", assign::scatter_kernel, dim3(scatter_grid_x(T, k, G, nw, a.slices), nbatch),
                          dim3(nw * 32), assign::scatter_smem_bytes(G, E, N, nw), s, a);
 }
 
@@ -1139,7 +1166,10 @@ int lb_decide(const int32_t *cnt_pred, const int32_t *cnt, const int32_t *ids, v
     a.offs = offs;
     a.ws = static_cast<int32_t *>(workspace);
     a.ws_stride = assign::ws_words(G, E, N);
-    const int nw = T > 0 ? scatter_warps(nbatch, T, k, G, E, N) : assign::SC_WARPS;
+    a.slices = scatter_slices(nbatch, T, k, G);
+    const int nw = T == 0 ? assign::SC_WARPS
+                          : a.slices > 1 ? std::min(slice_warps(T, G, a.slices), g_max_threads / 32)
+                                         : scatter_warps(nbatch, T, k, G, E, N);
     const size_t sm2 = assign::scatter_smem_bytes(G, E, N, nw);
     static SmemLimit lim0, lim1;
     if (!allow_smem(assign::scatter_kernel, g_lim_scatter, sm2, false)) return LB_ECUDA;
@@ -1176,7 +1206,7 @@ int lb_decide(const int32_t *cnt_pred, const int32_t *cnt, const int32_t *ids, v
                                dim3(std::min(assign::PREP_THREADS, g_max_threads)), smt, s, a);
     }
     if (rc != LB_OK || T == 0) return rc;
-    return launch_kernel("assign scatter", assign::scatter_kernel, dim3(scatter_grid_x(T, k, G, nw), nbatch),
+    return launch_kernel("assign scatter", assign::scatter_kernel, dim3(scatter_grid_x(T, k, G, nw, a.slices), nbatch),
                          dim3(nw * 32), sm2, s, a);
 }
 
@@ -1341,7 +1371,10 @@ extern "C" int lb_assign_noalloc(const int32_t *ids, const int32_t *cnt, const v
     a.offs = offs;
     a.ws = scratch;
     a.ws_stride = assign::ws_words(G, E, N);
-    const int nw = T > 0 ? scatter_warps(nbatch, T, k, G, E, N) : assign::SC_WARPS;
+    a.slices = scatter_slices(nbatch, T, k, G);
+    const int nw = T == 0 ? assign::SC_WARPS
+                          : a.slices > 1 ? std::min(slice_warps(T, G, a.slices), g_max_threads / 32)
+                                         : scatter_warps(nbatch, T, k, G, E, N);
     if (!allow_smem(assign::prep_kernel, g_lim_prep, assign::prep_smem_bytes(G, E, N), false) ||
         !allow_smem(assign::scatter_kernel, g_lim_scatter, assign::scatter_smem_bytes(G, E, N, nw), false))
         return LB_ECUDA;
@@ -1350,6 +1383,6 @@ extern "C" int lb_assign_noalloc(const int32_t *ids, const int32_t *cnt, const v
                       assign::prep_smem_bytes(G, E, N), s, a) != LB_OK)
         return LB_ECUDA;
     if (T == 0) return LB_OK;
-    return launch_kernel("assign scatter (noalloc)", assign::scatter_kernel, dim3(scatter_grid_x(T, k, G, nw), nbatch),
+    return launch_kernel("assign scatter (noalloc)", assign::scatter_kernel, dim3(scatter_grid_x(T, k, G, nw, a.slices), nbatch),
                          dim3(nw * 32), assign::scatter_smem_bytes(G, E, N, nw), s, a);
 }

@@ -13,8 +13,8 @@ both gates that read one hidden state in a single pass over it:
   tok, mass, loads = split(cnt, plan)                       lb_split
   dest, perm, offs = assign(ids, cnt, plan, split)          lb_assign
 (`solve` runs count, split and assign as lb_count + lb_decide: split and the
-assign's tables in one launch per problem, the scatter in a second; or, for
-problems of more than FUSED_ABOVE assignments, as one lb_solve launch.)
+assign's tables in one launch per problem, the scatter in a second;
+`solve_fused` as one lb_solve launch, which gives the same outputs.)
 """
 import torch
 
@@ -57,18 +57,13 @@ class DecisionPath:
     # assign by lb_decide (split and the assign's tables in one launch per
     # problem, the scatter in a second); solve_separate makes the same bytes
     # with lb_split and lb_assign
-    # Problems of more than this many assignments take the fused lb_solve
-    # (one cluster of up to 16 CTAs per problem spreads the scatter; measured
-    # per layer: Qwen3-235B-shaped 57.4 against 71.7 us); smaller ones
-    # lb_count + lb_decide (OLMoE-shaped 34.8 against 38.5 us, Qwen3-30B-shaped
-    # 51.2 against 55.3 us).  The outputs are identical either way.
-    FUSED_ABOVE = 131072
-
+    # lb_count + lb_decide: since the scatter spreads one problem's large
+    # source blocks over slices, this is the faster form on every measured
+    # shape (per layer, one problem: Qwen3-235B-shaped 38.6 against 51.6 us
+    # for the fused lb_solve, Qwen3-30B-shaped 36.1 against 43.7 us).  The
+    # outputs are identical either way.
     def solve(self, ids=None, counted=False):
         ids = self.ids if ids is None else ids
-        if self.T * self.k > self.FUSED_ABOVE:
-            self.solve_fused(ids)
-            return
         if not counted:
             _lib.lb_count(ids, self.G, self.E, cnt=self.cnt)
         self.decide(ids)
