@@ -590,10 +590,38 @@ int run_splitn(gate::Params &p, const void *h, const void *w, int nbatch, int mt
     return launch_gate_k<false, true>(p.k, ma, mb, p, mtiles, nbatch, smem, s);
 }
 
+// CTAs per source rank for the count: a cluster of up to 8 (rows of at
+// least 256 tokens each) while the problem's ranks alone underfill the GPU
+// (one Qwen3-235B-shaped problem: G = 8 ranks of 4096 tokens).
+int count_split(int nbatch, int T, int G) {
+    const long long ctas = static_cast<long long>(G) * nbatch;
+    const long long sms = device_sms();
+    int S = 1;
+    while (S < 8 && ctas * S * 2 <= sms && (T / G) / (S * 2) >= 256) S *= 2;
+    return S;
+}
+
 template <int K, bool VEC>
 int launch_count(const int32_t *ids, int nbatch, int T, int k, int E, int G, int32_t *cnt, cudaStream_t s) {
-    return launch_kernel("count", count::count_kernel<K, VEC>, dim3(G, nbatch), dim3(count::THREADS),
-                         E * sizeof(int), s, ids, T, k, E, G, cnt);
+    const int S = count_split(nbatch, T, G);
+    if (S == 1)
+        return launch_kernel("count", count::count_kernel<K, VEC>, dim3(G, nbatch), dim3(count::THREADS),
+                             E * sizeof(int), s, ids, T, k, E, G, cnt);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(G * S, nbatch, 1);
+    cfg.blockDim = dim3(count::THREADS, 1, 1);
+    cfg.dynamicSmemBytes = E * sizeof(int);
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = S;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, count::count_kernel_cluster<K, VEC>, ids, T, k, E, G, S, cnt);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaLaunchKernelEx(count, cluster)");
+    return launched("count (cluster)");
 }
 
 template <int K>
