@@ -45,7 +45,7 @@ __host__ __device__ inline size_t ws_words(int G, int E, int N) {
 __host__ __device__ inline size_t prep_smem_bytes(int G, int E, int N) {
     const size_t GN = static_cast<size_t>(G) * N;
     return static_cast<size_t>(E) * 8 + static_cast<size_t>(G) * E * 4 * 2 + static_cast<size_t>(E) * 4 * 3 +
-           (static_cast<size_t>(E) + 1) * 4 + GN * 4 * 7 + static_cast<size_t>(E) * 4 * 10 + 64;
+           (static_cast<size_t>(E) + 1) * 4 + GN * 4 * 7 + static_cast<size_t>(E) * 4 * 11 + 64;
 }
 
 // Shared memory of the scatter: per-expert tables (holders, replica count,
@@ -94,6 +94,7 @@ __device__ void prep_problem(const Args &a, int b, uint8_t *sm) {
     int32_t *csum = osz + NK;        // [E][8] remote counts per chunk of 8 blocks
     int32_t *qh = csum + E * 8;      // [E] remote assignments before the home block
     int32_t *bh = qh + E;            // [E] the home block's share of the edges' segments
+    int32_t *hc = bh + E;            // [E] cnt[home(e), e] (the counts' table then holds q0)
     __shared__ int wsum[32];
     __shared__ int bad;
 
@@ -232,9 +233,10 @@ __device__ void prep_problem(const Args &a, int b, uint8_t *sm) {
     // parallel steps (one thread per expert walking all blocks, with a hot
     // expert's tens of edges at its home block, held the CTA on that thread):
     // (1) remote counts per chunk of 8 blocks; (2) q0 of every block from the
-    // chunk prefixes, parked in base (global, read back by the same CTA after
-    // a barrier); (3) per edge, the home block's share of its segment and the
-    // replica holder's base; (4) every other (g, e).
+    // chunk prefixes, written over the counts' table in shared memory (each
+    // count is read before its slot is overwritten; only the home counts are
+    // needed later, kept in hc); (3) per edge, the home block's share of its
+    // segment and the replica holder's base; (4) every other (g, e).
     const int nch = (G + 7) >> 3;
     for (int x = tid; x < E * nch; x += blockDim.x) {
         const int e = x % E, c = x / E;
@@ -244,7 +246,10 @@ __device__ void prep_problem(const Args &a, int b, uint8_t *sm) {
             if (!((hm >> g) & 1ull)) sum += cnt_s[g * E + e];
         csum[e * 8 + c] = sum;
     }
-    for (int e = tid; e < E; e += blockDim.x) bh[e] = 0;
+    for (int e = tid; e < E; e += blockDim.x) {
+        bh[e] = 0;
+        hc[e] = cnt_s[(e / Eg) * E + e];
+    }
     __syncthreads();
     for (int x = tid; x < E * nch; x += blockDim.x) {
         const int e = x % E, c = x / E;
@@ -253,9 +258,10 @@ __device__ void prep_problem(const Args &a, int b, uint8_t *sm) {
         int q0 = 0;
         for (int c2 = 0; c2 < c; ++c2) q0 += csum[e * 8 + c2];
         for (int g = c * 8; g < min(G, c * 8 + 8); ++g) {
-            base[g * E + e] = q0;
+            const int cg = cnt_s[g * E + e];
+            cnt_s[g * E + e] = q0;
             if (g == h) qh[e] = q0;
-            if (!((hm >> g) & 1ull)) q0 += cnt_s[g * E + e];
+            if (!((hm >> g) & 1ull)) q0 += cg;
         }
     }
     __syncthreads();
@@ -266,7 +272,7 @@ __device__ void prep_problem(const Args &a, int b, uint8_t *sm) {
         if (e < 0 || e >= E || v < 0 || v >= G || rcnt[e] == 0) continue;
         atomicAdd(&bh[e], clampi(qh[e] - sq[i], 0, ms[i]));
         if (v != e / Eg && ((hold[e] >> v) & 1ull)) {
-            const int q0 = base[v * E + e];
+            const int q0 = cnt_s[v * E + e];
             base[v * E + e] = osz[v * E + e] + clampi(q0 - sq[i] - ms[i], 0, tk[i] - ms[i]);
         }
     }
@@ -277,10 +283,10 @@ __device__ void prep_problem(const Args &a, int b, uint8_t *sm) {
         const uint64_t hm = hold[e];
         const bool held = (hm >> g) & 1ull;
         if (held && g != h) continue;   // replica holders: set in (3)
-        const int m = rcnt[e], q0 = base[x];
+        const int m = rcnt[e], q0 = cnt_s[x];
         int out;
         if (held) out = osz[x] + (m == 0 ? q0 : bh[e]);
-        else if (m == 0) out = osz[h * E + e] + (h < g ? cnt_s[h * E + e] : 0) + q0;
+        else if (m == 0) out = osz[h * E + e] + (h < g ? hc[e] : 0) + q0;
         else out = q0;
         base[x] = out;
     }
