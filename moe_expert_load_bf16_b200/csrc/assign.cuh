@@ -69,13 +69,42 @@ struct Args {
     int32_t *dest, *perm, *offs, *ws;
     size_t ws_stride;   // words per problem
     int slices = 1;     // scatter CTAs per large source block (token-aligned slices)
+    int cta_blocks = 0; // 1: small blocks (<= WARP_BLOCK_MAX assignments) one per CTA as well
 };
 
 __device__ __forceinline__ int clampi(int x, int lo, int hi) { return min(max(x, lo), hi); }
 
+// Exclusive scan of one 64-bit value per thread over the CTA (every thread
+// calls it; wtot is 32 words of shared memory); `total` gets the CTA's sum.
+__device__ __forceinline__ uint64_t cta_exclusive_scan_u64(uint64_t x, uint64_t *wtot, uint64_t &total) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    uint64_t s = x;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const uint64_t y = __shfl_up_sync(kFull, s, off);
+        if (lane >= off) s += y;
+    }
+    if (lane == 31) wtot[warp] = s;
+    __syncthreads();
+    if (warp == 0) {
+        uint64_t w = lane < nw ? wtot[lane] : 0;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const uint64_t y = __shfl_up_sync(kFull, w, off);
+            if (lane >= off) w += y;
+        }
+        if (lane < nw) wtot[lane] = w;   // inclusive per warp
+    }
+    __syncthreads();
+    const uint64_t before = warp > 0 ? wtot[warp - 1] : 0;
+    total = wtot[nw - 1];
+    __syncthreads();   // wtot is reused by the next call
+    return before + s - x;
+}
+
 // Tables of problem b for its scatter: offs, base[g,e], replica segments.
 // All threads of the CTA call it; `sm` holds prep_smem_bytes(G,E,N) bytes.
-__device__ void prep_problem(const Args &a, int b, uint8_t *sm) {
+__device__ void prep_problem(const Args &a, int b, uint8_t *sm, int C = 1, int c = 0) {
     const int G = a.G, E = a.E, N = a.N, GN = G * N, NK = G * E;
     uint64_t *hold = reinterpret_cast<uint64_t *>(sm);
     int32_t *cnt_s = reinterpret_cast<int32_t *>(hold + E);
@@ -96,6 +125,7 @@ __device__ void prep_problem(const Args &a, int b, uint8_t *sm) {
     int32_t *bh = qh + E;            // [E] the home block's share of the edges' segments
     int32_t *hc = bh + E;            // [E] cnt[home(e), e] (the counts' table then holds q0)
     __shared__ int wsum[32];
+    __shared__ uint64_t wscan[32];
     __shared__ int bad;
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -109,6 +139,14 @@ __device__ void prep_problem(const Args &a, int b, uint8_t *sm) {
     int32_t *seg_cum = seg_qoff + GN;
     int32_t *seg_rep = seg_cum + GN;
     const int Eg = E / G;
+    // a cluster of C CTAs shares one problem (C divides G): CTA c owns the
+    // (rank, expert) keys of ranks [rlo, rhi); the per-expert work is done by
+    // every CTA, the per-key work by the owner, the scan's carries and the
+    // few home-rank offsets a CTA needs from another cross over distributed
+    // shared memory
+    const int rlo = c * (G / C), rhi = rlo + G / C;
+    const int K0 = rlo * E, K1 = rhi * E;
+    __shared__ int cta_total;
     int ne = hdr[0];
     if (tid == 0) bad = 0;
     if (ne < 0 || ne > GN) ne = 0;
@@ -132,9 +170,63 @@ __device__ void prep_problem(const Args &a, int b, uint8_t *sm) {
         }
         for (int e = tid; e <= E; e += blockDim.x) rep_ptr[e] = p_rep_ptr[e];
     }
+    // per-expert scratch of the segment scan below (the arrays' own contents
+    // are written later): the scan's value at e's first CSR position and
+    // past its last, for tok (high word) and mass (low word)
+    int32_t *hT = qh, *hM = bh, *eT = hc, *eM = csum;
+    for (int e = tid; e < E; e += blockDim.x) {
+        hold[e] = 0ull;
+        hT[e] = hM[e] = eT[e] = eM[e] = 0;
+    }
     __syncthreads();
 
-    // ---- per expert: holders, remote mass, replica segments
+    // ---- per CSR position j (in parallel: a hot expert's tens of edges
+    // would otherwise be one thread's serial walk): its edge and expert
+    // (checked against the expert's CSR range), the holder bit, and an
+    // exclusive scan of (tok, mass) over the positions.  A segment's start
+    // in q (and its mass before) is the scan at its position less the scan
+    // at its expert's first position.
+    {
+        uint64_t carry = 0;
+        for (int j0 = 0; j0 < ne; j0 += blockDim.x) {   // ne is the same in every thread
+            const int j = j0 + tid;
+            int i = -1, e = -1;
+            uint64_t val = 0;
+            if (j < ne) {
+                i = rep_edge[j];
+                if (i >= 0 && i < ne) {
+                    e = ee[i];
+                    const int v = ev[i];
+                    if (e < 0 || e >= E || v < 0 || v >= G || j < rep_ptr[e] || j >= rep_ptr[e + 1]) {
+                        e = -1;
+                    } else {
+                        atomicOr(reinterpret_cast<unsigned long long *>(&hold[e]), 1ull << v);
+                        val = (static_cast<uint64_t>(static_cast<uint32_t>(tk[i])) << 32) |
+                              static_cast<uint32_t>(ms[i]);
+                    }
+                }
+                if (e < 0) bad = 1;
+            }
+            uint64_t tot;
+            const uint64_t x = carry + cta_exclusive_scan_u64(val, wscan, tot);
+            carry += tot;
+            if (e >= 0) {
+                sq[i] = static_cast<int>(x >> 32);   // made relative to the expert's first position below
+                sc[i] = static_cast<int>(static_cast<uint32_t>(x));
+                if (j == rep_ptr[e]) {
+                    hT[e] = static_cast<int>(x >> 32);
+                    hM[e] = static_cast<int>(static_cast<uint32_t>(x));
+                }
+                if (j == rep_ptr[e + 1] - 1) {
+                    eT[e] = static_cast<int>((x + val) >> 32);
+                    eM[e] = static_cast<int>(static_cast<uint32_t>(x + val));
+                }
+            }
+        }
+    }
+    __syncthreads();
+
+    // ---- per expert: holders, remote mass; per edge: segment starts
     for (int e = tid; e < E; e += blockDim.x) {
         const int h = e / Eg;
         int r0 = rep_ptr[e], r1 = rep_ptr[e + 1];
@@ -142,20 +234,8 @@ __device__ void prep_problem(const Args &a, int b, uint8_t *sm) {
             bad = 1;
             r0 = r1 = 0;
         }
-        uint64_t hm = 1ull << h;
-        int qo = 0, cm = 0;
-        for (int j = r0; j < r1; ++j) {
-            const int i = rep_edge[j];
-            if (i < 0 || i >= ne || ee[i] != e || ev[i] < 0 || ev[i] >= G) {
-                bad = 1;
-                continue;
-            }
-            hm |= 1ull << ev[i];
-            sq[i] = qo;
-            sc[i] = cm;
-            qo += tk[i];
-            cm += ms[i];
-        }
+        const uint64_t hm = hold[e] | (1ull << h);
+        const int qo = r1 > r0 ? eT[e] - hT[e] : 0, cm = r1 > r0 ? eM[e] - hM[e] : 0;
         int R = 0;
         for (int g = 0; g < G; ++g)
             if (!((hm >> g) & 1ull)) R += cnt_s[g * E + e];
@@ -165,12 +245,19 @@ __device__ void prep_problem(const Args &a, int b, uint8_t *sm) {
         rtot[e] = R;
         homeadd[e] = (r1 > r0) ? cm : R;
     }
+    for (int i = tid; i < ne; i += blockDim.x) {
+        const int e = ee[i];
+        if (e >= 0 && e < E) {
+            sq[i] -= hT[e];
+            sc[i] -= hM[e];
+        }
+    }
     __syncthreads();
     LB_TICK(21);
 
     // ---- bucket sizes over keys r*E+e: own tokens of held experts, the home
     // share of each expert, and every edge's replica share (tok - mass)
-    for (int r = warp; r < G; r += (blockDim.x >> 5)) {
+    for (int r = rlo + warp; r < rhi; r += (blockDim.x >> 5)) {
         for (int e = lane; e < E; e += 32) {
             const uint64_t hm = hold[e];
             int sz = ((hm >> r) & 1ull) ? cnt_s[r * E + e] : 0;
@@ -179,18 +266,20 @@ __device__ void prep_problem(const Args &a, int b, uint8_t *sm) {
         }
     }
     __syncthreads();
+    LB_TICK(24);
     for (int i = tid; i < ne; i += blockDim.x) {
         const int e = ee[i], v = ev[i];
-        if (e >= 0 && e < E && v >= 0 && v < G) osz[v * E + e] += tk[i] - ms[i];   // one edge per (v, e)
+        if (e >= 0 && e < E && v >= rlo && v < rhi) osz[v * E + e] += tk[i] - ms[i];   // one edge per (v, e)
     }
     __syncthreads();
+    LB_TICK(25);
     // block-wide exclusive scan, in place: warp w scans its contiguous
     // segment of keys 32 at a time (conflict-free, coalesced), then the warp
     // totals are scanned and added back; offs (global) gets a copy
     {
         const int nw = blockDim.x >> 5;
-        const int seg = ((NK + nw - 1) / nw + 31) & ~31;
-        const int s0 = min(NK, warp * seg), s1 = min(NK, s0 + seg);
+        const int seg = ((K1 - K0 + nw - 1) / nw + 31) & ~31;
+        const int s0 = min(K1, K0 + warp * seg), s1 = min(K1, s0 + seg);
         int carry = 0;
         for (int kb = s0; kb < s1; kb += 32) {
             const int key = kb + lane;
@@ -207,18 +296,27 @@ __device__ void prep_problem(const Args &a, int b, uint8_t *sm) {
         if (lane == 0) wsum[warp] = carry;
         __syncthreads();
         if (warp == 0) {
-            const int c = lane < nw ? wsum[lane] : 0;
-            int x = c;
+            const int wc = lane < nw ? wsum[lane] : 0;
+            int x = wc;
 #pragma unroll
             for (int off = 1; off < 32; off <<= 1) {
                 const int y = __shfl_up_sync(kFull, x, off);
                 if (lane >= off) x += y;
             }
-            if (lane < nw) wsum[lane] = x - c;   // exclusive per warp
-            if (lane == nw - 1) offs[NK] = x;
+            if (lane < nw) wsum[lane] = x - wc;   // exclusive per warp
+            if (lane == nw - 1) cta_total = x;
         }
         __syncthreads();
-        const int add = wsum[warp];
+        LB_TICK(26);
+        // the keys of lower-ranked CTAs come first
+        int pre = 0;
+        if (C > 1) {
+            cluster_sync();
+            for (int q = 0; q < c; ++q) pre += ld_cluster_i32(mapa_shared(smem_u32(&cta_total), static_cast<uint32_t>(q)));
+        }
+        LB_TICK(27);
+        if (c == C - 1 && tid == 0) offs[NK] = pre + cta_total;
+        const int add = wsum[warp] + pre;
         for (int key = s0 + lane; key < s1; key += 32) {
             const int o = osz[key] + add;
             osz[key] = o;
@@ -239,25 +337,26 @@ __device__ void prep_problem(const Args &a, int b, uint8_t *sm) {
     // segment and the replica holder's base; (4) every other (g, e).
     const int nch = (G + 7) >> 3;
     for (int x = tid; x < E * nch; x += blockDim.x) {
-        const int e = x % E, c = x / E;
+        const int e = x % E, ch = x / E;
         const uint64_t hm = hold[e];
         int sum = 0;
-        for (int g = c * 8; g < min(G, c * 8 + 8); ++g)
+        for (int g = ch * 8; g < min(G, ch * 8 + 8); ++g)
             if (!((hm >> g) & 1ull)) sum += cnt_s[g * E + e];
-        csum[e * 8 + c] = sum;
+        csum[e * 8 + ch] = sum;
     }
     for (int e = tid; e < E; e += blockDim.x) {
         bh[e] = 0;
         hc[e] = cnt_s[(e / Eg) * E + e];
     }
     __syncthreads();
+    LB_TICK(28);
     for (int x = tid; x < E * nch; x += blockDim.x) {
-        const int e = x % E, c = x / E;
+        const int e = x % E, ch = x / E;
         const uint64_t hm = hold[e];
         const int h = e / Eg;
         int q0 = 0;
-        for (int c2 = 0; c2 < c; ++c2) q0 += csum[e * 8 + c2];
-        for (int g = c * 8; g < min(G, c * 8 + 8); ++g) {
+        for (int c2 = 0; c2 < ch; ++c2) q0 += csum[e * 8 + c2];
+        for (int g = ch * 8; g < min(G, ch * 8 + 8); ++g) {
             const int cg = cnt_s[g * E + e];
             cnt_s[g * E + e] = q0;
             if (g == h) qh[e] = q0;
@@ -265,19 +364,23 @@ __device__ void prep_problem(const Args &a, int b, uint8_t *sm) {
         }
     }
     __syncthreads();
+    LB_TICK(29);
     for (int i = tid; i < ne; i += blockDim.x) {
         // (in a plan every edge of e sits once in e's list; a list that does
         // not match its edges was flagged above)
         const int e = ee[i], v = ev[i];
         if (e < 0 || e >= E || v < 0 || v >= G || rcnt[e] == 0) continue;
         atomicAdd(&bh[e], clampi(qh[e] - sq[i], 0, ms[i]));
-        if (v != e / Eg && ((hold[e] >> v) & 1ull)) {
+        if (v != e / Eg && v >= rlo && v < rhi && ((hold[e] >> v) & 1ull)) {
             const int q0 = cnt_s[v * E + e];
             base[v * E + e] = osz[v * E + e] + clampi(q0 - sq[i] - ms[i], 0, tk[i] - ms[i]);
         }
     }
     __syncthreads();
-    for (int x = tid; x < NK; x += blockDim.x) {
+    LB_TICK(55);
+    if (C > 1) cluster_sync();   // every CTA's offsets final before the home-rank reads below
+    LB_TICK(56);
+    for (int x = K0 + tid; x < K1; x += blockDim.x) {
         const int g = x / E, e = x - g * E;
         const int h = e / Eg;
         const uint64_t hm = hold[e];
@@ -285,27 +388,51 @@ __device__ void prep_problem(const Args &a, int b, uint8_t *sm) {
         if (held && g != h) continue;   // replica holders: set in (3)
         const int m = rcnt[e], q0 = cnt_s[x];
         int out;
-        if (held) out = osz[x] + (m == 0 ? q0 : bh[e]);
-        else if (m == 0) out = osz[h * E + e] + (h < g ? hc[e] : 0) + q0;
-        else out = q0;
+        if (held) {
+            out = osz[x] + (m == 0 ? q0 : bh[e]);
+        } else if (m == 0) {
+            // the home rank's offset, from its owner (all scans are done:
+            // the cluster barrier above)
+            const int oh = (h >= rlo && h < rhi)
+                               ? osz[h * E + e]
+                               : ld_cluster_i32(mapa_shared(smem_u32(&osz[h * E + e]),
+                                                            static_cast<uint32_t>(h / (G / C))));
+            out = oh + (h < g ? hc[e] : 0) + q0;
+        } else {
+            out = q0;
+        }
         base[x] = out;
     }
+    LB_TICK(57);
     for (int i = tid; i < ne; i += blockDim.x) {
         const int e = ee[i], v = ev[i];
-        seg_qoff[i] = sq[i];
-        seg_cum[i] = sc[i];
-        seg_rep[i] = (e >= 0 && e < E && v >= 0 && v < G) ? osz[v * E + e] : 0;
+        const bool ok = e >= 0 && e < E && v >= 0 && v < G;
+        if (c == 0) {
+            seg_qoff[i] = sq[i];
+            seg_cum[i] = sc[i];
+            if (!ok) seg_rep[i] = 0;
+        }
+        if (ok && v >= rlo && v < rhi) seg_rep[i] = osz[v * E + e];   // by the rank's owner
     }
     __syncthreads();
     LB_TICK(23);
     if (tid == 0 && bad) flag(LB_DEV_BAD_SPLIT);
     __syncthreads();
+    if (C > 1) cluster_sync();   // no CTA leaves while another reads its offsets
 }
 
 __global__ void __launch_bounds__(PREP_THREADS) prep_kernel(const Args a) {
     extern __shared__ __align__(16) uint8_t sm[];
     pdl_begin();
     prep_problem(a, blockIdx.x, sm);
+}
+
+// One problem per cluster of gridDim.x CTAs (each owning G / gridDim.x ranks
+// of the key table), for a single problem's latency when G x E is large.
+__global__ void __launch_bounds__(PREP_THREADS) prep_kernel_cluster(const Args a) {
+    extern __shared__ __align__(16) uint8_t sm[];
+    pdl_begin();
+    prep_problem(a, blockIdx.y, sm, static_cast<int>(gridDim.x), static_cast<int>(cluster_ctarank()));
 }
 
 // ---- scatter ---------------------------------------------------------------
@@ -392,6 +519,7 @@ __device__ void scatter_setup(const Args &a, int b, const ScatterView &v) {
     int ne = hdr[0];
     if (ne < 0 || ne > GN) ne = 0;
     for (int e = tid; e <= E; e += blockDim.x) v.rep0[e] = p_rep_ptr[e];
+    for (int e = tid; e < E; e += blockDim.x) v.hold[e] = 1ull << (e / Eg);   // home; replica holders ORed below
     // per CSR position j (parallel): segment data
     for (int j = tid; j < ne; j += blockDim.x) {
         const int i = p_rep_edge[j];
@@ -419,15 +547,13 @@ __device__ void scatter_setup(const Args &a, int b, const ScatterView &v) {
             if (v.rep0[mid] <= j) lo = mid; else hi = mid - 1;
         }
         v.s_vcnt[j] = cnt[v.s_v[j] * E + lo];
+        if (v.s_tok[j] > 0 || v.s_qoff[j] != 0x7fffffff)
+            atomicOr(reinterpret_cast<unsigned long long *>(&v.hold[lo]), 1ull << v.s_v[j]);
     }
     for (int e = tid; e < E; e += blockDim.x) {
         const int h = e / Eg;
         int r0 = v.rep0[e], r1 = v.rep0[e + 1];
         if (r0 < 0 || r1 > ne || r1 < r0) r0 = r1 = 0;
-        uint64_t hm = 1ull << h;
-        for (int j = r0; j < r1; ++j)
-            if (v.s_tok[j] > 0 || v.s_qoff[j] != 0x7fffffff) hm |= 1ull << v.s_v[j];
-        v.hold[e] = hm;
         v.rcnt[e] = r1 - r0;
         v.homecnt[e] = cnt[h * E + e];
         v.homeoff[e] = offs[h * E + e];
@@ -710,8 +836,10 @@ __device__ void scatter_block_tok(const Args &a, int b, int g, int i0, int i1, c
         }
         v.sfirst[e] = sf;
     }
+    LB_TICK(58);
     for (int x = tid; x < nw * EP; x += blockDim.x) v.lmask[x] = 0u;
     __syncthreads();
+    LB_TICK(59);
     int32_t *wrow = v.wcnt + warp * EP;
     const int32_t *prow = v.wcnt + warp * EP;   // after the scan: the warp's prefixes
     uint32_t *lm = v.lmask + warp * EP;
@@ -918,8 +1046,9 @@ __device__ inline void scatter_block_cta_any(const Args &a, int b, int g, int i0
 // Scatter kernel: CTA (x, problem y) of W = blockDim.x / 32 warps (32 for
 // one problem's latency; 16 when many problems fill the GPU, so that two CTAs
 // share an SM and one's barriers overlap the other's work).  Small blocks:
-// CTA x takes blocks [x*W, (x+1)*W), one per warp.  Large blocks: CTA x
-// takes block x.
+// CTA x takes blocks [x*W, (x+1)*W), one per warp, unless a.cta_blocks asks
+// for one block per CTA (few problems: the blocks then spread over more SMs).
+// Large blocks: CTA x takes block x (or a slice of it).
 __global__ void __launch_bounds__(SC_THREADS) scatter_kernel(const Args a) {
     extern __shared__ __align__(16) uint8_t sm[];
     pdl_begin();
@@ -931,7 +1060,7 @@ __global__ void __launch_bounds__(SC_THREADS) scatter_kernel(const Args a) {
     scatter_setup(a, blockIdx.y, v);
     LB_TICK(11);
     const int nitems = (a.T / a.G) * a.k;
-    if (nitems <= WARP_BLOCK_MAX) {
+    if (nitems <= WARP_BLOCK_MAX && !a.cta_blocks) {
         const int g0 = blockIdx.x * nw;
         scatter_blocks_warp_any(a, blockIdx.y, g0, min(a.G, g0 + nw), v, &bad);
         __syncthreads();

@@ -633,9 +633,9 @@ int launch_count_v(bool vec, const int32_t *ids, int nbatch, int T, int k, int E
 
 // Scatter CTAs per problem: one per source block, or one per SC_WARPS small
 // blocks (one block per warp).
-int scatter_grid_x(int T, int k, int G, int nw = assign::SC_WARPS, int slices = 1) {
+int scatter_grid_x(int T, int k, int G, int nw = assign::SC_WARPS, int slices = 1, bool cta_blocks = false) {
     const long long nitems = static_cast<long long>(T / G) * k;
-    return nitems <= assign::WARP_BLOCK_MAX ? (G + nw - 1) / nw : G * slices;
+    return nitems <= assign::WARP_BLOCK_MAX && !cta_blocks ? (G + nw - 1) / nw : G * slices;
 }
 
 // Scatter CTAs per large source block: when one CTA per block leaves most
@@ -650,6 +650,39 @@ int scatter_slices(int nbatch, int T, int k, int G) {
     int S = 1;
     while (ctas * S * 2 <= sms && (T / G) / (S * 2) >= 256) S *= 2;
     return S;
+}
+
+// The assign's prep for one problem's latency on a cluster of 8 CTAs (each
+// owning G/8 ranks of the (rank, expert) key table) when the table is large:
+// at the decode shape (64 x 256 keys) one CTA is instruction-bound for about
+// 34 us.  Otherwise one CTA per problem.
+SmemLimit g_lim_prep_cluster;
+int launch_prep(const assign::Args &a, int nbatch, size_t smem, cudaStream_t s, const char *what) {
+    const int nt = std::min(assign::PREP_THREADS, g_max_threads);
+    const bool cl = static_cast<long long>(a.G) * a.E >= 8192 && a.G % 8 == 0 &&
+                    static_cast<long long>(nbatch) * 8 <= device_sms();
+    if (!cl) {
+        if (!allow_smem(assign::prep_kernel, g_lim_prep, smem, false)) return LB_ECUDA;
+        return launch_kernel(what, assign::prep_kernel, dim3(nbatch), dim3(nt), smem, s, a);
+    }
+    if (!allow_smem(assign::prep_kernel_cluster, g_lim_prep_cluster, smem, false)) return LB_ECUDA;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(8, nbatch, 1);
+    cfg.blockDim = dim3(nt, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 8;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = g_pdl ? 1 : 0;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, assign::prep_kernel_cluster, a);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaLaunchKernelEx(assign prep, cluster)");
+    return launched(what);
 }
 
 // Warps per scatter CTA for sliced blocks: one chunk of 32 tokens per warp
@@ -678,6 +711,30 @@ int scatter_warps(int nbatch, int T, int k, int G, int E, int N) {
     nw = std::min(nw, g_max_threads / 32);
     while (nw > 8 && assign::scatter_smem_bytes(G, E, N, nw) > 224 * 1024) nw >>= 1;
     return nw;
+}
+
+// Launch shape of the scatter for a.T, a.k, a.G, a.E, a.N over nbatch
+// problems: sets a.slices and a.cta_blocks, returns the warps per CTA (grid:
+// scatter_grid_x).  Small source blocks whose CTAs all fit one wave go one
+// block per CTA down the CTA path (token ranks from per-warp masks) rather
+// than one block per warp: one decode-shaped problem (G = 64 blocks of 128
+// tokens x top-8) otherwise keeps 8 SMs busy for most of the launch.
+int scatter_shape(assign::Args &a, int nbatch) {
+    const int T = a.T, k = a.k, G = a.G, E = a.E, N = a.N;
+    a.slices = scatter_slices(nbatch, T, k, G);
+    a.cta_blocks = 0;
+    if (T == 0) return assign::SC_WARPS;
+    if (a.slices > 1) return std::min(slice_warps(T, G, a.slices), g_max_threads / 32);
+    if (static_cast<long long>(T / G) * k <= assign::WARP_BLOCK_MAX &&
+        static_cast<long long>(G) * nbatch <= device_sms()) {
+        int nw = std::min(slice_warps(T, G, 1), g_max_threads / 32);
+        while (nw > 8 && assign::scatter_smem_bytes(G, E, N, nw) > 224 * 1024) nw >>= 1;
+        if (assign::scatter_smem_bytes(G, E, N, nw) <= 224 * 1024) {
+            a.cta_blocks = 1;
+            return nw;
+        }
+    }
+    return scatter_warps(nbatch, T, k, G, E, N);
 }
 
 bool plan_shape_ok(int G, int E, int N, int L) {
@@ -1143,19 +1200,12 @@ int lb_assign(const int32_t *ids, const int32_t *cnt, const void *plan, const in
     a.offs = offs;
     a.ws = static_cast<int32_t *>(workspace);
     a.ws_stride = assign::ws_words(G, E, N);
-    a.slices = scatter_slices(nbatch, T, k, G);
-    const int nw = T == 0 ? assign::SC_WARPS
-                          : a.slices > 1 ? std::min(slice_warps(T, G, a.slices), g_max_threads / 32)
-                                         : scatter_warps(nbatch, T, k, G, E, N);
+    const int nw = scatter_shape(a, nbatch);
     const size_t sm1 = assign::prep_smem_bytes(G, E, N), sm2 = assign::scatter_smem_bytes(G, E, N, nw);
-    if (!allow_smem(assign::prep_kernel, g_lim_prep, sm1, false) ||
-        !allow_smem(assign::scatter_kernel, g_lim_scatter, sm2, false))
-        return LB_ECUDA;
-    if (launch_kernel("assign prep", assign::prep_kernel, dim3(nbatch), dim3(std::min(assign::PREP_THREADS, g_max_threads)),
-                      sm1, s, a) != LB_OK)
-        return LB_ECUDA;
+    if (!allow_smem(assign::scatter_kernel, g_lim_scatter, sm2, false)) return LB_ECUDA;
+    if (launch_prep(a, nbatch, sm1, s, "assign prep") != LB_OK) return LB_ECUDA;
     if (T == 0) return LB_OK;
-    return launch_kernel("assign scatter", assign::scatter_kernel, dim3(scatter_grid_x(T, k, G, nw, a.slices), nbatch),
+    return launch_kernel("assign scatter", assign::scatter_kernel, dim3(scatter_grid_x(T, k, G, nw, a.slices, a.cta_blocks != 0), nbatch),
                          dim3(nw * 32), assign::scatter_smem_bytes(G, E, N, nw), s, a);
 }
 
@@ -1194,10 +1244,7 @@ int lb_decide(const int32_t *cnt_pred, const int32_t *cnt, const int32_t *ids, v
     a.offs = offs;
     a.ws = static_cast<int32_t *>(workspace);
     a.ws_stride = assign::ws_words(G, E, N);
-    a.slices = scatter_slices(nbatch, T, k, G);
-    const int nw = T == 0 ? assign::SC_WARPS
-                          : a.slices > 1 ? std::min(slice_warps(T, G, a.slices), g_max_threads / 32)
-                                         : scatter_warps(nbatch, T, k, G, E, N);
+    const int nw = scatter_shape(a, nbatch);
     const size_t sm2 = assign::scatter_smem_bytes(G, E, N, nw);
     static SmemLimit lim0, lim1;
     if (!allow_smem(assign::scatter_kernel, g_lim_scatter, sm2, false)) return LB_ECUDA;
@@ -1218,8 +1265,7 @@ int lb_decide(const int32_t *cnt_pred, const int32_t *cnt, const int32_t *ids, v
         const size_t smp = plan::smem_bytes(G, E, N), sms = split::smem_bytes(G, E, N),
                      smt = assign::prep_smem_bytes(G, E, N);
         if ((with_plan && !allow_smem(plan::plan_kernel, g_lim_plan, smp, false)) ||
-            !allow_smem(split::split_kernel, g_lim_split, sms, false) ||
-            !allow_smem(assign::prep_kernel, g_lim_prep, smt, false))
+            !allow_smem(split::split_kernel, g_lim_split, sms, false))
             return LB_ECUDA;
         rc = LB_OK;
         if (with_plan)
@@ -1229,12 +1275,10 @@ int lb_decide(const int32_t *cnt_pred, const int32_t *cnt, const int32_t *ids, v
             rc = launch_kernel("split", split::split_kernel, dim3(nbatch), dim3(split::THREADS), sms, s, cnt,
                                static_cast<const uint8_t *>(plan), stride, G, E, N, passes, tok, mass, loads,
                                passes_run);
-        if (rc == LB_OK)
-            rc = launch_kernel("assign prep", assign::prep_kernel, dim3(nbatch),
-                               dim3(std::min(assign::PREP_THREADS, g_max_threads)), smt, s, a);
+        if (rc == LB_OK) rc = launch_prep(a, nbatch, smt, s, "assign prep");
     }
     if (rc != LB_OK || T == 0) return rc;
-    return launch_kernel("assign scatter", assign::scatter_kernel, dim3(scatter_grid_x(T, k, G, nw, a.slices), nbatch),
+    return launch_kernel("assign scatter", assign::scatter_kernel, dim3(scatter_grid_x(T, k, G, nw, a.slices, a.cta_blocks != 0), nbatch),
                          dim3(nw * 32), sm2, s, a);
 }
 
@@ -1399,18 +1443,12 @@ extern "C" int lb_assign_noalloc(const int32_t *ids, const int32_t *cnt, const v
     a.offs = offs;
     a.ws = scratch;
     a.ws_stride = assign::ws_words(G, E, N);
-    a.slices = scatter_slices(nbatch, T, k, G);
-    const int nw = T == 0 ? assign::SC_WARPS
-                          : a.slices > 1 ? std::min(slice_warps(T, G, a.slices), g_max_threads / 32)
-                                         : scatter_warps(nbatch, T, k, G, E, N);
-    if (!allow_smem(assign::prep_kernel, g_lim_prep, assign::prep_smem_bytes(G, E, N), false) ||
-        !allow_smem(assign::scatter_kernel, g_lim_scatter, assign::scatter_smem_bytes(G, E, N, nw), false))
+    const int nw = scatter_shape(a, nbatch);
+    if (!allow_smem(assign::scatter_kernel, g_lim_scatter, assign::scatter_smem_bytes(G, E, N, nw), false))
         return LB_ECUDA;
-    if (launch_kernel("assign prep (noalloc)", assign::prep_kernel, dim3(nbatch),
-                      dim3(std::min(assign::PREP_THREADS, g_max_threads)),
-                      assign::prep_smem_bytes(G, E, N), s, a) != LB_OK)
+    if (launch_prep(a, nbatch, assign::prep_smem_bytes(G, E, N), s, "assign prep (noalloc)") != LB_OK)
         return LB_ECUDA;
     if (T == 0) return LB_OK;
-    return launch_kernel("assign scatter (noalloc)", assign::scatter_kernel, dim3(scatter_grid_x(T, k, G, nw, a.slices), nbatch),
+    return launch_kernel("assign scatter (noalloc)", assign::scatter_kernel, dim3(scatter_grid_x(T, k, G, nw, a.slices, a.cta_blocks != 0), nbatch),
                          dim3(nw * 32), assign::scatter_smem_bytes(G, E, N, nw), s, a);
 }

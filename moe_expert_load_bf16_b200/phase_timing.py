@@ -32,7 +32,14 @@ PHASES = {
                             (2, 8, "round table (thread 0's edges)"), (8, 3, "round table (wait for the others)"),
                             (3, 6, "passes"), (6, 4, "masses")]),
     "assign prep": (20, ["stage inputs + per-expert segments", "bucket sizes + scan", "block bases"]),
+    "assign prep detail": (None, [(21, 24, "bucket sizes"), (24, 25, "edge shares"), (25, 26, "scan in the CTA"),
+                                  (26, 27, "cluster barrier + carries"), (27, 22, "offsets written"),
+                                  (22, 28, "chunk sums"), (28, 29, "q0 per block"),
+                                  (29, 55, "edge shares + replica bases"), (55, 56, "cluster barrier"),
+                                  (56, 57, "other keys"), (57, 23, "segments")]),
     "assign scatter": (10, ["per-problem tables", "scatter"]),
+    "assign scatter detail (token path)": (None, [(11, 58, "block classes"), (58, 59, "mask clear + barrier"),
+                                                  (59, 13, "first ids")]),
     "assign scatter, first chunk (warp 0)": (None, [(13, 14, "ids, lane masks, in-warp ranks"), (14, 15, "scan down the warps (2 barriers)"),
                                                     (15, 16, "local and home slots placed, replicated queued"),
                                                     (16, 17, "replicated queue resolved"), (17, 18, "dest rows written"),
@@ -101,7 +108,8 @@ def main():
             fn()
             if lib.lb_debug_ticks(ticks, 64) != 0:
                 raise RuntimeError("lb_debug_ticks failed")
-            kernels = [name] if name != "assign" else ["assign prep", "assign scatter",
+            kernels = [name] if name != "assign" else ["assign prep", "assign prep detail", "assign scatter",
+                                                       "assign scatter detail (token path)",
                                                        "assign scatter, first chunk (warp 0)"]
             if name == "gate":
                 kernels = ["gate (pairs, H split)"]

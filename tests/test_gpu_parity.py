@@ -605,7 +605,8 @@ def test_assign_throughput_launch_equals_single(name, T, B):
     """Enough problems to fill the GPU twice over switch the scatter to
     512-thread CTAs (two per SM), in CTA mode (large source blocks) and in
     warp mode (small blocks); the bytes equal one-problem calls (1024-thread
-    CTAs) and pass the oracle check."""
+    CTAs for large blocks, one CTA per small block) and pass the oracle
+    check."""
     w = workloads.WORKLOADS[name]
     ids = workloads.decode_ids(w.with_(T=T), T, range(B + 1)).to(DEV)
     path = DecisionPath(B, T, 8, w.E, w.k, w.G, w.N, w.L, device=DEV)
@@ -656,6 +657,39 @@ def test_scatter_large_blocks_every_k(k):
     assert _lib.lb_get_status() == 0
     for a, b in zip(sep, (path.dest, path.perm, path.offs)):
         assert torch.equal(a, b)
+
+
+@pytest.mark.parametrize("k", [1, 2, 3, 4, 5, 8, 9])
+def test_scatter_small_blocks_every_k(k):
+    """Small source blocks (at most one warp's share) take one warp each when
+    many problems fill the GPU, and one CTA each when one problem's blocks fit
+    one wave: every top-k width through both, with ragged blocks; the bytes of
+    the two launches agree and pass the oracle check."""
+    rng = np.random.default_rng(70 + k)
+    G, E, N, L, B = 8, 32, 3, 1, 20      # G * B > the SM count: the batched launch is warp mode
+    T = G * (1500 // k + 3)
+    pr = rng.permutation(np.arange(1, E + 1)) ** -1.2
+    pr /= pr.sum()
+    rows = [rng.choice(E, k, replace=False, p=pr) for _ in range((B + 1) * T)]
+    ids_np = np.stack(rows).astype(np.int32).reshape(B + 1, T, k)
+    path = DecisionPath(B, T, 8, E, k, G, N, L, device=DEV)
+    path.ids_pred.copy_(torch.from_numpy(ids_np[0:1]).to(DEV).expand(B, -1, -1))
+    path.ids.copy_(torch.from_numpy(ids_np[1:]).to(DEV))
+    _lib.lb_count(path.ids_pred, G, E, cnt=path.cnt_pred)
+    _lib.lb_plan_replicas(path.cnt_pred, N, L, plan=path.plan)
+    path.solve()
+    torch.cuda.synchronize()
+    assert _lib.lb_get_status() == 0
+    for b in (0, B - 1):
+        parity.check_path(path, b, 12)
+        one = DecisionPath(1, T, 8, E, k, G, N, L, device=DEV)
+        one.ids.copy_(path.ids[b:b + 1])
+        one.plan.copy_(path.plan[b:b + 1])
+        one.solve()
+        torch.cuda.synchronize()
+        assert _lib.lb_get_status() == 0
+        for f in ("dest", "perm", "offs"):
+            assert torch.equal(getattr(one, f)[0], getattr(path, f)[b]), (f, b)
 
 
 def test_scatter_repeated_id_in_row_is_flagged_and_contained():
