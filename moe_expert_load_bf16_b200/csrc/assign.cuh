@@ -173,12 +173,13 @@ __device__ void prep_problem(const Args &a, int b, uint8_t *sm, int C = 1, int c
     // per-expert scratch of the segment scan below (the arrays' own contents
     // are written later): the scan's value at e's first CSR position and
     // past its last, for tok (high word) and mass (low word)
-    int32_t *hT = qh, *hM = bh, *eT = hc, *eM = csum;
+    int32_t *hT = rcnt, *hM = rtot, *eT = homeadd, *eM = qh;
     for (int e = tid; e < E; e += blockDim.x) {
         hold[e] = 0ull;
         hT[e] = hM[e] = eT[e] = eM[e] = 0;
     }
     __syncthreads();
+    LB_TICK(60);
 
     // ---- per CSR position j (in parallel: a hot expert's tens of edges
     // would otherwise be one thread's serial walk): its edge and expert
@@ -200,7 +201,7 @@ __device__ void prep_problem(const Args &a, int b, uint8_t *sm, int C = 1, int c
                     if (e < 0 || e >= E || v < 0 || v >= G || j < rep_ptr[e] || j >= rep_ptr[e + 1]) {
                         e = -1;
                     } else {
-                        atomicOr(reinterpret_cast<unsigned long long *>(&hold[e]), 1ull << v);
+                        or_bit64(&hold[e], v);
                         val = (static_cast<uint64_t>(static_cast<uint32_t>(tk[i])) << 32) |
                               static_cast<uint32_t>(ms[i]);
                     }
@@ -225,8 +226,34 @@ __device__ void prep_problem(const Args &a, int b, uint8_t *sm, int C = 1, int c
         }
     }
     __syncthreads();
+    LB_TICK(61);
 
-    // ---- per expert: holders, remote mass; per edge: segment starts
+    // ---- remote counts of e per chunk of 8 blocks (blocks that hold no copy
+    // of e); per edge, its segment's start relative to its expert's first
+    const int nch = (G + 7) >> 3;
+    for (int x = tid; x < E * nch; x += blockDim.x) {
+        const int e = x % E, ch = x / E;
+        const uint64_t hm = hold[e] | (1ull << (e / Eg));
+        int sum = 0;
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const int g = ch * 8 + u;
+            if (g < G && !((hm >> g) & 1ull)) sum += cnt_s[g * E + e];
+        }
+        csum[e * 8 + ch] = sum;
+    }
+    for (int i = tid; i < ne; i += blockDim.x) {
+        const int e = ee[i];
+        if (e >= 0 && e < E) {
+            sq[i] -= hT[e];
+            sc[i] -= hM[e];
+        }
+    }
+    __syncthreads();
+    LB_TICK(62);
+
+    // ---- per expert: holders, remote total, remote assignments before the
+    // home block (q0 there), the home count
     for (int e = tid; e < E; e += blockDim.x) {
         const int h = e / Eg;
         int r0 = rep_ptr[e], r1 = rep_ptr[e + 1];
@@ -235,22 +262,24 @@ __device__ void prep_problem(const Args &a, int b, uint8_t *sm, int C = 1, int c
             r0 = r1 = 0;
         }
         const uint64_t hm = hold[e] | (1ull << h);
+        // (the scan's scratch shares these arrays: read before they are written)
         const int qo = r1 > r0 ? eT[e] - hT[e] : 0, cm = r1 > r0 ? eM[e] - hM[e] : 0;
-        int R = 0;
-        for (int g = 0; g < G; ++g)
-            if (!((hm >> g) & 1ull)) R += cnt_s[g * E + e];
+        int R = 0, qhome = 0;
+        for (int c2 = 0; c2 < nch; ++c2) {
+            const int cs = csum[e * 8 + c2];
+            R += cs;
+            qhome += c2 < (h >> 3) ? cs : 0;
+        }
+        for (int g = h & ~7; g < h; ++g)
+            if (!((hm >> g) & 1ull)) qhome += cnt_s[g * E + e];
         if (r1 > r0 && qo != R) bad = 1;
         hold[e] = hm;
         rcnt[e] = r1 - r0;
         rtot[e] = R;
         homeadd[e] = (r1 > r0) ? cm : R;
-    }
-    for (int i = tid; i < ne; i += blockDim.x) {
-        const int e = ee[i];
-        if (e >= 0 && e < E) {
-            sq[i] -= hT[e];
-            sc[i] -= hM[e];
-        }
+        qh[e] = qhome;
+        bh[e] = 0;
+        hc[e] = cnt_s[h * E + e];
     }
     __syncthreads();
     LB_TICK(21);
@@ -312,7 +341,9 @@ __device__ void prep_problem(const Args &a, int b, uint8_t *sm, int C = 1, int c
         int pre = 0;
         if (C > 1) {
             cluster_sync();
-            for (int q = 0; q < c; ++q) pre += ld_cluster_i32(mapa_shared(smem_u32(&cta_total), static_cast<uint32_t>(q)));
+            // (every warp reads the lower CTAs' totals at once, one per lane)
+            const int t = lane < c ? ld_cluster_i32(mapa_shared(smem_u32(&cta_total), static_cast<uint32_t>(lane))) : 0;
+            pre = __reduce_add_sync(kFull, t);
         }
         LB_TICK(27);
         if (c == C - 1 && tid == 0) offs[NK] = pre + cta_total;
@@ -327,42 +358,30 @@ __device__ void prep_problem(const Args &a, int b, uint8_t *sm, int C = 1, int c
     LB_TICK(22);
 
     // ---- base per (block g, expert e).  q0(g, e) = remote assignments of e
-    // in the blocks before g (blocks that hold no copy of e).  In four
-    // parallel steps (one thread per expert walking all blocks, with a hot
-    // expert's tens of edges at its home block, held the CTA on that thread):
-    // (1) remote counts per chunk of 8 blocks; (2) q0 of every block from the
-    // chunk prefixes, written over the counts' table in shared memory (each
-    // count is read before its slot is overwritten; only the home counts are
-    // needed later, kept in hc); (3) per edge, the home block's share of its
-    // segment and the replica holder's base; (4) every other (g, e).
-    const int nch = (G + 7) >> 3;
-    for (int x = tid; x < E * nch; x += blockDim.x) {
-        const int e = x % E, ch = x / E;
-        const uint64_t hm = hold[e];
-        int sum = 0;
-        for (int g = ch * 8; g < min(G, ch * 8 + 8); ++g)
-            if (!((hm >> g) & 1ull)) sum += cnt_s[g * E + e];
-        csum[e * 8 + ch] = sum;
-    }
-    for (int e = tid; e < E; e += blockDim.x) {
-        bh[e] = 0;
-        hc[e] = cnt_s[(e / Eg) * E + e];
-    }
-    __syncthreads();
-    LB_TICK(28);
-    for (int x = tid; x < E * nch; x += blockDim.x) {
-        const int e = x % E, ch = x / E;
-        const uint64_t hm = hold[e];
-        const int h = e / Eg;
-        int q0 = 0;
-        for (int c2 = 0; c2 < ch; ++c2) q0 += csum[e * 8 + c2];
-        for (int g = ch * 8; g < min(G, ch * 8 + 8); ++g) {
-            const int cg = cnt_s[g * E + e];
-            cnt_s[g * E + e] = q0;
-            if (g == h) qh[e] = q0;
-            if (!((hm >> g) & 1ull)) q0 += cg;
+    // in the blocks before g (blocks that hold no copy of e).  In parallel
+    // steps: (1) q0 of the own rows' blocks from the chunk sums above,
+    // written over the counts' table in shared memory (each count is read
+    // before its slot is overwritten; the home counts were kept in hc, q0 at
+    // the home block in qh); (2) per edge, the home block's share of its
+    // segment and the replica holder's base; (3) every other (g, e).
+    {
+        const int ch0 = rlo >> 3, ch1 = (rhi + 7) >> 3;
+        for (int x = tid; x < E * (ch1 - ch0); x += blockDim.x) {
+            const int e = x % E, ch = ch0 + x / E;
+            const uint64_t hm = hold[e];
+            int q0 = 0;
+            for (int c2 = 0; c2 < ch; ++c2) q0 += csum[e * 8 + c2];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int g = ch * 8 + u;
+                if (g >= G) break;
+                const int cg = cnt_s[g * E + e];
+                if (g >= rlo && g < rhi) cnt_s[g * E + e] = q0;
+                if (!((hm >> g) & 1ull)) q0 += cg;
+            }
         }
     }
+    LB_TICK(28);
     __syncthreads();
     LB_TICK(29);
     for (int i = tid; i < ne; i += blockDim.x) {
@@ -539,6 +558,7 @@ __device__ void scatter_setup(const Args &a, int b, const ScatterView &v) {
         v.s_v[j] = w;
     }
     __syncthreads();
+    LB_TICK(63);
     for (int j = tid; j < ne; j += blockDim.x) {
         // the expert of CSR position j: last e with rep0[e] <= j
         int lo = 0, hi = E - 1;
@@ -548,8 +568,9 @@ __device__ void scatter_setup(const Args &a, int b, const ScatterView &v) {
         }
         v.s_vcnt[j] = cnt[v.s_v[j] * E + lo];
         if (v.s_tok[j] > 0 || v.s_qoff[j] != 0x7fffffff)
-            atomicOr(reinterpret_cast<unsigned long long *>(&v.hold[lo]), 1ull << v.s_v[j]);
+            or_bit64(&v.hold[lo], v.s_v[j]);
     }
+    LB_TICK(9);
     for (int e = tid; e < E; e += blockDim.x) {
         const int h = e / Eg;
         int r0 = v.rep0[e], r1 = v.rep0[e + 1];

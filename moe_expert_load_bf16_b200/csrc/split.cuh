@@ -279,7 +279,7 @@ __device__ int split_problem(const int32_t *__restrict__ cnt, const uint8_t *__r
             *bad = 1;
             continue;
         }
-        atomicOr(reinterpret_cast<unsigned long long *>(&v.hold[e]), 1ull << v.ev[i]);
+        or_bit64(&v.hold[e], v.ev[i]);
     }
     __syncthreads();
     // (c) per expert: remote mass R (tokens of ranks that hold no copy); the
@@ -314,9 +314,7 @@ __device__ int split_problem(const int32_t *__restrict__ cnt, const uint8_t *__r
         v.mv[i] = t;
         const int w = v.ev[i];
         if (v.ee[i] == e && v.eu[i] == e / Eg && w >= 0 && w < G) {
-            const unsigned long long bit = 1ull << w;
-            if (atomicAnd(reinterpret_cast<unsigned long long *>(&v.hold[e]), ~bit) & bit)
-                atomicAdd(&v.Ls[w], v.cnt[w * E + e]);
+            if (clear_bit64(&v.hold[e], w)) atomicAdd(&v.Ls[w], v.cnt[w * E + e]);
         }
     }
     LB_TICK(7);

@@ -31,14 +31,17 @@ PHASES = {
     "split detail": (None, [(1, 7, "per-expert setup (thread 0)"), (7, 2, "wait for the other experts"),
                             (2, 8, "round table (thread 0's edges)"), (8, 3, "round table (wait for the others)"),
                             (3, 6, "passes"), (6, 4, "masses")]),
-    "assign prep": (20, ["stage inputs + per-expert segments", "bucket sizes + scan", "block bases"]),
-    "assign prep detail": (None, [(21, 24, "bucket sizes"), (24, 25, "edge shares"), (25, 26, "scan in the CTA"),
+    "assign prep": (20, ["stage inputs, segment scan, chunk sums, per expert", "bucket sizes + scan",
+                         "block bases"]),
+    "assign prep detail": (None, [(20, 60, "stage inputs"), (60, 61, "segment scan"), (61, 62, "chunk sums"),
+                                  (62, 21, "per expert"), (21, 24, "bucket sizes"), (24, 25, "edge shares"), (25, 26, "scan in the CTA"),
                                   (26, 27, "cluster barrier + carries"), (27, 22, "offsets written"),
-                                  (22, 28, "chunk sums"), (28, 29, "q0 per block"),
+                                  (22, 28, "q0 of the own blocks"), (28, 29, "barrier"),
                                   (29, 55, "edge shares + replica bases"), (55, 56, "cluster barrier"),
                                   (56, 57, "other keys"), (57, 23, "segments")]),
     "assign scatter": (10, ["per-problem tables", "scatter"]),
-    "assign scatter detail (token path)": (None, [(11, 58, "block classes"), (58, 59, "mask clear + barrier"),
+    "assign scatter detail (token path)": (None, [(10, 63, "stage segments"), (63, 9, "segment experts"),
+                                                  (9, 11, "per expert"), (11, 58, "block classes"), (58, 59, "mask clear + barrier"),
                                                   (59, 13, "first ids")]),
     "assign scatter, first chunk (warp 0)": (None, [(13, 14, "ids, lane masks, in-warp ranks"), (14, 15, "scan down the warps (2 barriers)"),
                                                     (15, 16, "local and home slots placed, replicated queued"),
