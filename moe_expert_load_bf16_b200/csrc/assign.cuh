@@ -24,6 +24,7 @@
 // deterministic and stable.
 #pragma once
 #include "common.cuh"
+#include "maskbits.cuh"
 #include "plan.cuh"
 
 namespace lb {

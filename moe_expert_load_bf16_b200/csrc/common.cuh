@@ -345,18 +345,6 @@ __device__ __forceinline__ float4 ld_cluster_f4(uint32_t addr) {
     return v;
 }
 
-// Bit b (0..63) of a 64-bit mask in shared memory, set or cleared with a
-// 32-bit atomic on the word that holds it (a hot expert's tens of holders hit
-// one mask at once; the 32-bit forms are the fast ones under contention).
-__device__ __forceinline__ void or_bit64(uint64_t *m, int b) {
-    atomicOr(reinterpret_cast<unsigned *>(m) + (b >> 5), 1u << (b & 31));
-}
-// true if this call cleared the bit (it was set before)
-__device__ __forceinline__ bool clear_bit64(uint64_t *m, int b) {
-    const unsigned bit = 1u << (b & 31);
-    return (atomicAnd(reinterpret_cast<unsigned *>(m) + (b >> 5), ~bit) & bit) != 0u;
-}
-
 // ---------------------------------------------------------------- staging
 // Copy n int32 from global to shared memory with the whole CTA: 16-byte
 // loads when both sides are 16-byte aligned, four loads in flight per thread.

@@ -20,6 +20,7 @@
 // the loads in shared memory and __syncwarp between rounds.
 #pragma once
 #include "common.cuh"
+#include "maskbits.cuh"
 #include "plan.cuh"
 
 namespace lb {
