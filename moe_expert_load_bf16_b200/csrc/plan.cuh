@@ -13,9 +13,8 @@
 //            arg-min is one redux.sync plus a ballot.
 //   edges:   per-expert replica counts, warp scan, parallel edge emission
 //            (expert ascending, rank ascending).
-//   rounds:  greedy colouring in edge order by one warp, each rank's busy
-//            rounds as a 128-bit mask in a lane's registers (one thread with
-//            shared-memory masks past 128 rounds); the stable order by round
+//   rounds:  greedy colouring in edge order by one thread, each rank's busy
+//            rounds as 64-bit words in shared memory; the stable order by round
 //            from per-round counts, a warp scan and each edge's rank among
 //            the earlier edges of its round.
 #pragma once
@@ -327,55 +326,46 @@ __device__ void plan_problem(const int32_t *__restrict__ cnt, int G, int E, int 
     __syncthreads();
 
     LB_TICK(35);
-    // ---------------- greedy colouring, edge order: one warp, each rank's
-    // busy-round mask (rounds 0..127) in registers of lane (rank & 31)
-    __shared__ int overflow_s;
-    if (warp == 0) {
-        uint64_t a0 = 0, a1 = 0, b0 = 0, b1 = 0;   // ranks lane and lane+32
-        int nr = 0, overflow = 0;
-        for (int i = 0; i < ne; ++i) {
-            const int u = eu[i], v = ev[i];
-            const uint64_t mu0 = __shfl_sync(kFull, u < 32 ? a0 : b0, u & 31);
-            const uint64_t mu1 = __shfl_sync(kFull, u < 32 ? a1 : b1, u & 31);
-            const uint64_t mv0 = __shfl_sync(kFull, v < 32 ? a0 : b0, v & 31);
-            const uint64_t mv1 = __shfl_sync(kFull, v < 32 ? a1 : b1, v & 31);
-            const uint64_t f0 = ~(mu0 | mv0), f1 = ~(mu1 | mv1);
-            const int c = f0 ? __ffsll(static_cast<long long>(f0)) - 1
-                             : (f1 ? 64 + __ffsll(static_cast<long long>(f1)) - 1 : -1);
-            if (c < 0) {
-                overflow = 1;
-                break;
-            }
-            const uint64_t w0 = c < 64 ? (1ull << c) : 0ull, w1 = c >= 64 ? (1ull << (c - 64)) : 0ull;
-            const bool own_u = lane == (u & 31), own_v = lane == (v & 31);
-            a0 |= (own_u && u < 32) || (own_v && v < 32) ? w0 : 0ull;
-            a1 |= (own_u && u < 32) || (own_v && v < 32) ? w1 : 0ull;
-            b0 |= (own_u && u >= 32) || (own_v && v >= 32) ? w0 : 0ull;
-            b1 |= (own_u && u >= 32) || (own_v && v >= 32) ? w1 : 0ull;
-            if (lane == 0) er[i] = c;
-            nr = max(nr, c + 1);
-        }
-        if (lane == 0) {
-            n_rounds_s = nr;
-            overflow_s = overflow;
-        }
-    }
-    __syncthreads();
-    if (overflow_s && tid == 0) {
-        // more than 128 rounds: the same greedy colouring with W-word masks
+    // ---------------- greedy colouring, edge order: one thread, each rank's
+    // busy rounds as W 64-bit words in shared memory.  An edge costs one
+    // round of independent loads (both ranks' first two words), a find-first
+    // and two stores.  Measured at the decode shape (128 edges, 67 rounds):
+    // 17.5 us, against 22.1 us for a warp holding 128-bit masks in registers
+    // (eight shuffles per edge), 19.4 us for 32-bit words scanned in a loop,
+    // and 24.8 us with the next edge's words loaded ahead and forwarded in
+    // registers (a longer chain of 64-bit selects).
+    if (tid == 0) {
         int nr = 0;
         for (int i = 0; i < ne; ++i) {
-            const int u = eu[i], v = ev[i];
-            int c = 0;
-            for (int w = 0; w < W; ++w) {
-                const uint64_t x = busy[u * W + w] | busy[v * W + w];
-                if (~x) {
-                    c = w * 64 + __ffsll(static_cast<long long>(~x)) - 1;
-                    break;
+            uint64_t *bu = busy + eu[i] * W, *bv = busy + ev[i] * W;
+            const uint64_t u0 = bu[0], v0 = bv[0];
+            const uint64_t u1 = W > 1 ? bu[1] : ~0ull, v1 = W > 1 ? bv[1] : ~0ull;
+            int c;
+            uint64_t ou, ov;   // the words that take the round's bit
+            if (~(u0 | v0)) {
+                c = __ffsll(static_cast<long long>(~(u0 | v0))) - 1;
+                ou = u0;
+                ov = v0;
+            } else if (~(u1 | v1)) {
+                c = 64 + __ffsll(static_cast<long long>(~(u1 | v1))) - 1;
+                ou = u1;
+                ov = v1;
+            } else {
+                // past 128 rounds (W words cover more rounds than a plan has edges)
+                c = 0;
+                for (int w = 2; w < W; ++w) {
+                    const uint64_t x = bu[w] | bv[w];
+                    if (~x) {
+                        c = w * 64 + __ffsll(static_cast<long long>(~x)) - 1;
+                        break;
+                    }
                 }
+                ou = bu[c >> 6];
+                ov = bv[c >> 6];
             }
-            busy[u * W + (c >> 6)] |= 1ull << (c & 63);
-            busy[v * W + (c >> 6)] |= 1ull << (c & 63);
+            const uint64_t bit = 1ull << (c & 63);
+            bu[c >> 6] = ou | bit;
+            bv[c >> 6] = ov | bit;   // (an edge joins two ranks)
             er[i] = c;
             nr = max(nr, c + 1);
         }
