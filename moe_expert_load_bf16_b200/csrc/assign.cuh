@@ -441,9 +441,17 @@ __device__ void prep_problem(const Args &a, int b, uint8_t *sm, int C = 1, int c
     if (C > 1) cluster_sync();   // no CTA leaves while another reads its offsets
 }
 
+// Both prep kernels let the scatter launch as soon as every prep CTA has
+// passed its own wait (the scatter then builds its input tables and waits
+// for the prep to complete before reading the prep's outputs).
+__device__ __forceinline__ void pdl_signal_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 __global__ void __launch_bounds__(PREP_THREADS) prep_kernel(const Args a) {
     extern __shared__ __align__(16) uint8_t sm[];
     pdl_begin();
+    pdl_signal_dependents();
     prep_problem(a, blockIdx.x, sm);
 }
 
@@ -452,6 +460,7 @@ __global__ void __launch_bounds__(PREP_THREADS) prep_kernel(const Args a) {
 __global__ void __launch_bounds__(PREP_THREADS) prep_kernel_cluster(const Args a) {
     extern __shared__ __align__(16) uint8_t sm[];
     pdl_begin();
+    pdl_signal_dependents();
     prep_problem(a, blockIdx.y, sm, static_cast<int>(gridDim.x), static_cast<int>(cluster_ctarank()));
 }
 
@@ -518,7 +527,15 @@ __device__ inline ScatterView scatter_carve(uint8_t *sm, int G, int E, int N, in
 // earlier segments, bucket start on the replica rank, replica rank, the
 // replica rank's own count of e), and per expert its home bucket start and
 // home count.  The per-block terms are added per assignment.
-__device__ void scatter_setup(const Args &a, int b, const ScatterView &v) {
+//
+// In two parts.  scatter_setup_inputs reads only the counts, the plan and
+// the split (inputs that were final before the prep started); the scatter
+// kernel runs it before waiting on the prep, which signals its dependents as
+// soon as it starts, so this part overlaps the prep.  scatter_setup_tables
+// then reads the prep's outputs (segment starts, replica bucket starts,
+// offsets).  A kernel that launches the scatter must itself be complete, or
+// must have signalled only after its own wait, when these inputs are read.
+__device__ void scatter_setup_inputs(const Args &a, int b, const ScatterView &v) {
     const int G = a.G, E = a.E, N = a.N, GN = G * N, NK = G * E;
     const int tid = threadIdx.x;
     const int32_t *cnt = a.cnt + static_cast<int64_t>(b) * NK;
@@ -530,32 +547,30 @@ __device__ void scatter_setup(const Args &a, int b, const ScatterView &v) {
     const int32_t *p_rep_edge = reinterpret_cast<const int32_t *>(blob + LY.rep_edge);
     const int32_t *tok = a.tok + static_cast<int64_t>(b) * GN;
     const int32_t *mass = a.mass + static_cast<int64_t>(b) * GN;
-    const int32_t *offs = a.offs + static_cast<int64_t>(b) * (NK + 1);
-    const int32_t *ws = a.ws + static_cast<size_t>(b) * a.ws_stride;
-    const int32_t *seg_qoff = ws + NK;
-    const int32_t *seg_cum = seg_qoff + GN;
-    const int32_t *seg_rep = seg_cum + GN;
     const int Eg = E / G;
-    int ne = hdr[0];
+    // (loads through L2 only: the data is a completed kernel's output, read
+    // before this kernel's wait)
+    int ne = __ldcg(hdr);
     if (ne < 0 || ne > GN) ne = 0;
-    for (int e = tid; e <= E; e += blockDim.x) v.rep0[e] = p_rep_ptr[e];
+    for (int e = tid; e <= E; e += blockDim.x) v.rep0[e] = __ldcg(p_rep_ptr + e);
     for (int e = tid; e < E; e += blockDim.x) v.hold[e] = 1ull << (e / Eg);   // home; replica holders ORed below
-    // per CSR position j (parallel): segment data
+    // per CSR position j (parallel): segment data; s_qoff marks a position
+    // invalid (and holds 0 otherwise until the tables' part), s_cum holds
+    // the edge index until then
     for (int j = tid; j < ne; j += blockDim.x) {
-        const int i = p_rep_edge[j];
+        const int i = __ldcg(p_rep_edge + j);
         const bool ok = i >= 0 && i < ne;
-        const int w = ok ? p_ev[i] : -1;
+        const int w = ok ? __ldcg(p_ev + i) : -1;
         if (!ok || w < 0 || w >= G) {
             v.s_tok[j] = 0;   // an empty segment: never matched
             v.s_qoff[j] = 0x7fffffff;
             v.s_v[j] = 0;
             continue;
         }
-        v.s_qoff[j] = seg_qoff[i];
-        v.s_tok[j] = tok[i];
-        v.s_mass[j] = mass[i];
-        v.s_cum[j] = seg_cum[i];
-        v.s_rep[j] = seg_rep[i];
+        v.s_qoff[j] = 0;
+        v.s_cum[j] = i;
+        v.s_tok[j] = __ldcg(tok + i);
+        v.s_mass[j] = __ldcg(mass + i);
         v.s_v[j] = w;
     }
     __syncthreads();
@@ -567,9 +582,8 @@ __device__ void scatter_setup(const Args &a, int b, const ScatterView &v) {
             const int mid = (lo + hi + 1) >> 1;
             if (v.rep0[mid] <= j) lo = mid; else hi = mid - 1;
         }
-        v.s_vcnt[j] = cnt[v.s_v[j] * E + lo];
-        if (v.s_tok[j] > 0 || v.s_qoff[j] != 0x7fffffff)
-            or_bit64(&v.hold[lo], v.s_v[j]);
+        v.s_vcnt[j] = __ldcg(cnt + v.s_v[j] * E + lo);
+        if (v.s_qoff[j] != 0x7fffffff) or_bit64(&v.hold[lo], v.s_v[j]);
     }
     LB_TICK(9);
     for (int e = tid; e < E; e += blockDim.x) {
@@ -577,11 +591,39 @@ __device__ void scatter_setup(const Args &a, int b, const ScatterView &v) {
         int r0 = v.rep0[e], r1 = v.rep0[e + 1];
         if (r0 < 0 || r1 > ne || r1 < r0) r0 = r1 = 0;
         v.rcnt[e] = r1 - r0;
-        v.homecnt[e] = cnt[h * E + e];
-        v.homeoff[e] = offs[h * E + e];
+        v.homecnt[e] = __ldcg(cnt + h * E + e);
         v.home[e] = h;
     }
     __syncthreads();
+}
+
+__device__ void scatter_setup_tables(const Args &a, int b, const ScatterView &v) {
+    const int G = a.G, E = a.E, N = a.N, GN = G * N, NK = G * E;
+    const int tid = threadIdx.x;
+    const uint8_t *blob = a.plan + static_cast<size_t>(b) * a.plan_stride;
+    const int32_t *hdr = reinterpret_cast<const int32_t *>(blob + plan::layout(G, E, N).hdr);
+    const int32_t *offs = a.offs + static_cast<int64_t>(b) * (NK + 1);
+    const int32_t *ws = a.ws + static_cast<size_t>(b) * a.ws_stride;
+    const int32_t *seg_qoff = ws + NK;
+    const int32_t *seg_cum = seg_qoff + GN;
+    const int32_t *seg_rep = seg_cum + GN;
+    const int Eg = E / G;
+    int ne = hdr[0];
+    if (ne < 0 || ne > GN) ne = 0;
+    for (int j = tid; j < ne; j += blockDim.x) {
+        if (v.s_qoff[j] == 0x7fffffff) continue;
+        const int i = v.s_cum[j];
+        v.s_qoff[j] = seg_qoff[i];
+        v.s_cum[j] = seg_cum[i];
+        v.s_rep[j] = seg_rep[i];
+    }
+    for (int e = tid; e < E; e += blockDim.x) v.homeoff[e] = offs[(e / Eg) * E + e];
+    __syncthreads();
+}
+
+__device__ void scatter_setup(const Args &a, int b, const ScatterView &v) {
+    scatter_setup_inputs(a, b, v);
+    scatter_setup_tables(a, b, v);
 }
 
 // Destination rank and permutation slot of an assignment of expert e from
@@ -1073,13 +1115,17 @@ __device__ inline void scatter_block_cta_any(const Args &a, int b, int g, int i0
 // Large blocks: CTA x takes block x (or a slice of it).
 __global__ void __launch_bounds__(SC_THREADS) scatter_kernel(const Args a) {
     extern __shared__ __align__(16) uint8_t sm[];
-    pdl_begin();
     __shared__ int bad;
     if (threadIdx.x == 0) bad = 0;
     const int nw = blockDim.x >> 5;
     const ScatterView v = scatter_carve(sm, a.G, a.E, a.N, nw);
     LB_TICK(10);
-    scatter_setup(a, blockIdx.y, v);
+    // Launched after the prep (or the fused decide kernel): the counts, plan
+    // and split were final before the prep started, so the tables built from
+    // them are built before waiting on it.
+    scatter_setup_inputs(a, blockIdx.y, v);
+    pdl_begin();
+    scatter_setup_tables(a, blockIdx.y, v);
     LB_TICK(11);
     const int nitems = (a.T / a.G) * a.k;
     if (nitems <= WARP_BLOCK_MAX && !a.cta_blocks) {

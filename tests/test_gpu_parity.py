@@ -550,6 +550,56 @@ def test_programmatic_launch_is_invisible(graph):
         parity.check_path(b, l, 12)
 
 
+@pytest.mark.parametrize("graph", [False, True])
+@pytest.mark.parametrize("separate", [False, True])
+def test_programmatic_launch_prep_to_scatter(graph, separate):
+    """The decode-shaped path runs the split, the prep (a cluster of 8 CTAs)
+    and the scatter as separate launches, through lb_decide or through
+    lb_split + lb_assign.  With programmatic dependent launch the prep lets
+    the scatter start while it runs, and the scatter builds its tables from
+    the counts, plan and split before waiting on the prep.  Two steps run
+    back to back on one set of buffers, each step's count, split and prep
+    overwriting what the previous step's scatter read, eagerly and replayed
+    from a CUDA graph.  The bytes are the same with and without programmatic
+    launch, and they pass the oracle check."""
+    w = workloads.WORKLOADS["decode"]
+    T = 1024
+    ids = workloads.decode_ids(w.with_(T=T), T, [0, 1, 2]).to(DEV)
+    outs = []
+    try:
+        for pdl in (0, 1):
+            _lib.lb_launch_options(pdl, 0)
+            p = DecisionPath(1, T, w.H, w.E, w.k, w.G, w.N, w.L, device=DEV)
+            p.ids_pred.copy_(ids[0:1])
+            _lib.lb_count(p.ids_pred, w.G, w.E, cnt=p.cnt_pred)
+            _lib.lb_plan_replicas(p.cnt_pred, w.N, w.L, plan=p.plan)
+            step = p.solve_separate if separate else p.solve
+
+            def two_steps():
+                p.ids.copy_(ids[1:2])
+                step()
+                p.ids.copy_(ids[2:3])
+                step()
+            if graph:
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g):
+                    two_steps()
+                for _ in range(3):
+                    g.replay()
+            else:
+                for _ in range(3):
+                    two_steps()
+            torch.cuda.synchronize()
+            assert _lib.lb_get_status() == 0
+            outs.append(p)
+    finally:
+        _lib.lb_launch_options(1, 0)
+    a, b = outs
+    for f in ("cnt", "tok", "mass", "loads", "passes_run", "dest", "perm", "offs"):
+        assert torch.equal(getattr(a, f), getattr(b, f)), f
+    parity.check_path(b, 0, 12)
+
+
 @pytest.mark.parametrize("graph,narrow", [(False, False), (True, False), (True, True)])
 def test_step_pipeline_equals_serial(graph, narrow):
     """Two steps in flight (the gate of step i+1 on one stream beside the
