@@ -66,15 +66,19 @@ constexpr long long kWaitCycles = 2000000000LL;
 
 constexpr unsigned kFull = 0xffffffffu;
 
-// Programmatic dependent launch.  Every kernel of the library begins with
+// Programmatic dependent launch.  Every kernel of the library calls
 // pdl_begin(), which waits until the previous kernel on the stream has
 // completed and its memory operations are visible (a no-op for a kernel
-// launched without programmatic stream serialization).  Nothing before it
-// touches global memory, so a kernel never reads an input, or overwrites a
-// buffer, that its predecessor is still using.  No kernel signals its
-// dependents early (measured: an early signal let the next kernels' blocks
-// sit waiting on the SMs and made the step slower); the gain is the launch
-// processing of the next kernel, which overlaps the previous one's exit.
+// launched without programmatic stream serialization), before it touches
+// global memory, so a kernel never reads an input, or overwrites a buffer,
+// that its predecessor is still using.  The one exception is the assign's
+// scatter, which follows the prep: the prep signals its dependents once past
+// its own wait, and the scatter reads the inputs that were final before the
+// prep started (counts, plan, split; through L2) before its wait.  No other
+// kernel signals early (measured: an early signal let the next kernels'
+// blocks sit waiting on the SMs and made the step slower); the gain there is
+// the launch processing of the next kernel, which overlaps the previous
+// one's exit.
 __device__ __forceinline__ void pdl_begin() {
     asm volatile("griddepcontrol.wait;" ::: "memory");
 }
