@@ -112,11 +112,12 @@ __device__ int relax_passes_regs(int G, int nr, int passes, const View &v) {
         const int La0 = La, Lb0 = Lb;
         int4 A = v.tab[ca];
         int4 B = TWO ? v.tab[cb] : make_int4(0, 0, 0, 0);
-        // four rounds per loop body in the two-ranks-per-lane form: one
-        // round's table loads and mass stores then sit in the shadow of the
-        // next rounds' shuffle chains (decode shape, G = 64: the passes 15 %
-        // shorter; unrolling by 2 or 8, or for G <= 32, gained nothing)
-#pragma unroll(TWO ? 4 : 1)
+        // four rounds per loop body: one round's table loads and mass stores
+        // then sit in the shadow of the next rounds' shuffle chains (decode
+        // shape, G = 64: the passes 15 % shorter; unrolling by 2 or 8 gained
+        // nothing there; for G <= 32 four rounds measure the same as the
+        // compiler's own unrolling, and forcing none was 15-25 % slower)
+#pragma unroll 4
         for (int r = 0; r < nr; ++r) {
             const int4 a = A, b = B;
             // next round's slots (row nr is an idle row, so no bound check)
