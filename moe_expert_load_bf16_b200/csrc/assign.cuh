@@ -441,9 +441,11 @@ __device__ void prep_problem(const Args &a, int b, uint8_t *sm, int C = 1, int c
     if (C > 1) cluster_sync();   // no CTA leaves while another reads its offsets
 }
 
-// Both prep kernels let the scatter launch as soon as every prep CTA has
-// passed its own wait (the scatter then builds its input tables and waits
-// for the prep to complete before reading the prep's outputs).
+// Both prep kernels (and the fused decide kernel without its plan step) let
+// the scatter launch as soon as every CTA has passed its own wait (the
+// scatter then builds its tables from the counts and the plan, and waits for
+// its predecessor to complete before reading the split and the prep's
+// outputs).
 __device__ __forceinline__ void pdl_signal_dependents() {
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
@@ -528,13 +530,15 @@ __device__ inline ScatterView scatter_carve(uint8_t *sm, int G, int E, int N, in
 // replica rank's own count of e), and per expert its home bucket start and
 // home count.  The per-block terms are added per assignment.
 //
-// In two parts.  scatter_setup_inputs reads only the counts, the plan and
-// the split (inputs that were final before the prep started); the scatter
-// kernel runs it before waiting on the prep, which signals its dependents as
-// soon as it starts, so this part overlaps the prep.  scatter_setup_tables
-// then reads the prep's outputs (segment starts, replica bucket starts,
-// offsets).  A kernel that launches the scatter must itself be complete, or
-// must have signalled only after its own wait, when these inputs are read.
+// In two parts.  scatter_setup_inputs reads only the counts and the plan
+// (inputs that were final before the scatter's predecessor started); the
+// scatter kernel runs it before waiting on that predecessor (the prep, or
+// the fused decide kernel without its plan step), which signals its
+// dependents as soon as it is past its own wait, so this part overlaps it.
+// scatter_setup_tables then reads the split (tok, mass) and the prep's
+// outputs (segment starts, replica bucket starts, offsets).  A kernel that
+// precedes the scatter and writes the counts or the plan must not signal
+// early.
 __device__ void scatter_setup_inputs(const Args &a, int b, const ScatterView &v) {
     const int G = a.G, E = a.E, N = a.N, GN = G * N, NK = G * E;
     const int tid = threadIdx.x;
@@ -545,8 +549,6 @@ __device__ void scatter_setup_inputs(const Args &a, int b, const ScatterView &v)
     const int32_t *p_ev = reinterpret_cast<const int32_t *>(blob + LY.edge_v);
     const int32_t *p_rep_ptr = reinterpret_cast<const int32_t *>(blob + LY.rep_ptr);
     const int32_t *p_rep_edge = reinterpret_cast<const int32_t *>(blob + LY.rep_edge);
-    const int32_t *tok = a.tok + static_cast<int64_t>(b) * GN;
-    const int32_t *mass = a.mass + static_cast<int64_t>(b) * GN;
     const int Eg = E / G;
     // (loads through L2 only: the data is a completed kernel's output, read
     // before this kernel's wait)
@@ -569,8 +571,6 @@ __device__ void scatter_setup_inputs(const Args &a, int b, const ScatterView &v)
         }
         v.s_qoff[j] = 0;
         v.s_cum[j] = i;
-        v.s_tok[j] = __ldcg(tok + i);
-        v.s_mass[j] = __ldcg(mass + i);
         v.s_v[j] = w;
     }
     __syncthreads();
@@ -607,12 +607,16 @@ __device__ void scatter_setup_tables(const Args &a, int b, const ScatterView &v)
     const int32_t *seg_qoff = ws + NK;
     const int32_t *seg_cum = seg_qoff + GN;
     const int32_t *seg_rep = seg_cum + GN;
+    const int32_t *tok = a.tok + static_cast<int64_t>(b) * GN;
+    const int32_t *mass = a.mass + static_cast<int64_t>(b) * GN;
     const int Eg = E / G;
     int ne = hdr[0];
     if (ne < 0 || ne > GN) ne = 0;
     for (int j = tid; j < ne; j += blockDim.x) {
         if (v.s_qoff[j] == 0x7fffffff) continue;
         const int i = v.s_cum[j];
+        v.s_tok[j] = tok[i];
+        v.s_mass[j] = mass[i];
         v.s_qoff[j] = seg_qoff[i];
         v.s_cum[j] = seg_cum[i];
         v.s_rep[j] = seg_rep[i];
@@ -1120,9 +1124,9 @@ __global__ void __launch_bounds__(SC_THREADS) scatter_kernel(const Args a) {
     const int nw = blockDim.x >> 5;
     const ScatterView v = scatter_carve(sm, a.G, a.E, a.N, nw);
     LB_TICK(10);
-    // Launched after the prep (or the fused decide kernel): the counts, plan
-    // and split were final before the prep started, so the tables built from
-    // them are built before waiting on it.
+    // Launched after the prep or the fused decide kernel: the counts and the
+    // plan were final before either started, so the tables built from them
+    // are built before waiting on it.
     scatter_setup_inputs(a, blockIdx.y, v);
     pdl_begin();
     scatter_setup_tables(a, blockIdx.y, v);

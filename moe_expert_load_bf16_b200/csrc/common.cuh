@@ -72,9 +72,9 @@ constexpr unsigned kFull = 0xffffffffu;
 // launched without programmatic stream serialization), before it touches
 // global memory, so a kernel never reads an input, or overwrites a buffer,
 // that its predecessor is still using.  The one exception is the assign's
-// scatter, which follows the prep: the prep signals its dependents once past
-// its own wait, and the scatter reads the inputs that were final before the
-// prep started (counts, plan, split; through L2) before its wait.  No other
+// scatter: its predecessor signals its dependents once past its own wait,
+// and the scatter reads, before its wait, only inputs that were final before
+// that predecessor started (through L2; assign.cuh names them).  No other
 // kernel signals early (measured: an early signal let the next kernels'
 // blocks sit waiting on the SMs and made the step slower); the gain there is
 // the launch processing of the next kernel, which overlaps the previous

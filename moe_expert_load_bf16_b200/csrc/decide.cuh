@@ -49,6 +49,9 @@ __global__ void __launch_bounds__(THREADS)
                   int32_t *__restrict__ loads_all, int32_t *__restrict__ passes_run_all) {
     extern __shared__ __align__(16) uint8_t sm[];
     pdl_begin();
+    // without the plan step the scatter that follows may start now: what it
+    // reads before its own wait (the counts and the plan) is not written here
+    if (!PLAN) assign::pdl_signal_dependents();
     __shared__ int bad;
     const int tid = threadIdx.x, b = blockIdx.x;
     const int G = a.G, E = a.E, N = a.N, GN = G * N;
