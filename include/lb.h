@@ -155,10 +155,15 @@ int lb_gate_tuning(int stages, int split, int persistent, int kbox, int tiles_pe
 
 /* Launch options (process-wide; results are identical under every option).
  * programmatic_dependent_launch = 1 (the default): every kernel without a
- * thread-block cluster is launched with programmatic stream serialization,
- * so its launch is processed while the previous kernel on the stream runs;
- * each kernel waits for its predecessor's completion (and the visibility of
- * its writes) before it touches global memory.  0 = plain stream order.
+ * thread-block cluster, and lb_assign's clustered prep, is launched with
+ * programmatic stream serialization, so its launch is processed while the
+ * previous kernel on the stream runs; each kernel waits for its
+ * predecessor's completion (and the visibility of its writes) before it
+ * touches global memory.  The one exception: the prep of lb_assign and
+ * lb_decide (or lb_decide's fused kernel when it has no plan step) lets the
+ * scatter that follows it start once past its own wait, and the scatter
+ * reads the counts and the plan, which that kernel does not write, before
+ * its wait.  0 = plain stream order.
  * max_block_threads (0 = 1024, or 256, 512, 1024): the largest thread block
  * the integer kernels use (lb_assign's prep and scatter take up to 1024
  * threads; count, plan and split 512).  512 lets a block of every integer

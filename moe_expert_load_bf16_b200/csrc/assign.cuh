@@ -10,18 +10,22 @@
 //   base[g,e] = where block g's assignments of e start in their bucket
 //               (or q0 for a replicated expert's remote assignments, whose
 //               destination depends on their rank q among e's remote ones).
-// The prep kernel (one CTA per problem) computes these from cnt, plan and
+// The prep kernel (one CTA per problem, or a cluster of 8 CTAs per problem
+// when one problem's key table is large) computes these from cnt, plan and
 // split without reading the ids; counts and plan are staged in shared memory
-// first.  The scatter kernel (one CTA per (problem, source block), or one
-// warp per block when blocks are small) then needs only each assignment's
-// rank among the earlier assignments of the same expert in its block: warps
-// take consecutive 32-assignment steps, find each lane's peers (same expert)
-// with one ballot per bit of the expert id, keep per-warp counters in shared
-// memory, a per-expert scan down the warps' counters keeps block order, and each
-// assignment's slot is base + rank, or, for a replicated expert's remote
-// assignment, a binary search over the expert's replica segments (staged in
-// shared memory).  Positions never come from atomics, so the permutation is
-// deterministic and stable.
+// first.  The scatter kernel (one CTA per (problem, source block) or slice
+// of one, or one warp per block when many problems' small blocks fill the
+// GPU) then needs only each assignment's rank among the earlier assignments
+// of the same expert in its block: in the CTA forms with top-k up to 8, one
+// token per lane and per-warp lane masks of each expert (the rank is the
+// count of earlier lanes holding it); otherwise warps take consecutive
+// 32-assignment steps and find each lane's peers (same expert) with one
+// ballot per bit of the expert id.
+// Per-warp counters in shared memory and a per-expert scan down the warps'
+// counters keep block order, and each assignment's slot is base + rank, or,
+// for a replicated expert's remote assignment, found by searching the
+// expert's replica segments (staged in shared memory).  Positions never come
+// from atomics, so the permutation is deterministic and stable.
 #pragma once
 #include "common.cuh"
 #include "maskbits.cuh"
