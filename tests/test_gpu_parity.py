@@ -120,6 +120,36 @@ def test_decode_steps(T):
         parity.check_path(path, b, 12)
 
 
+@pytest.mark.parametrize("B", [2, 3])
+def test_decode_few_problems_per_launch(B):
+    """A few decode-shaped problems in one launch: the assign's prep runs one
+    cluster of 8 CTAs per problem, and the scatter one CTA per source block
+    of every problem while they fit one wave (B = 2: 128 CTAs) or one warp
+    per block once they do not (B = 3: 192 blocks); separate and fused forms
+    agree, and every problem passes the oracle check."""
+    w = workloads.WORKLOADS["decode"]
+    T = 1024
+    ids = workloads.decode_ids(w.with_(T=T), T, range(B + 1)).to(DEV)
+    path = DecisionPath(B, T, w.H, w.E, w.k, w.G, w.N, w.L, device=DEV)
+    cnt0 = _lib.lb_count(ids[0], w.G, w.E)
+    _lib.lb_plan_replicas(cnt0, w.N, w.L, plan=path.plan[0:1])
+    path.plan[1:].copy_(path.plan[0:1].expand(B - 1, -1))
+    path.ids.copy_(ids[1:])
+    path.ids_pred.copy_(ids[0:1].expand(B, -1, -1))
+    path.cnt_pred.copy_(cnt0.unsqueeze(0).expand(B, -1, -1))
+    path.solve()
+    torch.cuda.synchronize()
+    assert _lib.lb_get_status() == 0
+    for b in range(B):
+        parity.check_path(path, b, 12)
+    sep = [t.clone() for t in (path.dest, path.perm, path.offs)]
+    path.solve_separate()
+    torch.cuda.synchronize()
+    assert _lib.lb_get_status() == 0
+    for a, c in zip(sep, (path.dest, path.perm, path.offs)):
+        assert torch.equal(a, c)
+
+
 @pytest.mark.parametrize("mode", ["auto", "pairs_split_h2", "pairs_split_h3", "pairs_split_h4"])
 @pytest.mark.parametrize("T", [64, 1024, 4096, 8192])
 def test_decode_gate(T, mode):
