@@ -653,14 +653,48 @@ int scatter_slices(int nbatch, int T, int k, int G) {
 }
 
 // The assign's prep for one problem's latency on a cluster of 8 CTAs (each
-// owning G/8 ranks of the (rank, expert) key table) when the table is large:
-// at the decode shape (64 x 256 keys) one CTA is instruction-bound for about
-// 34 us.  Otherwise one CTA per problem.
+// owning G/8 ranks of the (rank, expert) key table) when the table is large
+// and the problems' clusters all fit the device at once (on a B200 about 15
+// clusters of 8 whole-SM CTAs): at the decode shape (64 x 256 keys) one CTA was
+// instruction-bound for about 34 us.  Otherwise one CTA per problem.
 SmemLimit g_lim_prep_cluster;
+
+// Clusters of 8 prep CTAs of nt threads that the device holds at once
+// (cached per device and block size; 0 if the query fails), asked with the
+// largest shared memory the prep may take.
+int prep_max_clusters(int nt) {
+    static int cached[kMaxDevices][3] = {};   // 0 not asked yet, -1 none or failed
+    const int dev = current_device();
+    const int t = nt >= 1024 ? 2 : nt >= 512 ? 1 : 0;
+    if (dev < 0) return 0;
+    if (cached[dev][t] != 0) return std::max(cached[dev][t], 0);
+    const size_t smem = 224 * 1024;
+    int n = 0;
+    if (allow_smem(assign::prep_kernel_cluster, g_lim_prep_cluster, smem, false)) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(8, 64, 1);
+        cfg.blockDim = dim3(nt, 1, 1);
+        cfg.dynamicSmemBytes = smem;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = 8;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        if (cudaOccupancyMaxActiveClusters(&n, assign::prep_kernel_cluster, &cfg) != cudaSuccess) {
+            cudaGetLastError();
+            n = 0;
+        }
+    }
+    cached[dev][t] = n > 0 ? n : -1;
+    return std::max(n, 0);
+}
+
 int launch_prep(const assign::Args &a, int nbatch, size_t smem, cudaStream_t s, const char *what) {
     const int nt = std::min(assign::PREP_THREADS, g_max_threads);
-    const bool cl = static_cast<long long>(a.G) * a.E >= 8192 && a.G % 8 == 0 &&
-                    static_cast<long long>(nbatch) * 8 <= device_sms();
+    // the cluster form only when every problem's cluster runs at once
+    const bool cl = static_cast<long long>(a.G) * a.E >= 8192 && a.G % 8 == 0 && nbatch <= prep_max_clusters(nt);
     if (!cl) {
         if (!allow_smem(assign::prep_kernel, g_lim_prep, smem, false)) return LB_ECUDA;
         return launch_kernel(what, assign::prep_kernel, dim3(nbatch), dim3(nt), smem, s, a);
