@@ -393,13 +393,16 @@ int launch_gate_pairk(const CUtensorMap &ma, const CUtensorMap &mb, const gate::
     cfg.blockDim = dim3(gate::Shape<4>::THREADS, 1, 1);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = s;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = 2 * KS;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    // (the kernel waits for its predecessor before it touches global memory)
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = g_pdl ? 1 : 0;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 2;
     const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, ma, mb, p);
     if (e != cudaSuccess) return cuda_fail(e, "cudaLaunchKernelEx(gate_topk pair, split H)");
     return launched("gate_topk pair, split H");
