@@ -946,8 +946,6 @@ __global__ void __launch_bounds__(Shape<4>::THREADS, 1)
         LB_CTA_TIME(0);
     }
 
-    for (int c = tid; c < p.Epad; c += Shape<4>::THREADS)
-        bias_s[c] = (p.bias != nullptr && c < p.E) ? p.bias[static_cast<int64_t>(b) * p.E + c] : 0.f;
     if (tid == 0) {
         for (int s = 0; s < stages; ++s) {
             mbar_init(&full_bar[s], 1);
@@ -1056,6 +1054,11 @@ __global__ void __launch_bounds__(Shape<4>::THREADS, 1)
     float *recv_f = stage_f + BM * SR;                   // [KS-1][RMAX][SR]
     bool ok = true;
     if (epi) {
+        // the bias, staged by the epilogue warps while the main loop runs (its
+        // load is off the path to the first tiles); the cluster barrier after
+        // the partials are staged orders it before the ranking reads it
+        for (int c = tid - 64; c < p.Epad; c += Shape<4>::EPI)
+            bias_s[c] = (p.bias != nullptr && c < p.E) ? p.bias[static_cast<int64_t>(b) * p.E + c] : 0.f;
         ok = mbar_wait(&acc_full, 0) && !*abort_flag;
         if (!ok && lane == 0) flag(LB_DEV_TIMEOUT);
         ok = __all_sync(kFull, ok);
